@@ -1,0 +1,136 @@
+"""Seeded synthetic inputs for the gated delta-rule layer.
+
+This module only draws random numbers and shapes them; it holds none of the
+layer's arithmetic.  Both the CUDA path (tests, bench) and the CPU oracle
+consume the same host tensors it returns, so the oracle sees the exact
+bf16-rounded values the GPU sees (upcast to fp64).
+
+Distributions follow the workloads the layer is described on (350M..3B-scale
+layers of a Gated DeltaNet / Kimi-Delta-Attention stack):
+
+* q, k ~ N(0,1), L2-normalised per token (fp32, eps 1e-6 under the root),
+  then cast to the compute dtype -- the block design normalises q and k;
+* v ~ N(0,1), not normalised;
+* beta = sigmoid(N(0,1));
+* log-gate g = -softplus(N(0,1) + shift): shift 0 for the small and the
+  long-context workloads, 2 for the 350M-scale and the channel-gate ones,
+  and -6 for the "slow gate" cases that keep the inter-chunk state alive;
+* optional initial state ~ N(0, std^2) in fp32; dO ~ N(0,1).
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+from typing import Optional
+
+import torch
+
+_DT = {"bf16": torch.bfloat16, "f32": torch.float32}
+
+
+@dataclass(frozen=True)
+class ChunkConfig:
+    name: str
+    B: int
+    T: int
+    H: int
+    dk: int
+    dv: int
+    chunk: int
+    dtype: str = "bf16"          # "bf16" or "f32" for q, k, v, o, dO
+    gate: str = "scalar"         # "scalar" or "channel"
+    g_shift: float = 0.0
+    h0_std: Optional[float] = None
+    backward: bool = True
+    dhT_std: Optional[float] = None
+    seed: int = 1000
+
+
+@dataclass(frozen=True)
+class DecodeConfig:
+    name: str
+    N: int
+    H: int
+    dk: int
+    dv: int
+    steps: int
+    dtype: str = "bf16"
+    gate: str = "scalar"
+    g_shift: float = 0.0
+    state_std: float = 0.02
+    seed: int = 1003
+
+
+# The five workloads.  Index 0 is the small case the oracle finishes in a
+# blink; "same distributions as the small case" is read for the long-context
+# and decode workloads (g shift 0).
+TINY = ChunkConfig("tiny B1 H1 T64 d16 C16 f32", 1, 64, 1, 16, 16, 16, "f32",
+                   "scalar", 0.0, None, False, None, 1000)
+L350M = ChunkConfig("350M-layer B8 H8 T2048 d128 C64 bf16", 8, 2048, 8, 128, 128,
+                    64, "bf16", "scalar", 2.0, None, True, None, 1001)
+LONG = ChunkConfig("long-context B1 H16 T8192 d128 C64 bf16", 1, 8192, 16, 128,
+                   128, 64, "bf16", "scalar", 0.0, 0.02, True, 1.0, 1002)
+DECODE = DecodeConfig("decode N256 H16 d128 x1000 steps", 256, 16, 128, 128,
+                      1000, "bf16", "scalar", 0.0, 0.02, 1003)
+KDA = ChunkConfig("kda B2 H32 T4096 d128 C64 bf16 channel-gate", 2, 4096, 32, 128,
+                  128, 64, "bf16", "channel", 2.0, None, True, None, 1004)
+
+
+def _gen(seed: int, idx: int) -> torch.Generator:
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed * 97 + idx)
+    return g
+
+
+def _l2norm(x: torch.Tensor) -> torch.Tensor:
+    return x * torch.rsqrt((x * x).sum(-1, keepdim=True) + 1e-6)
+
+
+def make_chunk_inputs(cfg: ChunkConfig, **over) -> dict:
+    """Host (CPU) tensors for one chunkwise fwd/bwd call.
+
+    Keyword overrides replace fields of ``cfg`` (e.g. T=100, g_shift=-6).
+    Returns q, k, v, dO in the config dtype; g, beta, h0, dhT in fp32."""
+    if over:
+        cfg = ChunkConfig(**{**cfg.__dict__, **over})
+    B, T, H, dk, dv = cfg.B, cfg.T, cfg.H, cfg.dk, cfg.dv
+    dt = _DT[cfg.dtype]
+    s = cfg.seed
+    q = _l2norm(torch.randn(B, T, H, dk, generator=_gen(s, 0))).to(dt)
+    k = _l2norm(torch.randn(B, T, H, dk, generator=_gen(s, 1))).to(dt)
+    v = torch.randn(B, T, H, dv, generator=_gen(s, 2)).to(dt)
+    gshape = (B, T, H, dk) if cfg.gate == "channel" else (B, T, H)
+    g = -torch.nn.functional.softplus(
+        torch.randn(*gshape, generator=_gen(s, 3)) + cfg.g_shift)
+    beta = torch.sigmoid(torch.randn(B, T, H, generator=_gen(s, 4)))
+    h0 = None
+    if cfg.h0_std is not None:
+        h0 = torch.randn(B, H, dv, dk, generator=_gen(s, 5)) * cfg.h0_std
+    dO = torch.randn(B, T, H, dv, generator=_gen(s, 6)).to(dt)
+    dhT = None
+    if cfg.dhT_std is not None:
+        dhT = torch.randn(B, H, dv, dk, generator=_gen(s, 7)) * cfg.dhT_std
+    return dict(q=q.contiguous(), k=k.contiguous(), v=v.contiguous(),
+                g=g.contiguous(), beta=beta.contiguous(), h0=h0, dO=dO.contiguous(),
+                dhT=dhT, cfg=cfg)
+
+
+def make_decode_inputs(cfg: DecodeConfig, steps: Optional[int] = None, **over) -> dict:
+    """Host tensors for ``steps`` successive single-token updates.
+    q, k [steps,N,H,dk], v [steps,N,H,dv] in the config dtype;
+    g [steps,N,H] (or [...,dk]), beta [steps,N,H], state0 [N,H,dv,dk] fp32."""
+    if over:
+        cfg = DecodeConfig(**{**cfg.__dict__, **over})
+    S = cfg.steps if steps is None else steps
+    N, H, dk, dv = cfg.N, cfg.H, cfg.dk, cfg.dv
+    dt = _DT[cfg.dtype]
+    s = cfg.seed
+    q = _l2norm(torch.randn(S, N, H, dk, generator=_gen(s, 0))).to(dt)
+    k = _l2norm(torch.randn(S, N, H, dk, generator=_gen(s, 1))).to(dt)
+    v = torch.randn(S, N, H, dv, generator=_gen(s, 2)).to(dt)
+    gshape = (S, N, H, dk) if cfg.gate == "channel" else (S, N, H)
+    g = -torch.nn.functional.softplus(
+        torch.randn(*gshape, generator=_gen(s, 3)) + cfg.g_shift)
+    beta = torch.sigmoid(torch.randn(S, N, H, generator=_gen(s, 4)))
+    state0 = torch.randn(N, H, dv, dk, generator=_gen(s, 5)) * cfg.state_std
+    return dict(q=q, k=k, v=v, g=g.contiguous(), beta=beta.contiguous(),
+                state0=state0, cfg=cfg)
