@@ -1,0 +1,235 @@
+"""Python binding of libgdn.so, the sm_100a gated delta-rule library.
+
+Argument marshalling only: every function below checks tensor shapes, dtypes
+and devices, allocates outputs with torch (device memory is torch's job),
+and calls the C entry point of the same name through ctypes on the current
+CUDA stream.  No arithmetic of the layer happens in Python, and there is no
+CPU fallback: if the compiled library is missing, the first call raises.
+
+Layouts follow the C ABI (include/gdn.h): q, k [B,T,H,dk]; v, o [B,T,H,dv];
+g [B,T,H] (scalar gate) or [B,T,H,dk] (channel gate) fp32; beta [B,T,H] fp32;
+states [B,H,dv,dk] fp32.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgdn.so")
+
+GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_WORKSPACE, GDN_ERR_CUDA, \
+    GDN_ERR_DEVICE_TIMEOUT = range(6)
+GDN_BF16, GDN_F32 = 0, 1
+GDN_GATE_SCALAR, GDN_GATE_CHANNEL = 0, 1
+
+# Every symbol include/gdn.h declares.
+EXPORTS = ("gdn_chunk_fwd_workspace", "gdn_chunk_fwd", "gdn_chunk_bwd_workspace",
+           "gdn_chunk_bwd", "gdn_recurrent_step", "gdn_query_device_status",
+           "gdn_status_string")
+
+
+class gdn_dims(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("T", ctypes.c_int), ("H", ctypes.c_int),
+                ("dk", ctypes.c_int), ("dv", ctypes.c_int), ("chunk", ctypes.c_int),
+                ("dtype", ctypes.c_int), ("gate", ctypes.c_int), ("scale", ctypes.c_float)]
+
+
+class GdnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)}")
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libgdn.so with argument types set.  Raises if it is absent."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(
+                    f"{LIB_PATH} is missing: build it with "
+                    "`python -m gated_delta_rule_153_b200.build` (nvcc, sm_100a)")
+            L = ctypes.CDLL(LIB_PATH)
+            vp, fp, sz = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t
+            dp = ctypes.POINTER(gdn_dims)
+            i, f = ctypes.c_int, ctypes.c_float
+            L.gdn_chunk_fwd_workspace.argtypes = [dp]
+            L.gdn_chunk_fwd_workspace.restype = sz
+            L.gdn_chunk_bwd_workspace.argtypes = [dp]
+            L.gdn_chunk_bwd_workspace.restype = sz
+            L.gdn_chunk_fwd.argtypes = [dp, vp, vp, vp, fp, fp, fp, vp, fp, vp, sz, vp]
+            L.gdn_chunk_fwd.restype = i
+            L.gdn_chunk_bwd.argtypes = [dp, vp, vp, vp, fp, fp, fp, vp, fp, vp, vp, vp,
+                                        fp, fp, fp, vp, sz, vp]
+            L.gdn_chunk_bwd.restype = i
+            L.gdn_recurrent_step.argtypes = [i, i, i, i, i, i, f, vp, vp, vp, fp, fp, fp,
+                                             vp, vp]
+            L.gdn_recurrent_step.restype = i
+            L.gdn_query_device_status.argtypes = [vp, vp]
+            L.gdn_query_device_status.restype = i
+            L.gdn_status_string.argtypes = [i]
+            L.gdn_status_string.restype = ctypes.c_char_p
+            _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().gdn_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str):
+    if status != GDN_OK:
+        raise GdnError(status, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype_code(t):
+    import torch
+    if t.dtype == torch.bfloat16:
+        return GDN_BF16
+    if t.dtype == torch.float32:
+        return GDN_F32
+    raise TypeError(f"q/k/v must be bfloat16 or float32, got {t.dtype}")
+
+
+def _need(t, name, dtype=None, shape=None):
+    import torch
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def make_dims(q, v, g, chunk=64, scale=1.0) -> gdn_dims:
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    gate = GDN_GATE_CHANNEL if g.dim() == 4 else GDN_GATE_SCALAR
+    return gdn_dims(B, T, H, dk, dv, int(chunk), _dtype_code(q), gate, float(scale))
+
+
+def gdn_chunk_fwd_workspace(dims: gdn_dims) -> int:
+    return int(lib().gdn_chunk_fwd_workspace(ctypes.byref(dims)))
+
+
+def gdn_chunk_bwd_workspace(dims: gdn_dims) -> int:
+    return int(lib().gdn_chunk_bwd_workspace(ctypes.byref(dims)))
+
+
+def _validate_chunk_inputs(q, k, v, g, beta, h0):
+    import torch
+    _need(q, "q")
+    B, T, H, dk = q.shape
+    _need(k, "k", q.dtype, (B, T, H, dk))
+    _need(v, "v", q.dtype)
+    if v.shape[:3] != (B, T, H):
+        raise ValueError("v must be [B,T,H,dv] matching q")
+    dv = v.shape[3]
+    _need(g, "g", torch.float32)
+    if tuple(g.shape) not in ((B, T, H), (B, T, H, dk)):
+        raise ValueError("g must be [B,T,H] or [B,T,H,dk]")
+    _need(beta, "beta", torch.float32, (B, T, H))
+    if h0 is not None:
+        _need(h0, "h0", torch.float32, (B, H, dv, dk))
+    return B, T, H, dk, dv
+
+
+def _workspace(nbytes, device, workspace):
+    import torch
+    if nbytes == 0:
+        return None
+    if workspace is not None:
+        if workspace.numel() * workspace.element_size() < nbytes:
+            raise ValueError(f"workspace too small: need {nbytes} bytes")
+        return workspace
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+def gdn_chunk_fwd(q, k, v, g, beta, h0=None, *, chunk=64, scale=1.0,
+                  output_final_state=True, o=None, hT=None, workspace=None, stream=None):
+    """Chunkwise forward.  Returns (o, hT); hT is None unless requested."""
+    import torch
+    B, T, H, dk, dv = _validate_chunk_inputs(q, k, v, g, beta, h0)
+    dims = make_dims(q, v, g, chunk, scale)
+    if o is None:
+        o = torch.empty(B, T, H, dv, dtype=q.dtype, device=q.device)
+    if output_final_state and hT is None:
+        hT = torch.empty(B, H, dv, dk, dtype=torch.float32, device=q.device)
+    nbytes = gdn_chunk_fwd_workspace(dims)
+    ws = _workspace(nbytes, q.device, workspace)
+    st = lib().gdn_chunk_fwd(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
+                             _ptr(beta), _ptr(h0), _ptr(o), _ptr(hT), _ptr(ws),
+                             nbytes if ws is None else ws.numel() * ws.element_size(),
+                             _stream(stream))
+    _check(st, "gdn_chunk_fwd")
+    return o, hT
+
+
+def gdn_chunk_bwd(q, k, v, g, beta, dO, h0=None, dhT=None, *, chunk=64, scale=1.0,
+                  workspace=None, stream=None):
+    """Chunkwise backward of <dO,o> + <dhT,hT>.  Returns a dict with dq, dk,
+    dv (dtype of q), dg (shape of g), dbeta, dh0 (None when h0 is None)."""
+    import torch
+    B, T, H, dk, dv = _validate_chunk_inputs(q, k, v, g, beta, h0)
+    _need(dO, "dO", q.dtype, (B, T, H, dv))
+    if dhT is not None:
+        _need(dhT, "dhT", torch.float32, (B, H, dv, dk))
+    dims = make_dims(q, v, g, chunk, scale)
+    out = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dv=torch.empty_like(v),
+               dg=torch.empty_like(g), dbeta=torch.empty_like(beta),
+               dh0=None if h0 is None else torch.empty_like(h0))
+    nbytes = gdn_chunk_bwd_workspace(dims)
+    ws = _workspace(nbytes, q.device, workspace)
+    st = lib().gdn_chunk_bwd(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
+                             _ptr(beta), _ptr(h0), _ptr(dO), _ptr(dhT), _ptr(out["dq"]),
+                             _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dg"]),
+                             _ptr(out["dbeta"]), _ptr(out["dh0"]), _ptr(ws),
+                             nbytes if ws is None else ws.numel() * ws.element_size(),
+                             _stream(stream))
+    _check(st, "gdn_chunk_bwd")
+    return out
+
+
+def gdn_recurrent_step(q, k, v, g, beta, state, *, scale=1.0, o=None, stream=None):
+    """One decode token, in place on ``state`` [N,H,dv,dk] fp32.  q,k [N,H,dk];
+    v [N,H,dv]; g [N,H] or [N,H,dk]; beta [N,H].  Returns o [N,H,dv]."""
+    import torch
+    _need(q, "q")
+    N, H, dk = q.shape
+    _need(k, "k", q.dtype, (N, H, dk))
+    _need(v, "v", q.dtype)
+    dv = v.shape[-1]
+    _need(g, "g", torch.float32)
+    gate = GDN_GATE_CHANNEL if g.dim() == 3 else GDN_GATE_SCALAR
+    _need(beta, "beta", torch.float32, (N, H))
+    _need(state, "state", torch.float32, (N, H, dv, dk))
+    if o is None:
+        o = torch.empty(N, H, dv, dtype=q.dtype, device=q.device)
+    st = lib().gdn_recurrent_step(N, H, dk, dv, _dtype_code(q), gate, float(scale), _ptr(q),
+                                  _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state),
+                                  _ptr(o), _stream(stream))
+    _check(st, "gdn_recurrent_step")
+    return o
+
+
+def gdn_query_device_status(workspace, stream=None) -> int:
+    """Status word of the most recent chunkwise call that used ``workspace``."""
+    return int(lib().gdn_query_device_status(_ptr(workspace), _stream(stream)))

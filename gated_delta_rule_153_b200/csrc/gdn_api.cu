@@ -1,0 +1,150 @@
+// gdn_api.cu -- the extern "C" entry points declared in include/gdn.h.
+//
+// Everything here runs on the host: argument validation (before any launch),
+// workspace sizing, and dispatch to the kernels.  Dispatch rule: bf16 with
+// dk = dv = 128 and chunk = 64 goes to the tensor-core kernels; every other
+// supported shape and GDN_F32 go to the fp32 SIMT kernels.  Both run on the
+// GPU; there is no host fallback.
+#include <math.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+using namespace gdn;
+
+namespace {
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+bool dim_ok(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
+
+gdn_status check_dims(const gdn_dims* d) {
+    if (!d) return GDN_ERR_INVALID_ARG;
+    if (d->B < 1 || d->T < 1 || d->H < 1) return GDN_ERR_INVALID_ARG;
+    if (d->chunk != 16 && d->chunk != 32 && d->chunk != 64) return GDN_ERR_INVALID_ARG;
+    if (d->dtype != GDN_BF16 && d->dtype != GDN_F32) return GDN_ERR_INVALID_ARG;
+    if (d->gate != GDN_GATE_SCALAR && d->gate != GDN_GATE_CHANNEL) return GDN_ERR_INVALID_ARG;
+    if (!isfinite(d->scale)) return GDN_ERR_INVALID_ARG;
+    // element counts must fit the kernels' 32-bit token index arithmetic
+    if ((double)d->B * d->T * d->H * 128.0 > 9.0e18) return GDN_ERR_INVALID_ARG;
+    if ((long long)d->B * d->H > 0x7fffffffLL) return GDN_ERR_INVALID_ARG;
+    if (!dim_ok(d->dk) || !dim_ok(d->dv)) return GDN_ERR_UNSUPPORTED;
+    return GDN_OK;
+}
+
+bool all_aligned(std::initializer_list<const void*> ps) {
+    for (const void* p : ps)
+        if (p && !aligned16(p)) return false;
+    return true;
+}
+
+gdn_status launch_status() {
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* gdn_status_string(gdn_status s) {
+    switch (s) {
+        case GDN_OK: return "GDN_OK";
+        case GDN_ERR_INVALID_ARG: return "GDN_ERR_INVALID_ARG";
+        case GDN_ERR_UNSUPPORTED: return "GDN_ERR_UNSUPPORTED";
+        case GDN_ERR_WORKSPACE: return "GDN_ERR_WORKSPACE";
+        case GDN_ERR_CUDA: return "GDN_ERR_CUDA";
+        case GDN_ERR_DEVICE_TIMEOUT: return "GDN_ERR_DEVICE_TIMEOUT";
+    }
+    return "GDN_UNKNOWN_STATUS";
+}
+
+size_t gdn_chunk_fwd_workspace(const gdn_dims* d) {
+    if (check_dims(d) != GDN_OK) return 0;
+    return tc_supported(*d) ? tc_fwd_workspace(*d) : simt_fwd_workspace(*d);
+}
+
+size_t gdn_chunk_bwd_workspace(const gdn_dims* d) {
+    if (check_dims(d) != GDN_OK) return 0;
+    return tc_supported(*d) ? tc_bwd_workspace(*d) : simt_bwd_workspace(*d);
+}
+
+gdn_status gdn_chunk_fwd(const gdn_dims* d, const void* q, const void* k, const void* v,
+                         const float* g, const float* beta, const float* h0, void* o,
+                         float* hT, void* ws, size_t ws_bytes, gdn_stream_t stream) {
+    gdn_status s = check_dims(d);
+    if (s != GDN_OK) return s;
+    if (!q || !k || !v || !g || !beta || !o) return GDN_ERR_INVALID_ARG;
+    if (!all_aligned({q, k, v, g, beta, h0, o, hT})) return GDN_ERR_INVALID_ARG;
+    if (h0 && hT && h0 == hT) return GDN_ERR_INVALID_ARG;
+    const size_t need = gdn_chunk_fwd_workspace(d);
+    if (ws_bytes < need || (need && !ws)) return GDN_ERR_WORKSPACE;
+    if (ws && ((uintptr_t)ws & 255u)) return GDN_ERR_WORKSPACE;
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaGetLastError();  // clear a stale error so it is not reported as ours
+    if (ws && cudaMemsetAsync(ws, 0, sizeof(unsigned int), st) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    if (tc_supported(*d)) launch_tc_fwd(*d, q, k, v, g, beta, h0, o, hT, ws, st);
+    else launch_simt_fwd(*d, q, k, v, g, beta, h0, o, hT, ws, st);
+    return launch_status();
+}
+
+gdn_status gdn_chunk_bwd(const gdn_dims* d, const void* q, const void* k, const void* v,
+                         const float* g, const float* beta, const float* h0, const void* dO,
+                         const float* dhT, void* dq, void* dk, void* dv, float* dg,
+                         float* dbeta, float* dh0, void* ws, size_t ws_bytes,
+                         gdn_stream_t stream) {
+    gdn_status s = check_dims(d);
+    if (s != GDN_OK) return s;
+    if (!q || !k || !v || !g || !beta || !dO || !dq || !dk || !dv || !dg || !dbeta)
+        return GDN_ERR_INVALID_ARG;
+    if ((h0 == nullptr) != (dh0 == nullptr)) return GDN_ERR_INVALID_ARG;
+    if (!all_aligned({q, k, v, g, beta, h0, dO, dhT, dq, dk, dv, dg, dbeta, dh0}))
+        return GDN_ERR_INVALID_ARG;
+    const size_t need = gdn_chunk_bwd_workspace(d);
+    if (ws_bytes < need || (need && !ws)) return GDN_ERR_WORKSPACE;
+    if (ws && ((uintptr_t)ws & 255u)) return GDN_ERR_WORKSPACE;
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaGetLastError();
+    if (ws && cudaMemsetAsync(ws, 0, sizeof(unsigned int), st) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    if (tc_supported(*d))
+        launch_tc_bwd(*d, q, k, v, g, beta, h0, dO, dhT, dq, dk, dv, dg, dbeta, dh0, ws, st);
+    else
+        launch_simt_bwd(*d, q, k, v, g, beta, h0, dO, dhT, dq, dk, dv, dg, dbeta, dh0, ws, st);
+    return launch_status();
+}
+
+gdn_status gdn_recurrent_step(int N, int H, int dk, int dv, gdn_dtype dtype, gdn_gate gate,
+                              float scale, const void* q, const void* k, const void* v,
+                              const float* g, const float* beta, float* state, void* o,
+                              gdn_stream_t stream) {
+    if (N < 1 || H < 1) return GDN_ERR_INVALID_ARG;
+    if ((long long)N * H > 0x7fffffffLL) return GDN_ERR_INVALID_ARG;
+    if (dtype != GDN_BF16 && dtype != GDN_F32) return GDN_ERR_INVALID_ARG;
+    if (gate != GDN_GATE_SCALAR && gate != GDN_GATE_CHANNEL) return GDN_ERR_INVALID_ARG;
+    if (!isfinite(scale)) return GDN_ERR_INVALID_ARG;
+    if (!q || !k || !v || !g || !beta || !state || !o) return GDN_ERR_INVALID_ARG;
+    if (!all_aligned({q, k, v, g, beta, state, o})) return GDN_ERR_INVALID_ARG;
+    if (!dim_ok(dk) || !dim_ok(dv)) return GDN_ERR_UNSUPPORTED;
+    cudaGetLastError();
+    launch_recurrent_step(N, H, dk, dv, dtype, gate, scale, q, k, v, g, beta, state, o,
+                          (cudaStream_t)stream);
+    return launch_status();
+}
+
+gdn_status gdn_query_device_status(void* ws, gdn_stream_t stream) {
+    if (!ws) return GDN_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return GDN_ERR_CUDA;
+    unsigned int word = 0;
+    if (cudaMemcpy(&word, ws, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    if (word == 0) return GDN_OK;
+    const unsigned int zero = 0;
+    if (cudaMemcpy(ws, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    return GDN_ERR_DEVICE_TIMEOUT;
+}
+
+}  // extern "C"

@@ -1,0 +1,39 @@
+// internal.h -- launchers shared between the C ABI layer and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+#include "../../include/gdn.h"
+
+namespace gdn {
+
+void launch_recurrent_step(int N, int H, int dk, int dv, gdn_dtype dtype, gdn_gate gate,
+                           float scale, const void* q, const void* k, const void* v,
+                           const float* g, const float* beta, float* state, void* o,
+                           cudaStream_t st);
+
+// Generic fp32-arithmetic chunkwise path (any supported dims, both dtypes).
+size_t simt_fwd_workspace(const gdn_dims& d);
+size_t simt_bwd_workspace(const gdn_dims& d);
+void launch_simt_fwd(const gdn_dims& d, const void* q, const void* k, const void* v,
+                     const float* g, const float* beta, const float* h0, void* o, float* hT,
+                     void* ws, cudaStream_t st);
+void launch_simt_bwd(const gdn_dims& d, const void* q, const void* k, const void* v,
+                     const float* g, const float* beta, const float* h0, const void* dO,
+                     const float* dhT, void* dq, void* dk, void* dv, float* dg, float* dbeta,
+                     float* dh0, void* ws, cudaStream_t st);
+
+// Tensor-core path (bf16, dk = dv = 128, chunk = 64).
+bool tc_supported(const gdn_dims& d);
+size_t tc_fwd_workspace(const gdn_dims& d);
+size_t tc_bwd_workspace(const gdn_dims& d);
+void launch_tc_fwd(const gdn_dims& d, const void* q, const void* k, const void* v,
+                   const float* g, const float* beta, const float* h0, void* o, float* hT,
+                   void* ws, cudaStream_t st);
+void launch_tc_bwd(const gdn_dims& d, const void* q, const void* k, const void* v,
+                   const float* g, const float* beta, const float* h0, const void* dO,
+                   const float* dhT, void* dq, void* dk, void* dv, float* dg, float* dbeta,
+                   float* dh0, void* ws, cudaStream_t st);
+
+}  // namespace gdn

@@ -124,13 +124,22 @@ def make_decode_inputs(cfg: DecodeConfig, steps: Optional[int] = None, **over) -
     N, H, dk, dv = cfg.N, cfg.H, cfg.dk, cfg.dv
     dt = _DT[cfg.dtype]
     s = cfg.seed
-    q = _l2norm(torch.randn(S, N, H, dk, generator=_gen(s, 0))).to(dt)
-    k = _l2norm(torch.randn(S, N, H, dk, generator=_gen(s, 1))).to(dt)
-    v = torch.randn(S, N, H, dv, generator=_gen(s, 2)).to(dt)
-    gshape = (S, N, H, dk) if cfg.gate == "channel" else (S, N, H)
-    g = -torch.nn.functional.softplus(
-        torch.randn(*gshape, generator=_gen(s, 3)) + cfg.g_shift)
-    beta = torch.sigmoid(torch.randn(S, N, H, generator=_gen(s, 4)))
-    state0 = torch.randn(N, H, dv, dk, generator=_gen(s, 5)) * cfg.state_std
+    gens = [_gen(s, i) for i in range(6)]
+    gshape = (N, H, dk) if cfg.gate == "channel" else (N, H)
+    q = torch.empty(S, N, H, dk, dtype=dt)
+    k = torch.empty(S, N, H, dk, dtype=dt)
+    v = torch.empty(S, N, H, dv, dtype=dt)
+    g = torch.empty(S, *gshape)
+    beta = torch.empty(S, N, H)
+    blk = 25  # steps drawn per block, to bound host memory at full size
+    for t0 in range(0, S, blk):
+        n = min(blk, S - t0)
+        q[t0:t0 + n] = _l2norm(torch.randn(n, N, H, dk, generator=gens[0])).to(dt)
+        k[t0:t0 + n] = _l2norm(torch.randn(n, N, H, dk, generator=gens[1])).to(dt)
+        v[t0:t0 + n] = torch.randn(n, N, H, dv, generator=gens[2]).to(dt)
+        g[t0:t0 + n] = -torch.nn.functional.softplus(
+            torch.randn(n, *gshape, generator=gens[3]) + cfg.g_shift)
+        beta[t0:t0 + n] = torch.sigmoid(torch.randn(n, N, H, generator=gens[4]))
+    state0 = torch.randn(N, H, dv, dk, generator=gens[5]) * cfg.state_std
     return dict(q=q, k=k, v=v, g=g.contiguous(), beta=beta.contiguous(),
                 state0=state0, cfg=cfg)

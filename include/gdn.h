@@ -1,0 +1,136 @@
+/*
+ * gdn.h -- C ABI of the gated delta-rule layer library (libgdn.so, sm_100a).
+ *
+ * The operation.  "Gated Delta Networks: Improving Mamba2 with Delta Rule"
+ * (paper review), section "Method": per (sequence b, head h) a matrix state
+ * S in R^{dv x dk} is updated token by token as
+ *
+ *     S_t = S_{t-1} a_t (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,   a_t = exp(g_t),
+ *
+ * and read out as o_t = S_t (scale * q_t).  GDN_GATE_SCALAR takes one log-gate
+ * g_t per (token, head); GDN_GATE_CHANNEL (the Kimi-Delta-Attention variant,
+ * named in the same review's linked reviews and in the "Linear Attention
+ * Architectures: Mechanisms, Trade-offs, and Cross-Layer Routing" abstract)
+ * takes g_t in R^{dk} and uses Diag(a_t) on the key index in place of a_t.
+ * The training calls compute the same values in the chunkwise-parallel form
+ * built on the WY representation and the UT transform (same review, sections
+ * "Goal" and "Method"); the decode call is the recurrent form, one token per
+ * call ("Background": O(1)-memory inference with a fixed-size state).
+ *
+ * Layouts (all row-major and contiguous; element strides are implied):
+ *   q, k          [B, T, H, dk]      q/k/v/o/dO/dq/dk/dv in `dtype`
+ *   v, o          [B, T, H, dv]
+ *   g             [B, T, H] (scalar gate) or [B, T, H, dk] (channel gate), fp32
+ *   beta          [B, T, H] fp32
+ *   h0, hT, dhT, dh0   [B, H, dv, dk] fp32 (row = value index, column = key index)
+ * Gradients come back in the dtype of their primal; dg, dbeta, dh0 are fp32.
+ *
+ * Precision.  GDN_BF16: bf16 inputs/outputs, fp32 accumulation, fp32 gate
+ * cumsums and an fp32 state.  GDN_F32: fp32 end to end (no tf32).
+ *
+ * Ownership and streams.  The caller owns every buffer, the workspace
+ * included.  The library never allocates, frees or synchronises (except
+ * gdn_query_device_status), keeps no state between calls, and enqueues all
+ * work on the stream it is given.  All pointers other than the host-side
+ * `dims` are device pointers.
+ *
+ * Errors.  Every argument is validated on the host before any launch; on
+ * error nothing is launched and the outputs are untouched:
+ *   GDN_ERR_INVALID_ARG  null required pointer, B/T/H < 1, bad enum, pointer
+ *                        not 16-byte aligned, dh0 given without h0 or the
+ *                        reverse, chunk not in {16, 32, 64}, scale not finite;
+ *   GDN_ERR_UNSUPPORTED  dk or dv not in {16, 32, 64, 128};
+ *   GDN_ERR_WORKSPACE    ws_bytes smaller than the *_workspace() size, or a
+ *                        null workspace when that size is non-zero;
+ *   GDN_ERR_CUDA         a launch failed (cudaGetLastError after launch).
+ * Value preconditions are documented, not checked: g finite and <= 0,
+ * beta in [0, 1] (the range the chunkwise algebra is tested on).
+ */
+#ifndef GDN_H
+#define GDN_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as the CUDA runtime's cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st *gdn_stream_t;
+
+typedef enum {
+    GDN_OK = 0,
+    GDN_ERR_INVALID_ARG = 1,
+    GDN_ERR_UNSUPPORTED = 2,
+    GDN_ERR_WORKSPACE = 3,
+    GDN_ERR_CUDA = 4,
+    GDN_ERR_DEVICE_TIMEOUT = 5
+} gdn_status;
+
+typedef enum { GDN_BF16 = 0, GDN_F32 = 1 } gdn_dtype;
+typedef enum { GDN_GATE_SCALAR = 0, GDN_GATE_CHANNEL = 1 } gdn_gate;
+
+/* Problem description shared by the chunkwise calls.
+ * chunk: tokens per chunk of the chunkwise algorithm (16, 32 or 64); the
+ * result does not depend on it beyond rounding.  T need not be a multiple of
+ * chunk (the tail chunk is shorter).  scale multiplies q (1 = o_t = S_t q_t). */
+typedef struct {
+    int B, T, H, dk, dv, chunk;
+    gdn_dtype dtype;
+    gdn_gate gate;
+    float scale;
+} gdn_dims;
+
+/* Bytes of device workspace gdn_chunk_fwd needs for `dims` (0 if dims are
+ * invalid).  The workspace must be 256-byte aligned. */
+size_t gdn_chunk_fwd_workspace(const gdn_dims *dims);
+
+/* Chunkwise forward.  Reads q, k, v, g, beta and, if not NULL, the initial
+ * state h0 (NULL = zero state).  Writes o and, if not NULL, the final state
+ * hT.  h0 and hT may not alias.  Chunkwise algorithm: per chunk the gate
+ * cumsum, the decayed K K^T, the UT transform T = (I + A)^{-1}, the WY
+ * factors, the inter-chunk fp32 state recurrence and the output products. */
+gdn_status gdn_chunk_fwd(const gdn_dims *dims, const void *q, const void *k,
+                         const void *v, const float *g, const float *beta,
+                         const float *h0, void *o, float *hT, void *ws,
+                         size_t ws_bytes, gdn_stream_t stream);
+
+/* Bytes of device workspace gdn_chunk_bwd needs for `dims`. */
+size_t gdn_chunk_bwd_workspace(const gdn_dims *dims);
+
+/* Chunkwise backward of L = <dO, o> + <dhT, hT> (dhT NULL = 0).  The call is
+ * stateless: it recomputes what it needs from the primal inputs.  Writes dq,
+ * dk, dv (primal dtype), dg (shape of g), dbeta, and dh0 (required exactly
+ * when h0 is given; NULL otherwise). */
+gdn_status gdn_chunk_bwd(const gdn_dims *dims, const void *q, const void *k,
+                         const void *v, const float *g, const float *beta,
+                         const float *h0, const void *dO, const float *dhT,
+                         void *dq, void *dk, void *dv, float *dg, float *dbeta,
+                         float *dh0, void *ws, size_t ws_bytes,
+                         gdn_stream_t stream);
+
+/* One decode token for N sequences x H heads, in place on the state.
+ * q, k [N, H, dk]; v, o [N, H, dv] in `dtype`; g [N, H] (scalar) or
+ * [N, H, dk] (channel) fp32; beta [N, H] fp32; state [N, H, dv, dk] fp32,
+ * read once and written once.  o_t uses the updated state. */
+gdn_status gdn_recurrent_step(int N, int H, int dk, int dv, gdn_dtype dtype,
+                              gdn_gate gate, float scale, const void *q,
+                              const void *k, const void *v, const float *g,
+                              const float *beta, float *state, void *o,
+                              gdn_stream_t stream);
+
+/* Synchronises `stream`, then reads and clears the status word kept in the
+ * first bytes of a chunkwise workspace.  Each chunkwise call clears that word
+ * (a 4-byte memset on its stream) before its kernels run, and a kernel whose
+ * bounded device wait gives up sets it, so the answer covers the most recent
+ * call on `ws`: GDN_ERR_DEVICE_TIMEOUT if a wait gave up, else GDN_OK. */
+gdn_status gdn_query_device_status(void *ws, gdn_stream_t stream);
+
+/* Static, human-readable name of a status code. */
+const char *gdn_status_string(gdn_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H */

@@ -1,0 +1,115 @@
+"""The C-ABI library loads, exports every symbol include/gdn.h declares, and
+rejects bad arguments on the host before touching the device (CPU only)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import gated_delta_rule_153_b200 as gdn
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for f in os.listdir(os.path.join(ROOT, "include")):
+        if f.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", f)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names |= set(re.findall(r"\b(gdn_[a-z_0-9]+)\s*\(", src))
+    return names
+
+
+def test_exports_every_declared_symbol():
+    L = gdn.lib()
+    declared = _declared()
+    assert declared, "no declarations found"
+    assert declared == set(gdn.EXPORTS)
+    for name in declared:
+        assert hasattr(L, name), name
+
+
+def _dims(**kw):
+    d = dict(B=1, T=64, H=2, dk=128, dv=128, chunk=64, dtype=gdn.GDN_BF16,
+             gate=gdn.GDN_GATE_SCALAR, scale=1.0)
+    d.update(kw)
+    return gdn.gdn_dims(**d)
+
+
+def test_status_strings():
+    assert gdn.status_string(gdn.GDN_OK) == "GDN_OK"
+    assert gdn.status_string(gdn.GDN_ERR_DEVICE_TIMEOUT) == "GDN_ERR_DEVICE_TIMEOUT"
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(B=0), gdn.GDN_ERR_INVALID_ARG), (dict(T=0), gdn.GDN_ERR_INVALID_ARG),
+    (dict(H=-1), gdn.GDN_ERR_INVALID_ARG), (dict(chunk=48), gdn.GDN_ERR_INVALID_ARG),
+    (dict(dtype=7), gdn.GDN_ERR_INVALID_ARG), (dict(gate=3), gdn.GDN_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), gdn.GDN_ERR_INVALID_ARG),
+    (dict(dk=96), gdn.GDN_ERR_UNSUPPORTED), (dict(dv=256), gdn.GDN_ERR_UNSUPPORTED),
+])
+def test_dims_rejected_before_launch(kw, code):
+    L = gdn.lib()
+    d = _dims(**kw)
+    p = ctypes.c_void_p(256)  # never dereferenced: validation fails first
+    assert L.gdn_chunk_fwd_workspace(ctypes.byref(d)) == 0
+    st = L.gdn_chunk_fwd(ctypes.byref(d), p, p, p, p, p, None, p, None, p, 1 << 40, None)
+    assert st == code
+    st = L.gdn_chunk_bwd(ctypes.byref(d), p, p, p, p, p, None, p, None, p, p, p, p, p, None,
+                         p, 1 << 40, None)
+    assert st == code
+
+
+def test_pointer_checks():
+    L = gdn.lib()
+    d = _dims()
+    p = ctypes.c_void_p(256)
+    mis = ctypes.c_void_p(258)
+    ws = ctypes.c_void_p(1 << 20)
+    big = 1 << 40
+    # null required pointer
+    assert L.gdn_chunk_fwd(ctypes.byref(d), None, p, p, p, p, None, p, None, ws, big,
+                           None) == gdn.GDN_ERR_INVALID_ARG
+    # misaligned pointer
+    assert L.gdn_chunk_fwd(ctypes.byref(d), p, mis, p, p, p, None, p, None, ws, big,
+                           None) == gdn.GDN_ERR_INVALID_ARG
+    # h0 aliasing hT
+    assert L.gdn_chunk_fwd(ctypes.byref(d), p, p, p, p, p, p, p, p, ws, big,
+                           None) == gdn.GDN_ERR_INVALID_ARG
+    # workspace too small / missing / misaligned
+    need = L.gdn_chunk_fwd_workspace(ctypes.byref(d))
+    assert need > 0
+    assert L.gdn_chunk_fwd(ctypes.byref(d), p, p, p, p, p, None, p, None, ws, need - 1,
+                           None) == gdn.GDN_ERR_WORKSPACE
+    assert L.gdn_chunk_fwd(ctypes.byref(d), p, p, p, p, p, None, p, None, None, big,
+                           None) == gdn.GDN_ERR_WORKSPACE
+    assert L.gdn_chunk_fwd(ctypes.byref(d), p, p, p, p, p, None, p, None,
+                           ctypes.c_void_p((1 << 20) + 16), big, None) == gdn.GDN_ERR_WORKSPACE
+    # dh0 given without h0 (and the reverse)
+    assert L.gdn_chunk_bwd(ctypes.byref(d), p, p, p, p, p, None, p, None, p, p, p, p, p, p,
+                           ws, big, None) == gdn.GDN_ERR_INVALID_ARG
+    assert L.gdn_chunk_bwd(ctypes.byref(d), p, p, p, p, p, p, p, None, p, p, p, p, p, None,
+                           ws, big, None) == gdn.GDN_ERR_INVALID_ARG
+
+
+def test_decode_checks():
+    L = gdn.lib()
+    p = ctypes.c_void_p(256)
+    assert L.gdn_recurrent_step(0, 16, 128, 128, 0, 0, 1.0, p, p, p, p, p, p, p,
+                                None) == gdn.GDN_ERR_INVALID_ARG
+    assert L.gdn_recurrent_step(4, 16, 100, 128, 0, 0, 1.0, p, p, p, p, p, p, p,
+                                None) == gdn.GDN_ERR_UNSUPPORTED
+    assert L.gdn_recurrent_step(4, 16, 128, 128, 0, 0, 1.0, p, p, p, p, p, None, p,
+                                None) == gdn.GDN_ERR_INVALID_ARG
+    assert L.gdn_recurrent_step(4, 16, 128, 128, 0, 5, 1.0, p, p, p, p, p, p, p,
+                                None) == gdn.GDN_ERR_INVALID_ARG
+    assert L.gdn_query_device_status(None, None) == gdn.GDN_ERR_INVALID_ARG
+
+
+def test_workspace_sizes_grow_with_problem():
+    L = gdn.lib()
+    a = L.gdn_chunk_bwd_workspace(ctypes.byref(_dims(T=64)))
+    b = L.gdn_chunk_bwd_workspace(ctypes.byref(_dims(T=4096)))
+    assert 0 < a < b
+    assert L.gdn_chunk_fwd_workspace(ctypes.byref(_dims(T=64))) % 4 == 0

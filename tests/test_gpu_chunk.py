@@ -1,0 +1,131 @@
+"""GPU parity of gdn_chunk_fwd / gdn_chunk_bwd against the fp64 oracle, on
+seeded inputs shaped like the layer's workloads, plus invariants that hold at
+any size (chunk-size invariance, resume, Euler identities, determinism)."""
+import numpy as np
+import pytest
+import torch
+
+from gated_delta_rule_153_b200.inputs import KDA, L350M, LONG, TINY, make_chunk_inputs
+from tests.parity import TOL, check_bwd, check_fwd, gpu_bwd, gpu_fwd, rel_err
+
+pytestmark = pytest.mark.gpu
+
+
+# ---- the small fp32 case (tolerance 1e-4) ---------------------------------
+def test_tiny_fwd(dev):
+    check_fwd(make_chunk_inputs(TINY), dev)
+
+
+def test_tiny_fwd_bwd_with_states(dev):
+    inp = make_chunk_inputs(TINY, h0_std=0.5, dhT_std=1.0)
+    check_fwd(inp, dev)
+    check_bwd(inp, dev)
+
+
+@pytest.mark.parametrize("dk,dv,T,C,gate", [
+    (16, 16, 1, 16, "scalar"), (16, 32, 7, 16, "scalar"), (32, 16, 100, 32, "channel"),
+    (64, 64, 130, 64, "scalar"), (128, 64, 77, 16, "channel"), (128, 128, 200, 64, "scalar"),
+    (128, 128, 129, 64, "channel"), (64, 128, 65, 32, "scalar"),
+])
+def test_f32_shapes_ragged(dev, dk, dv, T, C, gate):
+    inp = make_chunk_inputs(TINY, B=2, H=3, T=T, dk=dk, dv=dv, chunk=C, gate=gate,
+                            g_shift=-1.0, h0_std=0.3, dhT_std=0.5, seed=77 + T)
+    check_fwd(inp, dev)
+    check_bwd(inp, dev)
+
+
+# ---- bf16 at the layer's shapes (tolerance 2e-2) ---------------------------
+@pytest.mark.parametrize("dk,dv,T,gate", [(64, 64, 300, "scalar"), (32, 128, 97, "channel")])
+def test_bf16_small_dims(dev, dk, dv, T, gate):
+    inp = make_chunk_inputs(L350M, B=2, H=2, T=T, dk=dk, dv=dv, gate=gate, h0_std=0.1,
+                            dhT_std=0.3, seed=5 + T)
+    check_fwd(inp, dev)
+    check_bwd(inp, dev)
+
+
+def test_350m_fwd_bwd(dev):
+    inp = make_chunk_inputs(L350M)
+    check_fwd(inp, dev)
+    check_bwd(inp, dev)
+
+
+def test_long_context_fwd_bwd(dev):
+    inp = make_chunk_inputs(LONG)
+    check_fwd(inp, dev)
+    check_bwd(inp, dev)
+
+
+def test_kda_fwd_bwd(dev):
+    inp = make_chunk_inputs(KDA, B=1, H=8)
+    check_fwd(inp, dev)
+    check_bwd(inp, dev)
+
+
+@pytest.mark.parametrize("cfg,over", [
+    (L350M, dict(B=2, g_shift=-6.0, h0_std=0.1, dhT_std=0.5)),
+    (LONG, dict(H=4, g_shift=-6.0)),
+    (KDA, dict(B=1, H=4, T=1024, g_shift=-6.0, h0_std=0.1)),
+])
+def test_slow_gate_keeps_state_path_alive(dev, cfg, over):
+    """Gates near 1 so the inter-chunk state (and h0) matter for o."""
+    inp = make_chunk_inputs(cfg, **over)
+    check_fwd(inp, dev)
+    check_bwd(inp, dev)
+
+
+def test_zero_gate_small_beta(dev):
+    inp = make_chunk_inputs(L350M, B=1, H=4, T=512, h0_std=0.1)
+    inp["g"] = torch.zeros_like(inp["g"])
+    inp["beta"] = inp["beta"] * 0.05
+    check_fwd(inp, dev)
+    check_bwd(inp, dev)
+
+
+# ---- invariants -----------------------------------------------------------
+def test_chunk_size_invariance(dev):
+    inp = make_chunk_inputs(L350M, B=1, H=4, T=1000, dtype="f32", g_shift=-2.0, h0_std=0.2)
+    outs = [gpu_fwd(inp, dev, chunk=c) for c in (16, 32, 64)]
+    for o, hT in outs[1:]:
+        assert rel_err(o, outs[0][0].double().cpu().numpy()) < 1e-5
+        assert rel_err(hT, outs[0][1].double().cpu().numpy()) < 1e-5
+
+
+def test_resume_from_final_state(dev):
+    inp = make_chunk_inputs(L350M, B=2, H=4, T=768, g_shift=-3.0, h0_std=0.2)
+    o_full, h_full = gpu_fwd(inp, dev)
+    a = {n: (inp[n][:, :320] if n in ("q", "k", "v", "g", "beta") else inp[n]) for n in inp}
+    b = {n: (inp[n][:, 320:] if n in ("q", "k", "v", "g", "beta") else inp[n]) for n in inp}
+    a = {n: (x.contiguous() if torch.is_tensor(x) else x) for n, x in a.items()}
+    b = {n: (x.contiguous() if torch.is_tensor(x) else x) for n, x in b.items()}
+    oa, ha = gpu_fwd(a, dev)
+    b["h0"] = ha.cpu()
+    ob, hb = gpu_fwd(b, dev)
+    o_cat = torch.cat([oa, ob], 1)
+    assert rel_err(o_cat, o_full.double().cpu().numpy()) < 2e-2
+    assert rel_err(hb, h_full.double().cpu().numpy()) < 2e-2
+
+
+def test_euler_identities_full_size(dev):
+    """o, hT linear in (v, h0) and o linear in q:
+    <dv,v> + <dh0,h0> = <dO,o> + <dhT,hT>,  <dq,q> = <dO,o>."""
+    inp = make_chunk_inputs(LONG)
+    o, hT = gpu_fwd(inp, dev)
+    r = gpu_bwd(inp, dev)
+    f = lambda x: x.double().cpu()
+    dOo = float((f(inp["dO"]) * f(o)).sum())
+    rhs = dOo + float((f(inp["dhT"]) * f(hT)).sum())
+    lhs = float((f(r["dv"]) * f(inp["v"])).sum() + (f(r["dh0"]) * f(inp["h0"])).sum())
+    scale = float(f(inp["dO"]).abs().sum() * f(o).abs().max())
+    assert abs(lhs - rhs) <= 2e-2 * scale, (lhs, rhs)
+    lq = float((f(r["dq"]) * f(inp["q"])).sum())
+    assert abs(lq - dOo) <= 2e-2 * scale, (lq, dOo)
+
+
+def test_deterministic(dev):
+    inp = make_chunk_inputs(L350M, B=2, H=2, T=512)
+    o1, h1 = gpu_fwd(inp, dev)
+    o2, h2 = gpu_fwd(inp, dev)
+    assert torch.equal(o1, o2) and torch.equal(h1, h2)
+    r1, r2 = gpu_bwd(inp, dev), gpu_bwd(inp, dev)
+    for n in ("dq", "dk", "dv", "dg", "dbeta"):
+        assert torch.equal(r1[n], r2[n]), n
