@@ -1,0 +1,443 @@
+"""Benchmark of the gated delta-rule layer library on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one training pass of the layer over one batch of the 350M-scale
+workload (B=8, H=8, T=2048, d_k=d_v=128, chunk 64, bf16 q/k/v, fp32 gates and
+state): gdn_chunk_fwd then gdn_chunk_bwd, i.e. the gate cumsum, the decayed
+K K^T, the UT transform, the WY factors, the inter-chunk state recurrence,
+the outputs, the reverse state pass and the local gradients.  The headline
+value is tokens/s (B*T tokens per step, all heads) with inputs resident in
+HBM; the same line reports TFLOP/s against the tensor peak, the long-context
+forward (B=1, H=16, T=8192), the decode step (256 x 16 heads, 1000 steps,
+HBM GB/s), the channel-gate workload (B=2, H=32, T=4096), an end-to-end number
+through host buffers, the roofline of the dominant kernel, and the fp64 CPU
+oracle timed on this host as a baseline.
+
+With N > 1 (torchrun) every rank runs its own copy of the workload with a
+different seed (independent batches, no collective on the data path); value
+is the tokens of all ranks over the slowest rank's time (weak scaling).
+All inputs are synthetic (seeded generators, no datasets or weights).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = ("gated-delta-rule fwd+bwd tokens/s and TFLOP/s (% tensor peak); "
+          "decode HBM GB/s")
+
+# Algorithmic work per token-head at C=64, d_k=d_v=128 (triangular products
+# count half, recompute is not counted, the C^3 solve counts C^3/3 per chunk).
+FWD_FLOP = 140_629
+BWD_FLOP = 281_259
+FWD_BYTES = 1032      # q,k,v,o bf16 + g,beta fp32
+BWD_BYTES = 1808      # q,k,v,dO read; dq,dk,dv written; g,beta,dg,dbeta
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"],
+                    bf16_sustained=d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                    source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+# Per-kernel algorithmic traffic / work per launch for the roofline object.
+# Bytes are the unique bytes each kernel must read and write (inputs, its
+# workspace products, outputs); flops are its tensor-core products.
+def kernel_work(name, B, T, H):
+    th = B * T * H           # token-heads
+    nchunks = B * H * ((T + 63) // 64)
+    if name == "tc_prep":
+        # reads q,k,v (bf16), g, beta; writes W, U~ (bf16 C x 128), P (bf16 C x C), G
+        return dict(bound="hbm", bytes=th * (3 * 256 + 8 + 2 * 256 + 128 + 4))
+    if name in ("tc_walk_fwd",):
+        # reads W, Q, K, U~ (bf16), P, G; writes O
+        return dict(bound="hbm", bytes=th * (4 * 256 + 128 + 4 + 256))
+    if name in ("tc_walk_states",):
+        # reads W, K, U~, G; writes S0 per chunk (bf16) and U
+        return dict(bound="hbm", bytes=th * (3 * 256 + 4 + 256) + nchunks * 128 * 128 * 2)
+    if name == "tc_walk_bwd":
+        # reads P, dO, Q, K, W, G; writes dS per chunk (bf16), dU
+        return dict(bound="hbm", bytes=th * (128 + 4 * 256 + 4 + 256) + nchunks * 128 * 128 * 2)
+    if name == "tc_bwd_local":
+        # reads q,k,v,dO,U,dU (bf16), S0, dS per chunk, g, beta; writes dq,dk,dv, dg, dbeta
+        return dict(bound="hbm", bytes=th * (6 * 256 + 8 + 3 * 256 + 8)
+                    + nchunks * 2 * 128 * 128 * 2)
+    if name == "simt_bwd":
+        return dict(bound="hbm", bytes=th * BWD_BYTES)
+    if name == "simt_fwd":
+        return dict(bound="hbm", bytes=th * FWD_BYTES)
+    if name == "decode_step":
+        return dict(bound="hbm", bytes=B * H * (2 * 128 * 128 * 4 + 4 * 256 + 8))
+    return dict(bound="hbm", bytes=th * FWD_BYTES)
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason sampling during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, dev_index):
+        self.proc = None
+        self.dev = dev_index
+
+    def __enter__(self):
+        try:
+            ident = str(self.dev)
+            try:
+                uuid = str(torch.cuda.get_device_properties(self.dev).uuid)
+                ident = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            except Exception:
+                pass
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", ident, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.rows = []
+        if self.proc is None:
+            return
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out = ""
+        for line in out.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9:
+                self.rows.append(parts)
+
+    def summary(self):
+        if not getattr(self, "rows", None):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in self.rows if num(r[1])]
+        power = [num(r[3]) for r in self.rows if num(r[3])]
+        load = [s for s, p in zip(sm, power)] if sm else []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in self.rows for i in range(4)
+                          if r[5 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(load) if load else None,
+                "sm_max_mhz": num(self.rows[0][2]), "power_w_max": max(power) if power else None,
+                "samples": len(self.rows), "reasons": reasons}
+
+
+def timed(fn, steps, warmup, barrier=lambda: None):
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(steps):
+        fn()
+    e.record()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    return s.elapsed_time(e) / steps
+
+
+def chunk_step_fn(gdn, d, ws_f, ws_b, outs):
+    def step():
+        o, hT = gdn.gdn_chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["h0"],
+                                  o=outs["o"], hT=outs["hT"], workspace=ws_f)
+        gdn.gdn_chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["dO"], d["h0"],
+                          d["dhT"], workspace=ws_b)
+    return step
+
+
+def to_dev(inp, dev):
+    return {n: (x.to(dev) if torch.is_tensor(x) else x) for n, x in inp.items()}
+
+
+def workspaces(gdn, d):
+    dims = gdn.make_dims(d["q"], d["v"], d["g"])
+    wf = torch.empty(max(gdn.gdn_chunk_fwd_workspace(dims), 256), dtype=torch.uint8,
+                     device=d["q"].device)
+    wb = torch.empty(max(gdn.gdn_chunk_bwd_workspace(dims), 256), dtype=torch.uint8,
+                     device=d["q"].device)
+    return wf, wb
+
+
+def run_ours(args, rank, world, dev, barrier, max_over_ranks):
+    import gated_delta_rule_153_b200 as gdn
+    from gated_delta_rule_153_b200.inputs import DECODE, KDA, L350M, LONG, \
+        make_chunk_inputs, make_decode_inputs
+
+    pk = peaks()
+    cfg = L350M
+    inp = make_chunk_inputs(cfg, seed=cfg.seed + 7919 * rank)
+    d = to_dev(inp, dev)
+    outs = dict(o=torch.empty_like(d["v"]),
+                hT=torch.empty(cfg.B, cfg.H, cfg.dv, cfg.dk, device=dev))
+    ws_f, ws_b = workspaces(gdn, d)
+    step = chunk_step_fn(gdn, d, ws_f, ws_b, outs)
+
+    # ---- headline: fwd+bwd steps, inputs resident in HBM -------------------
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    cap = 64 * max(args.steps, 1)
+    idx = torch.cuda.current_device()
+    with ClockSampler(idx) as clk:
+        barrier()
+        torch.cuda.synchronize()
+        gdn.gdn_profile_begin(cap)
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        for _ in range(args.steps):
+            step()
+        e.record()
+        torch.cuda.synchronize()
+        nlaunch, launches = gdn.gdn_profile_end(cap)
+        barrier()
+        torch.cuda.synchronize()
+    ms_total = s.elapsed_time(e)
+    ms_total = max_over_ranks(ms_total)
+    ms_step = ms_total / args.steps
+    tokens = cfg.B * cfg.T
+    value = world * tokens * args.steps / (ms_total / 1e3)
+    th = cfg.B * cfg.T * cfg.H
+    flops_step = (FWD_FLOP + BWD_FLOP) * th
+    tflops = world * flops_step * args.steps / (ms_total / 1e3) / 1e12
+
+    # ---- roofline of the dominant kernel ------------------------------------
+    per = {}
+    for name, ms in launches:
+        per.setdefault(name, []).append(ms)
+    total_k = sum(sum(v) for v in per.values())
+    dom = max(per, key=lambda n: sum(per[n]))
+    dom_ms = statistics.mean(per[dom])
+    wk = kernel_work(dom, cfg.B, cfg.T, cfg.H)
+    achieved = wk["bytes"] / (dom_ms / 1e3) / 1e9
+    roofline = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1),
+                "peak": pk["hbm"], "unit": "GB/s", "frac": round(achieved / pk["hbm"], 4),
+                "peak_source": pk["source"], "traffic": None,
+                "avg_launch_ms": round(dom_ms, 4),
+                "share": round(sum(per[dom]) / total_k, 4),
+                "kernels": {n: {"launches": len(v), "avg_ms": round(statistics.mean(v), 4),
+                                "share": round(sum(v) / total_k, 4)} for n, v in per.items()}}
+
+    extra = {}
+    if not args.headline_only:
+        # ---- long-context forward (the 50%-of-tensor-peak target) ----------
+        li = to_dev(make_chunk_inputs(LONG, seed=LONG.seed + 7919 * rank), dev)
+        lws_f, _ = workspaces(gdn, li)
+        lo = torch.empty_like(li["v"])
+        lh = torch.empty(LONG.B, LONG.H, LONG.dv, LONG.dk, device=dev)
+        fwd = lambda: gdn.gdn_chunk_fwd(li["q"], li["k"], li["v"], li["g"], li["beta"], li["h0"],
+                                        o=lo, hT=lh, workspace=lws_f)
+        ms_f = timed(fwd, max(args.steps, 10), args.warmup, barrier)
+        lth = LONG.B * LONG.T * LONG.H
+        lt = FWD_FLOP * lth / (ms_f / 1e3) / 1e12
+        extra["long_context_fwd"] = {
+            "workload": LONG.name, "ms": round(ms_f, 4),
+            "tokens_per_s": round(LONG.B * LONG.T / (ms_f / 1e3), 1),
+            "tflops": round(lt, 2), "frac_tensor_peak": round(lt / pk["bf16"], 4),
+            "hbm_gbs": round(FWD_BYTES * lth / (ms_f / 1e3) / 1e9, 1)}
+        ms_fb = timed(chunk_step_fn(gdn, li, lws_f, workspaces(gdn, li)[1],
+                                    dict(o=lo, hT=lh)), 3, 1, barrier)
+        extra["long_context_fwd_bwd_ms"] = round(ms_fb, 3)
+        del li, lws_f
+        # ---- channel gate (KDA) fwd+bwd -------------------------------------
+        ki = to_dev(make_chunk_inputs(KDA, seed=KDA.seed + 7919 * rank), dev)
+        kws_f, kws_b = workspaces(gdn, ki)
+        ko = dict(o=torch.empty_like(ki["v"]), hT=None)
+        ms_k = timed(chunk_step_fn(gdn, ki, kws_f, kws_b, ko), 3, 1, barrier)
+        kth = KDA.B * KDA.T * KDA.H
+        extra["kda_fwd_bwd"] = {"workload": KDA.name, "ms": round(ms_k, 3),
+                                "tokens_per_s": round(KDA.B * KDA.T / (ms_k / 1e3), 1),
+                                "tflops": round((FWD_FLOP + BWD_FLOP) * kth / (ms_k / 1e3) / 1e12, 2)}
+        del ki, kws_f, kws_b
+        # ---- decode: 1000 successive single-token steps --------------------
+        dec = make_decode_inputs(DECODE, seed=DECODE.seed + 7919 * rank)
+        dd = to_dev(dec, dev)
+        st = dd["state0"].clone()
+        o = torch.empty(DECODE.N, DECODE.H, DECODE.dv, dtype=torch.bfloat16, device=dev)
+        S = DECODE.steps
+
+        def dec_run():
+            for t in range(S):
+                gdn.gdn_recurrent_step(dd["q"][t], dd["k"][t], dd["v"][t], dd["g"][t],
+                                       dd["beta"][t], st, o=o)
+        ms_d = timed(dec_run, 1, 1, barrier) / S
+        dbytes = DECODE.N * DECODE.H * (2 * DECODE.dv * DECODE.dk * 4 + 4 * 128 * 2 + 8)
+        gbs = dbytes / (ms_d / 1e3) / 1e9
+        extra["decode"] = {"workload": DECODE.name, "us_per_step": round(ms_d * 1e3, 2),
+                           "hbm_gbs": round(gbs, 1), "frac_hbm_peak": round(gbs / pk["hbm"], 4),
+                           "bytes_per_step": dbytes}
+        del dd, dec
+
+    # ---- end to end through host buffers ------------------------------------
+    names_in = ("q", "k", "v", "g", "beta", "dO")
+    host = {n: inp[n].pin_memory() for n in names_in}
+    h0 = d["h0"]
+    hout = {"o": torch.empty_like(inp["v"]).pin_memory()}
+    for n in ("dq", "dk", "dv", "dg", "dbeta"):
+        src = {"dq": "q", "dk": "k", "dv": "v", "dg": "g", "dbeta": "beta"}[n]
+        hout[n] = torch.empty_like(inp[src]).pin_memory()
+    dbuf = {n: torch.empty_like(d[n]) for n in names_in}
+
+    def e2e_step():
+        for n in names_in:
+            dbuf[n].copy_(host[n], non_blocking=True)
+        o, _ = gdn.gdn_chunk_fwd(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["g"], dbuf["beta"], h0,
+                                 o=outs["o"], hT=outs["hT"], workspace=ws_f)
+        r = gdn.gdn_chunk_bwd(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["g"], dbuf["beta"],
+                              dbuf["dO"], h0, None, workspace=ws_b)
+        hout["o"].copy_(o, non_blocking=True)
+        for n in ("dq", "dk", "dv", "dg", "dbeta"):
+            hout[n].copy_(r[n], non_blocking=True)
+    ms_e2e = max_over_ranks(timed(e2e_step, args.steps, 2, barrier))
+    h2d = sum(host[n].numel() * host[n].element_size() for n in names_in)
+    d2h = sum(x.numel() * x.element_size() for x in hout.values())
+
+    return dict(value=value, ms_step=ms_step, tflops=tflops, roofline=roofline, extra=extra,
+                e2e={"value": round(world * tokens / (ms_e2e / 1e3), 1), "unit": "tokens/s",
+                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                     "ms_per_step": round(ms_e2e, 3)},
+                gpu_launches=nlaunch, clocks=clk.summary(), peaks=pk, cfg=cfg)
+
+
+def cpu_baseline_oracle(sample_B):
+    """The fp64 oracle (as it stands) on host cores: fwd + bwd over the first
+    `sample_B` sequences of the 350M-scale workload.  Returns tokens/s."""
+    import oracle
+    from gated_delta_rule_153_b200.inputs import L350M, make_chunk_inputs
+    inp = make_chunk_inputs(L350M)
+    sl = {n: (inp[n][:sample_B] if n in ("q", "k", "v", "g", "beta", "dO") else inp[n])
+          for n in inp}
+    t0 = time.perf_counter()
+    oracle.fwd(sl["q"], sl["k"], sl["v"], sl["g"], sl["beta"], None)
+    oracle.bwd(sl["q"], sl["k"], sl["v"], sl["g"], sl["beta"], sl["dO"], None, None)
+    dt = time.perf_counter() - t0
+    return sample_B * L350M.T / dt, dt, oracle.threads()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--headline-only", action="store_true",
+                    help="skip the long-context, channel-gate and decode extras")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        from gated_delta_rule_153_b200.inputs import L350M
+        sample_B = 1
+        vals = []
+        for i in range(args.warmup + args.steps):
+            v, dt, cores = cpu_baseline_oracle(sample_B)
+            if i >= args.warmup:
+                vals.append((v, dt))
+        tot = sum(dt for _, dt in vals)
+        value = len(vals) * sample_B * L350M.T / tot
+        sample = (f"fwd+bwd of 1 of 8 sequences (T=2048, H=8, d=128) of the 350M-scale "
+                  f"workload per step, fp64 token loop, OpenMP over heads")
+        print(json.dumps({
+            "impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(1e3 * tot / len(vals), 2), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": L350M.name, "B": L350M.B, "T": L350M.T, "H": L350M.H,
+                       "d": 128, "chunk": 64, "l2": "n/a (CPU)"},
+            "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}))
+        return
+
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+        barrier = lambda: dist.barrier()
+
+        def max_over_ranks(x):
+            t = torch.tensor([x], dtype=torch.float64, device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            return float(t.item())
+    else:
+        barrier = lambda: None
+        max_over_ranks = lambda x: x
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+
+    r = run_ours(args, rank, world, dev, barrier, max_over_ranks)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, dt, cores = cpu_baseline_oracle(8)
+        cpu = {"value": round(v, 2), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": f"full 350M-scale workload (B=8, T=2048, H=8) fwd+bwd once, "
+                         f"fp64 token loop, {dt:.1f} s"}
+    cfg = r["cfg"]
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(r["value"], 1), "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(r["ms_step"], 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded generators; no datasets or trained weights)",
+            "config": {"workload": cfg.name, "B": cfg.B, "T": cfg.T, "H": cfg.H, "d_k": cfg.dk,
+                       "d_v": cfg.dv, "chunk": cfg.chunk, "gate": cfg.gate,
+                       "state": "fp32", "parallelism": f"replicas x{world} (independent batches)",
+                       "l2": "inputs larger than L2 (a step reads/writes > 0.5 GB); no flush"},
+            "tflops": round(r["tflops"], 2),
+            "frac_tensor_peak": round(r["tflops"] / r["peaks"]["bf16"], 4),
+            "roofline": r["roofline"],
+            "cpu_baseline": cpu,
+            "e2e": r["e2e"],
+            "gpu_launches": r["gpu_launches"],
+            "clocks": r["clocks"],
+        }
+        line.update(r["extra"])
+        print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -27,7 +27,7 @@ GDN_GATE_SCALAR, GDN_GATE_CHANNEL = 0, 1
 # Every symbol include/gdn.h declares.
 EXPORTS = ("gdn_chunk_fwd_workspace", "gdn_chunk_fwd", "gdn_chunk_bwd_workspace",
            "gdn_chunk_bwd", "gdn_recurrent_step", "gdn_query_device_status",
-           "gdn_status_string")
+           "gdn_status_string", "gdn_profile_begin", "gdn_profile_end")
 
 
 class gdn_dims(ctypes.Structure):
@@ -73,6 +73,11 @@ def lib() -> ctypes.CDLL:
             L.gdn_recurrent_step.restype = i
             L.gdn_query_device_status.argtypes = [vp, vp]
             L.gdn_query_device_status.restype = i
+            L.gdn_profile_begin.argtypes = [i]
+            L.gdn_profile_begin.restype = i
+            L.gdn_profile_end.argtypes = [ctypes.POINTER(ctypes.c_float),
+                                          ctypes.POINTER(ctypes.c_char_p), i]
+            L.gdn_profile_end.restype = i
             L.gdn_status_string.argtypes = [i]
             L.gdn_status_string.restype = ctypes.c_char_p
             _lib = L
@@ -228,6 +233,22 @@ def gdn_recurrent_step(q, k, v, g, beta, state, *, scale=1.0, o=None, stream=Non
                                   _ptr(o), _stream(stream))
     _check(st, "gdn_recurrent_step")
     return o
+
+
+def gdn_profile_begin(capacity: int) -> None:
+    """Start bracketing this thread's next ``capacity`` library launches with
+    CUDA events (a profiling aid)."""
+    _check(lib().gdn_profile_begin(int(capacity)), "gdn_profile_begin")
+
+
+def gdn_profile_end(capacity: int):
+    """Stop recording; returns (launch count, [(kernel name, ms), ...])."""
+    ms = (ctypes.c_float * capacity)()
+    names = (ctypes.c_char_p * capacity)()
+    n = lib().gdn_profile_end(ms, names, int(capacity))
+    if n < 0:
+        raise RuntimeError("gdn_profile_end: recording was not on or a CUDA call failed")
+    return n, [(names[i].decode(), float(ms[i])) for i in range(min(n, capacity))]
 
 
 def gdn_query_device_status(workspace, stream=None) -> int:

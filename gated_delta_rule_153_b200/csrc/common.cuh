@@ -24,6 +24,16 @@ template <> GDN_DEV __nv_bfloat16 from_f<__nv_bfloat16>(float x) { return __floa
 // device status word (non-zero after a bounded wait gave up).
 constexpr size_t kStatusBytes = 256;
 
+// Launch bracketing for gdn_profile_begin/end (no-ops unless enabled).
+void prof_before(cudaStream_t st);
+void prof_after(cudaStream_t st, const char* name);
+#define GDN_LAUNCH(name, st, ...)          \
+    do {                                   \
+        ::gdn::prof_before(st);            \
+        __VA_ARGS__;                       \
+        ::gdn::prof_after(st, name);       \
+    } while (0)
+
 GDN_DEV float warp_sum(float x) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);

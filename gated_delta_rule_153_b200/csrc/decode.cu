@@ -124,8 +124,10 @@ template <int DK, typename T, bool CHANNEL>
 static void launch_decode(int N, int H, int dv, float scale, const void* q, const void* k,
                           const void* v, const float* g, const float* beta, float* state,
                           void* o, cudaStream_t st) {
-    decode_step_kernel<DK, T, CHANNEL, 2><<<N * H, 256, 0, st>>>(
-        H, dv, scale, (const T*)q, (const T*)k, (const T*)v, g, beta, state, (T*)o);
+    GDN_LAUNCH("decode_step", st,
+               decode_step_kernel<DK, T, CHANNEL, 2><<<N * H, 256, 0, st>>>(
+                   H, dv, scale, (const T*)q, (const T*)k, (const T*)v, g, beta, state,
+                   (T*)o));
 }
 
 template <typename T, bool CHANNEL>

@@ -66,7 +66,7 @@ size_t gdn_chunk_fwd_workspace(const gdn_dims* d) {
 
 size_t gdn_chunk_bwd_workspace(const gdn_dims* d) {
     if (check_dims(d) != GDN_OK) return 0;
-    return tc_supported(*d) ? tc_bwd_workspace(*d) : simt_bwd_workspace(*d);
+    return tc_bwd_supported(*d) ? tc_bwd_workspace(*d) : simt_bwd_workspace(*d);
 }
 
 gdn_status gdn_chunk_fwd(const gdn_dims* d, const void* q, const void* k, const void* v,
@@ -108,7 +108,7 @@ gdn_status gdn_chunk_bwd(const gdn_dims* d, const void* q, const void* k, const 
     cudaGetLastError();
     if (ws && cudaMemsetAsync(ws, 0, sizeof(unsigned int), st) != cudaSuccess)
         return GDN_ERR_CUDA;
-    if (tc_supported(*d))
+    if (tc_bwd_supported(*d))
         launch_tc_bwd(*d, q, k, v, g, beta, h0, dO, dhT, dq, dk, dv, dg, dbeta, dh0, ws, st);
     else
         launch_simt_bwd(*d, q, k, v, g, beta, h0, dO, dhT, dq, dk, dv, dg, dbeta, dh0, ws, st);

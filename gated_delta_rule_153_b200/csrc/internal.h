@@ -26,6 +26,7 @@ void launch_simt_bwd(const gdn_dims& d, const void* q, const void* k, const void
 
 // Tensor-core path (bf16, dk = dv = 128, chunk = 64).
 bool tc_supported(const gdn_dims& d);
+bool tc_bwd_supported(const gdn_dims& d);
 size_t tc_fwd_workspace(const gdn_dims& d);
 size_t tc_bwd_workspace(const gdn_dims& d);
 void launch_tc_fwd(const gdn_dims& d, const void* q, const void* k, const void* v,

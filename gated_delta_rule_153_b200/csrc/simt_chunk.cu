@@ -462,11 +462,11 @@ void launch_simt_fwd(const gdn_dims& d, const void* q, const void* k, const void
     const int grid = d.B * d.H;
     const bool ch = d.gate == GDN_GATE_CHANNEL;
     if (d.dtype == GDN_BF16) {
-        if (ch) simt_fwd_kernel<__nv_bfloat16, true><<<grid, 256, 0, st>>>(a);
-        else simt_fwd_kernel<__nv_bfloat16, false><<<grid, 256, 0, st>>>(a);
+        if (ch) GDN_LAUNCH("simt_fwd", st, simt_fwd_kernel<__nv_bfloat16, true><<<grid, 256, 0, st>>>(a));
+        else GDN_LAUNCH("simt_fwd", st, simt_fwd_kernel<__nv_bfloat16, false><<<grid, 256, 0, st>>>(a));
     } else {
-        if (ch) simt_fwd_kernel<float, true><<<grid, 256, 0, st>>>(a);
-        else simt_fwd_kernel<float, false><<<grid, 256, 0, st>>>(a);
+        if (ch) GDN_LAUNCH("simt_fwd", st, simt_fwd_kernel<float, true><<<grid, 256, 0, st>>>(a));
+        else GDN_LAUNCH("simt_fwd", st, simt_fwd_kernel<float, false><<<grid, 256, 0, st>>>(a));
     }
 }
 
@@ -480,11 +480,11 @@ void launch_simt_bwd(const gdn_dims& d, const void* q, const void* k, const void
     const int grid = d.B * d.H;
     const bool ch = d.gate == GDN_GATE_CHANNEL;
     if (d.dtype == GDN_BF16) {
-        if (ch) simt_bwd_kernel<__nv_bfloat16, true><<<grid, 256, 0, st>>>(a);
-        else simt_bwd_kernel<__nv_bfloat16, false><<<grid, 256, 0, st>>>(a);
+        if (ch) GDN_LAUNCH("simt_bwd", st, simt_bwd_kernel<__nv_bfloat16, true><<<grid, 256, 0, st>>>(a));
+        else GDN_LAUNCH("simt_bwd", st, simt_bwd_kernel<__nv_bfloat16, false><<<grid, 256, 0, st>>>(a));
     } else {
-        if (ch) simt_bwd_kernel<float, true><<<grid, 256, 0, st>>>(a);
-        else simt_bwd_kernel<float, false><<<grid, 256, 0, st>>>(a);
+        if (ch) GDN_LAUNCH("simt_bwd", st, simt_bwd_kernel<float, true><<<grid, 256, 0, st>>>(a));
+        else GDN_LAUNCH("simt_bwd", st, simt_bwd_kernel<float, false><<<grid, 256, 0, st>>>(a));
     }
 }
 

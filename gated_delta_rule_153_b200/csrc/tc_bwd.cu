@@ -1,0 +1,765 @@
+// tc_bwd.cu -- tensor-core chunkwise backward of the gated delta rule
+// (bf16 q/k/v/dO, fp32 state gradients; dk = dv = 128, chunk 64, scalar gate).
+//
+// Reverse-mode through the chunk equations of the forward (see tc_chunk.cu):
+// with dS the gradient w.r.t. the state leaving a chunk and dO the output
+// gradient of its tokens,
+//   dU  = P^T dO + diag(e^{G_last-G}) K dS^T
+//   dS0 = e^{G_last} dS + (scale dO)^T diag(e^G) Q - dU^T W       (next chunk back)
+//   dQ' = diag(e^G) dO S0 + (dP .* D) K,          dP = lower(dO U^T)
+//   dK  = diag(e^{G_last-G}) U dS + diag(beta e^G) T^T dW + (dM + dM^T) K
+//         + (dP .* D)^T Q',                        dW = -dU S0
+//   dV  = diag(beta) T^T dU
+//   dA  = strict_lower(-T^T dT T^T),  dT = dW (diag(beta e^G) K)^T + dU (diag(beta) V)^T
+//   dM  = dA .* beta_i .* D
+// plus the gate and beta gradients from the matching row sums, and
+// dg = reverse within-chunk cumsum of dG.  (Q' = scale Q; dq = scale dQ'.)
+//
+// Kernels: tc_walk_bwd walks the chunks backwards for 16 rows of dS (the rows
+// of dS, like those of S, never mix) and stores dS and dU per chunk;
+// tc_bwd_local then computes every chunk's gradients in parallel from the
+// stored S0, U (forward recompute), dS and dU.
+#include "common.cuh"
+#include "internal.h"
+#include "mma.cuh"
+#include "tc_common.cuh"
+
+namespace gdn {
+namespace tc {
+void launch_prep(const ChunkPtrs& p, size_t nchunks, cudaStream_t st);
+void launch_walk_states(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& cp,
+                        const float* h0, void* ws, cudaStream_t st);
+}  // namespace tc
+
+namespace {
+using namespace tc;
+
+// ---------------------------------------------------------------------------
+// reverse walk: dS for 16 value-rows, chunks NT-1 .. 0
+// ---------------------------------------------------------------------------
+struct BwStage {
+    __nv_bfloat16 W[C * DK];
+    __nv_bfloat16 Q[C * DK];
+    __nv_bfloat16 K[C * DK];
+    __nv_bfloat16 P[C * C];
+    __nv_bfloat16 dO[C][16];
+    float G[C];
+};
+
+struct BwSmem {
+    BwStage st[2];
+    __nv_bfloat16 dS[16 * DK];  // bf16 copy of dS (rows x key columns)
+    __nv_bfloat16 dOt[16 * C];  // dO^T tile
+    __nv_bfloat16 dOg[16 * C];  // dO^T * scale * e^{G_i}
+    __nv_bfloat16 dU[16 * C];   // dU^T
+};
+
+struct BwPtrs {
+    const __nv_bfloat16 *q, *k, *dO;
+    const float* dhT;
+    const __nv_bfloat16 *W, *P;
+    const float* G;
+    __nv_bfloat16 *dSout, *dUout;
+    float* dh0;
+    int B, T, H, NT;
+    float scale;
+};
+
+__device__ void bw_issue(BwStage& st, const BwPtrs& p, int b, int h, int bh, int n, int a0,
+                         int tid) {
+    const int t0 = n * C;
+    const int L = min(C, p.T - t0);
+    const size_t row0 = ((size_t)b * p.T + t0) * p.H + h;
+    const size_t cid = (size_t)bh * p.NT + n;
+    load_tile_async<DK>(st.K, p.k + row0 * DK, (size_t)p.H * DK, C, L, tid, 128);
+    load_tile_async<DK>(st.Q, p.q + row0 * DK, (size_t)p.H * DK, C, L, tid, 128);
+    load_tile_async<DK>(st.W, p.W + cid * C * DK, DK, C, C, tid, 128);
+    load_tile_async<C>(st.P, p.P + cid * C * C, C, C, C, tid, 128);
+    for (int e = tid; e < C * 2; e += 128) {
+        const int r = e >> 1, c = e & 1;
+        const bool ok = r < L;
+        cp_async16_zfill(&st.dO[r][8 * c], p.dO + (row0 + (size_t)(ok ? r : 0) * p.H) * DV + a0 + 8 * c,
+                         ok);
+    }
+    for (int e = tid; e < C / 4; e += 128) cp_async16(&st.G[4 * e], p.G + cid * C + 4 * e);
+    cp_async_commit();
+}
+
+__global__ void __launch_bounds__(128) tc_walk_bwd_kernel(BwPtrs p) {
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    BwSmem& s = *reinterpret_cast<BwSmem*>(smem_raw);
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    const int tiles = DV / 16;
+    const int bh = blockIdx.x / tiles, a0 = (blockIdx.x % tiles) * 16;
+    const int b = bh / p.H, h = bh % p.H;
+    const int r_lo = lane >> 2;
+
+    float dS[4][4];
+    {
+        const float* src = p.dhT ? p.dhT + ((size_t)bh * DV + a0) * DK : nullptr;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int c = 32 * w + 8 * j + 2 * (lane & 3);
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                dS[j][e] = src ? src[(size_t)(r_lo + 8 * (e >> 1)) * DK + c + (e & 1)] : 0.f;
+        }
+    }
+    bw_issue(s.st[(p.NT - 1) & 1], p, b, h, bh, p.NT - 1, a0, tid);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) st_c<DK>(s.dS, 0, 32 * w + 8 * j, dS[j]);
+
+    for (int n = p.NT - 1; n >= 0; --n) {
+        BwStage& st = s.st[n & 1];
+        cp_async_wait<0>();
+        __syncthreads();
+        if (n > 0) bw_issue(s.st[(n - 1) & 1], p, b, h, bh, n - 1, a0, tid);
+        const size_t cid = (size_t)bh * p.NT + n;
+        // dO^T tiles, plain and scaled by scale*e^{G_i}
+        for (int e = tid; e < C * 16; e += 128) {
+            const int i = e >> 4, a = e & 15;
+            const float x = __bfloat162float(st.dO[i][a]);
+            s.dOt[swz<C>(a, i)] = st.dO[i][a];
+            s.dOg[swz<C>(a, i)] = __float2bfloat16_rn(x * p.scale * __expf(st.G[i]));
+        }
+        // dS leaving chunk n (bf16), rows a0.. of [dv][dk]
+        {
+            __nv_bfloat16* dst = p.dSout + (cid * DV + a0) * DK;
+            for (int e = tid; e < 16 * DK / 8; e += 128) {
+                const int r = e / (DK / 8), c8 = e % (DK / 8);
+                *reinterpret_cast<uint4*>(dst + (size_t)r * DK + 8 * c8) =
+                    *reinterpret_cast<const uint4*>(s.dS + swz<DK>(r, 8 * c8));
+            }
+        }
+        __syncthreads();
+        const float Gl = st.G[C - 1];
+        // dU^T (rows x tokens 16w..16w+15)
+        {
+            float a1[2][4] = {}, a2[2][4] = {};
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+                if (kk < w) continue;  // P[i][r] = 0 for i < r
+                uint32_t a[4], bp[4];
+                lda<C>(a, s.dOt, 0, 16 * kk);
+                ldb_kn<C>(bp, st.P, 16 * kk, 16 * w);
+                mma16816(a1[0], a, bp[0], bp[1]);
+                mma16816(a1[1], a, bp[2], bp[3]);
+            }
+#pragma unroll
+            for (int kk = 0; kk < DK / 16; ++kk) {
+                uint32_t a[4], bk[4];
+                lda<DK>(a, s.dS, 0, 16 * kk);
+                ldb_nk<DK>(bk, st.K, 16 * w, 16 * kk);
+                mma16816(a2[0], a, bk[0], bk[1]);
+                mma16816(a2[1], a, bk[2], bk[3]);
+            }
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int r0 = 16 * w + 8 * j + 2 * (lane & 3);
+                float u[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    u[e] = a1[j][e] + a2[j][e] * __expf(Gl - st.G[r0 + (e & 1)]);
+                st_c<C>(s.dU, 0, 16 * w + 8 * j, u);
+            }
+        }
+        __syncthreads();
+        {
+            __nv_bfloat16* dst = p.dUout + cid * C * DV + a0;
+            for (int e = tid; e < C * 16; e += 128) {
+                const int i = e >> 4, a = e & 15;
+                dst[(size_t)i * DV + a] = s.dU[swz<C>(a, i)];
+            }
+        }
+        // dS0 = e^{G_last} dS + dOg^T Q - dU^T W   (columns 32w..32w+31)
+        {
+            const float gam = __expf(Gl);
+            float y[4][4] = {}, z[4][4] = {};
+#pragma unroll
+            for (int kk = 0; kk < C / 16; ++kk) {
+                uint32_t ag[4], au[4];
+                lda<C>(ag, s.dOg, 0, 16 * kk);
+                lda<C>(au, s.dU, 0, 16 * kk);
+#pragma unroll
+                for (int np = 0; np < 2; ++np) {
+                    uint32_t bq[4], bw[4];
+                    ldb_kn<DK>(bq, st.Q, 16 * kk, 32 * w + 16 * np);
+                    ldb_kn<DK>(bw, st.W, 16 * kk, 32 * w + 16 * np);
+                    mma16816(y[2 * np], ag, bq[0], bq[1]);
+                    mma16816(y[2 * np + 1], ag, bq[2], bq[3]);
+                    mma16816(z[2 * np], au, bw[0], bw[1]);
+                    mma16816(z[2 * np + 1], au, bw[2], bw[3]);
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) dS[j][e] = gam * dS[j][e] + y[j][e] - z[j][e];
+        }
+        __syncthreads();
+#pragma unroll
+        for (int j = 0; j < 4; ++j) st_c<DK>(s.dS, 0, 32 * w + 8 * j, dS[j]);
+    }
+    if (p.dh0) {
+        float* dst = p.dh0 + ((size_t)bh * DV + a0) * DK;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int c = 32 * w + 8 * j + 2 * (lane & 3);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) dst[(size_t)(r_lo + 8 * (e >> 1)) * DK + c + (e & 1)] = dS[j][e];
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// local gradients: one CTA (8 warps) per chunk.  Warp w owns rows
+// 16*(w/2) .. +15 and column half (w%2) of every 64x128 result, and the
+// token-column half (w%2) of every 64x64 result.
+// ---------------------------------------------------------------------------
+struct LocSmem {
+    __nv_bfloat16 Q[C * DK], K[C * DK], V[C * DV], dO[C * DV], U[C * DV], dU[C * DV];
+    __nv_bfloat16 S0[DV * DK];  // rows a (value), cols c (key)
+    __nv_bfloat16 dS[DV * DK];
+    __nv_bfloat16 dW[C * DK];
+    __nv_bfloat16 Tb[C * C];
+    __nv_bfloat16 dPG[C * C];   // lower(dO U^T) .* D
+    __nv_bfloat16 dT[C * C];
+    __nv_bfloat16 X[C * C];     // dT T^T
+    __nv_bfloat16 dMM[C * C];   // dA .* beta_i .* D
+    float G[C], beta[C];
+    float red_b[8][C];   // partial dbeta (by row)
+    float red_g[8][C];   // partial dG (by token)
+    float red_s[8][2];   // partial scalars for G_last
+};
+
+struct LocPtrs {
+    const __nv_bfloat16 *q, *k, *v, *dO;
+    const float *g, *beta;
+    const __nv_bfloat16 *S0, *U, *dS, *dU, *Tb;
+    const float* G;
+    __nv_bfloat16 *dq, *dk, *dv;
+    float *dg, *dbeta;
+    int B, T, H, NT;
+    float scale;
+};
+
+// Row sums over the 4 lanes of a quad: lo -> row r_lo, hi -> row r_lo + 8.
+__device__ __forceinline__ void quad_rows(float& lo, float& hi) {
+    lo += __shfl_xor_sync(0xffffffffu, lo, 1);
+    lo += __shfl_xor_sync(0xffffffffu, lo, 2);
+    hi += __shfl_xor_sync(0xffffffffu, hi, 1);
+    hi += __shfl_xor_sync(0xffffffffu, hi, 2);
+}
+// Column sums over the 8 row-groups of a warp (lanes with equal lane%4).
+__device__ __forceinline__ float col_sum(float v) {
+    v += __shfl_xor_sync(0xffffffffu, v, 4);
+    v += __shfl_xor_sync(0xffffffffu, v, 8);
+    v += __shfl_xor_sync(0xffffffffu, v, 16);
+    return v;
+}
+
+__global__ void __launch_bounds__(256) tc_bwd_local_kernel(LocPtrs p) {
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    LocSmem& s = *reinterpret_cast<LocSmem*>(smem_raw);
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    const int rb = w >> 1, ch = w & 1;
+    const int m0 = 16 * rb;
+    const int cid = blockIdx.x;
+    const int bh = cid / p.NT, n = cid % p.NT, b = bh / p.H, h = bh % p.H;
+    const int t0 = n * C;
+    const int L = min(C, p.T - t0);
+    const size_t row0 = ((size_t)b * p.T + t0) * p.H + h;
+    const size_t rs = (size_t)p.H;
+    const int rl = m0 + (lane >> 2), rh = rl + 8;  // this thread's two rows
+
+    load_tile_async<DK>(s.Q, p.q + row0 * DK, rs * DK, C, L, tid, 256);
+    load_tile_async<DK>(s.K, p.k + row0 * DK, rs * DK, C, L, tid, 256);
+    load_tile_async<DV>(s.V, p.v + row0 * DV, rs * DV, C, L, tid, 256);
+    load_tile_async<DV>(s.dO, p.dO + row0 * DV, rs * DV, C, L, tid, 256);
+    load_tile_async<DV>(s.U, p.U + (size_t)cid * C * DV, DV, C, C, tid, 256);
+    load_tile_async<DV>(s.dU, p.dU + (size_t)cid * C * DV, DV, C, C, tid, 256);
+    load_tile_async<DK>(s.S0, p.S0 + (size_t)cid * DV * DK, DK, DV, DV, tid, 256);
+    load_tile_async<DK>(s.dS, p.dS + (size_t)cid * DV * DK, DK, DV, DV, tid, 256);
+    load_tile_async<C>(s.Tb, p.Tb + (size_t)cid * C * C, C, C, C, tid, 256);
+    cp_async_commit();
+    for (int e = tid; e < C; e += 256) {
+        s.G[e] = p.G[(size_t)cid * C + e];
+        s.beta[e] = e < L ? p.beta[row0 + e * rs] : 0.f;
+    }
+    for (int e = tid; e < 8 * C; e += 256) {
+        (&s.red_b[0][0])[e] = 0.f;
+        (&s.red_g[0][0])[e] = 0.f;
+    }
+    if (tid < 16) (&s.red_s[0][0])[tid] = 0.f;
+    cp_async_wait<0>();
+    __syncthreads();
+
+    const float Gl = s.G[C - 1];
+    const float egl = __expf(s.G[rl]), egh = __expf(s.G[rh]);
+    const float etl = __expf(Gl - s.G[rl]), eth = __expf(Gl - s.G[rh]);
+    const float bl = s.beta[rl], bhh = s.beta[rh];
+    float row_b_lo = 0.f, row_b_hi = 0.f;  // partial dbeta for rows rl, rh
+    float row_g_lo = 0.f, row_g_hi = 0.f;  // partial dG for rows rl, rh
+    float last_acc = 0.f;                  // partial dG_last (sum over rows of hkt)
+
+    // dQ' and dK accumulators: rows rl/rh, columns 64*ch + 8j + 2(lane%4) + {0,1}
+    float dQ[8][4], dK[8][4];
+
+    // ---- phase 1: contractions over the value dimension --------------------
+    {
+        float acc[8][4];
+        // dQg = dO S0  ->  dQ' = e^G dQg ;  dG += scale e^G sum_c dQg Q
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[j][e] = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < DV / 16; ++kk) {
+            uint32_t a[4];
+            lda<DV>(a, s.dO, m0, 16 * kk);
+#pragma unroll
+            for (int np = 0; np < 4; ++np) {
+                uint32_t bf[4];
+                ldb_kn<DK>(bf, s.S0, 16 * kk, 64 * ch + 16 * np);
+                mma16816(acc[2 * np], a, bf[0], bf[1]);
+                mma16816(acc[2 * np + 1], a, bf[2], bf[3]);
+            }
+        }
+        float hq_lo = 0.f, hq_hi = 0.f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int c = 64 * ch + 8 * j + 2 * (lane & 3);
+            const float2 ql = unpack_bf16(*reinterpret_cast<const uint32_t*>(s.Q + swz<DK>(rl, c)));
+            const float2 qh = unpack_bf16(*reinterpret_cast<const uint32_t*>(s.Q + swz<DK>(rh, c)));
+            hq_lo += acc[j][0] * ql.x + acc[j][1] * ql.y;
+            hq_hi += acc[j][2] * qh.x + acc[j][3] * qh.y;
+            dQ[j][0] = egl * acc[j][0]; dQ[j][1] = egl * acc[j][1];
+            dQ[j][2] = egh * acc[j][2]; dQ[j][3] = egh * acc[j][3];
+        }
+        row_g_lo += p.scale * egl * hq_lo;
+        row_g_hi += p.scale * egh * hq_hi;
+
+        // dKt = U dS  ->  dK = e^{Gl-G} dKt ;  hkt = e^{Gl-G} sum_c dKt K
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[j][e] = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < DV / 16; ++kk) {
+            uint32_t a[4];
+            lda<DV>(a, s.U, m0, 16 * kk);
+#pragma unroll
+            for (int np = 0; np < 4; ++np) {
+                uint32_t bf[4];
+                ldb_kn<DK>(bf, s.dS, 16 * kk, 64 * ch + 16 * np);
+                mma16816(acc[2 * np], a, bf[0], bf[1]);
+                mma16816(acc[2 * np + 1], a, bf[2], bf[3]);
+            }
+        }
+        float hk_lo = 0.f, hk_hi = 0.f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int c = 64 * ch + 8 * j + 2 * (lane & 3);
+            const float2 kl = unpack_bf16(*reinterpret_cast<const uint32_t*>(s.K + swz<DK>(rl, c)));
+            const float2 kh = unpack_bf16(*reinterpret_cast<const uint32_t*>(s.K + swz<DK>(rh, c)));
+            hk_lo += acc[j][0] * kl.x + acc[j][1] * kl.y;
+            hk_hi += acc[j][2] * kh.x + acc[j][3] * kh.y;
+            dK[j][0] = etl * acc[j][0]; dK[j][1] = etl * acc[j][1];
+            dK[j][2] = eth * acc[j][2]; dK[j][3] = eth * acc[j][3];
+        }
+        row_g_lo -= etl * hk_lo;
+        row_g_hi -= eth * hk_hi;
+        last_acc += etl * hk_lo + eth * hk_hi;
+
+        // dW = -dU S0  -> bf16 tile
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[j][e] = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < DV / 16; ++kk) {
+            uint32_t a[4];
+            lda<DV>(a, s.dU, m0, 16 * kk);
+#pragma unroll
+            for (int np = 0; np < 4; ++np) {
+                uint32_t bf[4];
+                ldb_kn<DK>(bf, s.S0, 16 * kk, 64 * ch + 16 * np);
+                mma16816(acc[2 * np], a, bf[0], bf[1]);
+                mma16816(acc[2 * np + 1], a, bf[2], bf[3]);
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            float x[4] = {-acc[j][0], -acc[j][1], -acc[j][2], -acc[j][3]};
+            st_c<DK>(s.dW, m0, 64 * ch + 8 * j, x);
+        }
+
+        // dP = lower(dO U^T), QK = Q K^T on tokens 32*ch .. +31
+        float dp[4][4] = {}, qk[4][4] = {};
+#pragma unroll
+        for (int kk = 0; kk < DV / 16; ++kk) {
+            uint32_t ad[4], aq[4];
+            lda<DV>(ad, s.dO, m0, 16 * kk);
+            lda<DK>(aq, s.Q, m0, 16 * kk);
+#pragma unroll
+            for (int np = 0; np < 2; ++np) {
+                uint32_t bu[4], bk[4];
+                ldb_nk<DV>(bu, s.U, 32 * ch + 16 * np, 16 * kk);
+                ldb_nk<DK>(bk, s.K, 32 * ch + 16 * np, 16 * kk);
+                mma16816(dp[2 * np], ad, bu[0], bu[1]);
+                mma16816(dp[2 * np + 1], ad, bu[2], bu[3]);
+                mma16816(qk[2 * np], aq, bk[0], bk[1]);
+                mma16816(qk[2 * np + 1], aq, bk[2], bk[3]);
+            }
+        }
+        // hP = dP .* (scale Q K^T .* D) ;  dPG = dP .* D
+        float colp[4][2];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int c0 = 32 * ch + 8 * j + 2 * (lane & 3);
+            float g[4];
+            colp[j][0] = colp[j][1] = 0.f;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int r = (e < 2) ? rl : rh, c = c0 + (e & 1);
+                const float d = (c <= r) ? __expf(s.G[r] - s.G[c]) : 0.f;
+                g[e] = dp[j][e] * d;
+                const float hp = g[e] * p.scale * qk[j][e];
+                if (e < 2) row_g_lo += hp; else row_g_hi += hp;
+                colp[j][e & 1] -= hp;
+            }
+            st_c<C>(s.dPG, m0, 32 * ch + 8 * j, g);
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const float v = col_sum(colp[j][e]);
+                if (lane < 4) s.red_g[w][32 * ch + 8 * j + 2 * lane + e] += v;
+            }
+        // e^{G_last} <dS, S0> (each warp a slice of the 128x128 elements)
+        float ss = 0.f;
+        for (int e = lane + 32 * w; e < DV * DK / 8; e += 256) {
+            const int r = e / (DK / 8), c8 = e % (DK / 8);
+            const uint4 x = *reinterpret_cast<const uint4*>(s.dS + swz<DK>(r, 8 * c8));
+            const uint4 y = *reinterpret_cast<const uint4*>(s.S0 + swz<DK>(r, 8 * c8));
+            const uint32_t xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                const float2 a = unpack_bf16(xs[t]), bb = unpack_bf16(ys[t]);
+                ss += a.x * bb.x + a.y * bb.y;
+            }
+        }
+        ss = warp_sum(ss);
+        last_acc = warp_sum(last_acc);  // over rows of this warp (both halves)
+        if (lane == 0) {
+            s.red_s[w][0] = ss;
+            s.red_s[w][1] = last_acc;
+        }
+    }
+
+    // ---- phase 2: K K^T (-> M), dT ---------------------------------------
+    float M[4][4];
+    {
+        float kkt[4][4] = {}, tw[4][4] = {}, tu[4][4] = {};
+#pragma unroll
+        for (int kk = 0; kk < DK / 16; ++kk) {
+            uint32_t ak[4];
+            lda<DK>(ak, s.K, m0, 16 * kk);
+#pragma unroll
+            for (int np = 0; np < 2; ++np) {
+                uint32_t bk[4];
+                ldb_nk<DK>(bk, s.K, 32 * ch + 16 * np, 16 * kk);
+                mma16816(kkt[2 * np], ak, bk[0], bk[1]);
+                mma16816(kkt[2 * np + 1], ak, bk[2], bk[3]);
+            }
+        }
+        __syncthreads();  // dW tile complete
+#pragma unroll
+        for (int kk = 0; kk < DK / 16; ++kk) {
+            uint32_t aw[4], au[4];
+            lda<DK>(aw, s.dW, m0, 16 * kk);
+            lda<DV>(au, s.dU, m0, 16 * kk);
+#pragma unroll
+            for (int np = 0; np < 2; ++np) {
+                uint32_t bk[4], bv[4];
+                ldb_nk<DK>(bk, s.K, 32 * ch + 16 * np, 16 * kk);
+                ldb_nk<DV>(bv, s.V, 32 * ch + 16 * np, 16 * kk);
+                mma16816(tw[2 * np], aw, bk[0], bk[1]);
+                mma16816(tw[2 * np + 1], aw, bk[2], bk[3]);
+                mma16816(tu[2 * np], au, bv[0], bv[1]);
+                mma16816(tu[2 * np + 1], au, bv[2], bv[3]);
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int c0 = 32 * ch + 8 * j + 2 * (lane & 3);
+            float dt[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int r = (e < 2) ? rl : rh, c = c0 + (e & 1);
+                const float bj = s.beta[c];
+                dt[e] = tw[j][e] * bj * __expf(s.G[c]) + tu[j][e] * bj;
+                M[j][e] = (c < r) ? kkt[j][e] * __expf(s.G[r] - s.G[c]) : 0.f;
+            }
+            st_c<C>(s.dT, m0, 32 * ch + 8 * j, dt);
+        }
+    }
+    __syncthreads();
+
+    // ---- phase 3: X = dT T^T ; dKg = T^T dW ; dVb = T^T dU ------------------
+    {
+        float x[4][4] = {};
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+            uint32_t a[4];
+            lda<C>(a, s.dT, m0, 16 * kk);
+#pragma unroll
+            for (int np = 0; np < 2; ++np) {
+                uint32_t bt[4];
+                ldb_nk<C>(bt, s.Tb, 32 * ch + 16 * np, 16 * kk);
+                mma16816(x[2 * np], a, bt[0], bt[1]);
+                mma16816(x[2 * np + 1], a, bt[2], bt[3]);
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) st_c<C>(s.X, m0, 32 * ch + 8 * j, x[j]);
+
+        float akg[8][4] = {}, avb[8][4] = {};
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+            if (kk < rb) continue;  // T[j][i] = 0 for j < i
+            uint32_t a[4];
+            lda_t<C>(a, s.Tb, m0, 16 * kk);
+#pragma unroll
+            for (int np = 0; np < 4; ++np) {
+                uint32_t bw[4], bu[4];
+                ldb_kn<DK>(bw, s.dW, 16 * kk, 64 * ch + 16 * np);
+                ldb_kn<DV>(bu, s.dU, 16 * kk, 64 * ch + 16 * np);
+                mma16816(akg[2 * np], a, bw[0], bw[1]);
+                mma16816(akg[2 * np + 1], a, bw[2], bw[3]);
+                mma16816(avb[2 * np], a, bu[0], bu[1]);
+                mma16816(avb[2 * np + 1], a, bu[2], bu[3]);
+            }
+        }
+        float hk_lo = 0.f, hk_hi = 0.f, hv_lo = 0.f, hv_hi = 0.f;
+        const bool okl = rl < L, okh = rh < L;
+        __nv_bfloat16* dvp = p.dv + row0 * DV;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int c = 64 * ch + 8 * j + 2 * (lane & 3);
+            const float2 kl = unpack_bf16(*reinterpret_cast<const uint32_t*>(s.K + swz<DK>(rl, c)));
+            const float2 kh = unpack_bf16(*reinterpret_cast<const uint32_t*>(s.K + swz<DK>(rh, c)));
+            const float2 vl = unpack_bf16(*reinterpret_cast<const uint32_t*>(s.V + swz<DV>(rl, c)));
+            const float2 vh = unpack_bf16(*reinterpret_cast<const uint32_t*>(s.V + swz<DV>(rh, c)));
+            hk_lo += akg[j][0] * kl.x + akg[j][1] * kl.y;
+            hk_hi += akg[j][2] * kh.x + akg[j][3] * kh.y;
+            hv_lo += avb[j][0] * vl.x + avb[j][1] * vl.y;
+            hv_hi += avb[j][2] * vh.x + avb[j][3] * vh.y;
+            dK[j][0] += bl * egl * akg[j][0]; dK[j][1] += bl * egl * akg[j][1];
+            dK[j][2] += bhh * egh * akg[j][2]; dK[j][3] += bhh * egh * akg[j][3];
+            if (okl)
+                *reinterpret_cast<uint32_t*>(dvp + (size_t)rl * rs * DV + c) =
+                    pack_bf16(bl * avb[j][0], bl * avb[j][1]);
+            if (okh)
+                *reinterpret_cast<uint32_t*>(dvp + (size_t)rh * rs * DV + c) =
+                    pack_bf16(bhh * avb[j][2], bhh * avb[j][3]);
+        }
+        row_b_lo += egl * hk_lo + hv_lo;
+        row_b_hi += egh * hk_hi + hv_hi;
+        row_g_lo += bl * egl * hk_lo;
+        row_g_hi += bhh * egh * hk_hi;
+    }
+    __syncthreads();
+
+    // ---- phase 4: dA = -T^T X (strictly lower) ------------------------------
+    {
+        float da[4][4] = {};
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+            if (kk < rb) continue;
+            uint32_t a[4];
+            lda_t<C>(a, s.Tb, m0, 16 * kk);
+#pragma unroll
+            for (int np = 0; np < 2; ++np) {
+                uint32_t bx[4];
+                ldb_kn<C>(bx, s.X, 16 * kk, 32 * ch + 16 * np);
+                mma16816(da[2 * np], a, bx[0], bx[1]);
+                mma16816(da[2 * np + 1], a, bx[2], bx[3]);
+            }
+        }
+        float colp[4][2];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int c0 = 32 * ch + 8 * j + 2 * (lane & 3);
+            float mm[4];
+            colp[j][0] = colp[j][1] = 0.f;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int r = (e < 2) ? rl : rh, c = c0 + (e & 1);
+                const float dA = (c < r) ? -da[j][e] : 0.f;
+                const float br = (e < 2) ? bl : bhh;
+                // M already carries the decay D
+                const float hA = dA * br * M[j][e];
+                if (e < 2) { row_b_lo += dA * M[j][e]; row_g_lo += hA; }
+                else { row_b_hi += dA * M[j][e]; row_g_hi += hA; }
+                colp[j][e & 1] -= hA;
+                mm[e] = (c < r) ? dA * br * __expf(s.G[r] - s.G[c]) : 0.f;
+            }
+            st_c<C>(s.dMM, m0, 32 * ch + 8 * j, mm);
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const float v = col_sum(colp[j][e]);
+                if (lane < 4) s.red_g[w][32 * ch + 8 * j + 2 * lane + e] += v;
+            }
+    }
+    __syncthreads();
+
+    // ---- phase 5: dK += dMM K + dMM^T K + scale dPG^T Q ; dQ' += dPG K -------
+    {
+        float tq[8][4] = {};
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+            uint32_t am[4], amt[4], ap[4], apt[4];
+            const bool lo = kk <= rb, hi = kk >= rb;
+            if (lo) { lda<C>(am, s.dMM, m0, 16 * kk); lda<C>(ap, s.dPG, m0, 16 * kk); }
+            if (hi) { lda_t<C>(amt, s.dMM, m0, 16 * kk); lda_t<C>(apt, s.dPG, m0, 16 * kk); }
+#pragma unroll
+            for (int np = 0; np < 4; ++np) {
+                uint32_t bk[4], bq[4];
+                ldb_kn<DK>(bk, s.K, 16 * kk, 64 * ch + 16 * np);
+                if (lo) {
+                    mma16816(dK[2 * np], am, bk[0], bk[1]);
+                    mma16816(dK[2 * np + 1], am, bk[2], bk[3]);
+                    mma16816(dQ[2 * np], ap, bk[0], bk[1]);
+                    mma16816(dQ[2 * np + 1], ap, bk[2], bk[3]);
+                }
+                if (hi) {
+                    ldb_kn<DK>(bq, s.Q, 16 * kk, 64 * ch + 16 * np);
+                    mma16816(dK[2 * np], amt, bk[0], bk[1]);
+                    mma16816(dK[2 * np + 1], amt, bk[2], bk[3]);
+                    mma16816(tq[2 * np], apt, bq[0], bq[1]);
+                    mma16816(tq[2 * np + 1], apt, bq[2], bq[3]);
+                }
+            }
+        }
+        const bool okl = rl < L, okh = rh < L;
+        __nv_bfloat16* dqp = p.dq + row0 * DK;
+        __nv_bfloat16* dkp = p.dk + row0 * DK;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int c = 64 * ch + 8 * j + 2 * (lane & 3);
+            if (okl) {
+                *reinterpret_cast<uint32_t*>(dqp + (size_t)rl * rs * DK + c) =
+                    pack_bf16(p.scale * dQ[j][0], p.scale * dQ[j][1]);
+                *reinterpret_cast<uint32_t*>(dkp + (size_t)rl * rs * DK + c) =
+                    pack_bf16(dK[j][0] + p.scale * tq[j][0], dK[j][1] + p.scale * tq[j][1]);
+            }
+            if (okh) {
+                *reinterpret_cast<uint32_t*>(dqp + (size_t)rh * rs * DK + c) =
+                    pack_bf16(p.scale * dQ[j][2], p.scale * dQ[j][3]);
+                *reinterpret_cast<uint32_t*>(dkp + (size_t)rh * rs * DK + c) =
+                    pack_bf16(dK[j][2] + p.scale * tq[j][2], dK[j][3] + p.scale * tq[j][3]);
+            }
+        }
+    }
+
+    // ---- per-token reductions: dbeta, dG -> dg --------------------------------
+    quad_rows(row_b_lo, row_b_hi);
+    quad_rows(row_g_lo, row_g_hi);
+    if ((lane & 3) == 0) {
+        s.red_b[w][rl] += row_b_lo;
+        s.red_b[w][rh] += row_b_hi;
+        s.red_g[w][rl] += row_g_lo;
+        s.red_g[w][rh] += row_g_hi;
+    }
+    __syncthreads();
+    if (w == 0) {
+        // red_s[w][0]: warp w's slice of <dS, S0>; red_s[w][1]: its rows' sum of
+        // e^{G_last-G_i} <dKt_i, k_i> over its column half.
+        float ssum = 0.f, lsum = 0.f;
+        for (int ww = 0; ww < 8; ++ww) {
+            ssum += s.red_s[ww][0];
+            lsum += s.red_s[ww][1];
+        }
+        float dG0 = 0.f, dG1 = 0.f, db0 = 0.f, db1 = 0.f;
+        for (int ww = 0; ww < 8; ++ww) {
+            dG0 += s.red_g[ww][lane];
+            dG1 += s.red_g[ww][lane + 32];
+            db0 += s.red_b[ww][lane];
+            db1 += s.red_b[ww][lane + 32];
+        }
+        if (lane == 31) dG1 += __expf(Gl) * ssum + lsum;
+        // reverse cumsum over the 64 tokens: dg_i = sum_{j >= i} dG_j
+        float x1 = dG1, x0 = dG0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float y1 = __shfl_down_sync(0xffffffffu, x1, o);
+            const float y0 = __shfl_down_sync(0xffffffffu, x0, o);
+            if (lane + o < 32) { x1 += y1; x0 += y0; }
+        }
+        x0 += __shfl_sync(0xffffffffu, x1, 0);
+        if (lane < L) {
+            p.dg[row0 + lane * rs] = x0;
+            p.dbeta[row0 + lane * rs] = db0;
+        }
+        if (lane + 32 < L) {
+            p.dg[row0 + (lane + 32) * rs] = x1;
+            p.dbeta[row0 + (lane + 32) * rs] = db1;
+        }
+    }
+}
+
+}  // namespace
+
+bool tc_bwd_supported(const gdn_dims& d) { return tc_supported(d); }
+
+void launch_tc_bwd(const gdn_dims& d, const void* q, const void* k, const void* v,
+                   const float* g, const float* beta, const float* h0, const void* dO,
+                   const float* dhT, void* dq, void* dk, void* dv, float* dg, float* dbeta,
+                   float* dh0, void* ws, cudaStream_t st) {
+    const TcLayout L = tc_layout(d, true);
+    char* base = (char*)ws;
+    ChunkPtrs cp{};
+    cp.q = (const __nv_bfloat16*)q; cp.k = (const __nv_bfloat16*)k; cp.v = (const __nv_bfloat16*)v;
+    cp.g = g; cp.beta = beta; cp.B = d.B; cp.T = d.T; cp.H = d.H; cp.NT = L.NT; cp.scale = d.scale;
+    cp.W = (__nv_bfloat16*)(base + L.W);
+    cp.Ut = (__nv_bfloat16*)(base + L.Ut);
+    cp.P = (__nv_bfloat16*)(base + L.P);
+    cp.G = (float*)(base + L.G);
+    cp.Tb = (__nv_bfloat16*)(base + L.Tb);
+    launch_prep(cp, L.nchunks, st);
+    launch_walk_states(d, L, cp, h0, ws, st);
+
+    BwPtrs bp{};
+    bp.q = cp.q; bp.k = cp.k; bp.dO = (const __nv_bfloat16*)dO; bp.dhT = dhT;
+    bp.W = cp.W; bp.P = cp.P; bp.G = cp.G;
+    bp.dSout = (__nv_bfloat16*)(base + L.dS);
+    bp.dUout = (__nv_bfloat16*)(base + L.dU);
+    bp.dh0 = dh0; bp.B = d.B; bp.T = d.T; bp.H = d.H; bp.NT = L.NT; bp.scale = d.scale;
+    {
+        const int smem = sizeof(BwSmem);
+        cudaFuncSetAttribute(tc_walk_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        GDN_LAUNCH("tc_walk_bwd", st,
+                   tc_walk_bwd_kernel<<<d.B * d.H * (DV / 16), 128, smem, st>>>(bp));
+    }
+    LocPtrs lp{};
+    lp.q = cp.q; lp.k = cp.k; lp.v = cp.v; lp.dO = bp.dO; lp.g = g; lp.beta = beta;
+    lp.S0 = (const __nv_bfloat16*)(base + L.S0);
+    lp.U = (const __nv_bfloat16*)(base + L.U);
+    lp.dS = bp.dSout; lp.dU = bp.dUout; lp.Tb = cp.Tb; lp.G = cp.G;
+    lp.dq = (__nv_bfloat16*)dq; lp.dk = (__nv_bfloat16*)dk; lp.dv = (__nv_bfloat16*)dv;
+    lp.dg = dg; lp.dbeta = dbeta;
+    lp.B = d.B; lp.T = d.T; lp.H = d.H; lp.NT = L.NT; lp.scale = d.scale;
+    {
+        const int smem = sizeof(LocSmem);
+        cudaFuncSetAttribute(tc_bwd_local_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        GDN_LAUNCH("tc_bwd_local", st,
+                   tc_bwd_local_kernel<<<(unsigned)L.nchunks, 256, smem, st>>>(lp));
+    }
+}
+
+}  // namespace gdn

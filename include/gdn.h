@@ -126,6 +126,18 @@ gdn_status gdn_recurrent_step(int N, int H, int dk, int dv, gdn_dtype dtype,
  * call on `ws`: GDN_ERR_DEVICE_TIMEOUT if a wait gave up, else GDN_OK. */
 gdn_status gdn_query_device_status(void *ws, gdn_stream_t stream);
 
+/* Per-launch timing, a profiling aid (off by default; no compute happens in
+ * these calls).  gdn_profile_begin(capacity) makes the calling host thread's
+ * next `capacity` kernel launches by this library record a CUDA event before
+ * and after each launch, on that launch's stream.  gdn_profile_end() stops
+ * recording, waits for the recorded events, writes up to `capacity` launch
+ * durations in milliseconds to `ms` and the kernel names (static strings) to
+ * `names` (either may be NULL), and returns how many launches were made while
+ * recording (may exceed what was stored), or -1 if recording was not on or a
+ * CUDA call failed.  Events are created on the first begin and kept. */
+gdn_status gdn_profile_begin(int capacity);
+int gdn_profile_end(float *ms, const char **names, int capacity);
+
 /* Static, human-readable name of a status code. */
 const char *gdn_status_string(gdn_status status);
 
