@@ -84,8 +84,11 @@ gdn_status gdn_chunk_fwd(const gdn_dims* d, const void* q, const void* k, const 
     cudaGetLastError();  // clear a stale error so it is not reported as ours
     if (ws && cudaMemsetAsync(ws, 0, sizeof(unsigned int), st) != cudaSuccess)
         return GDN_ERR_CUDA;
-    if (tc_supported(*d)) launch_tc_fwd(*d, q, k, v, g, beta, h0, o, hT, ws, st);
-    else launch_simt_fwd(*d, q, k, v, g, beta, h0, o, hT, ws, st);
+    if (tc_supported(*d)) {
+        if (!launch_tc_fwd(*d, q, k, v, g, beta, h0, o, hT, ws, st)) return GDN_ERR_CUDA;
+    } else {
+        launch_simt_fwd(*d, q, k, v, g, beta, h0, o, hT, ws, st);
+    }
     return launch_status();
 }
 
@@ -108,9 +111,10 @@ gdn_status gdn_chunk_bwd(const gdn_dims* d, const void* q, const void* k, const 
     cudaGetLastError();
     if (ws && cudaMemsetAsync(ws, 0, sizeof(unsigned int), st) != cudaSuccess)
         return GDN_ERR_CUDA;
-    if (tc_bwd_supported(*d))
-        launch_tc_bwd(*d, q, k, v, g, beta, h0, dO, dhT, dq, dk, dv, dg, dbeta, dh0, ws, st);
-    else
+    if (tc_bwd_supported(*d)) {
+        if (!launch_tc_bwd(*d, q, k, v, g, beta, h0, dO, dhT, dq, dk, dv, dg, dbeta, dh0, ws, st))
+            return GDN_ERR_CUDA;
+    } else
         launch_simt_bwd(*d, q, k, v, g, beta, h0, dO, dhT, dq, dk, dv, dg, dbeta, dh0, ws, st);
     return launch_status();
 }

@@ -29,10 +29,11 @@ bool tc_supported(const gdn_dims& d);
 bool tc_bwd_supported(const gdn_dims& d);
 size_t tc_fwd_workspace(const gdn_dims& d);
 size_t tc_bwd_workspace(const gdn_dims& d);
-void launch_tc_fwd(const gdn_dims& d, const void* q, const void* k, const void* v,
+// Return false if a TMA tensor map could not be encoded (nothing launched).
+bool launch_tc_fwd(const gdn_dims& d, const void* q, const void* k, const void* v,
                    const float* g, const float* beta, const float* h0, void* o, float* hT,
                    void* ws, cudaStream_t st);
-void launch_tc_bwd(const gdn_dims& d, const void* q, const void* k, const void* v,
+bool launch_tc_bwd(const gdn_dims& d, const void* q, const void* k, const void* v,
                    const float* g, const float* beta, const float* h0, const void* dO,
                    const float* dhT, void* dq, void* dk, void* dv, float* dg, float* dbeta,
                    float* dh0, void* ws, cudaStream_t st);

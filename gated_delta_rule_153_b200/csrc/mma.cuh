@@ -140,4 +140,78 @@ GDN_DEV void load_tile_async(__nv_bfloat16* X, const __nv_bfloat16* g, size_t gs
     }
 }
 
+// Copy a tile image (a contiguous run of `bytes`, multiple of 16) verbatim.
+GDN_DEV void load_image_async(void* X, const void* g, int bytes, int tid, int nthreads) {
+    for (int e = tid; e < bytes / 16; e += nthreads)
+        cp_async16((char*)X + 16 * e, (const char*)g + 16 * e);
+}
+
+}  // namespace gdn
+
+namespace gdn {
+
+// Layout classes: Swz<COLS> is the XOR-swizzled tile above; Pad<COLS> keeps
+// each row's COLS elements contiguous and in order (so a row can be filled by
+// one bulk copy) and pads the row pitch by 16 bytes, which also puts the
+// eight rows of an ldmatrix block in eight different bank groups.
+template <int COLS>
+struct Swz {
+    static constexpr int PITCH = COLS;
+    GDN_DEV static uint32_t off(int r, int c) { return swz<COLS>(r, c); }
+};
+template <int COLS>
+struct Pad {
+    static constexpr int PITCH = COLS + 8;
+    GDN_DEV static uint32_t off(int r, int c) { return r * PITCH + c; }
+};
+
+template <class LY>
+GDN_DEV void lda(uint32_t (&a)[4], const __nv_bfloat16* X, int m0, int k0) {
+    const int l = threadIdx.x & 31, idx = l >> 3;
+    ldsm_x4(a, smem_u32(X + LY::off(m0 + (l & 7) + (idx & 1) * 8, k0 + (idx >> 1) * 8)));
+}
+template <class LY>
+GDN_DEV void lda_t(uint32_t (&a)[4], const __nv_bfloat16* X, int m0, int k0) {
+    const int l = threadIdx.x & 31, idx = l >> 3;
+    ldsm_x4_t(a, smem_u32(X + LY::off(k0 + (l & 7) + (idx >> 1) * 8, m0 + (idx & 1) * 8)));
+}
+template <class LY>
+GDN_DEV void ldb_nk(uint32_t (&b)[4], const __nv_bfloat16* X, int n0, int k0) {
+    const int l = threadIdx.x & 31, idx = l >> 3;
+    ldsm_x4(b, smem_u32(X + LY::off(n0 + (l & 7) + (idx >> 1) * 8, k0 + (idx & 1) * 8)));
+}
+template <class LY>
+GDN_DEV void ldb_kn(uint32_t (&b)[4], const __nv_bfloat16* X, int k0, int n0) {
+    const int l = threadIdx.x & 31, idx = l >> 3;
+    ldsm_x4_t(b, smem_u32(X + LY::off(k0 + (l & 7) + (idx & 1) * 8, n0 + (idx >> 1) * 8)));
+}
+// Single n8 tile variants (x2): b[0], b[1] for n0..n0+7.
+GDN_DEV void ldsm_x2(uint32_t (&r)[2], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];\n"
+                 : "=r"(r[0]), "=r"(r[1]) : "r"(addr));
+}
+GDN_DEV void ldsm_x2_t(uint32_t (&r)[2], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];\n"
+                 : "=r"(r[0]), "=r"(r[1]) : "r"(addr));
+}
+// B[k][n] = X[n][k], one n8 tile: lanes 0-7 rows n0.., k0; lanes 8-15 rows n0.., k0+8.
+template <class LY>
+GDN_DEV void ldb_nk1(uint32_t (&b)[2], const __nv_bfloat16* X, int n0, int k0) {
+    const int l = threadIdx.x & 31, idx = (l >> 3) & 1;
+    ldsm_x2(b, smem_u32(X + LY::off(n0 + (l & 7), k0 + idx * 8)));
+}
+// B[k][n] = X[k][n], one n8 tile: lanes 0-7 rows k0.., lanes 8-15 rows k0+8..
+template <class LY>
+GDN_DEV void ldb_kn1(uint32_t (&b)[2], const __nv_bfloat16* X, int k0, int n0) {
+    const int l = threadIdx.x & 31, idx = (l >> 3) & 1;
+    ldsm_x2_t(b, smem_u32(X + LY::off(k0 + (l & 7) + idx * 8, n0)));
+}
+template <class LY>
+GDN_DEV void st_c(__nv_bfloat16* X, int m0, int n0, const float (&c)[4]) {
+    const int l = threadIdx.x & 31;
+    const int r = m0 + (l >> 2), col = n0 + 2 * (l & 3);
+    *reinterpret_cast<uint32_t*>(X + LY::off(r, col)) = pack_bf16(c[0], c[1]);
+    *reinterpret_cast<uint32_t*>(X + LY::off(r + 8, col)) = pack_bf16(c[2], c[3]);
+}
+
 }  // namespace gdn

@@ -27,6 +27,8 @@
 namespace gdn {
 namespace tc {
 void launch_prep(const ChunkPtrs& p, size_t nchunks, cudaStream_t st);
+bool chunk_ptrs(ChunkPtrs& p, const gdn_dims& d, const TcLayout& L, const void* q,
+                const void* k, const void* v, const float* g, const float* beta, void* ws);
 void launch_walk_states(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& cp,
                         const float* h0, void* ws, cudaStream_t st);
 }  // namespace tc
@@ -73,8 +75,8 @@ __device__ void bw_issue(BwStage& st, const BwPtrs& p, int b, int h, int bh, int
     const size_t cid = (size_t)bh * p.NT + n;
     load_tile_async<DK>(st.K, p.k + row0 * DK, (size_t)p.H * DK, C, L, tid, 128);
     load_tile_async<DK>(st.Q, p.q + row0 * DK, (size_t)p.H * DK, C, L, tid, 128);
-    load_tile_async<DK>(st.W, p.W + cid * C * DK, DK, C, C, tid, 128);
-    load_tile_async<C>(st.P, p.P + cid * C * C, C, C, C, tid, 128);
+    load_image_async(st.W, p.W + cid * C * DK, C * DK * 2, tid, 128);
+    load_image_async(st.P, p.P + cid * C * C, C * C * 2, tid, 128);
     for (int e = tid; e < C * 2; e += 128) {
         const int r = e >> 1, c = e & 1;
         const bool ok = r < L;
@@ -278,9 +280,9 @@ __global__ void __launch_bounds__(256) tc_bwd_local_kernel(LocPtrs p) {
     load_tile_async<DV>(s.dO, p.dO + row0 * DV, rs * DV, C, L, tid, 256);
     load_tile_async<DV>(s.U, p.U + (size_t)cid * C * DV, DV, C, C, tid, 256);
     load_tile_async<DV>(s.dU, p.dU + (size_t)cid * C * DV, DV, C, C, tid, 256);
-    load_tile_async<DK>(s.S0, p.S0 + (size_t)cid * DV * DK, DK, DV, DV, tid, 256);
+    load_image_async(s.S0, p.S0 + (size_t)cid * DV * DK, DV * DK * 2, tid, 256);
     load_tile_async<DK>(s.dS, p.dS + (size_t)cid * DV * DK, DK, DV, DV, tid, 256);
-    load_tile_async<C>(s.Tb, p.Tb + (size_t)cid * C * C, C, C, C, tid, 256);
+    load_image_async(s.Tb, p.Tb + (size_t)cid * C * C, C * C * 2, tid, 256);
     cp_async_commit();
     for (int e = tid; e < C; e += 256) {
         s.G[e] = p.G[(size_t)cid * C + e];
@@ -717,19 +719,14 @@ __global__ void __launch_bounds__(256) tc_bwd_local_kernel(LocPtrs p) {
 
 bool tc_bwd_supported(const gdn_dims& d) { return tc_supported(d); }
 
-void launch_tc_bwd(const gdn_dims& d, const void* q, const void* k, const void* v,
+bool launch_tc_bwd(const gdn_dims& d, const void* q, const void* k, const void* v,
                    const float* g, const float* beta, const float* h0, const void* dO,
                    const float* dhT, void* dq, void* dk, void* dv, float* dg, float* dbeta,
                    float* dh0, void* ws, cudaStream_t st) {
     const TcLayout L = tc_layout(d, true);
     char* base = (char*)ws;
-    ChunkPtrs cp{};
-    cp.q = (const __nv_bfloat16*)q; cp.k = (const __nv_bfloat16*)k; cp.v = (const __nv_bfloat16*)v;
-    cp.g = g; cp.beta = beta; cp.B = d.B; cp.T = d.T; cp.H = d.H; cp.NT = L.NT; cp.scale = d.scale;
-    cp.W = (__nv_bfloat16*)(base + L.W);
-    cp.Ut = (__nv_bfloat16*)(base + L.Ut);
-    cp.P = (__nv_bfloat16*)(base + L.P);
-    cp.G = (float*)(base + L.G);
+    ChunkPtrs cp;
+    if (!chunk_ptrs(cp, d, L, q, k, v, g, beta, ws)) return false;
     cp.Tb = (__nv_bfloat16*)(base + L.Tb);
     launch_prep(cp, L.nchunks, st);
     launch_walk_states(d, L, cp, h0, ws, st);
@@ -760,6 +757,7 @@ void launch_tc_bwd(const gdn_dims& d, const void* q, const void* k, const void* 
         GDN_LAUNCH("tc_bwd_local", st,
                    tc_bwd_local_kernel<<<(unsigned)L.nchunks, 256, smem, st>>>(lp));
     }
+    return true;
 }
 
 }  // namespace gdn

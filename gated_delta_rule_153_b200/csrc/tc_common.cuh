@@ -2,8 +2,10 @@
 // tensor-core chunkwise kernels (tc_chunk.cu forward pieces, tc_bwd.cu).
 #pragma once
 
+#include "async.cuh"
 #include "common.cuh"
 #include "mma.cuh"
+#include "tma.cuh"
 
 namespace gdn {
 namespace tc {
@@ -38,7 +40,16 @@ inline TcLayout tc_layout(const gdn_dims& d, bool bwd) {
     return L;
 }
 
+// Workspace images (written by prep with bulk stores, read back the same way):
+//   W   [chunk][64][128] bf16, Swz<128> tile image
+//   Ut  [chunk][8 tiles][64][16] bf16, value columns 16*tile .. +15, row-major
+//   P   [chunk][64][64]  bf16, Swz<64> tile image (scale folded in)
+//   G   [chunk][64] fp32 within-chunk cumsum of g (padding rows repeat the last)
+//   Tb  [chunk][64][64]  bf16, Swz<64> tile image of T = (I + A)^{-1}
+//   S0  [chunk][128][128] bf16, Swz<128> image of the chunk-start state
+//   U   [chunk][64][128] bf16 row-major;  dS, dU likewise (backward)
 struct ChunkPtrs {
+    CUtensorMap qmap, kmap, vmap;  // token maps of q, k, v (see tma.cuh)
     const __nv_bfloat16 *q, *k, *v;
     const float *g, *beta;
     int B, T, H, NT;
@@ -46,7 +57,14 @@ struct ChunkPtrs {
     __nv_bfloat16 *W, *Ut, *P;
     float* G;
     __nv_bfloat16* Tb;  // optional: bf16 T = (I + A)^{-1} per chunk (backward)
+    unsigned int* status;
 };
+
+// Round a dynamic shared-memory pointer up to the 1024-byte alignment that
+// 128-byte-swizzled TMA destinations need (launches request 1 KB extra).
+GDN_DEV unsigned char* align1k(unsigned char* p) {
+    return reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
 
 }  // namespace tc
 }  // namespace gdn
