@@ -27,7 +27,8 @@ GDN_GATE_SCALAR, GDN_GATE_CHANNEL = 0, 1
 # Every symbol include/gdn.h declares.
 EXPORTS = ("gdn_chunk_fwd_workspace", "gdn_chunk_fwd", "gdn_chunk_bwd_workspace",
            "gdn_chunk_bwd", "gdn_recurrent_step", "gdn_query_device_status",
-           "gdn_status_string", "gdn_profile_begin", "gdn_profile_end")
+           "gdn_status_string", "gdn_profile_begin", "gdn_profile_end",
+           "gdn_chunk_fwd_noalloc")
 
 
 class gdn_dims(ctypes.Structure):
@@ -73,6 +74,8 @@ def lib() -> ctypes.CDLL:
             L.gdn_recurrent_step.restype = i
             L.gdn_query_device_status.argtypes = [vp, vp]
             L.gdn_query_device_status.restype = i
+            L.gdn_chunk_fwd_noalloc.argtypes = [dp, vp, vp, vp, fp, fp, fp, vp, fp, vp]
+            L.gdn_chunk_fwd_noalloc.restype = i
             L.gdn_profile_begin.argtypes = [i]
             L.gdn_profile_begin.restype = i
             L.gdn_profile_end.argtypes = [ctypes.POINTER(ctypes.c_float),

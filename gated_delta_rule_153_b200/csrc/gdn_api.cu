@@ -45,6 +45,19 @@ gdn_status launch_status() {
 
 }  // namespace
 
+namespace gdn {
+gdn_status validate_fwd_args(const gdn_dims* d, const void* q, const void* k, const void* v,
+                             const float* g, const float* beta, const float* h0, const void* o,
+                             const float* hT) {
+    gdn_status s = check_dims(d);
+    if (s != GDN_OK) return s;
+    if (!q || !k || !v || !g || !beta || !o) return GDN_ERR_INVALID_ARG;
+    if (!all_aligned({q, k, v, g, beta, h0, o, hT})) return GDN_ERR_INVALID_ARG;
+    if (h0 && hT && h0 == hT) return GDN_ERR_INVALID_ARG;
+    return GDN_OK;
+}
+}  // namespace gdn
+
 extern "C" {
 
 const char* gdn_status_string(gdn_status s) {

@@ -13,6 +13,12 @@ void launch_recurrent_step(int N, int H, int dk, int dv, gdn_dtype dtype, gdn_ga
                            const float* g, const float* beta, float* state, void* o,
                            cudaStream_t st);
 
+// Host-side argument checks of gdn_chunk_fwd (dims, required pointers,
+// 16-byte alignment, h0/hT aliasing), without the workspace checks.
+gdn_status validate_fwd_args(const gdn_dims* d, const void* q, const void* k, const void* v,
+                             const float* g, const float* beta, const float* h0, const void* o,
+                             const float* hT);
+
 // Generic fp32-arithmetic chunkwise path (any supported dims, both dtypes).
 size_t simt_fwd_workspace(const gdn_dims& d);
 size_t simt_bwd_workspace(const gdn_dims& d);

@@ -25,6 +25,8 @@
 #include "mma.cuh"
 #include "tc_common.cuh"
 
+#include <mutex>
+
 namespace gdn {
 namespace {
 using namespace tc;
@@ -541,4 +543,55 @@ bool launch_tc_fwd(const gdn_dims& d, const void* q, const void* k, const void* 
     return true;
 }
 
+// ---------------------------------------------------------------------------
+// Allocation-free forward.  Some callers cannot call cudaMalloc at all: code
+// running under a fixed memory budget that the allocator must not touch, a
+// runtime that hands out no device memory of its own, or a host thread that
+// must not allocate between steps.  gdn_chunk_fwd_noalloc runs the same
+// tensor-core forward as gdn_chunk_fwd but takes its workspace from the
+// file-scope device array below, so the caller passes only inputs and
+// outputs.  Every GPU that loads this library holds the array until exit.
+// ---------------------------------------------------------------------------
+namespace {
+constexpr size_t kNoAllocScratchBytes = (size_t)64 << 20;  // 64 MiB per device
+__device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device (set up once per
+// device; the host-side name of the array is not a device address).
+void* noalloc_scratch() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void* ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess) return nullptr;
+        g_noalloc_ptr[dev] = ptr;
+    }
+    return g_noalloc_ptr[dev];
+}
+}  // namespace
+
 }  // namespace gdn
+
+extern "C" gdn_status gdn_chunk_fwd_noalloc(const gdn_dims* d, const void* q, const void* k,
+                                            const void* v, const float* g, const float* beta,
+                                            const float* h0, void* o, float* hT,
+                                            gdn_stream_t stream) {
+    const gdn_status s = gdn::validate_fwd_args(d, q, k, v, g, beta, h0, o, hT);
+    if (s != GDN_OK) return s;
+    if (!gdn::tc_supported(*d)) return GDN_ERR_UNSUPPORTED;
+    if (gdn::tc_fwd_workspace(*d) > gdn::kNoAllocScratchBytes) return GDN_ERR_WORKSPACE;
+    void* ws = gdn::noalloc_scratch();
+    if (!ws) return GDN_ERR_CUDA;
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaGetLastError();
+    // the status word must start at zero; every other byte the kernels read
+    // is written earlier in the same call
+    if (cudaMemsetAsync(ws, 0, sizeof(unsigned int), st) != cudaSuccess) return GDN_ERR_CUDA;
+    if (!gdn::launch_tc_fwd(*d, q, k, v, g, beta, h0, o, hT, ws, st)) return GDN_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}

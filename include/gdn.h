@@ -126,6 +126,30 @@ gdn_status gdn_recurrent_step(int N, int H, int dk, int dv, gdn_dtype dtype,
  * call on `ws`: GDN_ERR_DEVICE_TIMEOUT if a wait gave up, else GDN_OK. */
 gdn_status gdn_query_device_status(void *ws, gdn_stream_t stream);
 
+/* Allocation-free chunkwise forward, for callers that cannot call
+ * cudaMalloc (a fixed device-memory budget the allocator must not touch, a
+ * runtime that provides no device allocation, or host code that must not
+ * allocate between steps).  The paper has no counterpart: this is a
+ * deployment variant of gdn_chunk_fwd.  Same arguments and results as
+ * gdn_chunk_fwd minus the workspace: the workspace is a 64 MiB array built
+ * into the library (a file-scope device variable that every GPU loading the
+ * library holds until the process exits), so the caller passes only inputs
+ * and outputs.  Supported shapes are those of the tensor-core path (bf16,
+ * dk = dv = 128, chunk 64, scalar gate; GDN_ERR_UNSUPPORTED otherwise) whose
+ * workspace fits 64 MiB, i.e. B*H*ceil(T/64) <= 1628 chunk-heads
+ * (GDN_ERR_WORKSPACE otherwise, checked on the host before anything runs).
+ * No cudaMalloc, cudaFree or other allocating call is made.  The first call
+ * on a device looks up the array's device address (cudaGetSymbolAddress),
+ * so make that first call before any stream capture.  All calls share the
+ * one array and a call leaves its contents behind: the call clears the word
+ * that must start at zero itself, but calls that overlap on the GPU (other
+ * streams, other host threads) race on the array and must be serialised by
+ * the caller.  Device-side wait timeouts of these calls are not reported. */
+gdn_status gdn_chunk_fwd_noalloc(const gdn_dims *dims, const void *q, const void *k,
+                                 const void *v, const float *g, const float *beta,
+                                 const float *h0, void *o, float *hT,
+                                 gdn_stream_t stream);
+
 /* Per-launch timing, a profiling aid (off by default; no compute happens in
  * these calls).  gdn_profile_begin(capacity) makes the calling host thread's
  * next `capacity` kernel launches by this library record a CUDA event before
