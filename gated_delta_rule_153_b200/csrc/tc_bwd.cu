@@ -37,176 +37,187 @@ namespace {
 using namespace tc;
 
 // ---------------------------------------------------------------------------
-// reverse walk: dS for 16 value-rows, chunks NT-1 .. 0
+// reverse walk: dS for 16 value-rows, chunks NT-1 .. 0, 8 warps.
+// Warp w: tokens 8w..8w+7 of dU^T, key columns 16w..16w+15 of dS.
+// Chunk tiles arrive on a three-stage mbarrier ring (Q, K, dO by TMA tensor
+// maps; W, P, G by bulk copies of the workspace images).
 // ---------------------------------------------------------------------------
-struct BwStage {
-    __nv_bfloat16 W[C * DK];
-    __nv_bfloat16 Q[C * DK];
-    __nv_bfloat16 K[C * DK];
-    __nv_bfloat16 P[C * C];
-    __nv_bfloat16 dO[C][16];
+constexpr int BW_THREADS = 256;
+constexpr int BW_STAGES = 3;
+
+struct alignas(1024) BwStage {
+    __nv_bfloat16 Q[C * DK];   // Tma128
+    __nv_bfloat16 K[C * DK];   // Tma128
+    __nv_bfloat16 W[C * DK];   // Swz<128>
+    __nv_bfloat16 P[C * C];    // Swz<64>
+    __nv_bfloat16 dO[C * 16];  // [token][16 value columns]
     float G[C];
 };
 
 struct BwSmem {
-    BwStage st[2];
-    __nv_bfloat16 dS[16 * DK];  // bf16 copy of dS (rows x key columns)
-    __nv_bfloat16 dOt[16 * C];  // dO^T tile
-    __nv_bfloat16 dOg[16 * C];  // dO^T * scale * e^{G_i}
-    __nv_bfloat16 dU[16 * C];   // dU^T
+    BwStage st[BW_STAGES];
+    __nv_bfloat16 dS[16 * DK];  // Swz<128>: bf16 copy of dS (rows x key columns)
+    __nv_bfloat16 dOt[16 * C];  // Swz<64>: dO^T tile
+    __nv_bfloat16 dOg[16 * C];  // Swz<64>: dO^T * scale * e^{G_i}
+    __nv_bfloat16 dU[16 * C];   // Swz<64>: dU^T
+    __nv_bfloat16 dUst[C * 16]; // [token][row] staging for the dU store
+    uint64_t full[BW_STAGES];
 };
 
 struct BwPtrs {
-    const __nv_bfloat16 *q, *k, *dO;
+    CUtensorMap qmap, kmap, dOmap;
     const float* dhT;
     const __nv_bfloat16 *W, *P;
     const float* G;
     __nv_bfloat16 *dSout, *dUout;
     float* dh0;
+    unsigned int* status;
     int B, T, H, NT;
     float scale;
 };
 
-__device__ void bw_issue(BwStage& st, const BwPtrs& p, int b, int h, int bh, int n, int a0,
-                         int tid) {
-    const int t0 = n * C;
-    const int L = min(C, p.T - t0);
-    const size_t row0 = ((size_t)b * p.T + t0) * p.H + h;
+__device__ void bw_issue(BwStage& st, uint64_t* bar, const BwPtrs& p, int b, int h, int bh,
+                         int n, int a0) {
     const size_t cid = (size_t)bh * p.NT + n;
-    load_tile_async<DK>(st.K, p.k + row0 * DK, (size_t)p.H * DK, C, L, tid, 128);
-    load_tile_async<DK>(st.Q, p.q + row0 * DK, (size_t)p.H * DK, C, L, tid, 128);
-    load_image_async(st.W, p.W + cid * C * DK, C * DK * 2, tid, 128);
-    load_image_async(st.P, p.P + cid * C * C, C * C * 2, tid, 128);
-    for (int e = tid; e < C * 2; e += 128) {
-        const int r = e >> 1, c = e & 1;
-        const bool ok = r < L;
-        cp_async16_zfill(&st.dO[r][8 * c], p.dO + (row0 + (size_t)(ok ? r : 0) * p.H) * DV + a0 + 8 * c,
-                         ok);
-    }
-    for (int e = tid; e < C / 4; e += 128) cp_async16(&st.G[4 * e], p.G + cid * C + 4 * e);
-    cp_async_commit();
+    mbar_arrive_expect(bar, (3 * C * DK + C * C + C * 16) * 2 + C * 4);
+    const int tok = b * p.T + n * C;
+    tma_load_tile(st.Q, &p.qmap, h, tok, bar);
+    tma_load_tile(st.K, &p.kmap, h, tok, bar);
+    tma_load_3d(st.dO, &p.dOmap, a0, h, tok, bar);
+    bulk_g2s(st.W, p.W + cid * C * DK, C * DK * 2, bar);
+    bulk_g2s(st.P, p.P + cid * C * C, C * C * 2, bar);
+    bulk_g2s(st.G, p.G + cid * C, C * 4, bar);
 }
 
-__global__ void __launch_bounds__(128) tc_walk_bwd_kernel(BwPtrs p) {
-    extern __shared__ __align__(128) unsigned char smem_raw[];
-    BwSmem& s = *reinterpret_cast<BwSmem*>(smem_raw);
+__global__ void __launch_bounds__(BW_THREADS) tc_walk_bwd_kernel(const __grid_constant__ BwPtrs p) {
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    BwSmem& s = *reinterpret_cast<BwSmem*>(align1k(smem_raw));
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-    const int tiles = DV / 16;
-    const int bh = blockIdx.x / tiles, a0 = (blockIdx.x % tiles) * 16;
+    constexpr int TILES = DV / 16;
+    const int bh = blockIdx.x / TILES, a0 = (blockIdx.x % TILES) * 16;
     const int b = bh / p.H, h = bh % p.H;
     const int r_lo = lane >> 2;
+    const int i0 = 8 * w + 2 * (lane & 3);  // this thread's token pair in dU^T
 
-    float dS[4][4];
+    if (tid == 0) {
+        for (int i = 0; i < BW_STAGES; ++i) mbar_init(&s.full[i], 1);
+        fence_mbar_init();
+    }
+    // dS: rows r_lo, r_lo+8; columns 16w + 8j + 2(lane%4) + {0,1}
+    float dS[2][4];
     {
         const float* src = p.dhT ? p.dhT + ((size_t)bh * DV + a0) * DK : nullptr;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int c = 32 * w + 8 * j + 2 * (lane & 3);
+        for (int j = 0; j < 2; ++j) {
+            const int c = 16 * w + 8 * j + 2 * (lane & 3);
 #pragma unroll
             for (int e = 0; e < 4; ++e)
                 dS[j][e] = src ? src[(size_t)(r_lo + 8 * (e >> 1)) * DK + c + (e & 1)] : 0.f;
         }
     }
-    bw_issue(s.st[(p.NT - 1) & 1], p, b, h, bh, p.NT - 1, a0, tid);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) st_c<DK>(s.dS, 0, 32 * w + 8 * j, dS[j]);
-
-    for (int n = p.NT - 1; n >= 0; --n) {
-        BwStage& st = s.st[n & 1];
-        cp_async_wait<0>();
-        __syncthreads();
-        if (n > 0) bw_issue(s.st[(n - 1) & 1], p, b, h, bh, n - 1, a0, tid);
-        const size_t cid = (size_t)bh * p.NT + n;
-        // dO^T tiles, plain and scaled by scale*e^{G_i}
-        for (int e = tid; e < C * 16; e += 128) {
-            const int i = e >> 4, a = e & 15;
-            const float x = __bfloat162float(st.dO[i][a]);
-            s.dOt[swz<C>(a, i)] = st.dO[i][a];
-            s.dOg[swz<C>(a, i)] = __float2bfloat16_rn(x * p.scale * __expf(st.G[i]));
+    for (int j = 0; j < 2; ++j) st_c<Swz<128>>(s.dS, 0, 16 * w + 8 * j, dS[j]);
+    fence_async_smem();
+    __syncthreads();
+    if (tid == 0)
+        for (int k = 0; k < BW_STAGES - 1 && k < p.NT; ++k) {
+            const int n = p.NT - 1 - k;
+            bw_issue(s.st[k], &s.full[k], p, b, h, bh, n, a0);
         }
-        // dS leaving chunk n (bf16), rows a0.. of [dv][dk]
-        {
-            __nv_bfloat16* dst = p.dSout + (cid * DV + a0) * DK;
-            for (int e = tid; e < 16 * DK / 8; e += 128) {
-                const int r = e / (DK / 8), c8 = e % (DK / 8);
-                *reinterpret_cast<uint4*>(dst + (size_t)r * DK + 8 * c8) =
-                    *reinterpret_cast<const uint4*>(s.dS + swz<DK>(r, 8 * c8));
-            }
+
+    for (int k = 0; k < p.NT; ++k) {  // k-th step handles chunk n = NT-1-k
+        const int n = p.NT - 1 - k;
+        const int sk = k % BW_STAGES;
+        BwStage& st = s.st[sk];
+        if (!mbar_wait(&s.full[sk], (k / BW_STAGES) & 1, p.status)) return;
+        __syncthreads();  // stage landed; dS written; stage of step k-1 is free
+        if (tid == 0 && k + BW_STAGES - 1 < p.NT) {
+            const int kk = k + BW_STAGES - 1;
+            bw_issue(s.st[kk % BW_STAGES], &s.full[kk % BW_STAGES], p, b, h, bh, p.NT - 1 - kk, a0);
+        }
+        const size_t cid = (size_t)bh * p.NT + n;
+        const int L = min(C, p.T - n * C);
+        if (tid == 0) {  // dS leaving chunk n (Swz<128> image rows a0..)
+            bulk_s2g(p.dSout + (cid * DV + a0) * DK, s.dS, 16 * DK * 2);
+            bulk_commit();
+        }
+        // dO^T tiles (rows past the sequence end are zeroed: they are not ours)
+        for (int e = tid; e < C * 16; e += BW_THREADS) {
+            const int i = e >> 4, a = e & 15;
+            const float x = i < L ? __bfloat162float(st.dO[i * 16 + a]) : 0.f;
+            s.dOt[swz<C>(a, i)] = __float2bfloat16_rn(x);
+            s.dOg[swz<C>(a, i)] = __float2bfloat16_rn(x * p.scale * __expf(st.G[i]));
         }
         __syncthreads();
         const float Gl = st.G[C - 1];
-        // dU^T (rows x tokens 16w..16w+15)
+        // dU^T (rows x tokens 8w..8w+7) = dO^T P + (dS K^T) .* e^{G_last - G_r}
         {
-            float a1[2][4] = {}, a2[2][4] = {};
+            float a1[4] = {}, a2[2][4] = {};
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
-                if (kk < w) continue;  // P[i][r] = 0 for i < r
-                uint32_t a[4], bp[4];
-                lda<C>(a, s.dOt, 0, 16 * kk);
-                ldb_kn<C>(bp, st.P, 16 * kk, 16 * w);
-                mma16816(a1[0], a, bp[0], bp[1]);
-                mma16816(a1[1], a, bp[2], bp[3]);
+                if (16 * kk + 15 < 8 * w) continue;  // P[i][r] = 0 for i < r
+                uint32_t a[4], bp[2];
+                lda<Swz<64>>(a, s.dOt, 0, 16 * kk);
+                ldb_kn1<Swz<64>>(bp, st.P, 16 * kk, 8 * w);
+                mma16816(a1, a, bp[0], bp[1]);
             }
 #pragma unroll
             for (int kk = 0; kk < DK / 16; ++kk) {
-                uint32_t a[4], bk[4];
-                lda<DK>(a, s.dS, 0, 16 * kk);
-                ldb_nk<DK>(bk, st.K, 16 * w, 16 * kk);
-                mma16816(a2[0], a, bk[0], bk[1]);
-                mma16816(a2[1], a, bk[2], bk[3]);
+                uint32_t a[4], bk[2];
+                lda<Swz<128>>(a, s.dS, 0, 16 * kk);
+                ldb_nk1<Tma128>(bk, st.K, 8 * w, 16 * kk);
+                mma16816(a2[kk & 1], a, bk[0], bk[1]);
             }
+            float u[4];
 #pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                const int r0 = 16 * w + 8 * j + 2 * (lane & 3);
-                float u[4];
+            for (int e = 0; e < 4; ++e)  // padding tokens (past the sequence end) stay zero
+                u[e] = (i0 + (e & 1) < L)
+                           ? a1[e] + (a2[0][e] + a2[1][e]) * __expf(Gl - st.G[i0 + (e & 1)])
+                           : 0.f;
+            st_c<Swz<64>>(s.dU, 0, 8 * w, u);
 #pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    u[e] = a1[j][e] + a2[j][e] * __expf(Gl - st.G[r0 + (e & 1)]);
-                st_c<C>(s.dU, 0, 16 * w + 8 * j, u);
-            }
+            for (int e = 0; e < 4; ++e)
+                s.dUst[(i0 + (e & 1)) * 16 + r_lo + 8 * (e >> 1)] = __float2bfloat16_rn(u[e]);
         }
+        if (tid == 0) bulk_wait_read<0>();  // dS image read before it is rewritten
         __syncthreads();
-        {
-            __nv_bfloat16* dst = p.dUout + cid * C * DV + a0;
-            for (int e = tid; e < C * 16; e += 128) {
-                const int i = e >> 4, a = e & 15;
-                dst[(size_t)i * DV + a] = s.dU[swz<C>(a, i)];
-            }
-        }
-        // dS0 = e^{G_last} dS + dOg^T Q - dU^T W   (columns 32w..32w+31)
+        // dS0 = e^{G_last} dS + dOg^T Q - dU^T W   (columns 16w..16w+15)
         {
             const float gam = __expf(Gl);
-            float y[4][4] = {}, z[4][4] = {};
+            float y[2][4] = {}, z[2][4] = {};
 #pragma unroll
             for (int kk = 0; kk < C / 16; ++kk) {
-                uint32_t ag[4], au[4];
-                lda<C>(ag, s.dOg, 0, 16 * kk);
-                lda<C>(au, s.dU, 0, 16 * kk);
-#pragma unroll
-                for (int np = 0; np < 2; ++np) {
-                    uint32_t bq[4], bw[4];
-                    ldb_kn<DK>(bq, st.Q, 16 * kk, 32 * w + 16 * np);
-                    ldb_kn<DK>(bw, st.W, 16 * kk, 32 * w + 16 * np);
-                    mma16816(y[2 * np], ag, bq[0], bq[1]);
-                    mma16816(y[2 * np + 1], ag, bq[2], bq[3]);
-                    mma16816(z[2 * np], au, bw[0], bw[1]);
-                    mma16816(z[2 * np + 1], au, bw[2], bw[3]);
-                }
+                uint32_t ag[4], au[4], bq[4], bw[4];
+                lda<Swz<64>>(ag, s.dOg, 0, 16 * kk);
+                lda<Swz<64>>(au, s.dU, 0, 16 * kk);
+                ldb_kn<Tma128>(bq, st.Q, 16 * kk, 16 * w);
+                ldb_kn<Swz<128>>(bw, st.W, 16 * kk, 16 * w);
+                mma16816(y[0], ag, bq[0], bq[1]);
+                mma16816(y[1], ag, bq[2], bq[3]);
+                mma16816(z[0], au, bw[0], bw[1]);
+                mma16816(z[1], au, bw[2], bw[3]);
             }
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
+            for (int j = 0; j < 2; ++j)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) dS[j][e] = gam * dS[j][e] + y[j][e] - z[j][e];
         }
-        __syncthreads();
+        __syncthreads();  // everyone done with dS, dOt, dOg, dU; dU staged
 #pragma unroll
-        for (int j = 0; j < 4; ++j) st_c<DK>(s.dS, 0, 32 * w + 8 * j, dS[j]);
+        for (int j = 0; j < 2; ++j) st_c<Swz<128>>(s.dS, 0, 16 * w + 8 * j, dS[j]);
+        fence_async_smem();
+        if (tid < 2 * C) {  // dU rows (tokens x value rows a0..a0+15), 16-byte pieces
+            const int i = tid >> 1, hf = tid & 1;
+            *reinterpret_cast<uint4*>(p.dUout + (cid * C + i) * DV + a0 + 8 * hf) =
+                *reinterpret_cast<const uint4*>(&s.dUst[i * 16 + 8 * hf]);
+        }
     }
+    if (tid == 0) bulk_wait<0>();
     if (p.dh0) {
         float* dst = p.dh0 + ((size_t)bh * DV + a0) * DK;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int c = 32 * w + 8 * j + 2 * (lane & 3);
+        for (int j = 0; j < 2; ++j) {
+            const int c = 16 * w + 8 * j + 2 * (lane & 3);
 #pragma unroll
             for (int e = 0; e < 4; ++e) dst[(size_t)(r_lo + 8 * (e >> 1)) * DK + c + (e & 1)] = dS[j][e];
         }
@@ -281,7 +292,7 @@ __global__ void __launch_bounds__(256) tc_bwd_local_kernel(LocPtrs p) {
     load_tile_async<DV>(s.U, p.U + (size_t)cid * C * DV, DV, C, C, tid, 256);
     load_tile_async<DV>(s.dU, p.dU + (size_t)cid * C * DV, DV, C, C, tid, 256);
     load_image_async(s.S0, p.S0 + (size_t)cid * DV * DK, DV * DK * 2, tid, 256);
-    load_tile_async<DK>(s.dS, p.dS + (size_t)cid * DV * DK, DK, DV, DV, tid, 256);
+    load_image_async(s.dS, p.dS + (size_t)cid * DV * DK, DV * DK * 2, tid, 256);
     load_image_async(s.Tb, p.Tb + (size_t)cid * C * C, C * C * 2, tid, 256);
     cp_async_commit();
     for (int e = tid; e < C; e += 256) {
@@ -732,19 +743,22 @@ bool launch_tc_bwd(const gdn_dims& d, const void* q, const void* k, const void* 
     launch_walk_states(d, L, cp, h0, ws, st);
 
     BwPtrs bp{};
-    bp.q = cp.q; bp.k = cp.k; bp.dO = (const __nv_bfloat16*)dO; bp.dhT = dhT;
-    bp.W = cp.W; bp.P = cp.P; bp.G = cp.G;
+    bp.qmap = cp.qmap; bp.kmap = cp.kmap;
+    if (!encode_token_map(&bp.dOmap, dO, d.B, d.T, d.H, 16)) return false;
+    bp.dhT = dhT; bp.W = cp.W; bp.P = cp.P; bp.G = cp.G;
     bp.dSout = (__nv_bfloat16*)(base + L.dS);
     bp.dUout = (__nv_bfloat16*)(base + L.dU);
-    bp.dh0 = dh0; bp.B = d.B; bp.T = d.T; bp.H = d.H; bp.NT = L.NT; bp.scale = d.scale;
+    bp.dh0 = dh0; bp.status = cp.status;
+    bp.B = d.B; bp.T = d.T; bp.H = d.H; bp.NT = L.NT; bp.scale = d.scale;
     {
-        const int smem = sizeof(BwSmem);
+        const int smem = sizeof(BwSmem) + 1024;
         cudaFuncSetAttribute(tc_walk_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         GDN_LAUNCH("tc_walk_bwd", st,
-                   tc_walk_bwd_kernel<<<d.B * d.H * (DV / 16), 128, smem, st>>>(bp));
+                   tc_walk_bwd_kernel<<<d.B * d.H * (DV / 16), BW_THREADS, smem, st>>>(bp));
     }
     LocPtrs lp{};
-    lp.q = cp.q; lp.k = cp.k; lp.v = cp.v; lp.dO = bp.dO; lp.g = g; lp.beta = beta;
+    lp.q = cp.q; lp.k = cp.k; lp.v = cp.v; lp.dO = (const __nv_bfloat16*)dO; lp.g = g;
+    lp.beta = beta;
     lp.S0 = (const __nv_bfloat16*)(base + L.S0);
     lp.U = (const __nv_bfloat16*)(base + L.U);
     lp.dS = bp.dSout; lp.dU = bp.dUout; lp.Tb = cp.Tb; lp.G = cp.G;

@@ -145,7 +145,8 @@ __global__ void __launch_bounds__(128) tc_prep_kernel(const __grid_constant__ Ch
                 const int r = (e < 2) ? ra : rb2, c = c0 + (e & 1);
                 const float dec = (live && c <= r) ? __expf(((e < 2) ? Gra : Grb) - s.G[c]) : 0.f;
                 a[e] = (c < r) ? ((e < 2) ? bra : brb) * acck[j][e] * dec : 0.f;
-                pv[e] = accq[j][e] * dec * p.scale;
+                // rows past the sequence end are zero (their q rows are not ours)
+                pv[e] = (r < L) ? accq[j][e] * dec * p.scale : 0.f;
                 if ((j >> 1) == warp) s.Ad[warp][r - m0][c - m0] = a[e];
             }
             st_c<S64>(s.Ab, m0, 8 * j, a);

@@ -39,8 +39,11 @@ GDN_DEV void tma_load_tile(__nv_bfloat16* tile, const CUtensorMap* map, int head
     tma_load_3d(tile + 64 * 64, map, 64, head, token, bar);
 }
 
-// Host: encode the token map of a [B, T, H, 128] bf16 tensor.  Returns false
+// Host: encode the token map of a [B, T, H, 128] bf16 tensor.  box_cols 64
+// gives 128-byte-swizzled 64x64 boxes (Tma128 tiles); box_cols 16 gives
+// unswizzled 64-row x 16-column boxes (32-byte rows).  Returns false
 // if the driver entry point is unavailable or the encoder rejects the map.
-bool encode_token_map(CUtensorMap* map, const void* base, int B, int T, int H);
+bool encode_token_map(CUtensorMap* map, const void* base, int B, int T, int H,
+                      int box_cols = 64);
 
 }  // namespace gdn
