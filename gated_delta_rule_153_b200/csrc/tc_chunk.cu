@@ -278,21 +278,24 @@ __global__ void __launch_bounds__(128) tc_prep_kernel(const __grid_constant__ Ch
 constexpr int WALK_THREADS = 256;
 constexpr int WALK_STAGES = 3;
 
+// One CTA walks 16*MT value rows of one head's state (MT m-tiles per warp).
+template <int MT>
 struct alignas(1024) WalkStage {
     __nv_bfloat16 Q[C * DK];                 // Tma128
     __nv_bfloat16 K[C * DK];                 // Tma128
     __nv_bfloat16 W[C * DK];                 // Swz<128>
     __nv_bfloat16 P[C * C];                  // Swz<64>
-    __nv_bfloat16 Ut[C * 16];                // [token][16 value rows]
+    __nv_bfloat16 Ut[MT][C * 16];            // [tile][token][16 value rows]
     float G[C];
 };
 
+template <int MT>
 struct WalkSmem {
-    WalkStage st[WALK_STAGES];
-    __nv_bfloat16 S0[16 * DK];   // Swz<128>: bf16 copy of the state entering the chunk
-    __nv_bfloat16 Uu[16 * C];    // Swz<64>: U^T (rows of S x tokens)
-    __nv_bfloat16 Us[16 * C];    // Swz<64>: U^T scaled by e^{G_last - G_i}
-    __nv_bfloat16 O[C * 16];     // [token][row] staging (O, or U in MODE 1)
+    WalkStage<MT> st[WALK_STAGES];
+    __nv_bfloat16 S0[16 * MT * DK];   // Swz<128>: bf16 copy of the state entering the chunk
+    __nv_bfloat16 Uu[16 * MT * C];    // Swz<64>: U^T (rows of S x tokens)
+    __nv_bfloat16 Us[16 * MT * C];    // Swz<64>: U^T scaled by e^{G_last - G_i}
+    __nv_bfloat16 O[C * 16 * MT];     // [token][row] staging (O, or U in MODE 1)
     uint64_t full[WALK_STAGES];
 };
 
@@ -309,26 +312,28 @@ struct WalkPtrs {
     float scale;
 };
 
-__device__ void walk_issue(WalkStage& st, uint64_t* bar, const WalkPtrs& p, int b, int h,
-                           int bh, int n, int tile) {
+template <int MT>
+__device__ void walk_issue(WalkStage<MT>& st, uint64_t* bar, const WalkPtrs& p, int b, int h,
+                           int bh, int n, int tile0) {
     const size_t cid = (size_t)bh * p.NT + n;
-    mbar_arrive_expect(bar, (3 * C * DK + C * C + C * 16) * 2 + C * 4);
+    mbar_arrive_expect(bar, (3 * C * DK + C * C + MT * C * 16) * 2 + C * 4);
     const int tok = b * p.T + n * C;
     tma_load_tile(st.Q, &p.qmap, h, tok, bar);
     tma_load_tile(st.K, &p.kmap, h, tok, bar);
     bulk_g2s(st.W, p.W + cid * C * DK, C * DK * 2, bar);
     bulk_g2s(st.P, p.P + cid * C * C, C * C * 2, bar);
-    bulk_g2s(st.Ut, p.Ut + (cid * 8 + tile) * C * 16, C * 16 * 2, bar);
+    bulk_g2s(&st.Ut[0][0], p.Ut + (cid * 8 + tile0) * C * 16, MT * C * 16 * 2, bar);
     bulk_g2s(st.G, p.G + cid * C, C * 4, bar);
 }
 
-template <int MODE>
+template <int MT, int MODE>
 __global__ void __launch_bounds__(WALK_THREADS) tc_walk_kernel(const __grid_constant__ WalkPtrs p) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
-    WalkSmem& s = *reinterpret_cast<WalkSmem*>(align1k(smem_raw));
+    WalkSmem<MT>& s = *reinterpret_cast<WalkSmem<MT>*>(align1k(smem_raw));
+    constexpr int RT = 16 * MT;           // value rows of this CTA
+    constexpr int TILES = DV / RT;
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-    constexpr int TILES = DV / 16;
-    const int bh = blockIdx.x / TILES, tile = blockIdx.x % TILES, a0 = tile * 16;
+    const int bh = blockIdx.x / TILES, tile0 = (blockIdx.x % TILES) * MT, a0 = tile0 * 16;
     const int b = bh / p.H, h = bh % p.H;
     const int r_lo = lane >> 2;
     const int i0 = 8 * w + 2 * (lane & 3);  // this thread's token pair in the U/O tiles
@@ -337,118 +342,145 @@ __global__ void __launch_bounds__(WALK_THREADS) tc_walk_kernel(const __grid_cons
         for (int i = 0; i < WALK_STAGES; ++i) mbar_init(&s.full[i], 1);
         fence_mbar_init();
     }
-    // fp32 state: rows r_lo, r_lo+8; columns 16w + 8j + 2(lane%4) + {0,1}
-    float S[2][4];
+    // fp32 state: m-tile mt, rows 16mt + r_lo (+8); columns 16w + 8j + 2(lane%4) + {0,1}
+    float S[MT][2][4];
     {
         const float* h0 = p.h0 ? p.h0 + ((size_t)bh * DV + a0) * DK : nullptr;
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
-            const int c = 16 * w + 8 * j + 2 * (lane & 3);
+        for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-                S[j][e] = h0 ? h0[(size_t)(r_lo + 8 * (e >> 1)) * DK + c + (e & 1)] : 0.f;
-        }
+            for (int j = 0; j < 2; ++j) {
+                const int c = 16 * w + 8 * j + 2 * (lane & 3);
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    S[mt][j][e] = h0 ? h0[(size_t)(16 * mt + r_lo + 8 * (e >> 1)) * DK + c + (e & 1)] : 0.f;
+            }
     }
 #pragma unroll
-    for (int j = 0; j < 2; ++j) st_c<S128>(s.S0, 0, 16 * w + 8 * j, S[j]);
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) st_c<S128>(s.S0, 16 * mt, 16 * w + 8 * j, S[mt][j]);
     if (MODE == 1) fence_async_smem();
     __syncthreads();
     if (tid == 0)
         for (int n = 0; n < WALK_STAGES - 1 && n < p.NT; ++n)
-            walk_issue(s.st[n], &s.full[n], p, b, h, bh, n, tile);
+            walk_issue<MT>(s.st[n], &s.full[n], p, b, h, bh, n, tile0);
 
     for (int n = 0; n < p.NT; ++n) {
         const int sn = n % WALK_STAGES;
-        WalkStage& st = s.st[sn];
+        WalkStage<MT>& st = s.st[sn];
         if (!mbar_wait(&s.full[sn], (n / WALK_STAGES) & 1, p.status)) return;
         __syncthreads();  // stage n landed; S0 written; stage of chunk n-1 is free
         if (tid == 0 && n + WALK_STAGES - 1 < p.NT) {
             const int nn = n + WALK_STAGES - 1;
-            walk_issue(s.st[nn % WALK_STAGES], &s.full[nn % WALK_STAGES], p, b, h, bh, nn, tile);
+            walk_issue<MT>(s.st[nn % WALK_STAGES], &s.full[nn % WALK_STAGES], p, b, h, bh, nn, tile0);
         }
         const int L = min(C, p.T - n * C);
         const size_t cid = (size_t)bh * p.NT + n;
         if (MODE == 1 && tid == 0) {  // chunk-start state rows a0.. (Swz<128> image)
-            bulk_s2g(p.S0out + (cid * DV + a0) * DK, s.S0, 16 * DK * 2);
+            bulk_s2g(p.S0out + (cid * DV + a0) * DK, s.S0, RT * DK * 2);
             bulk_commit();
         }
+        const float Gl = st.G[C - 1];
+        const float et0 = __expf(Gl - st.G[i0]), et1 = __expf(Gl - st.G[i0 + 1]);
 
         // X = S0 W^T, Y = S0 Q^T for tokens 8w..8w+7 (two accumulators each)
-        float X[2][4] = {}, Y[2][4] = {};
+        float X[MT][2][4] = {}, Y[MT][2][4] = {};
 #pragma unroll
         for (int kk = 0; kk < DK / 16; ++kk) {
-            uint32_t a[4], bw[2];
-            lda<S128>(a, s.S0, 0, 16 * kk);
+            uint32_t bw[2], bq[2];
             ldb_nk1<S128>(bw, st.W, 8 * w, 16 * kk);
-            mma16816(X[kk & 1], a, bw[0], bw[1]);
-            if (MODE == 0) {
-                uint32_t bq[2];
-                ldb_nk1<Tma128>(bq, st.Q, 8 * w, 16 * kk);
-                mma16816(Y[kk & 1], a, bq[0], bq[1]);
+            if (MODE == 0) ldb_nk1<Tma128>(bq, st.Q, 8 * w, 16 * kk);
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                uint32_t a[4];
+                lda<S128>(a, s.S0, 16 * mt, 16 * kk);
+                mma16816(X[mt][kk & 1], a, bw[0], bw[1]);
+                if (MODE == 0) mma16816(Y[mt][kk & 1], a, bq[0], bq[1]);
             }
         }
-        const float Gl = st.G[C - 1];
-        float u[4], us[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int r = r_lo + 8 * (e >> 1), i = i0 + (e & 1);
-            u[e] = __bfloat162float(st.Ut[i * 16 + r]) - (X[0][e] + X[1][e]);
-            us[e] = u[e] * __expf(Gl - st.G[i]);
-        }
-        st_c<S64>(s.Uu, 0, 8 * w, u);
-        st_c<S64>(s.Us, 0, 8 * w, us);
-        if (MODE == 1) {
+        for (int mt = 0; mt < MT; ++mt) {
+            float u[4], us[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-                s.O[(i0 + (e & 1)) * 16 + r_lo + 8 * (e >> 1)] = __float2bfloat16_rn(u[e]);
-            if (tid == 0) bulk_wait_read<0>();  // S0 image read before it is rewritten
+            for (int e = 0; e < 4; ++e) {
+                const int r = r_lo + 8 * (e >> 1), i = i0 + (e & 1);
+                u[e] = __bfloat162float(st.Ut[mt][i * 16 + r]) - (X[mt][0][e] + X[mt][1][e]);
+                us[e] = u[e] * ((e & 1) ? et1 : et0);
+            }
+            st_c<S64>(s.Uu, 16 * mt, 8 * w, u);
+            st_c<S64>(s.Us, 16 * mt, 8 * w, us);
+            if (MODE == 1) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    s.O[(i0 + (e & 1)) * RT + 16 * mt + r_lo + 8 * (e >> 1)] = __float2bfloat16_rn(u[e]);
+            }
         }
+        if (MODE == 1 && tid == 0) bulk_wait_read<0>();  // S0 image read before it is rewritten
         __syncthreads();
 
         // S1 = e^{G_last} S0 + (U^T .* e^{G_last - G}) K, columns 16w..16w+15
         const float gam = __expf(Gl);
 #pragma unroll
-        for (int j = 0; j < 2; ++j)
+        for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) S[j][e] *= gam;
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) S[mt][j][e] *= gam;
 #pragma unroll
         for (int kk = 0; kk < C / 16; ++kk) {
-            uint32_t a[4], bk[4];
-            lda<S64>(a, s.Us, 0, 16 * kk);
+            uint32_t bk[4];
             ldb_kn<Tma128>(bk, st.K, 16 * kk, 16 * w);
-            mma16816(S[0], a, bk[0], bk[1]);
-            mma16816(S[1], a, bk[2], bk[3]);
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                uint32_t a[4];
+                lda<S64>(a, s.Us, 16 * mt, 16 * kk);
+                mma16816(S[mt][0], a, bk[0], bk[1]);
+                mma16816(S[mt][1], a, bk[2], bk[3]);
+            }
         }
         if (MODE == 0) {
             // O^T (rows x tokens 8w..) = scale e^{G_i} Y + U^T P^T
-            float o[4];
+            const float eg0 = p.scale * __expf(st.G[i0]), eg1 = p.scale * __expf(st.G[i0 + 1]);
+            float o[MT][4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-                o[e] = (Y[0][e] + Y[1][e]) * p.scale * __expf(st.G[i0 + (e & 1)]);
+            for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    o[mt][e] = (Y[mt][0][e] + Y[mt][1][e]) * ((e & 1) ? eg1 : eg0);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
                 if (16 * kk > 8 * w + 7) break;  // P[r][i] = 0 for i > r
-                uint32_t a[4], bp[2];
-                lda<S64>(a, s.Uu, 0, 16 * kk);
+                uint32_t bp[2];
                 ldb_nk1<S64>(bp, st.P, 8 * w, 16 * kk);
-                mma16816(o, a, bp[0], bp[1]);
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt) {
+                    uint32_t a[4];
+                    lda<S64>(a, s.Uu, 16 * mt, 16 * kk);
+                    mma16816(o[mt], a, bp[0], bp[1]);
+                }
             }
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-                s.O[(i0 + (e & 1)) * 16 + r_lo + 8 * (e >> 1)] = __float2bfloat16_rn(o[e]);
+            for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    s.O[(i0 + (e & 1)) * RT + 16 * mt + r_lo + 8 * (e >> 1)] = __float2bfloat16_rn(o[mt][e]);
         }
         __syncthreads();  // done with S0, Uu, Us; O / U staged
 #pragma unroll
-        for (int j = 0; j < 2; ++j) st_c<S128>(s.S0, 0, 16 * w + 8 * j, S[j]);
+        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+            for (int j = 0; j < 2; ++j) st_c<S128>(s.S0, 16 * mt, 16 * w + 8 * j, S[mt][j]);
         if (MODE == 1) fence_async_smem();
-        if (tid < 2 * L) {  // 16-byte row pieces of O (or U): row tid/2, half tid%2
-            const int i = tid >> 1, hf = tid & 1;
-            const uint4 v = *reinterpret_cast<const uint4*>(&s.O[i * 16 + 8 * hf]);
+        constexpr int PIECES = RT / 8;  // 16-byte pieces per token row
+        for (int e = tid; e < PIECES * L; e += WALK_THREADS) {
+            const int i = e / PIECES, pc = e % PIECES;
+            const uint4 v = *reinterpret_cast<const uint4*>(&s.O[i * RT + 8 * pc]);
             if (MODE == 0) {
                 const size_t row = ((size_t)b * p.T + n * C + i) * p.H + h;
-                *reinterpret_cast<uint4*>(p.o + row * DV + a0 + 8 * hf) = v;
+                *reinterpret_cast<uint4*>(p.o + row * DV + a0 + 8 * pc) = v;
             } else {
-                *reinterpret_cast<uint4*>(p.Uout + (cid * C + i) * DV + a0 + 8 * hf) = v;
+                *reinterpret_cast<uint4*>(p.Uout + (cid * C + i) * DV + a0 + 8 * pc) = v;
             }
         }
     }
@@ -456,11 +488,14 @@ __global__ void __launch_bounds__(WALK_THREADS) tc_walk_kernel(const __grid_cons
     if (MODE == 0 && p.hT) {
         float* hT = p.hT + ((size_t)bh * DV + a0) * DK;
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
-            const int c = 16 * w + 8 * j + 2 * (lane & 3);
+        for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) hT[(size_t)(r_lo + 8 * (e >> 1)) * DK + c + (e & 1)] = S[j][e];
-        }
+            for (int j = 0; j < 2; ++j) {
+                const int c = 16 * w + 8 * j + 2 * (lane & 3);
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    hT[(size_t)(16 * mt + r_lo + 8 * (e >> 1)) * DK + c + (e & 1)] = S[mt][j][e];
+            }
     }
 }
 
@@ -481,13 +516,24 @@ bool make_chunk_ptrs(ChunkPtrs& p, const gdn_dims& d, const TcLayout& L, const v
     return true;
 }
 
+template <int MT, int MODE>
+void launch_walk_mt(const WalkPtrs& p, cudaStream_t st) {
+    const int smem = sizeof(WalkSmem<MT>) + 1024;
+    cudaFuncSetAttribute(tc_walk_kernel<MT, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    const int grid = p.B * p.H * (DV / (16 * MT));
+    GDN_LAUNCH(MODE == 0 ? "tc_walk_fwd" : "tc_walk_states", st,
+               tc_walk_kernel<MT, MODE><<<grid, WALK_THREADS, smem, st>>>(p));
+}
+
+// Two m-tiles per warp halve the CTA count; use them only while the grid still
+// covers every SM at least once.
 template <int MODE>
 void launch_walk(const WalkPtrs& p, cudaStream_t st) {
-    const int smem = sizeof(WalkSmem) + 1024;
-    cudaFuncSetAttribute(tc_walk_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    const int grid = p.B * p.H * (DV / 16);
-    GDN_LAUNCH(MODE == 0 ? "tc_walk_fwd" : "tc_walk_states", st,
-               tc_walk_kernel<MODE><<<grid, WALK_THREADS, smem, st>>>(p));
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if ((long long)p.B * p.H * (DV / 32) >= sms) launch_walk_mt<2, MODE>(p, st);
+    else launch_walk_mt<1, MODE>(p, st);
 }
 
 WalkPtrs make_walk_ptrs(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& c, const float* h0) {
