@@ -728,7 +728,7 @@ __global__ void __launch_bounds__(256) tc_bwd_local_kernel(LocPtrs p) {
 
 }  // namespace
 
-bool tc_bwd_supported(const gdn_dims& d) { return tc_supported(d); }
+bool tc_bwd_supported(const gdn_dims& d) { return tc_supported(d) && d.gate == GDN_GATE_SCALAR; }
 
 bool launch_tc_bwd(const gdn_dims& d, const void* q, const void* k, const void* v,
                    const float* g, const float* beta, const float* h0, const void* dO,

@@ -28,6 +28,9 @@
 #include <mutex>
 
 namespace gdn {
+namespace tc {
+void launch_prep_kda(const ChunkPtrs& p, size_t nchunks, cudaStream_t st);
+}
 namespace {
 using namespace tc;
 using S128 = Swz<128>;
@@ -286,7 +289,7 @@ struct alignas(1024) WalkStage {
     __nv_bfloat16 W[C * DK];                 // Swz<128>
     __nv_bfloat16 P[C * C];                  // Swz<64>
     __nv_bfloat16 Ut[MT][C * 16];            // [tile][token][16 value rows]
-    float G[C];
+    float G[DK];                             // G (scalar gate) or e^{G_last,c} (channel gate)
 };
 
 template <int MT>
@@ -304,6 +307,7 @@ struct WalkPtrs {
     const float* h0;
     const __nv_bfloat16 *W, *Ut, *P;
     const float* G;
+    const __nv_bfloat16 *Qg, *Kt;  // channel gate: prepared Q and K images
     __nv_bfloat16* o;
     float* hT;
     __nv_bfloat16 *S0out, *Uout;
@@ -312,21 +316,29 @@ struct WalkPtrs {
     float scale;
 };
 
-template <int MT>
+// KDA: the chunk's Q and K arrive pre-scaled (scale Q .* e^G, K .* e^{G_last-G})
+// as workspace images, with the per-key chunk decay e^{G_last,c}.
+template <int MT, bool KDA>
 __device__ void walk_issue(WalkStage<MT>& st, uint64_t* bar, const WalkPtrs& p, int b, int h,
                            int bh, int n, int tile0) {
     const size_t cid = (size_t)bh * p.NT + n;
-    mbar_arrive_expect(bar, (3 * C * DK + C * C + MT * C * 16) * 2 + C * 4);
+    constexpr int GW = KDA ? DK : C;
+    mbar_arrive_expect(bar, (3 * C * DK + C * C + MT * C * 16) * 2 + GW * 4);
     const int tok = b * p.T + n * C;
-    tma_load_tile(st.Q, &p.qmap, h, tok, bar);
-    tma_load_tile(st.K, &p.kmap, h, tok, bar);
+    if (KDA) {
+        bulk_g2s(st.Q, p.Qg + cid * C * DK, C * DK * 2, bar);
+        bulk_g2s(st.K, p.Kt + cid * C * DK, C * DK * 2, bar);
+    } else {
+        tma_load_tile(st.Q, &p.qmap, h, tok, bar);
+        tma_load_tile(st.K, &p.kmap, h, tok, bar);
+    }
     bulk_g2s(st.W, p.W + cid * C * DK, C * DK * 2, bar);
     bulk_g2s(st.P, p.P + cid * C * C, C * C * 2, bar);
     bulk_g2s(&st.Ut[0][0], p.Ut + (cid * 8 + tile0) * C * 16, MT * C * 16 * 2, bar);
-    bulk_g2s(st.G, p.G + cid * C, C * 4, bar);
+    bulk_g2s(st.G, p.G + cid * GW, GW * 4, bar);
 }
 
-template <int MT, int MODE>
+template <int MT, int MODE, bool KDA>
 __global__ void __launch_bounds__(WALK_THREADS) tc_walk_kernel(const __grid_constant__ WalkPtrs p) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     WalkSmem<MT>& s = *reinterpret_cast<WalkSmem<MT>*>(align1k(smem_raw));
@@ -364,7 +376,7 @@ __global__ void __launch_bounds__(WALK_THREADS) tc_walk_kernel(const __grid_cons
     __syncthreads();
     if (tid == 0)
         for (int n = 0; n < WALK_STAGES - 1 && n < p.NT; ++n)
-            walk_issue<MT>(s.st[n], &s.full[n], p, b, h, bh, n, tile0);
+            walk_issue<MT, KDA>(s.st[n], &s.full[n], p, b, h, bh, n, tile0);
 
     for (int n = 0; n < p.NT; ++n) {
         const int sn = n % WALK_STAGES;
@@ -373,7 +385,8 @@ __global__ void __launch_bounds__(WALK_THREADS) tc_walk_kernel(const __grid_cons
         __syncthreads();  // stage n landed; S0 written; stage of chunk n-1 is free
         if (tid == 0 && n + WALK_STAGES - 1 < p.NT) {
             const int nn = n + WALK_STAGES - 1;
-            walk_issue<MT>(s.st[nn % WALK_STAGES], &s.full[nn % WALK_STAGES], p, b, h, bh, nn, tile0);
+            walk_issue<MT, KDA>(s.st[nn % WALK_STAGES], &s.full[nn % WALK_STAGES], p, b, h, bh, nn,
+                                tile0);
         }
         const int L = min(C, p.T - n * C);
         const size_t cid = (size_t)bh * p.NT + n;
@@ -381,8 +394,9 @@ __global__ void __launch_bounds__(WALK_THREADS) tc_walk_kernel(const __grid_cons
             bulk_s2g(p.S0out + (cid * DV + a0) * DK, s.S0, RT * DK * 2);
             bulk_commit();
         }
-        const float Gl = st.G[C - 1];
-        const float et0 = __expf(Gl - st.G[i0]), et1 = __expf(Gl - st.G[i0 + 1]);
+        const float Gl = KDA ? 0.f : st.G[C - 1];
+        const float et0 = KDA ? 1.f : __expf(Gl - st.G[i0]);
+        const float et1 = KDA ? 1.f : __expf(Gl - st.G[i0 + 1]);
 
         // X = S0 W^T, Y = S0 Q^T for tokens 8w..8w+7 (two accumulators each)
         float X[MT][2][4] = {}, Y[MT][2][4] = {};
@@ -420,13 +434,14 @@ __global__ void __launch_bounds__(WALK_THREADS) tc_walk_kernel(const __grid_cons
         __syncthreads();
 
         // S1 = e^{G_last} S0 + (U^T .* e^{G_last - G}) K, columns 16w..16w+15
-        const float gam = __expf(Gl);
+        const float gam = KDA ? 1.f : __expf(Gl);
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
             for (int j = 0; j < 2; ++j)
 #pragma unroll
-                for (int e = 0; e < 4; ++e) S[mt][j][e] *= gam;
+                for (int e = 0; e < 4; ++e)
+                    S[mt][j][e] *= KDA ? st.G[16 * w + 8 * j + 2 * (lane & 3) + (e & 1)] : gam;
 #pragma unroll
         for (int kk = 0; kk < C / 16; ++kk) {
             uint32_t bk[4];
@@ -441,7 +456,8 @@ __global__ void __launch_bounds__(WALK_THREADS) tc_walk_kernel(const __grid_cons
         }
         if (MODE == 0) {
             // O^T (rows x tokens 8w..) = scale e^{G_i} Y + U^T P^T
-            const float eg0 = p.scale * __expf(st.G[i0]), eg1 = p.scale * __expf(st.G[i0 + 1]);
+            const float eg0 = KDA ? 1.f : p.scale * __expf(st.G[i0]);
+            const float eg1 = KDA ? 1.f : p.scale * __expf(st.G[i0 + 1]);
             float o[MT][4];
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt)
@@ -512,34 +528,39 @@ bool make_chunk_ptrs(ChunkPtrs& p, const gdn_dims& d, const TcLayout& L, const v
     p.Ut = (__nv_bfloat16*)(base + L.Ut);
     p.P = (__nv_bfloat16*)(base + L.P);
     p.G = (float*)(base + L.G);
+    if (d.gate == GDN_GATE_CHANNEL) {
+        p.Qg = (__nv_bfloat16*)(base + L.Qg);
+        p.Kt = (__nv_bfloat16*)(base + L.Kt);
+    }
     p.status = (unsigned int*)ws;
     return true;
 }
 
-template <int MT, int MODE>
+template <int MT, int MODE, bool KDA>
 void launch_walk_mt(const WalkPtrs& p, cudaStream_t st) {
     const int smem = sizeof(WalkSmem<MT>) + 1024;
-    cudaFuncSetAttribute(tc_walk_kernel<MT, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaFuncSetAttribute(tc_walk_kernel<MT, MODE, KDA>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         smem);
     const int grid = p.B * p.H * (DV / (16 * MT));
     GDN_LAUNCH(MODE == 0 ? "tc_walk_fwd" : "tc_walk_states", st,
-               tc_walk_kernel<MT, MODE><<<grid, WALK_THREADS, smem, st>>>(p));
+               (tc_walk_kernel<MT, MODE, KDA><<<grid, WALK_THREADS, smem, st>>>(p)));
 }
 
 // Two m-tiles per warp halve the CTA count; use them only while the grid still
 // covers every SM at least once.
-template <int MODE>
+template <int MODE, bool KDA>
 void launch_walk(const WalkPtrs& p, cudaStream_t st) {
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess)
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if ((long long)p.B * p.H * (DV / 32) >= sms) launch_walk_mt<2, MODE>(p, st);
-    else launch_walk_mt<1, MODE>(p, st);
+    if ((long long)p.B * p.H * (DV / 32) >= sms) launch_walk_mt<2, MODE, KDA>(p, st);
+    else launch_walk_mt<1, MODE, KDA>(p, st);
 }
 
 WalkPtrs make_walk_ptrs(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& c, const float* h0) {
     WalkPtrs w{};
     w.qmap = c.qmap; w.kmap = c.kmap;
-    w.h0 = h0; w.W = c.W; w.Ut = c.Ut; w.P = c.P; w.G = c.G;
+    w.h0 = h0; w.W = c.W; w.Ut = c.Ut; w.P = c.P; w.G = c.G; w.Qg = c.Qg; w.Kt = c.Kt;
     w.status = c.status;
     w.B = d.B; w.T = d.T; w.H = d.H; w.NT = L.NT; w.scale = d.scale;
     return w;
@@ -564,13 +585,13 @@ void launch_walk_states(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& c
     WalkPtrs w = make_walk_ptrs(d, L, cp, h0);
     w.S0out = (__nv_bfloat16*)((char*)ws + L.S0);
     w.Uout = (__nv_bfloat16*)((char*)ws + L.U);
-    launch_walk<1>(w, st);
+    if (d.gate == GDN_GATE_CHANNEL) launch_walk<1, true>(w, st);
+    else launch_walk<1, false>(w, st);
 }
 }  // namespace tc
 
 bool tc_supported(const gdn_dims& d) {
-    return d.dtype == GDN_BF16 && d.dk == DK && d.dv == DV && d.chunk == C &&
-           d.gate == GDN_GATE_SCALAR;
+    return d.dtype == GDN_BF16 && d.dk == DK && d.dv == DV && d.chunk == C;
 }
 
 size_t tc_fwd_workspace(const gdn_dims& d) { return tc_layout(d, false).end; }
@@ -582,11 +603,14 @@ bool launch_tc_fwd(const gdn_dims& d, const void* q, const void* k, const void* 
     const TcLayout L = tc_layout(d, false);
     ChunkPtrs cp;
     if (!make_chunk_ptrs(cp, d, L, q, k, v, g, beta, ws)) return false;
-    launch_prep(cp, L.nchunks, st);
+    const bool kda = d.gate == GDN_GATE_CHANNEL;
+    if (kda) launch_prep_kda(cp, L.nchunks, st);
+    else launch_prep(cp, L.nchunks, st);
     WalkPtrs w = make_walk_ptrs(d, L, cp, h0);
     w.o = (__nv_bfloat16*)o;
     w.hT = hT;
-    launch_walk<0>(w, st);
+    if (kda) launch_walk<0, true>(w, st);
+    else launch_walk<0, false>(w, st);
     return true;
 }
 
@@ -630,7 +654,7 @@ extern "C" gdn_status gdn_chunk_fwd_noalloc(const gdn_dims* d, const void* q, co
                                             gdn_stream_t stream) {
     const gdn_status s = gdn::validate_fwd_args(d, q, k, v, g, beta, h0, o, hT);
     if (s != GDN_OK) return s;
-    if (!gdn::tc_supported(*d)) return GDN_ERR_UNSUPPORTED;
+    if (!gdn::tc_supported(*d) || d->gate != GDN_GATE_SCALAR) return GDN_ERR_UNSUPPORTED;
     if (gdn::tc_fwd_workspace(*d) > gdn::kNoAllocScratchBytes) return GDN_ERR_WORKSPACE;
     void* ws = gdn::noalloc_scratch();
     if (!ws) return GDN_ERR_CUDA;

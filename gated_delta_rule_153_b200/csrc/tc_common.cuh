@@ -16,7 +16,7 @@ struct TcLayout {
     int NT;
     size_t nchunks;
     // byte offsets into the workspace
-    size_t W, Ut, P, G, Tb, S0, U, dS, dU, end;
+    size_t W, Ut, P, G, Tb, S0, U, dS, dU, Qg, Kt, end;
 };
 
 inline TcLayout tc_layout(const gdn_dims& d, bool bwd) {
@@ -28,7 +28,11 @@ inline TcLayout tc_layout(const gdn_dims& d, bool bwd) {
     L.W = take(L.nchunks * C * DK * 2);
     L.Ut = take(L.nchunks * C * DV * 2);
     L.P = take(L.nchunks * C * C * 2);
-    L.G = take(L.nchunks * C * 4);
+    L.G = take(L.nchunks * (d.gate == GDN_GATE_CHANNEL ? DK : C) * 4);
+    if (d.gate == GDN_GATE_CHANNEL) {
+        L.Qg = take(L.nchunks * C * DK * 2);
+        L.Kt = take(L.nchunks * C * DK * 2);
+    }
     if (bwd) {
         L.Tb = take(L.nchunks * C * C * 2);
         L.S0 = take(L.nchunks * DV * DK * 2);
@@ -44,7 +48,10 @@ inline TcLayout tc_layout(const gdn_dims& d, bool bwd) {
 //   W   [chunk][64][128] bf16, Swz<128> tile image
 //   Ut  [chunk][8 tiles][64][16] bf16, value columns 16*tile .. +15, row-major
 //   P   [chunk][64][64]  bf16, Swz<64> tile image (scale folded in)
-//   G   [chunk][64] fp32 within-chunk cumsum of g (padding rows repeat the last)
+//   G   [chunk][64] fp32 within-chunk cumsum of g (padding rows repeat the last);
+//       channel gate: [chunk][128] fp32 e^{G_last,c}, the per-key decay of a chunk
+//   Qg  channel gate only: [chunk] Tma128 image of scale * Q .* e^{G}
+//   Kt  channel gate only: [chunk] Tma128 image of K .* e^{G_last - G}
 //   Tb  [chunk][64][64]  bf16, Swz<64> tile image of T = (I + A)^{-1}
 //   S0  [chunk][128][128] bf16, Swz<128> image of the chunk-start state
 //   U   [chunk][64][128] bf16 row-major;  dS, dU likewise (backward)
@@ -57,6 +64,7 @@ struct ChunkPtrs {
     __nv_bfloat16 *W, *Ut, *P;
     float* G;
     __nv_bfloat16* Tb;  // optional: bf16 T = (I + A)^{-1} per chunk (backward)
+    __nv_bfloat16 *Qg, *Kt;  // channel gate only
     unsigned int* status;
 };
 

@@ -129,3 +129,15 @@ def test_deterministic(dev):
     r1, r2 = gpu_bwd(inp, dev), gpu_bwd(inp, dev)
     for n in ("dq", "dk", "dv", "dg", "dbeta"):
         assert torch.equal(r1[n], r2[n]), n
+
+
+@pytest.mark.parametrize("over", [
+    dict(B=2, H=3, T=100, h0_std=0.1, dhT_std=0.3),             # ragged tail, MMA diagonal blocks
+    dict(B=1, H=4, T=200, g_shift=10.0, h0_std=0.1),            # spans > 80: exact diagonal blocks
+    dict(B=1, H=2, T=64, g_shift=-6.0, h0_std=0.2),             # slow gate, one chunk
+])
+def test_kda_tensor_core_forward(dev, over):
+    """Channel-gate forward through the tensor-core path against the oracle."""
+    inp = make_chunk_inputs(KDA, **over)
+    check_fwd(inp, dev)
+    check_bwd(inp, dev)
