@@ -45,22 +45,25 @@ using namespace tc;
 constexpr int BW_THREADS = 256;
 constexpr int BW_STAGES = 3;
 
+// One CTA walks 16*MT value rows of dS (MT m-tiles per warp).
+template <int MT>
 struct alignas(1024) BwStage {
-    __nv_bfloat16 Q[C * DK];   // Tma128
-    __nv_bfloat16 K[C * DK];   // Tma128
-    __nv_bfloat16 W[C * DK];   // Swz<128>
-    __nv_bfloat16 P[C * C];    // Swz<64>
-    __nv_bfloat16 dO[C * 16];  // [token][16 value columns]
+    __nv_bfloat16 Q[C * DK];       // Tma128
+    __nv_bfloat16 K[C * DK];       // Tma128
+    __nv_bfloat16 W[C * DK];       // Swz<128>
+    __nv_bfloat16 P[C * C];        // Swz<64>
+    __nv_bfloat16 dO[C * 16 * MT]; // [token][16*MT value columns]
     float G[C];
 };
 
+template <int MT>
 struct BwSmem {
-    BwStage st[BW_STAGES];
-    __nv_bfloat16 dS[16 * DK];  // Swz<128>: bf16 copy of dS (rows x key columns)
-    __nv_bfloat16 dOt[16 * C];  // Swz<64>: dO^T tile
-    __nv_bfloat16 dOg[16 * C];  // Swz<64>: dO^T * scale * e^{G_i}
-    __nv_bfloat16 dU[16 * C];   // Swz<64>: dU^T
-    __nv_bfloat16 dUst[C * 16]; // [token][row] staging for the dU store
+    BwStage<MT> st[BW_STAGES];
+    __nv_bfloat16 dS[16 * MT * DK];  // Swz<128>: bf16 copy of dS (rows x key columns)
+    __nv_bfloat16 dOt[16 * MT * C];  // Swz<64>: dO^T tile
+    __nv_bfloat16 dOg[16 * MT * C];  // Swz<64>: dO^T * scale * e^{G_i}
+    __nv_bfloat16 dU[16 * MT * C];   // Swz<64>: dU^T
+    __nv_bfloat16 dUst[C * 16 * MT]; // [token][row] staging for the dU store
     uint64_t full[BW_STAGES];
 };
 
@@ -76,10 +79,11 @@ struct BwPtrs {
     float scale;
 };
 
-__device__ void bw_issue(BwStage& st, uint64_t* bar, const BwPtrs& p, int b, int h, int bh,
+template <int MT>
+__device__ void bw_issue(BwStage<MT>& st, uint64_t* bar, const BwPtrs& p, int b, int h, int bh,
                          int n, int a0) {
     const size_t cid = (size_t)bh * p.NT + n;
-    mbar_arrive_expect(bar, (3 * C * DK + C * C + C * 16) * 2 + C * 4);
+    mbar_arrive_expect(bar, (3 * C * DK + C * C + C * 16 * MT) * 2 + C * 4);
     const int tok = b * p.T + n * C;
     tma_load_tile(st.Q, &p.qmap, h, tok, bar);
     tma_load_tile(st.K, &p.kmap, h, tok, bar);
@@ -89,12 +93,14 @@ __device__ void bw_issue(BwStage& st, uint64_t* bar, const BwPtrs& p, int b, int
     bulk_g2s(st.G, p.G + cid * C, C * 4, bar);
 }
 
+template <int MT>
 __global__ void __launch_bounds__(BW_THREADS) tc_walk_bwd_kernel(const __grid_constant__ BwPtrs p) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
-    BwSmem& s = *reinterpret_cast<BwSmem*>(align1k(smem_raw));
+    BwSmem<MT>& s = *reinterpret_cast<BwSmem<MT>*>(align1k(smem_raw));
+    constexpr int RT = 16 * MT;
+    constexpr int TILES = DV / RT;
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-    constexpr int TILES = DV / 16;
-    const int bh = blockIdx.x / TILES, a0 = (blockIdx.x % TILES) * 16;
+    const int bh = blockIdx.x / TILES, a0 = (blockIdx.x % TILES) * RT;
     const int b = bh / p.H, h = bh % p.H;
     const int r_lo = lane >> 2;
     const int i0 = 8 * w + 2 * (lane & 3);  // this thread's token pair in dU^T
@@ -103,124 +109,152 @@ __global__ void __launch_bounds__(BW_THREADS) tc_walk_bwd_kernel(const __grid_co
         for (int i = 0; i < BW_STAGES; ++i) mbar_init(&s.full[i], 1);
         fence_mbar_init();
     }
-    // dS: rows r_lo, r_lo+8; columns 16w + 8j + 2(lane%4) + {0,1}
-    float dS[2][4];
+    // dS: m-tile mt, rows 16mt + r_lo (+8); columns 16w + 8j + 2(lane%4) + {0,1}
+    float dS[MT][2][4];
     {
         const float* src = p.dhT ? p.dhT + ((size_t)bh * DV + a0) * DK : nullptr;
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
-            const int c = 16 * w + 8 * j + 2 * (lane & 3);
+        for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-                dS[j][e] = src ? src[(size_t)(r_lo + 8 * (e >> 1)) * DK + c + (e & 1)] : 0.f;
-        }
+            for (int j = 0; j < 2; ++j) {
+                const int c = 16 * w + 8 * j + 2 * (lane & 3);
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    dS[mt][j][e] =
+                        src ? src[(size_t)(16 * mt + r_lo + 8 * (e >> 1)) * DK + c + (e & 1)] : 0.f;
+            }
     }
 #pragma unroll
-    for (int j = 0; j < 2; ++j) st_c<Swz<128>>(s.dS, 0, 16 * w + 8 * j, dS[j]);
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) st_c<Swz<128>>(s.dS, 16 * mt, 16 * w + 8 * j, dS[mt][j]);
     fence_async_smem();
     __syncthreads();
     if (tid == 0)
-        for (int k = 0; k < BW_STAGES - 1 && k < p.NT; ++k) {
-            const int n = p.NT - 1 - k;
-            bw_issue(s.st[k], &s.full[k], p, b, h, bh, n, a0);
-        }
+        for (int k = 0; k < BW_STAGES - 1 && k < p.NT; ++k)
+            bw_issue<MT>(s.st[k], &s.full[k], p, b, h, bh, p.NT - 1 - k, a0);
 
-    for (int k = 0; k < p.NT; ++k) {  // k-th step handles chunk n = NT-1-k
+    for (int k = 0; k < p.NT; ++k) {  // step k handles chunk n = NT-1-k
         const int n = p.NT - 1 - k;
         const int sk = k % BW_STAGES;
-        BwStage& st = s.st[sk];
+        BwStage<MT>& st = s.st[sk];
         if (!mbar_wait(&s.full[sk], (k / BW_STAGES) & 1, p.status)) return;
         __syncthreads();  // stage landed; dS written; stage of step k-1 is free
         if (tid == 0 && k + BW_STAGES - 1 < p.NT) {
             const int kk = k + BW_STAGES - 1;
-            bw_issue(s.st[kk % BW_STAGES], &s.full[kk % BW_STAGES], p, b, h, bh, p.NT - 1 - kk, a0);
+            bw_issue<MT>(s.st[kk % BW_STAGES], &s.full[kk % BW_STAGES], p, b, h, bh, p.NT - 1 - kk, a0);
         }
         const size_t cid = (size_t)bh * p.NT + n;
         const int L = min(C, p.T - n * C);
         if (tid == 0) {  // dS leaving chunk n (Swz<128> image rows a0..)
-            bulk_s2g(p.dSout + (cid * DV + a0) * DK, s.dS, 16 * DK * 2);
+            bulk_s2g(p.dSout + (cid * DV + a0) * DK, s.dS, RT * DK * 2);
             bulk_commit();
         }
         // dO^T tiles (rows past the sequence end are zeroed: they are not ours)
-        for (int e = tid; e < C * 16; e += BW_THREADS) {
-            const int i = e >> 4, a = e & 15;
-            const float x = i < L ? __bfloat162float(st.dO[i * 16 + a]) : 0.f;
+        for (int e = tid; e < C * RT; e += BW_THREADS) {
+            const int i = e / RT, a = e % RT;
+            const float x = i < L ? __bfloat162float(st.dO[i * RT + a]) : 0.f;
             s.dOt[swz<C>(a, i)] = __float2bfloat16_rn(x);
             s.dOg[swz<C>(a, i)] = __float2bfloat16_rn(x * p.scale * __expf(st.G[i]));
         }
         __syncthreads();
         const float Gl = st.G[C - 1];
+        const float et0 = __expf(Gl - st.G[i0]), et1 = __expf(Gl - st.G[i0 + 1]);
         // dU^T (rows x tokens 8w..8w+7) = dO^T P + (dS K^T) .* e^{G_last - G_r}
         {
-            float a1[4] = {}, a2[2][4] = {};
+            float a1[MT][4] = {}, a2[MT][2][4] = {};
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
                 if (16 * kk + 15 < 8 * w) continue;  // P[i][r] = 0 for i < r
-                uint32_t a[4], bp[2];
-                lda<Swz<64>>(a, s.dOt, 0, 16 * kk);
+                uint32_t bp[2];
                 ldb_kn1<Swz<64>>(bp, st.P, 16 * kk, 8 * w);
-                mma16816(a1, a, bp[0], bp[1]);
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt) {
+                    uint32_t a[4];
+                    lda<Swz<64>>(a, s.dOt, 16 * mt, 16 * kk);
+                    mma16816(a1[mt], a, bp[0], bp[1]);
+                }
             }
 #pragma unroll
             for (int kk = 0; kk < DK / 16; ++kk) {
-                uint32_t a[4], bk[2];
-                lda<Swz<128>>(a, s.dS, 0, 16 * kk);
+                uint32_t bk[2];
                 ldb_nk1<Tma128>(bk, st.K, 8 * w, 16 * kk);
-                mma16816(a2[kk & 1], a, bk[0], bk[1]);
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt) {
+                    uint32_t a[4];
+                    lda<Swz<128>>(a, s.dS, 16 * mt, 16 * kk);
+                    mma16816(a2[mt][kk & 1], a, bk[0], bk[1]);
+                }
             }
-            float u[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e)  // padding tokens (past the sequence end) stay zero
-                u[e] = (i0 + (e & 1) < L)
-                           ? a1[e] + (a2[0][e] + a2[1][e]) * __expf(Gl - st.G[i0 + (e & 1)])
-                           : 0.f;
-            st_c<Swz<64>>(s.dU, 0, 8 * w, u);
+            for (int mt = 0; mt < MT; ++mt) {
+                float u[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-                s.dUst[(i0 + (e & 1)) * 16 + r_lo + 8 * (e >> 1)] = __float2bfloat16_rn(u[e]);
+                for (int e = 0; e < 4; ++e)  // padding tokens (past the sequence end) stay zero
+                    u[e] = (i0 + (e & 1) < L)
+                               ? a1[mt][e] + (a2[mt][0][e] + a2[mt][1][e]) * ((e & 1) ? et1 : et0)
+                               : 0.f;
+                st_c<Swz<64>>(s.dU, 16 * mt, 8 * w, u);
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    s.dUst[(i0 + (e & 1)) * RT + 16 * mt + r_lo + 8 * (e >> 1)] = __float2bfloat16_rn(u[e]);
+            }
         }
         if (tid == 0) bulk_wait_read<0>();  // dS image read before it is rewritten
         __syncthreads();
         // dS0 = e^{G_last} dS + dOg^T Q - dU^T W   (columns 16w..16w+15)
         {
             const float gam = __expf(Gl);
-            float y[2][4] = {}, z[2][4] = {};
+            float y[MT][2][4] = {}, z[MT][2][4] = {};
 #pragma unroll
             for (int kk = 0; kk < C / 16; ++kk) {
-                uint32_t ag[4], au[4], bq[4], bw[4];
-                lda<Swz<64>>(ag, s.dOg, 0, 16 * kk);
-                lda<Swz<64>>(au, s.dU, 0, 16 * kk);
+                uint32_t bq[4], bw[4];
                 ldb_kn<Tma128>(bq, st.Q, 16 * kk, 16 * w);
                 ldb_kn<Swz<128>>(bw, st.W, 16 * kk, 16 * w);
-                mma16816(y[0], ag, bq[0], bq[1]);
-                mma16816(y[1], ag, bq[2], bq[3]);
-                mma16816(z[0], au, bw[0], bw[1]);
-                mma16816(z[1], au, bw[2], bw[3]);
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt) {
+                    uint32_t ag[4], au[4];
+                    lda<Swz<64>>(ag, s.dOg, 16 * mt, 16 * kk);
+                    lda<Swz<64>>(au, s.dU, 16 * mt, 16 * kk);
+                    mma16816(y[mt][0], ag, bq[0], bq[1]);
+                    mma16816(y[mt][1], ag, bq[2], bq[3]);
+                    mma16816(z[mt][0], au, bw[0], bw[1]);
+                    mma16816(z[mt][1], au, bw[2], bw[3]);
+                }
             }
 #pragma unroll
-            for (int j = 0; j < 2; ++j)
+            for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-                for (int e = 0; e < 4; ++e) dS[j][e] = gam * dS[j][e] + y[j][e] - z[j][e];
+                for (int j = 0; j < 2; ++j)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        dS[mt][j][e] = gam * dS[mt][j][e] + y[mt][j][e] - z[mt][j][e];
         }
         __syncthreads();  // everyone done with dS, dOt, dOg, dU; dU staged
 #pragma unroll
-        for (int j = 0; j < 2; ++j) st_c<Swz<128>>(s.dS, 0, 16 * w + 8 * j, dS[j]);
+        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+            for (int j = 0; j < 2; ++j) st_c<Swz<128>>(s.dS, 16 * mt, 16 * w + 8 * j, dS[mt][j]);
         fence_async_smem();
-        if (tid < 2 * C) {  // dU rows (tokens x value rows a0..a0+15), 16-byte pieces
-            const int i = tid >> 1, hf = tid & 1;
-            *reinterpret_cast<uint4*>(p.dUout + (cid * C + i) * DV + a0 + 8 * hf) =
-                *reinterpret_cast<const uint4*>(&s.dUst[i * 16 + 8 * hf]);
+        constexpr int PIECES = RT / 8;
+        for (int e = tid; e < PIECES * C; e += BW_THREADS) {  // dU rows, 16-byte pieces
+            const int i = e / PIECES, pc = e % PIECES;
+            *reinterpret_cast<uint4*>(p.dUout + (cid * C + i) * DV + a0 + 8 * pc) =
+                *reinterpret_cast<const uint4*>(&s.dUst[i * RT + 8 * pc]);
         }
     }
     if (tid == 0) bulk_wait<0>();
     if (p.dh0) {
         float* dst = p.dh0 + ((size_t)bh * DV + a0) * DK;
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
-            const int c = 16 * w + 8 * j + 2 * (lane & 3);
+        for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) dst[(size_t)(r_lo + 8 * (e >> 1)) * DK + c + (e & 1)] = dS[j][e];
-        }
+            for (int j = 0; j < 2; ++j) {
+                const int c = 16 * w + 8 * j + 2 * (lane & 3);
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    dst[(size_t)(16 * mt + r_lo + 8 * (e >> 1)) * DK + c + (e & 1)] = dS[mt][j][e];
+            }
     }
 }
 
@@ -743,18 +777,27 @@ bool launch_tc_bwd(const gdn_dims& d, const void* q, const void* k, const void* 
     launch_walk_states(d, L, cp, h0, ws, st);
 
     BwPtrs bp{};
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const bool two = (long long)d.B * d.H * (DV / 32) >= sms;  // two m-tiles per warp
     bp.qmap = cp.qmap; bp.kmap = cp.kmap;
-    if (!encode_token_map(&bp.dOmap, dO, d.B, d.T, d.H, 16)) return false;
+    if (!encode_token_map(&bp.dOmap, dO, d.B, d.T, d.H, two ? 32 : 16)) return false;
     bp.dhT = dhT; bp.W = cp.W; bp.P = cp.P; bp.G = cp.G;
     bp.dSout = (__nv_bfloat16*)(base + L.dS);
     bp.dUout = (__nv_bfloat16*)(base + L.dU);
     bp.dh0 = dh0; bp.status = cp.status;
     bp.B = d.B; bp.T = d.T; bp.H = d.H; bp.NT = L.NT; bp.scale = d.scale;
-    {
-        const int smem = sizeof(BwSmem) + 1024;
-        cudaFuncSetAttribute(tc_walk_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (two) {
+        const int smem = sizeof(BwSmem<2>) + 1024;
+        cudaFuncSetAttribute(tc_walk_bwd_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         GDN_LAUNCH("tc_walk_bwd", st,
-                   tc_walk_bwd_kernel<<<d.B * d.H * (DV / 16), BW_THREADS, smem, st>>>(bp));
+                   tc_walk_bwd_kernel<2><<<d.B * d.H * (DV / 32), BW_THREADS, smem, st>>>(bp));
+    } else {
+        const int smem = sizeof(BwSmem<1>) + 1024;
+        cudaFuncSetAttribute(tc_walk_bwd_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        GDN_LAUNCH("tc_walk_bwd", st,
+                   tc_walk_bwd_kernel<1><<<d.B * d.H * (DV / 16), BW_THREADS, smem, st>>>(bp));
     }
     LocPtrs lp{};
     lp.q = cp.q; lp.k = cp.k; lp.v = cp.v; lp.dO = (const __nv_bfloat16*)dO; lp.g = g;
