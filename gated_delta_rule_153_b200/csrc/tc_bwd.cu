@@ -138,8 +138,7 @@ __global__ void __launch_bounds__(BW_THREADS) tc_walk_bwd_kernel(const __grid_co
         const int n = p.NT - 1 - k;
         const int sk = k % BW_STAGES;
         BwStage<MT>& st = s.st[sk];
-        if (!mbar_wait(&s.full[sk], (k / BW_STAGES) & 1, p.status)) return;
-        __syncthreads();  // stage landed; dS written; stage of step k-1 is free
+        if (__syncthreads_or(!mbar_wait(&s.full[sk], (k / BW_STAGES) & 1, p.status))) return;  // all threads agree; stage landed; dS written; stage of step k-1 is free
         if (tid == 0 && k + BW_STAGES - 1 < p.NT) {
             const int kk = k + BW_STAGES - 1;
             bw_issue<MT>(s.st[kk % BW_STAGES], &s.full[kk % BW_STAGES], p, b, h, bh, p.NT - 1 - kk, a0);
@@ -239,7 +238,7 @@ __global__ void __launch_bounds__(BW_THREADS) tc_walk_bwd_kernel(const __grid_co
         constexpr int PIECES = RT / 8;
         for (int e = tid; e < PIECES * C; e += BW_THREADS) {  // dU rows, 16-byte pieces
             const int i = e / PIECES, pc = e % PIECES;
-            *reinterpret_cast<uint4*>(p.dUout + (cid * C + i) * DV + a0 + 8 * pc) =
+            *reinterpret_cast<uint4*>(p.dUout + cid * C * DV + swz<DV>(i, a0 + 8 * pc)) =
                 *reinterpret_cast<const uint4*>(&s.dUst[i * RT + 8 * pc]);
         }
     }
@@ -259,11 +258,14 @@ __global__ void __launch_bounds__(BW_THREADS) tc_walk_bwd_kernel(const __grid_co
 }
 
 // ---------------------------------------------------------------------------
-// local gradients: one CTA (8 warps) per chunk.  Warp w owns rows
-// 16*(w/2) .. +15 and column half (w%2) of every 64x128 result, and the
-// token-column half (w%2) of every 64x64 result.
+// local gradients: one CTA (16 warps) per chunk.  Warp w owns rows
+// 16*(w/4) .. +15 and column quarter (w%4) of every 64x128 and every 64x64
+// result.
 // ---------------------------------------------------------------------------
+constexpr int LOC_WARPS = 16, LOC_THREADS = 32 * LOC_WARPS;
+
 struct LocSmem {
+    // Q, K, V, dO: Tma128 tiles (TMA); U, dU: Swz<128> images (bulk)
     __nv_bfloat16 Q[C * DK], K[C * DK], V[C * DV], dO[C * DV], U[C * DV], dU[C * DV];
     __nv_bfloat16 S0[DV * DK];  // rows a (value), cols c (key)
     __nv_bfloat16 dS[DV * DK];
@@ -274,18 +276,21 @@ struct LocSmem {
     __nv_bfloat16 X[C * C];     // dT T^T
     __nv_bfloat16 dMM[C * C];   // dA .* beta_i .* D
     float G[C], beta[C];
-    float red_b[8][C];   // partial dbeta (by row)
-    float red_g[8][C];   // partial dG (by token)
-    float red_s[8][2];   // partial scalars for G_last
+    float red_b[16][C];  // partial dbeta (by row), per warp
+    float red_g[16][C];  // partial dG (by token), per warp
+    float red_s[16][2];  // partial scalars for G_last, per warp
+    uint64_t bar[2];     // [0]: inputs of the value-dimension contractions, [1]: the rest
 };
 
 struct LocPtrs {
+    CUtensorMap qmap, kmap, vmap, dOmap;
     const __nv_bfloat16 *q, *k, *v, *dO;
     const float *g, *beta;
     const __nv_bfloat16 *S0, *U, *dS, *dU, *Tb;
     const float* G;
     __nv_bfloat16 *dq, *dk, *dv;
     float *dg, *dbeta;
+    unsigned int* status;
     int B, T, H, NT;
     float scale;
 };
@@ -305,11 +310,11 @@ __device__ __forceinline__ float col_sum(float v) {
     return v;
 }
 
-__global__ void __launch_bounds__(256) tc_bwd_local_kernel(LocPtrs p) {
-    extern __shared__ __align__(128) unsigned char smem_raw[];
-    LocSmem& s = *reinterpret_cast<LocSmem*>(smem_raw);
+__global__ void __launch_bounds__(LOC_THREADS) tc_bwd_local_kernel(const __grid_constant__ LocPtrs p) {
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    LocSmem& s = *reinterpret_cast<LocSmem*>(align1k(smem_raw));
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-    const int rb = w >> 1, ch = w & 1;
+    const int rb = w >> 2, cq = w & 3;
     const int m0 = 16 * rb;
     const int cid = blockIdx.x;
     const int bh = cid / p.NT, n = cid % p.NT, b = bh / p.H, h = bh % p.H;
@@ -319,26 +324,40 @@ __global__ void __launch_bounds__(256) tc_bwd_local_kernel(LocPtrs p) {
     const size_t rs = (size_t)p.H;
     const int rl = m0 + (lane >> 2), rh = rl + 8;  // this thread's two rows
 
-    load_tile_async<DK>(s.Q, p.q + row0 * DK, rs * DK, C, L, tid, 256);
-    load_tile_async<DK>(s.K, p.k + row0 * DK, rs * DK, C, L, tid, 256);
-    load_tile_async<DV>(s.V, p.v + row0 * DV, rs * DV, C, L, tid, 256);
-    load_tile_async<DV>(s.dO, p.dO + row0 * DV, rs * DV, C, L, tid, 256);
-    load_tile_async<DV>(s.U, p.U + (size_t)cid * C * DV, DV, C, C, tid, 256);
-    load_tile_async<DV>(s.dU, p.dU + (size_t)cid * C * DV, DV, C, C, tid, 256);
-    load_image_async(s.S0, p.S0 + (size_t)cid * DV * DK, DV * DK * 2, tid, 256);
-    load_image_async(s.dS, p.dS + (size_t)cid * DV * DK, DV * DK * 2, tid, 256);
-    load_image_async(s.Tb, p.Tb + (size_t)cid * C * C, C * C * 2, tid, 256);
-    cp_async_commit();
-    for (int e = tid; e < C; e += 256) {
-        s.G[e] = p.G[(size_t)cid * C + e];
-        s.beta[e] = e < L ? p.beta[row0 + e * rs] : 0.f;
+    if (tid == 0) {
+        mbar_init(&s.bar[0], 1);
+        mbar_init(&s.bar[1], 1);
+        fence_mbar_init();
+        const int tok = b * p.T + t0;
+        // phase 1 (contractions over the value dimension) needs dO, Q, K, U, dU,
+        // S0, dS, G; V and T are first used after it
+        mbar_arrive_expect(&s.bar[0], (5 * C * DK + 2 * DV * DK) * 2 + C * 4);
+        tma_load_tile(s.dO, &p.dOmap, h, tok, &s.bar[0]);
+        tma_load_tile(s.Q, &p.qmap, h, tok, &s.bar[0]);
+        tma_load_tile(s.K, &p.kmap, h, tok, &s.bar[0]);
+        bulk_g2s(s.U, p.U + (size_t)cid * C * DV, C * DV * 2, &s.bar[0]);
+        bulk_g2s(s.dU, p.dU + (size_t)cid * C * DV, C * DV * 2, &s.bar[0]);
+        bulk_g2s(s.S0, p.S0 + (size_t)cid * DV * DK, DV * DK * 2, &s.bar[0]);
+        bulk_g2s(s.dS, p.dS + (size_t)cid * DV * DK, DV * DK * 2, &s.bar[0]);
+        bulk_g2s(s.G, p.G + (size_t)cid * C, C * 4, &s.bar[0]);
+        mbar_arrive_expect(&s.bar[1], (C * DK + C * C) * 2);
+        tma_load_tile(s.V, &p.vmap, h, tok, &s.bar[1]);
+        bulk_g2s(s.Tb, p.Tb + (size_t)cid * C * C, C * C * 2, &s.bar[1]);
     }
-    for (int e = tid; e < 8 * C; e += 256) {
+    for (int e = tid; e < C; e += LOC_THREADS) s.beta[e] = e < L ? p.beta[row0 + e * rs] : 0.f;
+    for (int e = tid; e < LOC_WARPS * C; e += LOC_THREADS) {
         (&s.red_b[0][0])[e] = 0.f;
         (&s.red_g[0][0])[e] = 0.f;
     }
-    if (tid < 16) (&s.red_s[0][0])[tid] = 0.f;
-    cp_async_wait<0>();
+    if (tid < 2 * LOC_WARPS) (&s.red_s[0][0])[tid] = 0.f;
+    __syncthreads();
+    if (__syncthreads_or(!mbar_wait(&s.bar[0], 0, p.status))) return;
+    if (L < C) {  // dO rows past the sequence end belong to the next sequence: zero them
+        for (int e = tid; e < (C - L) * DV; e += LOC_THREADS) {
+            const int r = L + e / DV, c = e % DV;
+            s.dO[Tma128::off(r, c)] = __float2bfloat16_rn(0.f);
+        }
+    }
     __syncthreads();
 
     const float Gl = s.G[C - 1];
@@ -349,35 +368,35 @@ __global__ void __launch_bounds__(256) tc_bwd_local_kernel(LocPtrs p) {
     float row_g_lo = 0.f, row_g_hi = 0.f;  // partial dG for rows rl, rh
     float last_acc = 0.f;                  // partial dG_last (sum over rows of hkt)
 
-    // dQ' and dK accumulators: rows rl/rh, columns 64*ch + 8j + 2(lane%4) + {0,1}
-    float dQ[8][4], dK[8][4];
+    // dQ' and dK accumulators: rows rl/rh, columns 32*cq + 8j + 2(lane%4) + {0,1}
+    float dQ[4][4], dK[4][4];
 
     // ---- phase 1: contractions over the value dimension --------------------
     {
-        float acc[8][4];
+        float acc[4][4];
         // dQg = dO S0  ->  dQ' = e^G dQg ;  dG += scale e^G sum_c dQg Q
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
+        for (int j = 0; j < 4; ++j)
 #pragma unroll
             for (int e = 0; e < 4; ++e) acc[j][e] = 0.f;
 #pragma unroll
         for (int kk = 0; kk < DV / 16; ++kk) {
             uint32_t a[4];
-            lda<DV>(a, s.dO, m0, 16 * kk);
+            lda<Tma128>(a, s.dO, m0, 16 * kk);
 #pragma unroll
-            for (int np = 0; np < 4; ++np) {
+            for (int np = 0; np < 2; ++np) {
                 uint32_t bf[4];
-                ldb_kn<DK>(bf, s.S0, 16 * kk, 64 * ch + 16 * np);
+                ldb_kn<DK>(bf, s.S0, 16 * kk, 32 * cq + 16 * np);
                 mma16816(acc[2 * np], a, bf[0], bf[1]);
                 mma16816(acc[2 * np + 1], a, bf[2], bf[3]);
             }
         }
         float hq_lo = 0.f, hq_hi = 0.f;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int c = 64 * ch + 8 * j + 2 * (lane & 3);
-            const float2 ql = unpack_bf16(*reinterpret_cast<const uint32_t*>(s.Q + swz<DK>(rl, c)));
-            const float2 qh = unpack_bf16(*reinterpret_cast<const uint32_t*>(s.Q + swz<DK>(rh, c)));
+        for (int j = 0; j < 4; ++j) {
+            const int c = 32 * cq + 8 * j + 2 * (lane & 3);
+            const float2 ql = unpack_bf16(*reinterpret_cast<const uint32_t*>(s.Q + Tma128::off(rl, c)));
+            const float2 qh = unpack_bf16(*reinterpret_cast<const uint32_t*>(s.Q + Tma128::off(rh, c)));
             hq_lo += acc[j][0] * ql.x + acc[j][1] * ql.y;
             hq_hi += acc[j][2] * qh.x + acc[j][3] * qh.y;
             dQ[j][0] = egl * acc[j][0]; dQ[j][1] = egl * acc[j][1];
@@ -388,7 +407,7 @@ __global__ void __launch_bounds__(256) tc_bwd_local_kernel(LocPtrs p) {
 
         // dKt = U dS  ->  dK = e^{Gl-G} dKt ;  hkt = e^{Gl-G} sum_c dKt K
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
+        for (int j = 0; j < 4; ++j)
 #pragma unroll
             for (int e = 0; e < 4; ++e) acc[j][e] = 0.f;
 #pragma unroll
@@ -396,19 +415,19 @@ __global__ void __launch_bounds__(256) tc_bwd_local_kernel(LocPtrs p) {
             uint32_t a[4];
             lda<DV>(a, s.U, m0, 16 * kk);
 #pragma unroll
-            for (int np = 0; np < 4; ++np) {
+            for (int np = 0; np < 2; ++np) {
                 uint32_t bf[4];
-                ldb_kn<DK>(bf, s.dS, 16 * kk, 64 * ch + 16 * np);
+                ldb_kn<DK>(bf, s.dS, 16 * kk, 32 * cq + 16 * np);
                 mma16816(acc[2 * np], a, bf[0], bf[1]);
                 mma16816(acc[2 * np + 1], a, bf[2], bf[3]);
             }
         }
         float hk_lo = 0.f, hk_hi = 0.f;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int c = 64 * ch + 8 * j + 2 * (lane & 3);
-            const float2 kl = unpack_bf16(*reinterpret_cast<const uint32_t*>(s.K + swz<DK>(rl, c)));
-            const float2 kh = unpack_bf16(*reinterpret_cast<const uint32_t*>(s.K + swz<DK>(rh, c)));
+        for (int j = 0; j < 4; ++j) {
+            const int c = 32 * cq + 8 * j + 2 * (lane & 3);
+            const float2 kl = unpack_bf16(*reinterpret_cast<const uint32_t*>(s.K + Tma128::off(rl, c)));
+            const float2 kh = unpack_bf16(*reinterpret_cast<const uint32_t*>(s.K + Tma128::off(rh, c)));
             hk_lo += acc[j][0] * kl.x + acc[j][1] * kl.y;
             hk_hi += acc[j][2] * kh.x + acc[j][3] * kh.y;
             dK[j][0] = etl * acc[j][0]; dK[j][1] = etl * acc[j][1];
@@ -420,7 +439,7 @@ __global__ void __launch_bounds__(256) tc_bwd_local_kernel(LocPtrs p) {
 
         // dW = -dU S0  -> bf16 tile
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
+        for (int j = 0; j < 4; ++j)
 #pragma unroll
             for (int e = 0; e < 4; ++e) acc[j][e] = 0.f;
 #pragma unroll
@@ -428,31 +447,31 @@ __global__ void __launch_bounds__(256) tc_bwd_local_kernel(LocPtrs p) {
             uint32_t a[4];
             lda<DV>(a, s.dU, m0, 16 * kk);
 #pragma unroll
-            for (int np = 0; np < 4; ++np) {
+            for (int np = 0; np < 2; ++np) {
                 uint32_t bf[4];
-                ldb_kn<DK>(bf, s.S0, 16 * kk, 64 * ch + 16 * np);
+                ldb_kn<DK>(bf, s.S0, 16 * kk, 32 * cq + 16 * np);
                 mma16816(acc[2 * np], a, bf[0], bf[1]);
                 mma16816(acc[2 * np + 1], a, bf[2], bf[3]);
             }
         }
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+        for (int j = 0; j < 4; ++j) {
             float x[4] = {-acc[j][0], -acc[j][1], -acc[j][2], -acc[j][3]};
-            st_c<DK>(s.dW, m0, 64 * ch + 8 * j, x);
+            st_c<DK>(s.dW, m0, 32 * cq + 8 * j, x);
         }
 
-        // dP = lower(dO U^T), QK = Q K^T on tokens 32*ch .. +31
-        float dp[4][4] = {}, qk[4][4] = {};
+        // dP = lower(dO U^T), QK = Q K^T on tokens 16*cq .. +15
+        float dp[2][4] = {}, qk[2][4] = {};
 #pragma unroll
         for (int kk = 0; kk < DV / 16; ++kk) {
             uint32_t ad[4], aq[4];
-            lda<DV>(ad, s.dO, m0, 16 * kk);
-            lda<DK>(aq, s.Q, m0, 16 * kk);
+            lda<Tma128>(ad, s.dO, m0, 16 * kk);
+            lda<Tma128>(aq, s.Q, m0, 16 * kk);
 #pragma unroll
-            for (int np = 0; np < 2; ++np) {
+            for (int np = 0; np < 1; ++np) {
                 uint32_t bu[4], bk[4];
-                ldb_nk<DV>(bu, s.U, 32 * ch + 16 * np, 16 * kk);
-                ldb_nk<DK>(bk, s.K, 32 * ch + 16 * np, 16 * kk);
+                ldb_nk<DV>(bu, s.U, 16 * cq + 16 * np, 16 * kk);
+                ldb_nk<Tma128>(bk, s.K, 16 * cq + 16 * np, 16 * kk);
                 mma16816(dp[2 * np], ad, bu[0], bu[1]);
                 mma16816(dp[2 * np + 1], ad, bu[2], bu[3]);
                 mma16816(qk[2 * np], aq, bk[0], bk[1]);
@@ -460,10 +479,10 @@ __global__ void __launch_bounds__(256) tc_bwd_local_kernel(LocPtrs p) {
             }
         }
         // hP = dP .* (scale Q K^T .* D) ;  dPG = dP .* D
-        float colp[4][2];
+        float colp[2][2];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int c0 = 32 * ch + 8 * j + 2 * (lane & 3);
+        for (int j = 0; j < 2; ++j) {
+            const int c0 = 16 * cq + 8 * j + 2 * (lane & 3);
             float g[4];
             colp[j][0] = colp[j][1] = 0.f;
 #pragma unroll
@@ -475,18 +494,18 @@ __global__ void __launch_bounds__(256) tc_bwd_local_kernel(LocPtrs p) {
                 if (e < 2) row_g_lo += hp; else row_g_hi += hp;
                 colp[j][e & 1] -= hp;
             }
-            st_c<C>(s.dPG, m0, 32 * ch + 8 * j, g);
+            st_c<C>(s.dPG, m0, 16 * cq + 8 * j, g);
         }
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
+        for (int j = 0; j < 2; ++j)
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
                 const float v = col_sum(colp[j][e]);
-                if (lane < 4) s.red_g[w][32 * ch + 8 * j + 2 * lane + e] += v;
+                if (lane < 4) s.red_g[w][16 * cq + 8 * j + 2 * lane + e] += v;
             }
         // e^{G_last} <dS, S0> (each warp a slice of the 128x128 elements)
         float ss = 0.f;
-        for (int e = lane + 32 * w; e < DV * DK / 8; e += 256) {
+        for (int e = lane + 32 * w; e < DV * DK / 8; e += LOC_THREADS) {
             const int r = e / (DK / 8), c8 = e % (DK / 8);
             const uint4 x = *reinterpret_cast<const uint4*>(s.dS + swz<DK>(r, 8 * c8));
             const uint4 y = *reinterpret_cast<const uint4*>(s.S0 + swz<DK>(r, 8 * c8));
@@ -506,32 +525,32 @@ __global__ void __launch_bounds__(256) tc_bwd_local_kernel(LocPtrs p) {
     }
 
     // ---- phase 2: K K^T (-> M), dT ---------------------------------------
-    float M[4][4];
+    float M[2][4];
     {
-        float kkt[4][4] = {}, tw[4][4] = {}, tu[4][4] = {};
+        float kkt[2][4] = {}, tw[2][4] = {}, tu[2][4] = {};
 #pragma unroll
         for (int kk = 0; kk < DK / 16; ++kk) {
             uint32_t ak[4];
-            lda<DK>(ak, s.K, m0, 16 * kk);
+            lda<Tma128>(ak, s.K, m0, 16 * kk);
 #pragma unroll
-            for (int np = 0; np < 2; ++np) {
+            for (int np = 0; np < 1; ++np) {
                 uint32_t bk[4];
-                ldb_nk<DK>(bk, s.K, 32 * ch + 16 * np, 16 * kk);
+                ldb_nk<Tma128>(bk, s.K, 16 * cq + 16 * np, 16 * kk);
                 mma16816(kkt[2 * np], ak, bk[0], bk[1]);
                 mma16816(kkt[2 * np + 1], ak, bk[2], bk[3]);
             }
         }
-        __syncthreads();  // dW tile complete
+        if (__syncthreads_or(!mbar_wait(&s.bar[1], 0, p.status))) return;  // all threads agree; dW tile complete; V and T landed
 #pragma unroll
         for (int kk = 0; kk < DK / 16; ++kk) {
             uint32_t aw[4], au[4];
             lda<DK>(aw, s.dW, m0, 16 * kk);
             lda<DV>(au, s.dU, m0, 16 * kk);
 #pragma unroll
-            for (int np = 0; np < 2; ++np) {
+            for (int np = 0; np < 1; ++np) {
                 uint32_t bk[4], bv[4];
-                ldb_nk<DK>(bk, s.K, 32 * ch + 16 * np, 16 * kk);
-                ldb_nk<DV>(bv, s.V, 32 * ch + 16 * np, 16 * kk);
+                ldb_nk<Tma128>(bk, s.K, 16 * cq + 16 * np, 16 * kk);
+                ldb_nk<Tma128>(bv, s.V, 16 * cq + 16 * np, 16 * kk);
                 mma16816(tw[2 * np], aw, bk[0], bk[1]);
                 mma16816(tw[2 * np + 1], aw, bk[2], bk[3]);
                 mma16816(tu[2 * np], au, bv[0], bv[1]);
@@ -539,8 +558,8 @@ __global__ void __launch_bounds__(256) tc_bwd_local_kernel(LocPtrs p) {
             }
         }
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int c0 = 32 * ch + 8 * j + 2 * (lane & 3);
+        for (int j = 0; j < 2; ++j) {
+            const int c0 = 16 * cq + 8 * j + 2 * (lane & 3);
             float dt[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -549,40 +568,40 @@ __global__ void __launch_bounds__(256) tc_bwd_local_kernel(LocPtrs p) {
                 dt[e] = tw[j][e] * bj * __expf(s.G[c]) + tu[j][e] * bj;
                 M[j][e] = (c < r) ? kkt[j][e] * __expf(s.G[r] - s.G[c]) : 0.f;
             }
-            st_c<C>(s.dT, m0, 32 * ch + 8 * j, dt);
+            st_c<C>(s.dT, m0, 16 * cq + 8 * j, dt);
         }
     }
     __syncthreads();
 
     // ---- phase 3: X = dT T^T ; dKg = T^T dW ; dVb = T^T dU ------------------
     {
-        float x[4][4] = {};
+        float x[2][4] = {};
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
             uint32_t a[4];
             lda<C>(a, s.dT, m0, 16 * kk);
 #pragma unroll
-            for (int np = 0; np < 2; ++np) {
+            for (int np = 0; np < 1; ++np) {
                 uint32_t bt[4];
-                ldb_nk<C>(bt, s.Tb, 32 * ch + 16 * np, 16 * kk);
+                ldb_nk<C>(bt, s.Tb, 16 * cq + 16 * np, 16 * kk);
                 mma16816(x[2 * np], a, bt[0], bt[1]);
                 mma16816(x[2 * np + 1], a, bt[2], bt[3]);
             }
         }
 #pragma unroll
-        for (int j = 0; j < 4; ++j) st_c<C>(s.X, m0, 32 * ch + 8 * j, x[j]);
+        for (int j = 0; j < 2; ++j) st_c<C>(s.X, m0, 16 * cq + 8 * j, x[j]);
 
-        float akg[8][4] = {}, avb[8][4] = {};
+        float akg[4][4] = {}, avb[4][4] = {};
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
             if (kk < rb) continue;  // T[j][i] = 0 for j < i
             uint32_t a[4];
             lda_t<C>(a, s.Tb, m0, 16 * kk);
 #pragma unroll
-            for (int np = 0; np < 4; ++np) {
+            for (int np = 0; np < 2; ++np) {
                 uint32_t bw[4], bu[4];
-                ldb_kn<DK>(bw, s.dW, 16 * kk, 64 * ch + 16 * np);
-                ldb_kn<DV>(bu, s.dU, 16 * kk, 64 * ch + 16 * np);
+                ldb_kn<DK>(bw, s.dW, 16 * kk, 32 * cq + 16 * np);
+                ldb_kn<DV>(bu, s.dU, 16 * kk, 32 * cq + 16 * np);
                 mma16816(akg[2 * np], a, bw[0], bw[1]);
                 mma16816(akg[2 * np + 1], a, bw[2], bw[3]);
                 mma16816(avb[2 * np], a, bu[0], bu[1]);
@@ -593,12 +612,12 @@ __global__ void __launch_bounds__(256) tc_bwd_local_kernel(LocPtrs p) {
         const bool okl = rl < L, okh = rh < L;
         __nv_bfloat16* dvp = p.dv + row0 * DV;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int c = 64 * ch + 8 * j + 2 * (lane & 3);
-            const float2 kl = unpack_bf16(*reinterpret_cast<const uint32_t*>(s.K + swz<DK>(rl, c)));
-            const float2 kh = unpack_bf16(*reinterpret_cast<const uint32_t*>(s.K + swz<DK>(rh, c)));
-            const float2 vl = unpack_bf16(*reinterpret_cast<const uint32_t*>(s.V + swz<DV>(rl, c)));
-            const float2 vh = unpack_bf16(*reinterpret_cast<const uint32_t*>(s.V + swz<DV>(rh, c)));
+        for (int j = 0; j < 4; ++j) {
+            const int c = 32 * cq + 8 * j + 2 * (lane & 3);
+            const float2 kl = unpack_bf16(*reinterpret_cast<const uint32_t*>(s.K + Tma128::off(rl, c)));
+            const float2 kh = unpack_bf16(*reinterpret_cast<const uint32_t*>(s.K + Tma128::off(rh, c)));
+            const float2 vl = unpack_bf16(*reinterpret_cast<const uint32_t*>(s.V + Tma128::off(rl, c)));
+            const float2 vh = unpack_bf16(*reinterpret_cast<const uint32_t*>(s.V + Tma128::off(rh, c)));
             hk_lo += akg[j][0] * kl.x + akg[j][1] * kl.y;
             hk_hi += akg[j][2] * kh.x + akg[j][3] * kh.y;
             hv_lo += avb[j][0] * vl.x + avb[j][1] * vl.y;
@@ -621,24 +640,24 @@ __global__ void __launch_bounds__(256) tc_bwd_local_kernel(LocPtrs p) {
 
     // ---- phase 4: dA = -T^T X (strictly lower) ------------------------------
     {
-        float da[4][4] = {};
+        float da[2][4] = {};
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
             if (kk < rb) continue;
             uint32_t a[4];
             lda_t<C>(a, s.Tb, m0, 16 * kk);
 #pragma unroll
-            for (int np = 0; np < 2; ++np) {
+            for (int np = 0; np < 1; ++np) {
                 uint32_t bx[4];
-                ldb_kn<C>(bx, s.X, 16 * kk, 32 * ch + 16 * np);
+                ldb_kn<C>(bx, s.X, 16 * kk, 16 * cq + 16 * np);
                 mma16816(da[2 * np], a, bx[0], bx[1]);
                 mma16816(da[2 * np + 1], a, bx[2], bx[3]);
             }
         }
-        float colp[4][2];
+        float colp[2][2];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int c0 = 32 * ch + 8 * j + 2 * (lane & 3);
+        for (int j = 0; j < 2; ++j) {
+            const int c0 = 16 * cq + 8 * j + 2 * (lane & 3);
             float mm[4];
             colp[j][0] = colp[j][1] = 0.f;
 #pragma unroll
@@ -653,21 +672,21 @@ __global__ void __launch_bounds__(256) tc_bwd_local_kernel(LocPtrs p) {
                 colp[j][e & 1] -= hA;
                 mm[e] = (c < r) ? dA * br * __expf(s.G[r] - s.G[c]) : 0.f;
             }
-            st_c<C>(s.dMM, m0, 32 * ch + 8 * j, mm);
+            st_c<C>(s.dMM, m0, 16 * cq + 8 * j, mm);
         }
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
+        for (int j = 0; j < 2; ++j)
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
                 const float v = col_sum(colp[j][e]);
-                if (lane < 4) s.red_g[w][32 * ch + 8 * j + 2 * lane + e] += v;
+                if (lane < 4) s.red_g[w][16 * cq + 8 * j + 2 * lane + e] += v;
             }
     }
     __syncthreads();
 
     // ---- phase 5: dK += dMM K + dMM^T K + scale dPG^T Q ; dQ' += dPG K -------
     {
-        float tq[8][4] = {};
+        float tq[4][4] = {};
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
             uint32_t am[4], amt[4], ap[4], apt[4];
@@ -675,9 +694,9 @@ __global__ void __launch_bounds__(256) tc_bwd_local_kernel(LocPtrs p) {
             if (lo) { lda<C>(am, s.dMM, m0, 16 * kk); lda<C>(ap, s.dPG, m0, 16 * kk); }
             if (hi) { lda_t<C>(amt, s.dMM, m0, 16 * kk); lda_t<C>(apt, s.dPG, m0, 16 * kk); }
 #pragma unroll
-            for (int np = 0; np < 4; ++np) {
+            for (int np = 0; np < 2; ++np) {
                 uint32_t bk[4], bq[4];
-                ldb_kn<DK>(bk, s.K, 16 * kk, 64 * ch + 16 * np);
+                ldb_kn<Tma128>(bk, s.K, 16 * kk, 32 * cq + 16 * np);
                 if (lo) {
                     mma16816(dK[2 * np], am, bk[0], bk[1]);
                     mma16816(dK[2 * np + 1], am, bk[2], bk[3]);
@@ -685,7 +704,7 @@ __global__ void __launch_bounds__(256) tc_bwd_local_kernel(LocPtrs p) {
                     mma16816(dQ[2 * np + 1], ap, bk[2], bk[3]);
                 }
                 if (hi) {
-                    ldb_kn<DK>(bq, s.Q, 16 * kk, 64 * ch + 16 * np);
+                    ldb_kn<Tma128>(bq, s.Q, 16 * kk, 32 * cq + 16 * np);
                     mma16816(dK[2 * np], amt, bk[0], bk[1]);
                     mma16816(dK[2 * np + 1], amt, bk[2], bk[3]);
                     mma16816(tq[2 * np], apt, bq[0], bq[1]);
@@ -697,8 +716,8 @@ __global__ void __launch_bounds__(256) tc_bwd_local_kernel(LocPtrs p) {
         __nv_bfloat16* dqp = p.dq + row0 * DK;
         __nv_bfloat16* dkp = p.dk + row0 * DK;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int c = 64 * ch + 8 * j + 2 * (lane & 3);
+        for (int j = 0; j < 4; ++j) {
+            const int c = 32 * cq + 8 * j + 2 * (lane & 3);
             if (okl) {
                 *reinterpret_cast<uint32_t*>(dqp + (size_t)rl * rs * DK + c) =
                     pack_bf16(p.scale * dQ[j][0], p.scale * dQ[j][1]);
@@ -728,12 +747,12 @@ __global__ void __launch_bounds__(256) tc_bwd_local_kernel(LocPtrs p) {
         // red_s[w][0]: warp w's slice of <dS, S0>; red_s[w][1]: its rows' sum of
         // e^{G_last-G_i} <dKt_i, k_i> over its column half.
         float ssum = 0.f, lsum = 0.f;
-        for (int ww = 0; ww < 8; ++ww) {
+        for (int ww = 0; ww < LOC_WARPS; ++ww) {
             ssum += s.red_s[ww][0];
             lsum += s.red_s[ww][1];
         }
         float dG0 = 0.f, dG1 = 0.f, db0 = 0.f, db1 = 0.f;
-        for (int ww = 0; ww < 8; ++ww) {
+        for (int ww = 0; ww < LOC_WARPS; ++ww) {
             dG0 += s.red_g[ww][lane];
             dG1 += s.red_g[ww][lane + 32];
             db0 += s.red_b[ww][lane];
@@ -800,8 +819,10 @@ bool launch_tc_bwd(const gdn_dims& d, const void* q, const void* k, const void* 
                    tc_walk_bwd_kernel<1><<<d.B * d.H * (DV / 16), BW_THREADS, smem, st>>>(bp));
     }
     LocPtrs lp{};
+    lp.qmap = cp.qmap; lp.kmap = cp.kmap; lp.vmap = cp.vmap;
+    if (!encode_token_map(&lp.dOmap, dO, d.B, d.T, d.H)) return false;
     lp.q = cp.q; lp.k = cp.k; lp.v = cp.v; lp.dO = (const __nv_bfloat16*)dO; lp.g = g;
-    lp.beta = beta;
+    lp.beta = beta; lp.status = cp.status;
     lp.S0 = (const __nv_bfloat16*)(base + L.S0);
     lp.U = (const __nv_bfloat16*)(base + L.U);
     lp.dS = bp.dSout; lp.dU = bp.dUout; lp.Tb = cp.Tb; lp.G = cp.G;
@@ -809,10 +830,10 @@ bool launch_tc_bwd(const gdn_dims& d, const void* q, const void* k, const void* 
     lp.dg = dg; lp.dbeta = dbeta;
     lp.B = d.B; lp.T = d.T; lp.H = d.H; lp.NT = L.NT; lp.scale = d.scale;
     {
-        const int smem = sizeof(LocSmem);
+        const int smem = sizeof(LocSmem) + 1024;
         cudaFuncSetAttribute(tc_bwd_local_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         GDN_LAUNCH("tc_bwd_local", st,
-                   tc_bwd_local_kernel<<<(unsigned)L.nchunks, 256, smem, st>>>(lp));
+                   tc_bwd_local_kernel<<<(unsigned)L.nchunks, LOC_THREADS, smem, st>>>(lp));
     }
     return true;
 }

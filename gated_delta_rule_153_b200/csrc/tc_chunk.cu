@@ -110,7 +110,7 @@ __global__ void __launch_bounds__(128) tc_prep_kernel(const __grid_constant__ Ch
         s.sc1[lane + 32] = b1 * __expf(g1);
     }
     __syncthreads();
-    if (!mbar_wait(&s.bar, 0, p.status)) return;
+    if (__syncthreads_or(!mbar_wait(&s.bar, 0, p.status))) return;
 
     const int m0 = 16 * warp;
     // ---- decayed K K^T (-> A) and Q K^T (-> P) for row block `warp` --------
@@ -381,8 +381,7 @@ __global__ void __launch_bounds__(WALK_THREADS) tc_walk_kernel(const __grid_cons
     for (int n = 0; n < p.NT; ++n) {
         const int sn = n % WALK_STAGES;
         WalkStage<MT>& st = s.st[sn];
-        if (!mbar_wait(&s.full[sn], (n / WALK_STAGES) & 1, p.status)) return;
-        __syncthreads();  // stage n landed; S0 written; stage of chunk n-1 is free
+        if (__syncthreads_or(!mbar_wait(&s.full[sn], (n / WALK_STAGES) & 1, p.status))) return;  // all threads agree; stage n landed; S0 written; stage of chunk n-1 is free
         if (tid == 0 && n + WALK_STAGES - 1 < p.NT) {
             const int nn = n + WALK_STAGES - 1;
             walk_issue<MT, KDA>(s.st[nn % WALK_STAGES], &s.full[nn % WALK_STAGES], p, b, h, bh, nn,
@@ -495,8 +494,8 @@ __global__ void __launch_bounds__(WALK_THREADS) tc_walk_kernel(const __grid_cons
             if (MODE == 0) {
                 const size_t row = ((size_t)b * p.T + n * C + i) * p.H + h;
                 *reinterpret_cast<uint4*>(p.o + row * DV + a0 + 8 * pc) = v;
-            } else {
-                *reinterpret_cast<uint4*>(p.Uout + (cid * C + i) * DV + a0 + 8 * pc) = v;
+            } else {  // U image, Swz<128>: 16-byte piece at its swizzled position
+                *reinterpret_cast<uint4*>(p.Uout + cid * C * DV + swz<DV>(i, a0 + 8 * pc)) = v;
             }
         }
     }

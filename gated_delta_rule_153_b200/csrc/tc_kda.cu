@@ -111,7 +111,7 @@ __global__ void __launch_bounds__(128) tc_prep_kda_kernel(const __grid_constant_
         s.gl[c] = __expf(run);
     }
     __syncthreads();
-    if (!mbar_wait(&s.bar, 0, p.status)) return;
+    if (__syncthreads_or(!mbar_wait(&s.bar, 0, p.status))) return;
 
     // block spans and the six pair factors F_IJ
     if (warp < 4) {
