@@ -86,11 +86,40 @@ def kernel_work(name, B, T, H):
     return dict(bound="hbm", bytes=th * FWD_BYTES)
 
 
+# Kernel -> source file, for matching a recorded ncu traffic figure to the
+# code it was taken on (profiles/roofline_traffic.md).
+KERNEL_SOURCE = {"tc_prep": "tc_chunk.cu", "tc_walk_fwd": "tc_chunk.cu",
+                 "tc_walk_states": "tc_chunk.cu", "tc_walk_bwd": "tc_bwd.cu",
+                 "tc_bwd_local": "tc_bwd.cu", "tc_prep_kda": "tc_kda.cu",
+                 "decode_step": "decode.cu"}
+
+
+def recorded_traffic(kernel):
+    """DRAM bytes per launch (read + write) from the committed ncu summary,
+    or None when there is none or the kernel's source changed since."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "roofline_traffic.md")
+    src = KERNEL_SOURCE.get(kernel)
+    if not src or not os.path.exists(path):
+        return None
+    h = hashlib.sha256(open(os.path.join(ROOT, "gated_delta_rule_153_b200", "csrc", src),
+                            "rb").read()).hexdigest()[:16]
+    for line in open(path):
+        cells = [c.strip() for c in line.strip().strip("|").split("|")]
+        if len(cells) >= 4 and cells[0] == kernel and cells[2] == h:
+            try:
+                return float(cells[1])
+            except ValueError:
+                return None
+    return None
+
+
 class ClockSampler:
     """nvidia-smi clock / throttle-reason sampling during the timed region."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap,"
+              "utilization.gpu")
 
     def __init__(self, dev_index):
         self.proc = None
@@ -106,7 +135,7 @@ class ClockSampler:
                 pass
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", ident, f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             time.sleep(0.3)
         except Exception:
@@ -126,7 +155,7 @@ class ClockSampler:
             out = ""
         for line in out.strip().splitlines():
             parts = [x.strip() for x in line.split(",")]
-            if len(parts) >= 9:
+            if len(parts) >= 10:
                 self.rows.append(parts)
 
     def summary(self):
@@ -137,15 +166,15 @@ class ClockSampler:
                 return float(x)
             except ValueError:
                 return None
-        sm = [num(r[1]) for r in self.rows if num(r[1])]
-        power = [num(r[3]) for r in self.rows if num(r[3])]
-        load = [s for s, p in zip(sm, power)] if sm else []
+        busy = [r for r in self.rows if (num(r[9]) or 0) >= 50] or self.rows
+        sm = [num(r[1]) for r in busy if num(r[1])]
+        power = [num(r[3]) for r in busy if num(r[3])]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in self.rows for i in range(4)
+        reasons = sorted({names[i] for r in busy for i in range(4)
                           if r[5 + i].lower().startswith("active")})
-        return {"sm_mhz": statistics.median(load) if load else None,
+        return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": num(self.rows[0][2]), "power_w_max": max(power) if power else None,
-                "samples": len(self.rows), "reasons": reasons}
+                "samples": len(self.rows), "samples_under_load": len(busy), "reasons": reasons}
 
 
 def timed(fn, steps, warmup, barrier=lambda: None):
@@ -205,7 +234,7 @@ def run_ours(args, rank, world, dev, barrier, max_over_ranks):
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    cap = 64 * max(args.steps, 1)
+    cap = 8 * max(args.steps, 1) + 64
     idx = torch.cuda.current_device()
     with ClockSampler(idx) as clk:
         barrier()
@@ -238,9 +267,11 @@ def run_ours(args, rank, world, dev, barrier, max_over_ranks):
     dom_ms = statistics.mean(per[dom])
     wk = kernel_work(dom, cfg.B, cfg.T, cfg.H)
     achieved = wk["bytes"] / (dom_ms / 1e3) / 1e9
+    traffic = recorded_traffic(dom)
     roofline = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1),
                 "peak": pk["hbm"], "unit": "GB/s", "frac": round(achieved / pk["hbm"], 4),
-                "peak_source": pk["source"], "traffic": None,
+                "peak_source": pk["source"], "traffic": traffic,
+                "algorithmic_bytes": wk["bytes"],
                 "avg_launch_ms": round(dom_ms, 4),
                 "share": round(sum(per[dom]) / total_k, 4),
                 "kernels": {n: {"launches": len(v), "avg_ms": round(statistics.mean(v), 4),
@@ -345,7 +376,7 @@ def cpu_baseline_oracle(sample_B):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--headline-only", action="store_true",
