@@ -31,6 +31,10 @@ bool chunk_ptrs(ChunkPtrs& p, const gdn_dims& d, const TcLayout& L, const void* 
                 const void* k, const void* v, const float* g, const float* beta, void* ws);
 void launch_walk_states(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& cp,
                         const float* h0, void* ws, cudaStream_t st);
+void launch_prep_kda(const ChunkPtrs& p, size_t nchunks, cudaStream_t st);
+bool launch_bwd_local_kda(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& cp,
+                          const void* dO, void* dq, void* dk, void* dv, float* dg, float* dbeta,
+                          void* ws, cudaStream_t st);
 }  // namespace tc
 
 namespace {
@@ -53,7 +57,7 @@ struct alignas(1024) BwStage {
     __nv_bfloat16 W[C * DK];       // Swz<128>
     __nv_bfloat16 P[C * C];        // Swz<64>
     __nv_bfloat16 dO[C * 16 * MT]; // [token][16*MT value columns]
-    float G[C];
+    float G[DK];                   // G (scalar gate) or e^{G_last,c} (channel gate)
 };
 
 template <int MT>
@@ -71,6 +75,7 @@ struct BwPtrs {
     CUtensorMap qmap, kmap, dOmap;
     const float* dhT;
     const __nv_bfloat16 *W, *P;
+    const __nv_bfloat16 *Qg, *Kt;  // channel gate: prepared Q and K images
     const float* G;
     __nv_bfloat16 *dSout, *dUout;
     float* dh0;
@@ -79,21 +84,29 @@ struct BwPtrs {
     float scale;
 };
 
-template <int MT>
+// KDA: Q and K arrive pre-scaled (scale Q .* e^G, K .* e^{G_last-G}) as
+// workspace images, with the per-key chunk decay e^{G_last,c}.
+template <int MT, bool KDA>
 __device__ void bw_issue(BwStage<MT>& st, uint64_t* bar, const BwPtrs& p, int b, int h, int bh,
                          int n, int a0) {
     const size_t cid = (size_t)bh * p.NT + n;
-    mbar_arrive_expect(bar, (3 * C * DK + C * C + C * 16 * MT) * 2 + C * 4);
+    constexpr int GW = KDA ? DK : C;
+    mbar_arrive_expect(bar, (3 * C * DK + C * C + C * 16 * MT) * 2 + GW * 4);
     const int tok = b * p.T + n * C;
-    tma_load_tile(st.Q, &p.qmap, h, tok, bar);
-    tma_load_tile(st.K, &p.kmap, h, tok, bar);
+    if (KDA) {
+        bulk_g2s(st.Q, p.Qg + cid * C * DK, C * DK * 2, bar);
+        bulk_g2s(st.K, p.Kt + cid * C * DK, C * DK * 2, bar);
+    } else {
+        tma_load_tile(st.Q, &p.qmap, h, tok, bar);
+        tma_load_tile(st.K, &p.kmap, h, tok, bar);
+    }
     tma_load_3d(st.dO, &p.dOmap, a0, h, tok, bar);
     bulk_g2s(st.W, p.W + cid * C * DK, C * DK * 2, bar);
     bulk_g2s(st.P, p.P + cid * C * C, C * C * 2, bar);
-    bulk_g2s(st.G, p.G + cid * C, C * 4, bar);
+    bulk_g2s(st.G, p.G + cid * GW, GW * 4, bar);
 }
 
-template <int MT>
+template <int MT, bool KDA>
 __global__ void __launch_bounds__(BW_THREADS) tc_walk_bwd_kernel(const __grid_constant__ BwPtrs p) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     BwSmem<MT>& s = *reinterpret_cast<BwSmem<MT>*>(align1k(smem_raw));
@@ -132,7 +145,7 @@ __global__ void __launch_bounds__(BW_THREADS) tc_walk_bwd_kernel(const __grid_co
     __syncthreads();
     if (tid == 0)
         for (int k = 0; k < BW_STAGES - 1 && k < p.NT; ++k)
-            bw_issue<MT>(s.st[k], &s.full[k], p, b, h, bh, p.NT - 1 - k, a0);
+            bw_issue<MT, KDA>(s.st[k], &s.full[k], p, b, h, bh, p.NT - 1 - k, a0);
 
     for (int k = 0; k < p.NT; ++k) {  // step k handles chunk n = NT-1-k
         const int n = p.NT - 1 - k;
@@ -141,7 +154,8 @@ __global__ void __launch_bounds__(BW_THREADS) tc_walk_bwd_kernel(const __grid_co
         if (__syncthreads_or(!mbar_wait(&s.full[sk], (k / BW_STAGES) & 1, p.status))) return;  // all threads agree; stage landed; dS written; stage of step k-1 is free
         if (tid == 0 && k + BW_STAGES - 1 < p.NT) {
             const int kk = k + BW_STAGES - 1;
-            bw_issue<MT>(s.st[kk % BW_STAGES], &s.full[kk % BW_STAGES], p, b, h, bh, p.NT - 1 - kk, a0);
+            bw_issue<MT, KDA>(s.st[kk % BW_STAGES], &s.full[kk % BW_STAGES], p, b, h, bh,
+                              p.NT - 1 - kk, a0);
         }
         const size_t cid = (size_t)bh * p.NT + n;
         const int L = min(C, p.T - n * C);
@@ -154,11 +168,12 @@ __global__ void __launch_bounds__(BW_THREADS) tc_walk_bwd_kernel(const __grid_co
             const int i = e / RT, a = e % RT;
             const float x = i < L ? __bfloat162float(st.dO[i * RT + a]) : 0.f;
             s.dOt[swz<C>(a, i)] = __float2bfloat16_rn(x);
-            s.dOg[swz<C>(a, i)] = __float2bfloat16_rn(x * p.scale * __expf(st.G[i]));
+            s.dOg[swz<C>(a, i)] = __float2bfloat16_rn(KDA ? x : x * p.scale * __expf(st.G[i]));
         }
         __syncthreads();
-        const float Gl = st.G[C - 1];
-        const float et0 = __expf(Gl - st.G[i0]), et1 = __expf(Gl - st.G[i0 + 1]);
+        const float Gl = KDA ? 0.f : st.G[C - 1];
+        const float et0 = KDA ? 1.f : __expf(Gl - st.G[i0]);
+        const float et1 = KDA ? 1.f : __expf(Gl - st.G[i0 + 1]);
         // dU^T (rows x tokens 8w..8w+7) = dO^T P + (dS K^T) .* e^{G_last - G_r}
         {
             float a1[MT][4] = {}, a2[MT][2][4] = {};
@@ -203,7 +218,7 @@ __global__ void __launch_bounds__(BW_THREADS) tc_walk_bwd_kernel(const __grid_co
         __syncthreads();
         // dS0 = e^{G_last} dS + dOg^T Q - dU^T W   (columns 16w..16w+15)
         {
-            const float gam = __expf(Gl);
+            const float gam = KDA ? 1.f : __expf(Gl);
             float y[MT][2][4] = {}, z[MT][2][4] = {};
 #pragma unroll
             for (int kk = 0; kk < C / 16; ++kk) {
@@ -227,7 +242,10 @@ __global__ void __launch_bounds__(BW_THREADS) tc_walk_bwd_kernel(const __grid_co
                 for (int j = 0; j < 2; ++j)
 #pragma unroll
                     for (int e = 0; e < 4; ++e)
-                        dS[mt][j][e] = gam * dS[mt][j][e] + y[mt][j][e] - z[mt][j][e];
+                        dS[mt][j][e] =
+                            (KDA ? st.G[16 * w + 8 * j + 2 * (lane & 3) + (e & 1)] : gam) *
+                                dS[mt][j][e] +
+                            y[mt][j][e] - z[mt][j][e];
         }
         __syncthreads();  // everyone done with dS, dOt, dOg, dU; dU staged
 #pragma unroll
@@ -779,9 +797,19 @@ __global__ void __launch_bounds__(LOC_THREADS) tc_bwd_local_kernel(const __grid_
     }
 }
 
+template <int MT, bool KDA>
+void launch_walk_bwd(const BwPtrs& bp, cudaStream_t st) {
+    const int smem = sizeof(BwSmem<MT>) + 1024;
+    cudaFuncSetAttribute(tc_walk_bwd_kernel<MT, KDA>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         smem);
+    GDN_LAUNCH("tc_walk_bwd", st,
+               (tc_walk_bwd_kernel<MT, KDA><<<bp.B * bp.H * (DV / (16 * MT)), BW_THREADS, smem,
+                                              st>>>(bp)));
+}
+
 }  // namespace
 
-bool tc_bwd_supported(const gdn_dims& d) { return tc_supported(d) && d.gate == GDN_GATE_SCALAR; }
+bool tc_bwd_supported(const gdn_dims& d) { return tc_supported(d); }
 
 bool launch_tc_bwd(const gdn_dims& d, const void* q, const void* k, const void* v,
                    const float* g, const float* beta, const float* h0, const void* dO,
@@ -792,7 +820,9 @@ bool launch_tc_bwd(const gdn_dims& d, const void* q, const void* k, const void* 
     ChunkPtrs cp;
     if (!chunk_ptrs(cp, d, L, q, k, v, g, beta, ws)) return false;
     cp.Tb = (__nv_bfloat16*)(base + L.Tb);
-    launch_prep(cp, L.nchunks, st);
+    const bool kda_gate = d.gate == GDN_GATE_CHANNEL;
+    if (kda_gate) launch_prep_kda(cp, L.nchunks, st);
+    else launch_prep(cp, L.nchunks, st);
     launch_walk_states(d, L, cp, h0, ws, st);
 
     BwPtrs bp{};
@@ -807,17 +837,17 @@ bool launch_tc_bwd(const gdn_dims& d, const void* q, const void* k, const void* 
     bp.dUout = (__nv_bfloat16*)(base + L.dU);
     bp.dh0 = dh0; bp.status = cp.status;
     bp.B = d.B; bp.T = d.T; bp.H = d.H; bp.NT = L.NT; bp.scale = d.scale;
+    bp.Qg = cp.Qg; bp.Kt = cp.Kt;
+    const bool kda = d.gate == GDN_GATE_CHANNEL;
     if (two) {
-        const int smem = sizeof(BwSmem<2>) + 1024;
-        cudaFuncSetAttribute(tc_walk_bwd_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        GDN_LAUNCH("tc_walk_bwd", st,
-                   tc_walk_bwd_kernel<2><<<d.B * d.H * (DV / 32), BW_THREADS, smem, st>>>(bp));
+        if (kda) launch_walk_bwd<2, true>(bp, st);
+        else launch_walk_bwd<2, false>(bp, st);
     } else {
-        const int smem = sizeof(BwSmem<1>) + 1024;
-        cudaFuncSetAttribute(tc_walk_bwd_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        GDN_LAUNCH("tc_walk_bwd", st,
-                   tc_walk_bwd_kernel<1><<<d.B * d.H * (DV / 16), BW_THREADS, smem, st>>>(bp));
+        if (kda) launch_walk_bwd<1, true>(bp, st);
+        else launch_walk_bwd<1, false>(bp, st);
     }
+    if (kda_gate)
+        return launch_bwd_local_kda(d, L, cp, dO, dq, dk, dv, dg, dbeta, ws, st);
     LocPtrs lp{};
     lp.qmap = cp.qmap; lp.kmap = cp.kmap; lp.vmap = cp.vmap;
     if (!encode_token_map(&lp.dOmap, dO, d.B, d.T, d.H)) return false;

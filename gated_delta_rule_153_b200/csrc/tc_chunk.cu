@@ -488,7 +488,10 @@ __global__ void __launch_bounds__(WALK_THREADS) tc_walk_kernel(const __grid_cons
             for (int j = 0; j < 2; ++j) st_c<S128>(s.S0, 16 * mt, 16 * w + 8 * j, S[mt][j]);
         if (MODE == 1) fence_async_smem();
         constexpr int PIECES = RT / 8;  // 16-byte pieces per token row
-        for (int e = tid; e < PIECES * L; e += WALK_THREADS) {
+        // O: rows of the sequence only.  U image: all C rows, so the rows past a
+        // ragged end hold their exact value (zero) rather than stale workspace.
+        const int rows_out = MODE == 0 ? L : C;
+        for (int e = tid; e < PIECES * rows_out; e += WALK_THREADS) {
             const int i = e / PIECES, pc = e % PIECES;
             const uint4 v = *reinterpret_cast<const uint4*>(&s.O[i * RT + 8 * pc]);
             if (MODE == 0) {

@@ -347,3 +347,623 @@ void launch_prep_kda(const ChunkPtrs& p, size_t nchunks, cudaStream_t st) {
 
 }  // namespace tc
 }  // namespace gdn
+
+// ===========================================================================
+// Channel-gate backward, local gradients (one CTA of 16 warps per chunk).
+//
+// The products over the value dimension (dQg = dO S0, dKt = U dS, dW = -dU S0,
+// dP = lower(dO U^T)), the UT-transform chain (dT, X = dT T^T, dKg = T^T dW,
+// dVb = T^T dU, dA = -T^T X) and the state terms are those of the scalar gate.
+// Per-channel decays enter elementwise (e^{G_ic}, e^{G_last,c - G_ic}) and in
+// the four pair products, written with D_ijc = e^{G_ic - G_jc}:
+//   X1 = (dMM .* D) K,  X2 = (dMM .* D)^T K,  X3 = (dP .* D)^T Q,  X4 = (dP .* D) K
+// (dMM = dA .* beta_i), which give dK += X1 + X2 + scale X3, dQ' += X4 and
+// dG += K .* (X1 - X2 - scale X3) + scale Q .* X4.  They use the same block
+// factorisation as the forward: for j in block J < I,
+//   D_ijc = EL_ic F_IJc ER_jc,  F_IJc = e^{G_{16I,c} - G_{16J+15,c}},
+// so X1 over J < I is EL .* sum_J F_IJ .* (dMM_IJ (K .* ER)_J), and inside a
+// diagonal block D_ijc = EL_ic e^{G_{16I,c} - G_jc} (MMA form when the block's
+// span is at most 80, exact elementwise sums otherwise).  dg is the reverse
+// within-chunk cumsum of dG, per channel.
+// ===========================================================================
+namespace gdn {
+namespace tc {
+namespace {
+
+constexpr int KL_WARPS = 16, KL_THREADS = 32 * KL_WARPS;
+
+struct KdaLocSmem {
+    __nv_bfloat16 Q[C * DK];    // Tma128 (TMA)
+    __nv_bfloat16 K[C * DK];    // Tma128 (TMA)
+    __nv_bfloat16 dU[C * DV];   // Swz<128> image
+    __nv_bfloat16 dW[C * DK];   // Swz<128>
+    __nv_bfloat16 Tb[C * C];    // Swz<64> image
+    __nv_bfloat16 dP[C * C];    // Swz<64>: lower(dO U^T)
+    __nv_bfloat16 dT[C * C];    // Swz<64>: dT, then X = dT T^T, then dMM
+    union Scratch {
+        struct {
+            __nv_bfloat16 S[DV * DK];   // Swz<128>: S0, then dS
+            __nv_bfloat16 dO[C * DV];   // Tma128 (TMA)
+            __nv_bfloat16 U[C * DV];    // Swz<128> image
+        } p1;
+        struct {
+            __nv_bfloat16 Kl[C * DK], Kr[C * DK], Kd[C * DK], Ql[C * DK], Kg[C * DK];
+            __nv_bfloat16 V[C * DV];    // Tma128 (TMA), loaded at the start
+        } p2;
+        float dG[C][DK];
+    } u;
+    float G[C][DK];
+    float red_b[KL_WARPS][C];
+    float glp[2][4][DK];        // G_last column partials: [term][row block][channel]
+    float beta[C];
+    int diag_ok[4];
+    uint64_t bar[3];
+};
+
+struct KdaLocPtrs {
+    CUtensorMap qmap, kmap, vmap, dOmap;
+    const float *g, *beta;
+    const __nv_bfloat16 *S0, *U, *dS, *dU, *Tb;
+    __nv_bfloat16 *dq, *dk, *dv;
+    float *dg, *dbeta;
+    unsigned int* status;
+    int B, T, H, NT;
+    float scale;
+};
+
+using S128 = Swz<128>;
+using S64 = Swz<64>;
+
+__device__ __forceinline__ float bf(const __nv_bfloat16* t, uint32_t off) {
+    return __bfloat162float(t[off]);
+}
+
+// Sum over the 8 row groups of a warp (lanes with equal lane % 4).
+__device__ __forceinline__ float col_sum(float v) {
+    v += __shfl_xor_sync(0xffffffffu, v, 4);
+    v += __shfl_xor_sync(0xffffffffu, v, 8);
+    v += __shfl_xor_sync(0xffffffffu, v, 16);
+    return v;
+}
+
+__global__ void __launch_bounds__(KL_THREADS) tc_bwd_local_kda_kernel(const __grid_constant__ KdaLocPtrs p) {
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    KdaLocSmem& s = *reinterpret_cast<KdaLocSmem*>(align1k(smem_raw));
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    const int I = w >> 2, cq = w & 3, m0 = 16 * I;
+    const int cid = blockIdx.x;
+    const int bh = cid / p.NT, n = cid % p.NT, b = bh / p.H, h = bh % p.H;
+    const int t0 = n * C;
+    const int L = min(C, p.T - t0);
+    const size_t row0 = ((size_t)b * p.T + t0) * p.H + h;
+    const size_t rs = (size_t)p.H;
+    const int rl = m0 + (lane >> 2), rh = rl + 8;
+
+    if (tid == 0) {
+        for (int i = 0; i < 3; ++i) mbar_init(&s.bar[i], 1);
+        fence_mbar_init();
+        const int tok = b * p.T + t0;
+        // Q, K, dO, U, dU (five 64x128 tiles), S0 (128x128), T (64x64)
+        mbar_arrive_expect(&s.bar[0], (5 * C * DK + DV * DK + C * C) * 2);
+        tma_load_tile(s.Q, &p.qmap, h, tok, &s.bar[0]);
+        tma_load_tile(s.K, &p.kmap, h, tok, &s.bar[0]);
+        tma_load_tile(s.u.p1.dO, &p.dOmap, h, tok, &s.bar[0]);
+        bulk_g2s(s.u.p1.U, p.U + (size_t)cid * C * DV, C * DV * 2, &s.bar[0]);
+        bulk_g2s(s.dU, p.dU + (size_t)cid * C * DV, C * DV * 2, &s.bar[0]);
+        bulk_g2s(s.u.p1.S, p.S0 + (size_t)cid * DV * DK, DV * DK * 2, &s.bar[0]);
+        bulk_g2s(s.Tb, p.Tb + (size_t)cid * C * C, C * C * 2, &s.bar[0]);
+        mbar_arrive_expect(&s.bar[1], C * DV * 2);
+        tma_load_tile(s.u.p2.V, &p.vmap, h, tok, &s.bar[1]);
+    }
+    for (int e = tid; e < C * (DK / 4); e += KL_THREADS) {
+        const int r = e / (DK / 4), c4 = e % (DK / 4);
+        const bool ok = r < L;
+        cp_async16_zfill(&s.G[r][4 * c4], p.g + (row0 + (size_t)(ok ? r : 0) * rs) * DK + 4 * c4, ok);
+    }
+    cp_async_commit();
+    if (tid < C) s.beta[tid] = tid < L ? p.beta[row0 + tid * rs] : 0.f;
+    for (int e = tid; e < KL_WARPS * C; e += KL_THREADS) (&s.red_b[0][0])[e] = 0.f;
+    for (int e = tid; e < 2 * 4 * DK; e += KL_THREADS) (&s.glp[0][0][0])[e] = 0.f;
+    cp_async_wait<0>();
+    __syncthreads();
+    if (tid < DK) {  // per-channel within-chunk cumsum
+        float run = 0.f;
+        for (int i = 0; i < C; ++i) { run += s.G[i][tid]; s.G[i][tid] = run; }
+    }
+    __syncthreads();
+    if (w < 4) {
+        float sp = 0.f;
+        for (int c = lane; c < DK; c += 32) sp = fmaxf(sp, s.G[16 * w][c] - s.G[16 * w + 15][c]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) sp = fmaxf(sp, __shfl_xor_sync(0xffffffffu, sp, o));
+        if (lane == 0) s.diag_ok[w] = sp <= 80.f;
+    }
+    if (__syncthreads_or(!mbar_wait(&s.bar[0], 0, p.status))) return;
+    if (L < C) {  // dO rows past the sequence end belong to the next sequence
+        for (int e = tid; e < (C - L) * DV; e += KL_THREADS)
+            s.u.p1.dO[Tma128::off(L + e / DV, e % DV)] = __float2bfloat16_rn(0.f);
+    }
+    __syncthreads();
+
+    const float Gl_scale = 0.f;
+    (void)Gl_scale;
+    // this thread's 16 outputs of a 64x128 result: rows rl/rh, channels 32cq + 8j + 2(lane%4) + {0,1}
+    auto col = [&](int j, int e) { return 32 * cq + 8 * j + 2 * (lane & 3) + (e & 1); };
+    auto row = [&](int e) { return e < 2 ? rl : rh; };
+    float dQ[4][4], dK[4][4], dG[4][4];
+    float bsum_lo = 0.f, bsum_hi = 0.f;  // partial dbeta for rows rl, rh
+
+    // ---- phase 1a: dQg = dO S0, dW = -dU S0, dP = lower(dO U^T) ---------------
+    {
+        float aq[4][4] = {}, aw[4][4] = {};
+#pragma unroll
+        for (int kk = 0; kk < DV / 16; ++kk) {
+            uint32_t ad[4], au[4];
+            lda<Tma128>(ad, s.u.p1.dO, m0, 16 * kk);
+            lda<S128>(au, s.dU, m0, 16 * kk);
+#pragma unroll
+            for (int np = 0; np < 2; ++np) {
+                uint32_t bs[4];
+                ldb_kn<S128>(bs, s.u.p1.S, 16 * kk, 32 * cq + 16 * np);
+                mma16816(aq[2 * np], ad, bs[0], bs[1]);
+                mma16816(aq[2 * np + 1], ad, bs[2], bs[3]);
+                mma16816(aw[2 * np], au, bs[0], bs[1]);
+                mma16816(aw[2 * np + 1], au, bs[2], bs[3]);
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int r = row(e), c = col(j, e);
+                const float eg = __expf(s.G[r][c]);
+                dQ[j][e] = eg * aq[j][e];
+                dG[j][e] = p.scale * eg * aq[j][e] * bf(s.Q, Tma128::off(r, c));
+            }
+            float x[4] = {-aw[j][0], -aw[j][1], -aw[j][2], -aw[j][3]};
+            st_c<S128>(s.dW, m0, 32 * cq + 8 * j, x);
+        }
+        float dp[2][4] = {};
+#pragma unroll
+        for (int kk = 0; kk < DV / 16; ++kk) {
+            uint32_t ad[4], bu[4];
+            lda<Tma128>(ad, s.u.p1.dO, m0, 16 * kk);
+            ldb_nk<S128>(bu, s.u.p1.U, 16 * cq, 16 * kk);
+            mma16816(dp[0], ad, bu[0], bu[1]);
+            mma16816(dp[1], ad, bu[2], bu[3]);
+        }
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            float g[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int r = row(e), c = 16 * cq + 8 * j + 2 * (lane & 3) + (e & 1);
+                g[e] = c <= r ? dp[j][e] : 0.f;
+            }
+            st_c<S64>(s.dP, m0, 16 * cq + 8 * j, g);
+        }
+    }
+    // S0 elements this thread pairs with dS below (column c = tid % 128)
+    float s0r[32];
+    {
+        const int c = tid & (DK - 1), a0 = tid >> 7;
+#pragma unroll
+        for (int k = 0; k < 32; ++k) s0r[k] = bf(s.u.p1.S, swz<DK>(a0 + 4 * k, c));
+    }
+    __syncthreads();  // everyone done with S0
+    if (tid == 0) {
+        mbar_arrive_expect(&s.bar[2], DV * DK * 2);
+        bulk_g2s(s.u.p1.S, p.dS + (size_t)cid * DV * DK, DV * DK * 2, &s.bar[2]);
+    }
+    if (__syncthreads_or(!mbar_wait(&s.bar[2], 0, p.status))) return;
+
+    // ---- phase 1b: dKt = U dS, <dS, S0> per channel -----------------------------
+    {
+        float ak[4][4] = {};
+#pragma unroll
+        for (int kk = 0; kk < DV / 16; ++kk) {
+            uint32_t au[4];
+            lda<S128>(au, s.u.p1.U, m0, 16 * kk);
+#pragma unroll
+            for (int np = 0; np < 2; ++np) {
+                uint32_t bs[4];
+                ldb_kn<S128>(bs, s.u.p1.S, 16 * kk, 32 * cq + 16 * np);
+                mma16816(ak[2 * np], au, bs[0], bs[1]);
+                mma16816(ak[2 * np + 1], au, bs[2], bs[3]);
+            }
+        }
+        float colp[4][2] = {};
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int r = row(e), c = col(j, e);
+                const float et = __expf(s.G[C - 1][c] - s.G[r][c]);
+                dK[j][e] = et * ak[j][e];
+                const float hkt = et * ak[j][e] * bf(s.K, Tma128::off(r, c));
+                dG[j][e] -= hkt;
+                colp[j][e & 1] += hkt;
+            }
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const float v = col_sum(colp[j][e]);
+                if (lane < 4) s.glp[0][I][32 * cq + 8 * j + 2 * lane + e] = v;
+            }
+        const int c = tid & (DK - 1), a0 = tid >> 7;
+        float ss = 0.f;
+#pragma unroll
+        for (int k = 0; k < 32; ++k) ss += s0r[k] * bf(s.u.p1.S, swz<DK>(a0 + 4 * k, c));
+        s.glp[1][a0][c] = ss;
+    }
+    __syncthreads();  // phase-1 scratch is dead from here on
+
+    // ---- phase 2 prologue: scaled K / Q operands ----------------------------------
+    for (int e = tid; e < C * DK; e += KL_THREADS) {
+        const int i = e / DK, c = e % DK;
+        const int f = i & ~15, l = f + 15;
+        const float g = s.G[i][c];
+        const uint32_t o = Tma128::off(i, c);
+        const float kv = bf(s.K, o), qv = bf(s.Q, o);
+        const float el = __expf(g - s.G[f][c]);
+        s.u.p2.Kl[o] = __float2bfloat16_rn(kv * el);
+        s.u.p2.Ql[o] = __float2bfloat16_rn(qv * el);
+        s.u.p2.Kr[o] = __float2bfloat16_rn(kv * __expf(s.G[l][c] - g));
+        const float sp = s.G[f][c] - g;
+        s.u.p2.Kd[o] = __float2bfloat16_rn(sp <= 80.f ? kv * __expf(sp) : 0.f);
+        s.u.p2.Kg[o] = __float2bfloat16_rn(kv * __expf(g));
+    }
+    if (__syncthreads_or(!mbar_wait(&s.bar[1], 0, p.status))) return;
+    const bool dok = s.diag_ok[I];
+
+    // ---- phase 2: M (decayed K K^T, block J = cq) and dT -------------------------
+    float M[2][4];
+    {
+        const int J = cq;
+        float mk[2][4] = {}, tw[2][4] = {}, tu[2][4] = {};
+        const bool mma_m = J < I || (J == I && dok);
+#pragma unroll
+        for (int kk = 0; kk < DK / 16; ++kk) {
+            if (mma_m) {
+                uint32_t ak[4], bk[4];
+                lda<Tma128>(ak, s.u.p2.Kl, m0, 16 * kk);
+                if (J < I) {
+                    // scale the A fragment's channels by F_IJ
+                    const int k = 16 * kk + 2 * (lane & 3);
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) {
+                        const int kc = k + (r >> 1) * 8;
+                        const float f0 = __expf(s.G[16 * I][kc] - s.G[16 * J + 15][kc]);
+                        const float f1 = __expf(s.G[16 * I][kc + 1] - s.G[16 * J + 15][kc + 1]);
+                        float2 v = unpack_bf16(ak[r]);
+                        ak[r] = pack_bf16(v.x * f0, v.y * f1);
+                    }
+                    ldb_nk<Tma128>(bk, s.u.p2.Kr, 16 * J, 16 * kk);
+                } else {
+                    ldb_nk<Tma128>(bk, s.u.p2.Kd, 16 * J, 16 * kk);
+                }
+                mma16816(mk[0], ak, bk[0], bk[1]);
+                mma16816(mk[1], ak, bk[2], bk[3]);
+            }
+            uint32_t aw[4], au[4], bg[4], bv[4];
+            lda<S128>(aw, s.dW, m0, 16 * kk);
+            lda<S128>(au, s.dU, m0, 16 * kk);
+            ldb_nk<Tma128>(bg, s.u.p2.Kg, 16 * cq, 16 * kk);
+            ldb_nk<Tma128>(bv, s.u.p2.V, 16 * cq, 16 * kk);
+            mma16816(tw[0], aw, bg[0], bg[1]);
+            mma16816(tw[1], aw, bg[2], bg[3]);
+            mma16816(tu[0], au, bv[0], bv[1]);
+            mma16816(tu[1], au, bv[2], bv[3]);
+        }
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            float dt[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int r = row(e), c = 16 * cq + 8 * j + 2 * (lane & 3) + (e & 1);
+                dt[e] = s.beta[c] * (tw[j][e] + tu[j][e]);
+                float m = 0.f;
+                if (c < r) {
+                    if (mma_m) {
+                        m = mk[j][e];
+                    } else if (J == I) {  // exact: sum_ch k_r k_c e^{G_r - G_c}
+                        for (int ch = 0; ch < DK; ++ch)
+                            m += bf(s.K, Tma128::off(r, ch)) * bf(s.K, Tma128::off(c, ch)) *
+                                 __expf(s.G[r][ch] - s.G[c][ch]);
+                    }
+                }
+                M[j][e] = m;
+            }
+            st_c<S64>(s.dT, m0, 16 * cq + 8 * j, dt);
+        }
+    }
+    __syncthreads();
+
+    // ---- phase 3: X = dT T^T ; dKg = T^T dW ; dVb = T^T dU ---------------------
+    {
+        float x[2][4] = {};
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+            uint32_t a[4], bt[4];
+            lda<S64>(a, s.dT, m0, 16 * kk);
+            ldb_nk<S64>(bt, s.Tb, 16 * cq, 16 * kk);
+            mma16816(x[0], a, bt[0], bt[1]);
+            mma16816(x[1], a, bt[2], bt[3]);
+        }
+        float akg[4][4] = {}, avb[4][4] = {};
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+            if (kk < I) continue;  // T[j][i] = 0 for j < i
+            uint32_t a[4];
+            lda_t<S64>(a, s.Tb, m0, 16 * kk);
+#pragma unroll
+            for (int np = 0; np < 2; ++np) {
+                uint32_t bw[4], bu[4];
+                ldb_kn<S128>(bw, s.dW, 16 * kk, 32 * cq + 16 * np);
+                ldb_kn<S128>(bu, s.dU, 16 * kk, 32 * cq + 16 * np);
+                mma16816(akg[2 * np], a, bw[0], bw[1]);
+                mma16816(akg[2 * np + 1], a, bw[2], bw[3]);
+                mma16816(avb[2 * np], a, bu[0], bu[1]);
+                mma16816(avb[2 * np + 1], a, bu[2], bu[3]);
+            }
+        }
+        const float bl = s.beta[rl], bh2 = s.beta[rh];
+        __nv_bfloat16* dvp = p.dv + row0 * DV;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            float dvv[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int r = row(e), c = col(j, e);
+                const float br = e < 2 ? bl : bh2;
+                const float kgv = bf(s.u.p2.Kg, Tma128::off(r, c));  // k e^G
+                dK[j][e] += br * __expf(s.G[r][c]) * akg[j][e];
+                dG[j][e] += br * akg[j][e] * kgv;
+                const float hb = akg[j][e] * kgv + avb[j][e] * bf(s.u.p2.V, Tma128::off(r, c));
+                if (e < 2) bsum_lo += hb; else bsum_hi += hb;
+                dvv[e] = br * avb[j][e];
+            }
+            const int c = col(j, 0);
+            if (rl < L)
+                *reinterpret_cast<uint32_t*>(dvp + (size_t)rl * rs * DV + c) = pack_bf16(dvv[0], dvv[1]);
+            if (rh < L)
+                *reinterpret_cast<uint32_t*>(dvp + (size_t)rh * rs * DV + c) = pack_bf16(dvv[2], dvv[3]);
+        }
+        __syncthreads();  // everyone done reading dT
+#pragma unroll
+        for (int j = 0; j < 2; ++j) st_c<S64>(s.dT, m0, 16 * cq + 8 * j, x[j]);  // X
+    }
+    __syncthreads();
+
+    // ---- phase 4: dA = -T^T X (strictly lower), dbeta from M, dMM = dA beta_i ----
+    {
+        float da[2][4] = {};
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+            if (kk < I) continue;
+            uint32_t a[4], bx[4];
+            lda_t<S64>(a, s.Tb, m0, 16 * kk);
+            ldb_kn<S64>(bx, s.dT, 16 * kk, 16 * cq);
+            mma16816(da[0], a, bx[0], bx[1]);
+            mma16816(da[1], a, bx[2], bx[3]);
+        }
+        float mm[2][4];
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int r = row(e), c = 16 * cq + 8 * j + 2 * (lane & 3) + (e & 1);
+                const float dA = (c < r) ? -da[j][e] : 0.f;
+                if (e < 2) bsum_lo += dA * M[j][e]; else bsum_hi += dA * M[j][e];
+                mm[j][e] = dA * s.beta[r];
+            }
+        __syncthreads();  // everyone done reading X
+#pragma unroll
+        for (int j = 0; j < 2; ++j) st_c<S64>(s.dT, m0, 16 * cq + 8 * j, mm[j]);  // dMM
+    }
+    __syncthreads();
+
+    // ---- phase 5: the four decayed pair products ---------------------------------
+    {
+        // row side (X1, X4): blocks J < I scaled by F_IJ per channel, the diagonal
+        // block through Kd; everything then by EL = e^{G_r - G_f}
+        float x1[4][4] = {}, x4[4][4] = {};
+        for (int J = 0; J <= I; ++J) {
+            if (J == I && !dok) break;
+            float t1[4][4] = {}, t4[4][4] = {};
+            uint32_t am[4], ap[4];
+            lda<S64>(am, s.dT, m0, 16 * J);
+            lda<S64>(ap, s.dP, m0, 16 * J);
+            const __nv_bfloat16* B = J < I ? s.u.p2.Kr : s.u.p2.Kd;
+#pragma unroll
+            for (int np = 0; np < 2; ++np) {
+                uint32_t bk[4];
+                ldb_kn<Tma128>(bk, B, 16 * J, 32 * cq + 16 * np);
+                mma16816(t1[2 * np], am, bk[0], bk[1]);
+                mma16816(t1[2 * np + 1], am, bk[2], bk[3]);
+                mma16816(t4[2 * np], ap, bk[0], bk[1]);
+                mma16816(t4[2 * np + 1], ap, bk[2], bk[3]);
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int c = col(j, e);
+                    const float f = J < I ? __expf(s.G[16 * I][c] - s.G[16 * J + 15][c]) : 1.f;
+                    x1[j][e] += f * t1[j][e];
+                    x4[j][e] += f * t4[j][e];
+                }
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int r = row(e), c = col(j, e);
+                const float gr = s.G[r][c];
+                const float el = __expf(gr - s.G[m0][c]);
+                const float kv = bf(s.K, Tma128::off(r, c)), qv = bf(s.Q, Tma128::off(r, c));
+                const float dpd = bf(s.dP, swz<C>(r, r));
+                x1[j][e] *= el;
+                x4[j][e] *= el;
+                // The pair (r, r) has decay 1 and adds nothing to dG (its row- and
+                // column-side terms cancel).  Its rounded form is taken out of the dG
+                // sum here and on the column side, so that no bf16 residual of it
+                // swamps the small dg of a strongly decayed chunk.
+                float self4;
+                if (dok) {
+                    self4 = dpd * bf(s.u.p2.Kd, Tma128::off(r, c)) * el;
+                } else {  // exact diagonal-block sums, j < i inside block I
+                    for (int jj = m0; jj < r; ++jj) {
+                        const float d = __expf(gr - s.G[jj][c]);
+                        const float kj = bf(s.K, Tma128::off(jj, c));
+                        x1[j][e] += bf(s.dT, swz<C>(r, jj)) * d * kj;
+                        x4[j][e] += bf(s.dP, swz<C>(r, jj)) * d * kj;
+                    }
+                    self4 = dpd * kv;
+                    x4[j][e] += self4;
+                }
+                dK[j][e] += x1[j][e];
+                dQ[j][e] += x4[j][e];
+                dG[j][e] += kv * x1[j][e] + p.scale * qv * (x4[j][e] - self4);
+            }
+    }
+    {
+        // column side (X2, X3): blocks J > I scaled by ER_r F_JI, the diagonal
+        // block by e^{G_f - G_r} (its B operands carry EL_j)
+        float x2[4][4] = {}, x3[4][4] = {};
+        for (int J = I; J < 4; ++J) {
+            if (J == I && !dok) continue;
+            float t2[4][4] = {}, t3[4][4] = {};
+            uint32_t am[4], ap[4];
+            lda_t<S64>(am, s.dT, m0, 16 * J);
+            lda_t<S64>(ap, s.dP, m0, 16 * J);
+#pragma unroll
+            for (int np = 0; np < 2; ++np) {
+                uint32_t bk[4], bq[4];
+                ldb_kn<Tma128>(bk, s.u.p2.Kl, 16 * J, 32 * cq + 16 * np);
+                ldb_kn<Tma128>(bq, s.u.p2.Ql, 16 * J, 32 * cq + 16 * np);
+                mma16816(t2[2 * np], am, bk[0], bk[1]);
+                mma16816(t2[2 * np + 1], am, bk[2], bk[3]);
+                mma16816(t3[2 * np], ap, bq[0], bq[1]);
+                mma16816(t3[2 * np + 1], ap, bq[2], bq[3]);
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int r = row(e), c = col(j, e);
+                    const float gr = s.G[r][c];
+                    const float f = J > I ? __expf(s.G[m0 + 15][c] - gr + s.G[16 * J][c] -
+                                                   s.G[m0 + 15][c])
+                                          : __expf(s.G[m0][c] - gr);
+                    x2[j][e] += f * t2[j][e];
+                    x3[j][e] += f * t3[j][e];
+                }
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int r = row(e), c = col(j, e);
+                const float gr = s.G[r][c];
+                const float dpd = bf(s.dP, swz<C>(r, r));
+                float self3;  // the (r, r) pair's term, left out of dG as on the row side
+                if (dok) {
+                    self3 = dpd * bf(s.u.p2.Ql, Tma128::off(r, c)) * __expf(s.G[m0][c] - gr);
+                } else {  // exact diagonal-block sums, j > i inside block I
+                    for (int jj = r + 1; jj < m0 + 16; ++jj) {
+                        const float d = __expf(s.G[jj][c] - gr);
+                        x2[j][e] += bf(s.dT, swz<C>(jj, r)) * d * bf(s.K, Tma128::off(jj, c));
+                        x3[j][e] += bf(s.dP, swz<C>(jj, r)) * d * bf(s.Q, Tma128::off(jj, c));
+                    }
+                    self3 = dpd * bf(s.Q, Tma128::off(r, c));
+                    x3[j][e] += self3;
+                }
+                const float kv = bf(s.K, Tma128::off(r, c));
+                const float y = x2[j][e] + p.scale * x3[j][e];
+                dK[j][e] += y;
+                dG[j][e] -= kv * (x2[j][e] + p.scale * (x3[j][e] - self3));
+            }
+    }
+    {
+        const bool okl = rl < L, okh = rh < L;
+        __nv_bfloat16* dqp = p.dq + row0 * DK;
+        __nv_bfloat16* dkp = p.dk + row0 * DK;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int c = col(j, 0);
+            if (okl) {
+                *reinterpret_cast<uint32_t*>(dqp + (size_t)rl * rs * DK + c) =
+                    pack_bf16(p.scale * dQ[j][0], p.scale * dQ[j][1]);
+                *reinterpret_cast<uint32_t*>(dkp + (size_t)rl * rs * DK + c) = pack_bf16(dK[j][0], dK[j][1]);
+            }
+            if (okh) {
+                *reinterpret_cast<uint32_t*>(dqp + (size_t)rh * rs * DK + c) =
+                    pack_bf16(p.scale * dQ[j][2], p.scale * dQ[j][3]);
+                *reinterpret_cast<uint32_t*>(dkp + (size_t)rh * rs * DK + c) = pack_bf16(dK[j][2], dK[j][3]);
+            }
+        }
+    }
+    // ---- dbeta (row sums) and dg (per-channel reverse cumsum of dG) ---------------
+    {
+        float lo = bsum_lo, hi = bsum_hi;
+        lo += __shfl_xor_sync(0xffffffffu, lo, 1);
+        lo += __shfl_xor_sync(0xffffffffu, lo, 2);
+        hi += __shfl_xor_sync(0xffffffffu, hi, 1);
+        hi += __shfl_xor_sync(0xffffffffu, hi, 2);
+        if ((lane & 3) == 0) {
+            s.red_b[w][rl] = lo;
+            s.red_b[w][rh] = hi;
+        }
+    }
+    __syncthreads();  // phase-2 scratch is dead; dG goes there
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) s.u.dG[row(e)][col(j, e)] = dG[j][e];
+    __syncthreads();
+    if (tid < DK) {
+        const int c = tid;
+        float run = 0.f;
+        for (int rb = 0; rb < 4; ++rb)
+            run += s.glp[0][rb][c] + __expf(s.G[C - 1][c]) * s.glp[1][rb][c];
+        for (int i = C - 1; i >= 0; --i) {
+            run += s.u.dG[i][c];
+            if (i < L) p.dg[(row0 + (size_t)i * rs) * DK + c] = run;
+        }
+    } else if (tid < DK + C) {
+        const int i = tid - DK;
+        float sb = 0.f;
+        for (int ww = 0; ww < KL_WARPS; ++ww) sb += (ww >> 2) == (i >> 4) ? s.red_b[ww][i] : 0.f;
+        if (i < L) p.dbeta[row0 + (size_t)i * rs] = sb;
+    }
+}
+
+}  // namespace
+
+bool launch_bwd_local_kda(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& cp,
+                          const void* dO, void* dq, void* dk, void* dv, float* dg, float* dbeta,
+                          void* ws, cudaStream_t st) {
+    char* base = (char*)ws;
+    KdaLocPtrs lp{};
+    lp.qmap = cp.qmap; lp.kmap = cp.kmap; lp.vmap = cp.vmap;
+    if (!encode_token_map(&lp.dOmap, dO, d.B, d.T, d.H)) return false;
+    lp.g = cp.g; lp.beta = cp.beta;
+    lp.S0 = (const __nv_bfloat16*)(base + L.S0);
+    lp.U = (const __nv_bfloat16*)(base + L.U);
+    lp.dS = (const __nv_bfloat16*)(base + L.dS);
+    lp.dU = (const __nv_bfloat16*)(base + L.dU);
+    lp.Tb = cp.Tb;
+    lp.dq = (__nv_bfloat16*)dq; lp.dk = (__nv_bfloat16*)dk; lp.dv = (__nv_bfloat16*)dv;
+    lp.dg = dg; lp.dbeta = dbeta; lp.status = cp.status;
+    lp.B = d.B; lp.T = d.T; lp.H = d.H; lp.NT = L.NT; lp.scale = d.scale;
+    const int smem = sizeof(KdaLocSmem) + 1024;
+    cudaFuncSetAttribute(tc_bwd_local_kda_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    GDN_LAUNCH("tc_bwd_local_kda", st,
+               tc_bwd_local_kda_kernel<<<(unsigned)L.nchunks, KL_THREADS, smem, st>>>(lp));
+    return true;
+}
+
+}  // namespace tc
+}  // namespace gdn

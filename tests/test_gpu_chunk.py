@@ -73,6 +73,14 @@ def test_slow_gate_keeps_state_path_alive(dev, cfg, over):
     check_bwd(inp, dev)
 
 
+def test_strong_gate_ragged_tail(dev):
+    """g near -10 per token: the 8-token tail's gradients are tiny and must not
+    be swamped by rounding of the undecayed (i, i) pairs."""
+    inp = make_chunk_inputs(L350M, B=2, H=2, T=200, g_shift=10.0, h0_std=0.1, dhT_std=0.3)
+    check_fwd(inp, dev)
+    check_bwd(inp, dev)
+
+
 def test_zero_gate_small_beta(dev):
     inp = make_chunk_inputs(L350M, B=1, H=4, T=512, h0_std=0.1)
     inp["g"] = torch.zeros_like(inp["g"])
@@ -135,9 +143,11 @@ def test_deterministic(dev):
     dict(B=2, H=3, T=100, h0_std=0.1, dhT_std=0.3),             # ragged tail, MMA diagonal blocks
     dict(B=1, H=4, T=200, g_shift=10.0, h0_std=0.1),            # spans > 80: exact diagonal blocks
     dict(B=1, H=2, T=64, g_shift=-6.0, h0_std=0.2),             # slow gate, one chunk
+    dict(B=3, H=2, T=72, g_shift=4.0, h0_std=0.1),              # 8-token tails next to another sequence
+    dict(B=2, H=2, T=200, g_shift=10.0, dhT_std=0.3),           # strong gate: tiny dg in the short tail
 ])
-def test_kda_tensor_core_forward(dev, over):
-    """Channel-gate forward through the tensor-core path against the oracle."""
+def test_kda_tensor_core(dev, over):
+    """Channel-gate forward and backward through the tensor-core path against the oracle."""
     inp = make_chunk_inputs(KDA, **over)
     check_fwd(inp, dev)
     check_bwd(inp, dev)
