@@ -39,6 +39,11 @@ GDN_DEV void mbar_arrive_expect(uint64_t* bar, uint32_t bytes) {
                  ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
 }
 
+// Plain arrival (no transaction bytes).
+GDN_DEV void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 GDN_DEV bool mbar_try(uint64_t* bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(

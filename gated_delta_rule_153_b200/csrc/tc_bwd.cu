@@ -54,7 +54,7 @@ template <int MT>
 struct alignas(1024) BwStage {
     __nv_bfloat16 Q[C * DK];       // Tma128
     __nv_bfloat16 K[C * DK];       // Tma128
-    __nv_bfloat16 W[C * DK];       // Swz<128>
+    __nv_bfloat16 W[C * DK];       // Tma128
     __nv_bfloat16 P[C * C];        // Swz<64>
     __nv_bfloat16 dO[C * 16 * MT]; // [token][16*MT value columns]
     float G[DK];                   // G (scalar gate) or e^{G_last,c} (channel gate)
@@ -224,7 +224,7 @@ __global__ void __launch_bounds__(BW_THREADS) tc_walk_bwd_kernel(const __grid_co
             for (int kk = 0; kk < C / 16; ++kk) {
                 uint32_t bq[4], bw[4];
                 ldb_kn<Tma128>(bq, st.Q, 16 * kk, 16 * w);
-                ldb_kn<Swz<128>>(bw, st.W, 16 * kk, 16 * w);
+                ldb_kn<Tma128>(bw, st.W, 16 * kk, 16 * w);
 #pragma unroll
                 for (int mt = 0; mt < MT; ++mt) {
                     uint32_t ag[4], au[4];

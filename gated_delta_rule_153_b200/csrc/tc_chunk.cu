@@ -30,6 +30,8 @@
 namespace gdn {
 namespace tc {
 void launch_prep_kda(const ChunkPtrs& p, size_t nchunks, cudaStream_t st);
+void launch_walk5_fwd(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& c, const float* h0,
+                      void* o, float* hT, cudaStream_t st);
 }
 namespace {
 using namespace tc;
@@ -41,8 +43,8 @@ using P128 = Pad<128>;
 // prep: one CTA (4 warps) per chunk.  Warp w owns row block 16w..16w+15.
 // ---------------------------------------------------------------------------
 struct PrepSmem {
-    __nv_bfloat16 K[C * DK];   // Tma128; later: U~ staging [8][64][16]
-    __nv_bfloat16 Q[C * DK];   // Tma128; later: W staging (Swz<128> image)
+    __nv_bfloat16 K[C * DK];   // Tma128; later: U~^T staging (Swz<64>, 128 rows)
+    __nv_bfloat16 Q[C * DK];   // Tma128; later: W staging (Tma128 image)
     __nv_bfloat16 V[C * DV];   // Tma128
     __nv_bfloat16 P[C * C];    // Swz<64> image
     __nv_bfloat16 Ab[C * C];   // bf16 A (Swz<64>), strictly lower blocks used
@@ -249,15 +251,7 @@ __global__ void __launch_bounds__(128) tc_prep_kernel(const __grid_constant__ Ch
         }
     }
     __syncthreads();  // every warp is done reading K and V
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-        st_c<S128>(s.Q, m0, 8 * j, aw[j]);  // W image
-        // U~ staging: [tile = j/2][row][col 8*(j&1) + 2(lane%4) + {0,1}]
-        const int r = m0 + (lane >> 2), cc = 8 * (j & 1) + 2 * (lane & 3);
-        __nv_bfloat16* Ust = s.K + (j >> 1) * (C * 16);
-        *reinterpret_cast<uint32_t*>(Ust + r * 16 + cc) = pack_bf16(au[j][0], au[j][1]);
-        *reinterpret_cast<uint32_t*>(Ust + (r + 8) * 16 + cc) = pack_bf16(au[j][2], au[j][3]);
-    }
+    stage_w_ut(s.Q, s.K, aw, au, m0);  // W image in Q's slot, U~^T image in K's
     fence_async_smem();
     __syncthreads();
     if (tid == 0) {
@@ -286,9 +280,9 @@ template <int MT>
 struct alignas(1024) WalkStage {
     __nv_bfloat16 Q[C * DK];                 // Tma128
     __nv_bfloat16 K[C * DK];                 // Tma128
-    __nv_bfloat16 W[C * DK];                 // Swz<128>
+    __nv_bfloat16 W[C * DK];                 // Tma128
     __nv_bfloat16 P[C * C];                  // Swz<64>
-    __nv_bfloat16 Ut[MT][C * 16];            // [tile][token][16 value rows]
+    __nv_bfloat16 Ut[16 * MT * C];           // rows a0.. of the U~^T image (Swz<64>)
     float G[DK];                             // G (scalar gate) or e^{G_last,c} (channel gate)
 };
 
@@ -318,23 +312,25 @@ struct WalkPtrs {
 
 // KDA: the chunk's Q and K arrive pre-scaled (scale Q .* e^G, K .* e^{G_last-G})
 // as workspace images, with the per-key chunk decay e^{G_last,c}.
-template <int MT, bool KDA>
+// MODE 1 (state recompute) has no output, so it fetches neither Q nor P.
+template <int MT, int MODE, bool KDA>
 __device__ void walk_issue(WalkStage<MT>& st, uint64_t* bar, const WalkPtrs& p, int b, int h,
                            int bh, int n, int tile0) {
     const size_t cid = (size_t)bh * p.NT + n;
     constexpr int GW = KDA ? DK : C;
-    mbar_arrive_expect(bar, (3 * C * DK + C * C + MT * C * 16) * 2 + GW * 4);
+    constexpr int QP = MODE == 0 ? C * DK + C * C : 0;
+    mbar_arrive_expect(bar, (2 * C * DK + QP + MT * C * 16) * 2 + GW * 4);
     const int tok = b * p.T + n * C;
     if (KDA) {
-        bulk_g2s(st.Q, p.Qg + cid * C * DK, C * DK * 2, bar);
+        if (MODE == 0) bulk_g2s(st.Q, p.Qg + cid * C * DK, C * DK * 2, bar);
         bulk_g2s(st.K, p.Kt + cid * C * DK, C * DK * 2, bar);
     } else {
-        tma_load_tile(st.Q, &p.qmap, h, tok, bar);
+        if (MODE == 0) tma_load_tile(st.Q, &p.qmap, h, tok, bar);
         tma_load_tile(st.K, &p.kmap, h, tok, bar);
     }
     bulk_g2s(st.W, p.W + cid * C * DK, C * DK * 2, bar);
-    bulk_g2s(st.P, p.P + cid * C * C, C * C * 2, bar);
-    bulk_g2s(&st.Ut[0][0], p.Ut + (cid * 8 + tile0) * C * 16, MT * C * 16 * 2, bar);
+    if (MODE == 0) bulk_g2s(st.P, p.P + cid * C * C, C * C * 2, bar);
+    bulk_g2s(st.Ut, p.Ut + cid * C * DV + tile0 * 16 * C, MT * C * 16 * 2, bar);
     bulk_g2s(st.G, p.G + cid * GW, GW * 4, bar);
 }
 
@@ -376,7 +372,7 @@ __global__ void __launch_bounds__(WALK_THREADS) tc_walk_kernel(const __grid_cons
     __syncthreads();
     if (tid == 0)
         for (int n = 0; n < WALK_STAGES - 1 && n < p.NT; ++n)
-            walk_issue<MT, KDA>(s.st[n], &s.full[n], p, b, h, bh, n, tile0);
+            walk_issue<MT, MODE, KDA>(s.st[n], &s.full[n], p, b, h, bh, n, tile0);
 
     for (int n = 0; n < p.NT; ++n) {
         const int sn = n % WALK_STAGES;
@@ -384,7 +380,7 @@ __global__ void __launch_bounds__(WALK_THREADS) tc_walk_kernel(const __grid_cons
         if (__syncthreads_or(!mbar_wait(&s.full[sn], (n / WALK_STAGES) & 1, p.status))) return;  // all threads agree; stage n landed; S0 written; stage of chunk n-1 is free
         if (tid == 0 && n + WALK_STAGES - 1 < p.NT) {
             const int nn = n + WALK_STAGES - 1;
-            walk_issue<MT, KDA>(s.st[nn % WALK_STAGES], &s.full[nn % WALK_STAGES], p, b, h, bh, nn,
+            walk_issue<MT, MODE, KDA>(s.st[nn % WALK_STAGES], &s.full[nn % WALK_STAGES], p, b, h, bh, nn,
                                 tile0);
         }
         const int L = min(C, p.T - n * C);
@@ -402,7 +398,7 @@ __global__ void __launch_bounds__(WALK_THREADS) tc_walk_kernel(const __grid_cons
 #pragma unroll
         for (int kk = 0; kk < DK / 16; ++kk) {
             uint32_t bw[2], bq[2];
-            ldb_nk1<S128>(bw, st.W, 8 * w, 16 * kk);
+            ldb_nk1<Tma128>(bw, st.W, 8 * w, 16 * kk);
             if (MODE == 0) ldb_nk1<Tma128>(bq, st.Q, 8 * w, 16 * kk);
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt) {
@@ -418,7 +414,7 @@ __global__ void __launch_bounds__(WALK_THREADS) tc_walk_kernel(const __grid_cons
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int r = r_lo + 8 * (e >> 1), i = i0 + (e & 1);
-                u[e] = __bfloat162float(st.Ut[mt][i * 16 + r]) - (X[mt][0][e] + X[mt][1][e]);
+                u[e] = __bfloat162float(st.Ut[swz<C>(16 * mt + r, i)]) - (X[mt][0][e] + X[mt][1][e]);
                 us[e] = u[e] * ((e & 1) ? et1 : et0);
             }
             st_c<S64>(s.Uu, 16 * mt, 8 * w, u);
@@ -608,11 +604,19 @@ bool launch_tc_fwd(const gdn_dims& d, const void* q, const void* k, const void* 
     const bool kda = d.gate == GDN_GATE_CHANNEL;
     if (kda) launch_prep_kda(cp, L.nchunks, st);
     else launch_prep(cp, L.nchunks, st);
-    WalkPtrs w = make_walk_ptrs(d, L, cp, h0);
-    w.o = (__nv_bfloat16*)o;
-    w.hT = hT;
-    if (kda) launch_walk<0, true>(w, st);
-    else launch_walk<0, false>(w, st);
+    // The tcgen05 walk carries a whole head per CTA; with few heads the
+    // 16-row walk, which spreads each head over eight CTAs, fills more SMs.
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if ((long long)d.B * d.H * 4 >= sms) {
+        launch_walk5_fwd(d, L, cp, h0, o, hT, st);
+    } else {
+        WalkPtrs w = make_walk_ptrs(d, L, cp, h0);
+        w.o = (__nv_bfloat16*)o;
+        w.hT = hT;
+        if (kda) launch_walk<0, true>(w, st);
+        else launch_walk<0, false>(w, st);
+    }
     return true;
 }
 

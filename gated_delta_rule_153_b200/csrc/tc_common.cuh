@@ -45,8 +45,9 @@ inline TcLayout tc_layout(const gdn_dims& d, bool bwd) {
 }
 
 // Workspace images (written by prep with bulk stores, read back the same way):
-//   W   [chunk][64][128] bf16, Swz<128> tile image
-//   Ut  [chunk][8 tiles][64][16] bf16, value columns 16*tile .. +15, row-major
+//   W   [chunk] Tma128 image of the 64x128 W (two 64-column K-major panels)
+//   Ut  [chunk] Swz<64> image of U~^T: 128 value rows x 64 tokens, so any
+//       16-row slice of the state is one contiguous 2 KB range
 //   P   [chunk][64][64]  bf16, Swz<64> tile image (scale folded in)
 //   G   [chunk][64] fp32 within-chunk cumsum of g (padding rows repeat the last);
 //       channel gate: [chunk][128] fp32 e^{G_last,c}, the per-key decay of a chunk
@@ -67,6 +68,22 @@ struct ChunkPtrs {
     __nv_bfloat16 *Qg, *Kt;  // channel gate only
     unsigned int* status;
 };
+
+// Stage the W and U~ images from a warp's 16-row block of the W = T diag(.) K
+// and U~ = T diag(beta) V accumulators (m16n8 fragments, 16 n-blocks of 8).
+GDN_DEV void stage_w_ut(__nv_bfloat16* Wst, __nv_bfloat16* Ust, const float (&aw)[16][4],
+                        const float (&au)[16][4], int m0) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+        st_c<Tma128>(Wst, m0, 8 * j, aw[j]);
+        const int r = m0 + (lane >> 2), c = 8 * j + 2 * (lane & 3);
+        Ust[swz<C>(c, r)] = __float2bfloat16_rn(au[j][0]);
+        Ust[swz<C>(c + 1, r)] = __float2bfloat16_rn(au[j][1]);
+        Ust[swz<C>(c, r + 8)] = __float2bfloat16_rn(au[j][2]);
+        Ust[swz<C>(c + 1, r + 8)] = __float2bfloat16_rn(au[j][3]);
+    }
+}
 
 // Round a dynamic shared-memory pointer up to the 1024-byte alignment that
 // 128-byte-swizzled TMA destinations need (launches request 1 KB extra).

@@ -43,7 +43,7 @@ struct KdaPrepSmem {
     __nv_bfloat16 V[C * DV];    // Tma128 (TMA)
     __nv_bfloat16 Kl[C * DK];   // K .* EL; later K .* e^G (W operand), then W image
     __nv_bfloat16 Ql[C * DK];   // Q .* EL; later Kt image
-    __nv_bfloat16 Kr[C * DK];   // K .* ER; later U~ staging
+    __nv_bfloat16 Kr[C * DK];   // K .* ER; later U~^T staging
     __nv_bfloat16 Kd[C * DK];   // K .* e^{G_f - G} (diagonal blocks whose span passed)
     float G[C][DK];             // per-channel cumsum
     __nv_bfloat16 P[C * C];     // Swz<64> image
@@ -314,14 +314,7 @@ __global__ void __launch_bounds__(128) tc_prep_kda_kernel(const __grid_constant_
         }
     }
     __syncthreads();  // done reading Kl and V
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-        st_c<S128>(s.Kl, m0, 8 * j, aw[j]);  // W image
-        const int r = m0 + (lane >> 2), cc = 8 * (j & 1) + 2 * (lane & 3);
-        __nv_bfloat16* Ust = s.Kr + (j >> 1) * (C * 16);
-        *reinterpret_cast<uint32_t*>(Ust + r * 16 + cc) = pack_bf16(au[j][0], au[j][1]);
-        *reinterpret_cast<uint32_t*>(Ust + (r + 8) * 16 + cc) = pack_bf16(au[j][2], au[j][3]);
-    }
+    stage_w_ut(s.Kl, s.Kr, aw, au, m0);  // W image in Kl's slot, U~^T image in Kr's
     fence_async_smem();
     __syncthreads();
     if (tid == 0) {

@@ -89,6 +89,20 @@ def test_zero_gate_small_beta(dev):
     check_bwd(inp, dev)
 
 
+@pytest.mark.parametrize("cfg,over", [
+    (L350M, dict(B=3, H=16, T=200, h0_std=0.1, dhT_std=0.3)),             # ragged tail, h0
+    (L350M, dict(B=3, H=16, T=72, g_shift=10.0, h0_std=0.1)),             # strong gate, 8-token tails
+    (KDA, dict(B=3, H=16, T=200, h0_std=0.1)),
+    (KDA, dict(B=3, H=16, T=130, g_shift=10.0, h0_std=0.1)),
+    (KDA, dict(B=3, H=16, T=64, g_shift=-6.0, h0_std=0.2)),               # slow gate: the state dominates
+])
+def test_whole_head_walk(dev, cfg, over):
+    """Enough heads for the forward to carry one whole head per CTA on the
+    fifth-generation tensor cores (state in registers, operands in TMEM)."""
+    inp = make_chunk_inputs(cfg, **over)
+    check_fwd(inp, dev)
+
+
 # ---- invariants -----------------------------------------------------------
 def test_chunk_size_invariance(dev):
     inp = make_chunk_inputs(L350M, B=1, H=4, T=1000, dtype="f32", g_shift=-2.0, h0_std=0.2)
