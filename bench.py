@@ -64,7 +64,7 @@ def kernel_work(name, B, T, H):
     if name == "tc_prep":
         # reads q,k,v (bf16), g, beta; writes W, U~ (bf16 C x 128), P (bf16 C x C), G
         return dict(bound="hbm", bytes=th * (3 * 256 + 8 + 2 * 256 + 128 + 4))
-    if name in ("tc_walk_fwd",):
+    if name in ("tc_walk_fwd", "tc5_walk_fwd"):
         # reads W, Q, K, U~ (bf16), P, G; writes O
         return dict(bound="hbm", bytes=th * (4 * 256 + 128 + 4 + 256))
     if name in ("tc_walk_states",):
@@ -89,6 +89,7 @@ def kernel_work(name, B, T, H):
 # Kernel -> source file, for matching a recorded ncu traffic figure to the
 # code it was taken on (profiles/roofline_traffic.md).
 KERNEL_SOURCE = {"tc_prep": "tc_chunk.cu", "tc_walk_fwd": "tc_chunk.cu",
+                 "tc5_walk_fwd": "tc5_walk.cu",
                  "tc_walk_states": "tc_chunk.cu", "tc_walk_bwd": "tc_bwd.cu",
                  "tc_bwd_local": "tc_bwd.cu", "tc_prep_kda": "tc_kda.cu",
                  "decode_step": "decode.cu"}

@@ -44,13 +44,12 @@ using P128 = Pad<128>;
 // ---------------------------------------------------------------------------
 struct PrepSmem {
     __nv_bfloat16 K[C * DK];   // Tma128; later: U~^T staging (Swz<64>, 128 rows)
-    __nv_bfloat16 Q[C * DK];   // Tma128; later: W staging (Tma128 image)
+    __nv_bfloat16 Q[C * DK];   // Tma128; then the fp32 diagonal blocks of A and the
+                               // 16x16 scratch of the block solve; then W staging
     __nv_bfloat16 V[C * DV];   // Tma128
     __nv_bfloat16 P[C * C];    // Swz<64> image
     __nv_bfloat16 Ab[C * C];   // bf16 A (Swz<64>), strictly lower blocks used
     __nv_bfloat16 Tb[C * C];   // bf16 T (Swz<64>)
-    __nv_bfloat16 X[4][16 * 16];
-    float Ad[4][16][17];       // fp32 diagonal blocks of A
     float G[C];
     float beta[C];
     float sc1[C];              // beta_j e^{G_j}
@@ -115,6 +114,11 @@ __global__ void __launch_bounds__(128) tc_prep_kernel(const __grid_constant__ Ch
     if (__syncthreads_or(!mbar_wait(&s.bar, 0, p.status))) return;
 
     const int m0 = 16 * warp;
+    // Q is dead once Q K^T is formed: its space holds the diagonal blocks of A
+    // (fp32, padded rows) and each warp's 16x16 bf16 scratch.
+    auto Ad = reinterpret_cast<float(*)[16][17]>(s.Q);
+    auto Xs = reinterpret_cast<__nv_bfloat16(*)[16 * 16]>(reinterpret_cast<unsigned char*>(s.Q) +
+                                                          4 * 16 * 17 * sizeof(float));
     // ---- decayed K K^T (-> A) and Q K^T (-> P) for row block `warp` --------
     {
         float acck[8][4], accq[8][4];
@@ -138,6 +142,7 @@ __global__ void __launch_bounds__(128) tc_prep_kernel(const __grid_constant__ Ch
                 mma16816(accq[2 * np + 1], aq, bf[2], bf[3]);
             }
         }
+        __syncthreads();  // every warp is done reading Q
         const int ra = m0 + (lane >> 2), rb2 = ra + 8;
         const float Gra = s.G[ra], Grb = s.G[rb2], bra = s.beta[ra], brb = s.beta[rb2];
 #pragma unroll
@@ -152,7 +157,7 @@ __global__ void __launch_bounds__(128) tc_prep_kernel(const __grid_constant__ Ch
                 a[e] = (c < r) ? ((e < 2) ? bra : brb) * acck[j][e] * dec : 0.f;
                 // rows past the sequence end are zero (their q rows are not ours)
                 pv[e] = (r < L) ? accq[j][e] * dec * p.scale : 0.f;
-                if ((j >> 1) == warp) s.Ad[warp][r - m0][c - m0] = a[e];
+                if ((j >> 1) == warp) Ad[warp][r - m0][c - m0] = a[e];
             }
             st_c<S64>(s.Ab, m0, 8 * j, a);
             st_c<S64>(s.P, m0, 8 * j, pv);
@@ -169,7 +174,7 @@ __global__ void __launch_bounds__(128) tc_prep_kernel(const __grid_constant__ Ch
         for (int i = 0; i < 16; ++i) {
             float v = (i == c) ? 1.f : 0.f;
 #pragma unroll
-            for (int j = 0; j < i; ++j) v -= s.Ad[warp][i][j] * t[j];
+            for (int j = 0; j < i; ++j) v -= Ad[warp][i][j] * t[j];
             t[i] = (i < c) ? 0.f : v;
         }
         if (lane < 16) {
@@ -200,8 +205,8 @@ __global__ void __launch_bounds__(128) tc_prep_kernel(const __grid_constant__ Ch
 #pragma unroll
             for (int jn = 0; jn < 2; ++jn) {
                 const int r = lane >> 2, cc = 8 * jn + 2 * (lane & 3);
-                *reinterpret_cast<uint32_t*>(&s.X[warp][r * 16 + cc]) = pack_bf16(x[jn][0], x[jn][1]);
-                *reinterpret_cast<uint32_t*>(&s.X[warp][(r + 8) * 16 + cc]) = pack_bf16(x[jn][2], x[jn][3]);
+                *reinterpret_cast<uint32_t*>(&Xs[warp][r * 16 + cc]) = pack_bf16(x[jn][0], x[jn][1]);
+                *reinterpret_cast<uint32_t*>(&Xs[warp][(r + 8) * 16 + cc]) = pack_bf16(x[jn][2], x[jn][3]);
             }
             __syncwarp();
             uint32_t a[4], bx[4];
@@ -210,7 +215,7 @@ __global__ void __launch_bounds__(128) tc_prep_kernel(const __grid_constant__ Ch
                 // B[k][n] = X[k][n]
                 const int idx = lane >> 3;
                 const int row = (lane & 7) + (idx & 1) * 8, col = (idx >> 1) * 8;
-                ldsm_x4_t(bx, smem_u32(&s.X[warp][row * 16 + col]));
+                ldsm_x4_t(bx, smem_u32(&Xs[warp][row * 16 + col]));
             }
             float y[2][4] = {};
             mma16816(y[0], a, bx[0], bx[1]);
