@@ -25,6 +25,11 @@
 // epilogue-only operand, is read from global memory into registers one chunk
 // ahead.
 //
+// MODE 1 (state recompute for the backward) has no output: it fetches
+// neither Q nor P, runs X = S0 W^T alone in place of [X|Y], skips Z, and
+// stores each chunk's entering state (bf16, Swz<128> image) and U (Swz<128>,
+// token rows) for the backward kernels.
+//
 // Channel gate: Q and K arrive as prepared images (scale Q .* e^G and
 // K .* e^{G_last - G}), G holds e^{G_last,c}, Us = U, and the decay of the
 // state is per key column.
@@ -48,6 +53,7 @@ constexpr int W5_STAGES = 3;
 // 64 columns), U and Us (32 columns each)
 constexpr int TXY = 0, TD = 128, TZ = 256, TAS = 320, TAU = 384, TAUS = 416, TCOLS = 512;
 constexpr uint32_t ID_XY = tc5::idesc_bf16(128, 128, false, false);
+constexpr uint32_t ID_X = tc5::idesc_bf16(128, 64, false, false);
 constexpr uint32_t ID_D = tc5::idesc_bf16(128, 128, false, true);
 constexpr uint32_t ID_Z = tc5::idesc_bf16(128, 64, false, false);
 
@@ -74,32 +80,35 @@ struct W5Ptrs {
     const float* G;
     __nv_bfloat16* o;
     float* hT;
+    __nv_bfloat16 *S0out, *Uout;  // MODE 1
     unsigned int* status;
     int B, T, H, NT;
     float scale;
 };
 
-template <bool KDA>
+template <bool KDA, int MODE>
 __device__ void w5_issue(W5Stage& st, uint64_t* bar, const W5Ptrs& p, int b, int h, int bh, int n) {
     const size_t cid = (size_t)bh * p.NT + n;
     constexpr int GW = KDA ? DK : C;
     constexpr int PANEL = C * 64;  // elements of one 64x64 panel
-    mbar_arrive_expect(bar, (3 * C * DK + C * C) * 2 + GW * 4);
+    mbar_arrive_expect(bar, (MODE == 0 ? 3 * C * DK + C * C : 2 * C * DK) * 2 + GW * 4);
     const __nv_bfloat16* W = p.W + cid * C * DK;
     bulk_g2s(st.WQ, W, PANEL * 2, bar);
     bulk_g2s(st.WQ + 2 * PANEL, W + PANEL, PANEL * 2, bar);
-    if (KDA) {
-        const __nv_bfloat16* Qg = p.Qg + cid * C * DK;
-        bulk_g2s(st.WQ + PANEL, Qg, PANEL * 2, bar);
-        bulk_g2s(st.WQ + 3 * PANEL, Qg + PANEL, PANEL * 2, bar);
-        bulk_g2s(st.K, p.Kt + cid * C * DK, C * DK * 2, bar);
-    } else {
-        const int tok = b * p.T + n * C;
-        tma_load_3d(st.WQ + PANEL, &p.qmap, 0, h, tok, bar);
-        tma_load_3d(st.WQ + 3 * PANEL, &p.qmap, 64, h, tok, bar);
-        tma_load_tile(st.K, &p.kmap, h, tok, bar);
+    const int tok = b * p.T + n * C;
+    if (MODE == 0) {
+        if (KDA) {
+            const __nv_bfloat16* Qg = p.Qg + cid * C * DK;
+            bulk_g2s(st.WQ + PANEL, Qg, PANEL * 2, bar);
+            bulk_g2s(st.WQ + 3 * PANEL, Qg + PANEL, PANEL * 2, bar);
+        } else {
+            tma_load_3d(st.WQ + PANEL, &p.qmap, 0, h, tok, bar);
+            tma_load_3d(st.WQ + 3 * PANEL, &p.qmap, 64, h, tok, bar);
+        }
+        bulk_g2s(st.P, p.P + cid * C * C, C * C * 2, bar);
     }
-    bulk_g2s(st.P, p.P + cid * C * C, C * C * 2, bar);
+    if (KDA) bulk_g2s(st.K, p.Kt + cid * C * DK, C * DK * 2, bar);
+    else tma_load_tile(st.K, &p.kmap, h, tok, bar);
     bulk_g2s(st.G, p.G + cid * GW, GW * 4, bar);
 }
 
@@ -115,7 +124,7 @@ GDN_DEV void warp_arrive(uint64_t* bar) {
 }
 
 
-template <bool KDA>
+template <bool KDA, int MODE>
 __global__ void __launch_bounds__(W5_THREADS) tc5_walk_kernel(const __grid_constant__ W5Ptrs p) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     W5Smem& s = *reinterpret_cast<W5Smem*>(align1k(smem_raw));
@@ -147,7 +156,7 @@ __global__ void __launch_bounds__(W5_THREADS) tc5_walk_kernel(const __grid_const
             for (int n = 0; n < p.NT; ++n) {
                 const int sn = n % W5_STAGES;
                 if (n >= W5_STAGES && !mbar_wait(&s.empty[sn], ((n / W5_STAGES) - 1) & 1, p.status)) break;
-                w5_issue<KDA>(s.st[sn], &s.full[sn], p, b, h, bh, n);
+                w5_issue<KDA, MODE>(s.st[sn], &s.full[sn], p, b, h, bh, n);
                 issued = n + 1;
             }
             // Leave no load in flight (returns at once for stages already consumed).
@@ -167,7 +176,8 @@ __global__ void __launch_bounds__(W5_THREADS) tc5_walk_kernel(const __grid_const
                 const uint32_t sWQ = smem_u32(st.WQ), sK = smem_u32(st.K), sP = smem_u32(st.P);
 #pragma unroll
                 for (int kk = 0; kk < DK / 16; ++kk)
-                    tc5::mma_ts(tm + TXY, tm + TAS + 8 * kk, tc5::kmajor<2 * C>(sWQ, kk), ID_XY, kk > 0);
+                    tc5::mma_ts(tm + TXY, tm + TAS + 8 * kk, tc5::kmajor<2 * C>(sWQ, kk),
+                                MODE == 0 ? ID_XY : ID_X, kk > 0);
                 tc5::commit(&s.x_done);
                 if (!mbar_wait(&s.u_ready, n & 1, p.status)) break;
                 tc5::fence_after();
@@ -175,10 +185,12 @@ __global__ void __launch_bounds__(W5_THREADS) tc5_walk_kernel(const __grid_const
                 for (int kk = 0; kk < C / 16; ++kk)
                     tc5::mma_ts(tm + TD, aUs + 8 * kk, tc5::mnmajor(sK, kk, C * 128), ID_D, kk > 0);
                 tc5::commit(&s.d_done);
+                if (MODE == 0) {
 #pragma unroll
-                for (int kk = 0; kk < C / 16; ++kk)
-                    tc5::mma_ts(tm + TZ, tm + TAU + 8 * kk, tc5::kmajor<C>(sP, kk), ID_Z, kk > 0);
-                tc5::commit(&s.o_done);
+                    for (int kk = 0; kk < C / 16; ++kk)
+                        tc5::mma_ts(tm + TZ, tm + TAU + 8 * kk, tc5::kmajor<C>(sP, kk), ID_Z, kk > 0);
+                    tc5::commit(&s.o_done);
+                }
                 tc5::commit(&s.empty[sn]);
             }
             // Leave nothing in flight: every MMA retired.
@@ -208,7 +220,19 @@ __global__ void __launch_bounds__(W5_THREADS) tc5_walk_kernel(const __grid_const
             tc5::st16(trow + TAS + 16 * cg, r);
             tc5::wait_st();
         };
+        // MODE 1: bf16 state entering chunk n, Swz<128> image (64 contiguous bytes)
+        auto store_s0 = [&](int n) {
+            __nv_bfloat16* dst = p.S0out + ((size_t)bh * p.NT + n) * DV * DK;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int c = 32 * cg + 8 * j;
+                *reinterpret_cast<uint4*>(dst + swz<DK>(a, c)) =
+                    make_uint4(pack_bf16(S[c - 32 * cg], S[c - 32 * cg + 1]), pack_bf16(S[c - 32 * cg + 2], S[c - 32 * cg + 3]),
+                               pack_bf16(S[c - 32 * cg + 4], S[c - 32 * cg + 5]), pack_bf16(S[c - 32 * cg + 6], S[c - 32 * cg + 7]));
+            }
+        };
         store_state();
+        if (MODE == 1) store_s0(0);
         tc5::fence_before();
         warp_arrive(&s.s_ready);
 
@@ -238,7 +262,7 @@ __global__ void __launch_bounds__(W5_THREADS) tc5_walk_kernel(const __grid_const
             {
                 float x[16];
                 tc5::ld16(x, trow + TXY + t0);
-                tc5::ld16(y, trow + TXY + C + t0);
+                if (MODE == 0) tc5::ld16(y, trow + TXY + C + t0);
                 tc5::wait_ld();
                 const __nv_bfloat16* ua = reinterpret_cast<const __nv_bfloat16*>(&ut0);
                 const __nv_bfloat16* ub = reinterpret_cast<const __nv_bfloat16*>(&ut1);
@@ -255,9 +279,18 @@ __global__ void __launch_bounds__(W5_THREADS) tc5_walk_kernel(const __grid_const
                 tc5::st8(trow + TAU + 8 * cg, ru);
                 if (!KDA) tc5::st8(trow + TAUS + 8 * cg, rs);
                 tc5::wait_st();
+                tc5::fence_before();
+                warp_arrive(&s.u_ready);
+                if (MODE == 1) {  // U image, token rows (64 contiguous bytes per warp store)
+                    __nv_bfloat16* dst = p.Uout + ((size_t)bh * p.NT + n) * C * DV;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(&ru[j]);
+                        dst[swz<DV>(t0 + 2 * j, a)] = v.x;
+                        dst[swz<DV>(t0 + 2 * j + 1, a)] = v.y;
+                    }
+                }
             }
-            tc5::fence_before();
-            warp_arrive(&s.u_ready);
             if (n + 1 < p.NT) {  // next chunk's U~^T, consumed one step later
                 const __nv_bfloat16* Un = Ut + (size_t)(n + 1) * C * DV;
                 ut0 = *reinterpret_cast<const uint4*>(Un + uo0);
@@ -279,6 +312,11 @@ __global__ void __launch_bounds__(W5_THREADS) tc5_walk_kernel(const __grid_const
             store_state();
             tc5::fence_before();
             warp_arrive(&s.s_ready);
+            if (MODE == 1) {
+                warp_arrive(&s.empty[sn]);
+                if (n + 1 < p.NT) store_s0(n + 1);
+                continue;
+            }
             // ---- O^T = scale e^{G_i} Y + Z, tokens t0 .. t0+15 of row a ---------
             if (!wait_all(&s.o_done, n & 1, p.status)) break;
             tc5::fence_after();
@@ -296,7 +334,7 @@ __global__ void __launch_bounds__(W5_THREADS) tc5_walk_kernel(const __grid_const
             tc5::fence_before();
             warp_arrive(&s.empty[sn]);
         }
-        if (p.hT) {
+        if (MODE == 0 && p.hT) {
             float* hT = p.hT + ((size_t)bh * DV + a) * DK + 32 * cg;
 #pragma unroll
             for (int j = 0; j < 32; j += 4)
@@ -311,11 +349,12 @@ __global__ void __launch_bounds__(W5_THREADS) tc5_walk_kernel(const __grid_const
     }
 }
 
-template <bool KDA>
+template <bool KDA, int MODE>
 void launch_w5(const W5Ptrs& p, cudaStream_t st) {
     const int smem = sizeof(W5Smem) + 1024;
-    cudaFuncSetAttribute(tc5_walk_kernel<KDA>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    GDN_LAUNCH("tc5_walk_fwd", st, (tc5_walk_kernel<KDA><<<p.B * p.H, W5_THREADS, smem, st>>>(p)));
+    cudaFuncSetAttribute(tc5_walk_kernel<KDA, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    GDN_LAUNCH(MODE == 0 ? "tc5_walk_fwd" : "tc5_walk_states", st,
+               (tc5_walk_kernel<KDA, MODE><<<p.B * p.H, W5_THREADS, smem, st>>>(p)));
 }
 
 }  // namespace
@@ -328,8 +367,21 @@ void launch_walk5_fwd(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& c, 
     w.h0 = h0; w.W = c.W; w.Ut = c.Ut; w.P = c.P; w.G = c.G; w.Qg = c.Qg; w.Kt = c.Kt;
     w.o = (__nv_bfloat16*)o; w.hT = hT; w.status = c.status;
     w.B = d.B; w.T = d.T; w.H = d.H; w.NT = L.NT; w.scale = d.scale;
-    if (d.gate == GDN_GATE_CHANNEL) launch_w5<true>(w, st);
-    else launch_w5<false>(w, st);
+    if (d.gate == GDN_GATE_CHANNEL) launch_w5<true, 0>(w, st);
+    else launch_w5<false, 0>(w, st);
+}
+
+void launch_walk5_states(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& c, const float* h0,
+                         void* ws, cudaStream_t st) {
+    W5Ptrs w{};
+    w.qmap = c.qmap; w.kmap = c.kmap;
+    w.h0 = h0; w.W = c.W; w.Ut = c.Ut; w.P = c.P; w.G = c.G; w.Qg = c.Qg; w.Kt = c.Kt;
+    w.S0out = (__nv_bfloat16*)((char*)ws + L.S0);
+    w.Uout = (__nv_bfloat16*)((char*)ws + L.U);
+    w.status = c.status;
+    w.B = d.B; w.T = d.T; w.H = d.H; w.NT = L.NT; w.scale = d.scale;
+    if (d.gate == GDN_GATE_CHANNEL) launch_w5<true, 1>(w, st);
+    else launch_w5<false, 1>(w, st);
 }
 }  // namespace tc
 }  // namespace gdn

@@ -32,6 +32,8 @@ namespace tc {
 void launch_prep_kda(const ChunkPtrs& p, size_t nchunks, cudaStream_t st);
 void launch_walk5_fwd(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& c, const float* h0,
                       void* o, float* hT, cudaStream_t st);
+void launch_walk5_states(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& c, const float* h0,
+                         void* ws, cudaStream_t st);
 }
 namespace {
 using namespace tc;
@@ -569,6 +571,14 @@ WalkPtrs make_walk_ptrs(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& c
     return w;
 }
 
+// The tcgen05 walk carries a whole head per CTA; with few heads the 16-row
+// walk, which spreads each head over eight CTAs, fills more SMs.
+bool whole_head_walk(const gdn_dims& d) {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    return (long long)d.B * d.H * 4 >= sms;
+}
+
 }  // namespace
 
 namespace tc {
@@ -585,6 +595,10 @@ bool chunk_ptrs(ChunkPtrs& p, const gdn_dims& d, const TcLayout& L, const void* 
 
 void launch_walk_states(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& cp,
                         const float* h0, void* ws, cudaStream_t st) {
+    if (whole_head_walk(d)) {
+        launch_walk5_states(d, L, cp, h0, ws, st);
+        return;
+    }
     WalkPtrs w = make_walk_ptrs(d, L, cp, h0);
     w.S0out = (__nv_bfloat16*)((char*)ws + L.S0);
     w.Uout = (__nv_bfloat16*)((char*)ws + L.U);
@@ -609,11 +623,7 @@ bool launch_tc_fwd(const gdn_dims& d, const void* q, const void* k, const void* 
     const bool kda = d.gate == GDN_GATE_CHANNEL;
     if (kda) launch_prep_kda(cp, L.nchunks, st);
     else launch_prep(cp, L.nchunks, st);
-    // The tcgen05 walk carries a whole head per CTA; with few heads the
-    // 16-row walk, which spreads each head over eight CTAs, fills more SMs.
-    int dev = 0, sms = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if ((long long)d.B * d.H * 4 >= sms) {
+    if (whole_head_walk(d)) {
         launch_walk5_fwd(d, L, cp, h0, o, hT, st);
     } else {
         WalkPtrs w = make_walk_ptrs(d, L, cp, h0);

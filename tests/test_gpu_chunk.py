@@ -97,10 +97,12 @@ def test_zero_gate_small_beta(dev):
     (KDA, dict(B=3, H=16, T=64, g_shift=-6.0, h0_std=0.2)),               # slow gate: the state dominates
 ])
 def test_whole_head_walk(dev, cfg, over):
-    """Enough heads for the forward to carry one whole head per CTA on the
-    fifth-generation tensor cores (state in registers, operands in TMEM)."""
+    """Enough heads for the forward, and the backward's state recompute, to
+    carry one whole head per CTA on the fifth-generation tensor cores (state
+    in registers, operands in TMEM)."""
     inp = make_chunk_inputs(cfg, **over)
     check_fwd(inp, dev)
+    check_bwd(inp, dev)
 
 
 # ---- invariants -----------------------------------------------------------
