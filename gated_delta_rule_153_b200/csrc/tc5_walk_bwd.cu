@@ -1,0 +1,335 @@
+// tc5_walk_bwd.cu -- the backward's reverse chunk chain on the fifth-generation
+// tensor cores.
+//
+// Reverse mode through the chunk chain of the forward (tc5_walk.cu): with dS
+// the gradient of the state leaving chunk n and dO the output gradient of
+// its tokens,
+//   dU^T = dO^T P + (dS K^T) .* e^{G_last - G_i}          (value rows x tokens)
+//   dS0  = e^{G_last} dS + dO^T (scale e^G .* Q) - dU^T W  (the state entering n)
+// One CTA walks one head's 128 value rows of dS backwards through the chunks:
+//   F = dO^T P  (128 x 64)     E = dS K^T   (128 x 64)        [A: dO tile, dS]
+//   T = dO^T Q^ - dU^T W (128 x 128, one accumulator; the second product
+//       enters with its A operand negated)                    [A: dO tile, dU]
+// dS stays fp32 in the epilogue threads' registers; its bf16 copy and dU are
+// written straight into tensor memory as A operands.  The dO tile is read
+// as an MN-major A operand from shared memory; Q is scaled in place to
+// Q^ = scale e^{G_i} Q (rows past the sequence end zeroed) before T.
+// Each chunk's dS (bf16, Swz<128>) and dU (Swz<128>, token rows) are stored
+// for the local-gradient kernel; dh0 is the dS left after chunk 0.
+//
+// Warp roles as in tc5_walk.cu: 16 epilogue warps (TMEM lane quarter =
+// warp % 4, column group = warp / 4), one MMA warp, one load warp with a
+// three-stage ring.  Chain per step: E -> dU -> T -> dS update -> next E;
+// F and the first half of T depend only on the chunk's tiles.
+//
+// Channel gate: Q and K arrive as prepared images (scale Q .* e^G and
+// K .* e^{G_last - G}), G holds e^{G_last,c}, no per-token factors apply, and
+// the decay of dS is per key column.
+#include "async.cuh"
+#include "common.cuh"
+#include "internal.h"
+#include "mma.cuh"
+#include "tc5.cuh"
+#include "tc_common.cuh"
+
+namespace gdn {
+namespace {
+using namespace tc;
+
+constexpr int RB_EPI_WARPS = 16;
+constexpr int RB_THREADS = 32 * (RB_EPI_WARPS + 2);
+constexpr int RB_CTRL = RB_EPI_WARPS;
+constexpr int RB_PROD = RB_EPI_WARPS + 1;
+constexpr int RB_STAGES = 3;
+// tensor-memory columns: accumulators E, F, T; A operands dS (bf16 pairs), dU
+constexpr int TE = 0, TF = 64, TT = 128, TADS = 256, TADU = 320, RCOLS = 512;
+constexpr uint32_t ID_E = tc5::idesc_bf16(128, 64, false, false);
+constexpr uint32_t ID_F = tc5::idesc_bf16(128, 64, true, true);
+constexpr uint32_t ID_Y = tc5::idesc_bf16(128, 128, true, true);
+constexpr uint32_t ID_Z = tc5::idesc_bf16(128, 128, false, true) | (1u << 13);  // A negated
+
+struct alignas(1024) RbStage {
+    __nv_bfloat16 Q[C * DK];   // Tma128 [token][key]; scaled in place (B of T, MN-major)
+    __nv_bfloat16 K[C * DK];   // Tma128 [token][key]: K-major B of E
+    __nv_bfloat16 W[C * DK];   // Tma128 [token][key]: MN-major B of T
+    __nv_bfloat16 dO[C * DV];  // Tma128 [token][value]: MN-major A of F and T
+    __nv_bfloat16 P[C * C];    // Swz<64> [j][i]: MN-major B of F
+    float G[DK];               // G (scalar gate, C used) or e^{G_last,c}
+};
+
+struct RbSmem {
+    RbStage st[RB_STAGES];
+    uint64_t full[RB_STAGES], empty[RB_STAGES];
+    uint64_t ds_ready, q_ready, du_ready, e_done, t_done, fin;
+    uint32_t tmem;
+};
+
+struct RbPtrs {
+    CUtensorMap qmap, kmap, dOmap;
+    const float* dhT;
+    const __nv_bfloat16 *W, *P, *Qg, *Kt;
+    const float* G;
+    __nv_bfloat16 *dSout, *dUout;
+    float* dh0;
+    unsigned int* status;
+    int B, T, H, NT;
+    float scale;
+};
+
+template <bool KDA>
+__device__ void rb_issue(RbStage& st, uint64_t* bar, const RbPtrs& p, int b, int h, int bh, int n) {
+    const size_t cid = (size_t)bh * p.NT + n;
+    constexpr int GW = KDA ? DK : C;
+    mbar_arrive_expect(bar, (4 * C * DK + C * C) * 2 + GW * 4);
+    const int tok = b * p.T + n * C;
+    if (KDA) {
+        bulk_g2s(st.Q, p.Qg + cid * C * DK, C * DK * 2, bar);
+        bulk_g2s(st.K, p.Kt + cid * C * DK, C * DK * 2, bar);
+    } else {
+        tma_load_tile(st.Q, &p.qmap, h, tok, bar);
+        tma_load_tile(st.K, &p.kmap, h, tok, bar);
+    }
+    tma_load_tile(st.dO, &p.dOmap, h, tok, bar);
+    bulk_g2s(st.W, p.W + cid * C * DK, C * DK * 2, bar);
+    bulk_g2s(st.P, p.P + cid * C * C, C * C * 2, bar);
+    bulk_g2s(st.G, p.G + cid * GW, GW * 4, bar);
+}
+
+GDN_DEV bool rb_wait_all(uint64_t* bar, uint32_t parity, unsigned int* status) {
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, status));
+}
+
+GDN_DEV void rb_warp_arrive(uint64_t* bar) {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
+
+template <bool KDA>
+__global__ void __launch_bounds__(RB_THREADS) tc5_walk_bwd_kernel(const __grid_constant__ RbPtrs p) {
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    RbSmem& s = *reinterpret_cast<RbSmem*>(align1k(smem_raw));
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int bh = blockIdx.x, b = bh / p.H, h = bh % p.H;
+
+    if (tid == 0) {
+        for (int i = 0; i < RB_STAGES; ++i) {
+            mbar_init(&s.full[i], 1);
+            mbar_init(&s.empty[i], 1 + RB_EPI_WARPS);
+        }
+        mbar_init(&s.ds_ready, RB_EPI_WARPS);
+        mbar_init(&s.q_ready, RB_EPI_WARPS);
+        mbar_init(&s.du_ready, RB_EPI_WARPS);
+        mbar_init(&s.e_done, 1);
+        mbar_init(&s.t_done, 1);
+        mbar_init(&s.fin, 1);
+        fence_mbar_init();
+    }
+    if (warp == RB_CTRL) tc5::alloc(&s.tmem, RCOLS);
+    tc5::fence_before();
+    __syncthreads();
+    tc5::fence_after();
+    const uint32_t tm = s.tmem;
+
+    if (warp == RB_PROD) {
+        if (lane == 0) {
+            int issued = 0;
+            for (int k = 0; k < p.NT; ++k) {  // step k carries chunk NT-1-k
+                const int sk = k % RB_STAGES;
+                if (k >= RB_STAGES && !mbar_wait(&s.empty[sk], ((k / RB_STAGES) - 1) & 1, p.status)) break;
+                rb_issue<KDA>(s.st[sk], &s.full[sk], p, b, h, bh, p.NT - 1 - k);
+                issued = k + 1;
+            }
+            for (int k = max(0, issued - RB_STAGES); k < issued; ++k)
+                mbar_wait(&s.full[k % RB_STAGES], (k / RB_STAGES) & 1, p.status);
+        }
+        __syncwarp();
+    } else if (warp == RB_CTRL) {
+        if (lane == 0) {
+            for (int k = 0; k < p.NT; ++k) {
+                const int sk = k % RB_STAGES;
+                RbStage& st = s.st[sk];
+                if (!mbar_wait(&s.full[sk], (k / RB_STAGES) & 1, p.status)) break;
+                const uint32_t sQ = smem_u32(st.Q), sK = smem_u32(st.K), sW = smem_u32(st.W),
+                               sdO = smem_u32(st.dO), sP = smem_u32(st.P);
+#pragma unroll
+                for (int kk = 0; kk < C / 16; ++kk)  // F = dO^T P
+                    tc5::mma(tm + TF, tc5::mnmajor(sdO, kk, C * 128), tc5::mnmajor(sP, kk, C * 128), ID_F,
+                             kk > 0);
+                if (!mbar_wait(&s.ds_ready, k & 1, p.status)) break;
+                tc5::fence_after();
+#pragma unroll
+                for (int kk = 0; kk < DK / 16; ++kk)  // E = dS K^T
+                    tc5::mma_ts(tm + TE, tm + TADS + 8 * kk, tc5::kmajor<C>(sK, kk), ID_E, kk > 0);
+                tc5::commit(&s.e_done);
+                if (!mbar_wait(&s.q_ready, k & 1, p.status)) break;
+                tc5::fence_after();
+#pragma unroll
+                for (int kk = 0; kk < C / 16; ++kk)  // T = dO^T Q^
+                    tc5::mma(tm + TT, tc5::mnmajor(sdO, kk, C * 128), tc5::mnmajor(sQ, kk, C * 128), ID_Y,
+                             kk > 0);
+                if (!mbar_wait(&s.du_ready, k & 1, p.status)) break;
+                tc5::fence_after();
+#pragma unroll
+                for (int kk = 0; kk < C / 16; ++kk)  // T -= dU^T W
+                    tc5::mma_ts(tm + TT, tm + TADU + 8 * kk, tc5::mnmajor(sW, kk, C * 128), ID_Z, true);
+                tc5::commit(&s.t_done);
+                tc5::commit(&s.empty[sk]);
+            }
+            tc5::commit(&s.fin);
+            mbar_wait(&s.fin, 0, p.status);
+        }
+        __syncwarp();
+    } else {
+        // ---- epilogue: thread = value row a; key columns 32*cg .. +31 of dS,
+        // tokens 16*cg .. +15 of dU -------------------------------------------
+        const int q = warp & 3, cg = warp >> 2, a = 32 * q + lane;
+        const uint32_t trow = tm + ((uint32_t)(32 * q) << 16);
+        const int t0 = 16 * cg;
+        float dS[32];
+        {
+            const float* src = p.dhT ? p.dhT + ((size_t)bh * DV + a) * DK + 32 * cg : nullptr;
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) {
+                const float4 v = src ? *reinterpret_cast<const float4*>(src + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+                dS[j] = v.x; dS[j + 1] = v.y; dS[j + 2] = v.z; dS[j + 3] = v.w;
+            }
+        }
+        auto store_ds_tmem = [&]() {
+            uint32_t r[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) r[j] = pack_bf16(dS[2 * j], dS[2 * j + 1]);
+            tc5::st16(trow + TADS + 16 * cg, r);
+            tc5::wait_st();
+        };
+        store_ds_tmem();
+        tc5::fence_before();
+        rb_warp_arrive(&s.ds_ready);
+
+        for (int k = 0; k < p.NT; ++k) {
+            const int n = p.NT - 1 - k, sk = k % RB_STAGES;
+            RbStage& st = s.st[sk];
+            const int L = min(C, p.T - n * C);
+            const size_t cid = (size_t)bh * p.NT + n;
+            if (!rb_wait_all(&s.full[sk], (k / RB_STAGES) & 1, p.status)) break;
+            {   // dS leaving chunk n: bf16 Swz<128> image, 64 contiguous bytes
+                __nv_bfloat16* dst = p.dSout + cid * DV * DK;
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    *reinterpret_cast<uint4*>(dst + swz<DK>(a, 32 * cg + 8 * j)) =
+                        make_uint4(pack_bf16(dS[8 * j], dS[8 * j + 1]), pack_bf16(dS[8 * j + 2], dS[8 * j + 3]),
+                                   pack_bf16(dS[8 * j + 4], dS[8 * j + 5]), pack_bf16(dS[8 * j + 6], dS[8 * j + 7]));
+            }
+            // Q^ = scale e^{G_i} Q in place, rows past the sequence end zeroed
+            if (!KDA || L < C) {
+#pragma unroll
+                for (int rep = 0; rep < 2; ++rep) {
+                    const int ci = tid + 32 * RB_EPI_WARPS * rep;  // 16-byte piece of the tile
+                    const int i = (ci & 511) >> 3;
+                    const float f = i < L ? (KDA ? 1.f : p.scale * __expf(st.G[i])) : 0.f;
+                    uint4* ptr = reinterpret_cast<uint4*>(st.Q) + ci;
+                    uint4 v = *ptr;
+                    __nv_bfloat162* e2 = reinterpret_cast<__nv_bfloat162*>(&v);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const float2 x = __bfloat1622float2(e2[j]);
+                        e2[j] = __floats2bfloat162_rn(x.x * f, x.y * f);
+                    }
+                    *ptr = v;
+                }
+            }
+            tc5::fence_proxy_async();
+            rb_warp_arrive(&s.q_ready);
+            // ---- dU = F + E .* e^{G_last - G_i}, zero past the sequence end ----
+            float et = 1.f, gam = 1.f;
+            if (!KDA) {
+                const float gl = st.G[C - 1];
+                et = __expf(gl - st.G[t0 + (lane & 15)]);
+                gam = __expf(gl);
+            }
+            if (!rb_wait_all(&s.e_done, k & 1, p.status)) break;
+            tc5::fence_after();
+            {
+                float e[16], f[16];
+                tc5::ld16(e, trow + TE + t0);
+                tc5::ld16(f, trow + TF + t0);
+                tc5::wait_ld();
+                uint32_t ru[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const float e0 = KDA ? 1.f : __shfl_sync(0xffffffffu, et, 2 * j);
+                    const float e1 = KDA ? 1.f : __shfl_sync(0xffffffffu, et, 2 * j + 1);
+                    const float u0 = t0 + 2 * j < L ? fmaf(e[2 * j], e0, f[2 * j]) : 0.f;
+                    const float u1 = t0 + 2 * j + 1 < L ? fmaf(e[2 * j + 1], e1, f[2 * j + 1]) : 0.f;
+                    ru[j] = pack_bf16(u0, u1);
+                }
+                tc5::st8(trow + TADU + 8 * cg, ru);
+                tc5::wait_st();
+                tc5::fence_before();
+                rb_warp_arrive(&s.du_ready);
+                __nv_bfloat16* dst = p.dUout + cid * C * DV;  // dU image, token rows
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(&ru[j]);
+                    dst[swz<DV>(t0 + 2 * j, a)] = v.x;
+                    dst[swz<DV>(t0 + 2 * j + 1, a)] = v.y;
+                }
+            }
+            // ---- dS0 = gamma dS + T ---------------------------------------------
+            if (!rb_wait_all(&s.t_done, k & 1, p.status)) break;
+            tc5::fence_after();
+            {
+                float t[32];
+                tc5::ld32(t, trow + TT + 32 * cg);
+                tc5::wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const float gj = KDA ? st.G[32 * cg + j] : gam;
+                    dS[j] = fmaf(gj, dS[j], t[j]);
+                }
+            }
+            store_ds_tmem();
+            tc5::fence_before();
+            rb_warp_arrive(&s.ds_ready);
+            rb_warp_arrive(&s.empty[sk]);
+        }
+        if (p.dh0) {
+            float* dst = p.dh0 + ((size_t)bh * DV + a) * DK + 32 * cg;
+#pragma unroll
+            for (int j = 0; j < 32; j += 4)
+                *reinterpret_cast<float4*>(dst + j) = make_float4(dS[j], dS[j + 1], dS[j + 2], dS[j + 3]);
+        }
+    }
+    tc5::fence_before();
+    __syncthreads();
+    if (warp == RB_CTRL) {
+        tc5::fence_after();
+        tc5::dealloc(tm, RCOLS);
+    }
+}
+
+template <bool KDA>
+void launch_rb(const RbPtrs& p, cudaStream_t st) {
+    const int smem = sizeof(RbSmem) + 1024;
+    cudaFuncSetAttribute(tc5_walk_bwd_kernel<KDA>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    GDN_LAUNCH("tc5_walk_bwd", st, (tc5_walk_bwd_kernel<KDA><<<p.B * p.H, RB_THREADS, smem, st>>>(p)));
+}
+
+}  // namespace
+
+namespace tc {
+bool launch_walk5_bwd(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& c, const void* dO,
+                      const float* dhT, float* dh0, void* ws, cudaStream_t st) {
+    RbPtrs p{};
+    p.qmap = c.qmap; p.kmap = c.kmap;
+    if (!encode_token_map(&p.dOmap, dO, d.B, d.T, d.H)) return false;
+    p.dhT = dhT; p.W = c.W; p.P = c.P; p.Qg = c.Qg; p.Kt = c.Kt; p.G = c.G;
+    p.dSout = (__nv_bfloat16*)((char*)ws + L.dS);
+    p.dUout = (__nv_bfloat16*)((char*)ws + L.dU);
+    p.dh0 = dh0; p.status = c.status;
+    p.B = d.B; p.T = d.T; p.H = d.H; p.NT = L.NT; p.scale = d.scale;
+    if (d.gate == GDN_GATE_CHANNEL) launch_rb<true>(p, st);
+    else launch_rb<false>(p, st);
+    return true;
+}
+}  // namespace tc
+}  // namespace gdn

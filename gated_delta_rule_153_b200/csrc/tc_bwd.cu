@@ -35,6 +35,9 @@ void launch_prep_kda(const ChunkPtrs& p, size_t nchunks, cudaStream_t st);
 bool launch_bwd_local_kda(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& cp,
                           const void* dO, void* dq, void* dk, void* dv, float* dg, float* dbeta,
                           void* ws, cudaStream_t st);
+bool whole_head_walk(const gdn_dims& d);
+bool launch_walk5_bwd(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& c, const void* dO,
+                      const float* dhT, float* dh0, void* ws, cudaStream_t st);
 }  // namespace tc
 
 namespace {
@@ -807,6 +810,30 @@ void launch_walk_bwd(const BwPtrs& bp, cudaStream_t st) {
                                               st>>>(bp)));
 }
 
+// The 16-row reverse walk (few heads): bp carries the dS / dU outputs.
+bool launch_walk_bwd16(const gdn_dims& d, const ChunkPtrs& cp, const void* dO, const float* dhT,
+                       float* dh0, BwPtrs& bp, cudaStream_t st) {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const bool two = (long long)d.B * d.H * (DV / 32) >= sms;  // two m-tiles per warp
+    bp.qmap = cp.qmap; bp.kmap = cp.kmap;
+    if (!encode_token_map(&bp.dOmap, dO, d.B, d.T, d.H, two ? 32 : 16)) return false;
+    bp.dhT = dhT; bp.W = cp.W; bp.P = cp.P; bp.G = cp.G;
+    bp.dh0 = dh0; bp.status = cp.status;
+    bp.B = d.B; bp.T = d.T; bp.H = d.H; bp.NT = cp.NT; bp.scale = d.scale;
+    bp.Qg = cp.Qg; bp.Kt = cp.Kt;
+    const bool kda = d.gate == GDN_GATE_CHANNEL;
+    if (two) {
+        if (kda) launch_walk_bwd<2, true>(bp, st);
+        else launch_walk_bwd<2, false>(bp, st);
+    } else {
+        if (kda) launch_walk_bwd<1, true>(bp, st);
+        else launch_walk_bwd<1, false>(bp, st);
+    }
+    return true;
+}
+
 }  // namespace
 
 bool tc_bwd_supported(const gdn_dims& d) { return tc_supported(d); }
@@ -826,25 +853,12 @@ bool launch_tc_bwd(const gdn_dims& d, const void* q, const void* k, const void* 
     launch_walk_states(d, L, cp, h0, ws, st);
 
     BwPtrs bp{};
-    int dev = 0, sms = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess)
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const bool two = (long long)d.B * d.H * (DV / 32) >= sms;  // two m-tiles per warp
-    bp.qmap = cp.qmap; bp.kmap = cp.kmap;
-    if (!encode_token_map(&bp.dOmap, dO, d.B, d.T, d.H, two ? 32 : 16)) return false;
-    bp.dhT = dhT; bp.W = cp.W; bp.P = cp.P; bp.G = cp.G;
     bp.dSout = (__nv_bfloat16*)(base + L.dS);
     bp.dUout = (__nv_bfloat16*)(base + L.dU);
-    bp.dh0 = dh0; bp.status = cp.status;
-    bp.B = d.B; bp.T = d.T; bp.H = d.H; bp.NT = L.NT; bp.scale = d.scale;
-    bp.Qg = cp.Qg; bp.Kt = cp.Kt;
-    const bool kda = d.gate == GDN_GATE_CHANNEL;
-    if (two) {
-        if (kda) launch_walk_bwd<2, true>(bp, st);
-        else launch_walk_bwd<2, false>(bp, st);
-    } else {
-        if (kda) launch_walk_bwd<1, true>(bp, st);
-        else launch_walk_bwd<1, false>(bp, st);
+    if (whole_head_walk(d)) {
+        if (!launch_walk5_bwd(d, L, cp, dO, dhT, dh0, ws, st)) return false;
+    } else if (!launch_walk_bwd16(d, cp, dO, dhT, dh0, bp, st)) {
+        return false;
     }
     if (kda_gate)
         return launch_bwd_local_kda(d, L, cp, dO, dq, dk, dv, dg, dbeta, ws, st);

@@ -571,17 +571,17 @@ WalkPtrs make_walk_ptrs(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& c
     return w;
 }
 
-// The tcgen05 walk carries a whole head per CTA; with few heads the 16-row
-// walk, which spreads each head over eight CTAs, fills more SMs.
+}  // namespace
+
+namespace tc {
+// The tcgen05 walks carry a whole head per CTA; with few heads the 16-row
+// walks, which spread each head over eight CTAs, fill more SMs.
 bool whole_head_walk(const gdn_dims& d) {
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     return (long long)d.B * d.H * 4 >= sms;
 }
 
-}  // namespace
-
-namespace tc {
 void launch_prep(const ChunkPtrs& p, size_t nchunks, cudaStream_t st) {
     const int smem = sizeof(PrepSmem) + 1024;
     cudaFuncSetAttribute(tc_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -623,7 +623,7 @@ bool launch_tc_fwd(const gdn_dims& d, const void* q, const void* k, const void* 
     const bool kda = d.gate == GDN_GATE_CHANNEL;
     if (kda) launch_prep_kda(cp, L.nchunks, st);
     else launch_prep(cp, L.nchunks, st);
-    if (whole_head_walk(d)) {
+    if (tc::whole_head_walk(d)) {
         launch_walk5_fwd(d, L, cp, h0, o, hT, st);
     } else {
         WalkPtrs w = make_walk_ptrs(d, L, cp, h0);
