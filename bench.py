@@ -217,6 +217,27 @@ def workspaces(gdn, d):
     return wf, wb
 
 
+def replica_seed(base, rank):
+    """Seed of rank `rank`'s replica: every rank runs its own batch."""
+    return base + 7919 * rank
+
+
+def whole_job_rate(units_per_rank, world, steps, ms_max):
+    """Units per second of the whole job: all ranks' units over the slowest
+    rank's time (weak scaling: each rank holds the full per-GPU workload)."""
+    return world * units_per_rank * steps / (ms_max / 1e3)
+
+
+def rank_reducers(dist, device):
+    """(barrier, max_over_ranks) over the default process group; `device`
+    holds the reduction tensor (cuda under NCCL, cpu under gloo)."""
+    def max_over_ranks(x):
+        t = torch.tensor([x], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+    return (lambda: dist.barrier()), max_over_ranks
+
+
 def run_ours(args, rank, world, dev, barrier, max_over_ranks):
     import gated_delta_rule_153_b200 as gdn
     from gated_delta_rule_153_b200.inputs import DECODE, KDA, L350M, LONG, \
@@ -224,7 +245,7 @@ def run_ours(args, rank, world, dev, barrier, max_over_ranks):
 
     pk = peaks()
     cfg = L350M
-    inp = make_chunk_inputs(cfg, seed=cfg.seed + 7919 * rank)
+    inp = make_chunk_inputs(cfg, seed=replica_seed(cfg.seed, rank))
     d = to_dev(inp, dev)
     outs = dict(o=torch.empty_like(d["v"]),
                 hT=torch.empty(cfg.B, cfg.H, cfg.dv, cfg.dk, device=dev))
@@ -254,7 +275,7 @@ def run_ours(args, rank, world, dev, barrier, max_over_ranks):
     ms_total = max_over_ranks(ms_total)
     ms_step = ms_total / args.steps
     tokens = cfg.B * cfg.T
-    value = world * tokens * args.steps / (ms_total / 1e3)
+    value = whole_job_rate(tokens, world, args.steps, ms_total)
     th = cfg.B * cfg.T * cfg.H
     flops_step = (FWD_FLOP + BWD_FLOP) * th
     tflops = world * flops_step * args.steps / (ms_total / 1e3) / 1e12
@@ -423,12 +444,7 @@ def main():
         torch.cuda.set_device(local)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
-        barrier = lambda: dist.barrier()
-
-        def max_over_ranks(x):
-            t = torch.tensor([x], dtype=torch.float64, device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            return float(t.item())
+        barrier, max_over_ranks = rank_reducers(dist, torch.device("cuda", local))
     else:
         barrier = lambda: None
         max_over_ranks = lambda x: x

@@ -167,3 +167,15 @@ def test_kda_tensor_core(dev, over):
     inp = make_chunk_inputs(KDA, **over)
     check_fwd(inp, dev)
     check_bwd(inp, dev)
+
+
+def test_status_word_reports_and_clears(dev):
+    """A bounded wait that runs out sets the workspace's status word; the
+    query reports it once and clears it (the word is preset here: no kernel
+    is made to time out)."""
+    import gated_delta_rule_153_b200 as gdn
+    ws = torch.zeros(256, dtype=torch.uint8, device=dev)
+    assert gdn.gdn_query_device_status(ws) == gdn.GDN_OK
+    ws[0] = 1
+    assert gdn.gdn_query_device_status(ws) == gdn.GDN_ERR_DEVICE_TIMEOUT
+    assert gdn.gdn_query_device_status(ws) == gdn.GDN_OK
