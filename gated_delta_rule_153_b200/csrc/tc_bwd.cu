@@ -314,6 +314,7 @@ struct LocPtrs {
     unsigned int* status;
     int B, T, H, NT;
     float scale;
+    int pf_stride;  // chunks a wave ahead; 0: no prefetch
 };
 
 // Row sums over the 4 lanes of a quad: lo -> row r_lo, hi -> row r_lo + 8.
@@ -364,6 +365,21 @@ __global__ void __launch_bounds__(LOC_THREADS) tc_bwd_local_kernel(const __grid_
         mbar_arrive_expect(&s.bar[1], (C * DK + C * C) * 2);
         tma_load_tile(s.V, &p.vmap, h, tok, &s.bar[1]);
         bulk_g2s(s.Tb, p.Tb + (size_t)cid * C * C, C * C * 2, &s.bar[1]);
+        // the chunk a wave ahead: its tiles and images wait in L2 when its CTA starts
+        const int pc = cid + p.pf_stride;
+        if (p.pf_stride > 0 && pc < (int)gridDim.x) {
+            const int pbh = pc / p.NT, pn = pc % p.NT;
+            const int ptok = (pbh / p.H) * p.T + pn * C, ph = pbh % p.H;
+            tma_prefetch_tile(&p.dOmap, ph, ptok);
+            tma_prefetch_tile(&p.qmap, ph, ptok);
+            tma_prefetch_tile(&p.kmap, ph, ptok);
+            tma_prefetch_tile(&p.vmap, ph, ptok);
+            bulk_prefetch_l2(p.U + (size_t)pc * C * DV, C * DV * 2);
+            bulk_prefetch_l2(p.dU + (size_t)pc * C * DV, C * DV * 2);
+            bulk_prefetch_l2(p.S0 + (size_t)pc * DV * DK, DV * DK * 2);
+            bulk_prefetch_l2(p.dS + (size_t)pc * DV * DK, DV * DK * 2);
+            bulk_prefetch_l2(p.Tb + (size_t)pc * C * C, C * C * 2);
+        }
     }
     for (int e = tid; e < C; e += LOC_THREADS) s.beta[e] = e < L ? p.beta[row0 + e * rs] : 0.f;
     for (int e = tid; e < LOC_WARPS * C; e += LOC_THREADS) {
@@ -876,6 +892,9 @@ bool launch_tc_bwd(const gdn_dims& d, const void* q, const void* k, const void* 
     {
         const int smem = sizeof(LocSmem) + 1024;
         cudaFuncSetAttribute(tc_bwd_local_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        int dev = 0, sms = 148;
+        if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        lp.pf_stride = sms;  // one CTA per SM
         GDN_LAUNCH("tc_bwd_local", st,
                    tc_bwd_local_kernel<<<(unsigned)L.nchunks, LOC_THREADS, smem, st>>>(lp));
     }

@@ -39,6 +39,20 @@ GDN_DEV void tma_load_tile(__nv_bfloat16* tile, const CUtensorMap* map, int head
     tma_load_3d(tile + 64 * 64, map, 64, head, token, bar);
 }
 
+// Hint: pull box (x, y, z) of the map's tensor into L2 ahead of a load.
+GDN_DEV void tma_prefetch_3d(const CUtensorMap* map, int x, int y, int z) {
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global [%0, {%1, %2, %3}];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(x), "r"(y), "r"(z)
+                 : "memory");
+}
+
+// Both 64-channel halves of rows token .. token+63 of head `head`.
+GDN_DEV void tma_prefetch_tile(const CUtensorMap* map, int head, int token) {
+    tma_prefetch_3d(map, 0, head, token);
+    tma_prefetch_3d(map, 64, head, token);
+}
+
 // Host: encode the token map of a [B, T, H, 128] bf16 tensor.  box_cols 64
 // gives 128-byte-swizzled 64x64 boxes (Tma128 tiles); box_cols 16 gives
 // unswizzled 64-row x 16-column boxes (32-byte rows).  Returns false

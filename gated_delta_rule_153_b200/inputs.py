@@ -43,6 +43,8 @@ class ChunkConfig:
     backward: bool = True
     dhT_std: Optional[float] = None
     seed: int = 1000
+    beta_max: float = 1.0        # beta = beta_max * sigmoid(N(0,1)); 2 allows I - beta k k^T
+                                 # a negative eigenvalue along k
 
 
 @dataclass(frozen=True)
@@ -58,6 +60,7 @@ class DecodeConfig:
     g_shift: float = 0.0
     state_std: float = 0.02
     seed: int = 1003
+    beta_max: float = 1.0
 
 
 # The five workloads.  Index 0 is the small case the oracle finishes in a
@@ -101,7 +104,7 @@ def make_chunk_inputs(cfg: ChunkConfig, **over) -> dict:
     gshape = (B, T, H, dk) if cfg.gate == "channel" else (B, T, H)
     g = -torch.nn.functional.softplus(
         torch.randn(*gshape, generator=_gen(s, 3)) + cfg.g_shift)
-    beta = torch.sigmoid(torch.randn(B, T, H, generator=_gen(s, 4)))
+    beta = cfg.beta_max * torch.sigmoid(torch.randn(B, T, H, generator=_gen(s, 4)))
     h0 = None
     if cfg.h0_std is not None:
         h0 = torch.randn(B, H, dv, dk, generator=_gen(s, 5)) * cfg.h0_std
@@ -139,7 +142,7 @@ def make_decode_inputs(cfg: DecodeConfig, steps: Optional[int] = None, **over) -
         v[t0:t0 + n] = torch.randn(n, N, H, dv, generator=gens[2]).to(dt)
         g[t0:t0 + n] = -torch.nn.functional.softplus(
             torch.randn(n, *gshape, generator=gens[3]) + cfg.g_shift)
-        beta[t0:t0 + n] = torch.sigmoid(torch.randn(n, N, H, generator=gens[4]))
+        beta[t0:t0 + n] = cfg.beta_max * torch.sigmoid(torch.randn(n, N, H, generator=gens[4]))
     state0 = torch.randn(N, H, dv, dk, generator=gens[5]) * cfg.state_std
     return dict(q=q, k=k, v=v, g=g.contiguous(), beta=beta.contiguous(),
                 state0=state0, cfg=cfg)

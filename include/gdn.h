@@ -44,7 +44,11 @@
  *                        null workspace when that size is non-zero;
  *   GDN_ERR_CUDA         a launch failed (cudaGetLastError after launch).
  * Value preconditions are documented, not checked: g finite and <= 0,
- * beta in [0, 1] (the range the chunkwise algebra is tested on).
+ * beta in [0, 2].  beta in (1, 2] is the negative-eigenvalue transition that
+ * "Gated Delta Networks: Improving Mamba2 with Delta Rule" (paper review),
+ * section "Future work", names as an extension: I - beta k k^T then flips the
+ * sign along a unit k (a reflection at beta = 2).  The arithmetic is the same;
+ * both ranges are tested.
  */
 #ifndef GDN_H
 #define GDN_H

@@ -10,7 +10,9 @@ Page citations: "Gated Delta Networks: Improving Mamba2 with Delta Rule"
 (paper review) -- section "Method" (the recurrence; the delta rule as one
 test-time SGD step with learning rate b_t and the gate as a weight decay),
 section "Key idea" (a_t -> 0 erases, a_t -> 1 is the pure delta rule),
-section "Background" (the state as an associative key->value memory).
+section "Background" (the state as an associative key->value memory),
+section "Future work" (negative-eigenvalue transitions: b in (0, 2), so that
+I - b k k^T may flip the sign along k).
 """
 from __future__ import annotations
 
@@ -31,13 +33,13 @@ def _unit(rng, shape):
     return x / np.linalg.norm(x, axis=-1, keepdims=True)
 
 
-def _inputs(rng, B=1, T=6, H=1, dk=4, dv=3, channel=False, g_shift=0.0):
+def _inputs(rng, B=1, T=6, H=1, dk=4, dv=3, channel=False, g_shift=0.0, beta_max=1.0):
     q = _unit(rng, (B, T, H, dk))
     k = _unit(rng, (B, T, H, dk))
     v = rng.standard_normal((B, T, H, dv))
     gshape = (B, T, H, dk) if channel else (B, T, H)
     g = -np.log1p(np.exp(rng.standard_normal(gshape) + g_shift))
-    beta = 1.0 / (1.0 + np.exp(-rng.standard_normal((B, T, H))))
+    beta = beta_max / (1.0 + np.exp(-rng.standard_normal((B, T, H))))
     h0 = 0.5 * rng.standard_normal((B, H, dv, dk))
     return q, k, v, g, beta, h0
 
@@ -143,8 +145,8 @@ def pin_erase_limit(lib=None):
 
 
 def pin_contraction(lib=None):
-    """Unit keys, b in (0,1), a <= 1, v = 0: every step is a contraction, so
-    ||S_t||_F never grows (and strictly shrinks when a < 1)."""
+    """Unit keys, b in (0,2), a <= 1, v = 0: every step is a contraction
+    (|1 - b| < 1 along k), so ||S_t||_F never grows."""
     rng = np.random.default_rng(5)
     for channel in (False, True):
         N, H, d = 3, 2, 5
@@ -154,7 +156,7 @@ def pin_contraction(lib=None):
             q = _unit(rng, (N, H, d)); k = _unit(rng, (N, H, d))
             v = np.zeros((N, H, d))
             g = -np.log1p(np.exp(rng.standard_normal((N, H, d) if channel else (N, H))))
-            b = 1 / (1 + np.exp(-rng.standard_normal((N, H))))
+            b = (1 + (t % 2)) / (1 + np.exp(-rng.standard_normal((N, H))))  # (0,1) or (0,2)
             _, S = oracle.step(q, k, v, g, b, S, lib=lib)
             now = np.linalg.norm(S, axis=(2, 3))
             assert np.all(now < prev + 1e-15), "state norm grew"
@@ -243,6 +245,45 @@ def pin_chunkwise(lib=None):
                 _close(r[n], r2[n], 1e-11, f"chunk bwd {n} T={T} C={C}")
 
 
+def pin_negative_eigenvalue(lib=None):
+    """b in (0, 2) (the negative-eigenvalue extension).  With unit k and v = 0
+    one token maps S0 to a S0 (I - b k k^T), whose Frobenius norm satisfies
+    ||S1||^2 = a^2 (||S0||^2 - b (2 - b) ||S0 k||^2); at b = 2, a = 1 the map
+    is the Householder reflection through k's orthogonal complement
+    (S1 k = -S0 k, S1 x = S0 x for x orthogonal to k).  The chunkwise algebra
+    still equals the token loop with b up to 2."""
+    rng = np.random.default_rng(13)
+    dk, dv = 5, 4
+    for trial in range(4):
+        q, k, v, g, beta, h0 = _inputs(rng, T=1, dk=dk, dv=dv, beta_max=2.0)
+        v = np.zeros_like(v)
+        _, S1 = oracle.fwd(q, k, v, g, beta, h0, lib=lib)
+        a, b, kk = np.exp(g[0, 0, 0]), beta[0, 0, 0], k[0, 0, 0]
+        want = a * a * (np.sum(h0[0, 0] ** 2) - b * (2 - b) * np.sum((h0[0, 0] @ kk) ** 2))
+        _close(np.sum(S1[0, 0] ** 2), want, 1e-12, "norm drop")
+        beta2 = np.full_like(beta, 2.0)
+        _, R = oracle.fwd(q, k, v, np.zeros_like(g), beta2, h0, lib=lib)
+        x = rng.standard_normal(dk)
+        x -= (x @ kk) * kk
+        _close(R[0, 0] @ kk, -(h0[0, 0] @ kk), 1e-12, "reflected direction")
+        _close(R[0, 0] @ x, h0[0, 0] @ x, 1e-12, "fixed complement")
+        _close(np.linalg.norm(R[0, 0]), np.linalg.norm(h0[0, 0]), 1e-12, "reflection norm")
+    for channel in (False, True):
+        q, k, v, g, beta, h0 = _inputs(rng, B=1, T=37, H=2, dk=5, dv=4, channel=channel,
+                                      g_shift=-1.0, beta_max=2.0)
+        assert beta.max() > 1.0
+        dO = rng.standard_normal(v.shape)
+        dhT = rng.standard_normal(h0.shape)
+        o, S = oracle.fwd(q, k, v, g, beta, h0, lib=lib)
+        o2, S2 = chunkwise.chunk_forward(q, k, v, g, beta, h0, C=16)
+        _close(o, o2, 1e-11, "chunk fwd o, b in (0,2)")
+        _close(S, S2, 1e-11, "chunk fwd state, b in (0,2)")
+        r = oracle.bwd(q, k, v, g, beta, dO, h0, dhT, ckpt=3, lib=lib)
+        r2 = chunkwise.chunk_backward(q, k, v, g, beta, dO, h0, dhT, C=16)
+        for n in r:
+            _close(r[n], r2[n], 1e-10, f"chunk bwd {n}, b in (0,2)")
+
+
 def pin_channel_equals_scalar(lib=None):
     """A channel gate with the same value in every channel is the scalar gate
     (forward, and the scalar dg is the channel sum of the channel dg)."""
@@ -326,6 +367,7 @@ def pin_euler(lib=None):
 
 
 ALL_PINS = [pin_golden, pin_overwrite, pin_one_token_geometry, pin_identity_and_decay,
-            pin_erase_limit, pin_contraction, pin_sgd_view, pin_dense_closed_form,
+            pin_erase_limit, pin_contraction, pin_negative_eigenvalue, pin_sgd_view,
+            pin_dense_closed_form,
             pin_chunkwise, pin_channel_equals_scalar, pin_step_and_resume,
             pin_bwd_finite_differences, pin_euler]

@@ -105,6 +105,22 @@ def test_whole_head_walk(dev, cfg, over):
     check_bwd(inp, dev)
 
 
+@pytest.mark.parametrize("cfg,over", [
+    (TINY, dict(B=2, H=3, T=77, dk=64, dv=32, chunk=16, h0_std=0.3, dhT_std=0.5)),       # SIMT fp32
+    (L350M, dict(B=2, H=2, T=200, h0_std=0.1, dhT_std=0.3)),                           # 16-row walks
+    (L350M, dict(B=3, H=16, T=130, h0_std=0.1, dhT_std=0.3)),                          # whole-head walks
+    (KDA, dict(B=1, H=4, T=200, h0_std=0.1, dhT_std=0.3)),
+    (KDA, dict(B=3, H=16, T=100, h0_std=0.1)),
+])
+def test_negative_eigenvalue(dev, cfg, over):
+    """beta in (0, 2) (negative-eigenvalue transitions): the same kernels, a
+    wider input range."""
+    inp = make_chunk_inputs(cfg, beta_max=2.0, **over)
+    assert float(inp["beta"].max()) > 1.0
+    check_fwd(inp, dev)
+    check_bwd(inp, dev)
+
+
 # ---- invariants -----------------------------------------------------------
 def test_chunk_size_invariance(dev):
     inp = make_chunk_inputs(L350M, B=1, H=4, T=1000, dtype="f32", g_shift=-2.0, h0_std=0.2)

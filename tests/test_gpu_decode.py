@@ -75,3 +75,19 @@ def test_decode_matches_chunk_fwd(dev):
     torch.cuda.synchronize()
     assert rel_err(o_dec, o_chunk.double().cpu().numpy()) < 1e-4
     assert rel_err(st, hT.double().cpu().numpy()) < 1e-4
+
+
+@pytest.mark.parametrize("dtype,gate", [("f32", "scalar"), ("bf16", "channel")])
+def test_decode_negative_eigenvalue(dev, dtype, gate):
+    """beta in (0, 2): I - beta k k^T may flip the sign along k."""
+    inp = make_decode_inputs(DECODE, steps=20, N=3, H=5, dk=128, dv=128, dtype=dtype, gate=gate,
+                             beta_max=2.0)
+    assert float(inp["beta"].max()) > 1.0
+    o, st = _run_steps(inp, dev, 20)
+    s_ref = inp["state0"].double().numpy()
+    tol = 1e-4 if dtype == "f32" else 2e-2
+    for t in range(20):
+        o_ref, s_ref = oracle.step(inp["q"][t], inp["k"][t], inp["v"][t], inp["g"][t],
+                                   inp["beta"][t], s_ref)
+        assert rel_err(o[t], o_ref) <= tol, t
+    assert rel_err(st, s_ref) <= tol
