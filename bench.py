@@ -67,10 +67,10 @@ def kernel_work(name, B, T, H):
     if name in ("tc_walk_fwd", "tc5_walk_fwd"):
         # reads W, Q, K, U~ (bf16), P, G; writes O
         return dict(bound="hbm", bytes=th * (4 * 256 + 128 + 4 + 256))
-    if name in ("tc_walk_states",):
+    if name in ("tc_walk_states", "tc5_walk_states"):
         # reads W, K, U~, G; writes S0 per chunk (bf16) and U
         return dict(bound="hbm", bytes=th * (3 * 256 + 4 + 256) + nchunks * 128 * 128 * 2)
-    if name == "tc_walk_bwd":
+    if name in ("tc_walk_bwd", "tc5_walk_bwd"):
         # reads P, dO, Q, K, W, G; writes dS per chunk (bf16), dU
         return dict(bound="hbm", bytes=th * (128 + 4 * 256 + 4 + 256) + nchunks * 128 * 128 * 2)
     if name == "tc_bwd_local":
@@ -89,7 +89,8 @@ def kernel_work(name, B, T, H):
 # Kernel -> source file, for matching a recorded ncu traffic figure to the
 # code it was taken on (profiles/roofline_traffic.md).
 KERNEL_SOURCE = {"tc_prep": "tc_chunk.cu", "tc_walk_fwd": "tc_chunk.cu",
-                 "tc5_walk_fwd": "tc5_walk.cu",
+                 "tc5_walk_fwd": "tc5_walk.cu", "tc5_walk_states": "tc5_walk.cu",
+                 "tc5_walk_bwd": "tc5_walk_bwd.cu",
                  "tc_walk_states": "tc_chunk.cu", "tc_walk_bwd": "tc_bwd.cu",
                  "tc_bwd_local": "tc_bwd.cu", "tc_prep_kda": "tc_kda.cu",
                  "decode_step": "decode.cu"}
@@ -302,7 +303,7 @@ def run_ours(args, rank, world, dev, barrier, max_over_ranks):
     extra = {}
     if not args.headline_only:
         # ---- long-context forward (the 50%-of-tensor-peak target) ----------
-        li = to_dev(make_chunk_inputs(LONG, seed=LONG.seed + 7919 * rank), dev)
+        li = to_dev(make_chunk_inputs(LONG, seed=replica_seed(LONG.seed, rank)), dev)
         lws_f, _ = workspaces(gdn, li)
         lo = torch.empty_like(li["v"])
         lh = torch.empty(LONG.B, LONG.H, LONG.dv, LONG.dk, device=dev)
@@ -321,7 +322,7 @@ def run_ours(args, rank, world, dev, barrier, max_over_ranks):
         extra["long_context_fwd_bwd_ms"] = round(ms_fb, 3)
         del li, lws_f
         # ---- channel gate (KDA) fwd+bwd -------------------------------------
-        ki = to_dev(make_chunk_inputs(KDA, seed=KDA.seed + 7919 * rank), dev)
+        ki = to_dev(make_chunk_inputs(KDA, seed=replica_seed(KDA.seed, rank)), dev)
         kws_f, kws_b = workspaces(gdn, ki)
         ko = dict(o=torch.empty_like(ki["v"]), hT=None)
         ms_k = timed(chunk_step_fn(gdn, ki, kws_f, kws_b, ko), 3, 1, barrier)
@@ -331,7 +332,7 @@ def run_ours(args, rank, world, dev, barrier, max_over_ranks):
                                 "tflops": round((FWD_FLOP + BWD_FLOP) * kth / (ms_k / 1e3) / 1e12, 2)}
         del ki, kws_f, kws_b
         # ---- decode: 1000 successive single-token steps --------------------
-        dec = make_decode_inputs(DECODE, seed=DECODE.seed + 7919 * rank)
+        dec = make_decode_inputs(DECODE, seed=replica_seed(DECODE.seed, rank))
         dd = to_dev(dec, dev)
         st = dd["state0"].clone()
         o = torch.empty(DECODE.N, DECODE.H, DECODE.dv, dtype=torch.bfloat16, device=dev)
