@@ -60,6 +60,11 @@ struct KdaPrepSmem {
 
 __device__ __forceinline__ int pair_index(int I, int J) { return I * (I - 1) / 2 + J; }
 
+// Eight warps: warp w works on row block w % 4; in the A/P products it takes
+// the column blocks J of parity w / 4, in the W / U~ products the column half
+// w / 4; the block solve runs on warps 0..3.
+constexpr int KP_THREADS = 256;
+
 GDN_DEV void scale_a_cols_f(uint32_t (&a)[4], const float* f, int k0) {
     const int l = threadIdx.x & 31;
     const int k = k0 + 2 * (l & 3);
@@ -71,7 +76,7 @@ GDN_DEV void scale_a_cols_f(uint32_t (&a)[4], const float* f, int k0) {
     }
 }
 
-__global__ void __launch_bounds__(128) tc_prep_kda_kernel(const __grid_constant__ ChunkPtrs p) {
+__global__ void __launch_bounds__(KP_THREADS) tc_prep_kda_kernel(const __grid_constant__ ChunkPtrs p) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     KdaPrepSmem& s = *reinterpret_cast<KdaPrepSmem*>(align1k(smem_raw));
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -92,7 +97,7 @@ __global__ void __launch_bounds__(128) tc_prep_kda_kernel(const __grid_constant_
         tma_load_tile(s.V, &p.vmap, h, tok, &s.bar);
     }
     // log-gates (rows past the sequence end add 0) and beta
-    for (int e = tid; e < C * (DK / 4); e += 128) {
+    for (int e = tid; e < C * (DK / 4); e += KP_THREADS) {
         const int r = e / (DK / 4), c4 = e % (DK / 4);
         const bool ok = r < L;
         cp_async16_zfill(&s.G[r][4 * c4], p.g + (row0 + (size_t)(ok ? r : 0) * rs) * DK + 4 * c4, ok);
@@ -101,7 +106,7 @@ __global__ void __launch_bounds__(128) tc_prep_kda_kernel(const __grid_constant_
     if (tid < C) s.beta[tid] = tid < L ? p.beta[row0 + tid * rs] : 0.f;
     cp_async_wait<0>();
     __syncthreads();
-    {   // per-channel cumsum: thread c owns channel c
+    if (tid < DK) {   // per-channel cumsum: thread c owns channel c
         const int c = tid;
         float run = 0.f;
         for (int i = 0; i < C; ++i) {
@@ -121,14 +126,14 @@ __global__ void __launch_bounds__(128) tc_prep_kda_kernel(const __grid_constant_
         for (int o = 16; o > 0; o >>= 1) sp = fmaxf(sp, __shfl_xor_sync(0xffffffffu, sp, o));
         if (lane == 0) s.diag_ok[warp] = sp <= 80.f;
     }
-    for (int e = tid; e < 6 * DK; e += 128) {
+    for (int e = tid; e < 6 * DK; e += KP_THREADS) {
         const int pi = e / DK, c = e % DK;
         const int I = pi < 1 ? 1 : (pi < 3 ? 2 : 3);
         const int J = pi - I * (I - 1) / 2;
         s.F[pi][c] = __expf(s.G[16 * I][c] - s.G[16 * J + 15][c]);
     }
     // scaled operands
-    for (int e = tid; e < C * DK; e += 128) {
+    for (int e = tid; e < C * DK; e += KP_THREADS) {
         const int i = e / DK, c = e % DK;
         const int f = i & ~15, l = f + 15;
         const float g = s.G[i][c];
@@ -143,8 +148,8 @@ __global__ void __launch_bounds__(128) tc_prep_kda_kernel(const __grid_constant_
     }
     __syncthreads();
 
-    const int m0 = 16 * warp, I = warp;
-    // ---- A and P, row block I -------------------------------------------
+    const int I = warp & 3, m0 = 16 * I, half = warp >> 2;
+    // ---- A and P, row block I, column blocks J of parity `half` ----------
     {
         float acck[4][2][4], accq[4][2][4];  // [J][n-tile][e]
 #pragma unroll
@@ -162,6 +167,7 @@ __global__ void __launch_bounds__(128) tc_prep_kda_kernel(const __grid_constant_
 #pragma unroll
             for (int J = 0; J < 4; ++J) {
                 if (J > I) break;
+                if ((J & 1) != half) continue;
                 uint32_t ak[4], aq[4], bf[4];
 #pragma unroll
                 for (int r = 0; r < 4; ++r) { ak[r] = ak0[r]; aq[r] = aq0[r]; }
@@ -182,6 +188,7 @@ __global__ void __launch_bounds__(128) tc_prep_kda_kernel(const __grid_constant_
         const int ra = m0 + (lane >> 2), rb = ra + 8;
 #pragma unroll
         for (int J = 0; J < 4; ++J) {
+            if ((J & 1) != half) continue;
 #pragma unroll
             for (int t = 0; t < 2; ++t) {
                 const int c0 = 16 * J + 8 * t + 2 * (lane & 3);
@@ -198,7 +205,7 @@ __global__ void __launch_bounds__(128) tc_prep_kda_kernel(const __grid_constant_
                 st_c<S64>(s.P, m0, 16 * J + 8 * t, pv);
             }
         }
-        if (!dok) {
+        if (!dok && (I & 1) == half) {
             // exact diagonal block: pairs (i, j), j <= i, summed over channels
             __syncwarp();
             for (int e = lane; e < 16 * 16; e += 32) {
@@ -219,10 +226,10 @@ __global__ void __launch_bounds__(128) tc_prep_kda_kernel(const __grid_constant_
             }
         }
     }
-    __syncwarp();
+    __syncthreads();  // A's diagonal blocks complete (either warp of a pair wrote them)
 
-    // ---- UT transform (identical to the scalar-gate prep) -----------------
-    {
+    // ---- UT transform (identical to the scalar-gate prep), warps 0..3 ------
+    if (warp < 4) {
         const int c = lane & 15;
         float t[16];
 #pragma unroll
@@ -244,7 +251,7 @@ __global__ void __launch_bounds__(128) tc_prep_kda_kernel(const __grid_constant_
     __syncthreads();
     for (int dgl = 1; dgl < 4; ++dgl) {
         const int J = warp, I2 = warp + dgl;
-        if (I2 < 4) {
+        if (warp < 4 && I2 < 4) {
             float x[2][4] = {};
             for (int Kb = J; Kb < I2; ++Kb) {
                 uint32_t a[4], bt[4];
@@ -280,7 +287,7 @@ __global__ void __launch_bounds__(128) tc_prep_kda_kernel(const __grid_constant_
     }
 
     // ---- K .* e^G (W operand), Qg = scale Q .* e^G, Kt = K .* e^{G_last - G}
-    for (int e = tid; e < C * DK; e += 128) {
+    for (int e = tid; e < C * DK; e += KP_THREADS) {
         const int i = e / DK, c = e % DK;
         const uint32_t o = Tma128::off(i, c);
         const float g = s.G[i][c];
@@ -291,22 +298,23 @@ __global__ void __launch_bounds__(128) tc_prep_kda_kernel(const __grid_constant_
         s.Q[o] = __float2bfloat16_rn(p.scale * __bfloat162float(s.Q[o]) * eg);  // Qg image
     }
     __syncthreads();
-    float aw[16][4], au[16][4];
+    // W, U~ for row block I, columns 64*half .. +63
+    float aw[8][4], au[8][4];
 #pragma unroll
-    for (int j = 0; j < 16; ++j)
+    for (int j = 0; j < 8; ++j)
 #pragma unroll
         for (int e = 0; e < 4; ++e) aw[j][e] = au[j][e] = 0.f;
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk) {
-        if (kk > warp) break;
+        if (kk > I) break;
         uint32_t a1[4];
         lda<S64>(a1, s.Tb, m0, 16 * kk);
         scale_a_cols_f(a1, s.beta, 16 * kk);
 #pragma unroll
-        for (int np = 0; np < 8; ++np) {
+        for (int np = 0; np < 4; ++np) {
             uint32_t bk[4], bv[4];
-            ldb_kn<Tma128>(bk, s.Kl, 16 * kk, 16 * np);
-            ldb_kn<Tma128>(bv, s.V, 16 * kk, 16 * np);
+            ldb_kn<Tma128>(bk, s.Kl, 16 * kk, 64 * half + 16 * np);
+            ldb_kn<Tma128>(bv, s.V, 16 * kk, 64 * half + 16 * np);
             mma16816(aw[2 * np], a1, bk[0], bk[1]);
             mma16816(aw[2 * np + 1], a1, bk[2], bk[3]);
             mma16816(au[2 * np], a1, bv[0], bv[1]);
@@ -314,7 +322,7 @@ __global__ void __launch_bounds__(128) tc_prep_kda_kernel(const __grid_constant_
         }
     }
     __syncthreads();  // done reading Kl and V
-    stage_w_ut(s.Kl, s.Kr, aw, au, m0);  // W image in Kl's slot, U~^T image in Kr's
+    stage_w_ut_cols(s.Kl, s.Kr, aw, au, m0, 64 * half);  // W image in Kl's slot, U~^T in Kr's
     fence_async_smem();
     __syncthreads();
     if (tid == 0) {
@@ -335,7 +343,7 @@ __global__ void __launch_bounds__(128) tc_prep_kda_kernel(const __grid_constant_
 void launch_prep_kda(const ChunkPtrs& p, size_t nchunks, cudaStream_t st) {
     const int smem = sizeof(KdaPrepSmem) + 1024;
     cudaFuncSetAttribute(tc_prep_kda_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    GDN_LAUNCH("tc_prep_kda", st, tc_prep_kda_kernel<<<(unsigned)nchunks, 128, smem, st>>>(p));
+    GDN_LAUNCH("tc_prep_kda", st, tc_prep_kda_kernel<<<(unsigned)nchunks, KP_THREADS, smem, st>>>(p));
 }
 
 }  // namespace tc
