@@ -85,12 +85,13 @@ GDN_DEV void stage_w_ut(__nv_bfloat16* Wst, __nv_bfloat16* Ust, const float (&aw
     }
 }
 
-// The same for 64 of the 128 columns, starting at column n0.
-GDN_DEV void stage_w_ut_cols(__nv_bfloat16* Wst, __nv_bfloat16* Ust, const float (&aw)[8][4],
-                             const float (&au)[8][4], int m0, int n0) {
+// The same for 8*NB of the 128 columns, starting at column n0.
+template <int NB>
+GDN_DEV void stage_w_ut_cols(__nv_bfloat16* Wst, __nv_bfloat16* Ust, const float (&aw)[NB][4],
+                             const float (&au)[NB][4], int m0, int n0) {
     const int lane = threadIdx.x & 31;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
+    for (int j = 0; j < NB; ++j) {
         st_c<Tma128>(Wst, m0, n0 + 8 * j, aw[j]);
         const int r = m0 + (lane >> 2), c = n0 + 8 * j + 2 * (lane & 3);
         Ust[swz<C>(c, r)] = __float2bfloat16_rn(au[j][0]);

@@ -60,10 +60,10 @@ struct KdaPrepSmem {
 
 __device__ __forceinline__ int pair_index(int I, int J) { return I * (I - 1) / 2 + J; }
 
-// Eight warps: warp w works on row block w % 4; in the A/P products it takes
-// the column blocks J of parity w / 4, in the W / U~ products the column half
-// w / 4; the block solve runs on warps 0..3.
-constexpr int KP_THREADS = 256;
+// Sixteen warps: warp w works on row block w % 4; in the A/P products it takes
+// column block J = w / 4, in the W / U~ products the column quarter w / 4;
+// the block solve runs on warps 0..3.
+constexpr int KP_THREADS = 512;
 
 GDN_DEV void scale_a_cols_f(uint32_t (&a)[4], const float* f, int k0) {
     const int l = threadIdx.x & 31;
@@ -148,8 +148,8 @@ __global__ void __launch_bounds__(KP_THREADS) tc_prep_kda_kernel(const __grid_co
     }
     __syncthreads();
 
-    const int I = warp & 3, m0 = 16 * I, half = warp >> 2;
-    // ---- A and P, row block I, column blocks J of parity `half` ----------
+    const int I = warp & 3, m0 = 16 * I, grp = warp >> 2;
+    // ---- A and P, row block I, column block J = grp ----------------------
     {
         float acck[4][2][4], accq[4][2][4];  // [J][n-tile][e]
 #pragma unroll
@@ -167,7 +167,7 @@ __global__ void __launch_bounds__(KP_THREADS) tc_prep_kda_kernel(const __grid_co
 #pragma unroll
             for (int J = 0; J < 4; ++J) {
                 if (J > I) break;
-                if ((J & 1) != half) continue;
+                if (J != grp) continue;
                 uint32_t ak[4], aq[4], bf[4];
 #pragma unroll
                 for (int r = 0; r < 4; ++r) { ak[r] = ak0[r]; aq[r] = aq0[r]; }
@@ -188,7 +188,7 @@ __global__ void __launch_bounds__(KP_THREADS) tc_prep_kda_kernel(const __grid_co
         const int ra = m0 + (lane >> 2), rb = ra + 8;
 #pragma unroll
         for (int J = 0; J < 4; ++J) {
-            if ((J & 1) != half) continue;
+            if (J != grp) continue;
 #pragma unroll
             for (int t = 0; t < 2; ++t) {
                 const int c0 = 16 * J + 8 * t + 2 * (lane & 3);
@@ -205,7 +205,7 @@ __global__ void __launch_bounds__(KP_THREADS) tc_prep_kda_kernel(const __grid_co
                 st_c<S64>(s.P, m0, 16 * J + 8 * t, pv);
             }
         }
-        if (!dok && (I & 1) == half) {
+        if (!dok && I == grp) {
             // exact diagonal block: pairs (i, j), j <= i, summed over channels
             __syncwarp();
             for (int e = lane; e < 16 * 16; e += 32) {
@@ -298,10 +298,10 @@ __global__ void __launch_bounds__(KP_THREADS) tc_prep_kda_kernel(const __grid_co
         s.Q[o] = __float2bfloat16_rn(p.scale * __bfloat162float(s.Q[o]) * eg);  // Qg image
     }
     __syncthreads();
-    // W, U~ for row block I, columns 64*half .. +63
-    float aw[8][4], au[8][4];
+    // W, U~ for row block I, columns 32*grp .. +31
+    float aw[4][4], au[4][4];
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
+    for (int j = 0; j < 4; ++j)
 #pragma unroll
         for (int e = 0; e < 4; ++e) aw[j][e] = au[j][e] = 0.f;
 #pragma unroll
@@ -311,10 +311,10 @@ __global__ void __launch_bounds__(KP_THREADS) tc_prep_kda_kernel(const __grid_co
         lda<S64>(a1, s.Tb, m0, 16 * kk);
         scale_a_cols_f(a1, s.beta, 16 * kk);
 #pragma unroll
-        for (int np = 0; np < 4; ++np) {
+        for (int np = 0; np < 2; ++np) {
             uint32_t bk[4], bv[4];
-            ldb_kn<Tma128>(bk, s.Kl, 16 * kk, 64 * half + 16 * np);
-            ldb_kn<Tma128>(bv, s.V, 16 * kk, 64 * half + 16 * np);
+            ldb_kn<Tma128>(bk, s.Kl, 16 * kk, 32 * grp + 16 * np);
+            ldb_kn<Tma128>(bv, s.V, 16 * kk, 32 * grp + 16 * np);
             mma16816(aw[2 * np], a1, bk[0], bk[1]);
             mma16816(aw[2 * np + 1], a1, bk[2], bk[3]);
             mma16816(au[2 * np], a1, bv[0], bv[1]);
@@ -322,7 +322,7 @@ __global__ void __launch_bounds__(KP_THREADS) tc_prep_kda_kernel(const __grid_co
         }
     }
     __syncthreads();  // done reading Kl and V
-    stage_w_ut_cols(s.Kl, s.Kr, aw, au, m0, 64 * half);  // W image in Kl's slot, U~^T in Kr's
+    stage_w_ut_cols(s.Kl, s.Kr, aw, au, m0, 32 * grp);  // W image in Kl's slot, U~^T in Kr's
     fence_async_smem();
     __syncthreads();
     if (tid == 0) {
