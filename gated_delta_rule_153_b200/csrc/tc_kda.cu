@@ -391,9 +391,11 @@ struct KdaLocSmem {
             __nv_bfloat16 Kl[C * DK], Kr[C * DK], Kd[C * DK], Ql[C * DK], Kg[C * DK];
             __nv_bfloat16 V[C * DV];    // Tma128 (TMA), loaded at the start
         } p2;
-        float dG[C][DK];
+        float dG[C][DK + 4];
     } u;
-    float G[C][DK];
+    // Rows padded by 4 floats: a warp reading its MMA fragment's (row, column)
+    // positions (8 rows x 4 columns) then hits 2 lanes per bank instead of 8.
+    float G[C][DK + 4];
     float red_b[KL_WARPS][C];
     float glp[2][4][DK];        // G_last column partials: [term][row block][channel]
     float beta[C];
@@ -766,10 +768,15 @@ __global__ void __launch_bounds__(KL_THREADS) tc_bwd_local_kda_kernel(const __gr
     __syncthreads();
 
     // ---- phase 5: the four decayed pair products ---------------------------------
+    // Each column block's contribution goes straight into dQ, dK and dG, so no
+    // per-side accumulators stay live across the blocks.  The pair (r, r) has
+    // decay 1 and adds nothing to dG (its row- and column-side terms cancel): its
+    // rounded form is left out of the dG sums on both sides, so that no bf16
+    // residual of it swamps the small dg of a strongly decayed chunk.
     {
-        // row side (X1, X4): blocks J < I scaled by F_IJ per channel, the diagonal
-        // block through Kd; everything then by EL = e^{G_r - G_f}
-        float x1[4][4] = {}, x4[4][4] = {};
+        // row side: X1 = dMM (K .* decay), X4 = dP (K .* decay); blocks J < I
+        // through Kr, the diagonal block through Kd, then each by its factor
+        // e^{G_r - G_l} (J < I, l = last row of J) or e^{G_r - G_f} (J = I)
         for (int J = 0; J <= I; ++J) {
             if (J == I && !dok) break;
             float t1[4][4] = {}, t4[4][4] = {};
@@ -786,53 +793,46 @@ __global__ void __launch_bounds__(KL_THREADS) tc_bwd_local_kda_kernel(const __gr
                 mma16816(t4[2 * np], ap, bk[0], bk[1]);
                 mma16816(t4[2 * np + 1], ap, bk[2], bk[3]);
             }
+            const int ref = J < I ? 16 * J + 15 : m0;
 #pragma unroll
             for (int j = 0; j < 4; ++j)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const int c = col(j, e);
-                    const float f = J < I ? __expf(s.G[16 * I][c] - s.G[16 * J + 15][c]) : 1.f;
-                    x1[j][e] += f * t1[j][e];
-                    x4[j][e] += f * t4[j][e];
+                    const int r = row(e), c = col(j, e);
+                    const uint32_t o = Tma128::off(r, c);
+                    const float f = __expf(s.G[r][c] - s.G[ref][c]);
+                    const float x1 = f * t1[j][e], x4 = f * t4[j][e];
+                    const float self4 = J == I ? bf(s.dP, swz<C>(r, r)) * bf(s.u.p2.Kd, o) * f : 0.f;
+                    dK[j][e] += x1;
+                    dQ[j][e] += x4;
+                    dG[j][e] += bf(s.K, o) * x1 + p.scale * bf(s.Q, o) * (x4 - self4);
                 }
         }
+        if (!dok) {  // exact diagonal-block sums, j <= i inside block I
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
+            for (int j = 0; j < 4; ++j)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int r = row(e), c = col(j, e);
-                const float gr = s.G[r][c];
-                const float el = __expf(gr - s.G[m0][c]);
-                const float kv = bf(s.K, Tma128::off(r, c)), qv = bf(s.Q, Tma128::off(r, c));
-                const float dpd = bf(s.dP, swz<C>(r, r));
-                x1[j][e] *= el;
-                x4[j][e] *= el;
-                // The pair (r, r) has decay 1 and adds nothing to dG (its row- and
-                // column-side terms cancel).  Its rounded form is taken out of the dG
-                // sum here and on the column side, so that no bf16 residual of it
-                // swamps the small dg of a strongly decayed chunk.
-                float self4;
-                if (dok) {
-                    self4 = dpd * bf(s.u.p2.Kd, Tma128::off(r, c)) * el;
-                } else {  // exact diagonal-block sums, j < i inside block I
+                for (int e = 0; e < 4; ++e) {
+                    const int r = row(e), c = col(j, e);
+                    const float gr = s.G[r][c];
+                    float x1 = 0.f, x4 = 0.f;
                     for (int jj = m0; jj < r; ++jj) {
                         const float d = __expf(gr - s.G[jj][c]);
                         const float kj = bf(s.K, Tma128::off(jj, c));
-                        x1[j][e] += bf(s.dT, swz<C>(r, jj)) * d * kj;
-                        x4[j][e] += bf(s.dP, swz<C>(r, jj)) * d * kj;
+                        x1 += bf(s.dT, swz<C>(r, jj)) * d * kj;
+                        x4 += bf(s.dP, swz<C>(r, jj)) * d * kj;
                     }
-                    self4 = dpd * kv;
-                    x4[j][e] += self4;
+                    const float kv = bf(s.K, Tma128::off(r, c)), qv = bf(s.Q, Tma128::off(r, c));
+                    dK[j][e] += x1;
+                    dQ[j][e] += x4 + bf(s.dP, swz<C>(r, r)) * kv;
+                    dG[j][e] += kv * x1 + p.scale * qv * x4;
                 }
-                dK[j][e] += x1[j][e];
-                dQ[j][e] += x4[j][e];
-                dG[j][e] += kv * x1[j][e] + p.scale * qv * (x4[j][e] - self4);
-            }
+        }
     }
     {
-        // column side (X2, X3): blocks J > I scaled by ER_r F_JI, the diagonal
-        // block by e^{G_f - G_r} (its B operands carry EL_j)
-        float x2[4][4] = {}, x3[4][4] = {};
+        // column side: X2 = dMM^T (K .* decay), X3 = dP^T (Q .* decay); blocks J > I
+        // by e^{G_f(J) - G_r}, the diagonal block by e^{G_f - G_r} (its B operands
+        // carry EL_j)
         for (int J = I; J < 4; ++J) {
             if (J == I && !dok) continue;
             float t2[4][4] = {}, t3[4][4] = {};
@@ -854,38 +854,32 @@ __global__ void __launch_bounds__(KL_THREADS) tc_bwd_local_kda_kernel(const __gr
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int r = row(e), c = col(j, e);
-                    const float gr = s.G[r][c];
-                    const float f = J > I ? __expf(s.G[m0 + 15][c] - gr + s.G[16 * J][c] -
-                                                   s.G[m0 + 15][c])
-                                          : __expf(s.G[m0][c] - gr);
-                    x2[j][e] += f * t2[j][e];
-                    x3[j][e] += f * t3[j][e];
+                    const uint32_t o = Tma128::off(r, c);
+                    const float f = __expf(s.G[16 * J][c] - s.G[r][c]);
+                    const float x2 = f * t2[j][e], x3 = f * t3[j][e];
+                    const float self3 = J == I ? bf(s.dP, swz<C>(r, r)) * bf(s.u.p2.Ql, o) * f : 0.f;
+                    dK[j][e] += x2 + p.scale * x3;
+                    dG[j][e] -= bf(s.K, o) * (x2 + p.scale * (x3 - self3));
                 }
         }
+        if (!dok) {  // exact diagonal-block sums, j > i inside block I
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
+            for (int j = 0; j < 4; ++j)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int r = row(e), c = col(j, e);
-                const float gr = s.G[r][c];
-                const float dpd = bf(s.dP, swz<C>(r, r));
-                float self3;  // the (r, r) pair's term, left out of dG as on the row side
-                if (dok) {
-                    self3 = dpd * bf(s.u.p2.Ql, Tma128::off(r, c)) * __expf(s.G[m0][c] - gr);
-                } else {  // exact diagonal-block sums, j > i inside block I
+                for (int e = 0; e < 4; ++e) {
+                    const int r = row(e), c = col(j, e);
+                    const float gr = s.G[r][c];
+                    float x2 = 0.f, x3 = 0.f;
                     for (int jj = r + 1; jj < m0 + 16; ++jj) {
                         const float d = __expf(s.G[jj][c] - gr);
-                        x2[j][e] += bf(s.dT, swz<C>(jj, r)) * d * bf(s.K, Tma128::off(jj, c));
-                        x3[j][e] += bf(s.dP, swz<C>(jj, r)) * d * bf(s.Q, Tma128::off(jj, c));
+                        x2 += bf(s.dT, swz<C>(jj, r)) * d * bf(s.K, Tma128::off(jj, c));
+                        x3 += bf(s.dP, swz<C>(jj, r)) * d * bf(s.Q, Tma128::off(jj, c));
                     }
-                    self3 = dpd * bf(s.Q, Tma128::off(r, c));
-                    x3[j][e] += self3;
+                    const float kv = bf(s.K, Tma128::off(r, c));
+                    dK[j][e] += x2 + p.scale * (x3 + bf(s.dP, swz<C>(r, r)) * bf(s.Q, Tma128::off(r, c)));
+                    dG[j][e] -= kv * (x2 + p.scale * x3);
                 }
-                const float kv = bf(s.K, Tma128::off(r, c));
-                const float y = x2[j][e] + p.scale * x3[j][e];
-                dK[j][e] += y;
-                dG[j][e] -= kv * (x2[j][e] + p.scale * (x3[j][e] - self3));
-            }
+        }
     }
     {
         const bool okl = rl < L, okh = rh < L;
