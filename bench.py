@@ -331,6 +331,20 @@ def run_ours(args, rank, world, dev, barrier, max_over_ranks):
                                 "tokens_per_s": round(KDA.B * KDA.T / (ms_k / 1e3), 1),
                                 "tflops": round((FWD_FLOP + BWD_FLOP) * kth / (ms_k / 1e3) / 1e12, 2)}
         del ki, kws_f, kws_b
+        # ---- gated DeltaProduct, n = 2 steps per token, 350M-scale shape -----
+        from gated_delta_rule_153_b200.inputs import make_product_inputs
+        pi = to_dev(make_product_inputs(cfg, 2, seed=replica_seed(cfg.seed + 1, rank)), dev)
+
+        def product_step():
+            gdn.gdn_product_fwd(pi["q"], pi["k"], pi["v"], pi["g"], pi["beta"], pi["h0"])
+            gdn.gdn_product_bwd(pi["q"], pi["k"], pi["v"], pi["g"], pi["beta"], pi["dO"],
+                                pi["h0"], pi["dhT"])
+        ms_p = timed(product_step, 3, 1, barrier)
+        extra["deltaproduct_fwd_bwd"] = {
+            "workload": f"{cfg.name}, n=2 delta steps per token", "ms": round(ms_p, 3),
+            "tokens_per_s": round(cfg.B * cfg.T / (ms_p / 1e3), 1),
+            "sub_tokens_per_s": round(2 * cfg.B * cfg.T / (ms_p / 1e3), 1)}
+        del pi
         # ---- decode: 1000 successive single-token steps --------------------
         dec = make_decode_inputs(DECODE, seed=replica_seed(DECODE.seed, rank))
         dd = to_dev(dec, dev)

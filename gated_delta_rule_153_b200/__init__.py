@@ -28,7 +28,8 @@ GDN_GATE_SCALAR, GDN_GATE_CHANNEL = 0, 1
 EXPORTS = ("gdn_chunk_fwd_workspace", "gdn_chunk_fwd", "gdn_chunk_bwd_workspace",
            "gdn_chunk_bwd", "gdn_recurrent_step", "gdn_query_device_status",
            "gdn_status_string", "gdn_profile_begin", "gdn_profile_end",
-           "gdn_chunk_fwd_noalloc")
+           "gdn_chunk_fwd_noalloc", "gdn_product_fwd_workspace", "gdn_product_fwd",
+           "gdn_product_bwd_workspace", "gdn_product_bwd")
 
 
 class gdn_dims(ctypes.Structure):
@@ -76,6 +77,15 @@ def lib() -> ctypes.CDLL:
             L.gdn_query_device_status.restype = i
             L.gdn_chunk_fwd_noalloc.argtypes = [dp, vp, vp, vp, fp, fp, fp, vp, fp, vp]
             L.gdn_chunk_fwd_noalloc.restype = i
+            L.gdn_product_fwd_workspace.argtypes = [dp, i]
+            L.gdn_product_fwd_workspace.restype = sz
+            L.gdn_product_bwd_workspace.argtypes = [dp, i]
+            L.gdn_product_bwd_workspace.restype = sz
+            L.gdn_product_fwd.argtypes = [dp, i, vp, vp, vp, fp, fp, fp, vp, fp, vp, sz, vp]
+            L.gdn_product_fwd.restype = i
+            L.gdn_product_bwd.argtypes = [dp, i, vp, vp, vp, fp, fp, fp, vp, fp, vp, vp, vp,
+                                          fp, fp, fp, vp, sz, vp]
+            L.gdn_product_bwd.restype = i
             L.gdn_profile_begin.argtypes = [i]
             L.gdn_profile_begin.restype = i
             L.gdn_profile_end.argtypes = [ctypes.POINTER(ctypes.c_float),
@@ -257,3 +267,70 @@ def gdn_profile_end(capacity: int):
 def gdn_query_device_status(workspace, stream=None) -> int:
     """Status word of the most recent chunkwise call that used ``workspace``."""
     return int(lib().gdn_query_device_status(_ptr(workspace), _stream(stream)))
+
+
+# ---- gated DeltaProduct (n delta-rule steps per token) ---------------------
+def _validate_product_inputs(q, k, v, g, beta, h0):
+    import torch
+    _need(q, "q")
+    B, T, H, dk = q.shape
+    if k.dim() != 5:
+        raise ValueError("k must be [B,T,n,H,dk]")
+    n = k.shape[2]
+    _need(k, "k", q.dtype, (B, T, n, H, dk))
+    _need(v, "v", q.dtype)
+    if v.dim() != 5 or v.shape[:4] != (B, T, n, H):
+        raise ValueError("v must be [B,T,n,H,dv] matching k")
+    dv = v.shape[4]
+    _need(g, "g", torch.float32)
+    if tuple(g.shape) not in ((B, T, H), (B, T, H, dk)):
+        raise ValueError("g must be [B,T,H] or [B,T,H,dk]")
+    _need(beta, "beta", torch.float32, (B, T, n, H))
+    if h0 is not None:
+        _need(h0, "h0", torch.float32, (B, H, dv, dk))
+    return B, T, n, H, dk, dv
+
+
+def gdn_product_fwd(q, k, v, g, beta, h0=None, *, chunk=64, scale=1.0,
+                    output_final_state=True, workspace=None, stream=None):
+    """Gated DeltaProduct forward: k [B,T,n,H,dk], v [B,T,n,H,dv],
+    beta [B,T,n,H]; q, g, h0 as for gdn_chunk_fwd.  Returns (o, hT)."""
+    import torch
+    B, T, n, H, dk, dv = _validate_product_inputs(q, k, v, g, beta, h0)
+    dims = make_dims(q, v, g, chunk, scale)
+    o = torch.empty(B, T, H, dv, dtype=q.dtype, device=q.device)
+    hT = torch.empty(B, H, dv, dk, dtype=torch.float32, device=q.device) \
+        if output_final_state else None
+    nbytes = int(lib().gdn_product_fwd_workspace(ctypes.byref(dims), n))
+    ws = _workspace(nbytes, q.device, workspace)
+    st = lib().gdn_product_fwd(ctypes.byref(dims), n, _ptr(q), _ptr(k), _ptr(v), _ptr(g),
+                               _ptr(beta), _ptr(h0), _ptr(o), _ptr(hT), _ptr(ws),
+                               nbytes if ws is None else ws.numel() * ws.element_size(),
+                               _stream(stream))
+    _check(st, "gdn_product_fwd")
+    return o, hT
+
+
+def gdn_product_bwd(q, k, v, g, beta, dO, h0=None, dhT=None, *, chunk=64, scale=1.0,
+                    workspace=None, stream=None):
+    """Gated DeltaProduct backward of <dO,o> + <dhT,hT>: gradients in the
+    shapes of their primals (dh0 None when h0 is None)."""
+    import torch
+    B, T, n, H, dk, dv = _validate_product_inputs(q, k, v, g, beta, h0)
+    _need(dO, "dO", q.dtype, (B, T, H, dv))
+    if dhT is not None:
+        _need(dhT, "dhT", torch.float32, (B, H, dv, dk))
+    dims = make_dims(q, v, g, chunk, scale)
+    out = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dv=torch.empty_like(v),
+               dg=torch.empty_like(g), dbeta=torch.empty_like(beta),
+               dh0=None if h0 is None else torch.empty_like(h0))
+    nbytes = int(lib().gdn_product_bwd_workspace(ctypes.byref(dims), n))
+    ws = _workspace(nbytes, q.device, workspace)
+    st = lib().gdn_product_bwd(ctypes.byref(dims), n, _ptr(q), _ptr(k), _ptr(v), _ptr(g),
+                               _ptr(beta), _ptr(h0), _ptr(dO), _ptr(dhT), _ptr(out["dq"]),
+                               _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dg"]),
+                               _ptr(out["dbeta"]), _ptr(out["dh0"]), _ptr(ws),
+                               nbytes if ws is None else ws.numel() * ws.element_size(),
+                               _stream(stream))
+    _check(st, "gdn_product_bwd")
+    return out

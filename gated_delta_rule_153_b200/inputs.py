@@ -146,3 +146,18 @@ def make_decode_inputs(cfg: DecodeConfig, steps: Optional[int] = None, **over) -
     state0 = torch.randn(N, H, dv, dk, generator=gens[5]) * cfg.state_std
     return dict(q=q, k=k, v=v, g=g.contiguous(), beta=beta.contiguous(),
                 state0=state0, cfg=cfg)
+
+
+def make_product_inputs(cfg: ChunkConfig, n: int, **over) -> dict:
+    """Host tensors for the gated DeltaProduct with n steps per token:
+    k, v [B,T,n,H,d] and beta [B,T,n,H] are the n*T-token draw of
+    ``make_chunk_inputs`` viewed per token; q, g, h0, dO, dhT come from the
+    T-token draw."""
+    tok = make_chunk_inputs(cfg, **over)
+    c = tok["cfg"]
+    sub = make_chunk_inputs(c, T=c.T * n, seed=c.seed + 500)
+    B, T, H = c.B, c.T, c.H
+    return dict(q=tok["q"], g=tok["g"], h0=tok["h0"], dO=tok["dO"], dhT=tok["dhT"],
+                k=sub["k"].reshape(B, T, n, H, c.dk).contiguous(),
+                v=sub["v"].reshape(B, T, n, H, c.dv).contiguous(),
+                beta=sub["beta"].reshape(B, T, n, H).contiguous(), n=n, cfg=c)

@@ -113,6 +113,41 @@ gdn_status gdn_chunk_bwd(const gdn_dims *dims, const void *q, const void *k,
                          float *dh0, void *ws, size_t ws_bytes,
                          gdn_stream_t stream);
 
+/* Gated DeltaProduct: "DeltaProduct: Improving State-Tracking in Linear RNNs
+ * via Householder Products" (in the list of related papers of the "Linear
+ * Attention Architectures: Mechanisms, Trade-offs, and Cross-Layer Routing"
+ * summary page) with the gate of "Gated Delta Networks: Improving Mamba2
+ * with Delta Rule" (paper review), whose section "Future work" names
+ * products of Householder matrices as an extension.  The pages give no
+ * equation; the reading: each token applies its gate once, then n delta-rule
+ * steps with its own keys, values and betas in order j = 1..n, and is read
+ * out after the last,
+ *     S <- S D_t;  S <- S (I - b_tj k_tj k_tj^T) + b_tj v_tj k_tj^T;  o_t = S (scale q_t).
+ * That is the gated delta rule on the n*T sub-tokens (t, 1) .. (t, n) with
+ * g_t on the first and q_t read at the last, and it runs as exactly that:
+ * gdn_chunk_fwd / gdn_chunk_bwd over T' = n*T, around device copies that
+ * spread q, g (and dO) over the sub-tokens and gather o (dq, dg) back.
+ * dims->T is the token count; 1 <= n <= 64 and n*T must fit an int.
+ * Layouts (contiguous): q [B,T,H,dk]; k [B,T,n,H,dk]; v [B,T,n,H,dv];
+ * beta [B,T,n,H] fp32; g, h0, hT as in gdn_chunk_fwd; o [B,T,H,dv].  The
+ * gradients take the shapes of their primals.  The workspace holds the inner
+ * call's workspace first, so gdn_query_device_status works on it.
+ * Errors: GDN_ERR_INVALID_ARG for n out of range or a null q, g, o (dO, dq,
+ * dg); otherwise those of gdn_chunk_fwd / gdn_chunk_bwd for T' = n*T. */
+size_t gdn_product_fwd_workspace(const gdn_dims *dims, int n);
+gdn_status gdn_product_fwd(const gdn_dims *dims, int n, const void *q,
+                           const void *k, const void *v, const float *g,
+                           const float *beta, const float *h0, void *o,
+                           float *hT, void *ws, size_t ws_bytes,
+                           gdn_stream_t stream);
+size_t gdn_product_bwd_workspace(const gdn_dims *dims, int n);
+gdn_status gdn_product_bwd(const gdn_dims *dims, int n, const void *q,
+                           const void *k, const void *v, const float *g,
+                           const float *beta, const float *h0, const void *dO,
+                           const float *dhT, void *dq, void *dk, void *dv,
+                           float *dg, float *dbeta, float *dh0, void *ws,
+                           size_t ws_bytes, gdn_stream_t stream);
+
 /* One decode token for N sequences x H heads, in place on the state.
  * q, k [N, H, dk]; v, o [N, H, dv] in `dtype`; g [N, H] (scalar) or
  * [N, H, dk] (channel) fp32; beta [N, H] fp32; state [N, H, dv, dk] fp32,

@@ -3,8 +3,10 @@
 Only ``tests/`` may import this module; the CUDA library never uses it.
 
 Source: "DeltaProduct: Improving State-Tracking in Linear RNNs via
-Householder Products" (listed on the pages by title) and the "Gated Delta
-Networks: Improving Mamba2 with Delta Rule" review, section "Future work",
+Householder Products" (listed by title among the related papers of the
+"Linear Attention Architectures: Mechanisms, Trade-offs, and Cross-Layer
+Routing" summary page) and the "Gated Delta Networks: Improving Mamba2 with
+Delta Rule" review, section "Future work",
 which names products of Householder matrices as an extension of the gated
 delta rule.  The pages give no equation; the reading taken here: each token t
 carries n keys, values and betas, applies its gate once, then performs n

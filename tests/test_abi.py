@@ -113,3 +113,17 @@ def test_workspace_sizes_grow_with_problem():
     b = L.gdn_chunk_bwd_workspace(ctypes.byref(_dims(T=4096)))
     assert 0 < a < b
     assert L.gdn_chunk_fwd_workspace(ctypes.byref(_dims(T=64))) % 4 == 0
+
+
+def test_product_checks():
+    """gdn_product_*: n out of range is rejected on the host (no launch)."""
+    L = gdn.lib()
+    d = gdn.gdn_dims(1, 64, 2, 128, 128, 64, gdn.GDN_BF16, gdn.GDN_GATE_SCALAR, 1.0)
+    assert L.gdn_product_fwd_workspace(ctypes.byref(d), 0) == 0
+    assert L.gdn_product_fwd_workspace(ctypes.byref(d), 65) == 0
+    assert L.gdn_product_fwd_workspace(ctypes.byref(d), 2) > L.gdn_chunk_fwd_workspace(ctypes.byref(d))
+    assert L.gdn_product_bwd_workspace(ctypes.byref(d), 3) > 0
+    p = ctypes.c_void_p(256)
+    for n in (0, 65):
+        assert L.gdn_product_fwd(ctypes.byref(d), n, p, p, p, p, p, None, p, None, p, 1 << 30,
+                                 None) == gdn.GDN_ERR_INVALID_ARG
