@@ -195,3 +195,26 @@ def test_status_word_reports_and_clears(dev):
     ws[0] = 1
     assert gdn.gdn_query_device_status(ws) == gdn.GDN_ERR_DEVICE_TIMEOUT
     assert gdn.gdn_query_device_status(ws) == gdn.GDN_OK
+
+
+@pytest.mark.parametrize("T", [1, 63, 65, 129])
+@pytest.mark.parametrize("cfg,over", [
+    (L350M, dict(B=1, H=3)),          # 16-row walks
+    (L350M, dict(B=3, H=16)),         # whole-head walks
+    (KDA, dict(B=1, H=3)),
+    (KDA, dict(B=3, H=16)),
+])
+def test_tensor_core_edge_lengths(dev, T, cfg, over):
+    """A single token, one token short of / past a chunk, and past two chunks,
+    on both walks and both gates (the tail chunk's padding rows and the
+    one-step chains)."""
+    inp = make_chunk_inputs(cfg, T=T, h0_std=0.2, dhT_std=0.3, seed=900 + T, **over)
+    check_fwd(inp, dev)
+    check_bwd(inp, dev)
+
+
+def test_many_chunks_one_head(dev):
+    """256 chunks in one chain (T = 16384, one head, 16-row walks)."""
+    inp = make_chunk_inputs(L350M, B=1, H=1, T=16384, g_shift=-3.0, h0_std=0.1, dhT_std=0.2)
+    check_fwd(inp, dev)
+    check_bwd(inp, dev)
