@@ -29,7 +29,8 @@ EXPORTS = ("gdn_chunk_fwd_workspace", "gdn_chunk_fwd", "gdn_chunk_bwd_workspace"
            "gdn_chunk_bwd", "gdn_recurrent_step", "gdn_query_device_status",
            "gdn_status_string", "gdn_profile_begin", "gdn_profile_end",
            "gdn_chunk_fwd_noalloc", "gdn_product_fwd_workspace", "gdn_product_fwd",
-           "gdn_product_bwd_workspace", "gdn_product_bwd")
+           "gdn_product_bwd_workspace", "gdn_product_bwd", "gdn_chunk_fwd_varlen_workspace",
+           "gdn_chunk_fwd_varlen", "gdn_chunk_bwd_varlen_workspace", "gdn_chunk_bwd_varlen")
 
 
 class gdn_dims(ctypes.Structure):
@@ -86,6 +87,16 @@ def lib() -> ctypes.CDLL:
             L.gdn_product_bwd.argtypes = [dp, i, vp, vp, vp, fp, fp, fp, vp, fp, vp, vp, vp,
                                           fp, fp, fp, vp, sz, vp]
             L.gdn_product_bwd.restype = i
+            L.gdn_chunk_fwd_varlen_workspace.argtypes = [dp, i]
+            L.gdn_chunk_fwd_varlen_workspace.restype = sz
+            L.gdn_chunk_bwd_varlen_workspace.argtypes = [dp, i]
+            L.gdn_chunk_bwd_varlen_workspace.restype = sz
+            L.gdn_chunk_fwd_varlen.argtypes = [dp, vp, i, vp, vp, vp, fp, fp, fp, vp, fp, vp,
+                                               sz, vp]
+            L.gdn_chunk_fwd_varlen.restype = i
+            L.gdn_chunk_bwd_varlen.argtypes = [dp, vp, i, vp, vp, vp, fp, fp, fp, vp, fp, vp,
+                                               vp, vp, fp, fp, fp, vp, sz, vp]
+            L.gdn_chunk_bwd_varlen.restype = i
             L.gdn_profile_begin.argtypes = [i]
             L.gdn_profile_begin.restype = i
             L.gdn_profile_end.argtypes = [ctypes.POINTER(ctypes.c_float),
@@ -333,4 +344,68 @@ def gdn_product_bwd(q, k, v, g, beta, dO, h0=None, dhT=None, *, chunk=64, scale=
                                nbytes if ws is None else ws.numel() * ws.element_size(),
                                _stream(stream))
     _check(st, "gdn_product_bwd")
+    return out
+
+
+# ---- packed variable-length batches ----------------------------------------
+def _validate_varlen(q, k, v, g, beta, cu_seqlens, h0):
+    import torch
+    B, T, H, dk, dv = _validate_chunk_inputs(q, k, v, g, beta, None)
+    if B != 1:
+        raise ValueError("packed sequences take q [1, total_tokens, H, dk]")
+    _need(cu_seqlens, "cu_seqlens", torch.int32)
+    if cu_seqlens.dim() != 1 or cu_seqlens.numel() < 2:
+        raise ValueError("cu_seqlens must be [nseq + 1] int32")
+    nseq = cu_seqlens.numel() - 1
+    if h0 is not None:
+        _need(h0, "h0", torch.float32, (nseq, H, dv, dk))
+    return nseq, T, H, dk, dv
+
+
+def gdn_chunk_fwd_varlen(q, k, v, g, beta, cu_seqlens, h0=None, *, scale=1.0,
+                         output_final_state=True, workspace=None, stream=None):
+    """Chunkwise forward over packed sequences: q [1,T,H,dk] etc. hold nseq
+    sequences back to back, sequence s at tokens cu_seqlens[s]..cu_seqlens[s+1]-1
+    (cu_seqlens int32 on the device).  h0 / hT are [nseq,H,dv,dk].  Returns
+    (o, hT)."""
+    import torch
+    nseq, T, H, dk, dv = _validate_varlen(q, k, v, g, beta, cu_seqlens, h0)
+    dims = make_dims(q, v, g, 64, scale)
+    o = torch.empty(1, T, H, dv, dtype=q.dtype, device=q.device)
+    hT = torch.empty(nseq, H, dv, dk, dtype=torch.float32, device=q.device) \
+        if output_final_state else None
+    nbytes = int(lib().gdn_chunk_fwd_varlen_workspace(ctypes.byref(dims), nseq))
+    ws = _workspace(nbytes, q.device, workspace)
+    st = lib().gdn_chunk_fwd_varlen(ctypes.byref(dims), _ptr(cu_seqlens), nseq, _ptr(q),
+                                    _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0), _ptr(o),
+                                    _ptr(hT), _ptr(ws),
+                                    nbytes if ws is None else ws.numel() * ws.element_size(),
+                                    _stream(stream))
+    _check(st, "gdn_chunk_fwd_varlen")
+    return o, hT
+
+
+def gdn_chunk_bwd_varlen(q, k, v, g, beta, cu_seqlens, dO, h0=None, dhT=None, *, scale=1.0,
+                         workspace=None, stream=None):
+    """Backward of gdn_chunk_fwd_varlen: gradients in the shapes of their
+    primals (dh0 None when h0 is None)."""
+    import torch
+    nseq, T, H, dk, dv = _validate_varlen(q, k, v, g, beta, cu_seqlens, h0)
+    _need(dO, "dO", q.dtype, (1, T, H, dv))
+    if dhT is not None:
+        _need(dhT, "dhT", torch.float32, (nseq, H, dv, dk))
+    dims = make_dims(q, v, g, 64, scale)
+    out = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dv=torch.empty_like(v),
+               dg=torch.empty_like(g), dbeta=torch.empty_like(beta),
+               dh0=None if h0 is None else torch.empty_like(h0))
+    nbytes = int(lib().gdn_chunk_bwd_varlen_workspace(ctypes.byref(dims), nseq))
+    ws = _workspace(nbytes, q.device, workspace)
+    st = lib().gdn_chunk_bwd_varlen(ctypes.byref(dims), _ptr(cu_seqlens), nseq, _ptr(q),
+                                    _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0), _ptr(dO),
+                                    _ptr(dhT), _ptr(out["dq"]), _ptr(out["dk"]),
+                                    _ptr(out["dv"]), _ptr(out["dg"]), _ptr(out["dbeta"]),
+                                    _ptr(out["dh0"]), _ptr(ws),
+                                    nbytes if ws is None else ws.numel() * ws.element_size(),
+                                    _stream(stream))
+    _check(st, "gdn_chunk_bwd_varlen")
     return out

@@ -38,6 +38,20 @@ bool all_aligned(std::initializer_list<const void*> ps) {
     return true;
 }
 
+// Packed sequences: one row of T tokens in all (B = 1) split by device
+// offsets into nseq sequences; tensor-core shapes only.
+gdn_status check_varlen(const gdn_dims* d, int nseq) {
+    gdn_status s = check_dims(d);
+    if (s != GDN_OK) return s;
+    if (d->B != 1 || nseq < 1) return GDN_ERR_INVALID_ARG;
+    if ((long long)nseq * d->H > 0x7fffffffLL) return GDN_ERR_INVALID_ARG;
+    // chunk slots: ceil(T / 64) + nseq per head must fit an int
+    if ((long long)d->H * ((d->T + 63) / 64 + (long long)nseq) > 0x7fffffffLL)
+        return GDN_ERR_INVALID_ARG;
+    if (!tc_supported(*d)) return GDN_ERR_UNSUPPORTED;
+    return GDN_OK;
+}
+
 gdn_status launch_status() {
     cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
@@ -161,7 +175,61 @@ gdn_status gdn_query_device_status(void* ws, gdn_stream_t stream) {
     const unsigned int zero = 0;
     if (cudaMemcpy(ws, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
         return GDN_ERR_CUDA;
-    return GDN_ERR_DEVICE_TIMEOUT;
+    return (word & 1u) ? GDN_ERR_DEVICE_TIMEOUT : GDN_ERR_INVALID_ARG;
+}
+
+size_t gdn_chunk_fwd_varlen_workspace(const gdn_dims* d, int nseq) {
+    if (check_varlen(d, nseq) != GDN_OK) return 0;
+    return tc_fwd_workspace(*d, nseq);
+}
+
+size_t gdn_chunk_bwd_varlen_workspace(const gdn_dims* d, int nseq) {
+    if (check_varlen(d, nseq) != GDN_OK) return 0;
+    return tc_bwd_workspace(*d, nseq);
+}
+
+gdn_status gdn_chunk_fwd_varlen(const gdn_dims* d, const int* cu_seqlens, int nseq, const void* q,
+                                const void* k, const void* v, const float* g, const float* beta,
+                                const float* h0, void* o, float* hT, void* ws, size_t ws_bytes,
+                                gdn_stream_t stream) {
+    gdn_status s = check_varlen(d, nseq);
+    if (s != GDN_OK) return s;
+    if (!cu_seqlens || ((uintptr_t)cu_seqlens & 3u)) return GDN_ERR_INVALID_ARG;
+    if (!q || !k || !v || !g || !beta || !o) return GDN_ERR_INVALID_ARG;
+    if (!all_aligned({q, k, v, g, beta, h0, o, hT})) return GDN_ERR_INVALID_ARG;
+    if (h0 && hT && h0 == hT) return GDN_ERR_INVALID_ARG;
+    const size_t need = tc_fwd_workspace(*d, nseq);
+    if (!ws || ws_bytes < need || ((uintptr_t)ws & 255u)) return GDN_ERR_WORKSPACE;
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaGetLastError();
+    if (cudaMemsetAsync(ws, 0, sizeof(unsigned int), st) != cudaSuccess) return GDN_ERR_CUDA;
+    if (!launch_tc_fwd(*d, q, k, v, g, beta, h0, o, hT, ws, st, cu_seqlens, nseq))
+        return GDN_ERR_CUDA;
+    return launch_status();
+}
+
+gdn_status gdn_chunk_bwd_varlen(const gdn_dims* d, const int* cu_seqlens, int nseq, const void* q,
+                                const void* k, const void* v, const float* g, const float* beta,
+                                const float* h0, const void* dO, const float* dhT, void* dq,
+                                void* dk, void* dv, float* dg, float* dbeta, float* dh0, void* ws,
+                                size_t ws_bytes, gdn_stream_t stream) {
+    gdn_status s = check_varlen(d, nseq);
+    if (s != GDN_OK) return s;
+    if (!cu_seqlens || ((uintptr_t)cu_seqlens & 3u)) return GDN_ERR_INVALID_ARG;
+    if (!q || !k || !v || !g || !beta || !dO || !dq || !dk || !dv || !dg || !dbeta)
+        return GDN_ERR_INVALID_ARG;
+    if ((h0 == nullptr) != (dh0 == nullptr)) return GDN_ERR_INVALID_ARG;
+    if (!all_aligned({q, k, v, g, beta, h0, dO, dhT, dq, dk, dv, dg, dbeta, dh0}))
+        return GDN_ERR_INVALID_ARG;
+    const size_t need = tc_bwd_workspace(*d, nseq);
+    if (!ws || ws_bytes < need || ((uintptr_t)ws & 255u)) return GDN_ERR_WORKSPACE;
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaGetLastError();
+    if (cudaMemsetAsync(ws, 0, sizeof(unsigned int), st) != cudaSuccess) return GDN_ERR_CUDA;
+    if (!launch_tc_bwd(*d, q, k, v, g, beta, h0, dO, dhT, dq, dk, dv, dg, dbeta, dh0, ws, st,
+                       cu_seqlens, nseq))
+        return GDN_ERR_CUDA;
+    return launch_status();
 }
 
 }  // extern "C"

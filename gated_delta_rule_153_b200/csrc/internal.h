@@ -33,15 +33,22 @@ void launch_simt_bwd(const gdn_dims& d, const void* q, const void* k, const void
 // Tensor-core path (bf16, dk = dv = 128, chunk = 64).
 bool tc_supported(const gdn_dims& d);
 bool tc_bwd_supported(const gdn_dims& d);
-size_t tc_fwd_workspace(const gdn_dims& d);
-size_t tc_bwd_workspace(const gdn_dims& d);
+// nseq > 0: a packed batch of nseq sequences (d.B = 1, d.T tokens in all,
+// device offsets cu[0..nseq]); states are [nseq, H, dv, dk].
+size_t tc_fwd_workspace(const gdn_dims& d, int nseq = 0);
+size_t tc_bwd_workspace(const gdn_dims& d, int nseq = 0);
 // Return false if a TMA tensor map could not be encoded (nothing launched).
 bool launch_tc_fwd(const gdn_dims& d, const void* q, const void* k, const void* v,
                    const float* g, const float* beta, const float* h0, void* o, float* hT,
-                   void* ws, cudaStream_t st);
+                   void* ws, cudaStream_t st, const int* cu = nullptr, int nseq = 0);
 bool launch_tc_bwd(const gdn_dims& d, const void* q, const void* k, const void* v,
                    const float* g, const float* beta, const float* h0, const void* dO,
                    const float* dhT, void* dq, void* dk, void* dv, float* dg, float* dbeta,
-                   float* dh0, void* ws, cudaStream_t st);
+                   float* dh0, void* ws, cudaStream_t st, const int* cu = nullptr, int nseq = 0);
+// Chunk offsets of a packed batch: cstart[s] = sum over s' < s of ceil(len_s' / 64).
+// An offset table that is not non-decreasing from 0 to T sets status bit 1 and
+// yields no chunks.
+void launch_varlen_setup(const int* cu, int nseq, int T, int* cstart, unsigned int* status,
+                         cudaStream_t st);
 
 }  // namespace gdn

@@ -84,18 +84,19 @@ struct W5Ptrs {
     unsigned int* status;
     int B, T, H, NT;
     float scale;
+    SeqMap seq;
 };
 
 template <bool KDA, int MODE>
-__device__ void w5_issue(W5Stage& st, uint64_t* bar, const W5Ptrs& p, int b, int h, int bh, int n) {
-    const size_t cid = (size_t)bh * p.NT + n;
+__device__ void w5_issue(W5Stage& st, uint64_t* bar, const W5Ptrs& p, const Chain& ch, int h, int n) {
+    const size_t cid = (size_t)ch.img * p.NT + ch.n0 + n;  // step n of the chain
     constexpr int GW = KDA ? DK : C;
     constexpr int PANEL = C * 64;  // elements of one 64x64 panel
     mbar_arrive_expect(bar, (MODE == 0 ? 3 * C * DK + C * C : 2 * C * DK) * 2 + GW * 4);
     const __nv_bfloat16* W = p.W + cid * C * DK;
     bulk_g2s(st.WQ, W, PANEL * 2, bar);
     bulk_g2s(st.WQ + 2 * PANEL, W + PANEL, PANEL * 2, bar);
-    const int tok = b * p.T + n * C;
+    const int tok = ch.tok0 + n * C;
     if (MODE == 0) {
         if (KDA) {
             const __nv_bfloat16* Qg = p.Qg + cid * C * DK;
@@ -129,7 +130,9 @@ __global__ void __launch_bounds__(W5_THREADS) tc5_walk_kernel(const __grid_const
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     W5Smem& s = *reinterpret_cast<W5Smem*>(align1k(smem_raw));
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int bh = blockIdx.x, b = bh / p.H, h = bh % p.H;
+    const int bh = blockIdx.x, h = bh % p.H;  // bh: state row (sequence * H + head)
+    const Chain ch = chain_of(p.seq, p.T, p.H, p.NT, bh / p.H, h);
+    const int nsteps = ch.n1 - ch.n0;
 
     if (tid == 0) {
         for (int i = 0; i < W5_STAGES; ++i) {
@@ -153,10 +156,10 @@ __global__ void __launch_bounds__(W5_THREADS) tc5_walk_kernel(const __grid_const
     if (warp == W5_PROD) {
         if (lane == 0) {
             int issued = 0;
-            for (int n = 0; n < p.NT; ++n) {
+            for (int n = 0; n < nsteps; ++n) {
                 const int sn = n % W5_STAGES;
                 if (n >= W5_STAGES && !mbar_wait(&s.empty[sn], ((n / W5_STAGES) - 1) & 1, p.status)) break;
-                w5_issue<KDA, MODE>(s.st[sn], &s.full[sn], p, b, h, bh, n);
+                w5_issue<KDA, MODE>(s.st[sn], &s.full[sn], p, ch, h, n);
                 issued = n + 1;
             }
             // Leave no load in flight (returns at once for stages already consumed).
@@ -167,7 +170,7 @@ __global__ void __launch_bounds__(W5_THREADS) tc5_walk_kernel(const __grid_const
     } else if (warp == W5_CTRL) {
         if (lane == 0) {
             const uint32_t aUs = tm + (KDA ? TAU : TAUS);
-            for (int n = 0; n < p.NT; ++n) {
+            for (int n = 0; n < nsteps; ++n) {
                 const int sn = n % W5_STAGES;
                 W5Stage& st = s.st[sn];
                 if (!mbar_wait(&s.full[sn], (n / W5_STAGES) & 1, p.status)) break;
@@ -222,7 +225,7 @@ __global__ void __launch_bounds__(W5_THREADS) tc5_walk_kernel(const __grid_const
         };
         // MODE 1: bf16 state entering chunk n, Swz<128> image (64 contiguous bytes)
         auto store_s0 = [&](int n) {
-            __nv_bfloat16* dst = p.S0out + ((size_t)bh * p.NT + n) * DV * DK;
+            __nv_bfloat16* dst = p.S0out + ((size_t)ch.img * p.NT + ch.n0 + n) * DV * DK;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const int c = 32 * cg + 8 * j;
@@ -232,20 +235,23 @@ __global__ void __launch_bounds__(W5_THREADS) tc5_walk_kernel(const __grid_const
             }
         };
         store_state();
-        if (MODE == 1) store_s0(0);
+        if (MODE == 1 && nsteps > 0) store_s0(0);
         tc5::fence_before();
         warp_arrive(&s.s_ready);
 
         // U~^T of row a, tokens t0..t0+15: two 16-byte pieces of its Swz<64> row
         const uint32_t uo0 = swz<C>(a, t0), uo1 = swz<C>(a, t0 + 8);
-        const __nv_bfloat16* Ut = p.Ut + (size_t)bh * p.NT * C * DV;
-        uint4 ut0 = *reinterpret_cast<const uint4*>(Ut + uo0);
-        uint4 ut1 = *reinterpret_cast<const uint4*>(Ut + uo1);
+        const __nv_bfloat16* Ut = p.Ut + ((size_t)ch.img * p.NT + ch.n0) * C * DV;
+        uint4 ut0 = make_uint4(0, 0, 0, 0), ut1 = ut0;
+        if (nsteps > 0) {
+            ut0 = *reinterpret_cast<const uint4*>(Ut + uo0);
+            ut1 = *reinterpret_cast<const uint4*>(Ut + uo1);
+        }
 
-        for (int n = 0; n < p.NT; ++n) {
+        for (int n = 0; n < nsteps; ++n) {
             const int sn = n % W5_STAGES;
             const W5Stage& st = s.st[sn];
-            const int L = min(C, p.T - n * C);
+            const int L = min(C, ch.end - (ch.tok0 + n * C));
             if (!wait_all(&s.full[sn], (n / W5_STAGES) & 1, p.status)) break;
             // per-token factors, lane j (mod 16) <-> token t0 + j
             float dec = 1.f, sce = 1.f, gam = 1.f;
@@ -282,7 +288,7 @@ __global__ void __launch_bounds__(W5_THREADS) tc5_walk_kernel(const __grid_const
                 tc5::fence_before();
                 warp_arrive(&s.u_ready);
                 if (MODE == 1) {  // U image, token rows (64 contiguous bytes per warp store)
-                    __nv_bfloat16* dst = p.Uout + ((size_t)bh * p.NT + n) * C * DV;
+                    __nv_bfloat16* dst = p.Uout + ((size_t)ch.img * p.NT + ch.n0 + n) * C * DV;
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
                         const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(&ru[j]);
@@ -291,7 +297,7 @@ __global__ void __launch_bounds__(W5_THREADS) tc5_walk_kernel(const __grid_const
                     }
                 }
             }
-            if (n + 1 < p.NT) {  // next chunk's U~^T, consumed one step later
+            if (n + 1 < nsteps) {  // next chunk's U~^T, consumed one step later
                 const __nv_bfloat16* Un = Ut + (size_t)(n + 1) * C * DV;
                 ut0 = *reinterpret_cast<const uint4*>(Un + uo0);
                 ut1 = *reinterpret_cast<const uint4*>(Un + uo1);
@@ -314,7 +320,7 @@ __global__ void __launch_bounds__(W5_THREADS) tc5_walk_kernel(const __grid_const
             warp_arrive(&s.s_ready);
             if (MODE == 1) {
                 warp_arrive(&s.empty[sn]);
-                if (n + 1 < p.NT) store_s0(n + 1);
+                if (n + 1 < nsteps) store_s0(n + 1);
                 continue;
             }
             // ---- O^T = scale e^{G_i} Y + Z, tokens t0 .. t0+15 of row a ---------
@@ -324,7 +330,7 @@ __global__ void __launch_bounds__(W5_THREADS) tc5_walk_kernel(const __grid_const
                 float z[16];
                 tc5::ld16(z, trow + TZ + t0);
                 tc5::wait_ld();
-                __nv_bfloat16* o = p.o + (((size_t)b * p.T + n * C + t0) * p.H + h) * DV + a;
+                __nv_bfloat16* o = p.o + (((size_t)ch.tok0 + n * C + t0) * p.H + h) * DV + a;
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
                     const float f = KDA ? 1.f : __shfl_sync(0xffffffffu, sce, j);
@@ -366,7 +372,8 @@ void launch_walk5_fwd(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& c, 
     w.qmap = c.qmap; w.kmap = c.kmap;
     w.h0 = h0; w.W = c.W; w.Ut = c.Ut; w.P = c.P; w.G = c.G; w.Qg = c.Qg; w.Kt = c.Kt;
     w.o = (__nv_bfloat16*)o; w.hT = hT; w.status = c.status;
-    w.B = d.B; w.T = d.T; w.H = d.H; w.NT = L.NT; w.scale = d.scale;
+    w.B = chain_batches(d.B, c.seq); w.T = d.T; w.H = d.H; w.NT = L.NT; w.scale = d.scale;
+    w.seq = c.seq;
     if (d.gate == GDN_GATE_CHANNEL) launch_w5<true, 0>(w, st);
     else launch_w5<false, 0>(w, st);
 }
@@ -379,7 +386,8 @@ void launch_walk5_states(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& 
     w.S0out = (__nv_bfloat16*)((char*)ws + L.S0);
     w.Uout = (__nv_bfloat16*)((char*)ws + L.U);
     w.status = c.status;
-    w.B = d.B; w.T = d.T; w.H = d.H; w.NT = L.NT; w.scale = d.scale;
+    w.B = chain_batches(d.B, c.seq); w.T = d.T; w.H = d.H; w.NT = L.NT; w.scale = d.scale;
+    w.seq = c.seq;
     if (d.gate == GDN_GATE_CHANNEL) launch_w5<true, 1>(w, st);
     else launch_w5<false, 1>(w, st);
 }

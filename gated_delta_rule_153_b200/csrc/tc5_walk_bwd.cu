@@ -74,14 +74,15 @@ struct RbPtrs {
     unsigned int* status;
     int B, T, H, NT;
     float scale;
+    SeqMap seq;
 };
 
 template <bool KDA>
-__device__ void rb_issue(RbStage& st, uint64_t* bar, const RbPtrs& p, int b, int h, int bh, int n) {
-    const size_t cid = (size_t)bh * p.NT + n;
+__device__ void rb_issue(RbStage& st, uint64_t* bar, const RbPtrs& p, const Chain& ch, int h, int j) {
+    const size_t cid = (size_t)ch.img * p.NT + ch.n0 + j;  // chunk j of the chain
     constexpr int GW = KDA ? DK : C;
     mbar_arrive_expect(bar, (4 * C * DK + C * C) * 2 + GW * 4);
-    const int tok = b * p.T + n * C;
+    const int tok = ch.tok0 + j * C;
     if (KDA) {
         bulk_g2s(st.Q, p.Qg + cid * C * DK, C * DK * 2, bar);
         bulk_g2s(st.K, p.Kt + cid * C * DK, C * DK * 2, bar);
@@ -109,7 +110,9 @@ __global__ void __launch_bounds__(RB_THREADS) tc5_walk_bwd_kernel(const __grid_c
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     RbSmem& s = *reinterpret_cast<RbSmem*>(align1k(smem_raw));
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int bh = blockIdx.x, b = bh / p.H, h = bh % p.H;
+    const int bh = blockIdx.x, h = bh % p.H;  // bh: state row (sequence * H + head)
+    const Chain ch = chain_of(p.seq, p.T, p.H, p.NT, bh / p.H, h);
+    const int nsteps = ch.n1 - ch.n0;
 
     if (tid == 0) {
         for (int i = 0; i < RB_STAGES; ++i) {
@@ -133,10 +136,10 @@ __global__ void __launch_bounds__(RB_THREADS) tc5_walk_bwd_kernel(const __grid_c
     if (warp == RB_PROD) {
         if (lane == 0) {
             int issued = 0;
-            for (int k = 0; k < p.NT; ++k) {  // step k carries chunk NT-1-k
+            for (int k = 0; k < nsteps; ++k) {  // step k carries chunk nsteps-1-k of the chain
                 const int sk = k % RB_STAGES;
                 if (k >= RB_STAGES && !mbar_wait(&s.empty[sk], ((k / RB_STAGES) - 1) & 1, p.status)) break;
-                rb_issue<KDA>(s.st[sk], &s.full[sk], p, b, h, bh, p.NT - 1 - k);
+                rb_issue<KDA>(s.st[sk], &s.full[sk], p, ch, h, nsteps - 1 - k);
                 issued = k + 1;
             }
             for (int k = max(0, issued - RB_STAGES); k < issued; ++k)
@@ -145,7 +148,7 @@ __global__ void __launch_bounds__(RB_THREADS) tc5_walk_bwd_kernel(const __grid_c
         __syncwarp();
     } else if (warp == RB_CTRL) {
         if (lane == 0) {
-            for (int k = 0; k < p.NT; ++k) {
+            for (int k = 0; k < nsteps; ++k) {
                 const int sk = k % RB_STAGES;
                 RbStage& st = s.st[sk];
                 if (!mbar_wait(&s.full[sk], (k / RB_STAGES) & 1, p.status)) break;
@@ -205,11 +208,11 @@ __global__ void __launch_bounds__(RB_THREADS) tc5_walk_bwd_kernel(const __grid_c
         tc5::fence_before();
         rb_warp_arrive(&s.ds_ready);
 
-        for (int k = 0; k < p.NT; ++k) {
-            const int n = p.NT - 1 - k, sk = k % RB_STAGES;
+        for (int k = 0; k < nsteps; ++k) {
+            const int j = nsteps - 1 - k, sk = k % RB_STAGES;  // chunk j of the chain
             RbStage& st = s.st[sk];
-            const int L = min(C, p.T - n * C);
-            const size_t cid = (size_t)bh * p.NT + n;
+            const int L = min(C, ch.end - (ch.tok0 + j * C));
+            const size_t cid = (size_t)ch.img * p.NT + ch.n0 + j;
             if (!rb_wait_all(&s.full[sk], (k / RB_STAGES) & 1, p.status)) break;
             {   // dS leaving chunk n: bf16 Swz<128> image, 64 contiguous bytes
                 __nv_bfloat16* dst = p.dSout + cid * DV * DK;
@@ -326,7 +329,8 @@ bool launch_walk5_bwd(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& c, 
     p.dSout = (__nv_bfloat16*)((char*)ws + L.dS);
     p.dUout = (__nv_bfloat16*)((char*)ws + L.dU);
     p.dh0 = dh0; p.status = c.status;
-    p.B = d.B; p.T = d.T; p.H = d.H; p.NT = L.NT; p.scale = d.scale;
+    p.B = chain_batches(d.B, c.seq); p.T = d.T; p.H = d.H; p.NT = L.NT; p.scale = d.scale;
+    p.seq = c.seq;
     if (d.gate == GDN_GATE_CHANNEL) launch_rb<true>(p, st);
     else launch_rb<false>(p, st);
     return true;

@@ -35,7 +35,7 @@ void launch_prep_kda(const ChunkPtrs& p, size_t nchunks, cudaStream_t st);
 bool launch_bwd_local_kda(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& cp,
                           const void* dO, void* dq, void* dk, void* dv, float* dg, float* dbeta,
                           void* ws, cudaStream_t st);
-bool whole_head_walk(const gdn_dims& d);
+bool whole_head_walk(const gdn_dims& d, const SeqMap& seq);
 bool launch_walk5_bwd(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& c, const void* dO,
                       const float* dhT, float* dh0, void* ws, cudaStream_t st);
 }  // namespace tc
@@ -85,17 +85,18 @@ struct BwPtrs {
     unsigned int* status;
     int B, T, H, NT;
     float scale;
+    SeqMap seq;
 };
 
 // KDA: Q and K arrive pre-scaled (scale Q .* e^G, K .* e^{G_last-G}) as
 // workspace images, with the per-key chunk decay e^{G_last,c}.
 template <int MT, bool KDA>
-__device__ void bw_issue(BwStage<MT>& st, uint64_t* bar, const BwPtrs& p, int b, int h, int bh,
-                         int n, int a0) {
-    const size_t cid = (size_t)bh * p.NT + n;
+__device__ void bw_issue(BwStage<MT>& st, uint64_t* bar, const BwPtrs& p, const Chain& ch, int h,
+                         int j, int a0) {
+    const size_t cid = (size_t)ch.img * p.NT + ch.n0 + j;  // chunk j of the chain
     constexpr int GW = KDA ? DK : C;
     mbar_arrive_expect(bar, (3 * C * DK + C * C + C * 16 * MT) * 2 + GW * 4);
-    const int tok = b * p.T + n * C;
+    const int tok = ch.tok0 + j * C;
     if (KDA) {
         bulk_g2s(st.Q, p.Qg + cid * C * DK, C * DK * 2, bar);
         bulk_g2s(st.K, p.Kt + cid * C * DK, C * DK * 2, bar);
@@ -117,7 +118,9 @@ __global__ void __launch_bounds__(BW_THREADS) tc_walk_bwd_kernel(const __grid_co
     constexpr int TILES = DV / RT;
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
     const int bh = blockIdx.x / TILES, a0 = (blockIdx.x % TILES) * RT;
-    const int b = bh / p.H, h = bh % p.H;
+    const int h = bh % p.H;  // bh: state row (sequence * H + head)
+    const Chain ch = chain_of(p.seq, p.T, p.H, p.NT, bh / p.H, h);
+    const int nsteps = ch.n1 - ch.n0;
     const int r_lo = lane >> 2;
     const int i0 = 8 * w + 2 * (lane & 3);  // this thread's token pair in dU^T
 
@@ -147,21 +150,21 @@ __global__ void __launch_bounds__(BW_THREADS) tc_walk_bwd_kernel(const __grid_co
     fence_async_smem();
     __syncthreads();
     if (tid == 0)
-        for (int k = 0; k < BW_STAGES - 1 && k < p.NT; ++k)
-            bw_issue<MT, KDA>(s.st[k], &s.full[k], p, b, h, bh, p.NT - 1 - k, a0);
+        for (int k = 0; k < BW_STAGES - 1 && k < nsteps; ++k)
+            bw_issue<MT, KDA>(s.st[k], &s.full[k], p, ch, h, nsteps - 1 - k, a0);
 
-    for (int k = 0; k < p.NT; ++k) {  // step k handles chunk n = NT-1-k
-        const int n = p.NT - 1 - k;
+    for (int k = 0; k < nsteps; ++k) {  // step k handles chunk j = nsteps-1-k of the chain
+        const int j = nsteps - 1 - k;
         const int sk = k % BW_STAGES;
         BwStage<MT>& st = s.st[sk];
         if (__syncthreads_or(!mbar_wait(&s.full[sk], (k / BW_STAGES) & 1, p.status))) return;  // all threads agree; stage landed; dS written; stage of step k-1 is free
-        if (tid == 0 && k + BW_STAGES - 1 < p.NT) {
+        if (tid == 0 && k + BW_STAGES - 1 < nsteps) {
             const int kk = k + BW_STAGES - 1;
-            bw_issue<MT, KDA>(s.st[kk % BW_STAGES], &s.full[kk % BW_STAGES], p, b, h, bh,
-                              p.NT - 1 - kk, a0);
+            bw_issue<MT, KDA>(s.st[kk % BW_STAGES], &s.full[kk % BW_STAGES], p, ch, h,
+                              nsteps - 1 - kk, a0);
         }
-        const size_t cid = (size_t)bh * p.NT + n;
-        const int L = min(C, p.T - n * C);
+        const size_t cid = (size_t)ch.img * p.NT + ch.n0 + j;
+        const int L = min(C, ch.end - (ch.tok0 + j * C));
         if (tid == 0) {  // dS leaving chunk n (Swz<128> image rows a0..)
             bulk_s2g(p.dSout + (cid * DV + a0) * DK, s.dS, RT * DK * 2);
             bulk_commit();
@@ -315,6 +318,7 @@ struct LocPtrs {
     int B, T, H, NT;
     float scale;
     int pf_stride;  // chunks a wave ahead; 0: no prefetch
+    SeqMap seq;
 };
 
 // Row sums over the 4 lanes of a quad: lo -> row r_lo, hi -> row r_lo + 8.
@@ -339,10 +343,11 @@ __global__ void __launch_bounds__(LOC_THREADS) tc_bwd_local_kernel(const __grid_
     const int rb = w >> 2, cq = w & 3;
     const int m0 = 16 * rb;
     const int cid = blockIdx.x;
-    const int bh = cid / p.NT, n = cid % p.NT, b = bh / p.H, h = bh % p.H;
-    const int t0 = n * C;
-    const int L = min(C, p.T - t0);
-    const size_t row0 = ((size_t)b * p.T + t0) * p.H + h;
+    const int bh = cid / p.NT, n = cid % p.NT, h = bh % p.H;
+    const ChunkLoc cl = chunk_loc(p.seq, p.T, p.H, bh, n);
+    if (!cl.valid) return;  // past the last chunk of a packed batch
+    const int L = cl.L;
+    const size_t row0 = (size_t)cl.tok * p.H + h;
     const size_t rs = (size_t)p.H;
     const int rl = m0 + (lane >> 2), rh = rl + 8;  // this thread's two rows
 
@@ -350,7 +355,7 @@ __global__ void __launch_bounds__(LOC_THREADS) tc_bwd_local_kernel(const __grid_
         mbar_init(&s.bar[0], 1);
         mbar_init(&s.bar[1], 1);
         fence_mbar_init();
-        const int tok = b * p.T + t0;
+        const int tok = cl.tok;
         // phase 1 (contractions over the value dimension) needs dO, Q, K, U, dU,
         // S0, dS, G; V and T are first used after it
         mbar_arrive_expect(&s.bar[0], (5 * C * DK + 2 * DV * DK) * 2 + C * 4);
@@ -368,8 +373,9 @@ __global__ void __launch_bounds__(LOC_THREADS) tc_bwd_local_kernel(const __grid_
         // the chunk a wave ahead: its tiles and images wait in L2 when its CTA starts
         const int pc = cid + p.pf_stride;
         if (p.pf_stride > 0 && pc < (int)gridDim.x) {
-            const int pbh = pc / p.NT, pn = pc % p.NT;
-            const int ptok = (pbh / p.H) * p.T + pn * C, ph = pbh % p.H;
+            const int pbh = pc / p.NT, pn = pc % p.NT, ph = pbh % p.H;
+            const ChunkLoc pl = chunk_loc(p.seq, p.T, p.H, pbh, pn);
+            const int ptok = pl.valid ? pl.tok : 0;
             tma_prefetch_tile(&p.dOmap, ph, ptok);
             tma_prefetch_tile(&p.qmap, ph, ptok);
             tma_prefetch_tile(&p.kmap, ph, ptok);
@@ -832,12 +838,13 @@ bool launch_walk_bwd16(const gdn_dims& d, const ChunkPtrs& cp, const void* dO, c
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess)
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const bool two = (long long)d.B * d.H * (DV / 32) >= sms;  // two m-tiles per warp
+    const bool two = (long long)chain_batches(d.B, cp.seq) * d.H * (DV / 32) >= sms;  // two m-tiles per warp
     bp.qmap = cp.qmap; bp.kmap = cp.kmap;
     if (!encode_token_map(&bp.dOmap, dO, d.B, d.T, d.H, two ? 32 : 16)) return false;
     bp.dhT = dhT; bp.W = cp.W; bp.P = cp.P; bp.G = cp.G;
     bp.dh0 = dh0; bp.status = cp.status;
-    bp.B = d.B; bp.T = d.T; bp.H = d.H; bp.NT = cp.NT; bp.scale = d.scale;
+    bp.B = chain_batches(d.B, cp.seq); bp.T = d.T; bp.H = d.H; bp.NT = cp.NT; bp.scale = d.scale;
+    bp.seq = cp.seq;
     bp.Qg = cp.Qg; bp.Kt = cp.Kt;
     const bool kda = d.gate == GDN_GATE_CHANNEL;
     if (two) {
@@ -857,12 +864,17 @@ bool tc_bwd_supported(const gdn_dims& d) { return tc_supported(d); }
 bool launch_tc_bwd(const gdn_dims& d, const void* q, const void* k, const void* v,
                    const float* g, const float* beta, const float* h0, const void* dO,
                    const float* dhT, void* dq, void* dk, void* dv, float* dg, float* dbeta,
-                   float* dh0, void* ws, cudaStream_t st) {
-    const TcLayout L = tc_layout(d, true);
+                   float* dh0, void* ws, cudaStream_t st, const int* cu, int nseq) {
+    const TcLayout L = tc_layout(d, true, nseq);
     char* base = (char*)ws;
     ChunkPtrs cp;
     if (!chunk_ptrs(cp, d, L, q, k, v, g, beta, ws)) return false;
     cp.Tb = (__nv_bfloat16*)(base + L.Tb);
+    if (nseq) {
+        int* cstart = (int*)(base + L.cstart);
+        launch_varlen_setup(cu, nseq, d.T, cstart, cp.status, st);
+        cp.seq = SeqMap{cu, cstart, nseq};
+    }
     const bool kda_gate = d.gate == GDN_GATE_CHANNEL;
     if (kda_gate) launch_prep_kda(cp, L.nchunks, st);
     else launch_prep(cp, L.nchunks, st);
@@ -871,7 +883,7 @@ bool launch_tc_bwd(const gdn_dims& d, const void* q, const void* k, const void* 
     BwPtrs bp{};
     bp.dSout = (__nv_bfloat16*)(base + L.dS);
     bp.dUout = (__nv_bfloat16*)(base + L.dU);
-    if (whole_head_walk(d)) {
+    if (whole_head_walk(d, cp.seq)) {
         if (!launch_walk5_bwd(d, L, cp, dO, dhT, dh0, ws, st)) return false;
     } else if (!launch_walk_bwd16(d, cp, dO, dhT, dh0, bp, st)) {
         return false;
@@ -889,6 +901,7 @@ bool launch_tc_bwd(const gdn_dims& d, const void* q, const void* k, const void* 
     lp.dq = (__nv_bfloat16*)dq; lp.dk = (__nv_bfloat16*)dk; lp.dv = (__nv_bfloat16*)dv;
     lp.dg = dg; lp.dbeta = dbeta;
     lp.B = d.B; lp.T = d.T; lp.H = d.H; lp.NT = L.NT; lp.scale = d.scale;
+    lp.seq = cp.seq;
     {
         const int smem = sizeof(LocSmem) + 1024;
         cudaFuncSetAttribute(tc_bwd_local_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);

@@ -75,11 +75,12 @@ __global__ void __launch_bounds__(128) tc_prep_kernel(const __grid_constant__ Ch
     PrepSmem& s = *reinterpret_cast<PrepSmem*>(align1k(smem_raw));
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int cid = blockIdx.x;
-    const int bh = cid / p.NT, n = cid % p.NT, b = bh / p.H, h = bh % p.H;
-    const int t0 = n * C;
-    const int L = min(C, p.T - t0);
-    const size_t row0 = ((size_t)b * p.T + t0) * p.H + h;  // token-head index of row 0
-    const size_t rs = (size_t)p.H;                        // token-head stride between rows
+    const int bh = cid / p.NT, n = cid % p.NT, h = bh % p.H;
+    const ChunkLoc cl = chunk_loc(p.seq, p.T, p.H, bh, n);
+    if (!cl.valid) return;  // past the last chunk of a packed batch
+    const int L = cl.L;
+    const size_t row0 = (size_t)cl.tok * p.H + h;  // token-head index of row 0
+    const size_t rs = (size_t)p.H;                 // token-head stride between rows
 
     if (tid == 0) {
         mbar_init(&s.bar, 1);
@@ -87,7 +88,7 @@ __global__ void __launch_bounds__(128) tc_prep_kernel(const __grid_constant__ Ch
         // rows past L hold the next sequence's tokens (or zeros past the
         // tensor): finite, and annihilated by beta = 0 on those rows
         mbar_arrive_expect(&s.bar, 3 * C * DK * 2);
-        const int tok = b * p.T + t0;
+        const int tok = cl.tok;
         tma_load_tile(s.K, &p.kmap, h, tok, &s.bar);
         tma_load_tile(s.Q, &p.qmap, h, tok, &s.bar);
         tma_load_tile(s.V, &p.vmap, h, tok, &s.bar);
@@ -315,19 +316,20 @@ struct WalkPtrs {
     unsigned int* status;
     int B, T, H, NT;
     float scale;
+    SeqMap seq;
 };
 
 // KDA: the chunk's Q and K arrive pre-scaled (scale Q .* e^G, K .* e^{G_last-G})
 // as workspace images, with the per-key chunk decay e^{G_last,c}.
 // MODE 1 (state recompute) has no output, so it fetches neither Q nor P.
 template <int MT, int MODE, bool KDA>
-__device__ void walk_issue(WalkStage<MT>& st, uint64_t* bar, const WalkPtrs& p, int b, int h,
-                           int bh, int n, int tile0) {
-    const size_t cid = (size_t)bh * p.NT + n;
+__device__ void walk_issue(WalkStage<MT>& st, uint64_t* bar, const WalkPtrs& p, const Chain& ch,
+                           int h, int k, int tile0) {
+    const size_t cid = (size_t)ch.img * p.NT + ch.n0 + k;  // step k of the chain
     constexpr int GW = KDA ? DK : C;
     constexpr int QP = MODE == 0 ? C * DK + C * C : 0;
     mbar_arrive_expect(bar, (2 * C * DK + QP + MT * C * 16) * 2 + GW * 4);
-    const int tok = b * p.T + n * C;
+    const int tok = ch.tok0 + k * C;
     if (KDA) {
         if (MODE == 0) bulk_g2s(st.Q, p.Qg + cid * C * DK, C * DK * 2, bar);
         bulk_g2s(st.K, p.Kt + cid * C * DK, C * DK * 2, bar);
@@ -349,7 +351,9 @@ __global__ void __launch_bounds__(WALK_THREADS) tc_walk_kernel(const __grid_cons
     constexpr int TILES = DV / RT;
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
     const int bh = blockIdx.x / TILES, tile0 = (blockIdx.x % TILES) * MT, a0 = tile0 * 16;
-    const int b = bh / p.H, h = bh % p.H;
+    const int h = bh % p.H;
+    const Chain ch = chain_of(p.seq, p.T, p.H, p.NT, bh / p.H, h);
+    const int nsteps = ch.n1 - ch.n0;
     const int r_lo = lane >> 2;
     const int i0 = 8 * w + 2 * (lane & 3);  // this thread's token pair in the U/O tiles
 
@@ -378,20 +382,21 @@ __global__ void __launch_bounds__(WALK_THREADS) tc_walk_kernel(const __grid_cons
     if (MODE == 1) fence_async_smem();
     __syncthreads();
     if (tid == 0)
-        for (int n = 0; n < WALK_STAGES - 1 && n < p.NT; ++n)
-            walk_issue<MT, MODE, KDA>(s.st[n], &s.full[n], p, b, h, bh, n, tile0);
+        for (int k = 0; k < WALK_STAGES - 1 && k < nsteps; ++k)
+            walk_issue<MT, MODE, KDA>(s.st[k], &s.full[k], p, ch, h, k, tile0);
 
-    for (int n = 0; n < p.NT; ++n) {
-        const int sn = n % WALK_STAGES;
+    for (int k = 0; k < nsteps; ++k) {  // step k: chunk ch.n0 + k
+        const int sn = k % WALK_STAGES;
         WalkStage<MT>& st = s.st[sn];
-        if (__syncthreads_or(!mbar_wait(&s.full[sn], (n / WALK_STAGES) & 1, p.status))) return;  // all threads agree; stage n landed; S0 written; stage of chunk n-1 is free
-        if (tid == 0 && n + WALK_STAGES - 1 < p.NT) {
-            const int nn = n + WALK_STAGES - 1;
-            walk_issue<MT, MODE, KDA>(s.st[nn % WALK_STAGES], &s.full[nn % WALK_STAGES], p, b, h, bh, nn,
+        if (__syncthreads_or(!mbar_wait(&s.full[sn], (k / WALK_STAGES) & 1, p.status))) return;  // all threads agree; stage k landed; S0 written; stage of step k-1 is free
+        if (tid == 0 && k + WALK_STAGES - 1 < nsteps) {
+            const int kk = k + WALK_STAGES - 1;
+            walk_issue<MT, MODE, KDA>(s.st[kk % WALK_STAGES], &s.full[kk % WALK_STAGES], p, ch, h, kk,
                                 tile0);
         }
-        const int L = min(C, p.T - n * C);
-        const size_t cid = (size_t)bh * p.NT + n;
+        const int tok = ch.tok0 + k * C;
+        const int L = min(C, ch.end - tok);
+        const size_t cid = (size_t)ch.img * p.NT + ch.n0 + k;
         if (MODE == 1 && tid == 0) {  // chunk-start state rows a0.. (Swz<128> image)
             bulk_s2g(p.S0out + (cid * DV + a0) * DK, s.S0, RT * DK * 2);
             bulk_commit();
@@ -498,7 +503,7 @@ __global__ void __launch_bounds__(WALK_THREADS) tc_walk_kernel(const __grid_cons
             const int i = e / PIECES, pc = e % PIECES;
             const uint4 v = *reinterpret_cast<const uint4*>(&s.O[i * RT + 8 * pc]);
             if (MODE == 0) {
-                const size_t row = ((size_t)b * p.T + n * C + i) * p.H + h;
+                const size_t row = ((size_t)tok + i) * p.H + h;
                 *reinterpret_cast<uint4*>(p.o + row * DV + a0 + 8 * pc) = v;
             } else {  // U image, Swz<128>: 16-byte piece at its swizzled position
                 *reinterpret_cast<uint4*>(p.Uout + cid * C * DV + swz<DV>(i, a0 + 8 * pc)) = v;
@@ -567,7 +572,8 @@ WalkPtrs make_walk_ptrs(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& c
     w.qmap = c.qmap; w.kmap = c.kmap;
     w.h0 = h0; w.W = c.W; w.Ut = c.Ut; w.P = c.P; w.G = c.G; w.Qg = c.Qg; w.Kt = c.Kt;
     w.status = c.status;
-    w.B = d.B; w.T = d.T; w.H = d.H; w.NT = L.NT; w.scale = d.scale;
+    w.B = chain_batches(d.B, c.seq); w.T = d.T; w.H = d.H; w.NT = L.NT; w.scale = d.scale;
+    w.seq = c.seq;
     return w;
 }
 
@@ -576,10 +582,10 @@ WalkPtrs make_walk_ptrs(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& c
 namespace tc {
 // The tcgen05 walks carry a whole head per CTA; with few heads the 16-row
 // walks, which spread each head over eight CTAs, fill more SMs.
-bool whole_head_walk(const gdn_dims& d) {
+bool whole_head_walk(const gdn_dims& d, const SeqMap& seq) {
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    return (long long)d.B * d.H * 4 >= sms;
+    return (long long)chain_batches(d.B, seq) * d.H * 4 >= sms;
 }
 
 void launch_prep(const ChunkPtrs& p, size_t nchunks, cudaStream_t st) {
@@ -595,7 +601,7 @@ bool chunk_ptrs(ChunkPtrs& p, const gdn_dims& d, const TcLayout& L, const void* 
 
 void launch_walk_states(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& cp,
                         const float* h0, void* ws, cudaStream_t st) {
-    if (whole_head_walk(d)) {
+    if (whole_head_walk(d, cp.seq)) {
         launch_walk5_states(d, L, cp, h0, ws, st);
         return;
     }
@@ -611,19 +617,68 @@ bool tc_supported(const gdn_dims& d) {
     return d.dtype == GDN_BF16 && d.dk == DK && d.dv == DV && d.chunk == C;
 }
 
-size_t tc_fwd_workspace(const gdn_dims& d) { return tc_layout(d, false).end; }
-size_t tc_bwd_workspace(const gdn_dims& d) { return tc_layout(d, true).end; }
+size_t tc_fwd_workspace(const gdn_dims& d, int nseq) { return tc_layout(d, false, nseq).end; }
+size_t tc_bwd_workspace(const gdn_dims& d, int nseq) { return tc_layout(d, true, nseq).end; }
+
+namespace {
+// One CTA: per-sequence chunk counts over each thread's run of sequences, a
+// block scan of the run totals, then the offsets.
+constexpr int kSetupThreads = 256;
+__global__ void __launch_bounds__(kSetupThreads) varlen_setup_kernel(const int* cu, int nseq, int T,
+                                                                     int* cstart, unsigned int* status) {
+    __shared__ int part[kSetupThreads];
+    __shared__ int bad;
+    const int tid = threadIdx.x;
+    if (tid == 0) bad = (cu[0] != 0 || cu[nseq] != T) ? 1 : 0;
+    __syncthreads();
+    const int per = (nseq + kSetupThreads - 1) / kSetupThreads;
+    const int s0 = min(nseq, tid * per), s1 = min(nseq, s0 + per);
+    int sum = 0;
+    for (int s = s0; s < s1; ++s) {
+        const int len = cu[s + 1] - cu[s];
+        if (len < 0) bad = 1;
+        sum += (max(len, 0) + C - 1) / C;
+    }
+    part[tid] = sum;
+    __syncthreads();
+    for (int o = 1; o < kSetupThreads; o <<= 1) {  // inclusive scan
+        const int x = tid >= o ? part[tid - o] : 0;
+        __syncthreads();
+        part[tid] += x;
+        __syncthreads();
+    }
+    const bool ok = bad == 0;
+    int run = ok ? part[tid] - sum : 0;
+    for (int s = s0; s < s1; ++s) {
+        cstart[s] = run;
+        if (ok) run += (cu[s + 1] - cu[s] + C - 1) / C;
+    }
+    if (tid == kSetupThreads - 1) cstart[nseq] = ok ? part[tid] : 0;
+    if (tid == 0 && !ok && status) atomicOr(status, 2u);
+}
+}  // namespace
+
+void launch_varlen_setup(const int* cu, int nseq, int T, int* cstart, unsigned int* status,
+                         cudaStream_t st) {
+    GDN_LAUNCH("varlen_setup", st,
+               varlen_setup_kernel<<<1, kSetupThreads, 0, st>>>(cu, nseq, T, cstart, status));
+}
 
 bool launch_tc_fwd(const gdn_dims& d, const void* q, const void* k, const void* v,
                    const float* g, const float* beta, const float* h0, void* o, float* hT,
-                   void* ws, cudaStream_t st) {
-    const TcLayout L = tc_layout(d, false);
+                   void* ws, cudaStream_t st, const int* cu, int nseq) {
+    const TcLayout L = tc_layout(d, false, nseq);
     ChunkPtrs cp;
     if (!make_chunk_ptrs(cp, d, L, q, k, v, g, beta, ws)) return false;
+    if (nseq) {  // chains then run one per (packed sequence, head)
+        int* cstart = (int*)((char*)ws + L.cstart);
+        launch_varlen_setup(cu, nseq, d.T, cstart, cp.status, st);
+        cp.seq = SeqMap{cu, cstart, nseq};
+    }
     const bool kda = d.gate == GDN_GATE_CHANNEL;
     if (kda) launch_prep_kda(cp, L.nchunks, st);
     else launch_prep(cp, L.nchunks, st);
-    if (tc::whole_head_walk(d)) {
+    if (tc::whole_head_walk(d, cp.seq)) {
         launch_walk5_fwd(d, L, cp, h0, o, hT, st);
     } else {
         WalkPtrs w = make_walk_ptrs(d, L, cp, h0);

@@ -16,15 +16,18 @@ struct TcLayout {
     int NT;
     size_t nchunks;
     // byte offsets into the workspace
-    size_t W, Ut, P, G, Tb, S0, U, dS, dU, Qg, Kt, end;
+    size_t W, Ut, P, G, Tb, S0, U, dS, dU, Qg, Kt, cstart, end;
 };
 
-inline TcLayout tc_layout(const gdn_dims& d, bool bwd) {
+// nseq > 0: a packed batch of nseq sequences in one row of d.T tokens; the
+// chunk count is bounded by ceil(T / C) + nseq.
+inline TcLayout tc_layout(const gdn_dims& d, bool bwd, int nseq = 0) {
     TcLayout L{};
-    L.NT = (d.T + C - 1) / C;
-    L.nchunks = (size_t)d.B * d.H * L.NT;
+    L.NT = (d.T + C - 1) / C + nseq;
+    L.nchunks = (size_t)(nseq ? 1 : d.B) * d.H * L.NT;
     size_t o = kStatusBytes;
     auto take = [&](size_t bytes) { size_t r = o; o += (bytes + 255) & ~(size_t)255; return r; };
+    if (nseq) L.cstart = take((size_t)(nseq + 1) * 4);
     L.W = take(L.nchunks * C * DK * 2);
     L.Ut = take(L.nchunks * C * DV * 2);
     L.P = take(L.nchunks * C * C * 2);
@@ -42,6 +45,63 @@ inline TcLayout tc_layout(const gdn_dims& d, bool bwd) {
     }
     L.end = o;
     return L;
+}
+
+// Packed variable-length batches.  With `cu` null the batch is B sequences of
+// T tokens and chunk n of (sequence b, head h) has image index (b*H + h)*NT + n.
+// With `cu` set the tokens of N sequences are packed in one row of T tokens
+// (sequence s = tokens cu[s] .. cu[s+1]-1), chunks are numbered over all
+// sequences (cstart[s] = first chunk of s, cstart[N] = their count) and the
+// image index is h*NT + n; NT bounds the chunk count.
+struct SeqMap {
+    const int* cu;      // [N+1] token offsets, or null
+    const int* cstart;  // [N+1] chunk offsets (set on the device from cu)
+    int N;
+};
+
+// Number of sequences the chains run over: B rows of T, or the N packed ones.
+inline int chain_batches(int B, const SeqMap& m) { return m.cu ? m.N : B; }
+
+// Token start and length of chunk n of image row bh, and its sequence.
+struct ChunkLoc {
+    int tok, L, seq;
+    bool valid;
+};
+GDN_DEV ChunkLoc chunk_loc(const SeqMap& m, int T, int H, int bh, int n) {
+    ChunkLoc c;
+    if (!m.cu) {
+        c.seq = bh / H;
+        c.tok = c.seq * T + n * C;
+        c.L = min(C, T - n * C);
+        c.valid = true;
+        return c;
+    }
+    c.valid = n < m.cstart[m.N];
+    if (!c.valid) return c;
+    int lo = 0, hi = m.N - 1;  // the last s with cstart[s] <= n
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (m.cstart[mid] <= n) lo = mid; else hi = mid - 1;
+    }
+    c.seq = lo;
+    c.tok = m.cu[lo] + (n - m.cstart[lo]) * C;
+    c.L = min(C, m.cu[lo + 1] - c.tok);
+    return c;
+}
+
+// The chain of (sequence s, head h): its chunks n0 .. n1-1, their image row,
+// and the first token.  The state of the chain is row s*H + h of h0 / hT.
+struct Chain {
+    int n0, n1, img, tok0, end;  // end: one past the chain's last token
+};
+GDN_DEV Chain chain_of(const SeqMap& m, int T, int H, int NT, int s, int h) {
+    Chain c;
+    if (!m.cu) {
+        c.n0 = 0; c.n1 = NT; c.img = s * H + h; c.tok0 = s * T; c.end = (s + 1) * T;
+    } else {
+        c.n0 = m.cstart[s]; c.n1 = m.cstart[s + 1]; c.img = h; c.tok0 = m.cu[s]; c.end = m.cu[s + 1];
+    }
+    return c;
 }
 
 // Workspace images (written by prep with bulk stores, read back the same way):
@@ -67,6 +127,7 @@ struct ChunkPtrs {
     __nv_bfloat16* Tb;  // optional: bf16 T = (I + A)^{-1} per chunk (backward)
     __nv_bfloat16 *Qg, *Kt;  // channel gate only
     unsigned int* status;
+    SeqMap seq;
 };
 
 // Stage the W and U~ images from a warp's 16-row block of the W = T diag(.) K

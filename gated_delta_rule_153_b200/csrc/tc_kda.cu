@@ -81,17 +81,18 @@ __global__ void __launch_bounds__(KP_THREADS) tc_prep_kda_kernel(const __grid_co
     KdaPrepSmem& s = *reinterpret_cast<KdaPrepSmem*>(align1k(smem_raw));
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int cid = blockIdx.x;
-    const int bh = cid / p.NT, n = cid % p.NT, b = bh / p.H, h = bh % p.H;
-    const int t0 = n * C;
-    const int L = min(C, p.T - t0);
-    const size_t row0 = ((size_t)b * p.T + t0) * p.H + h;
+    const int bh = cid / p.NT, n = cid % p.NT, h = bh % p.H;
+    const ChunkLoc cl = chunk_loc(p.seq, p.T, p.H, bh, n);
+    if (!cl.valid) return;  // past the last chunk of a packed batch
+    const int L = cl.L;
+    const size_t row0 = (size_t)cl.tok * p.H + h;
     const size_t rs = (size_t)p.H;
 
     if (tid == 0) {
         mbar_init(&s.bar, 1);
         fence_mbar_init();
         mbar_arrive_expect(&s.bar, 3 * C * DK * 2);
-        const int tok = b * p.T + t0;
+        const int tok = cl.tok;
         tma_load_tile(s.K, &p.kmap, h, tok, &s.bar);
         tma_load_tile(s.Q, &p.qmap, h, tok, &s.bar);
         tma_load_tile(s.V, &p.vmap, h, tok, &s.bar);
@@ -412,6 +413,7 @@ struct KdaLocPtrs {
     unsigned int* status;
     int B, T, H, NT;
     float scale;
+    SeqMap seq;
 };
 
 using S128 = Swz<128>;
@@ -435,17 +437,18 @@ __global__ void __launch_bounds__(KL_THREADS) tc_bwd_local_kda_kernel(const __gr
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
     const int I = w >> 2, cq = w & 3, m0 = 16 * I;
     const int cid = blockIdx.x;
-    const int bh = cid / p.NT, n = cid % p.NT, b = bh / p.H, h = bh % p.H;
-    const int t0 = n * C;
-    const int L = min(C, p.T - t0);
-    const size_t row0 = ((size_t)b * p.T + t0) * p.H + h;
+    const int bh = cid / p.NT, n = cid % p.NT, h = bh % p.H;
+    const ChunkLoc cl = chunk_loc(p.seq, p.T, p.H, bh, n);
+    if (!cl.valid) return;  // past the last chunk of a packed batch
+    const int L = cl.L;
+    const size_t row0 = (size_t)cl.tok * p.H + h;
     const size_t rs = (size_t)p.H;
     const int rl = m0 + (lane >> 2), rh = rl + 8;
 
     if (tid == 0) {
         for (int i = 0; i < 3; ++i) mbar_init(&s.bar[i], 1);
         fence_mbar_init();
-        const int tok = b * p.T + t0;
+        const int tok = cl.tok;
         // Q, K, dO, U, dU (five 64x128 tiles), S0 (128x128), T (64x64)
         mbar_arrive_expect(&s.bar[0], (5 * C * DK + DV * DK + C * C) * 2);
         tma_load_tile(s.Q, &p.qmap, h, tok, &s.bar[0]);
@@ -953,6 +956,7 @@ bool launch_bwd_local_kda(const gdn_dims& d, const TcLayout& L, const ChunkPtrs&
     lp.dq = (__nv_bfloat16*)dq; lp.dk = (__nv_bfloat16*)dk; lp.dv = (__nv_bfloat16*)dv;
     lp.dg = dg; lp.dbeta = dbeta; lp.status = cp.status;
     lp.B = d.B; lp.T = d.T; lp.H = d.H; lp.NT = L.NT; lp.scale = d.scale;
+    lp.seq = cp.seq;
     const int smem = sizeof(KdaLocSmem) + 1024;
     cudaFuncSetAttribute(tc_bwd_local_kda_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     GDN_LAUNCH("tc_bwd_local_kda", st,

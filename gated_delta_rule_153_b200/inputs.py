@@ -161,3 +161,17 @@ def make_product_inputs(cfg: ChunkConfig, n: int, **over) -> dict:
                 k=sub["k"].reshape(B, T, n, H, c.dk).contiguous(),
                 v=sub["v"].reshape(B, T, n, H, c.dv).contiguous(),
                 beta=sub["beta"].reshape(B, T, n, H).contiguous(), n=n, cfg=c)
+
+
+def make_varlen_inputs(cfg: ChunkConfig, lens, **over) -> dict:
+    """Host tensors for a packed batch of len(lens) sequences of the given
+    token counts: q, k, v, g, beta, dO [1, sum(lens), H, ...] drawn as one
+    row, h0 / dhT [len(lens), H, dv, dk] (when the config draws them) and
+    cu_seqlens [len(lens) + 1] int32 (0, then the running sums)."""
+    lens = [int(n) for n in lens]
+    tok = make_chunk_inputs(cfg, B=1, T=max(1, sum(lens)), **over)
+    c = tok["cfg"]
+    states = make_chunk_inputs(c, B=len(lens), T=1, seed=c.seed + 700)
+    cu = torch.zeros(len(lens) + 1, dtype=torch.int32)
+    cu[1:] = torch.cumsum(torch.tensor(lens, dtype=torch.int64), 0).to(torch.int32)
+    return dict(tok, h0=states["h0"], dhT=states["dhT"], cu_seqlens=cu, lens=lens)

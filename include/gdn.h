@@ -113,6 +113,41 @@ gdn_status gdn_chunk_bwd(const gdn_dims *dims, const void *q, const void *k,
                          float *dh0, void *ws, size_t ws_bytes,
                          gdn_stream_t stream);
 
+/* Packed variable-length batches.  Each sequence of a packed batch is its own
+ * instance of the recurrence of "Gated Delta Networks: Improving Mamba2 with
+ * Delta Rule" (paper review), section "Method": its state starts from its
+ * own h0 (or zero) and no state crosses a sequence boundary, so the result
+ * for sequence s equals gdn_chunk_fwd / gdn_chunk_bwd on that sequence alone.
+ * The tokens of nseq sequences sit back to back in one row: dims->B must be 1
+ * and dims->T is the total token count; sequence s holds tokens
+ * cu_seqlens[s] .. cu_seqlens[s+1]-1 (a device array of nseq + 1 ints,
+ * 4-byte aligned, cu_seqlens[0] = 0, non-decreasing, cu_seqlens[nseq] = T;
+ * empty sequences are allowed and pass h0 through to hT).  q, k, v, g, beta,
+ * o and their gradients take the [1, T, H, ...] layouts above; h0, hT, dhT,
+ * dh0 are [nseq, H, dv, dk].  Chunks never straddle a boundary: each sequence
+ * is cut into chunks of 64 from its own first token.
+ * Tensor-core shapes only (GDN_BF16, dk = dv = 128, chunk = 64), else
+ * GDN_ERR_UNSUPPORTED; nseq < 1 or B != 1 is GDN_ERR_INVALID_ARG.  The offsets
+ * are device data and are checked on the device: offsets that break the rules
+ * above leave the outputs unspecified and make gdn_query_device_status on
+ * this workspace return GDN_ERR_INVALID_ARG.  The workspace depends on nseq. */
+size_t gdn_chunk_fwd_varlen_workspace(const gdn_dims *dims, int nseq);
+gdn_status gdn_chunk_fwd_varlen(const gdn_dims *dims, const int *cu_seqlens,
+                                int nseq, const void *q, const void *k,
+                                const void *v, const float *g,
+                                const float *beta, const float *h0, void *o,
+                                float *hT, void *ws, size_t ws_bytes,
+                                gdn_stream_t stream);
+size_t gdn_chunk_bwd_varlen_workspace(const gdn_dims *dims, int nseq);
+gdn_status gdn_chunk_bwd_varlen(const gdn_dims *dims, const int *cu_seqlens,
+                                int nseq, const void *q, const void *k,
+                                const void *v, const float *g,
+                                const float *beta, const float *h0,
+                                const void *dO, const float *dhT, void *dq,
+                                void *dk, void *dv, float *dg, float *dbeta,
+                                float *dh0, void *ws, size_t ws_bytes,
+                                gdn_stream_t stream);
+
 /* Gated DeltaProduct: "DeltaProduct: Improving State-Tracking in Linear RNNs
  * via Householder Products" (in the list of related papers of the "Linear
  * Attention Architectures: Mechanisms, Trade-offs, and Cross-Layer Routing"
@@ -162,7 +197,8 @@ gdn_status gdn_recurrent_step(int N, int H, int dk, int dv, gdn_dtype dtype,
  * first bytes of a chunkwise workspace.  Each chunkwise call clears that word
  * (a 4-byte memset on its stream) before its kernels run, and a kernel whose
  * bounded device wait gives up sets it, so the answer covers the most recent
- * call on `ws`: GDN_ERR_DEVICE_TIMEOUT if a wait gave up, else GDN_OK. */
+ * call on `ws`: GDN_ERR_DEVICE_TIMEOUT if a wait gave up, GDN_ERR_INVALID_ARG
+ * if the offsets of a packed batch were invalid, else GDN_OK. */
 gdn_status gdn_query_device_status(void *ws, gdn_stream_t stream);
 
 /* Allocation-free chunkwise forward, for callers that cannot call

@@ -127,3 +127,38 @@ def test_product_checks():
     for n in (0, 65):
         assert L.gdn_product_fwd(ctypes.byref(d), n, p, p, p, p, p, None, p, None, p, 1 << 30,
                                  None) == gdn.GDN_ERR_INVALID_ARG
+
+
+def test_varlen_checks():
+    """gdn_chunk_*_varlen: B != 1, nseq < 1 and a null or misaligned offset
+    array are rejected on the host, non-tensor-core shapes are unsupported;
+    the workspace grows with the number of sequences."""
+    L = gdn.lib()
+    d = gdn.gdn_dims(1, 1000, 4, 128, 128, 64, gdn.GDN_BF16, gdn.GDN_GATE_SCALAR, 1.0)
+    w1 = L.gdn_chunk_fwd_varlen_workspace(ctypes.byref(d), 1)
+    w9 = L.gdn_chunk_fwd_varlen_workspace(ctypes.byref(d), 9)
+    assert 0 < w1 < w9
+    assert L.gdn_chunk_bwd_varlen_workspace(ctypes.byref(d), 9) > w9
+    assert L.gdn_chunk_fwd_varlen_workspace(ctypes.byref(d), 0) == 0
+    d2 = gdn.gdn_dims(2, 1000, 4, 128, 128, 64, gdn.GDN_BF16, gdn.GDN_GATE_SCALAR, 1.0)
+    assert L.gdn_chunk_fwd_varlen_workspace(ctypes.byref(d2), 3) == 0
+    f32 = gdn.gdn_dims(1, 1000, 4, 128, 128, 64, gdn.GDN_F32, gdn.GDN_GATE_SCALAR, 1.0)
+    assert L.gdn_chunk_bwd_varlen_workspace(ctypes.byref(f32), 3) == 0
+    p = ctypes.c_void_p(256)
+    ws = 1 << 40
+    fwd = L.gdn_chunk_fwd_varlen
+    assert fwd(ctypes.byref(d), p, 0, p, p, p, p, p, None, p, None, p, ws, None) == \
+        gdn.GDN_ERR_INVALID_ARG
+    assert fwd(ctypes.byref(d2), p, 3, p, p, p, p, p, None, p, None, p, ws, None) == \
+        gdn.GDN_ERR_INVALID_ARG
+    assert fwd(ctypes.byref(d), None, 3, p, p, p, p, p, None, p, None, p, ws, None) == \
+        gdn.GDN_ERR_INVALID_ARG
+    assert fwd(ctypes.byref(d), ctypes.c_void_p(258), 3, p, p, p, p, p, None, p, None, p, ws,
+               None) == gdn.GDN_ERR_INVALID_ARG
+    assert fwd(ctypes.byref(f32), p, 3, p, p, p, p, p, None, p, None, p, ws, None) == \
+        gdn.GDN_ERR_UNSUPPORTED
+    assert fwd(ctypes.byref(d), p, 3, p, p, p, p, p, None, p, None, p, 16, None) == \
+        gdn.GDN_ERR_WORKSPACE
+    bwd = L.gdn_chunk_bwd_varlen
+    assert bwd(ctypes.byref(d), p, 3, p, p, p, p, p, p, p, None, p, p, p, p, p, None, p, ws,
+               None) == gdn.GDN_ERR_INVALID_ARG  # dh0 without h0
