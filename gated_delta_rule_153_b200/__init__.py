@@ -30,7 +30,8 @@ EXPORTS = ("gdn_chunk_fwd_workspace", "gdn_chunk_fwd", "gdn_chunk_bwd_workspace"
            "gdn_status_string", "gdn_profile_begin", "gdn_profile_end",
            "gdn_chunk_fwd_noalloc", "gdn_product_fwd_workspace", "gdn_product_fwd",
            "gdn_product_bwd_workspace", "gdn_product_bwd", "gdn_chunk_fwd_varlen_workspace",
-           "gdn_chunk_fwd_varlen", "gdn_chunk_bwd_varlen_workspace", "gdn_chunk_bwd_varlen")
+           "gdn_chunk_fwd_varlen", "gdn_chunk_bwd_varlen_workspace", "gdn_chunk_bwd_varlen",
+           "gdn_tree_verify", "gdn_tree_commit")
 
 
 class gdn_dims(ctypes.Structure):
@@ -97,6 +98,12 @@ def lib() -> ctypes.CDLL:
             L.gdn_chunk_bwd_varlen.argtypes = [dp, vp, i, vp, vp, vp, fp, fp, fp, vp, fp, vp,
                                                vp, vp, fp, fp, fp, vp, sz, vp]
             L.gdn_chunk_bwd_varlen.restype = i
+            L.gdn_tree_verify.argtypes = [i, i, i, i, i, i, i, f, vp, vp, vp, vp, fp, fp, fp,
+                                          vp, vp, vp]
+            L.gdn_tree_verify.restype = i
+            L.gdn_tree_commit.argtypes = [i, i, i, i, i, i, i, vp, vp, vp, vp, fp, fp, fp, vp,
+                                          vp]
+            L.gdn_tree_commit.restype = i
             L.gdn_profile_begin.argtypes = [i]
             L.gdn_profile_begin.restype = i
             L.gdn_profile_end.argtypes = [ctypes.POINTER(ctypes.c_float),
@@ -409,3 +416,56 @@ def gdn_chunk_bwd_varlen(q, k, v, g, beta, cu_seqlens, dO, h0=None, dhT=None, *,
                                     _stream(stream))
     _check(st, "gdn_chunk_bwd_varlen")
     return out
+
+
+# ---- draft-tree verification and commit ------------------------------------
+def _validate_tree(parent, k, v, g, beta, state):
+    import torch
+    _need(parent, "parent", torch.int32)
+    if parent.dim() != 2:
+        raise ValueError("parent must be [N, M] int32")
+    N, M = parent.shape
+    _need(k, "k")
+    if k.dim() != 4 or tuple(k.shape[:2]) != (N, M):
+        raise ValueError("k must be [N, M, H, dk]")
+    H, dk = k.shape[2], k.shape[3]
+    _need(v, "v", k.dtype)
+    if v.dim() != 4 or tuple(v.shape[:3]) != (N, M, H):
+        raise ValueError("v must be [N, M, H, dv]")
+    dv = v.shape[3]
+    gate = GDN_GATE_CHANNEL if g.dim() == 4 else GDN_GATE_SCALAR
+    _need(g, "g", torch.float32)
+    if tuple(g.shape[:3]) != (N, M, H):
+        raise ValueError("g must be [N, M, H]")
+    _need(beta, "beta", torch.float32, (N, M, H))
+    _need(state, "state", torch.float32, (N, H, dv, dk))
+    return N, M, H, dk, dv, gate
+
+
+def gdn_tree_verify(parent, q, k, v, g, beta, state, *, scale=1.0, o=None, status=None,
+                    stream=None):
+    """Outputs of every draft-tree node: o [N,M,H,dv], node i read out after
+    the tokens of its root path, from ``state`` [N,H,dv,dk] (not modified)."""
+    import torch
+    N, M, H, dk, dv, gate = _validate_tree(parent, k, v, g, beta, state)
+    _need(q, "q", k.dtype, tuple(k.shape))
+    if o is None:
+        o = torch.empty(N, M, H, dv, dtype=q.dtype, device=q.device)
+    st = lib().gdn_tree_verify(N, M, H, dk, dv, _dtype_code(q), gate, float(scale),
+                               _ptr(parent), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                               _ptr(state), _ptr(o), _ptr(status), _stream(stream))
+    _check(st, "gdn_tree_verify")
+    return o
+
+
+def gdn_tree_commit(parent, accepted, k, v, g, beta, state, *, status=None, stream=None):
+    """In place on ``state``: the state after the root path of node
+    accepted[n] (int32 [N]; -1 leaves state[n] as it is)."""
+    import torch
+    N, M, H, dk, dv, gate = _validate_tree(parent, k, v, g, beta, state)
+    _need(accepted, "accepted", torch.int32, (N,))
+    st = lib().gdn_tree_commit(N, M, H, dk, dv, _dtype_code(k), gate, _ptr(parent),
+                               _ptr(accepted), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                               _ptr(state), _ptr(status), _stream(stream))
+    _check(st, "gdn_tree_commit")
+    return state

@@ -1,0 +1,465 @@
+// tree.cu -- draft-tree verification and commit for the gated delta rule.
+//
+// "TreeWY: Speculative Verification for Gated DeltaNet Hybrids" (paper list
+// of the "Linear Attention Architectures: Mechanisms, Trade-offs, and
+// Cross-Layer Routing" summary page): score every node of a speculative draft
+// tree against the committed state with one triangular solve instead of one
+// state snapshot per node, and rebuild only the accepted state on commit.
+//
+// A tree of M <= 64 nodes hangs below the committed state S0 of each
+// (sequence, head); parent[i] in [-1, i) (-1: S0 itself).  Node i's output is
+// the gated delta rule ("Gated Delta Networks: Improving Mamba2 with Delta
+// Rule", section "Method") run from S0 over its root path.  With G_i the sum
+// of g over the root path of i (inclusive) and anc(i) its strict ancestors,
+// the chunkwise algebra of that review carries over with the causal mask
+// replaced by the ancestor relation:
+//     A_ij = beta_i e^{G_i - G_j} k_i.k_j        (j in anc(i), else 0)
+//     T    = (I + A)^{-1}                         (lower triangular: parents first)
+//     W    = T diag(beta e^G) K,   U~ = T diag(beta) V,   U = U~ - W S0^T
+//     P_ij = scale e^{G_i - G_j} q_i.k_j          (j in anc(i) or j = i)
+//     O    = scale diag(e^G) Q S0^T + P U.
+// Row i of U is the delta-rule correction u_i of node i given the state at its
+// parent, so O_i is exactly node i's read-out.  Commit runs the recurrent form
+// along the accepted node's root path on the fp32 state: one read and one
+// write of each state row.
+#include <math.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "mma.cuh"
+
+namespace gdn {
+namespace {
+
+constexpr int TD = 128;           // d_k = d_v
+constexpr int TREE_THREADS = 256;  // 8 warps
+constexpr int kMaxTreeNodes = 64;
+
+template <int MP>
+struct TreeSmem {
+    __nv_bfloat16 K[MP * TD];  // Swz<128>; rows of U (value index as column) once W is built
+    __nv_bfloat16 Q[MP * TD];
+    __nv_bfloat16 V[MP * TD];
+    union {
+        float A[MP][MP + 1];          // masked, decayed beta K K^T
+        __nv_bfloat16 Wn[MP * TD];    // -W, Swz<128>
+    };
+    float T[MP][MP + 1];              // (I + A)^{-1}
+    alignas(128) __nv_bfloat16 Tw[MP * 64];  // T diag(beta e^G), Swz<64> (columns < MP used)
+    __nv_bfloat16 Tu[MP * 64];        // T diag(beta)
+    __nv_bfloat16 P[MP * 64];
+    float G[MP], g[MP], beta[MP];
+    unsigned long long anc[MP];
+    int par[MP];
+};
+
+// One CTA per (sequence n, head h).  MB = number of 16-node blocks.
+template <int MB>
+__global__ void __launch_bounds__(TREE_THREADS)
+tree_verify_kernel(int M, int H, float scale, const int* __restrict__ parent,
+                   const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
+                   const __nv_bfloat16* __restrict__ v, const float* __restrict__ g,
+                   const float* __restrict__ beta, const float* __restrict__ state,
+                   __nv_bfloat16* __restrict__ o, unsigned int* status) {
+    constexpr int MP = 16 * MB;
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    TreeSmem<MP>& s = *reinterpret_cast<TreeSmem<MP>*>(smem_raw);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int nh = blockIdx.x, n = nh / H, h = nh % H;
+    const size_t rs = (size_t)H * TD;                        // token row stride
+    const size_t row0 = ((size_t)n * M * H + h) * TD;       // node 0 of (n, h)
+
+    // ---- loads: node tokens into shared tiles, the state into registers ----
+    load_tile_async<TD>(s.K, k + row0, rs, MP, M, tid, TREE_THREADS);
+    load_tile_async<TD>(s.Q, q + row0, rs, MP, M, tid, TREE_THREADS);
+    load_tile_async<TD>(s.V, v + row0, rs, MP, M, tid, TREE_THREADS);
+    cp_async_commit();
+    if (tid < MP) {
+        int p = -1;
+        float gi = 0.f, bi = 0.f;
+        if (tid < M) {
+            p = parent[(size_t)n * M + tid];
+            if (p < -1 || p >= tid) {  // not a tree in topological order
+                if (status) atomicOr(status, 2u);
+                p = -1;
+            }
+            gi = g[((size_t)n * M + tid) * H + h];
+            bi = beta[((size_t)n * M + tid) * H + h];
+        }
+        s.par[tid] = p;
+        s.g[tid] = gi;
+        s.beta[tid] = bi;
+    }
+    // B fragments of S0^T for this warp's 16 value rows a0.. (B[k = c][n = a] = S0[a][c]).
+    const int a0 = 16 * warp;
+    uint32_t sf[2][8][2];
+    {
+        const float* S0 = state + (size_t)nh * TD * TD;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            const float* row = S0 + (size_t)(a0 + 8 * nt + (lane >> 2)) * TD + 2 * (lane & 3);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const float2 x = __ldcs(reinterpret_cast<const float2*>(row + 16 * kk));
+                const float2 y = __ldcs(reinterpret_cast<const float2*>(row + 16 * kk + 8));
+                sf[nt][kk][0] = pack_bf16(x.x, x.y);
+                sf[nt][kk][1] = pack_bf16(y.x, y.y);
+            }
+        }
+    }
+    cp_async_wait<0>();
+    __syncthreads();
+
+    // ---- path sums of g and ancestor sets (parents precede children) ------
+    if (tid < MP) {
+        float Gi = s.g[tid];
+        unsigned long long m = 0;
+        for (int j = s.par[tid]; j >= 0; j = s.par[j]) {
+            m |= 1ull << j;
+            Gi += s.g[j];
+        }
+        s.G[tid] = Gi;
+        s.anc[tid] = m;
+    }
+    __syncthreads();
+
+    // ---- A (warps 0-3) and P (warps 4-7): 16 node rows each -----------------
+    {
+        const int mat = warp >> 2, mb = warp & 3;
+        if (mb < MB) {
+            float acc[2 * MB][4];
+#pragma unroll
+            for (int t = 0; t < 2 * MB; ++t)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) acc[t][e] = 0.f;
+#pragma unroll
+            for (int kk = 0; kk < TD / 16; ++kk) {
+                uint32_t a[4];
+                lda<TD>(a, mat ? s.Q : s.K, 16 * mb, 16 * kk);
+#pragma unroll
+                for (int np = 0; np < MB; ++np) {
+                    uint32_t b[4];
+                    ldb_nk<TD>(b, s.K, 16 * np, 16 * kk);
+                    mma16816(acc[2 * np], a, b[0], b[1]);
+                    mma16816(acc[2 * np + 1], a, b[2], b[3]);
+                }
+            }
+#pragma unroll
+            for (int t = 0; t < 2 * MB; ++t)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int i = 16 * mb + (lane >> 2) + 8 * (e >> 1);
+                    const int j = 8 * t + 2 * (lane & 3) + (e & 1);
+                    const bool is_anc = (s.anc[i] >> j) & 1ull;
+                    if (mat == 0) {
+                        s.A[i][j] = is_anc ? s.beta[i] * __expf(s.G[i] - s.G[j]) * acc[t][e] : 0.f;
+                    } else {
+                        const float pv = (is_anc || j == i) ? scale * __expf(s.G[i] - s.G[j]) * acc[t][e] : 0.f;
+                        s.P[swz<64>(i, j)] = __float2bfloat16_rn(pv);
+                    }
+                }
+        }
+    }
+    __syncthreads();
+
+    // ---- T = (I + A)^{-1} by forward substitution, 4 lanes per column -------
+    {
+        const int c = tid >> 2, part = tid & 3;
+        if (c < MP) {  // whole warps: 8 columns each
+            for (int i = 0; i < MP; ++i) {
+                float sum = 0.f;
+                for (int j = c + part; j < i; j += 4) sum += s.A[i][j] * s.T[j][c];
+                sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+                sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+                if (part == 0) s.T[i][c] = i == c ? 1.f : (i > c ? -sum : 0.f);
+                __syncwarp();
+            }
+        }
+    }
+    __syncthreads();
+    for (int e = tid; e < MP * MP; e += TREE_THREADS) {
+        const int i = e / MP, j = e % MP;
+        const float t = s.T[i][j] * s.beta[j];
+        s.Tw[swz<64>(i, j)] = __float2bfloat16_rn(t * __expf(s.G[j]));
+        s.Tu[swz<64>(i, j)] = __float2bfloat16_rn(t);
+    }
+    __syncthreads();
+
+    // ---- -W = -T diag(beta e^G) K: 16 node rows x 64 key columns per warp ----
+    {
+        const int mb = warp & 3, c0 = 64 * (warp >> 2);
+        if (mb < MB) {
+            float acc[8][4];
+#pragma unroll
+            for (int t = 0; t < 8; ++t)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) acc[t][e] = 0.f;
+#pragma unroll
+            for (int kk = 0; kk < MB; ++kk) {
+                uint32_t a[4];
+                lda<64>(a, s.Tw, 16 * mb, 16 * kk);
+#pragma unroll
+                for (int np = 0; np < 4; ++np) {
+                    uint32_t b[4];
+                    ldb_kn<TD>(b, s.K, 16 * kk, c0 + 16 * np);
+                    mma16816(acc[2 * np], a, b[0], b[1]);
+                    mma16816(acc[2 * np + 1], a, b[2], b[3]);
+                }
+            }
+#pragma unroll
+            for (int t = 0; t < 8; ++t) {
+                float ng[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) ng[e] = -acc[t][e];
+                st_c<TD>(s.Wn, 16 * mb, c0 + 8 * t, ng);
+            }
+        }
+    }
+    __syncthreads();  // K is read for the last time above; U takes its place
+
+    // ---- U = U~ - W S0^T and O = scale e^G Q S0^T + P U, value rows a0..a0+15 ----
+    __nv_bfloat16* Ub = s.K;
+    float acco[MB][2][4];
+#pragma unroll
+    for (int mb = 0; mb < MB; ++mb) {
+        float u[2][4];
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) { u[nt][e] = 0.f; acco[mb][nt][e] = 0.f; }
+#pragma unroll
+        for (int kk = 0; kk <= mb; ++kk) {  // T is lower triangular
+            uint32_t a[4], b[4];
+            lda<64>(a, s.Tu, 16 * mb, 16 * kk);
+            ldb_kn<TD>(b, s.V, 16 * kk, a0);
+            mma16816(u[0], a, b[0], b[1]);
+            mma16816(u[1], a, b[2], b[3]);
+        }
+#pragma unroll
+        for (int kk = 0; kk < TD / 16; ++kk) {
+            uint32_t a[4];
+            lda<TD>(a, s.Wn, 16 * mb, 16 * kk);
+            mma16816(u[0], a, sf[0][kk][0], sf[0][kk][1]);
+            mma16816(u[1], a, sf[1][kk][0], sf[1][kk][1]);
+            lda<TD>(a, s.Q, 16 * mb, 16 * kk);
+            mma16816(acco[mb][0], a, sf[0][kk][0], sf[0][kk][1]);
+            mma16816(acco[mb][1], a, sf[1][kk][0], sf[1][kk][1]);
+        }
+        st_c<TD>(Ub, 16 * mb, a0, u[0]);
+        st_c<TD>(Ub, 16 * mb, a0 + 8, u[1]);
+        const int r = 16 * mb + (lane >> 2);
+        const float f0 = scale * __expf(s.G[r]), f1 = scale * __expf(s.G[r + 8]);
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            acco[mb][nt][0] *= f0; acco[mb][nt][1] *= f0;
+            acco[mb][nt][2] *= f1; acco[mb][nt][3] *= f1;
+        }
+    }
+    __syncwarp();  // this warp's U columns, written above, are all it reads below
+#pragma unroll
+    for (int mb = 0; mb < MB; ++mb) {
+#pragma unroll
+        for (int kk = 0; kk <= mb; ++kk) {  // P is lower triangular
+            uint32_t a[4], b[4];
+            lda<64>(a, s.P, 16 * mb, 16 * kk);
+            ldb_kn<TD>(b, Ub, 16 * kk, a0);
+            mma16816(acco[mb][0], a, b[0], b[1]);
+            mma16816(acco[mb][1], a, b[2], b[3]);
+        }
+        const int r = 16 * mb + (lane >> 2);
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            const int col = a0 + 8 * nt + 2 * (lane & 3);
+            if (r < M)
+                *reinterpret_cast<uint32_t*>(o + row0 + (size_t)r * rs + col) =
+                    pack_bf16(acco[mb][nt][0], acco[mb][nt][1]);
+            if (r + 8 < M)
+                *reinterpret_cast<uint32_t*>(o + row0 + (size_t)(r + 8) * rs + col) =
+                    pack_bf16(acco[mb][nt][2], acco[mb][nt][3]);
+        }
+    }
+}
+
+// ---- commit: the recurrent form along the accepted node's root path --------
+struct CommitSmem {
+    float k[kMaxTreeNodes][TD];  // keys of the path tokens, in path order
+    float v[kMaxTreeNodes][TD];
+    float alpha[kMaxTreeNodes], beta[kMaxTreeNodes];
+    int path[kMaxTreeNodes];
+    int len;
+};
+
+// One CTA per (n, h); a state row is covered by 8 lanes of 16 columns each
+// (column 4*(sub + 8j) + e), and each thread keeps four rows in registers for
+// the whole path: one streaming read and one streaming write per element.
+__global__ void __launch_bounds__(TREE_THREADS)
+tree_commit_kernel(int M, int H, const int* __restrict__ parent, const int* __restrict__ accepted,
+                   const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
+                   const float* __restrict__ g, const float* __restrict__ beta,
+                   float* __restrict__ state, unsigned int* status) {
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    CommitSmem& s = *reinterpret_cast<CommitSmem*>(smem_raw);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int nh = blockIdx.x, n = nh / H, h = nh % H;
+    if (tid == 0) {
+        int a = accepted[n];
+        if (a < -1 || a >= M) {
+            if (status) atomicOr(status, 2u);
+            a = -1;
+        }
+        int len = 0;
+        for (int j = a; j >= 0 && len < kMaxTreeNodes;) {  // leaf to root
+            s.path[len++] = j;
+            const int p = parent[(size_t)n * M + j];
+            if (p < -1 || p >= j) {
+                if (status) atomicOr(status, 2u);
+                break;  // an invalid parent reads as -1, as in verification
+            }
+            j = p;
+        }
+        for (int x = 0; x < len / 2; ++x) {  // root to leaf
+            const int t = s.path[x];
+            s.path[x] = s.path[len - 1 - x];
+            s.path[len - 1 - x] = t;
+        }
+        s.len = len;
+    }
+    __syncthreads();
+    const int len = s.len;
+    if (len == 0) return;  // nothing accepted: the state stays as it is
+    for (int e = tid; e < len * TD; e += TREE_THREADS) {
+        const int p = e / TD, c = e % TD;
+        const size_t row = (((size_t)n * M + s.path[p]) * H + h) * TD;
+        s.k[p][c] = __bfloat162float(k[row + c]);
+        s.v[p][c] = __bfloat162float(v[row + c]);
+    }
+    if (tid < len) {
+        const size_t i = ((size_t)n * M + s.path[tid]) * H + h;
+        s.alpha[tid] = __expf(g[i]);
+        s.beta[tid] = beta[i];
+    }
+    float* S = state + (size_t)nh * TD * TD;
+    const int sub = lane & 7, grp = lane >> 3;
+    float4 st[4][4];
+#pragma unroll
+    for (int rr = 0; rr < 4; ++rr) {
+        const float4* src = reinterpret_cast<const float4*>(S + (size_t)(32 * rr + 4 * warp + grp) * TD);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) st[rr][j] = __ldcs(src + sub + 8 * j);
+    }
+    __syncthreads();
+    for (int p = 0; p < len; ++p) {
+        float kr[16];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float4 x = *reinterpret_cast<const float4*>(&s.k[p][4 * (sub + 8 * j)]);
+            kr[4 * j] = x.x; kr[4 * j + 1] = x.y; kr[4 * j + 2] = x.z; kr[4 * j + 3] = x.w;
+        }
+        const float al = s.alpha[p], be = s.beta[p];
+#pragma unroll
+        for (int rr = 0; rr < 4; ++rr) {
+            float dot = 0.f;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                st[rr][j].x *= al; st[rr][j].y *= al; st[rr][j].z *= al; st[rr][j].w *= al;
+                dot += st[rr][j].x * kr[4 * j] + st[rr][j].y * kr[4 * j + 1] +
+                       st[rr][j].z * kr[4 * j + 2] + st[rr][j].w * kr[4 * j + 3];
+            }
+            dot += __shfl_xor_sync(0xffffffffu, dot, 1);
+            dot += __shfl_xor_sync(0xffffffffu, dot, 2);
+            dot += __shfl_xor_sync(0xffffffffu, dot, 4);
+            const float u = be * (s.v[p][32 * rr + 4 * warp + grp] - dot);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                st[rr][j].x += u * kr[4 * j]; st[rr][j].y += u * kr[4 * j + 1];
+                st[rr][j].z += u * kr[4 * j + 2]; st[rr][j].w += u * kr[4 * j + 3];
+            }
+        }
+    }
+#pragma unroll
+    for (int rr = 0; rr < 4; ++rr) {
+        float4* dst = reinterpret_cast<float4*>(S + (size_t)(32 * rr + 4 * warp + grp) * TD);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) __stcs(dst + sub + 8 * j, st[rr][j]);
+    }
+}
+
+template <int MB>
+void launch_verify(int N, int M, int H, float scale, const int* parent, const void* q,
+                   const void* k, const void* v, const float* g, const float* beta,
+                   const float* state, void* o, unsigned int* status, cudaStream_t st) {
+    const int smem = sizeof(TreeSmem<16 * MB>);
+    cudaFuncSetAttribute(tree_verify_kernel<MB>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    GDN_LAUNCH("tree_verify", st,
+               (tree_verify_kernel<MB><<<(unsigned)(N * H), TREE_THREADS, smem, st>>>(
+                   M, H, scale, parent, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k,
+                   (const __nv_bfloat16*)v, g, beta, state, (__nv_bfloat16*)o, status)));
+}
+
+bool aligned(const void* p, unsigned a) { return ((uintptr_t)p & (a - 1)) == 0; }
+
+gdn_status check_tree(int N, int M, int H, int dk, int dv, gdn_dtype dtype, gdn_gate gate) {
+    if (N < 1 || H < 1 || M < 1) return GDN_ERR_INVALID_ARG;
+    if ((long long)N * H > 0x7fffffffLL) return GDN_ERR_INVALID_ARG;
+    if (dtype != GDN_BF16 && dtype != GDN_F32) return GDN_ERR_INVALID_ARG;
+    if (gate != GDN_GATE_SCALAR && gate != GDN_GATE_CHANNEL) return GDN_ERR_INVALID_ARG;
+    if (M > kMaxTreeNodes) return GDN_ERR_UNSUPPORTED;
+    if (dtype != GDN_BF16 || gate != GDN_GATE_SCALAR || dk != TD || dv != TD)
+        return GDN_ERR_UNSUPPORTED;
+    return GDN_OK;
+}
+
+gdn_status launched() { return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA; }
+
+}  // namespace
+}  // namespace gdn
+
+extern "C" {
+
+gdn_status gdn_tree_verify(int N, int M, int H, int dk, int dv, gdn_dtype dtype, gdn_gate gate,
+                           float scale, const int* parent, const void* q, const void* k,
+                           const void* v, const float* g, const float* beta, const float* state,
+                           void* o, unsigned int* status, gdn_stream_t stream) {
+    using namespace gdn;
+    const gdn_status s = check_tree(N, M, H, dk, dv, dtype, gate);
+    if (s != GDN_OK) return s;
+    if (!isfinite(scale)) return GDN_ERR_INVALID_ARG;
+    if (!parent || !q || !k || !v || !g || !beta || !state || !o) return GDN_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(state, 16) ||
+        !aligned(o, 16) || !aligned(parent, 4) || !aligned(g, 4) || !aligned(beta, 4) ||
+        !aligned(status, 4))
+        return GDN_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaGetLastError();
+    switch ((M + 15) / 16) {
+        case 1: launch_verify<1>(N, M, H, scale, parent, q, k, v, g, beta, state, o, status, st); break;
+        case 2: launch_verify<2>(N, M, H, scale, parent, q, k, v, g, beta, state, o, status, st); break;
+        case 3: launch_verify<3>(N, M, H, scale, parent, q, k, v, g, beta, state, o, status, st); break;
+        default: launch_verify<4>(N, M, H, scale, parent, q, k, v, g, beta, state, o, status, st); break;
+    }
+    return launched();
+}
+
+gdn_status gdn_tree_commit(int N, int M, int H, int dk, int dv, gdn_dtype dtype, gdn_gate gate,
+                           const int* parent, const int* accepted, const void* k, const void* v,
+                           const float* g, const float* beta, float* state, unsigned int* status,
+                           gdn_stream_t stream) {
+    using namespace gdn;
+    const gdn_status s = check_tree(N, M, H, dk, dv, dtype, gate);
+    if (s != GDN_OK) return s;
+    if (!parent || !accepted || !k || !v || !g || !beta || !state) return GDN_ERR_INVALID_ARG;
+    if (!aligned(k, 16) || !aligned(v, 16) || !aligned(state, 16) || !aligned(parent, 4) ||
+        !aligned(accepted, 4) || !aligned(g, 4) || !aligned(beta, 4) || !aligned(status, 4))
+        return GDN_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaGetLastError();
+    const int smem = sizeof(CommitSmem);
+    cudaFuncSetAttribute(tree_commit_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    GDN_LAUNCH("tree_commit", st,
+               (tree_commit_kernel<<<(unsigned)(N * H), TREE_THREADS, smem, st>>>(
+                   M, H, parent, accepted, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, g,
+                   beta, state, status)));
+    return launched();
+}
+
+}  // extern "C"

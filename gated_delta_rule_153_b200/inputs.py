@@ -175,3 +175,39 @@ def make_varlen_inputs(cfg: ChunkConfig, lens, **over) -> dict:
     cu = torch.zeros(len(lens) + 1, dtype=torch.int32)
     cu[1:] = torch.cumsum(torch.tensor(lens, dtype=torch.int64), 0).to(torch.int32)
     return dict(tok, h0=states["h0"], dhT=states["dhT"], cu_seqlens=cu, lens=lens)
+
+
+def tree_parents(N: int, M: int, shape: str = "random", seed: int = 0) -> torch.Tensor:
+    """Parent indices [N, M] int32 of draft trees (parent[i] in [-1, i)):
+    "random" draws each parent uniformly from -1 .. i-1, "chain" is
+    i - 1, "star" is -1 everywhere, "kary4" is the complete 4-ary tree in
+    breadth-first order below a root node 0."""
+    if shape == "chain":
+        p = torch.arange(M) - 1
+        return p.repeat(N, 1).to(torch.int32).contiguous()
+    if shape == "star":
+        return torch.full((N, M), -1, dtype=torch.int32)
+    if shape == "kary4":
+        p = torch.tensor([-1] + [(i - 1) // 4 for i in range(1, M)])
+        return p.repeat(N, 1).to(torch.int32).contiguous()
+    gen = _gen(seed, 11)
+    u = torch.rand(N, M, generator=gen)
+    idx = torch.arange(M)
+    return (torch.floor(u * (idx + 1)).to(torch.int64) - 1).to(torch.int32).contiguous()
+
+
+def make_tree_inputs(N: int, M: int, H: int, shape: str = "random", seed: int = 1200,
+                     g_shift: float = 0.0, beta_max: float = 1.0,
+                     state_std: float = 0.02) -> dict:
+    """Host tensors for draft-tree verification: q, k [N,M,H,128] and v
+    [N,M,H,128] bf16 (q, k L2-normalised), g, beta [N,M,H] fp32 drawn as in
+    make_chunk_inputs, state [N,H,128,128] fp32, parent [N,M] int32 and
+    accepted [N] int32 (uniform over -1 .. M-1)."""
+    cfg = ChunkConfig("tree", N, M, H, 128, 128, 64, "bf16", "scalar", g_shift, None,
+                      False, None, seed, beta_max)
+    tok = make_chunk_inputs(cfg)
+    state = torch.randn(N, H, 128, 128, generator=_gen(seed, 12)) * state_std
+    accepted = (torch.floor(torch.rand(N, generator=_gen(seed, 13)) * (M + 1)) - 1)
+    return dict(q=tok["q"], k=tok["k"], v=tok["v"], g=tok["g"], beta=tok["beta"],
+                state=state, parent=tree_parents(N, M, shape, seed),
+                accepted=accepted.to(torch.int32), N=N, M=M, H=H)

@@ -148,6 +148,44 @@ gdn_status gdn_chunk_bwd_varlen(const gdn_dims *dims, const int *cu_seqlens,
                                 float *dh0, void *ws, size_t ws_bytes,
                                 gdn_stream_t stream);
 
+/* Draft-tree verification and commit: "TreeWY: Speculative Verification for
+ * Gated DeltaNet Hybrids" (paper list of the "Linear Attention
+ * Architectures: Mechanisms, Trade-offs, and Cross-Layer Routing" summary
+ * page).  Per (sequence n, head h) a speculative draft tree of M nodes hangs
+ * below the committed state S = state[n, h]: node i carries one token and a
+ * parent index parent[n, i] in [-1, i) (-1: the node follows S directly;
+ * parents precede children).  Node i's output is the gated delta rule of
+ * gdn_chunk_fwd run from S over the tokens of its root path, read out at i.
+ * gdn_tree_verify computes all M outputs in one pass without any per-node
+ * state: the chunkwise WY/UT algebra with the causal mask replaced by the
+ * ancestor relation (one triangular solve per tree), reading S once.
+ * gdn_tree_commit replaces S by the state after the root path of node
+ * accepted[n] (-1 or nothing accepted: S is left untouched), by the
+ * recurrent form along that path on the fp32 state.
+ * Layouts (contiguous): parent [N, M] int32; accepted [N] int32; q, k
+ * [N, M, H, dk]; v, o [N, M, H, dv]; g, beta [N, M, H] fp32; state
+ * [N, H, dv, dk] fp32 (row = value index).  All device pointers.
+ * Supported: GDN_BF16, GDN_GATE_SCALAR, dk = dv = 128, 1 <= M <= 64 (else
+ * GDN_ERR_UNSUPPORTED); N, H, M < 1, null pointers or misalignment (16 bytes
+ * for q, k, v, o, state; 4 for the rest) are GDN_ERR_INVALID_ARG.
+ * Tree indices are device data and are checked on the device: a parent out
+ * of [-1, i) is read as -1 and an accepted index out of [-1, M) as -1; either
+ * sets bit 1 (value 2) of the optional device word *status (may be NULL),
+ * which gdn_query_device_status(status, stream) then reports as
+ * GDN_ERR_INVALID_ARG.  state is read-only in gdn_tree_verify and updated in
+ * place by gdn_tree_commit; q, k, v, g, beta may be shared by both calls. */
+gdn_status gdn_tree_verify(int N, int M, int H, int dk, int dv, gdn_dtype dtype,
+                           gdn_gate gate, float scale, const int *parent,
+                           const void *q, const void *k, const void *v,
+                           const float *g, const float *beta,
+                           const float *state, void *o, unsigned int *status,
+                           gdn_stream_t stream);
+gdn_status gdn_tree_commit(int N, int M, int H, int dk, int dv, gdn_dtype dtype,
+                           gdn_gate gate, const int *parent, const int *accepted,
+                           const void *k, const void *v, const float *g,
+                           const float *beta, float *state, unsigned int *status,
+                           gdn_stream_t stream);
+
 /* Gated DeltaProduct: "DeltaProduct: Improving State-Tracking in Linear RNNs
  * via Householder Products" (in the list of related papers of the "Linear
  * Attention Architectures: Mechanisms, Trade-offs, and Cross-Layer Routing"

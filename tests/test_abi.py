@@ -162,3 +162,28 @@ def test_varlen_checks():
     bwd = L.gdn_chunk_bwd_varlen
     assert bwd(ctypes.byref(d), p, 3, p, p, p, p, p, p, p, None, p, p, p, p, p, None, p, ws,
                None) == gdn.GDN_ERR_INVALID_ARG  # dh0 without h0
+
+
+def test_tree_checks():
+    """gdn_tree_*: host-side rejection before any launch."""
+    L = gdn.lib()
+    p = ctypes.c_void_p(256)
+    bf, sc, ch = gdn.GDN_BF16, gdn.GDN_GATE_SCALAR, gdn.GDN_GATE_CHANNEL
+    v = L.gdn_tree_verify
+    args = (p, p, p, p, p, p, p, p, None, None)
+    assert v(2, 0, 4, 128, 128, bf, sc, 1.0, *args) == gdn.GDN_ERR_INVALID_ARG
+    assert v(2, 65, 4, 128, 128, bf, sc, 1.0, *args) == gdn.GDN_ERR_UNSUPPORTED
+    assert v(2, 8, 4, 64, 128, bf, sc, 1.0, *args) == gdn.GDN_ERR_UNSUPPORTED
+    assert v(2, 8, 4, 128, 128, gdn.GDN_F32, sc, 1.0, *args) == gdn.GDN_ERR_UNSUPPORTED
+    assert v(2, 8, 4, 128, 128, bf, ch, 1.0, *args) == gdn.GDN_ERR_UNSUPPORTED
+    assert v(2, 8, 4, 128, 128, bf, sc, float("nan"), *args) == gdn.GDN_ERR_INVALID_ARG
+    assert v(2, 8, 4, 128, 128, bf, sc, 1.0, None, *args[1:]) == gdn.GDN_ERR_INVALID_ARG
+    assert v(2, 8, 4, 128, 128, bf, sc, 1.0, p, ctypes.c_void_p(264), *args[2:]) == \
+        gdn.GDN_ERR_INVALID_ARG
+    c = L.gdn_tree_commit
+    assert c(0, 8, 4, 128, 128, bf, sc, p, p, p, p, p, p, p, None, None) == \
+        gdn.GDN_ERR_INVALID_ARG
+    assert c(2, 8, 4, 128, 128, bf, sc, p, None, p, p, p, p, p, None, None) == \
+        gdn.GDN_ERR_INVALID_ARG
+    assert c(2, 8, 4, 128, 128, bf, sc, p, ctypes.c_void_p(258), p, p, p, p, p, None,
+             None) == gdn.GDN_ERR_INVALID_ARG
