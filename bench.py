@@ -363,6 +363,45 @@ def run_ours(args, rank, world, dev, barrier, max_over_ranks):
                            "hbm_gbs": round(gbs, 1), "frac_hbm_peak": round(gbs / pk["hbm"], 4),
                            "bytes_per_step": dbytes}
         del dd, dec
+        # ---- draft-tree verification and commit, decode-sized batch ----------
+        from gated_delta_rule_153_b200.inputs import make_tree_inputs
+        TN, TM, TH = DECODE.N, 32, DECODE.H
+        tr = to_dev(make_tree_inputs(TN, TM, TH, shape="kary4",
+                                     seed=replica_seed(1200, rank)), dev)
+        to = torch.empty_like(tr["v"])
+        REP = 20
+
+        def tree_verify_run():
+            for _ in range(REP):
+                gdn.gdn_tree_verify(tr["parent"], tr["q"], tr["k"], tr["v"], tr["g"], tr["beta"],
+                                    tr["state"], o=to)
+
+        def tree_commit_run():
+            for _ in range(REP):
+                gdn.gdn_tree_commit(tr["parent"], tr["accepted"], tr["k"], tr["v"], tr["g"],
+                                    tr["beta"], tr["state"])
+        ms_v = timed(tree_verify_run, 3, 1, barrier) / REP
+        ms_c = timed(tree_commit_run, 3, 1, barrier) / REP
+        state_b = TN * TH * DECODE.dv * DECODE.dk * 4
+        vbytes = state_b + TN * TH * TM * (4 * 128 * 2 + 8) + TN * TM * 4
+        par = tr["parent"].cpu().numpy()
+        path_len = 0
+        for n, a in enumerate(tr["accepted"].cpu().tolist()):
+            while a >= 0:
+                path_len += 1
+                a = int(par[n, a])
+        committed = int((tr["accepted"] >= 0).sum().item())
+        cbytes = committed * TH * 2 * DECODE.dv * DECODE.dk * 4 + path_len * TH * (2 * 128 * 2 + 8)
+        extra["draft_tree"] = {
+            "workload": f"N{TN} H{TH} d128, {TM}-node 4-ary draft trees, bf16, fp32 state",
+            "verify_us": round(ms_v * 1e3, 2), "verify_bytes": vbytes,
+            "verify_hbm_gbs": round(vbytes / (ms_v / 1e3) / 1e9, 1),
+            "verify_frac_hbm_peak": round(vbytes / (ms_v / 1e3) / 1e9 / pk["hbm"], 4),
+            "commit_us": round(ms_c * 1e3, 2), "commit_bytes": cbytes,
+            "commit_hbm_gbs": round(cbytes / (ms_c / 1e3) / 1e9, 1),
+            "commit_frac_hbm_peak": round(cbytes / (ms_c / 1e3) / 1e9 / pk["hbm"], 4),
+            "nodes_verified_per_s": round(TN * TM / (ms_v / 1e3), 1)}
+        del tr, to
 
     # ---- end to end through host buffers ------------------------------------
     names_in = ("q", "k", "v", "g", "beta", "dO")

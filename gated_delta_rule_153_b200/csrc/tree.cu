@@ -24,6 +24,7 @@
 // write of each state row.
 #include <math.h>
 
+#include "async.cuh"
 #include "common.cuh"
 #include "internal.h"
 #include "mma.cuh"
@@ -50,12 +51,13 @@ struct TreeSmem {
     __nv_bfloat16 P[MP * 64];
     float G[MP], g[MP], beta[MP];
     unsigned long long anc[MP];
-    int par[MP];
+    int par[MP], depth[MP];
+    int maxdepth;
 };
 
 // One CTA per (sequence n, head h).  MB = number of 16-node blocks.
 template <int MB>
-__global__ void __launch_bounds__(TREE_THREADS)
+__global__ void __launch_bounds__(TREE_THREADS, MB <= 2 ? 4 : 2)  // 4 CTAs per SM up to 32 nodes
 tree_verify_kernel(int M, int H, float scale, const int* __restrict__ parent,
                    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                    const __nv_bfloat16* __restrict__ v, const float* __restrict__ g,
@@ -69,7 +71,11 @@ tree_verify_kernel(int M, int H, float scale, const int* __restrict__ parent,
     const size_t rs = (size_t)H * TD;                        // token row stride
     const size_t row0 = ((size_t)n * M * H + h) * TD;       // node 0 of (n, h)
 
-    // ---- loads: node tokens into shared tiles, the state into registers ----
+    // ---- loads: node tokens into shared tiles; the state is pulled into L2
+    // now and read as MMA fragments in the last phase ------------------------
+    const float* S0 = state + (size_t)nh * TD * TD;
+    if (tid < 4) bulk_prefetch_l2(S0 + tid * (TD * TD / 4), TD * TD);  // 4 x 16 KiB
+    if (tid == 0) s.maxdepth = 0;
     load_tile_async<TD>(s.K, k + row0, rs, MP, M, tid, TREE_THREADS);
     load_tile_async<TD>(s.Q, q + row0, rs, MP, M, tid, TREE_THREADS);
     load_tile_async<TD>(s.V, v + row0, rs, MP, M, tid, TREE_THREADS);
@@ -90,23 +96,6 @@ tree_verify_kernel(int M, int H, float scale, const int* __restrict__ parent,
         s.g[tid] = gi;
         s.beta[tid] = bi;
     }
-    // B fragments of S0^T for this warp's 16 value rows a0.. (B[k = c][n = a] = S0[a][c]).
-    const int a0 = 16 * warp;
-    uint32_t sf[2][8][2];
-    {
-        const float* S0 = state + (size_t)nh * TD * TD;
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-            const float* row = S0 + (size_t)(a0 + 8 * nt + (lane >> 2)) * TD + 2 * (lane & 3);
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                const float2 x = __ldcs(reinterpret_cast<const float2*>(row + 16 * kk));
-                const float2 y = __ldcs(reinterpret_cast<const float2*>(row + 16 * kk + 8));
-                sf[nt][kk][0] = pack_bf16(x.x, x.y);
-                sf[nt][kk][1] = pack_bf16(y.x, y.y);
-            }
-        }
-    }
     cp_async_wait<0>();
     __syncthreads();
 
@@ -120,6 +109,8 @@ tree_verify_kernel(int M, int H, float scale, const int* __restrict__ parent,
         }
         s.G[tid] = Gi;
         s.anc[tid] = m;
+        s.depth[tid] = __popcll(m);
+        atomicMax(&s.maxdepth, __popcll(m));
     }
     __syncthreads();
 
@@ -162,21 +153,31 @@ tree_verify_kernel(int M, int H, float scale, const int* __restrict__ parent,
     }
     __syncthreads();
 
-    // ---- T = (I + A)^{-1} by forward substitution, 4 lanes per column -------
+    // ---- T = (I + A)^{-1}, one tree level at a time --------------------------
+    // Row i of T is e_i - sum over ancestors l of A_il T_l, and T_ic is non-zero
+    // only for c an ancestor of i or i itself; so every node of one depth is
+    // solved at once from the rows of shallower nodes (a chain: one per level).
     {
-        const int c = tid >> 2, part = tid & 3;
-        if (c < MP) {  // whole warps: 8 columns each
-            for (int i = 0; i < MP; ++i) {
-                float sum = 0.f;
-                for (int j = c + part; j < i; j += 4) sum += s.A[i][j] * s.T[j][c];
-                sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-                sum += __shfl_xor_sync(0xffffffffu, sum, 2);
-                if (part == 0) s.T[i][c] = i == c ? 1.f : (i > c ? -sum : 0.f);
-                __syncwarp();
+        const int levels = s.maxdepth;
+        for (int d = 0; d <= levels; ++d) {
+            for (int e = tid; e < MP * MP; e += TREE_THREADS) {
+                const int i = e / MP, c = e % MP;
+                if (s.depth[i] != d) continue;
+                const unsigned long long ai = s.anc[i];
+                float t = c == i ? 1.f : 0.f;
+                if ((ai >> c) & 1ull) {
+                    float sum = 0.f;
+                    for (unsigned long long m = ai & ~((1ull << c) - 1ull); m; m &= m - 1ull) {
+                        const int l = __ffsll((long long)m) - 1;  // ancestors l >= c
+                        sum += s.A[i][l] * s.T[l][c];
+                    }
+                    t = -sum;
+                }
+                s.T[i][c] = t;
             }
+            __syncthreads();
         }
     }
-    __syncthreads();
     for (int e = tid; e < MP * MP; e += TREE_THREADS) {
         const int i = e / MP, j = e % MP;
         const float t = s.T[i][j] * s.beta[j];
@@ -218,35 +219,52 @@ tree_verify_kernel(int M, int H, float scale, const int* __restrict__ parent,
     __syncthreads();  // K is read for the last time above; U takes its place
 
     // ---- U = U~ - W S0^T and O = scale e^G Q S0^T + P U, value rows a0..a0+15 ----
+    const int a0 = 16 * warp;
     __nv_bfloat16* Ub = s.K;
-    float acco[MB][2][4];
+    float accu[MB][2][4], acco[MB][2][4];
 #pragma unroll
-    for (int mb = 0; mb < MB; ++mb) {
-        float u[2][4];
+    for (int mb = 0; mb < MB; ++mb)
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) { u[nt][e] = 0.f; acco[mb][nt][e] = 0.f; }
+            for (int e = 0; e < 4; ++e) { accu[mb][nt][e] = 0.f; acco[mb][nt][e] = 0.f; }
+#pragma unroll
+    for (int mb = 0; mb < MB; ++mb)
 #pragma unroll
         for (int kk = 0; kk <= mb; ++kk) {  // T is lower triangular
             uint32_t a[4], b[4];
             lda<64>(a, s.Tu, 16 * mb, 16 * kk);
             ldb_kn<TD>(b, s.V, 16 * kk, a0);
-            mma16816(u[0], a, b[0], b[1]);
-            mma16816(u[1], a, b[2], b[3]);
+            mma16816(accu[mb][0], a, b[0], b[1]);
+            mma16816(accu[mb][1], a, b[2], b[3]);
         }
+    // B fragments of S0^T (B[k = c][n = a] = S0[a][c]) straight from L2, one
+    // K = 16 step at a time, shared by every node block.
+    const float* srow0 = S0 + (size_t)(a0 + (lane >> 2)) * TD + 2 * (lane & 3);
+    const float* srow1 = srow0 + 8 * TD;
 #pragma unroll
-        for (int kk = 0; kk < TD / 16; ++kk) {
+    for (int kk = 0; kk < TD / 16; ++kk) {
+        const float2 x0 = __ldcs(reinterpret_cast<const float2*>(srow0 + 16 * kk));
+        const float2 y0 = __ldcs(reinterpret_cast<const float2*>(srow0 + 16 * kk + 8));
+        const float2 x1 = __ldcs(reinterpret_cast<const float2*>(srow1 + 16 * kk));
+        const float2 y1 = __ldcs(reinterpret_cast<const float2*>(srow1 + 16 * kk + 8));
+        const uint32_t b00 = pack_bf16(x0.x, x0.y), b01 = pack_bf16(y0.x, y0.y);
+        const uint32_t b10 = pack_bf16(x1.x, x1.y), b11 = pack_bf16(y1.x, y1.y);
+#pragma unroll
+        for (int mb = 0; mb < MB; ++mb) {
             uint32_t a[4];
             lda<TD>(a, s.Wn, 16 * mb, 16 * kk);
-            mma16816(u[0], a, sf[0][kk][0], sf[0][kk][1]);
-            mma16816(u[1], a, sf[1][kk][0], sf[1][kk][1]);
+            mma16816(accu[mb][0], a, b00, b01);
+            mma16816(accu[mb][1], a, b10, b11);
             lda<TD>(a, s.Q, 16 * mb, 16 * kk);
-            mma16816(acco[mb][0], a, sf[0][kk][0], sf[0][kk][1]);
-            mma16816(acco[mb][1], a, sf[1][kk][0], sf[1][kk][1]);
+            mma16816(acco[mb][0], a, b00, b01);
+            mma16816(acco[mb][1], a, b10, b11);
         }
-        st_c<TD>(Ub, 16 * mb, a0, u[0]);
-        st_c<TD>(Ub, 16 * mb, a0 + 8, u[1]);
+    }
+#pragma unroll
+    for (int mb = 0; mb < MB; ++mb) {
+        st_c<TD>(Ub, 16 * mb, a0, accu[mb][0]);
+        st_c<TD>(Ub, 16 * mb, a0 + 8, accu[mb][1]);
         const int r = 16 * mb + (lane >> 2);
         const float f0 = scale * __expf(s.G[r]), f1 = scale * __expf(s.G[r + 8]);
 #pragma unroll
