@@ -402,6 +402,60 @@ def run_ours(args, rank, world, dev, barrier, max_over_ranks):
             "commit_frac_hbm_peak": round(cbytes / (ms_c / 1e3) / 1e9 / pk["hbm"], 4),
             "nodes_verified_per_s": round(TN * TM / (ms_v / 1e3), 1)}
         del tr, to
+        # ---- q/k/v prologue (short conv, SiLU, L2 norm), 350M-scale shape ----
+        from gated_delta_rule_153_b200.inputs import make_prologue_inputs
+        pr = {n: make_prologue_inputs(cfg.B, cfg.T, cfg.H, seed=replica_seed(1400 + i, rank))
+              for i, n in enumerate("qkv")}
+        pr = {n: {m: t.to(dev) for m, t in v.items() if torch.is_tensor(t)} for n, v in pr.items()}
+        py = {n: torch.empty_like(pr[n]["x"]) for n in "qkv"}
+        pws = torch.empty(gdn.lib().gdn_short_conv_bwd_workspace(cfg.B, cfg.T, cfg.H, 128, 4),
+                          dtype=torch.uint8, device=dev)
+
+        def prologue_fwd():
+            for n in "qkv":
+                gdn.gdn_short_conv_fwd(pr[n]["x"], pr[n]["w"], l2norm=n != "v", y=py[n])
+
+        def prologue_bwd():
+            for n in "qkv":
+                gdn.gdn_short_conv_bwd(pr[n]["x"], pr[n]["w"], pr[n]["dy"], l2norm=n != "v",
+                                       workspace=pws)
+        # Each call is a few microseconds of device work behind tens of
+        # microseconds of Python argument checks, so the step is captured in a
+        # CUDA graph and the replays are timed: device time, not launch rate.
+        def graph_ms(fn, reps=20):
+            fn()
+            torch.cuda.synchronize()
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                fn()
+            graph.replay()
+            torch.cuda.synchronize()
+            barrier()
+            t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            t0.record()
+            for _ in range(reps):
+                graph.replay()
+            t1.record()
+            torch.cuda.synchronize()
+            del graph
+            return t0.elapsed_time(t1) / reps
+        try:
+            ms_pf, ms_pb, ptiming = graph_ms(prologue_fwd), graph_ms(prologue_bwd), "cuda graph"
+        except RuntimeError as err:  # capture refused: time the eager calls instead
+            ms_pf, ms_pb = timed(prologue_fwd, 5, 2, barrier), timed(prologue_bwd, 5, 2, barrier)
+            ptiming = f"eager (graph capture failed: {str(err)[:80]})"
+        th = cfg.B * cfg.T * cfg.H
+        pf_bytes = 3 * th * 2 * 256             # read x, write y, bf16 d = 128
+        pb_bytes = 3 * th * 3 * 256             # read x, dy, write dx
+        extra["prologue"] = {
+            "workload": f"{cfg.name}: q, k (L2 norm) and v, K = 4 taps", "timing": ptiming,
+            "fwd_us": round(ms_pf * 1e3, 1), "fwd_bytes": pf_bytes,
+            "fwd_hbm_gbs": round(pf_bytes / (ms_pf / 1e3) / 1e9, 1),
+            "fwd_frac_hbm_peak": round(pf_bytes / (ms_pf / 1e3) / 1e9 / pk["hbm"], 4),
+            "bwd_us": round(ms_pb * 1e3, 1), "bwd_bytes": pb_bytes,
+            "bwd_hbm_gbs": round(pb_bytes / (ms_pb / 1e3) / 1e9, 1),
+            "bwd_frac_hbm_peak": round(pb_bytes / (ms_pb / 1e3) / 1e9 / pk["hbm"], 4)}
+        del pr, py, pws
 
     # ---- end to end through host buffers ------------------------------------
     names_in = ("q", "k", "v", "g", "beta", "dO")

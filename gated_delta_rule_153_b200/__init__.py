@@ -31,7 +31,8 @@ EXPORTS = ("gdn_chunk_fwd_workspace", "gdn_chunk_fwd", "gdn_chunk_bwd_workspace"
            "gdn_chunk_fwd_noalloc", "gdn_product_fwd_workspace", "gdn_product_fwd",
            "gdn_product_bwd_workspace", "gdn_product_bwd", "gdn_chunk_fwd_varlen_workspace",
            "gdn_chunk_fwd_varlen", "gdn_chunk_bwd_varlen_workspace", "gdn_chunk_bwd_varlen",
-           "gdn_tree_verify", "gdn_tree_commit")
+           "gdn_tree_verify", "gdn_tree_commit", "gdn_short_conv_fwd",
+           "gdn_short_conv_bwd_workspace", "gdn_short_conv_bwd")
 
 
 class gdn_dims(ctypes.Structure):
@@ -104,6 +105,12 @@ def lib() -> ctypes.CDLL:
             L.gdn_tree_commit.argtypes = [i, i, i, i, i, i, i, vp, vp, vp, vp, fp, fp, fp, vp,
                                           vp]
             L.gdn_tree_commit.restype = i
+            L.gdn_short_conv_fwd.argtypes = [i, i, i, i, i, i, i, vp, fp, vp, vp]
+            L.gdn_short_conv_fwd.restype = i
+            L.gdn_short_conv_bwd_workspace.argtypes = [i, i, i, i, i]
+            L.gdn_short_conv_bwd_workspace.restype = sz
+            L.gdn_short_conv_bwd.argtypes = [i, i, i, i, i, i, i, vp, fp, vp, vp, fp, vp, sz, vp]
+            L.gdn_short_conv_bwd.restype = i
             L.gdn_profile_begin.argtypes = [i]
             L.gdn_profile_begin.restype = i
             L.gdn_profile_end.argtypes = [ctypes.POINTER(ctypes.c_float),
@@ -469,3 +476,46 @@ def gdn_tree_commit(parent, accepted, k, v, g, beta, state, *, status=None, stre
                                _ptr(state), _ptr(status), _stream(stream))
     _check(st, "gdn_tree_commit")
     return state
+
+
+# ---- q/k/v prologue: short causal convolution, SiLU, L2 norm ---------------
+def _validate_conv(x, w):
+    import torch
+    _need(x, "x")
+    if x.dim() != 4:
+        raise ValueError("x must be [B, T, H, d]")
+    B, T, H, d = x.shape
+    _need(w, "w", torch.float32)
+    if w.dim() != 3 or tuple(w.shape[:2]) != (H, d):
+        raise ValueError("w must be [H, d, K] fp32")
+    return B, T, H, d, w.shape[2]
+
+
+def gdn_short_conv_fwd(x, w, *, l2norm=True, y=None, stream=None):
+    """y = (L2-normalised) SiLU(causal depthwise conv of x with w): x
+    [B,T,H,d] bf16/fp32, w [H,d,K] fp32.  Returns y (shape and dtype of x)."""
+    import torch
+    B, T, H, d, K = _validate_conv(x, w)
+    if y is None:
+        y = torch.empty_like(x)
+    st = lib().gdn_short_conv_fwd(B, T, H, d, K, _dtype_code(x), int(bool(l2norm)), _ptr(x),
+                                  _ptr(w), _ptr(y), _stream(stream))
+    _check(st, "gdn_short_conv_fwd")
+    return y
+
+
+def gdn_short_conv_bwd(x, w, dy, *, l2norm=True, workspace=None, stream=None):
+    """Gradients of <dy, y> for gdn_short_conv_fwd: returns (dx, dw)."""
+    import torch
+    B, T, H, d, K = _validate_conv(x, w)
+    _need(dy, "dy", x.dtype, tuple(x.shape))
+    dx = torch.empty_like(x)
+    dw = torch.empty_like(w)
+    nbytes = int(lib().gdn_short_conv_bwd_workspace(B, T, H, d, K))
+    ws = _workspace(nbytes, x.device, workspace)
+    st = lib().gdn_short_conv_bwd(B, T, H, d, K, _dtype_code(x), int(bool(l2norm)), _ptr(x),
+                                  _ptr(w), _ptr(dy), _ptr(dx), _ptr(dw), _ptr(ws),
+                                  nbytes if ws is None else ws.numel() * ws.element_size(),
+                                  _stream(stream))
+    _check(st, "gdn_short_conv_bwd")
+    return dx, dw

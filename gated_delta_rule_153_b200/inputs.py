@@ -211,3 +211,15 @@ def make_tree_inputs(N: int, M: int, H: int, shape: str = "random", seed: int = 
     return dict(q=tok["q"], k=tok["k"], v=tok["v"], g=tok["g"], beta=tok["beta"],
                 state=state, parent=tree_parents(N, M, shape, seed),
                 accepted=accepted.to(torch.int32), N=N, M=M, H=H)
+
+
+def make_prologue_inputs(B: int, T: int, H: int, d: int = 128, K: int = 4,
+                         dtype: str = "bf16", seed: int = 1400) -> dict:
+    """Host tensors for the short-conv prologue: projected activations x and
+    an upstream gradient dy [B,T,H,d] in ``dtype`` (N(0,1)), filters w
+    [H,d,K] fp32 (N(0, 1/K))."""
+    dt = _DT[dtype]
+    x = torch.randn(B, T, H, d, generator=_gen(seed, 20)).to(dt)
+    w = torch.randn(H, d, K, generator=_gen(seed, 21)) / K ** 0.5
+    dy = torch.randn(B, T, H, d, generator=_gen(seed, 22)).to(dt)
+    return dict(x=x.contiguous(), w=w.contiguous(), dy=dy.contiguous(), dtype=dtype)

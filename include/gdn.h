@@ -148,6 +148,31 @@ gdn_status gdn_chunk_bwd_varlen(const gdn_dims *dims, const int *cu_seqlens,
                                 float *dh0, void *ws, size_t ws_bytes,
                                 gdn_stream_t stream);
 
+/* The q/k/v prologue: "Gated Delta Networks: Improving Mamba2 with Delta
+ * Rule" (paper review), section "Method": q and k pass through a short
+ * convolution and SiLU, then L2 normalisation; v takes the same path without
+ * the norm.  Read as a causal depthwise filter of K taps per channel with
+ * zeros before each sequence's first token (no bias):
+ *     z_t[c] = sum_{j<K} w[h, c, j] x_t-j[c],   s = z * sigmoid(z),
+ *     y = s / sqrt(sum_c s_c^2 + 1e-6)  over the d channels of one head
+ *     (l2norm != 0; otherwise y = s).
+ * gdn_short_conv_fwd writes y; gdn_short_conv_bwd writes dx and dw for the
+ * loss <dy, y> (dw is overwritten, not accumulated, and summed in a fixed
+ * order, so it is deterministic).  Layouts (contiguous, device): x, y, dy, dx
+ * [B, T, H, d] in `dtype` (bf16 or fp32); w, dw [H, d, K] fp32.  x and y may
+ * not alias, nor dx and x or dy.  d in {32, 64, 128} and 1 <= K <= 4 (else
+ * GDN_ERR_UNSUPPORTED / GDN_ERR_INVALID_ARG); x, y, dy, dx 16-byte aligned;
+ * the backward workspace (gdn_short_conv_bwd_workspace bytes, 256-byte
+ * aligned) holds one weight-gradient partial per 32-token tile of a head. */
+gdn_status gdn_short_conv_fwd(int B, int T, int H, int d, int K, gdn_dtype dtype,
+                              int l2norm, const void *x, const float *w, void *y,
+                              gdn_stream_t stream);
+size_t gdn_short_conv_bwd_workspace(int B, int T, int H, int d, int K);
+gdn_status gdn_short_conv_bwd(int B, int T, int H, int d, int K, gdn_dtype dtype,
+                              int l2norm, const void *x, const float *w,
+                              const void *dy, void *dx, float *dw, void *ws,
+                              size_t ws_bytes, gdn_stream_t stream);
+
 /* Draft-tree verification and commit: "TreeWY: Speculative Verification for
  * Gated DeltaNet Hybrids" (paper list of the "Linear Attention
  * Architectures: Mechanisms, Trade-offs, and Cross-Layer Routing" summary

@@ -187,3 +187,24 @@ def test_tree_checks():
         gdn.GDN_ERR_INVALID_ARG
     assert c(2, 8, 4, 128, 128, bf, sc, p, ctypes.c_void_p(258), p, p, p, p, p, None,
              None) == gdn.GDN_ERR_INVALID_ARG
+
+
+def test_short_conv_checks():
+    L = gdn.lib()
+    p = ctypes.c_void_p(256)
+    bf = gdn.GDN_BF16
+    f = L.gdn_short_conv_fwd
+    assert f(0, 8, 2, 128, 4, bf, 1, p, p, ctypes.c_void_p(512), None) == gdn.GDN_ERR_INVALID_ARG
+    assert f(1, 8, 2, 96, 4, bf, 1, p, p, ctypes.c_void_p(512), None) == gdn.GDN_ERR_UNSUPPORTED
+    assert f(1, 8, 2, 128, 5, bf, 1, p, p, ctypes.c_void_p(512), None) == gdn.GDN_ERR_UNSUPPORTED
+    assert f(1, 8, 2, 128, 0, bf, 1, p, p, ctypes.c_void_p(512), None) == gdn.GDN_ERR_INVALID_ARG
+    assert f(1, 8, 2, 128, 4, bf, 1, p, p, p, None) == gdn.GDN_ERR_INVALID_ARG  # y aliases x
+    assert f(1, 8, 2, 128, 4, bf, 1, ctypes.c_void_p(264), p, ctypes.c_void_p(512),
+             None) == gdn.GDN_ERR_INVALID_ARG
+    assert L.gdn_short_conv_bwd_workspace(2, 100, 3, 128, 4) == 2 * 4 * 3 * 128 * 4 * 4
+    b = L.gdn_short_conv_bwd
+    q = ctypes.c_void_p(1024)
+    assert b(2, 100, 3, 128, 4, bf, 1, p, p, ctypes.c_void_p(512), q, p, p, 16, None) == \
+        gdn.GDN_ERR_WORKSPACE
+    assert b(2, 100, 3, 128, 4, bf, 1, p, p, ctypes.c_void_p(512), p, p, p, 1 << 30, None) == \
+        gdn.GDN_ERR_INVALID_ARG  # dx aliases x
