@@ -198,9 +198,10 @@ short_conv_fwd_kernel(int Tn, int H, int K, int tiles, const T* __restrict__ x,
     load_filters<CPL>(wr, w + ((size_t)r.h * D + c0) * K, K);
 #pragma unroll
     for (int j = 0; j < KT - 1; ++j) unpack(win[KT - 2 - j], xs[j]);  // win[0] = x_{t0-1}
+    // Straight-line over the run, so the reductions of different tokens
+    // overlap; tokens past the end are computed and not stored.
 #pragma unroll
     for (int u = 0; u < RUN; ++u) {
-        if (r.t0 + u >= r.t1) break;  // uniform over the warp
         float xv[CPL], s[CPL];
         unpack(xv, xs[u + KT - 1]);
         conv_at<CPL>(s, wr, xv, win);
@@ -216,8 +217,59 @@ short_conv_fwd_kernel(int Tn, int H, int K, int tiles, const T* __restrict__ x,
 #pragma unroll
             for (int i = 0; i < CPL; ++i) s[i] *= inv;
         }
-        store_ch<T, CPL>(y + base + (size_t)(r.t0 + u) * rs, s);
+        if (r.t0 + u < r.t1) store_ch<T, CPL>(y + base + (size_t)(r.t0 + u) * rs, s);
     }
+}
+
+// dz_t from x_t, the window x_{t-1..t-3} and dy_t (a whole warp: the norm's
+// sums are warp reductions).
+template <int CPL, bool NORM, typename R>
+GDN_DEV void dz_at(float (&dz)[CPL], const float (&wr)[CPL][KT], const float (&xv)[CPL],
+                   const float (&win)[KT - 1][CPL], R dyraw) {
+    float z[CPL], sg[CPL], sv[CPL], g[CPL];
+    conv_at<CPL>(z, wr, xv, win);
+    unpack(g, dyraw);
+    float ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) {
+        sg[i] = __fdividef(1.f, 1.f + __expf(-z[i]));
+        sv[i] = z[i] * sg[i];
+        ss += sv[i] * sv[i];
+    }
+    if (NORM) {
+        const float inv = rsqrtf(warp_sum(ss) + kNormEps);
+        float dot = 0.f;
+#pragma unroll
+        for (int i = 0; i < CPL; ++i) dot += sv[i] * inv * g[i];
+        dot = warp_sum(dot);
+#pragma unroll
+        for (int i = 0; i < CPL; ++i) g[i] = (g[i] - sv[i] * inv * dot) * inv;
+    }
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) dz[i] = g[i] * sg[i] * (1.f + z[i] * (1.f - sg[i]));
+}
+
+template <int CPL>
+GDN_DEV void push_dz(float (&dzw)[KT][CPL], const float (&dz)[CPL]) {
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) {
+        dzw[3][i] = dzw[2][i];
+        dzw[2][i] = dzw[1][i];
+        dzw[1][i] = dzw[0][i];
+        dzw[0][i] = dz[i];
+    }
+}
+
+// dx_te = sum_j w_j dz_{te+j} once dz_{te+KT-1} is in dzw[0] (te in [t0, t1)).
+template <typename T, int CPL>
+GDN_DEV void emit_dx(T* dxb, size_t rs, const float (&wr)[CPL][KT], const float (&dzw)[KT][CPL],
+                     int te, int t0, int t1) {
+    if (te < t0 || te >= t1) return;
+    float gx[CPL];
+#pragma unroll
+    for (int i = 0; i < CPL; ++i)
+        gx[i] = wr[i][0] * dzw[3][i] + wr[i][1] * dzw[2][i] + wr[i][2] * dzw[1][i] + wr[i][3] * dzw[0][i];
+    store_ch<T, CPL>(dxb + (size_t)te * rs, gx);
 }
 
 // The backward: dz over the run and the KT-1 tokens after it (dx of the run
@@ -243,83 +295,78 @@ short_conv_bwd_kernel(int Tn, int H, int K, int tiles, const T* __restrict__ x,
     for (int i = 0; i < CPL; ++i)
 #pragma unroll
         for (int j = 0; j < KT; ++j) dw[i][j] = 0.f;
-    if (active) {
-        const size_t rs = (size_t)H * D;
-        const size_t base = ((size_t)r.b * Tn * H + r.h) * D + c0;
-        const int tz = min(Tn, r.t1 + KT - 1);  // tokens that have a dz
-        R xs[NX], dys[NZ];                      // every load of the run in flight at once
+    __shared__ float head[PW][KT - 1][D];  // each warp's first KT-1 dz, for the warp before it
+    const size_t rs = (size_t)H * D;
+    const size_t base = ((size_t)r.b * Tn * H + r.h) * D + c0;
+    const bool last = warp == PW - 1;  // recomputes the KT-1 dz past the CTA's tokens
+    R xs[NX], dys[NZ];
+    float dzw[KT][CPL], win[KT - 1][CPL];  // dzw[j] = dz_{t-j}; win[j] = x_{t-1-j}
 #pragma unroll
-        for (int u = 0; u < NX; ++u) {
+    for (int j = 0; j < KT; ++j)
+#pragma unroll
+        for (int i = 0; i < CPL; ++i) dzw[j][i] = 0.f;
+    if (active) {
+        const int tz = min(Tn, r.t1 + KT - 1);  // tokens that have a dz
+#pragma unroll
+        for (int u = 0; u < NX; ++u) {  // every load of the run in flight at once
             const int t = r.t0 - (KT - 1) + u;
-            xs[u] = load_raw<T, CPL>(x + base + (size_t)max(t, 0) * rs, t >= 0 && t < tz);
+            const bool need = u < RUN + KT - 1 || last;
+            xs[u] = load_raw<T, CPL>(x + base + (size_t)max(t, 0) * rs, need && t >= 0 && t < tz);
         }
 #pragma unroll
         for (int u = 0; u < NZ; ++u)
-            dys[u] = load_raw<T, CPL>(dy + base + (size_t)(r.t0 + u) * rs, r.t0 + u < tz);
-        float dzw[KT][CPL];  // dzw[j] = dz_{t-j}
-#pragma unroll
-        for (int j = 0; j < KT; ++j)
-#pragma unroll
-            for (int i = 0; i < CPL; ++i) dzw[j][i] = 0.f;
-        float win[KT - 1][CPL];
+            dys[u] = load_raw<T, CPL>(dy + base + (size_t)(r.t0 + u) * rs,
+                                      (u < RUN || last) && r.t0 + u < tz);
 #pragma unroll
         for (int j = 0; j < KT - 1; ++j) unpack(win[KT - 2 - j], xs[j]);  // win[0] = x_{t0-1}
+        // The run's own tokens, straight-line: past the end dy reads as zero,
+        // which gives dz = 0 exactly, so nothing but stores is guarded.
 #pragma unroll
-        for (int u = 0; u < NZ; ++u) {
+        for (int u = 0; u < RUN; ++u) {
             float dz[CPL], xv[CPL];
             unpack(xv, xs[u + KT - 1]);
-            if (r.t0 + u < tz) {  // uniform over the warp
-                float z[CPL], sg[CPL], sv[CPL], g[CPL];
-                conv_at<CPL>(z, wr, xv, win);
-                unpack(g, dys[u]);
-                float ss = 0.f;
+            dz_at<CPL, NORM>(dz, wr, xv, win, dys[u]);
 #pragma unroll
-                for (int i = 0; i < CPL; ++i) {
-                    sg[i] = __fdividef(1.f, 1.f + __expf(-z[i]));
-                    sv[i] = z[i] * sg[i];
-                    ss += sv[i] * sv[i];
-                }
-                if (NORM) {
-                    const float inv = rsqrtf(warp_sum(ss) + kNormEps);
-                    float dot = 0.f;
+            for (int i = 0; i < CPL; ++i) {
+                dw[i][0] += dz[i] * xv[i];
+                dw[i][1] += dz[i] * win[0][i];
+                dw[i][2] += dz[i] * win[1][i];
+                dw[i][3] += dz[i] * win[2][i];
+            }
+            if (u < KT - 1) {
 #pragma unroll
-                    for (int i = 0; i < CPL; ++i) dot += sv[i] * inv * g[i];
-                    dot = warp_sum(dot);
+                for (int i = 0; i < CPL; ++i) head[warp][u][c0 + i] = dz[i];
+            }
+            shift_in<CPL>(win, xv);
+            push_dz<CPL>(dzw, dz);
+            emit_dx<T, CPL>(dx + base, rs, wr, dzw, r.t0 + u - (KT - 1), r.t0, r.t1);
+        }
+    } else {
 #pragma unroll
-                    for (int i = 0; i < CPL; ++i) g[i] = (g[i] - sv[i] * inv * dot) * inv;
-                }
+        for (int k = 0; k < KT - 1; ++k)
 #pragma unroll
-                for (int i = 0; i < CPL; ++i) dz[i] = g[i] * sg[i] * (1.f + z[i] * (1.f - sg[i]));
-                if (u < RUN && r.t0 + u < r.t1) {  // this run's share of the weight gradient
+            for (int i = 0; i < CPL; ++i) head[warp][k][c0 + i] = 0.f;
+    }
+    __syncthreads();
+    if (active) {  // dx of the run's last KT-1 tokens needs the next KT-1 dz
 #pragma unroll
-                    for (int i = 0; i < CPL; ++i) {
-                        dw[i][0] += dz[i] * xv[i];
-                        dw[i][1] += dz[i] * win[0][i];
-                        dw[i][2] += dz[i] * win[1][i];
-                        dw[i][3] += dz[i] * win[2][i];
-                    }
-                }
+        for (int k = 0; k < KT - 1; ++k) {
+            const int t = r.t0 + RUN + k;
+            float dz[CPL];
+            if (!last) {
+#pragma unroll
+                for (int i = 0; i < CPL; ++i) dz[i] = head[warp + 1][k][c0 + i];
+            } else if (t < Tn) {  // uniform over the warp
+                float xv[CPL];
+                unpack(xv, xs[RUN + KT - 1 + k]);
+                dz_at<CPL, NORM>(dz, wr, xv, win, dys[RUN + k]);
+                shift_in<CPL>(win, xv);
             } else {
 #pragma unroll
                 for (int i = 0; i < CPL; ++i) dz[i] = 0.f;
             }
-            shift_in<CPL>(win, xv);
-#pragma unroll
-            for (int i = 0; i < CPL; ++i) {
-                dzw[3][i] = dzw[2][i];
-                dzw[2][i] = dzw[1][i];
-                dzw[1][i] = dzw[0][i];
-                dzw[0][i] = dz[i];
-            }
-            const int te = r.t0 + u - (KT - 1);  // dx_te = sum_j w_j dz_{te+j}
-            if (te >= r.t0 && te < r.t1) {
-                float gx[CPL];
-#pragma unroll
-                for (int i = 0; i < CPL; ++i)
-                    gx[i] = wr[i][0] * dzw[3][i] + wr[i][1] * dzw[2][i] + wr[i][2] * dzw[1][i] +
-                            wr[i][3] * dzw[0][i];
-                store_ch<T, CPL>(dx + base + (size_t)te * rs, gx);
-            }
+            push_dz<CPL>(dzw, dz);
+            emit_dx<T, CPL>(dx + base, rs, wr, dzw, t - (KT - 1), r.t0, r.t1);
         }
     }
     // The CTA's weight-gradient partial: warps summed in a fixed order.
