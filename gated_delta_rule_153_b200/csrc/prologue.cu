@@ -285,7 +285,7 @@ short_conv_bwd_kernel(int Tn, int H, int K, int tiles, const T* __restrict__ x,
     constexpr int RUN = RUN_B;
     constexpr int NZ = RUN + KT - 1;        // dz_{t0} .. dz_{t0+RUN+2}
     constexpr int NX = NZ + KT - 1;         // x_{t0-3} .. x_{t0+RUN+2}
-    __shared__ float red[PW][D * KT];
+    __shared__ float red[PW][KT][D];  // tap-major: a lane's CPL channels are contiguous
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, c0 = lane * CPL;
     const Tile r = tile_of<RUN>(H, tiles, Tn);
     const bool active = r.t0 < r.t1;  // uniform over the warp
@@ -335,7 +335,7 @@ short_conv_bwd_kernel(int Tn, int H, int K, int tiles, const T* __restrict__ x,
             }
             if (u < KT - 1) {
 #pragma unroll
-                for (int i = 0; i < CPL; ++i) head[warp][u][c0 + i] = dz[i];
+                for (int i = 0; i < CPL; ++i) head[warp][u][c0 + i] = dz[i];  // contiguous per lane
             }
             shift_in<CPL>(win, xv);
             push_dz<CPL>(dzw, dz);
@@ -371,39 +371,40 @@ short_conv_bwd_kernel(int Tn, int H, int K, int tiles, const T* __restrict__ x,
     }
     // The CTA's weight-gradient partial: warps summed in a fixed order.
 #pragma unroll
-    for (int i = 0; i < CPL; ++i)
+    for (int j = 0; j < KT; ++j)
 #pragma unroll
-        for (int j = 0; j < KT; ++j) red[warp][(c0 + i) * KT + j] = dw[i][j];
+        for (int i = 0; i < CPL; ++i) red[warp][j][c0 + i] = dw[i][j];
     __syncthreads();
     for (int e = threadIdx.x; e < D * K; e += PW * 32) {
         const int c = e / K, j = e % K;
         float acc = 0.f;
 #pragma unroll
-        for (int q = 0; q < PW; ++q) acc += red[q][c * KT + j];
+        for (int q = 0; q < PW; ++q) acc += red[q][j][c];
         part[(size_t)blockIdx.x * D * K + e] = acc;  // slot (b, tile, h) = blockIdx.x
     }
 }
 
-// dw[e] = sum over the (b, tile) partials of e, in that order.  A CTA owns 32
-// consecutive e (one per lane); its warps take interleaved partials, then add
-// their sums in warp order.
-__global__ void __launch_bounds__(PW * 32)
+// dw[e] = sum over the (b, tile) partials of e, in a fixed order.  A CTA owns
+// 32 consecutive e (one per lane); its RW warps take interleaved partials (a
+// coalesced 128-byte row each), then their sums are added in warp order.
+constexpr int RW = 32;
+__global__ void __launch_bounds__(RW * 32)
 short_conv_dw_reduce_kernel(const float* __restrict__ part, int nparts, int per,
                             float* __restrict__ dw) {
-    __shared__ float red[PW][32];
+    __shared__ float red[RW][33];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int e = blockIdx.x * 32 + lane;
     float acc = 0.f;
     if (e < per) {
-#pragma unroll 8
-        for (int p = warp; p < nparts; p += PW) acc += part[(size_t)p * per + e];
+#pragma unroll 4
+        for (int p = warp; p < nparts; p += RW) acc += part[(size_t)p * per + e];
     }
     red[warp][lane] = acc;
     __syncthreads();
     if (warp == 0 && e < per) {
         float t = 0.f;
 #pragma unroll
-        for (int q = 0; q < PW; ++q) t += red[q][lane];
+        for (int q = 0; q < RW; ++q) t += red[q][lane];
         dw[e] = t;
     }
 }
@@ -517,7 +518,7 @@ gdn_status gdn_short_conv_bwd(int B, int T, int H, int d, int K, gdn_dtype dtype
         dispatch_bwd<float>(B, T, H, d, K, l2norm != 0, x, w, dy, dx, part, st);
     const int per = H * d * K;
     GDN_LAUNCH("short_conv_dw_reduce", st,
-               (short_conv_dw_reduce_kernel<<<(per + 31) / 32, PW * 32, 0, st>>>(
+               (short_conv_dw_reduce_kernel<<<(per + 31) / 32, RW * 32, 0, st>>>(
                    part, B * tiles_of(T, RUN_B), per, dw)));
     return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
