@@ -67,6 +67,7 @@ def _failed_pins(lib):
     return failed
 
 
+@pytest.mark.filterwarnings("ignore::RuntimeWarning")  # a mutant's numbers may overflow
 @pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
 def test_pins_catch_mutant(name, old, new):
     with tempfile.TemporaryDirectory() as d:
