@@ -35,36 +35,6 @@ constexpr int PW = 8;          // warps per CTA
 constexpr float kNormEps = 1e-6f;
 
 template <typename T, int CPL>
-GDN_DEV void load_ch(float (&v)[CPL], const T* p);
-template <>
-GDN_DEV void load_ch<__nv_bfloat16, 4>(float (&v)[4], const __nv_bfloat16* p) {
-    const uint2 u = *reinterpret_cast<const uint2*>(p);
-    const float2 a = unpack_bf16(u.x), b = unpack_bf16(u.y);
-    v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
-}
-template <>
-GDN_DEV void load_ch<__nv_bfloat16, 2>(float (&v)[2], const __nv_bfloat16* p) {
-    const float2 a = unpack_bf16(*reinterpret_cast<const uint32_t*>(p));
-    v[0] = a.x; v[1] = a.y;
-}
-template <>
-GDN_DEV void load_ch<__nv_bfloat16, 1>(float (&v)[1], const __nv_bfloat16* p) {
-    v[0] = __bfloat162float(*p);
-}
-template <>
-GDN_DEV void load_ch<float, 4>(float (&v)[4], const float* p) {
-    const float4 a = *reinterpret_cast<const float4*>(p);
-    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-}
-template <>
-GDN_DEV void load_ch<float, 2>(float (&v)[2], const float* p) {
-    const float2 a = *reinterpret_cast<const float2*>(p);
-    v[0] = a.x; v[1] = a.y;
-}
-template <>
-GDN_DEV void load_ch<float, 1>(float (&v)[1], const float* p) { v[0] = *p; }
-
-template <typename T, int CPL>
 GDN_DEV void store_ch(T* p, const float (&v)[CPL]);
 template <>
 GDN_DEV void store_ch<__nv_bfloat16, 4>(__nv_bfloat16* p, const float (&v)[4]) {
