@@ -208,3 +208,17 @@ def test_short_conv_checks():
         gdn.GDN_ERR_WORKSPACE
     assert b(2, 100, 3, 128, 4, bf, 1, p, p, ctypes.c_void_p(512), p, p, p, 1 << 30, None) == \
         gdn.GDN_ERR_INVALID_ARG  # dx aliases x
+
+
+def test_header_is_plain_c(tmp_path):
+    """include/gdn.h compiles as C11 on its own, and every entry point it
+    declares can be named from C (taking each one's address)."""
+    import subprocess
+    names = sorted(_declared())
+    src = tmp_path / "use.c"
+    src.write_text('#include "gdn.h"\ntypedef void (*entry)(void);\n' +
+                   "entry gdn_entry_points[] = {\n" +
+                   "".join(f"    (entry)&{n},\n" for n in names) + "};\n")
+    subprocess.run(["gcc", "-std=c11", "-Wall", "-Werror", "-pedantic", "-c",
+                    "-I", os.path.join(ROOT, "include"), str(src), "-o", str(tmp_path / "use.o")],
+                   check=True)
