@@ -55,40 +55,40 @@ def peaks():
     return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
 
 
-# Per-kernel algorithmic traffic / work per launch for the roofline object.
-# Bytes are the unique bytes each kernel must read and write (inputs, its
-# workspace products, outputs); flops are its tensor-core products.
+# Per-kernel algorithmic bytes per launch for the roofline object: the bytes
+# of the layer's own tensors (q, k, v, g, beta, o, dO, dq, dk, dv, dg, dbeta,
+# states) that the kernel must read or write, counted once per launch.  The
+# workspace images the kernels pass to each other are implementation traffic,
+# not algorithmic bytes: they show up in the measured DRAM traffic, and the
+# ratio traffic / algorithmic is reported as the waste factor.
+TH_BYTES = {
+    # reads q, k, v (bf16) and g, beta (fp32)
+    "tc_prep": 3 * 256 + 8, "tc5_prep": 3 * 256 + 8,
+    # reads q, k; writes o
+    "tc_walk_fwd": 3 * 256, "tc5_walk_fwd": 3 * 256, "tc5_seg_fwd": 3 * 256,
+    # reads k (and v through the prepared images): k only
+    "tc_walk_states": 256, "tc5_walk_states": 256, "tc5_seg_map": 256,
+    # reads q, k, dO
+    "tc_walk_bwd": 3 * 256, "tc5_walk_bwd": 3 * 256,
+    # reads q, k, v, dO, g, beta; writes dq, dk, dv, dg, dbeta: the whole
+    # backward's method bytes
+    "tc_bwd_local": BWD_BYTES, "tc5_bwd_local": BWD_BYTES,
+    "simt_bwd": BWD_BYTES, "simt_fwd": FWD_BYTES,
+}
+
+
 def kernel_work(name, B, T, H):
     th = B * T * H           # token-heads
-    nchunks = B * H * ((T + 63) // 64)
-    if name == "tc_prep":
-        # reads q,k,v (bf16), g, beta; writes W, U~ (bf16 C x 128), P (bf16 C x C), G
-        return dict(bound="hbm", bytes=th * (3 * 256 + 8 + 2 * 256 + 128 + 4))
-    if name in ("tc_walk_fwd", "tc5_walk_fwd"):
-        # reads W, Q, K, U~ (bf16), P, G; writes O
-        return dict(bound="hbm", bytes=th * (4 * 256 + 128 + 4 + 256))
-    if name in ("tc_walk_states", "tc5_walk_states"):
-        # reads W, K, U~, G; writes S0 per chunk (bf16) and U
-        return dict(bound="hbm", bytes=th * (3 * 256 + 4 + 256) + nchunks * 128 * 128 * 2)
-    if name in ("tc_walk_bwd", "tc5_walk_bwd"):
-        # reads P, dO, Q, K, W, G; writes dS per chunk (bf16), dU
-        return dict(bound="hbm", bytes=th * (128 + 4 * 256 + 4 + 256) + nchunks * 128 * 128 * 2)
-    if name == "tc_bwd_local":
-        # reads q,k,v,dO,U,dU (bf16), S0, dS per chunk, g, beta; writes dq,dk,dv, dg, dbeta
-        return dict(bound="hbm", bytes=th * (6 * 256 + 8 + 3 * 256 + 8)
-                    + nchunks * 2 * 128 * 128 * 2)
-    if name == "simt_bwd":
-        return dict(bound="hbm", bytes=th * BWD_BYTES)
-    if name == "simt_fwd":
-        return dict(bound="hbm", bytes=th * FWD_BYTES)
     if name == "decode_step":
         return dict(bound="hbm", bytes=B * H * (2 * 128 * 128 * 4 + 4 * 256 + 8))
-    return dict(bound="hbm", bytes=th * FWD_BYTES)
+    return dict(bound="hbm", bytes=th * TH_BYTES.get(name, FWD_BYTES))
 
 
 # Kernel -> source file, for matching a recorded ncu traffic figure to the
 # code it was taken on (profiles/roofline_traffic.md).
 KERNEL_SOURCE = {"tc_prep": "tc_chunk.cu", "tc_walk_fwd": "tc_chunk.cu",
+                 "tc5_prep": "tc5_prep.cu", "tc5_bwd_local": "tc5_bwd_local.cu",
+                 "tc5_seg_fwd": "tc5_walk.cu", "tc5_seg_map": "tc5_walk.cu",
                  "tc5_walk_fwd": "tc5_walk.cu", "tc5_walk_states": "tc5_walk.cu",
                  "tc5_walk_bwd": "tc5_walk_bwd.cu",
                  "tc_walk_states": "tc_chunk.cu", "tc_walk_bwd": "tc_bwd.cu",
@@ -257,19 +257,16 @@ def run_ours(args, rank, world, dev, barrier, max_over_ranks):
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    cap = 8 * max(args.steps, 1) + 64
     idx = torch.cuda.current_device()
     with ClockSampler(idx) as clk:
         barrier()
         torch.cuda.synchronize()
-        gdn.gdn_profile_begin(cap)
         s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         s.record()
         for _ in range(args.steps):
             step()
         e.record()
         torch.cuda.synchronize()
-        nlaunch, launches = gdn.gdn_profile_end(cap)
         barrier()
         torch.cuda.synchronize()
     ms_total = s.elapsed_time(e)
@@ -280,6 +277,20 @@ def run_ours(args, rank, world, dev, barrier, max_over_ranks):
     th = cfg.B * cfg.T * cfg.H
     flops_step = (FWD_FLOP + BWD_FLOP) * th
     tflops = world * flops_step * args.steps / (ms_total / 1e3) / 1e12
+
+    # ---- per-kernel times: a separate pass with the launch hook on -----------
+    # (two events per launch on the launching stream; kept out of the
+    # headline's timed region)
+    psteps = min(max(args.steps // 5, 5), 50)
+    cap = 16 * psteps + 64
+    torch.cuda.synchronize()
+    gdn.gdn_profile_begin(cap)
+    for _ in range(psteps):
+        step()
+    torch.cuda.synchronize()
+    nlaunch_p, launches = gdn.gdn_profile_end(cap)
+    per_step_launches = nlaunch_p / psteps
+    nlaunch = int(round(per_step_launches * args.steps))
 
     # ---- roofline of the dominant kernel ------------------------------------
     per = {}
@@ -293,12 +304,22 @@ def run_ours(args, rank, world, dev, barrier, max_over_ranks):
     traffic = recorded_traffic(dom)
     roofline = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1),
                 "peak": pk["hbm"], "unit": "GB/s", "frac": round(achieved / pk["hbm"], 4),
-                "peak_source": pk["source"], "traffic": traffic,
+                "peak_source": pk["source"] + " (burst copy, MEASURED_PEAKS.json)",
+                "traffic": traffic,
+                "waste": round(traffic / wk["bytes"], 3) if traffic else None,
                 "algorithmic_bytes": wk["bytes"],
+                "algorithmic_bytes_rule": "layer tensors the kernel reads or writes "
+                                          "(per token-head: fwd 1032 B, bwd 1808 B in all)",
                 "avg_launch_ms": round(dom_ms, 4),
                 "share": round(sum(per[dom]) / total_k, 4),
                 "kernels": {n: {"launches": len(v), "avg_ms": round(statistics.mean(v), 4),
                                 "share": round(sum(v) / total_k, 4)} for n, v in per.items()}}
+    step_bytes = (FWD_BYTES + BWD_BYTES) * th
+    step_hbm = step_bytes / (ms_step / 1e3) / 1e9
+    roofline["step"] = {"algorithmic_bytes": step_bytes, "hbm_gbs": round(step_hbm, 1),
+                        "frac_hbm": round(step_hbm / pk["hbm"], 4),
+                        "tflops": round(flops_step / (ms_step / 1e3) / 1e12, 2),
+                        "frac_tensor": round(flops_step / (ms_step / 1e3) / 1e12 / pk["bf16"], 4)}
 
     extra = {}
     if not args.headline_only:
@@ -312,11 +333,22 @@ def run_ours(args, rank, world, dev, barrier, max_over_ranks):
         ms_f = timed(fwd, max(args.steps, 10), args.warmup, barrier)
         lth = LONG.B * LONG.T * LONG.H
         lt = FWD_FLOP * lth / (ms_f / 1e3) / 1e12
+        lflop = FWD_FLOP * lth
+        lbytes = FWD_BYTES * lth + 2 * LONG.B * LONG.H * LONG.dv * LONG.dk * 4  # + h0, hT
+        intensity = lflop / lbytes
+        attainable = min(pk["bf16"], intensity * pk["hbm"] / 1e3)  # TFLOP/s
         extra["long_context_fwd"] = {
             "workload": LONG.name, "ms": round(ms_f, 4),
             "tokens_per_s": round(LONG.B * LONG.T / (ms_f / 1e3), 1),
             "tflops": round(lt, 2), "frac_tensor_peak": round(lt / pk["bf16"], 4),
-            "hbm_gbs": round(FWD_BYTES * lth / (ms_f / 1e3) / 1e9, 1)}
+            "hbm_gbs": round(lbytes / (ms_f / 1e3) / 1e9, 1),
+            "roofline": {"bound": "tensor", "achieved": round(lt, 2), "peak": pk["bf16"],
+                         "unit": "TFLOP/s", "frac": round(lt / pk["bf16"], 4),
+                         "flop_per_launch": lflop, "algorithmic_bytes": lbytes,
+                         "intensity_flop_per_byte": round(intensity, 1),
+                         "attainable_tflops": round(attainable, 1),
+                         "frac_attainable": round(lt / attainable, 4),
+                         "peak_source": pk["source"] + " (burst cuBLAS bf16)"}}
         ms_fb = timed(chunk_step_fn(gdn, li, lws_f, workspaces(gdn, li)[1],
                                     dict(o=lo, hT=lh)), 3, 1, barrier)
         extra["long_context_fwd_bwd_ms"] = round(ms_fb, 3)
@@ -523,7 +555,7 @@ def main():
         if rank != 0:
             return
         from gated_delta_rule_153_b200.inputs import L350M
-        sample_B = 1
+        sample_B = L350M.B
         vals = []
         for i in range(args.warmup + args.steps):
             v, dt, cores = cpu_baseline_oracle(sample_B)
@@ -531,8 +563,8 @@ def main():
                 vals.append((v, dt))
         tot = sum(dt for _, dt in vals)
         value = len(vals) * sample_B * L350M.T / tot
-        sample = (f"fwd+bwd of 1 of 8 sequences (T=2048, H=8, d=128) of the 350M-scale "
-                  f"workload per step, fp64 token loop, OpenMP over heads")
+        sample = (f"fwd+bwd of all {sample_B} sequences (T=2048, H=8, d=128) of the 350M-scale "
+                  f"workload per step, fp64 token loop, OpenMP over (sequence, head)")
         print(json.dumps({
             "impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": "tokens/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,

@@ -742,3 +742,9 @@ extern "C" gdn_status gdn_chunk_fwd_noalloc(const gdn_dims* d, const void* q, co
     if (!gdn::launch_tc_fwd(*d, q, k, v, g, beta, h0, o, hT, ws, st)) return GDN_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
+
+extern "C" gdn_status gdn_noalloc_device_status(gdn_stream_t stream) {
+    void* ws = gdn::noalloc_scratch();
+    if (!ws) return GDN_ERR_CUDA;
+    return gdn_query_device_status(ws, stream);
+}

@@ -1,8 +1,8 @@
 // tree.cu -- draft-tree verification and commit for the gated delta rule.
 //
-// "TreeWY: Speculative Verification for Gated DeltaNet Hybrids" (paper list
-// of the "Linear Attention Architectures: Mechanisms, Trade-offs, and
-// Cross-Layer Routing" summary page): score every node of a speculative draft
+// "TreeWY: Speculative Verification for Gated DeltaNet Hybrids" (the
+// "Linked reviews" entry of the "Gated Delta Networks: Improving Mamba2
+// with Delta Rule" review page): score every node of a speculative draft
 // tree against the committed state with one triangular solve instead of one
 // state snapshot per node, and rebuild only the accepted state on commit.
 //

@@ -174,9 +174,8 @@ gdn_status gdn_short_conv_bwd(int B, int T, int H, int d, int K, gdn_dtype dtype
                               size_t ws_bytes, gdn_stream_t stream);
 
 /* Draft-tree verification and commit: "TreeWY: Speculative Verification for
- * Gated DeltaNet Hybrids" (paper list of the "Linear Attention
- * Architectures: Mechanisms, Trade-offs, and Cross-Layer Routing" summary
- * page).  Per (sequence n, head h) a speculative draft tree of M nodes hangs
+ * Gated DeltaNet Hybrids" (the "Linked reviews" entry of the "Gated Delta
+ * Networks: Improving Mamba2 with Delta Rule" review page).  Per (sequence n, head h) a speculative draft tree of M nodes hangs
  * below the committed state S = state[n, h]: node i carries one token and a
  * parent index parent[n, i] in [-1, i) (-1: the node follows S directly;
  * parents precede children).  Node i's output is the gated delta rule of
@@ -282,11 +281,25 @@ gdn_status gdn_query_device_status(void *ws, gdn_stream_t stream);
  * one array and a call leaves its contents behind: the call clears the word
  * that must start at zero itself, but calls that overlap on the GPU (other
  * streams, other host threads) race on the array and must be serialised by
- * the caller.  Device-side wait timeouts of these calls are not reported. */
+ * the caller.  The array's address is looked up once per device and kept
+ * for the life of the process, so these calls must not be used after
+ * cudaDeviceReset (or anything else that destroys the device's primary
+ * context) in the same process.  A device wait of these calls that gives up
+ * is reported by gdn_noalloc_device_status, not by the return value. */
 gdn_status gdn_chunk_fwd_noalloc(const gdn_dims *dims, const void *q, const void *k,
                                  const void *v, const float *g, const float *beta,
                                  const float *h0, void *o, float *hT,
                                  gdn_stream_t stream);
+
+/* Companion of gdn_chunk_fwd_noalloc, with no counterpart in the paper
+ * either: synchronises `stream`, then reads and clears the status word at
+ * the start of the library's built-in array on the current device, exactly
+ * as gdn_query_device_status does for a caller's workspace.  The answer
+ * covers the most recent gdn_chunk_fwd_noalloc call on this device:
+ * GDN_ERR_DEVICE_TIMEOUT if one of its bounded device waits gave up (its
+ * o / hT are then not valid), else GDN_OK; GDN_ERR_CUDA if a CUDA call
+ * failed.  Allocates nothing. */
+gdn_status gdn_noalloc_device_status(gdn_stream_t stream);
 
 /* Per-launch timing, a profiling aid (off by default; no compute happens in
  * these calls).  gdn_profile_begin(capacity) makes the calling host thread's

@@ -4,9 +4,9 @@ INFRASTRUCTURE ONLY.
 Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU legs of ``bench.py``
 may import this module; the CUDA library never uses it.
 
-Source: "TreeWY: Speculative Verification for Gated DeltaNet Hybrids" (in the
-paper list of the "Linear Attention Architectures: Mechanisms, Trade-offs, and
-Cross-Layer Routing" summary page).  The page gives the goal, not the
+Source: "TreeWY: Speculative Verification for Gated DeltaNet Hybrids" (the
+"Linked reviews" entry of the "Gated Delta Networks: Improving Mamba2 with
+Delta Rule" review page).  The page gives the goal, not the
 equations: score every node of a speculative draft tree against the committed
 recurrent state without keeping one state snapshot per draft position, and on
 commit rebuild only the state of the accepted node.  The reading taken here:

@@ -218,3 +218,21 @@ def test_many_chunks_one_head(dev):
     inp = make_chunk_inputs(L350M, B=1, H=1, T=16384, g_shift=-3.0, h0_std=0.1, dhT_std=0.2)
     check_fwd(inp, dev)
     check_bwd(inp, dev)
+
+
+def test_kda_full_size_fwd_bwd(dev):
+    """The channel-gate workload at its own size (B=2, H=32, T=4096): 64
+    heads take the whole-head tcgen05 walks with the channel gate over
+    64-chunk chains, forward, state recompute and reverse walk."""
+    inp = make_chunk_inputs(KDA, dhT_std=0.3)
+    check_fwd(inp, dev)
+    check_bwd(inp, dev)
+
+
+def test_kda_slow_gate_whole_head_long_chain(dev):
+    """Channel gate near 1 (g shift -6) on the whole-head walks over
+    16-chunk chains, with h0 and dhT: the inter-chunk path carries the
+    signal, so a wrong per-key decay of the state would show."""
+    inp = make_chunk_inputs(KDA, T=1024, g_shift=-6.0, h0_std=0.1, dhT_std=0.3)
+    check_fwd(inp, dev)
+    check_bwd(inp, dev)

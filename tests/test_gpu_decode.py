@@ -41,13 +41,21 @@ def test_decode_small(dev, dtype, gate, dk, dv):
 
 def test_decode_full_config_1000_steps(dev):
     """256 sequences x 16 heads, 1000 steps; every output and the final
-    states of a seeded sample of 48 (sequence, head) pairs against the oracle,
-    and all final states checked finite and bounded."""
+    states of a sample of (sequence, head) pairs against the oracle, and all
+    final states checked finite.  The sample holds the first and the last
+    pair, one pair from every block of 16 sequences (so an indexing fault
+    confined to high sequence numbers cannot slip through), one pair of every
+    head, and 48 seeded random pairs."""
     inp = make_decode_inputs(DECODE)
     S = DECODE.steps
     o, st = _run_steps(inp, dev, S)
     rng = np.random.default_rng(0)
-    pairs = rng.choice(DECODE.N * DECODE.H, size=48, replace=False)
+    NH = DECODE.N * DECODE.H
+    blocks = [16 * blk + int(rng.integers(16)) for blk in range(DECODE.N // 16)]
+    per_block = [n * DECODE.H + int(rng.integers(DECODE.H)) for n in blocks]
+    per_head = [int(rng.integers(DECODE.N)) * DECODE.H + h for h in range(DECODE.H)]
+    pairs = np.unique(np.concatenate([[0, NH - 1], per_block, per_head,
+                                      rng.choice(NH, size=48, replace=False)]))
     n_idx, h_idx = pairs // DECODE.H, pairs % DECODE.H
     sel = lambda x: x[:, n_idx, h_idx][:, :, None]   # [S, P, 1, ...] as N=P, H=1
     q, k, v, g, b = (sel(inp[n]) for n in ("q", "k", "v", "g", "beta"))

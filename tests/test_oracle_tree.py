@@ -3,8 +3,8 @@ other than the oracle itself: the C token-loop oracle on chains, stars and the
 root paths of random trees, plus two structural invariants (only descendants
 see a node's token; relabelling the nodes in another topological order
 relabels the outputs).  Page citation: "TreeWY: Speculative Verification for
-Gated DeltaNet Hybrids" (paper list of the "Linear Attention Architectures"
-summary page) and the gated delta rule of the "Gated Delta Networks" review,
+Gated DeltaNet Hybrids" (the "Linked reviews" entry of the "Gated Delta Networks"
+review page) and the gated delta rule of the "Gated Delta Networks" review,
 section "Method"."""
 import numpy as np
 
