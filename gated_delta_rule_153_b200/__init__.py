@@ -28,7 +28,7 @@ GDN_GATE_SCALAR, GDN_GATE_CHANNEL = 0, 1
 EXPORTS = ("gdn_chunk_fwd_workspace", "gdn_chunk_fwd", "gdn_chunk_bwd_workspace",
            "gdn_chunk_bwd", "gdn_recurrent_step", "gdn_query_device_status",
            "gdn_status_string", "gdn_profile_begin", "gdn_profile_end",
-           "gdn_chunk_fwd_noalloc", "gdn_noalloc_device_status", "gdn_product_fwd_workspace", "gdn_product_fwd",
+           "gdn_chunk_fwd_noalloc", "gdn_noalloc_device_status", "gdn_test_stalled_fwd", "gdn_product_fwd_workspace", "gdn_product_fwd",
            "gdn_product_bwd_workspace", "gdn_product_bwd", "gdn_chunk_fwd_varlen_workspace",
            "gdn_chunk_fwd_varlen", "gdn_chunk_bwd_varlen_workspace", "gdn_chunk_bwd_varlen",
            "gdn_tree_verify", "gdn_tree_commit", "gdn_short_conv_fwd",
@@ -80,6 +80,9 @@ def lib() -> ctypes.CDLL:
             L.gdn_query_device_status.restype = i
             L.gdn_chunk_fwd_noalloc.argtypes = [dp, vp, vp, vp, fp, fp, fp, vp, fp, vp]
             L.gdn_chunk_fwd_noalloc.restype = i
+            L.gdn_test_stalled_fwd.argtypes = [dp, vp, vp, vp, fp, fp, fp, vp, fp, vp, sz, i,
+                                               ctypes.c_ulonglong, vp]
+            L.gdn_test_stalled_fwd.restype = i
             L.gdn_noalloc_device_status.argtypes = [vp]
             L.gdn_noalloc_device_status.restype = i
             L.gdn_product_fwd_workspace.argtypes = [dp, i]

@@ -55,14 +55,17 @@ GDN_DEV bool mbar_try(uint64_t* bar, uint32_t parity) {
 }
 
 // Bounded wait for phase `parity` of `bar`.  Returns false (and flags the
-// status word) if it did not complete within kWaitNs.
-GDN_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned int* status) {
+// status word) if it did not complete within `limit_ns` (default kWaitNs).
+// A wait that guards a copy or an MMA still in flight when the CTA is about
+// to exit (the drains before teardown) always uses the default limit.
+GDN_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned int* status,
+                       unsigned long long limit_ns = kWaitNs) {
     if (mbar_try(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     for (;;) {
         for (int i = 0; i < 64; ++i)
             if (mbar_try(bar, parity)) return true;
-        if (globaltimer() - t0 > kWaitNs) {
+        if (globaltimer() - t0 > limit_ns) {
             if (status) atomicOr(status, 1u);
             return false;
         }

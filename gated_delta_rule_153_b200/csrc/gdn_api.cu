@@ -164,6 +164,24 @@ gdn_status gdn_recurrent_step(int N, int H, int dk, int dv, gdn_dtype dtype, gdn
     return launch_status();
 }
 
+gdn_status gdn_test_stalled_fwd(const gdn_dims* d, const void* q, const void* k, const void* v,
+                                const float* g, const float* beta, const float* h0, void* o,
+                                float* hT, void* ws, size_t ws_bytes, int stall_at,
+                                unsigned long long wait_ns, gdn_stream_t stream) {
+    gdn_status s = validate_fwd_args(d, q, k, v, g, beta, h0, o, hT);
+    if (s != GDN_OK) return s;
+    if (stall_at < 0 || wait_ns == 0 || wait_ns > 1000000000ull) return GDN_ERR_INVALID_ARG;
+    if (!tc_supported(*d) || !tc_fwd_whole_head(*d)) return GDN_ERR_UNSUPPORTED;
+    const size_t need = tc_fwd_workspace(*d);
+    if (!ws || ws_bytes < need || ((uintptr_t)ws & 255u)) return GDN_ERR_WORKSPACE;
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaGetLastError();
+    if (cudaMemsetAsync(ws, 0, sizeof(unsigned int), st) != cudaSuccess) return GDN_ERR_CUDA;
+    if (!launch_tc_fwd(*d, q, k, v, g, beta, h0, o, hT, ws, st, nullptr, 0, wait_ns, stall_at))
+        return GDN_ERR_CUDA;
+    return launch_status();
+}
+
 gdn_status gdn_query_device_status(void* ws, gdn_stream_t stream) {
     if (!ws) return GDN_ERR_INVALID_ARG;
     cudaStream_t st = (cudaStream_t)stream;

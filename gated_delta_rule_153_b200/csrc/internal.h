@@ -38,9 +38,14 @@ bool tc_bwd_supported(const gdn_dims& d);
 size_t tc_fwd_workspace(const gdn_dims& d, int nseq = 0);
 size_t tc_bwd_workspace(const gdn_dims& d, int nseq = 0);
 // Return false if a TMA tensor map could not be encoded (nothing launched).
+// wait_ns / stall_at: the bounded-wait limit and the stall test hook of the
+// tcgen05 forward walk (defaults: 1 s, no stall).
 bool launch_tc_fwd(const gdn_dims& d, const void* q, const void* k, const void* v,
                    const float* g, const float* beta, const float* h0, void* o, float* hT,
-                   void* ws, cudaStream_t st, const int* cu = nullptr, int nseq = 0);
+                   void* ws, cudaStream_t st, const int* cu = nullptr, int nseq = 0,
+                   unsigned long long wait_ns = 1000000000ull, int stall_at = -1);
+// True when the forward of these dims runs its chain on the tcgen05 whole-head walk.
+bool tc_fwd_whole_head(const gdn_dims& d);
 bool launch_tc_bwd(const gdn_dims& d, const void* q, const void* k, const void* v,
                    const float* g, const float* beta, const float* h0, const void* dO,
                    const float* dhT, void* dq, void* dk, void* dv, float* dg, float* dbeta,

@@ -1,0 +1,342 @@
+// tc5_prep.cu -- per-chunk WY preparation of the gated delta rule on the
+// fifth-generation tensor cores (scalar gate, bf16, dk = dv = 128, chunk 64).
+//
+// For one chunk of one head, with G the within-chunk cumsum of the log-gate
+// ("Gated Delta Networks: Improving Mamba2 with Delta Rule" (paper review),
+// section "Method": the gated delta rule in its chunkwise WY / UT-transform
+// form):
+//   A  = strict_lower(diag(beta) (K K^T .* D)),  D_ij = exp(G_i - G_j)
+//   T  = (I + A)^{-1}                                 (UT transform)
+//   W  = T diag(beta) (diag(e^G) K),   U~ = T diag(beta) V
+//   P  = scale lower(Q K^T .* D)
+// The products run as tcgen05 MMAs with fp32 accumulators in tensor memory:
+//   [K K^T ; Q K^T] = [K ; Q] K^T           one M = 128, N = 64 product: rows
+//                                           0..63 give A, rows 64..127 give P
+//   W^T  = (e^G K)^T (T diag(beta))^T       M = 128 (key), N = 64 (token)
+//   U~^T = V^T (T diag(beta))^T             M = 128 (value), N = 64 (token)
+// with K and Q stacked in one K-major operand (the TMA tiles of both land in
+// the same 128-row panels), and the transposed products reading the K and V
+// tiles as MN-major A operands, so no tile is copied or transposed in shared
+// memory.  The row scale e^{G_j} of W is applied to K in place once Q K^T and
+// K K^T are done, so both transposed products share the B operand T diag(beta).
+// The triangular solve keeps the 16x16 diagonal blocks of T exact in fp32
+// registers (forward substitution) and combines the off-diagonal blocks one
+// block diagonal at a time with warp-level MMAs (T_IJ = -T_II sum_K A_IK T_KJ).
+//
+// One CTA of four warps per chunk; thread t owns TMEM lane t in both
+// epilogues (row t of [K K^T ; Q K^T], then key / value row t of W^T / U~^T).
+// Shared memory ~74 KB and 128 TMEM columns, so three CTAs share an SM.
+// Outputs (bulk stores into the workspace): the W image (Tma128), the U~^T
+// image (Swz<64>, 128 value rows), P (Swz<64>), G, and optionally T (Swz<64>);
+// the K~ = diag(e^{G_last - G}) K image (Tma128) goes out with plain 16-byte
+// stores straight from the K tile.
+#include "async.cuh"
+#include "common.cuh"
+#include "internal.h"
+#include "mma.cuh"
+#include "tc5.cuh"
+#include "tc_common.cuh"
+
+namespace gdn {
+namespace {
+using namespace tc;
+
+constexpr int P5_THREADS = 128;
+constexpr uint32_t P5_TCOLS = 128;  // D1 = [KK^T; QK^T] in 0..63; then W^T 0..63, U~^T 64..127
+constexpr uint32_t ID_KQ = tc5::idesc_bf16(128, 64, false, false);
+constexpr uint32_t ID_WU = tc5::idesc_bf16(128, 64, true, false);
+constexpr int KQ_PANEL = 2 * C * 64;  // elements of one 128-row, 64-column panel
+
+struct alignas(1024) P5Smem {
+    // [K p0 | Q p0 | K p1 | Q p1], 8 KB each: panel p holds key columns 64p..64p+63
+    // of the 64 K rows then the 64 Q rows.  Once the first product is done the
+    // Q quarters hold the bf16 A (Swz<64>) and the fp32 diagonal blocks of A
+    // with the solve's scratch; once the transposed products are done the
+    // whole region holds the W image (16 KB) and the U~^T image (16 KB).
+    __nv_bfloat16 KQ[2 * KQ_PANEL];
+    __nv_bfloat16 V[C * DV];  // Tma128
+    __nv_bfloat16 P[C * C];   // Swz<64>
+    __nv_bfloat16 T[C * C];   // Swz<64>: T = (I + A)^{-1}
+    __nv_bfloat16 T2[C * C];  // Swz<64>: T diag(beta)
+    float G[C];
+    float beta[C];
+    uint64_t bar_ld, bar_mma;
+    uint32_t tmem;
+};
+
+__global__ void __launch_bounds__(P5_THREADS, 3) tc5_prep_kernel(const __grid_constant__ ChunkPtrs p) {
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    P5Smem& s = *reinterpret_cast<P5Smem*>(align1k(smem_raw));
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int cid = blockIdx.x;
+    const int bh = cid / p.NT, n = cid % p.NT, h = bh % p.H;
+    const ChunkLoc cl = chunk_loc(p.seq, p.T, p.H, bh, n);
+    if (!cl.valid) return;  // past the last chunk of a packed batch
+    const int L = cl.L;
+    const size_t row0 = (size_t)cl.tok * p.H + h;  // token-head index of row 0
+    const size_t rs = (size_t)p.H;                 // token-head stride between rows
+
+    if (tid == 0) {
+        mbar_init(&s.bar_ld, 1);
+        mbar_init(&s.bar_mma, 1);
+        fence_mbar_init();
+        // rows past L hold the next sequence's tokens (or zeros past the
+        // tensor): finite, and annihilated by beta = 0 on those rows
+        mbar_arrive_expect(&s.bar_ld, 3 * C * DK * 2);
+        tma_load_3d(s.KQ, &p.kmap, 0, h, cl.tok, &s.bar_ld);
+        tma_load_3d(s.KQ + C * 64, &p.qmap, 0, h, cl.tok, &s.bar_ld);
+        tma_load_3d(s.KQ + KQ_PANEL, &p.kmap, 64, h, cl.tok, &s.bar_ld);
+        tma_load_3d(s.KQ + KQ_PANEL + C * 64, &p.qmap, 64, h, cl.tok, &s.bar_ld);
+        tma_load_tile(s.V, &p.vmap, h, cl.tok, &s.bar_ld);
+    }
+    if (warp == 0) {
+        tc5::alloc(&s.tmem, P5_TCOLS);
+        // inclusive cumsum of the log-gate over the chunk (rows past L add 0)
+        float g0 = lane < L ? p.g[row0 + lane * rs] : 0.f;
+        float g1 = lane + 32 < L ? p.g[row0 + (lane + 32) * rs] : 0.f;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float x0 = __shfl_up_sync(0xffffffffu, g0, o);
+            const float x1 = __shfl_up_sync(0xffffffffu, g1, o);
+            if (lane >= o) { g0 += x0; g1 += x1; }
+        }
+        g1 += __shfl_sync(0xffffffffu, g0, 31);
+        s.G[lane] = g0;
+        s.G[lane + 32] = g1;
+        s.beta[lane] = lane < L ? p.beta[row0 + lane * rs] : 0.f;
+        s.beta[lane + 32] = lane + 32 < L ? p.beta[row0 + (lane + 32) * rs] : 0.f;
+    }
+    tc5::fence_before();
+    __syncthreads();
+    tc5::fence_after();
+    const uint32_t tm = s.tmem;
+    const uint32_t sKQ = smem_u32(s.KQ);
+    bool ok = true;
+
+    // ---- [K K^T ; Q K^T] ---------------------------------------------------
+    if (tid == 0) {
+        ok = mbar_wait(&s.bar_ld, 0, p.status);
+        if (ok) {
+#pragma unroll
+            for (int kk = 0; kk < DK / 16; ++kk)
+                tc5::mma(tm, tc5::kmajor<2 * C>(sKQ, kk), tc5::kmajor<2 * C>(sKQ, kk), ID_KQ, kk > 0);
+            tc5::commit(&s.bar_mma);
+        }
+    }
+    if (__syncthreads_or(!ok)) goto done;
+    ok = mbar_wait(&s.bar_mma, 0, p.status);
+    if (__syncthreads_or(!ok)) goto done;
+    tc5::fence_after();
+
+    // Q is dead: its first quarter holds the bf16 A, its second the fp32
+    // diagonal blocks of A and each warp's 16x16 scratch of the solve.
+    {
+        __nv_bfloat16* Abf = s.KQ + C * 64;
+        auto Ad = reinterpret_cast<float(*)[16][17]>(s.KQ + KQ_PANEL + C * 64);
+        auto Xs = reinterpret_cast<__nv_bfloat16(*)[16 * 16]>(
+            reinterpret_cast<unsigned char*>(s.KQ + KQ_PANEL + C * 64) + 4 * 16 * 17 * sizeof(float));
+
+        // ---- epilogue 1: thread t = row t of [K K^T ; Q K^T] ---------------
+        {
+            const uint32_t trow = tm + ((uint32_t)(32 * warp) << 16);
+            float v[64];
+            tc5::ld32(*reinterpret_cast<float(*)[32]>(&v[0]), trow);
+            tc5::ld32(*reinterpret_cast<float(*)[32]>(&v[32]), trow + 32);
+            tc5::wait_ld();
+            const bool is_a = tid < C;
+            const int r = is_a ? tid : tid - C;
+            const float Gr = s.G[r];
+            // A row r: beta_r (k_r . k_c) e^{G_r - G_c} for c < r;
+            // P row r: scale (q_r . k_c) e^{G_r - G_c} for c <= r (rows past L zero)
+            const float f = is_a ? s.beta[r] : (r < L ? p.scale : 0.f);
+            const int lim = is_a ? r : r + 1;
+#pragma unroll
+            for (int c = 0; c < 64; ++c) v[c] = (c < lim) ? f * v[c] * __expf(Gr - s.G[c]) : 0.f;
+            __nv_bfloat16* dst = is_a ? Abf : s.P;
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                *reinterpret_cast<uint4*>(dst + swz<C>(r, 8 * j)) =
+                    make_uint4(pack_bf16(v[8 * j], v[8 * j + 1]), pack_bf16(v[8 * j + 2], v[8 * j + 3]),
+                               pack_bf16(v[8 * j + 4], v[8 * j + 5]), pack_bf16(v[8 * j + 6], v[8 * j + 7]));
+            if (is_a) {
+                const int b = r >> 4;
+#pragma unroll
+                for (int c = 0; c < 64; ++c)
+                    if ((c >> 4) == b) Ad[b][r & 15][c & 15] = v[c];
+            }
+        }
+        tc5::fence_before();
+        __syncthreads();
+
+        // ---- K~ = diag(e^{G_last - G}) K to the workspace (the walks' B of
+        // the state update), and K <- diag(e^G) K in place (the row scale of W)
+        {
+            const int r = tid >> 1, pn = tid & 1;
+            const float e = __expf(s.G[r]), dec = __expf(s.G[C - 1] - s.G[r]);
+            __nv_bfloat16* row = s.KQ + pn * KQ_PANEL + r * 64;
+            // same swizzled position in the Tma128 image (panel pn at pn * 4096)
+            __nv_bfloat16* kt = p.Kt + (size_t)cid * C * DK + pn * (C * 64) + r * 64;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                uint4 x = *reinterpret_cast<uint4*>(row + 8 * j), y;
+                uint32_t* w = reinterpret_cast<uint32_t*>(&x);
+                uint32_t* wt = reinterpret_cast<uint32_t*>(&y);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float2 f2 = unpack_bf16(w[i]);
+                    w[i] = pack_bf16(f2.x * e, f2.y * e);
+                    wt[i] = pack_bf16(f2.x * dec, f2.y * dec);
+                }
+                *reinterpret_cast<uint4*>(row + 8 * j) = x;
+                *reinterpret_cast<uint4*>(kt + 8 * j) = y;
+            }
+        }
+
+        // ---- UT transform, diagonal block `warp`: forward substitution ------
+        // Lane c (< 16) owns column c of T_ww in registers.
+        const int m0 = 16 * warp;
+        {
+            const int c = lane & 15;
+            float t[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                float v = (i == c) ? 1.f : 0.f;
+#pragma unroll
+                for (int j = 0; j < i; ++j) v -= Ad[warp][i][j] * t[j];
+                t[i] = (i < c) ? 0.f : v;
+            }
+            if (lane < 16) {
+                const float bc = s.beta[m0 + c];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    s.T[swz<C>(m0 + i, m0 + c)] = __float2bfloat16_rn(t[i]);
+                    s.T2[swz<C>(m0 + i, m0 + c)] = __float2bfloat16_rn(t[i] * bc);
+                }
+            }
+            // zero this warp's row block right of the diagonal block
+            for (int e = lane; e < 16 * C; e += 32) {
+                const int r = e >> 6, cc = e & 63;
+                if (cc >= m0 + 16) {
+                    s.T[swz<C>(m0 + r, cc)] = __float2bfloat16_rn(0.f);
+                    s.T2[swz<C>(m0 + r, cc)] = __float2bfloat16_rn(0.f);
+                }
+            }
+        }
+        __syncthreads();
+        // ---- off-diagonal blocks, one block diagonal at a time --------------
+        //   T_IJ = -T_II sum_{K=J}^{I-1} A_IK T_KJ
+        for (int dgl = 1; dgl < 4; ++dgl) {
+            const int J = warp, I = warp + dgl;
+            if (I < 4) {
+                float x[2][4] = {};
+                for (int Kb = J; Kb < I; ++Kb) {
+                    uint32_t a[4], bt[4];
+                    lda<Swz<64>>(a, Abf, 16 * I, 16 * Kb);
+                    ldb_kn<Swz<64>>(bt, s.T, 16 * Kb, 16 * J);
+                    mma16816(x[0], a, bt[0], bt[1]);
+                    mma16816(x[1], a, bt[2], bt[3]);
+                }
+#pragma unroll
+                for (int jn = 0; jn < 2; ++jn) {
+                    const int r = lane >> 2, cc = 8 * jn + 2 * (lane & 3);
+                    *reinterpret_cast<uint32_t*>(&Xs[warp][r * 16 + cc]) = pack_bf16(x[jn][0], x[jn][1]);
+                    *reinterpret_cast<uint32_t*>(&Xs[warp][(r + 8) * 16 + cc]) = pack_bf16(x[jn][2], x[jn][3]);
+                }
+                __syncwarp();
+                uint32_t a[4], bx[4];
+                lda<Swz<64>>(a, s.T, 16 * I, 16 * I);
+                {
+                    const int idx = lane >> 3;
+                    const int row = (lane & 7) + (idx & 1) * 8, col = (idx >> 1) * 8;
+                    ldsm_x4_t(bx, smem_u32(&Xs[warp][row * 16 + col]));
+                }
+                float y[2][4] = {};
+                mma16816(y[0], a, bx[0], bx[1]);
+                mma16816(y[1], a, bx[2], bx[3]);
+#pragma unroll
+                for (int jn = 0; jn < 2; ++jn) {
+                    const int cc = 16 * J + 8 * jn + 2 * (lane & 3);
+                    const float b0 = s.beta[cc], b1 = s.beta[cc + 1];
+                    float z[4] = {-y[jn][0], -y[jn][1], -y[jn][2], -y[jn][3]};
+                    float z2[4] = {z[0] * b0, z[1] * b1, z[2] * b0, z[3] * b1};
+                    st_c<Swz<64>>(s.T, 16 * I, 16 * J + 8 * jn, z);
+                    st_c<Swz<64>>(s.T2, 16 * I, 16 * J + 8 * jn, z2);
+                }
+            }
+            __syncthreads();
+        }
+    }
+
+    // ---- W^T = (e^G K)^T T2^T ; U~^T = V^T T2^T ------------------------------
+    fence_async_smem();  // scaled K and T2 (generic writes) -> tensor-core reads
+    tc5::fence_before();
+    __syncthreads();
+    if (tid == 0) {
+        tc5::fence_after();
+        const uint32_t sT2 = smem_u32(s.T2), sV = smem_u32(s.V);
+#pragma unroll
+        for (int kk = 0; kk < C / 16; ++kk)
+            tc5::mma(tm, tc5::mnmajor(sKQ, kk, KQ_PANEL * 2), tc5::kmajor<C>(sT2, kk), ID_WU, kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < C / 16; ++kk)
+            tc5::mma(tm + 64, tc5::mnmajor(sV, kk, C * 128), tc5::kmajor<C>(sT2, kk), ID_WU, kk > 0);
+        tc5::commit(&s.bar_mma);
+    }
+    ok = mbar_wait(&s.bar_mma, 1, p.status);
+    if (__syncthreads_or(!ok)) goto done;
+    tc5::fence_after();
+
+    // ---- epilogue 2: thread t = key row t of W^T and value row t of U~^T -----
+    {
+        __nv_bfloat16* Wimg = s.KQ;             // Tma128, 16 KB
+        __nv_bfloat16* Uimg = s.KQ + C * DK;    // Swz<64>, 128 rows x 64 tokens
+        const uint32_t trow = tm + ((uint32_t)(32 * warp) << 16);
+        float x[32];
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            tc5::ld32(x, trow + 32 * half);
+            tc5::wait_ld();
+#pragma unroll
+            for (int t = 0; t < 32; ++t) Wimg[Tma128::off(32 * half + t, tid)] = __float2bfloat16_rn(x[t]);
+        }
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            tc5::ld32(x, trow + 64 + 32 * half);
+            tc5::wait_ld();
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                *reinterpret_cast<uint4*>(Uimg + swz<C>(tid, 32 * half + 8 * j)) =
+                    make_uint4(pack_bf16(x[8 * j], x[8 * j + 1]), pack_bf16(x[8 * j + 2], x[8 * j + 3]),
+                               pack_bf16(x[8 * j + 4], x[8 * j + 5]), pack_bf16(x[8 * j + 6], x[8 * j + 7]));
+        }
+    }
+    fence_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+        bulk_s2g(p.W + (size_t)cid * C * DK, s.KQ, C * DK * 2);
+        bulk_s2g(p.Ut + (size_t)cid * C * DV, s.KQ + C * DK, C * DV * 2);
+        bulk_s2g(p.P + (size_t)cid * C * C, s.P, C * C * 2);
+        bulk_s2g(p.G + (size_t)cid * C, s.G, C * 4);
+        if (p.Tb) bulk_s2g(p.Tb + (size_t)cid * C * C, s.T, C * C * 2);
+        bulk_commit();
+        bulk_wait_read<0>();
+    }
+done:
+    tc5::fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc5::fence_after();
+        tc5::dealloc(tm, P5_TCOLS);
+    }
+}
+
+}  // namespace
+
+namespace tc {
+void launch_prep5(const ChunkPtrs& p, size_t nchunks, cudaStream_t st) {
+    const int smem = sizeof(P5Smem) + 1024;
+    cudaFuncSetAttribute(tc5_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    GDN_LAUNCH("tc5_prep", st, tc5_prep_kernel<<<(unsigned)nchunks, P5_THREADS, smem, st>>>(p));
+}
+}  // namespace tc
+}  // namespace gdn

@@ -5,40 +5,44 @@
 // review), section "Method": U = U~ - W S0^T, O = scale diag(e^G) Q S0^T + P U,
 // S1 = e^{G_last} S0 + U^T diag(e^{G_last - G}) K), with every product on
 // tcgen05 MMAs whose accumulators sit in tensor memory:
-//   [X | Y] = S0 [W ; Q]^T   (128 x 128: X = S0 W^T, Y = S0 Q^T; one N = 128 MMA
-//                             per K step)
-//   D = Us^T K  (128 x 128)   Z = U^T P^T (128 x 64)
-// The A operands (the bf16 state and the U images) are written by the
-// epilogue straight into tensor memory, so shared memory carries only the
-// chunk tiles (B operands) and the MMAs read nothing from it twice.  The fp32
-// state lives in the epilogue threads' registers (thread = state row, 32 key
-// columns each); every step they add D to it and store its bf16 copy as the
-// next step's A operand, so the state itself never leaves fp32.
+//   [X | Y] = -S0 [W ; Q]^T  (128 x 128, B negated in the instruction
+//                             descriptor; one N = 128 MMA per K step)
+//   X      += U~^T           (four N = 16 MMAs against a 16x16 identity), so X
+//                             is U itself and Y = -S0 Q^T
+//   D = U^T K~  (128 x 128, K~ = diag(e^{G_last - G}) K, an image from prep)
+//   Z = U^T P^T (128 x 64)
+// The A operands of the chain (the bf16 state and U) are written by the
+// epilogue straight into tensor memory; U~^T arrives in shared memory with the
+// chunk's other tiles and enters the accumulator through the identity, so the
+// epilogue neither loads nor subtracts it.  The fp32 state lives in the
+// epilogue threads' registers (thread = state row, 32 key columns each);
+// every step they add D to it and store its bf16 copy as the next step's A
+// operand, so the state itself never leaves fp32.
 //
 // Warp roles: warps 0..15 are the epilogue (TMEM lane quarter = warp % 4,
 // column group = warp / 4); warp 16 allocates TMEM and its lane 0 issues
 // every MMA; lane 0 of warp 17 issues the chunk loads into a three-stage
 // ring as stages are released.  Per step the chain is
-//   [X|Y] -> U, Us -> D -> S update + state image -> next [X|Y],
+//   [X|Y], X += U~ -> U -> D -> S update + state image -> next [X|Y],
 // with Z and the output store off the chain.  The epilogue reads X and Y
-// together, so each accumulator needs only one buffer.  U~^T, an
-// epilogue-only operand, is read from global memory into registers one chunk
-// ahead.
+// together, so each accumulator needs only one buffer.
 //
 // MODE 1 (state recompute for the backward) has no output: it fetches
-// neither Q nor P, runs X = S0 W^T alone in place of [X|Y], skips Z, and
-// stores each chunk's entering state (bf16, Swz<128> image) and U (Swz<128>,
-// token rows) for the backward kernels.
+// neither Q nor P, runs X alone in place of [X|Y], skips Z, and stores each
+// chunk's entering state (bf16, Swz<128> image) and U (Swz<128>, token rows)
+// for the backward kernels.
 //
-// Channel gate: Q and K arrive as prepared images (scale Q .* e^G and
-// K .* e^{G_last - G}), G holds e^{G_last,c}, Us = U, and the decay of the
-// state is per key column.
+// Channel gate: Q arrives as the prepared image scale Q .* e^G, K~ is
+// K .* e^{G_last - G} per key channel, G holds e^{G_last,c}, and the decay of
+// the state is per key column.
 #include "async.cuh"
 #include "common.cuh"
 #include "internal.h"
 #include "mma.cuh"
 #include "tc5.cuh"
 #include "tc_common.cuh"
+
+#include <type_traits>
 
 namespace gdn {
 namespace {
@@ -48,33 +52,54 @@ constexpr int W5_EPI_WARPS = 16;
 constexpr int W5_THREADS = 32 * (W5_EPI_WARPS + 2);
 constexpr int W5_CTRL = W5_EPI_WARPS;      // MMA warp
 constexpr int W5_PROD = W5_EPI_WARPS + 1;  // load warp
-constexpr int W5_STAGES = 3;
-// tensor-memory columns: accumulators [X|Y], D, Z; A operands S (bf16 pairs,
-// 64 columns), U and Us (32 columns each)
-constexpr int TXY = 0, TD = 128, TZ = 256, TAS = 320, TAU = 384, TAUS = 416, TCOLS = 512;
-constexpr uint32_t ID_XY = tc5::idesc_bf16(128, 128, false, false);
-constexpr uint32_t ID_X = tc5::idesc_bf16(128, 64, false, false);
+constexpr uint32_t NEG_B = 1u << 14;       // instruction descriptor: negate B
+constexpr uint32_t ID_XY = tc5::idesc_bf16(128, 128, false, false) | NEG_B;
+constexpr uint32_t ID_X = tc5::idesc_bf16(128, 64, false, false) | NEG_B;
+constexpr uint32_t ID_UI = tc5::idesc_bf16(128, 16, false, false);
 constexpr uint32_t ID_D = tc5::idesc_bf16(128, 128, false, true);
 constexpr uint32_t ID_Z = tc5::idesc_bf16(128, 64, false, false);
 
+// MODE 0: forward (O, hT).  MODE 1: state recompute for the backward (chunk
+// states S0 and U stored).  MODE 2: a segment's affine map (final state only).
+// Forward stage: [W p0 | Q p0 | W p1 | Q p1] (K-major B of [X|Y], 128 rows per
+// 64-key panel, 8 KB each), K~, U~^T, P.
 struct alignas(1024) W5Stage {
-    // K-major B of [X|Y], 128 rows (64 W tokens, then 64 Q tokens) per
-    // 64-key panel: [W p0 | Q p0 | W p1 | Q p1], 8 KB each
     __nv_bfloat16 WQ[2 * C * DK];
-    __nv_bfloat16 K[C * DK];  // Tma128: MN-major B of D
-    __nv_bfloat16 P[C * C];   // Swz<64>: K-major B of Z
-    float G[DK];              // G (scalar gate, C used) or e^{G_last,c}
+    __nv_bfloat16 K[C * DK];   // Tma128 image of K .* e^{G_last - G}: MN-major B of D
+    __nv_bfloat16 Ut[DV * C];  // Swz<64> U~^T (value rows x tokens): K-major A of X += U~^T
+    __nv_bfloat16 P[C * C];    // Swz<64>: K-major B of Z
+};
+// Stage without outputs: W (Tma128, K-major B of X), K~, U~^T.
+struct alignas(1024) W5LeanStage {
+    __nv_bfloat16 W[C * DK];
+    __nv_bfloat16 K[C * DK];
+    __nv_bfloat16 Ut[DV * C];
 };
 
+template <int MODE>
+struct W5Cfg {
+    static constexpr bool FULL = MODE == 0;
+    static constexpr int STAGES = FULL ? 3 : 2;
+    // tensor-memory columns.  Forward: [X|Y] 0..127, D, Z, then the A operands
+    // S (bf16 pairs) and U.  Lean: X and D share columns 0..127 (D is issued
+    // only after the epilogue has read X), so two CTAs fit an SM.
+    static constexpr int TXY = 0, TD = FULL ? 128 : 0, TZ = 256, TAS = FULL ? 320 : 128,
+                         TAU = FULL ? 384 : 192, TCOLS = FULL ? 512 : 256;
+};
+
+template <int MODE>
 struct W5Smem {
-    W5Stage st[W5_STAGES];
-    uint64_t full[W5_STAGES], empty[W5_STAGES];
+    using Stage = typename std::conditional<W5Cfg<MODE>::FULL, W5Stage, W5LeanStage>::type;
+    Stage st[W5Cfg<MODE>::STAGES];
+    __nv_bfloat16 I16[16 * 64];  // 16x16 identity, Swz<64> rows: B of X += U~^T
+    float G[W5Cfg<MODE>::STAGES][DK];  // G (scalar gate, C used) or e^{G_last,c}
+    uint64_t full[W5Cfg<MODE>::STAGES], empty[W5Cfg<MODE>::STAGES];
     uint64_t s_ready, u_ready, x_done, d_done, o_done, fin;
     uint32_t tmem;
 };
 
 struct W5Ptrs {
-    CUtensorMap qmap, kmap;
+    CUtensorMap qmap;
     const float* h0;
     const __nv_bfloat16 *W, *Ut, *P, *Qg, *Kt;
     const float* G;
@@ -85,19 +110,32 @@ struct W5Ptrs {
     int B, T, H, NT;
     float scale;
     SeqMap seq;
+    // Segments: each chain of chunks is cut into nseg runs of seglen chunks
+    // (nseg = 1: one run).  E[(bh*nseg + j)] holds the fp32 state entering
+    // run j (j >= 1); MODE 2 writes E[..+1] from run 0 and the maps M, N of
+    // runs 1 .. nseg-2 (state after the run from I without U~, from 0 with U~).
+    int nseg, seglen;
+    float *E, *Mmap, *Nmap;
+    // Bounded waits: limit of every wait that does not guard a copy or an MMA
+    // in flight at teardown (those use the default), and a test hook that
+    // stops the loads before step stall_at (-1: never) so that the waits on
+    // that stage, which nothing will complete, run out.
+    unsigned long long wait_ns;
+    int stall_at;
 };
 
 template <bool KDA, int MODE>
-__device__ void w5_issue(W5Stage& st, uint64_t* bar, const W5Ptrs& p, const Chain& ch, int h, int n) {
+__device__ void w5_issue(typename W5Smem<MODE>::Stage& st, float* G, uint64_t* bar, const W5Ptrs& p,
+                         const Chain& ch, int h, int n, bool use_u) {
     const size_t cid = (size_t)ch.img * p.NT + ch.n0 + n;  // step n of the chain
     constexpr int GW = KDA ? DK : C;
     constexpr int PANEL = C * 64;  // elements of one 64x64 panel
-    mbar_arrive_expect(bar, (MODE == 0 ? 3 * C * DK + C * C : 2 * C * DK) * 2 + GW * 4);
     const __nv_bfloat16* W = p.W + cid * C * DK;
-    bulk_g2s(st.WQ, W, PANEL * 2, bar);
-    bulk_g2s(st.WQ + 2 * PANEL, W + PANEL, PANEL * 2, bar);
     const int tok = ch.tok0 + n * C;
-    if (MODE == 0) {
+    if constexpr (MODE == 0) {
+        mbar_arrive_expect(bar, (3 * C * DK + DV * C + C * C) * 2 + GW * 4);  // W, Q, K~, U~^T, P
+        bulk_g2s(st.WQ, W, PANEL * 2, bar);
+        bulk_g2s(st.WQ + 2 * PANEL, W + PANEL, PANEL * 2, bar);
         if (KDA) {
             const __nv_bfloat16* Qg = p.Qg + cid * C * DK;
             bulk_g2s(st.WQ + PANEL, Qg, PANEL * 2, bar);
@@ -107,15 +145,20 @@ __device__ void w5_issue(W5Stage& st, uint64_t* bar, const W5Ptrs& p, const Chai
             tma_load_3d(st.WQ + 3 * PANEL, &p.qmap, 64, h, tok, bar);
         }
         bulk_g2s(st.P, p.P + cid * C * C, C * C * 2, bar);
+        bulk_g2s(st.Ut, p.Ut + cid * C * DV, DV * C * 2, bar);
+    } else {
+        mbar_arrive_expect(bar, (2 * C * DK + (use_u ? DV * C : 0)) * 2 + GW * 4);  // W, K~, U~^T
+        bulk_g2s(st.W, W, C * DK * 2, bar);
+        if (use_u) bulk_g2s(st.Ut, p.Ut + cid * C * DV, DV * C * 2, bar);
     }
-    if (KDA) bulk_g2s(st.K, p.Kt + cid * C * DK, C * DK * 2, bar);
-    else tma_load_tile(st.K, &p.kmap, h, tok, bar);
-    bulk_g2s(st.G, p.G + cid * GW, GW * 4, bar);
+    bulk_g2s(st.K, p.Kt + cid * C * DK, C * DK * 2, bar);
+    bulk_g2s(G, p.G + cid * GW, GW * 4, bar);
 }
 
 // Warp-uniform bounded wait: every lane agrees on the outcome.
-GDN_DEV bool wait_all(uint64_t* bar, uint32_t parity, unsigned int* status) {
-    return __all_sync(0xffffffffu, mbar_wait(bar, parity, status));
+GDN_DEV bool wait_all(uint64_t* bar, uint32_t parity, unsigned int* status,
+                      unsigned long long limit_ns) {
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, status, limit_ns));
 }
 
 // One arrival per warp, after all of its lanes' prior writes.
@@ -124,18 +167,63 @@ GDN_DEV void warp_arrive(uint64_t* bar) {
     if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
 }
 
+// What one CTA walks: chain steps n_begin .. n_end-1 of state row bh, from
+// `start` (kStartH0: h0 or zero; kStartE: the run's entry state; kStartI: the
+// identity; kStartZero), with or without U~, ending in `out` (hT, E, M or N).
+enum { kStartH0, kStartE, kStartI, kStartZero };
+struct W5Job {
+    int bh, n_begin, n_end, start;
+    bool use_u;
+    float* out;
+};
+
+template <int MODE>
+GDN_DEV W5Job w5_job(const W5Ptrs& p, int nsteps_of_chain_unused) {
+    W5Job jb;
+    (void)nsteps_of_chain_unused;
+    if constexpr (MODE == 2) {
+        const int per = 2 * p.nseg - 3;  // run 0 from h0, then (M, N) of runs 1 .. nseg-2
+        const int b = blockIdx.x / per, job = blockIdx.x % per;
+        jb.bh = b;
+        const int j = job == 0 ? 0 : 1 + (job - 1) / 2;
+        jb.n_begin = j * p.seglen;
+        jb.n_end = jb.n_begin + p.seglen;
+        const size_t slot = ((size_t)b * p.nseg + j) * DV * DK;
+        if (job == 0) {
+            jb.start = kStartH0; jb.use_u = true; jb.out = p.E + slot + (size_t)DV * DK;
+        } else if ((job - 1) % 2 == 0) {
+            jb.start = kStartI; jb.use_u = false; jb.out = p.Mmap + slot;
+        } else {
+            jb.start = kStartZero; jb.use_u = true; jb.out = p.Nmap + slot;
+        }
+    } else {
+        const int b = blockIdx.x / p.nseg, j = blockIdx.x % p.nseg;
+        jb.bh = b;
+        jb.n_begin = j * p.seglen;
+        jb.n_end = (j + 1) * p.seglen;  // clipped to the chain below
+        jb.start = j == 0 ? kStartH0 : kStartE;
+        jb.use_u = true;
+        jb.out = (MODE == 0 && j == p.nseg - 1 && p.hT) ? p.hT + (size_t)b * DV * DK : nullptr;
+    }
+    return jb;
+}
 
 template <bool KDA, int MODE>
 __global__ void __launch_bounds__(W5_THREADS) tc5_walk_kernel(const __grid_constant__ W5Ptrs p) {
+    using Cfg = W5Cfg<MODE>;
+    using Smem = W5Smem<MODE>;
+    constexpr int NST = Cfg::STAGES;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
-    W5Smem& s = *reinterpret_cast<W5Smem*>(align1k(smem_raw));
+    Smem& s = *reinterpret_cast<Smem*>(align1k(smem_raw));
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int bh = blockIdx.x, h = bh % p.H;  // bh: state row (sequence * H + head)
+    W5Job jb = w5_job<MODE>(p, 0);
+    const int bh = jb.bh, h = bh % p.H;  // bh: state row (sequence * H + head)
     const Chain ch = chain_of(p.seq, p.T, p.H, p.NT, bh / p.H, h);
-    const int nsteps = ch.n1 - ch.n0;
+    const int n_begin = min(jb.n_begin, ch.n1 - ch.n0), n_end = min(jb.n_end, ch.n1 - ch.n0);
+    const int nsteps = n_end - n_begin;  // steps of this CTA (chain steps n_begin ..)
 
     if (tid == 0) {
-        for (int i = 0; i < W5_STAGES; ++i) {
+        for (int i = 0; i < NST; ++i) {
             mbar_init(&s.full[i], 1);
             mbar_init(&s.empty[i], 1 + W5_EPI_WARPS);
         }
@@ -147,7 +235,13 @@ __global__ void __launch_bounds__(W5_THREADS) tc5_walk_kernel(const __grid_const
         mbar_init(&s.fin, 1);
         fence_mbar_init();
     }
-    if (warp == W5_CTRL) tc5::alloc(&s.tmem, TCOLS);
+    // the 16x16 identity (rows of 64 elements, 128-byte swizzle)
+    for (int e = tid; e < 16 * 64; e += W5_THREADS) {
+        const int r = e >> 6, c = e & 63;
+        s.I16[swz<64>(r, c)] = __float2bfloat16_rn(r == c ? 1.f : 0.f);
+    }
+    fence_async_smem();
+    if (warp == W5_CTRL) tc5::alloc(&s.tmem, Cfg::TCOLS);
     tc5::fence_before();
     __syncthreads();
     tc5::fence_after();
@@ -157,41 +251,61 @@ __global__ void __launch_bounds__(W5_THREADS) tc5_walk_kernel(const __grid_const
         if (lane == 0) {
             int issued = 0;
             for (int n = 0; n < nsteps; ++n) {
-                const int sn = n % W5_STAGES;
-                if (n >= W5_STAGES && !mbar_wait(&s.empty[sn], ((n / W5_STAGES) - 1) & 1, p.status)) break;
-                w5_issue<KDA, MODE>(s.st[sn], &s.full[sn], p, ch, h, n);
+                const int sn = n % NST;
+                if (n == p.stall_at) break;  // test hook: leave this stage unloaded
+                if (n >= NST && !mbar_wait(&s.empty[sn], ((n / NST) - 1) & 1, p.status, p.wait_ns)) break;
+                w5_issue<KDA, MODE>(s.st[sn], s.G[sn], &s.full[sn], p, ch, h, n_begin + n, jb.use_u);
                 issued = n + 1;
             }
             // Leave no load in flight (returns at once for stages already consumed).
-            for (int n = max(0, issued - W5_STAGES); n < issued; ++n)
-                mbar_wait(&s.full[n % W5_STAGES], (n / W5_STAGES) & 1, p.status);
+            for (int n = max(0, issued - NST); n < issued; ++n)
+                mbar_wait(&s.full[n % NST], (n / NST) & 1, p.status);
         }
         __syncwarp();
     } else if (warp == W5_CTRL) {
         if (lane == 0) {
-            const uint32_t aUs = tm + (KDA ? TAU : TAUS);
+            const uint32_t sI = smem_u32(s.I16);
             for (int n = 0; n < nsteps; ++n) {
-                const int sn = n % W5_STAGES;
-                W5Stage& st = s.st[sn];
-                if (!mbar_wait(&s.full[sn], (n / W5_STAGES) & 1, p.status)) break;
-                if (!mbar_wait(&s.s_ready, n & 1, p.status)) break;
+                const int sn = n % NST;
+                auto& st = s.st[sn];
+                if (!mbar_wait(&s.full[sn], (n / NST) & 1, p.status, p.wait_ns)) break;
+                if (!mbar_wait(&s.s_ready, n & 1, p.status, p.wait_ns)) break;
                 tc5::fence_after();
-                const uint32_t sWQ = smem_u32(st.WQ), sK = smem_u32(st.K), sP = smem_u32(st.P);
+                const uint32_t sK = smem_u32(st.K), sU = smem_u32(st.Ut);
+                // [X|Y] = -S0 [W;Q]^T (X alone without outputs), then X += U~^T:
+                // X is U itself
+                if constexpr (MODE == 0) {
+                    const uint32_t sWQ = smem_u32(st.WQ);
 #pragma unroll
-                for (int kk = 0; kk < DK / 16; ++kk)
-                    tc5::mma_ts(tm + TXY, tm + TAS + 8 * kk, tc5::kmajor<2 * C>(sWQ, kk),
-                                MODE == 0 ? ID_XY : ID_X, kk > 0);
+                    for (int kk = 0; kk < DK / 16; ++kk)
+                        tc5::mma_ts(tm + Cfg::TXY, tm + Cfg::TAS + 8 * kk, tc5::kmajor<2 * C>(sWQ, kk),
+                                    ID_XY, kk > 0);
+                } else {
+                    const uint32_t sW = smem_u32(st.W);
+#pragma unroll
+                    for (int kk = 0; kk < DK / 16; ++kk)
+                        tc5::mma_ts(tm + Cfg::TXY, tm + Cfg::TAS + 8 * kk, tc5::kmajor<C>(sW, kk), ID_X,
+                                    kk > 0);
+                }
+                if (jb.use_u) {
+#pragma unroll
+                    for (int kk = 0; kk < C / 16; ++kk)
+                        tc5::mma(tm + Cfg::TXY + 16 * kk, tc5::kmajor<DV>(sU, kk), tc5::kmajor<16>(sI, 0),
+                                 ID_UI, true);
+                }
                 tc5::commit(&s.x_done);
-                if (!mbar_wait(&s.u_ready, n & 1, p.status)) break;
+                if (!mbar_wait(&s.u_ready, n & 1, p.status, p.wait_ns)) break;
                 tc5::fence_after();
 #pragma unroll
                 for (int kk = 0; kk < C / 16; ++kk)
-                    tc5::mma_ts(tm + TD, aUs + 8 * kk, tc5::mnmajor(sK, kk, C * 128), ID_D, kk > 0);
+                    tc5::mma_ts(tm + Cfg::TD, tm + Cfg::TAU + 8 * kk, tc5::mnmajor(sK, kk, C * 128), ID_D,
+                                kk > 0);
                 tc5::commit(&s.d_done);
-                if (MODE == 0) {
+                if constexpr (MODE == 0) {
+                    const uint32_t sP = smem_u32(st.P);
 #pragma unroll
                     for (int kk = 0; kk < C / 16; ++kk)
-                        tc5::mma_ts(tm + TZ, tm + TAU + 8 * kk, tc5::kmajor<C>(sP, kk), ID_Z, kk > 0);
+                        tc5::mma_ts(tm + Cfg::TZ, tm + Cfg::TAU + 8 * kk, tc5::kmajor<C>(sP, kk), ID_Z, kk > 0);
                     tc5::commit(&s.o_done);
                 }
                 tc5::commit(&s.empty[sn]);
@@ -209,86 +323,67 @@ __global__ void __launch_bounds__(W5_THREADS) tc5_walk_kernel(const __grid_const
         const int t0 = 16 * cg;  // first token of this thread's U / O columns
         float S[32];
         {
-            const float* h0 = p.h0 ? p.h0 + ((size_t)bh * DV + a) * DK + 32 * cg : nullptr;
+            const float* src = nullptr;
+            if (jb.start == kStartH0 && p.h0) src = p.h0 + (size_t)bh * DV * DK;
+            if (jb.start == kStartE) src = p.E + ((size_t)bh * p.nseg + jb.n_begin / p.seglen) * DV * DK;
+            if (src) src += (size_t)a * DK + 32 * cg;
 #pragma unroll
             for (int j = 0; j < 32; j += 4) {
-                const float4 v = h0 ? *reinterpret_cast<const float4*>(h0 + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+                const float4 v = src ? *reinterpret_cast<const float4*>(src + j) : make_float4(0.f, 0.f, 0.f, 0.f);
                 S[j] = v.x; S[j + 1] = v.y; S[j + 2] = v.z; S[j + 3] = v.w;
+            }
+            if (jb.start == kStartI) {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) S[j] = (32 * cg + j == a) ? 1.f : 0.f;
             }
         }
         auto store_state = [&]() {  // bf16 pairs of this thread's 32 key columns
             uint32_t r[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) r[j] = pack_bf16(S[2 * j], S[2 * j + 1]);
-            tc5::st16(trow + TAS + 16 * cg, r);
+            tc5::st16(trow + Cfg::TAS + 16 * cg, r);
             tc5::wait_st();
         };
-        // MODE 1: bf16 state entering chunk n, Swz<128> image (64 contiguous bytes)
+        // MODE 1: bf16 state entering chain step n, Swz<128> image (64 contiguous bytes)
         auto store_s0 = [&](int n) {
             __nv_bfloat16* dst = p.S0out + ((size_t)ch.img * p.NT + ch.n0 + n) * DV * DK;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const int c = 32 * cg + 8 * j;
                 *reinterpret_cast<uint4*>(dst + swz<DK>(a, c)) =
-                    make_uint4(pack_bf16(S[c - 32 * cg], S[c - 32 * cg + 1]), pack_bf16(S[c - 32 * cg + 2], S[c - 32 * cg + 3]),
-                               pack_bf16(S[c - 32 * cg + 4], S[c - 32 * cg + 5]), pack_bf16(S[c - 32 * cg + 6], S[c - 32 * cg + 7]));
+                    make_uint4(pack_bf16(S[8 * j], S[8 * j + 1]), pack_bf16(S[8 * j + 2], S[8 * j + 3]),
+                               pack_bf16(S[8 * j + 4], S[8 * j + 5]), pack_bf16(S[8 * j + 6], S[8 * j + 7]));
             }
         };
         store_state();
-        if (MODE == 1 && nsteps > 0) store_s0(0);
+        if (MODE == 1 && nsteps > 0) store_s0(n_begin);
         tc5::fence_before();
         warp_arrive(&s.s_ready);
 
-        // U~^T of row a, tokens t0..t0+15: two 16-byte pieces of its Swz<64> row
-        const uint32_t uo0 = swz<C>(a, t0), uo1 = swz<C>(a, t0 + 8);
-        const __nv_bfloat16* Ut = p.Ut + ((size_t)ch.img * p.NT + ch.n0) * C * DV;
-        uint4 ut0 = make_uint4(0, 0, 0, 0), ut1 = ut0;
-        if (nsteps > 0) {
-            ut0 = *reinterpret_cast<const uint4*>(Ut + uo0);
-            ut1 = *reinterpret_cast<const uint4*>(Ut + uo1);
-        }
-
         for (int n = 0; n < nsteps; ++n) {
-            const int sn = n % W5_STAGES;
-            const W5Stage& st = s.st[sn];
-            const int L = min(C, ch.end - (ch.tok0 + n * C));
-            if (!wait_all(&s.full[sn], (n / W5_STAGES) & 1, p.status)) break;
-            // per-token factors, lane j (mod 16) <-> token t0 + j
-            float dec = 1.f, sce = 1.f, gam = 1.f;
-            if (!KDA) {
-                const float gi = st.G[t0 + (lane & 15)], gl = st.G[C - 1];
-                dec = __expf(gl - gi);
-                sce = p.scale * __expf(gi);
-                gam = __expf(gl);
-            }
-            // ---- U = U~ - X; Y kept for the output ------------------------------
-            if (!wait_all(&s.x_done, n & 1, p.status)) break;
+            const int sn = n % NST;
+            const float* G = s.G[sn];
+            const int cn = n_begin + n;  // chain step
+            const int L = min(C, ch.end - (ch.tok0 + cn * C));
+            if (!wait_all(&s.full[sn], (n / NST) & 1, p.status, p.wait_ns)) break;
+            // ---- U = X (= U~ - S0 W^T); -Y kept for the output -------------
+            if (!wait_all(&s.x_done, n & 1, p.status, p.wait_ns)) break;
             tc5::fence_after();
             float y[16];
             {
                 float x[16];
-                tc5::ld16(x, trow + TXY + t0);
-                if (MODE == 0) tc5::ld16(y, trow + TXY + C + t0);
+                tc5::ld16(x, trow + Cfg::TXY + t0);
+                if (MODE == 0) tc5::ld16(y, trow + Cfg::TXY + C + t0);
                 tc5::wait_ld();
-                const __nv_bfloat16* ua = reinterpret_cast<const __nv_bfloat16*>(&ut0);
-                const __nv_bfloat16* ub = reinterpret_cast<const __nv_bfloat16*>(&ut1);
-                uint32_t ru[8], rs[8];
+                uint32_t ru[8];
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const float u0 = __bfloat162float(j < 4 ? ua[2 * j] : ub[2 * j - 8]) - x[2 * j];
-                    const float u1 = __bfloat162float(j < 4 ? ua[2 * j + 1] : ub[2 * j - 7]) - x[2 * j + 1];
-                    ru[j] = pack_bf16(u0, u1);
-                    if (!KDA)
-                        rs[j] = pack_bf16(u0 * __shfl_sync(0xffffffffu, dec, 2 * j),
-                                          u1 * __shfl_sync(0xffffffffu, dec, 2 * j + 1));
-                }
-                tc5::st8(trow + TAU + 8 * cg, ru);
-                if (!KDA) tc5::st8(trow + TAUS + 8 * cg, rs);
+                for (int j = 0; j < 8; ++j) ru[j] = pack_bf16(x[2 * j], x[2 * j + 1]);
+                tc5::st8(trow + Cfg::TAU + 8 * cg, ru);
                 tc5::wait_st();
                 tc5::fence_before();
                 warp_arrive(&s.u_ready);
                 if (MODE == 1) {  // U image, token rows (64 contiguous bytes per warp store)
-                    __nv_bfloat16* dst = p.Uout + ((size_t)ch.img * p.NT + ch.n0 + n) * C * DV;
+                    __nv_bfloat16* dst = p.Uout + ((size_t)ch.img * p.NT + ch.n0 + cn) * C * DV;
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
                         const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(&ru[j]);
@@ -297,99 +392,161 @@ __global__ void __launch_bounds__(W5_THREADS) tc5_walk_kernel(const __grid_const
                     }
                 }
             }
-            if (n + 1 < nsteps) {  // next chunk's U~^T, consumed one step later
-                const __nv_bfloat16* Un = Ut + (size_t)(n + 1) * C * DV;
-                ut0 = *reinterpret_cast<const uint4*>(Un + uo0);
-                ut1 = *reinterpret_cast<const uint4*>(Un + uo1);
-            }
             // ---- S1 = gamma S0 + D, and the bf16 state image -------------------
-            if (!wait_all(&s.d_done, n & 1, p.status)) break;
+            if (!wait_all(&s.d_done, n & 1, p.status, p.wait_ns)) break;
             tc5::fence_after();
             {
                 float d[32];
-                tc5::ld32(d, trow + TD + 32 * cg);
+                tc5::ld32(d, trow + Cfg::TD + 32 * cg);
                 tc5::wait_ld();
+                const float gam = KDA ? 1.f : __expf(G[C - 1]);
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const float gj = KDA ? st.G[32 * cg + j] : gam;
-                    S[j] = fmaf(gj, S[j], d[j]);
-                }
+                for (int j = 0; j < 32; ++j) S[j] = fmaf(KDA ? G[32 * cg + j] : gam, S[j], d[j]);
             }
             store_state();
             tc5::fence_before();
             warp_arrive(&s.s_ready);
-            if (MODE == 1) {
+            if (MODE != 0) {
                 warp_arrive(&s.empty[sn]);
-                if (n + 1 < nsteps) store_s0(n + 1);
+                if (MODE == 1 && n + 1 < nsteps) store_s0(cn + 1);
                 continue;
             }
-            // ---- O^T = scale e^{G_i} Y + Z, tokens t0 .. t0+15 of row a ---------
-            if (!wait_all(&s.o_done, n & 1, p.status)) break;
+            // ---- O^T = scale e^{G_i} S0 Q^T + U^T P^T, tokens t0 .. t0+15 of row a
+            const float sce = KDA ? 1.f : p.scale * __expf(G[t0 + (lane & 15)]);
+            if (!wait_all(&s.o_done, n & 1, p.status, p.wait_ns)) break;
             tc5::fence_after();
             {
                 float z[16];
-                tc5::ld16(z, trow + TZ + t0);
+                tc5::ld16(z, trow + Cfg::TZ + t0);
                 tc5::wait_ld();
-                __nv_bfloat16* o = p.o + (((size_t)ch.tok0 + n * C + t0) * p.H + h) * DV + a;
+                __nv_bfloat16* o = p.o + (((size_t)ch.tok0 + cn * C + t0) * p.H + h) * DV + a;
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
                     const float f = KDA ? 1.f : __shfl_sync(0xffffffffu, sce, j);
-                    if (t0 + j < L) o[(size_t)j * p.H * DV] = __float2bfloat16_rn(fmaf(f, y[j], z[j]));
+                    if (t0 + j < L) o[(size_t)j * p.H * DV] = __float2bfloat16_rn(fmaf(-f, y[j], z[j]));
                 }
             }
             tc5::fence_before();
             warp_arrive(&s.empty[sn]);
         }
-        if (MODE == 0 && p.hT) {
-            float* hT = p.hT + ((size_t)bh * DV + a) * DK + 32 * cg;
+        if (jb.out) {
+            float* out = jb.out + (size_t)a * DK + 32 * cg;
 #pragma unroll
             for (int j = 0; j < 32; j += 4)
-                *reinterpret_cast<float4*>(hT + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+                *reinterpret_cast<float4*>(out + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
         }
     }
     tc5::fence_before();
     __syncthreads();
     if (warp == W5_CTRL) {
         tc5::fence_after();
-        tc5::dealloc(tm, TCOLS);
+        tc5::dealloc(tm, Cfg::TCOLS);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Scan over the runs of each chain: E_{j+1} = E_j M_j + N_j for j = 1 ..
+// nseg-2, in fp32 (E_1 comes from run 0).  One CTA per (state row block of
+// 8 rows, chain); M_j is staged through shared memory a 64-row half at a time.
+// ---------------------------------------------------------------------------
+constexpr int SC_THREADS = 256, SC_ROWS = 8;
+__global__ void __launch_bounds__(SC_THREADS) tc5_seg_scan_kernel(float* E, const float* Mmap,
+                                                                  const float* Nmap, int nseg) {
+    __shared__ __align__(16) float Ms[64][DK];
+    __shared__ __align__(16) float Er[SC_ROWS][DK];
+    const int tid = threadIdx.x;
+    const int b = blockIdx.y, r0 = blockIdx.x * SC_ROWS;
+    const int r = tid >> 5, c0 = (tid & 31) * 4;  // row r0 + r, columns c0 .. c0+3
+    for (int j = 1; j + 1 < nseg; ++j) {
+        const size_t slot = ((size_t)b * nseg + j) * DV * DK;
+        for (int e = tid; e < SC_ROWS * DK / 4; e += SC_THREADS)
+            reinterpret_cast<float4*>(&Er[0][0])[e] =
+                reinterpret_cast<const float4*>(E + slot + (size_t)r0 * DK)[e];
+        float4 acc = reinterpret_cast<const float4*>(Nmap + slot + (size_t)(r0 + r) * DK)[c0 / 4];
+        for (int half = 0; half < 2; ++half) {
+            __syncthreads();
+            for (int e = tid; e < 64 * DK / 4; e += SC_THREADS)
+                reinterpret_cast<float4*>(&Ms[0][0])[e] =
+                    reinterpret_cast<const float4*>(Mmap + slot + (size_t)64 * half * DK)[e];
+            __syncthreads();
+#pragma unroll 8
+            for (int k = 0; k < 64; ++k) {
+                const float e = Er[r][64 * half + k];
+                const float4 m = *reinterpret_cast<const float4*>(&Ms[k][c0]);
+                acc.x = fmaf(e, m.x, acc.x); acc.y = fmaf(e, m.y, acc.y);
+                acc.z = fmaf(e, m.z, acc.z); acc.w = fmaf(e, m.w, acc.w);
+            }
+        }
+        reinterpret_cast<float4*>(E + slot + (size_t)DV * DK + (size_t)(r0 + r) * DK)[c0 / 4] = acc;
+        __syncthreads();
     }
 }
 
 template <bool KDA, int MODE>
-void launch_w5(const W5Ptrs& p, cudaStream_t st) {
-    const int smem = sizeof(W5Smem) + 1024;
+void launch_w5(const W5Ptrs& p, int grid, cudaStream_t st) {
+    const int smem = sizeof(W5Smem<MODE>) + 1024;
     cudaFuncSetAttribute(tc5_walk_kernel<KDA, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    GDN_LAUNCH(MODE == 0 ? "tc5_walk_fwd" : "tc5_walk_states", st,
-               (tc5_walk_kernel<KDA, MODE><<<p.B * p.H, W5_THREADS, smem, st>>>(p)));
+    GDN_LAUNCH(MODE == 0 ? "tc5_walk_fwd" : MODE == 1 ? "tc5_walk_states" : "tc5_seg_map", st,
+               (tc5_walk_kernel<KDA, MODE><<<grid, W5_THREADS, smem, st>>>(p)));
+}
+
+W5Ptrs w5_ptrs(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& c, const float* h0) {
+    W5Ptrs w{};
+    w.qmap = c.qmap;
+    w.h0 = h0; w.W = c.W; w.Ut = c.Ut; w.P = c.P; w.G = c.G; w.Qg = c.Qg; w.Kt = c.Kt;
+    w.status = c.status;
+    w.wait_ns = c.wait_ns; w.stall_at = c.stall_at;
+    w.B = chain_batches(d.B, c.seq); w.T = d.T; w.H = d.H; w.NT = L.NT; w.scale = d.scale;
+    w.seq = c.seq;
+    w.nseg = 1; w.seglen = L.NT;
+    return w;
+}
+
+// Runs the segment maps and the scan, so that E holds every run's entry state.
+template <bool KDA>
+void run_segments(W5Ptrs& w, const TcLayout& L, void* ws, cudaStream_t st) {
+    w.E = (float*)((char*)ws + L.segE);
+    w.Mmap = (float*)((char*)ws + L.segM);
+    w.Nmap = (float*)((char*)ws + L.segN);
+    launch_w5<KDA, 2>(w, w.B * w.H * (2 * w.nseg - 3), st);
+    if (w.nseg > 2)
+        GDN_LAUNCH("tc5_seg_scan", st,
+                   (tc5_seg_scan_kernel<<<dim3(DV / SC_ROWS, w.B * w.H), SC_THREADS, 0, st>>>(
+                       w.E, w.Mmap, w.Nmap, w.nseg)));
 }
 
 }  // namespace
 
 namespace tc {
 void launch_walk5_fwd(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& c, const float* h0,
-                      void* o, float* hT, cudaStream_t st) {
-    W5Ptrs w{};
-    w.qmap = c.qmap; w.kmap = c.kmap;
-    w.h0 = h0; w.W = c.W; w.Ut = c.Ut; w.P = c.P; w.G = c.G; w.Qg = c.Qg; w.Kt = c.Kt;
-    w.o = (__nv_bfloat16*)o; w.hT = hT; w.status = c.status;
-    w.B = chain_batches(d.B, c.seq); w.T = d.T; w.H = d.H; w.NT = L.NT; w.scale = d.scale;
-    w.seq = c.seq;
-    if (d.gate == GDN_GATE_CHANNEL) launch_w5<true, 0>(w, st);
-    else launch_w5<false, 0>(w, st);
+                      void* o, float* hT, void* ws, cudaStream_t st) {
+    W5Ptrs w = w5_ptrs(d, L, c, h0);
+    w.o = (__nv_bfloat16*)o; w.hT = hT;
+    const bool kda = d.gate == GDN_GATE_CHANNEL;
+    w.nseg = L.nseg;
+    w.seglen = L.seglen;
+    if (w.nseg > 1) {
+        if (kda) run_segments<true>(w, L, ws, st);
+        else run_segments<false>(w, L, ws, st);
+    }
+    if (kda) launch_w5<true, 0>(w, w.B * w.H * w.nseg, st);
+    else launch_w5<false, 0>(w, w.B * w.H * w.nseg, st);
 }
 
 void launch_walk5_states(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& c, const float* h0,
                          void* ws, cudaStream_t st) {
-    W5Ptrs w{};
-    w.qmap = c.qmap; w.kmap = c.kmap;
-    w.h0 = h0; w.W = c.W; w.Ut = c.Ut; w.P = c.P; w.G = c.G; w.Qg = c.Qg; w.Kt = c.Kt;
+    W5Ptrs w = w5_ptrs(d, L, c, h0);
     w.S0out = (__nv_bfloat16*)((char*)ws + L.S0);
     w.Uout = (__nv_bfloat16*)((char*)ws + L.U);
-    w.status = c.status;
-    w.B = chain_batches(d.B, c.seq); w.T = d.T; w.H = d.H; w.NT = L.NT; w.scale = d.scale;
-    w.seq = c.seq;
-    if (d.gate == GDN_GATE_CHANNEL) launch_w5<true, 1>(w, st);
-    else launch_w5<false, 1>(w, st);
+    const bool kda = d.gate == GDN_GATE_CHANNEL;
+    w.nseg = L.nseg;
+    w.seglen = L.seglen;
+    if (w.nseg > 1) {
+        if (kda) run_segments<true>(w, L, ws, st);
+        else run_segments<false>(w, L, ws, st);
+    }
+    if (kda) launch_w5<true, 1>(w, w.B * w.H * w.nseg, st);
+    else launch_w5<false, 1>(w, w.B * w.H * w.nseg, st);
 }
 }  // namespace tc
 }  // namespace gdn

@@ -4,10 +4,10 @@
 // Reverse mode through the chunk chain of the forward (tc5_walk.cu): with dS
 // the gradient of the state leaving chunk n and dO the output gradient of
 // its tokens,
-//   dU^T = dO^T P + (dS K^T) .* e^{G_last - G_i}          (value rows x tokens)
+//   dU^T = dO^T P + dS K~^T,  K~ = diag(e^{G_last - G}) K  (value rows x tokens)
 //   dS0  = e^{G_last} dS + dO^T (scale e^G .* Q) - dU^T W  (the state entering n)
 // One CTA walks one head's 128 value rows of dS backwards through the chunks:
-//   F = dO^T P  (128 x 64)     E = dS K^T   (128 x 64)        [A: dO tile, dS]
+//   F = dO^T P  (128 x 64)     E = dS K~^T  (128 x 64)        [A: dO tile, dS]
 //   T = dO^T Q^ - dU^T W (128 x 128, one accumulator; the second product
 //       enters with its A operand negated)                    [A: dO tile, dU]
 // dS stays fp32 in the epilogue threads' registers; its bf16 copy and dU are
@@ -22,9 +22,10 @@
 // three-stage ring.  Chain per step: E -> dU -> T -> dS update -> next E;
 // F and the first half of T depend only on the chunk's tiles.
 //
-// Channel gate: Q and K arrive as prepared images (scale Q .* e^G and
-// K .* e^{G_last - G}), G holds e^{G_last,c}, no per-token factors apply, and
-// the decay of dS is per key column.
+// K~ is the prepared image K .* e^{G_last - G} (per token for the scalar
+// gate, per key channel for the channel gate).  Channel gate: Q arrives as
+// the prepared image scale Q .* e^G, G holds e^{G_last,c}, no per-token
+// factors apply, and the decay of dS is per key column.
 #include "async.cuh"
 #include "common.cuh"
 #include "internal.h"
@@ -50,7 +51,7 @@ constexpr uint32_t ID_Z = tc5::idesc_bf16(128, 128, false, true) | (1u << 13);  
 
 struct alignas(1024) RbStage {
     __nv_bfloat16 Q[C * DK];   // Tma128 [token][key]; scaled in place (B of T, MN-major)
-    __nv_bfloat16 K[C * DK];   // Tma128 [token][key]: K-major B of E
+    __nv_bfloat16 K[C * DK];   // Tma128 image of K .* e^{G_last - G}: K-major B of E
     __nv_bfloat16 W[C * DK];   // Tma128 [token][key]: MN-major B of T
     __nv_bfloat16 dO[C * DV];  // Tma128 [token][value]: MN-major A of F and T
     __nv_bfloat16 P[C * C];    // Swz<64> [j][i]: MN-major B of F
@@ -83,13 +84,9 @@ __device__ void rb_issue(RbStage& st, uint64_t* bar, const RbPtrs& p, const Chai
     constexpr int GW = KDA ? DK : C;
     mbar_arrive_expect(bar, (4 * C * DK + C * C) * 2 + GW * 4);
     const int tok = ch.tok0 + j * C;
-    if (KDA) {
-        bulk_g2s(st.Q, p.Qg + cid * C * DK, C * DK * 2, bar);
-        bulk_g2s(st.K, p.Kt + cid * C * DK, C * DK * 2, bar);
-    } else {
-        tma_load_tile(st.Q, &p.qmap, h, tok, bar);
-        tma_load_tile(st.K, &p.kmap, h, tok, bar);
-    }
+    if (KDA) bulk_g2s(st.Q, p.Qg + cid * C * DK, C * DK * 2, bar);
+    else tma_load_tile(st.Q, &p.qmap, h, tok, bar);
+    bulk_g2s(st.K, p.Kt + cid * C * DK, C * DK * 2, bar);
     tma_load_tile(st.dO, &p.dOmap, h, tok, bar);
     bulk_g2s(st.W, p.W + cid * C * DK, C * DK * 2, bar);
     bulk_g2s(st.P, p.P + cid * C * C, C * C * 2, bar);
@@ -242,13 +239,9 @@ __global__ void __launch_bounds__(RB_THREADS) tc5_walk_bwd_kernel(const __grid_c
             }
             tc5::fence_proxy_async();
             rb_warp_arrive(&s.q_ready);
-            // ---- dU = F + E .* e^{G_last - G_i}, zero past the sequence end ----
-            float et = 1.f, gam = 1.f;
-            if (!KDA) {
-                const float gl = st.G[C - 1];
-                et = __expf(gl - st.G[t0 + (lane & 15)]);
-                gam = __expf(gl);
-            }
+            // ---- dU = F + E, zero past the sequence end (E = dS K~^T carries
+            // the factors e^{G_last - G_i}) ---------------------------------------
+            const float gam = KDA ? 1.f : __expf(st.G[C - 1]);
             if (!rb_wait_all(&s.e_done, k & 1, p.status)) break;
             tc5::fence_after();
             {
@@ -259,10 +252,8 @@ __global__ void __launch_bounds__(RB_THREADS) tc5_walk_bwd_kernel(const __grid_c
                 uint32_t ru[8];
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
-                    const float e0 = KDA ? 1.f : __shfl_sync(0xffffffffu, et, 2 * j);
-                    const float e1 = KDA ? 1.f : __shfl_sync(0xffffffffu, et, 2 * j + 1);
-                    const float u0 = t0 + 2 * j < L ? fmaf(e[2 * j], e0, f[2 * j]) : 0.f;
-                    const float u1 = t0 + 2 * j + 1 < L ? fmaf(e[2 * j + 1], e1, f[2 * j + 1]) : 0.f;
+                    const float u0 = t0 + 2 * j < L ? e[2 * j] + f[2 * j] : 0.f;
+                    const float u1 = t0 + 2 * j + 1 < L ? e[2 * j + 1] + f[2 * j + 1] : 0.f;
                     ru[j] = pack_bf16(u0, u1);
                 }
                 tc5::st8(trow + TADU + 8 * cg, ru);

@@ -30,8 +30,9 @@
 namespace gdn {
 namespace tc {
 void launch_prep_kda(const ChunkPtrs& p, size_t nchunks, cudaStream_t st);
+void launch_prep5(const ChunkPtrs& p, size_t nchunks, cudaStream_t st);
 void launch_walk5_fwd(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& c, const float* h0,
-                      void* o, float* hT, cudaStream_t st);
+                      void* o, float* hT, void* ws, cudaStream_t st);
 void launch_walk5_states(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& c, const float* h0,
                          void* ws, cudaStream_t st);
 }
@@ -538,10 +539,8 @@ bool make_chunk_ptrs(ChunkPtrs& p, const gdn_dims& d, const TcLayout& L, const v
     p.Ut = (__nv_bfloat16*)(base + L.Ut);
     p.P = (__nv_bfloat16*)(base + L.P);
     p.G = (float*)(base + L.G);
-    if (d.gate == GDN_GATE_CHANNEL) {
-        p.Qg = (__nv_bfloat16*)(base + L.Qg);
-        p.Kt = (__nv_bfloat16*)(base + L.Kt);
-    }
+    p.Kt = (__nv_bfloat16*)(base + L.Kt);
+    if (d.gate == GDN_GATE_CHANNEL) p.Qg = (__nv_bfloat16*)(base + L.Qg);
     p.status = (unsigned int*)ws;
     return true;
 }
@@ -583,16 +582,16 @@ namespace tc {
 // The tcgen05 walks carry a whole head per CTA; with few heads the 16-row
 // walks, which spread each head over eight CTAs, fill more SMs.
 bool whole_head_walk(const gdn_dims& d, const SeqMap& seq) {
-    int dev = 0, sms = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    return (long long)chain_batches(d.B, seq) * d.H * 4 >= sms;
+    return (long long)chain_batches(d.B, seq) * d.H * 4 >= sm_count();
 }
 
-void launch_prep(const ChunkPtrs& p, size_t nchunks, cudaStream_t st) {
-    const int smem = sizeof(PrepSmem) + 1024;
-    cudaFuncSetAttribute(tc_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    GDN_LAUNCH("tc_prep", st, tc_prep_kernel<<<(unsigned)nchunks, 128, smem, st>>>(p));
+// The forward chain (and the backward's state recompute) also takes the
+// tcgen05 walk when its chains are cut into runs.
+bool whole_head_fwd(const gdn_dims& d, const TcLayout& L, const SeqMap& seq) {
+    return whole_head_walk(d, seq) || L.nseg > 1;
 }
+
+void launch_prep(const ChunkPtrs& p, size_t nchunks, cudaStream_t st) { launch_prep5(p, nchunks, st); }
 
 bool chunk_ptrs(ChunkPtrs& p, const gdn_dims& d, const TcLayout& L, const void* q,
                 const void* k, const void* v, const float* g, const float* beta, void* ws) {
@@ -601,7 +600,7 @@ bool chunk_ptrs(ChunkPtrs& p, const gdn_dims& d, const TcLayout& L, const void* 
 
 void launch_walk_states(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& cp,
                         const float* h0, void* ws, cudaStream_t st) {
-    if (whole_head_walk(d, cp.seq)) {
+    if (whole_head_fwd(d, L, cp.seq)) {
         launch_walk5_states(d, L, cp, h0, ws, st);
         return;
     }
@@ -664,12 +663,19 @@ void launch_varlen_setup(const int* cu, int nseq, int T, int* cstart, unsigned i
                varlen_setup_kernel<<<1, kSetupThreads, 0, st>>>(cu, nseq, T, cstart, status));
 }
 
+bool tc_fwd_whole_head(const gdn_dims& d) {
+    return tc::whole_head_fwd(d, tc_layout(d, false), SeqMap{});
+}
+
 bool launch_tc_fwd(const gdn_dims& d, const void* q, const void* k, const void* v,
                    const float* g, const float* beta, const float* h0, void* o, float* hT,
-                   void* ws, cudaStream_t st, const int* cu, int nseq) {
+                   void* ws, cudaStream_t st, const int* cu, int nseq,
+                   unsigned long long wait_ns, int stall_at) {
     const TcLayout L = tc_layout(d, false, nseq);
     ChunkPtrs cp;
     if (!make_chunk_ptrs(cp, d, L, q, k, v, g, beta, ws)) return false;
+    cp.wait_ns = wait_ns;
+    cp.stall_at = stall_at;
     if (nseq) {  // chains then run one per (packed sequence, head)
         int* cstart = (int*)((char*)ws + L.cstart);
         launch_varlen_setup(cu, nseq, d.T, cstart, cp.status, st);
@@ -678,8 +684,8 @@ bool launch_tc_fwd(const gdn_dims& d, const void* q, const void* k, const void* 
     const bool kda = d.gate == GDN_GATE_CHANNEL;
     if (kda) launch_prep_kda(cp, L.nchunks, st);
     else launch_prep(cp, L.nchunks, st);
-    if (tc::whole_head_walk(d, cp.seq)) {
-        launch_walk5_fwd(d, L, cp, h0, o, hT, st);
+    if (tc::whole_head_fwd(d, L, cp.seq)) {
+        launch_walk5_fwd(d, L, cp, h0, o, hT, ws, st);
     } else {
         WalkPtrs w = make_walk_ptrs(d, L, cp, h0);
         w.o = (__nv_bfloat16*)o;

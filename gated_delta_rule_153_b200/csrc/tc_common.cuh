@@ -15,9 +15,43 @@ constexpr int C = 64, DK = 128, DV = 128;
 struct TcLayout {
     int NT;
     size_t nchunks;
+    int nseg, seglen;  // runs per chain of the segmented tcgen05 walks (1: unsegmented)
+                       // and chunks per run (the last run may be shorter, never empty)
     // byte offsets into the workspace
-    size_t W, Ut, P, G, Tb, S0, U, dS, dU, Qg, Kt, cstart, end;
+    size_t W, Ut, P, G, Tb, S0, U, dS, dU, Qg, Kt, cstart, segE, segM, segN, end;
 };
+
+// Streaming multiprocessors of the current device (148 when it cannot be read).
+inline int sm_count() {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && sms > 0)
+        return sms;
+    cudaGetLastError();
+    return 148;
+}
+
+// Runs per chain for the forward chain (and the backward's state recompute).
+// With few chains, each chain of NT chunks can be cut into n runs: the maps
+// of the runs (2n - 3 CTAs per chain, one per SM), a scan, then the runs
+// themselves (n CTAs per chain, one per SM).  The estimate counts chain steps
+// on the critical path, (waves of maps + waves of runs) x run length, plus
+// half a step per scan step, against NT steps unsegmented; 3 .. 16 runs of at
+// least 4 chunks are considered.
+inline int seg_runs(int chains, int NT) {
+    const int sms = sm_count();
+    if (chains < 1) chains = 1;
+    int best = 1;
+    double best_cost = (double)NT * ((chains + sms - 1) / sms);
+    for (int n = 3; n <= 16; ++n) {
+        const int len = (NT + n - 1) / n;
+        if (len < 4) break;
+        const long long maps = (long long)chains * (2 * n - 3), runs = (long long)chains * n;
+        const double cost = (double)len * ((maps + sms - 1) / sms + (runs + sms - 1) / sms) + 0.5 * (n - 2);
+        if (cost < best_cost) { best_cost = cost; best = n; }
+    }
+    return best;
+}
 
 // nseq > 0: a packed batch of nseq sequences in one row of d.T tokens; the
 // chunk count is bounded by ceil(T / C) + nseq.
@@ -25,17 +59,24 @@ inline TcLayout tc_layout(const gdn_dims& d, bool bwd, int nseq = 0) {
     TcLayout L{};
     L.NT = (d.T + C - 1) / C + nseq;
     L.nchunks = (size_t)(nseq ? 1 : d.B) * d.H * L.NT;
+    L.nseg = nseq ? 1 : seg_runs(d.B * d.H, L.NT);
+    L.seglen = (L.NT + L.nseg - 1) / L.nseg;
+    L.nseg = (L.NT + L.seglen - 1) / L.seglen;
     size_t o = kStatusBytes;
     auto take = [&](size_t bytes) { size_t r = o; o += (bytes + 255) & ~(size_t)255; return r; };
     if (nseq) L.cstart = take((size_t)(nseq + 1) * 4);
+    if (L.nseg > 1) {  // fp32 states: run entries E, and the maps M, N of each run
+        const size_t seg = (size_t)d.B * d.H * L.nseg * DV * DK * 4;
+        L.segE = take(seg);
+        L.segM = take(seg);
+        L.segN = take(seg);
+    }
     L.W = take(L.nchunks * C * DK * 2);
     L.Ut = take(L.nchunks * C * DV * 2);
     L.P = take(L.nchunks * C * C * 2);
     L.G = take(L.nchunks * (d.gate == GDN_GATE_CHANNEL ? DK : C) * 4);
-    if (d.gate == GDN_GATE_CHANNEL) {
-        L.Qg = take(L.nchunks * C * DK * 2);
-        L.Kt = take(L.nchunks * C * DK * 2);
-    }
+    L.Kt = take(L.nchunks * C * DK * 2);
+    if (d.gate == GDN_GATE_CHANNEL) L.Qg = take(L.nchunks * C * DK * 2);
     if (bwd) {
         L.Tb = take(L.nchunks * C * C * 2);
         L.S0 = take(L.nchunks * DV * DK * 2);
@@ -112,7 +153,8 @@ GDN_DEV Chain chain_of(const SeqMap& m, int T, int H, int NT, int s, int h) {
 //   G   [chunk][64] fp32 within-chunk cumsum of g (padding rows repeat the last);
 //       channel gate: [chunk][128] fp32 e^{G_last,c}, the per-key decay of a chunk
 //   Qg  channel gate only: [chunk] Tma128 image of scale * Q .* e^{G}
-//   Kt  channel gate only: [chunk] Tma128 image of K .* e^{G_last - G}
+//   Kt  [chunk] Tma128 image of K .* e^{G_last - G} (per key channel for the
+//       channel gate, per token for the scalar gate)
 //   Tb  [chunk][64][64]  bf16, Swz<64> tile image of T = (I + A)^{-1}
 //   S0  [chunk][128][128] bf16, Swz<128> image of the chunk-start state
 //   U   [chunk][64][128] bf16 row-major;  dS, dU likewise (backward)
@@ -125,9 +167,13 @@ struct ChunkPtrs {
     __nv_bfloat16 *W, *Ut, *P;
     float* G;
     __nv_bfloat16* Tb;  // optional: bf16 T = (I + A)^{-1} per chunk (backward)
-    __nv_bfloat16 *Qg, *Kt;  // channel gate only
+    __nv_bfloat16 *Qg;  // channel gate only
+    __nv_bfloat16* Kt;
     unsigned int* status;
     SeqMap seq;
+    // bounded waits of the tcgen05 forward walks (see tc5_walk.cu)
+    unsigned long long wait_ns = kWaitNs;
+    int stall_at = -1;
 };
 
 // Stage the W and U~ images from a warp's 16-row block of the W = T diag(.) K

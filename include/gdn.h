@@ -255,6 +255,24 @@ gdn_status gdn_recurrent_step(int N, int H, int dk, int dv, gdn_dtype dtype,
                               const float *beta, float *state, void *o,
                               gdn_stream_t stream);
 
+/* Test hook for the bounded device waits (no counterpart in the paper): runs
+ * gdn_chunk_fwd's tensor-core forward with the loads of chain step
+ * `stall_at` (and after) never issued, so the waits on that step, which no
+ * copy, MMA or thread will ever complete, give up after `wait_ns`
+ * nanoseconds (1 .. 1e9).  Every role then stops; loads and MMAs already
+ * issued are drained (those waits keep the 1 s limit), tensor memory is
+ * freed, and the kernel returns with bit 0 of the workspace's status word
+ * set, so gdn_query_device_status reports GDN_ERR_DEVICE_TIMEOUT.  o and hT
+ * are then not valid.  Only shapes whose forward chain runs on the tcgen05
+ * whole-head walk are accepted (bf16, dk = dv = 128, chunk 64, scalar or
+ * channel gate, B*H*4 >= the SM count; GDN_ERR_UNSUPPORTED otherwise).
+ * Arguments and workspace as gdn_chunk_fwd. */
+gdn_status gdn_test_stalled_fwd(const gdn_dims *dims, const void *q, const void *k,
+                                const void *v, const float *g, const float *beta,
+                                const float *h0, void *o, float *hT, void *ws,
+                                size_t ws_bytes, int stall_at, unsigned long long wait_ns,
+                                gdn_stream_t stream);
+
 /* Synchronises `stream`, then reads and clears the status word kept in the
  * first bytes of a chunkwise workspace.  Each chunkwise call clears that word
  * (a 4-byte memset on its stream) before its kernels run, and a kernel whose

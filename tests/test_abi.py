@@ -222,3 +222,22 @@ def test_header_is_plain_c(tmp_path):
     subprocess.run(["gcc", "-std=c11", "-Wall", "-Werror", "-pedantic", "-c",
                     "-I", os.path.join(ROOT, "include"), str(src), "-o", str(tmp_path / "use.o")],
                    check=True)
+
+
+def test_stalled_fwd_hook_checks():
+    """The wait-timeout test hook rejects bad hook arguments and shapes that
+    do not take the tcgen05 whole-head walk, on the host."""
+    L = gdn.lib()
+    p = ctypes.c_void_p(256)
+    ws = ctypes.c_void_p(1 << 20)
+    big = 1 << 40
+    wide = gdn.gdn_dims(1, 512, 40, 128, 128, 64, gdn.GDN_BF16, gdn.GDN_GATE_SCALAR, 1.0)
+    narrow = gdn.gdn_dims(1, 512, 1, 128, 128, 64, gdn.GDN_BF16, gdn.GDN_GATE_SCALAR, 1.0)
+    f32 = gdn.gdn_dims(1, 512, 40, 128, 128, 64, gdn.GDN_F32, gdn.GDN_GATE_SCALAR, 1.0)
+    call = lambda d, stall, ns: L.gdn_test_stalled_fwd(ctypes.byref(d), p, p, p, p, p, None, p,
+                                                       None, ws, big, stall, ns, None)
+    assert call(wide, -1, 1000) == gdn.GDN_ERR_INVALID_ARG
+    assert call(wide, 2, 0) == gdn.GDN_ERR_INVALID_ARG
+    assert call(wide, 2, 2_000_000_000) == gdn.GDN_ERR_INVALID_ARG
+    assert call(narrow, 2, 1000) == gdn.GDN_ERR_UNSUPPORTED
+    assert call(f32, 2, 1000) == gdn.GDN_ERR_UNSUPPORTED

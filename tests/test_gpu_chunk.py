@@ -236,3 +236,49 @@ def test_kda_slow_gate_whole_head_long_chain(dev):
     inp = make_chunk_inputs(KDA, T=1024, g_shift=-6.0, h0_std=0.1, dhT_std=0.3)
     check_fwd(inp, dev)
     check_bwd(inp, dev)
+
+
+def test_walk_wait_runs_out_and_context_survives(dev):
+    """A bounded device wait that actually runs out: the tcgen05 forward walk
+    is run with the loads of chain step 3 never issued, so the waits on that
+    stage (which no copy, MMA or thread completes) give up after 200 us.  The
+    call returns, the status word reports the timeout once, and a normal call
+    on the same stream afterwards still matches the oracle."""
+    import ctypes
+    import gated_delta_rule_153_b200 as gdn
+    inp = make_chunk_inputs(L350M, B=1, H=40, T=512, h0_std=0.1, seed=31)
+    q, k, v, g, beta, h0 = (inp[n].to(dev) for n in ("q", "k", "v", "g", "beta", "h0"))
+    dims = gdn.make_dims(q, v, g)
+    ws = torch.zeros(gdn.gdn_chunk_fwd_workspace(dims), dtype=torch.uint8, device=dev)
+    o = torch.empty_like(v)
+    hT = torch.empty(1, 40, 128, 128, device=dev)
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    st = gdn.lib().gdn_test_stalled_fwd(ctypes.byref(dims), q.data_ptr(), k.data_ptr(),
+                                        v.data_ptr(), g.data_ptr(), beta.data_ptr(),
+                                        h0.data_ptr(), o.data_ptr(), hT.data_ptr(),
+                                        ws.data_ptr(), ws.numel(), 3, 200_000, stream)
+    assert st == gdn.GDN_OK, gdn.status_string(st)
+    assert gdn.gdn_query_device_status(ws) == gdn.GDN_ERR_DEVICE_TIMEOUT
+    assert gdn.gdn_query_device_status(ws) == gdn.GDN_OK
+    check_fwd(inp, dev)
+
+
+@pytest.mark.parametrize("cfg,over", [
+    # 6 chains of 43 chunks (runs of 4, the last one shorter); ragged tail, slow gate
+    (L350M, dict(B=2, H=3, T=64 * 43 - 17, g_shift=-6.0, h0_std=0.1, dhT_std=0.3)),
+    # no initial state: run 0 starts from zero
+    (L350M, dict(B=1, H=4, T=64 * 40, g_shift=-4.0, dhT_std=0.3)),
+    # one chain cut into the most runs (16), fast and slow gates
+    (LONG, dict(H=1, T=64 * 130, g_shift=-6.0)),
+    (LONG, dict(H=2, T=64 * 96)),
+    # channel gate
+    (KDA, dict(B=1, H=4, T=4096, g_shift=-6.0, h0_std=0.1, dhT_std=0.3)),
+])
+def test_segmented_chains(dev, cfg, over):
+    """Few chains: each chain is cut into runs whose affine maps (walked from
+    the identity and from zero) are scanned into the runs' entry states, then
+    every run is walked from its entry state in parallel.  Slow gates keep the
+    state, and so every map and every scan step, in the outputs."""
+    inp = make_chunk_inputs(cfg, **over)
+    check_fwd(inp, dev)
+    check_bwd(inp, dev)
