@@ -29,8 +29,8 @@
 //
 // MODE 1 (state recompute for the backward) has no output: it fetches
 // neither Q nor P, runs X alone in place of [X|Y], skips Z, and stores each
-// chunk's entering state (bf16, Swz<128> image) and U (Swz<128>, token rows)
-// for the backward kernels.
+// chunk's entering state (bf16, Kp<128> image: two 64-key panels of 128
+// rows) and U (Tma128, token rows) for the backward kernels.
 //
 // Channel gate: Q arrives as the prepared image scale Q .* e^G, K~ is
 // K .* e^{G_last - G} per key channel, G holds e^{G_last,c}, and the decay of
@@ -45,6 +45,10 @@
 #include <type_traits>
 
 namespace gdn {
+namespace tc {
+void launch_seg_scan(float* E, const float* Mmap, const float* Nmap, int nseg, int chains,
+                     cudaStream_t st);
+}
 namespace {
 using namespace tc;
 
@@ -344,13 +348,13 @@ __global__ void __launch_bounds__(W5_THREADS) tc5_walk_kernel(const __grid_const
             tc5::st16(trow + Cfg::TAS + 16 * cg, r);
             tc5::wait_st();
         };
-        // MODE 1: bf16 state entering chain step n, Swz<128> image (64 contiguous bytes)
+        // MODE 1: bf16 state entering chain step n, Kp<128> image (64 contiguous bytes)
         auto store_s0 = [&](int n) {
             __nv_bfloat16* dst = p.S0out + ((size_t)ch.img * p.NT + ch.n0 + n) * DV * DK;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const int c = 32 * cg + 8 * j;
-                *reinterpret_cast<uint4*>(dst + swz<DK>(a, c)) =
+                *reinterpret_cast<uint4*>(dst + Kp<DV>::off(a, c)) =
                     make_uint4(pack_bf16(S[8 * j], S[8 * j + 1]), pack_bf16(S[8 * j + 2], S[8 * j + 3]),
                                pack_bf16(S[8 * j + 4], S[8 * j + 5]), pack_bf16(S[8 * j + 6], S[8 * j + 7]));
             }
@@ -382,13 +386,13 @@ __global__ void __launch_bounds__(W5_THREADS) tc5_walk_kernel(const __grid_const
                 tc5::wait_st();
                 tc5::fence_before();
                 warp_arrive(&s.u_ready);
-                if (MODE == 1) {  // U image, token rows (64 contiguous bytes per warp store)
+                if (MODE == 1) {  // U image, Tma128 token rows (64 contiguous bytes per warp store)
                     __nv_bfloat16* dst = p.Uout + ((size_t)ch.img * p.NT + ch.n0 + cn) * C * DV;
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
                         const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(&ru[j]);
-                        dst[swz<DV>(t0 + 2 * j, a)] = v.x;
-                        dst[swz<DV>(t0 + 2 * j + 1, a)] = v.y;
+                        dst[Tma128::off(t0 + 2 * j, a)] = v.x;
+                        dst[Tma128::off(t0 + 2 * j + 1, a)] = v.y;
                     }
                 }
             }
@@ -509,15 +513,19 @@ void run_segments(W5Ptrs& w, const TcLayout& L, void* ws, cudaStream_t st) {
     w.Mmap = (float*)((char*)ws + L.segM);
     w.Nmap = (float*)((char*)ws + L.segN);
     launch_w5<KDA, 2>(w, w.B * w.H * (2 * w.nseg - 3), st);
-    if (w.nseg > 2)
-        GDN_LAUNCH("tc5_seg_scan", st,
-                   (tc5_seg_scan_kernel<<<dim3(DV / SC_ROWS, w.B * w.H), SC_THREADS, 0, st>>>(
-                       w.E, w.Mmap, w.Nmap, w.nseg)));
+    if (w.nseg > 2) tc::launch_seg_scan(w.E, w.Mmap, w.Nmap, w.nseg, w.B * w.H, st);
 }
 
 }  // namespace
 
 namespace tc {
+void launch_seg_scan(float* E, const float* Mmap, const float* Nmap, int nseg, int chains,
+                     cudaStream_t st) {
+    GDN_LAUNCH("tc5_seg_scan", st,
+               (tc5_seg_scan_kernel<<<dim3(DV / SC_ROWS, chains), SC_THREADS, 0, st>>>(
+                   E, Mmap, Nmap, nseg)));
+}
+
 void launch_walk5_fwd(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& c, const float* h0,
                       void* o, float* hT, void* ws, cudaStream_t st) {
     W5Ptrs w = w5_ptrs(d, L, c, h0);

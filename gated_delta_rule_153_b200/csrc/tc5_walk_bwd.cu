@@ -14,7 +14,7 @@
 // written straight into tensor memory as A operands.  The dO tile is read
 // as an MN-major A operand from shared memory; Q is scaled in place to
 // Q^ = scale e^{G_i} Q (rows past the sequence end zeroed) before T.
-// Each chunk's dS (bf16, Swz<128>) and dU (Swz<128>, token rows) are stored
+// Each chunk's dS (bf16, Kp<128>) and dU (Tma128, token rows) are stored
 // for the local-gradient kernel; dh0 is the dS left after chunk 0.
 //
 // Warp roles as in tc5_walk.cu: 16 epilogue warps (TMEM lane quarter =
@@ -76,20 +76,30 @@ struct RbPtrs {
     int B, T, H, NT;
     float scale;
     SeqMap seq;
+    // Runs (see tc5_walk.cu), counted from the end of the chain: run i holds
+    // chunks of forward run nseg-1-i.  E[(bh*nseg + i)] is the fp32 gradient
+    // entering run i (i >= 1); MODE 2 writes E[..+1] from run 0 (entered with
+    // dhT) and the reverse maps dS -> dS R + Q' of runs 1 .. nseg-2 (R: from I
+    // without the dO terms; Q': from 0 with them).
+    int nseg, seglen;
+    float *E, *Mmap, *Nmap;
 };
 
 template <bool KDA>
-__device__ void rb_issue(RbStage& st, uint64_t* bar, const RbPtrs& p, const Chain& ch, int h, int j) {
+__device__ void rb_issue(RbStage& st, uint64_t* bar, const RbPtrs& p, const Chain& ch, int h, int j,
+                         bool use_do) {
     const size_t cid = (size_t)ch.img * p.NT + ch.n0 + j;  // chunk j of the chain
     constexpr int GW = KDA ? DK : C;
-    mbar_arrive_expect(bar, (4 * C * DK + C * C) * 2 + GW * 4);
+    mbar_arrive_expect(bar, ((use_do ? 4 : 2) * C * DK + (use_do ? C * C : 0)) * 2 + GW * 4);
     const int tok = ch.tok0 + j * C;
-    if (KDA) bulk_g2s(st.Q, p.Qg + cid * C * DK, C * DK * 2, bar);
-    else tma_load_tile(st.Q, &p.qmap, h, tok, bar);
+    if (use_do) {  // the dO terms: Q (scaled in place), dO, P
+        if (KDA) bulk_g2s(st.Q, p.Qg + cid * C * DK, C * DK * 2, bar);
+        else tma_load_tile(st.Q, &p.qmap, h, tok, bar);
+        tma_load_tile(st.dO, &p.dOmap, h, tok, bar);
+        bulk_g2s(st.P, p.P + cid * C * C, C * C * 2, bar);
+    }
     bulk_g2s(st.K, p.Kt + cid * C * DK, C * DK * 2, bar);
-    tma_load_tile(st.dO, &p.dOmap, h, tok, bar);
     bulk_g2s(st.W, p.W + cid * C * DK, C * DK * 2, bar);
-    bulk_g2s(st.P, p.P + cid * C * C, C * C * 2, bar);
     bulk_g2s(st.G, p.G + cid * GW, GW * 4, bar);
 }
 
@@ -102,14 +112,42 @@ GDN_DEV void rb_warp_arrive(uint64_t* bar) {
     if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
 }
 
-template <bool KDA>
+enum { kRbStartDhT, kRbStartE, kRbStartI, kRbStartZero };
+
+// MODE 0: the reverse walk proper (dS, dU images per chunk; dh0).  MODE 2:
+// a run's reverse map (final gradient only).
+template <bool KDA, int MODE>
 __global__ void __launch_bounds__(RB_THREADS) tc5_walk_bwd_kernel(const __grid_constant__ RbPtrs p) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     RbSmem& s = *reinterpret_cast<RbSmem*>(align1k(smem_raw));
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int bh = blockIdx.x, h = bh % p.H;  // bh: state row (sequence * H + head)
+    // ---- which run of which chain, from where, to where ----------------------
+    int bh, run, start;
+    bool use_do;
+    float* out;
+    if (MODE == 2) {
+        const int per = 2 * p.nseg - 3, job = blockIdx.x % per;
+        bh = blockIdx.x / per;
+        run = job == 0 ? 0 : 1 + (job - 1) / 2;
+        const size_t slot = ((size_t)bh * p.nseg + run) * DV * DK;
+        if (job == 0) { start = kRbStartDhT; use_do = true; out = p.E + slot + (size_t)DV * DK; }
+        else if ((job - 1) % 2 == 0) { start = kRbStartI; use_do = false; out = p.Mmap + slot; }
+        else { start = kRbStartZero; use_do = true; out = p.Nmap + slot; }
+    } else {
+        bh = blockIdx.x / p.nseg;
+        run = blockIdx.x % p.nseg;
+        start = run == 0 ? kRbStartDhT : kRbStartE;
+        use_do = true;
+        // the run holding chunk 0 of the chain ends in dh0
+        out = (run == p.nseg - 1 && p.dh0) ? p.dh0 + (size_t)bh * DV * DK : nullptr;
+    }
+    const int h = bh % p.H;  // bh: state row (sequence * H + head)
     const Chain ch = chain_of(p.seq, p.T, p.H, p.NT, bh / p.H, h);
-    const int nsteps = ch.n1 - ch.n0;
+    const int nch = ch.n1 - ch.n0;
+    // forward run nseg-1-run covers chain chunks [c_lo, c_hi); walked downwards
+    const int fr = p.nseg - 1 - run;
+    const int c_lo = min(fr * p.seglen, nch), c_hi = min((fr + 1) * p.seglen, nch);
+    const int nsteps = c_hi - c_lo;
 
     if (tid == 0) {
         for (int i = 0; i < RB_STAGES; ++i) {
@@ -133,10 +171,10 @@ __global__ void __launch_bounds__(RB_THREADS) tc5_walk_bwd_kernel(const __grid_c
     if (warp == RB_PROD) {
         if (lane == 0) {
             int issued = 0;
-            for (int k = 0; k < nsteps; ++k) {  // step k carries chunk nsteps-1-k of the chain
+            for (int k = 0; k < nsteps; ++k) {  // step k carries chunk c_hi-1-k of the chain
                 const int sk = k % RB_STAGES;
                 if (k >= RB_STAGES && !mbar_wait(&s.empty[sk], ((k / RB_STAGES) - 1) & 1, p.status)) break;
-                rb_issue<KDA>(s.st[sk], &s.full[sk], p, ch, h, nsteps - 1 - k);
+                rb_issue<KDA>(s.st[sk], &s.full[sk], p, ch, h, c_hi - 1 - k, use_do);
                 issued = k + 1;
             }
             for (int k = max(0, issued - RB_STAGES); k < issued; ++k)
@@ -151,27 +189,32 @@ __global__ void __launch_bounds__(RB_THREADS) tc5_walk_bwd_kernel(const __grid_c
                 if (!mbar_wait(&s.full[sk], (k / RB_STAGES) & 1, p.status)) break;
                 const uint32_t sQ = smem_u32(st.Q), sK = smem_u32(st.K), sW = smem_u32(st.W),
                                sdO = smem_u32(st.dO), sP = smem_u32(st.P);
+                if (use_do) {
 #pragma unroll
-                for (int kk = 0; kk < C / 16; ++kk)  // F = dO^T P
-                    tc5::mma(tm + TF, tc5::mnmajor(sdO, kk, C * 128), tc5::mnmajor(sP, kk, C * 128), ID_F,
-                             kk > 0);
+                    for (int kk = 0; kk < C / 16; ++kk)  // F = dO^T P
+                        tc5::mma(tm + TF, tc5::mnmajor(sdO, kk, C * 128), tc5::mnmajor(sP, kk, C * 128), ID_F,
+                                 kk > 0);
+                }
                 if (!mbar_wait(&s.ds_ready, k & 1, p.status)) break;
                 tc5::fence_after();
 #pragma unroll
-                for (int kk = 0; kk < DK / 16; ++kk)  // E = dS K^T
+                for (int kk = 0; kk < DK / 16; ++kk)  // E = dS K~^T
                     tc5::mma_ts(tm + TE, tm + TADS + 8 * kk, tc5::kmajor<C>(sK, kk), ID_E, kk > 0);
                 tc5::commit(&s.e_done);
-                if (!mbar_wait(&s.q_ready, k & 1, p.status)) break;
-                tc5::fence_after();
+                if (use_do) {
+                    if (!mbar_wait(&s.q_ready, k & 1, p.status)) break;
+                    tc5::fence_after();
 #pragma unroll
-                for (int kk = 0; kk < C / 16; ++kk)  // T = dO^T Q^
-                    tc5::mma(tm + TT, tc5::mnmajor(sdO, kk, C * 128), tc5::mnmajor(sQ, kk, C * 128), ID_Y,
-                             kk > 0);
+                    for (int kk = 0; kk < C / 16; ++kk)  // T = dO^T Q^
+                        tc5::mma(tm + TT, tc5::mnmajor(sdO, kk, C * 128), tc5::mnmajor(sQ, kk, C * 128), ID_Y,
+                                 kk > 0);
+                }
                 if (!mbar_wait(&s.du_ready, k & 1, p.status)) break;
                 tc5::fence_after();
 #pragma unroll
                 for (int kk = 0; kk < C / 16; ++kk)  // T -= dU^T W
-                    tc5::mma_ts(tm + TT, tm + TADU + 8 * kk, tc5::mnmajor(sW, kk, C * 128), ID_Z, true);
+                    tc5::mma_ts(tm + TT, tm + TADU + 8 * kk, tc5::mnmajor(sW, kk, C * 128), ID_Z,
+                                use_do || kk > 0);
                 tc5::commit(&s.t_done);
                 tc5::commit(&s.empty[sk]);
             }
@@ -187,11 +230,18 @@ __global__ void __launch_bounds__(RB_THREADS) tc5_walk_bwd_kernel(const __grid_c
         const int t0 = 16 * cg;
         float dS[32];
         {
-            const float* src = p.dhT ? p.dhT + ((size_t)bh * DV + a) * DK + 32 * cg : nullptr;
+            const float* src = nullptr;
+            if (start == kRbStartDhT && p.dhT) src = p.dhT + (size_t)bh * DV * DK;
+            if (start == kRbStartE) src = p.E + ((size_t)bh * p.nseg + run) * DV * DK;
+            if (src) src += (size_t)a * DK + 32 * cg;
 #pragma unroll
             for (int j = 0; j < 32; j += 4) {
                 const float4 v = src ? *reinterpret_cast<const float4*>(src + j) : make_float4(0.f, 0.f, 0.f, 0.f);
                 dS[j] = v.x; dS[j + 1] = v.y; dS[j + 2] = v.z; dS[j + 3] = v.w;
+            }
+            if (start == kRbStartI) {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) dS[j] = (32 * cg + j == a) ? 1.f : 0.f;
             }
         }
         auto store_ds_tmem = [&]() {
@@ -206,21 +256,21 @@ __global__ void __launch_bounds__(RB_THREADS) tc5_walk_bwd_kernel(const __grid_c
         rb_warp_arrive(&s.ds_ready);
 
         for (int k = 0; k < nsteps; ++k) {
-            const int j = nsteps - 1 - k, sk = k % RB_STAGES;  // chunk j of the chain
+            const int j = c_hi - 1 - k, sk = k % RB_STAGES;  // chunk j of the chain
             RbStage& st = s.st[sk];
             const int L = min(C, ch.end - (ch.tok0 + j * C));
             const size_t cid = (size_t)ch.img * p.NT + ch.n0 + j;
             if (!rb_wait_all(&s.full[sk], (k / RB_STAGES) & 1, p.status)) break;
-            {   // dS leaving chunk n: bf16 Swz<128> image, 64 contiguous bytes
+            if (MODE == 0) {   // dS leaving chunk n: bf16 Kp<128> image, 64 contiguous bytes
                 __nv_bfloat16* dst = p.dSout + cid * DV * DK;
 #pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    *reinterpret_cast<uint4*>(dst + swz<DK>(a, 32 * cg + 8 * j)) =
-                        make_uint4(pack_bf16(dS[8 * j], dS[8 * j + 1]), pack_bf16(dS[8 * j + 2], dS[8 * j + 3]),
-                                   pack_bf16(dS[8 * j + 4], dS[8 * j + 5]), pack_bf16(dS[8 * j + 6], dS[8 * j + 7]));
+                for (int jj = 0; jj < 4; ++jj)
+                    *reinterpret_cast<uint4*>(dst + Kp<DV>::off(a, 32 * cg + 8 * jj)) =
+                        make_uint4(pack_bf16(dS[8 * jj], dS[8 * jj + 1]), pack_bf16(dS[8 * jj + 2], dS[8 * jj + 3]),
+                                   pack_bf16(dS[8 * jj + 4], dS[8 * jj + 5]), pack_bf16(dS[8 * jj + 6], dS[8 * jj + 7]));
             }
             // Q^ = scale e^{G_i} Q in place, rows past the sequence end zeroed
-            if (!KDA || L < C) {
+            if (use_do && (!KDA || L < C)) {
 #pragma unroll
                 for (int rep = 0; rep < 2; ++rep) {
                     const int ci = tid + 32 * RB_EPI_WARPS * rep;  // 16-byte piece of the tile
@@ -230,9 +280,9 @@ __global__ void __launch_bounds__(RB_THREADS) tc5_walk_bwd_kernel(const __grid_c
                     uint4 v = *ptr;
                     __nv_bfloat162* e2 = reinterpret_cast<__nv_bfloat162*>(&v);
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const float2 x = __bfloat1622float2(e2[j]);
-                        e2[j] = __floats2bfloat162_rn(x.x * f, x.y * f);
+                    for (int jj = 0; jj < 4; ++jj) {
+                        const float2 x = __bfloat1622float2(e2[jj]);
+                        e2[jj] = __floats2bfloat162_rn(x.x * f, x.y * f);
                     }
                     *ptr = v;
                 }
@@ -247,25 +297,27 @@ __global__ void __launch_bounds__(RB_THREADS) tc5_walk_bwd_kernel(const __grid_c
             {
                 float e[16], f[16];
                 tc5::ld16(e, trow + TE + t0);
-                tc5::ld16(f, trow + TF + t0);
+                if (use_do) tc5::ld16(f, trow + TF + t0);
                 tc5::wait_ld();
                 uint32_t ru[8];
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const float u0 = t0 + 2 * j < L ? e[2 * j] + f[2 * j] : 0.f;
-                    const float u1 = t0 + 2 * j + 1 < L ? e[2 * j + 1] + f[2 * j + 1] : 0.f;
-                    ru[j] = pack_bf16(u0, u1);
+                for (int jj = 0; jj < 8; ++jj) {
+                    const float u0 = t0 + 2 * jj < L ? e[2 * jj] + (use_do ? f[2 * jj] : 0.f) : 0.f;
+                    const float u1 = t0 + 2 * jj + 1 < L ? e[2 * jj + 1] + (use_do ? f[2 * jj + 1] : 0.f) : 0.f;
+                    ru[jj] = pack_bf16(u0, u1);
                 }
                 tc5::st8(trow + TADU + 8 * cg, ru);
                 tc5::wait_st();
                 tc5::fence_before();
                 rb_warp_arrive(&s.du_ready);
-                __nv_bfloat16* dst = p.dUout + cid * C * DV;  // dU image, token rows
+                if (MODE == 0) {
+                    __nv_bfloat16* dst = p.dUout + cid * C * DV;  // dU image, Tma128 token rows
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(&ru[j]);
-                    dst[swz<DV>(t0 + 2 * j, a)] = v.x;
-                    dst[swz<DV>(t0 + 2 * j + 1, a)] = v.y;
+                    for (int jj = 0; jj < 8; ++jj) {
+                        const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(&ru[jj]);
+                        dst[Tma128::off(t0 + 2 * jj, a)] = v.x;
+                        dst[Tma128::off(t0 + 2 * jj + 1, a)] = v.y;
+                    }
                 }
             }
             // ---- dS0 = gamma dS + T ---------------------------------------------
@@ -276,9 +328,9 @@ __global__ void __launch_bounds__(RB_THREADS) tc5_walk_bwd_kernel(const __grid_c
                 tc5::ld32(t, trow + TT + 32 * cg);
                 tc5::wait_ld();
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const float gj = KDA ? st.G[32 * cg + j] : gam;
-                    dS[j] = fmaf(gj, dS[j], t[j]);
+                for (int jj = 0; jj < 32; ++jj) {
+                    const float gj = KDA ? st.G[32 * cg + jj] : gam;
+                    dS[jj] = fmaf(gj, dS[jj], t[jj]);
                 }
             }
             store_ds_tmem();
@@ -286,11 +338,11 @@ __global__ void __launch_bounds__(RB_THREADS) tc5_walk_bwd_kernel(const __grid_c
             rb_warp_arrive(&s.ds_ready);
             rb_warp_arrive(&s.empty[sk]);
         }
-        if (p.dh0) {
-            float* dst = p.dh0 + ((size_t)bh * DV + a) * DK + 32 * cg;
+        if (out) {
+            float* dst = out + (size_t)a * DK + 32 * cg;
 #pragma unroll
-            for (int j = 0; j < 32; j += 4)
-                *reinterpret_cast<float4*>(dst + j) = make_float4(dS[j], dS[j + 1], dS[j + 2], dS[j + 3]);
+            for (int jj = 0; jj < 32; jj += 4)
+                *reinterpret_cast<float4*>(dst + jj) = make_float4(dS[jj], dS[jj + 1], dS[jj + 2], dS[jj + 3]);
         }
     }
     tc5::fence_before();
@@ -301,16 +353,20 @@ __global__ void __launch_bounds__(RB_THREADS) tc5_walk_bwd_kernel(const __grid_c
     }
 }
 
-template <bool KDA>
-void launch_rb(const RbPtrs& p, cudaStream_t st) {
+template <bool KDA, int MODE>
+void launch_rb(const RbPtrs& p, int grid, cudaStream_t st) {
     const int smem = sizeof(RbSmem) + 1024;
-    cudaFuncSetAttribute(tc5_walk_bwd_kernel<KDA>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    GDN_LAUNCH("tc5_walk_bwd", st, (tc5_walk_bwd_kernel<KDA><<<p.B * p.H, RB_THREADS, smem, st>>>(p)));
+    cudaFuncSetAttribute(tc5_walk_bwd_kernel<KDA, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    GDN_LAUNCH(MODE == 0 ? "tc5_walk_bwd" : "tc5_seg_map_bwd", st,
+               (tc5_walk_bwd_kernel<KDA, MODE><<<grid, RB_THREADS, smem, st>>>(p)));
 }
 
 }  // namespace
 
 namespace tc {
+void launch_seg_scan(float* E, const float* Mmap, const float* Nmap, int nseg, int chains,
+                     cudaStream_t st);
+
 bool launch_walk5_bwd(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& c, const void* dO,
                       const float* dhT, float* dh0, void* ws, cudaStream_t st) {
     RbPtrs p{};
@@ -322,8 +378,19 @@ bool launch_walk5_bwd(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& c, 
     p.dh0 = dh0; p.status = c.status;
     p.B = chain_batches(d.B, c.seq); p.T = d.T; p.H = d.H; p.NT = L.NT; p.scale = d.scale;
     p.seq = c.seq;
-    if (d.gate == GDN_GATE_CHANNEL) launch_rb<true>(p, st);
-    else launch_rb<false>(p, st);
+    p.nseg = L.nseg; p.seglen = L.seglen;
+    const bool kda = d.gate == GDN_GATE_CHANNEL;
+    const int chains = p.B * p.H;
+    if (p.nseg > 1) {
+        p.E = (float*)((char*)ws + L.segE);
+        p.Mmap = (float*)((char*)ws + L.segM);
+        p.Nmap = (float*)((char*)ws + L.segN);
+        if (kda) launch_rb<true, 2>(p, chains * (2 * p.nseg - 3), st);
+        else launch_rb<false, 2>(p, chains * (2 * p.nseg - 3), st);
+        if (p.nseg > 2) launch_seg_scan(p.E, p.Mmap, p.Nmap, p.nseg, chains, st);
+    }
+    if (kda) launch_rb<true, 0>(p, chains * p.nseg, st);
+    else launch_rb<false, 0>(p, chains * p.nseg, st);
     return true;
 }
 }  // namespace tc

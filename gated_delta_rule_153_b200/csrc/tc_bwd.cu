@@ -22,6 +22,7 @@
 #include "common.cuh"
 #include "internal.h"
 #include "mma.cuh"
+#include "tc5.cuh"
 #include "tc_common.cuh"
 
 namespace gdn {
@@ -38,6 +39,8 @@ bool launch_bwd_local_kda(const gdn_dims& d, const TcLayout& L, const ChunkPtrs&
 bool whole_head_walk(const gdn_dims& d, const SeqMap& seq);
 bool launch_walk5_bwd(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& c, const void* dO,
                       const float* dhT, float* dh0, void* ws, cudaStream_t st);
+bool launch_bwd_local5(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& cp, const void* dO,
+                       void* dq, void* dk, void* dv, float* dg, float* dbeta, void* ws, cudaStream_t st);
 }  // namespace tc
 
 namespace {
@@ -165,9 +168,12 @@ __global__ void __launch_bounds__(BW_THREADS) tc_walk_bwd_kernel(const __grid_co
         }
         const size_t cid = (size_t)ch.img * p.NT + ch.n0 + j;
         const int L = min(C, ch.end - (ch.tok0 + j * C));
-        if (tid == 0) {  // dS leaving chunk n (Swz<128> image rows a0..)
-            bulk_s2g(p.dSout + (cid * DV + a0) * DK, s.dS, RT * DK * 2);
-            bulk_commit();
+        // dS leaving chunk n: rows a0.. into the Kp<128> image (a0 is a multiple
+        // of 16, so a 16-byte piece keeps its swizzled position)
+        for (int e = tid; e < RT * 16; e += BW_THREADS) {
+            const int r = e >> 4, pos = e & 15;
+            *reinterpret_cast<uint4*>(p.dSout + cid * DV * DK + (pos >> 3) * (DV * 64) + (a0 + r) * 64 +
+                                      (pos & 7) * 8) = *reinterpret_cast<const uint4*>(s.dS + r * DK + pos * 8);
         }
         // dO^T tiles (rows past the sequence end are zeroed: they are not ours)
         for (int e = tid; e < C * RT; e += BW_THREADS) {
@@ -220,7 +226,6 @@ __global__ void __launch_bounds__(BW_THREADS) tc_walk_bwd_kernel(const __grid_co
                     s.dUst[(i0 + (e & 1)) * RT + 16 * mt + r_lo + 8 * (e >> 1)] = __float2bfloat16_rn(u[e]);
             }
         }
-        if (tid == 0) bulk_wait_read<0>();  // dS image read before it is rewritten
         __syncthreads();
         // dS0 = e^{G_last} dS + dOg^T Q - dU^T W   (columns 16w..16w+15)
         {
@@ -262,11 +267,10 @@ __global__ void __launch_bounds__(BW_THREADS) tc_walk_bwd_kernel(const __grid_co
         constexpr int PIECES = RT / 8;
         for (int e = tid; e < PIECES * C; e += BW_THREADS) {  // dU rows, 16-byte pieces
             const int i = e / PIECES, pc = e % PIECES;
-            *reinterpret_cast<uint4*>(p.dUout + cid * C * DV + swz<DV>(i, a0 + 8 * pc)) =
+            *reinterpret_cast<uint4*>(p.dUout + cid * C * DV + Tma128::off(i, a0 + 8 * pc)) =
                 *reinterpret_cast<const uint4*>(&s.dUst[i * RT + 8 * pc]);
         }
     }
-    if (tid == 0) bulk_wait<0>();
     if (p.dh0) {
         float* dst = p.dh0 + ((size_t)bh * DV + a0) * DK;
 #pragma unroll
@@ -289,9 +293,9 @@ __global__ void __launch_bounds__(BW_THREADS) tc_walk_bwd_kernel(const __grid_co
 constexpr int LOC_WARPS = 16, LOC_THREADS = 32 * LOC_WARPS;
 
 struct LocSmem {
-    // Q, K, V, dO: Tma128 tiles (TMA); U, dU: Swz<128> images (bulk)
+    // Q, K, V, dO: Tma128 tiles (TMA); U, dU: Tma128 images (bulk)
     __nv_bfloat16 Q[C * DK], K[C * DK], V[C * DV], dO[C * DV], U[C * DV], dU[C * DV];
-    __nv_bfloat16 S0[DV * DK];  // rows a (value), cols c (key)
+    __nv_bfloat16 S0[DV * DK];  // Kp<128>: rows a (value), cols c (key)
     __nv_bfloat16 dS[DV * DK];
     __nv_bfloat16 dW[C * DK];
     __nv_bfloat16 Tb[C * C];
@@ -429,7 +433,7 @@ __global__ void __launch_bounds__(LOC_THREADS) tc_bwd_local_kernel(const __grid_
 #pragma unroll
             for (int np = 0; np < 2; ++np) {
                 uint32_t bf[4];
-                ldb_kn<DK>(bf, s.S0, 16 * kk, 32 * cq + 16 * np);
+                ldb_kn<Kp<DV>>(bf, s.S0, 16 * kk, 32 * cq + 16 * np);
                 mma16816(acc[2 * np], a, bf[0], bf[1]);
                 mma16816(acc[2 * np + 1], a, bf[2], bf[3]);
             }
@@ -456,11 +460,11 @@ __global__ void __launch_bounds__(LOC_THREADS) tc_bwd_local_kernel(const __grid_
 #pragma unroll
         for (int kk = 0; kk < DV / 16; ++kk) {
             uint32_t a[4];
-            lda<DV>(a, s.U, m0, 16 * kk);
+            lda<Tma128>(a, s.U, m0, 16 * kk);
 #pragma unroll
             for (int np = 0; np < 2; ++np) {
                 uint32_t bf[4];
-                ldb_kn<DK>(bf, s.dS, 16 * kk, 32 * cq + 16 * np);
+                ldb_kn<Kp<DV>>(bf, s.dS, 16 * kk, 32 * cq + 16 * np);
                 mma16816(acc[2 * np], a, bf[0], bf[1]);
                 mma16816(acc[2 * np + 1], a, bf[2], bf[3]);
             }
@@ -488,11 +492,11 @@ __global__ void __launch_bounds__(LOC_THREADS) tc_bwd_local_kernel(const __grid_
 #pragma unroll
         for (int kk = 0; kk < DV / 16; ++kk) {
             uint32_t a[4];
-            lda<DV>(a, s.dU, m0, 16 * kk);
+            lda<Tma128>(a, s.dU, m0, 16 * kk);
 #pragma unroll
             for (int np = 0; np < 2; ++np) {
                 uint32_t bf[4];
-                ldb_kn<DK>(bf, s.S0, 16 * kk, 32 * cq + 16 * np);
+                ldb_kn<Kp<DV>>(bf, s.S0, 16 * kk, 32 * cq + 16 * np);
                 mma16816(acc[2 * np], a, bf[0], bf[1]);
                 mma16816(acc[2 * np + 1], a, bf[2], bf[3]);
             }
@@ -513,7 +517,7 @@ __global__ void __launch_bounds__(LOC_THREADS) tc_bwd_local_kernel(const __grid_
 #pragma unroll
             for (int np = 0; np < 1; ++np) {
                 uint32_t bu[4], bk[4];
-                ldb_nk<DV>(bu, s.U, 16 * cq + 16 * np, 16 * kk);
+                ldb_nk<Tma128>(bu, s.U, 16 * cq + 16 * np, 16 * kk);
                 ldb_nk<Tma128>(bk, s.K, 16 * cq + 16 * np, 16 * kk);
                 mma16816(dp[2 * np], ad, bu[0], bu[1]);
                 mma16816(dp[2 * np + 1], ad, bu[2], bu[3]);
@@ -588,7 +592,7 @@ __global__ void __launch_bounds__(LOC_THREADS) tc_bwd_local_kernel(const __grid_
         for (int kk = 0; kk < DK / 16; ++kk) {
             uint32_t aw[4], au[4];
             lda<DK>(aw, s.dW, m0, 16 * kk);
-            lda<DV>(au, s.dU, m0, 16 * kk);
+            lda<Tma128>(au, s.dU, m0, 16 * kk);
 #pragma unroll
             for (int np = 0; np < 1; ++np) {
                 uint32_t bk[4], bv[4];
@@ -644,7 +648,7 @@ __global__ void __launch_bounds__(LOC_THREADS) tc_bwd_local_kernel(const __grid_
             for (int np = 0; np < 2; ++np) {
                 uint32_t bw[4], bu[4];
                 ldb_kn<DK>(bw, s.dW, 16 * kk, 32 * cq + 16 * np);
-                ldb_kn<DV>(bu, s.dU, 16 * kk, 32 * cq + 16 * np);
+                ldb_kn<Tma128>(bu, s.dU, 16 * kk, 32 * cq + 16 * np);
                 mma16816(akg[2 * np], a, bw[0], bw[1]);
                 mma16816(akg[2 * np + 1], a, bw[2], bw[3]);
                 mma16816(avb[2 * np], a, bu[0], bu[1]);
@@ -883,13 +887,14 @@ bool launch_tc_bwd(const gdn_dims& d, const void* q, const void* k, const void* 
     BwPtrs bp{};
     bp.dSout = (__nv_bfloat16*)(base + L.dS);
     bp.dUout = (__nv_bfloat16*)(base + L.dU);
-    if (whole_head_walk(d, cp.seq)) {
+    if (whole_head_walk(d, cp.seq) || L.nseg > 1) {
         if (!launch_walk5_bwd(d, L, cp, dO, dhT, dh0, ws, st)) return false;
     } else if (!launch_walk_bwd16(d, cp, dO, dhT, dh0, bp, st)) {
         return false;
     }
     if (kda_gate)
         return launch_bwd_local_kda(d, L, cp, dO, dq, dk, dv, dg, dbeta, ws, st);
+    return launch_bwd_local5(d, L, cp, dO, dq, dk, dv, dg, dbeta, ws, st);
     LocPtrs lp{};
     lp.qmap = cp.qmap; lp.kmap = cp.kmap; lp.vmap = cp.vmap;
     if (!encode_token_map(&lp.dOmap, dO, d.B, d.T, d.H)) return false;

@@ -398,9 +398,15 @@ __global__ void __launch_bounds__(WALK_THREADS) tc_walk_kernel(const __grid_cons
         const int tok = ch.tok0 + k * C;
         const int L = min(C, ch.end - tok);
         const size_t cid = (size_t)ch.img * p.NT + ch.n0 + k;
-        if (MODE == 1 && tid == 0) {  // chunk-start state rows a0.. (Swz<128> image)
-            bulk_s2g(p.S0out + (cid * DV + a0) * DK, s.S0, RT * DK * 2);
-            bulk_commit();
+        if (MODE == 1) {  // chunk-start state rows a0.. into the Kp<128> image
+            // (a0 is a multiple of 16, so a 16-byte piece keeps its swizzled
+            // position: the first half of a Swz<128> row is panel 0, the second panel 1)
+            for (int e = tid; e < RT * 16; e += WALK_THREADS) {
+                const int r = e >> 4, pos = e & 15;
+                *reinterpret_cast<uint4*>(p.S0out + cid * DV * DK + (pos >> 3) * (DV * 64) +
+                                          (a0 + r) * 64 + (pos & 7) * 8) =
+                    *reinterpret_cast<const uint4*>(s.S0 + r * DK + pos * 8);
+            }
         }
         const float Gl = KDA ? 0.f : st.G[C - 1];
         const float et0 = KDA ? 1.f : __expf(Gl - st.G[i0]);
@@ -438,7 +444,6 @@ __global__ void __launch_bounds__(WALK_THREADS) tc_walk_kernel(const __grid_cons
                     s.O[(i0 + (e & 1)) * RT + 16 * mt + r_lo + 8 * (e >> 1)] = __float2bfloat16_rn(u[e]);
             }
         }
-        if (MODE == 1 && tid == 0) bulk_wait_read<0>();  // S0 image read before it is rewritten
         __syncthreads();
 
         // S1 = e^{G_last} S0 + (U^T .* e^{G_last - G}) K, columns 16w..16w+15
@@ -506,12 +511,11 @@ __global__ void __launch_bounds__(WALK_THREADS) tc_walk_kernel(const __grid_cons
             if (MODE == 0) {
                 const size_t row = ((size_t)tok + i) * p.H + h;
                 *reinterpret_cast<uint4*>(p.o + row * DV + a0 + 8 * pc) = v;
-            } else {  // U image, Swz<128>: 16-byte piece at its swizzled position
-                *reinterpret_cast<uint4*>(p.Uout + cid * C * DV + swz<DV>(i, a0 + 8 * pc)) = v;
+            } else {  // U image, Tma128: 16-byte piece at its swizzled position
+                *reinterpret_cast<uint4*>(p.Uout + cid * C * DV + Tma128::off(i, a0 + 8 * pc)) = v;
             }
         }
     }
-    if (MODE == 1 && tid == 0) bulk_wait<0>();
     if (MODE == 0 && p.hT) {
         float* hT = p.hT + ((size_t)bh * DV + a0) * DK;
 #pragma unroll

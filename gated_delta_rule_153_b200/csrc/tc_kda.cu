@@ -28,6 +28,7 @@
 #include "common.cuh"
 #include "internal.h"
 #include "mma.cuh"
+#include "tc5.cuh"
 #include "tc_common.cuh"
 
 namespace gdn {
@@ -506,11 +507,11 @@ __global__ void __launch_bounds__(KL_THREADS) tc_bwd_local_kda_kernel(const __gr
         for (int kk = 0; kk < DV / 16; ++kk) {
             uint32_t ad[4], au[4];
             lda<Tma128>(ad, s.u.p1.dO, m0, 16 * kk);
-            lda<S128>(au, s.dU, m0, 16 * kk);
+            lda<Tma128>(au, s.dU, m0, 16 * kk);
 #pragma unroll
             for (int np = 0; np < 2; ++np) {
                 uint32_t bs[4];
-                ldb_kn<S128>(bs, s.u.p1.S, 16 * kk, 32 * cq + 16 * np);
+                ldb_kn<Kp<DV>>(bs, s.u.p1.S, 16 * kk, 32 * cq + 16 * np);
                 mma16816(aq[2 * np], ad, bs[0], bs[1]);
                 mma16816(aq[2 * np + 1], ad, bs[2], bs[3]);
                 mma16816(aw[2 * np], au, bs[0], bs[1]);
@@ -534,7 +535,7 @@ __global__ void __launch_bounds__(KL_THREADS) tc_bwd_local_kda_kernel(const __gr
         for (int kk = 0; kk < DV / 16; ++kk) {
             uint32_t ad[4], bu[4];
             lda<Tma128>(ad, s.u.p1.dO, m0, 16 * kk);
-            ldb_nk<S128>(bu, s.u.p1.U, 16 * cq, 16 * kk);
+            ldb_nk<Tma128>(bu, s.u.p1.U, 16 * cq, 16 * kk);
             mma16816(dp[0], ad, bu[0], bu[1]);
             mma16816(dp[1], ad, bu[2], bu[3]);
         }
@@ -554,7 +555,7 @@ __global__ void __launch_bounds__(KL_THREADS) tc_bwd_local_kda_kernel(const __gr
     {
         const int c = tid & (DK - 1), a0 = tid >> 7;
 #pragma unroll
-        for (int k = 0; k < 32; ++k) s0r[k] = bf(s.u.p1.S, swz<DK>(a0 + 4 * k, c));
+        for (int k = 0; k < 32; ++k) s0r[k] = bf(s.u.p1.S, Kp<DV>::off(a0 + 4 * k, c));
     }
     __syncthreads();  // everyone done with S0
     if (tid == 0) {
@@ -569,11 +570,11 @@ __global__ void __launch_bounds__(KL_THREADS) tc_bwd_local_kda_kernel(const __gr
 #pragma unroll
         for (int kk = 0; kk < DV / 16; ++kk) {
             uint32_t au[4];
-            lda<S128>(au, s.u.p1.U, m0, 16 * kk);
+            lda<Tma128>(au, s.u.p1.U, m0, 16 * kk);
 #pragma unroll
             for (int np = 0; np < 2; ++np) {
                 uint32_t bs[4];
-                ldb_kn<S128>(bs, s.u.p1.S, 16 * kk, 32 * cq + 16 * np);
+                ldb_kn<Kp<DV>>(bs, s.u.p1.S, 16 * kk, 32 * cq + 16 * np);
                 mma16816(ak[2 * np], au, bs[0], bs[1]);
                 mma16816(ak[2 * np + 1], au, bs[2], bs[3]);
             }
@@ -600,7 +601,7 @@ __global__ void __launch_bounds__(KL_THREADS) tc_bwd_local_kda_kernel(const __gr
         const int c = tid & (DK - 1), a0 = tid >> 7;
         float ss = 0.f;
 #pragma unroll
-        for (int k = 0; k < 32; ++k) ss += s0r[k] * bf(s.u.p1.S, swz<DK>(a0 + 4 * k, c));
+        for (int k = 0; k < 32; ++k) ss += s0r[k] * bf(s.u.p1.S, Kp<DV>::off(a0 + 4 * k, c));
         s.glp[1][a0][c] = ss;
     }
     __syncthreads();  // phase-1 scratch is dead from here on
@@ -654,7 +655,7 @@ __global__ void __launch_bounds__(KL_THREADS) tc_bwd_local_kda_kernel(const __gr
             }
             uint32_t aw[4], au[4], bg[4], bv[4];
             lda<S128>(aw, s.dW, m0, 16 * kk);
-            lda<S128>(au, s.dU, m0, 16 * kk);
+            lda<Tma128>(au, s.dU, m0, 16 * kk);
             ldb_nk<Tma128>(bg, s.u.p2.Kg, 16 * cq, 16 * kk);
             ldb_nk<Tma128>(bv, s.u.p2.V, 16 * cq, 16 * kk);
             mma16816(tw[0], aw, bg[0], bg[1]);
@@ -707,7 +708,7 @@ __global__ void __launch_bounds__(KL_THREADS) tc_bwd_local_kda_kernel(const __gr
             for (int np = 0; np < 2; ++np) {
                 uint32_t bw[4], bu[4];
                 ldb_kn<S128>(bw, s.dW, 16 * kk, 32 * cq + 16 * np);
-                ldb_kn<S128>(bu, s.dU, 16 * kk, 32 * cq + 16 * np);
+                ldb_kn<Tma128>(bu, s.dU, 16 * kk, 32 * cq + 16 * np);
                 mma16816(akg[2 * np], a, bw[0], bw[1]);
                 mma16816(akg[2 * np + 1], a, bw[2], bw[3]);
                 mma16816(avb[2 * np], a, bu[0], bu[1]);

@@ -291,7 +291,8 @@ gdn_status gdn_query_device_status(void *ws, gdn_stream_t stream);
  * library holds until the process exits), so the caller passes only inputs
  * and outputs.  Supported shapes are those of the tensor-core path (bf16,
  * dk = dv = 128, chunk 64, scalar gate; GDN_ERR_UNSUPPORTED otherwise) whose
- * workspace fits 64 MiB, i.e. B*H*ceil(T/64) <= 1628 chunk-heads
+ * workspace, as gdn_chunk_fwd_workspace reports it, fits 64 MiB: about 72 KiB
+ * per chunk-head, plus 192 KiB per run when few chains are cut into runs
  * (GDN_ERR_WORKSPACE otherwise, checked on the host before anything runs).
  * No cudaMalloc, cudaFree or other allocating call is made.  The first call
  * on a device looks up the array's device address (cudaGetSymbolAddress),
