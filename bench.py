@@ -520,19 +520,21 @@ def run_ours(args, rank, world, dev, barrier, max_over_ranks):
                 gpu_launches=nlaunch, clocks=clk.summary(), peaks=pk, cfg=cfg)
 
 
-def cpu_baseline_oracle(sample_B):
+def cpu_baseline_oracle(sample_B, sample_T=None, inp=None):
     """The fp64 oracle (as it stands) on host cores: fwd + bwd over the first
-    `sample_B` sequences of the 350M-scale workload.  Returns tokens/s."""
+    `sample_B` sequences (first `sample_T` tokens of each, default all) of the
+    350M-scale workload.  Returns tokens/s, seconds and the thread count."""
     import oracle
     from gated_delta_rule_153_b200.inputs import L350M, make_chunk_inputs
-    inp = make_chunk_inputs(L350M)
-    sl = {n: (inp[n][:sample_B] if n in ("q", "k", "v", "g", "beta", "dO") else inp[n])
-          for n in inp}
+    inp = inp if inp is not None else make_chunk_inputs(L350M)
+    Ts = sample_T or L350M.T
+    sl = {n: (inp[n][:sample_B, :Ts].contiguous() if n in ("q", "k", "v", "g", "beta", "dO")
+              else inp[n]) for n in inp}
     t0 = time.perf_counter()
     oracle.fwd(sl["q"], sl["k"], sl["v"], sl["g"], sl["beta"], None)
     oracle.bwd(sl["q"], sl["k"], sl["v"], sl["g"], sl["beta"], sl["dO"], None, None)
     dt = time.perf_counter() - t0
-    return sample_B * L350M.T / dt, dt, oracle.threads()
+    return sample_B * Ts / dt, dt, oracle.threads()
 
 
 def main():
@@ -554,17 +556,26 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return
-        from gated_delta_rule_153_b200.inputs import L350M
-        sample_B = L350M.B
+        from gated_delta_rule_153_b200.inputs import L350M, make_chunk_inputs
+        inp = make_chunk_inputs(L350M)
+        sample_B = L350M.B  # all 8 sequences x 8 heads: every core busy
+        # Each step is the first sample_T tokens of every sequence, sized from a
+        # probe step so that warm-up plus timed steps take about two minutes.
+        probe_T = 256
+        v0, dt0, _ = cpu_baseline_oracle(sample_B, probe_T, inp)
+        per_tok = dt0 / (sample_B * probe_T)
+        budget = 120.0 / (args.warmup + args.steps)
+        sample_T = int(max(128, min(L350M.T, budget / (per_tok * sample_B))) // 64 * 64)
         vals = []
         for i in range(args.warmup + args.steps):
-            v, dt, cores = cpu_baseline_oracle(sample_B)
+            v, dt, cores = cpu_baseline_oracle(sample_B, sample_T, inp)
             if i >= args.warmup:
                 vals.append((v, dt))
         tot = sum(dt for _, dt in vals)
-        value = len(vals) * sample_B * L350M.T / tot
-        sample = (f"fwd+bwd of all {sample_B} sequences (T=2048, H=8, d=128) of the 350M-scale "
-                  f"workload per step, fp64 token loop, OpenMP over (sequence, head)")
+        value = len(vals) * sample_B * sample_T / tot
+        sample = (f"fwd+bwd of the first {sample_T} of T=2048 tokens of all {sample_B} sequences "
+                  f"(H=8, d=128) of the 350M-scale workload per step, fp64 token loop, OpenMP "
+                  f"over (sequence, head); tokens/s is linear-time work, so the rate holds for T=2048")
         print(json.dumps({
             "impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": "tokens/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,

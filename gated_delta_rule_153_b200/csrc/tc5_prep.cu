@@ -7,25 +7,26 @@
 // form):
 //   A  = strict_lower(diag(beta) (K K^T .* D)),  D_ij = exp(G_i - G_j)
 //   T  = (I + A)^{-1}                                 (UT transform)
-//   W  = T diag(beta) (diag(e^G) K),   U~ = T diag(beta) V
+//   W  = T (diag(beta e^G) K),   U~ = T (diag(beta) V)
 //   P  = scale lower(Q K^T .* D)
 // The products run as tcgen05 MMAs with fp32 accumulators in tensor memory:
 //   [K K^T ; Q K^T] = [K ; Q] K^T           one M = 128, N = 64 product: rows
 //                                           0..63 give A, rows 64..127 give P
-//   W^T  = (e^G K)^T (T diag(beta))^T       M = 128 (key), N = 64 (token)
-//   U~^T = V^T (T diag(beta))^T             M = 128 (value), N = 64 (token)
+//   W^T  = (beta e^G K)^T T^T               M = 128 (key), N = 64 (token)
+//   U~^T = (beta V)^T T^T                   M = 128 (value), N = 64 (token)
 // with K and Q stacked in one K-major operand (the TMA tiles of both land in
 // the same 128-row panels), and the transposed products reading the K and V
 // tiles as MN-major A operands, so no tile is copied or transposed in shared
-// memory.  The row scale e^{G_j} of W is applied to K in place once Q K^T and
-// K K^T are done, so both transposed products share the B operand T diag(beta).
+// memory.  The row scales beta e^G of W and beta of U~ are applied to the K
+// and V tiles in place once Q K^T and K K^T are done, so both transposed
+// products share the B operand T.
 // The triangular solve keeps the 16x16 diagonal blocks of T exact in fp32
 // registers (forward substitution) and combines the off-diagonal blocks one
 // block diagonal at a time with warp-level MMAs (T_IJ = -T_II sum_K A_IK T_KJ).
 //
 // One CTA of four warps per chunk; thread t owns TMEM lane t in both
 // epilogues (row t of [K K^T ; Q K^T], then key / value row t of W^T / U~^T).
-// Shared memory ~74 KB and 128 TMEM columns, so three CTAs share an SM.
+// Shared memory 74 KB and 128 TMEM columns, so three CTAs share an SM.
 // Outputs (bulk stores into the workspace): the W image (Tma128), the U~^T
 // image (Swz<64>, 128 value rows), P (Swz<64>), G, and optionally T (Swz<64>);
 // the K~ = diag(e^{G_last - G}) K image (Tma128) goes out with plain 16-byte
@@ -57,7 +58,6 @@ struct alignas(1024) P5Smem {
     __nv_bfloat16 V[C * DV];  // Tma128
     __nv_bfloat16 P[C * C];   // Swz<64>
     __nv_bfloat16 T[C * C];   // Swz<64>: T = (I + A)^{-1}
-    __nv_bfloat16 T2[C * C];  // Swz<64>: T diag(beta)
     float G[C];
     float beta[C];
     uint64_t bar_ld, bar_mma;
@@ -169,10 +169,11 @@ __global__ void __launch_bounds__(P5_THREADS, 3) tc5_prep_kernel(const __grid_co
         __syncthreads();
 
         // ---- K~ = diag(e^{G_last - G}) K to the workspace (the walks' B of
-        // the state update), and K <- diag(e^G) K in place (the row scale of W)
+        // the state update); K <- diag(beta e^G) K and V <- diag(beta) V in
+        // place (the row scales of W and U~)
         {
             const int r = tid >> 1, pn = tid & 1;
-            const float e = __expf(s.G[r]), dec = __expf(s.G[C - 1] - s.G[r]);
+            const float e = s.beta[r] * __expf(s.G[r]), dec = __expf(s.G[C - 1] - s.G[r]);
             __nv_bfloat16* row = s.KQ + pn * KQ_PANEL + r * 64;
             // same swizzled position in the Tma128 image (panel pn at pn * 4096)
             __nv_bfloat16* kt = p.Kt + (size_t)cid * C * DK + pn * (C * 64) + r * 64;
@@ -190,6 +191,19 @@ __global__ void __launch_bounds__(P5_THREADS, 3) tc5_prep_kernel(const __grid_co
                 *reinterpret_cast<uint4*>(row + 8 * j) = x;
                 *reinterpret_cast<uint4*>(kt + 8 * j) = y;
             }
+            const float b = s.beta[r];
+            __nv_bfloat16* vrow = s.V + pn * (C * 64) + r * 64;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                uint4 x = *reinterpret_cast<uint4*>(vrow + 8 * j);
+                uint32_t* w = reinterpret_cast<uint32_t*>(&x);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float2 f2 = unpack_bf16(w[i]);
+                    w[i] = pack_bf16(f2.x * b, f2.y * b);
+                }
+                *reinterpret_cast<uint4*>(vrow + 8 * j) = x;
+            }
         }
 
         // ---- UT transform, diagonal block `warp`: forward substitution ------
@@ -206,20 +220,13 @@ __global__ void __launch_bounds__(P5_THREADS, 3) tc5_prep_kernel(const __grid_co
                 t[i] = (i < c) ? 0.f : v;
             }
             if (lane < 16) {
-                const float bc = s.beta[m0 + c];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    s.T[swz<C>(m0 + i, m0 + c)] = __float2bfloat16_rn(t[i]);
-                    s.T2[swz<C>(m0 + i, m0 + c)] = __float2bfloat16_rn(t[i] * bc);
-                }
+                for (int i = 0; i < 16; ++i) s.T[swz<C>(m0 + i, m0 + c)] = __float2bfloat16_rn(t[i]);
             }
             // zero this warp's row block right of the diagonal block
             for (int e = lane; e < 16 * C; e += 32) {
                 const int r = e >> 6, cc = e & 63;
-                if (cc >= m0 + 16) {
-                    s.T[swz<C>(m0 + r, cc)] = __float2bfloat16_rn(0.f);
-                    s.T2[swz<C>(m0 + r, cc)] = __float2bfloat16_rn(0.f);
-                }
+                if (cc >= m0 + 16) s.T[swz<C>(m0 + r, cc)] = __float2bfloat16_rn(0.f);
             }
         }
         __syncthreads();
@@ -255,31 +262,27 @@ __global__ void __launch_bounds__(P5_THREADS, 3) tc5_prep_kernel(const __grid_co
                 mma16816(y[1], a, bx[2], bx[3]);
 #pragma unroll
                 for (int jn = 0; jn < 2; ++jn) {
-                    const int cc = 16 * J + 8 * jn + 2 * (lane & 3);
-                    const float b0 = s.beta[cc], b1 = s.beta[cc + 1];
                     float z[4] = {-y[jn][0], -y[jn][1], -y[jn][2], -y[jn][3]};
-                    float z2[4] = {z[0] * b0, z[1] * b1, z[2] * b0, z[3] * b1};
                     st_c<Swz<64>>(s.T, 16 * I, 16 * J + 8 * jn, z);
-                    st_c<Swz<64>>(s.T2, 16 * I, 16 * J + 8 * jn, z2);
                 }
             }
             __syncthreads();
         }
     }
 
-    // ---- W^T = (e^G K)^T T2^T ; U~^T = V^T T2^T ------------------------------
-    fence_async_smem();  // scaled K and T2 (generic writes) -> tensor-core reads
+    // ---- W^T = (beta e^G K)^T T^T ; U~^T = (beta V)^T T^T -----------------------
+    fence_async_smem();  // scaled K, V and T (generic writes) -> tensor-core reads
     tc5::fence_before();
     __syncthreads();
     if (tid == 0) {
         tc5::fence_after();
-        const uint32_t sT2 = smem_u32(s.T2), sV = smem_u32(s.V);
+        const uint32_t sT = smem_u32(s.T), sV = smem_u32(s.V);
 #pragma unroll
         for (int kk = 0; kk < C / 16; ++kk)
-            tc5::mma(tm, tc5::mnmajor(sKQ, kk, KQ_PANEL * 2), tc5::kmajor<C>(sT2, kk), ID_WU, kk > 0);
+            tc5::mma(tm, tc5::mnmajor(sKQ, kk, KQ_PANEL * 2), tc5::kmajor<C>(sT, kk), ID_WU, kk > 0);
 #pragma unroll
         for (int kk = 0; kk < C / 16; ++kk)
-            tc5::mma(tm + 64, tc5::mnmajor(sV, kk, C * 128), tc5::kmajor<C>(sT2, kk), ID_WU, kk > 0);
+            tc5::mma(tm + 64, tc5::mnmajor(sV, kk, C * 128), tc5::kmajor<C>(sT, kk), ID_WU, kk > 0);
         tc5::commit(&s.bar_mma);
     }
     ok = mbar_wait(&s.bar_mma, 1, p.status);
