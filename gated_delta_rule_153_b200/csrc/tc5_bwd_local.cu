@@ -27,9 +27,10 @@
 //   [dU ; dO] V^T     -> dU V^T             [dW ; .] K^T  -> dW K^T
 //   [dT ; .] T^T -> X,  [T^T ; .] X -> T^T X,  [T^T ; .] dW,  [T^T ; .] dU
 //   dk += [dMM ; .] K + [dMM^T ; .] K + [sdPG^T ; .] Q,   dq += [. ; sdPG] K
-// One thread owns one TMEM lane (one token row) in every epilogue; column sums
-// over tokens go through a shared-memory transpose.  One CTA of four warps per
-// chunk; thread 0 issues the loads and the MMAs.
+// In every epilogue four warps share a TMEM lane quarter (one token row per
+// thread) and split the row's columns; per-token sums meet in shared-memory
+// atomics, and column sums over tokens go through a shared-memory transpose.
+// One CTA of sixteen warps per chunk; thread 0 issues the loads and the MMAs.
 #include "async.cuh"
 #include "common.cuh"
 #include "internal.h"
@@ -41,7 +42,7 @@ namespace gdn {
 namespace {
 using namespace tc;
 
-constexpr int BL_THREADS = 128;
+constexpr int BL_THREADS = 512;  // warp w: TMEM lane quarter w % 4, column group w / 4
 constexpr int PAIR = 128 * 64;  // elements of one 128-row, 64-column panel
 // tensor-memory columns
 constexpr uint32_t TA = 0,     // [-dW ; dq accumulator]          128
@@ -68,8 +69,12 @@ struct alignas(1024) BlSmem {
     // rows 64..127
     __nv_bfloat16 T[2 * C * C];
     float G[C], beta[C];
-    float colG[C], colB[C];      // column sums into dG and dbeta
-    float red[4][2];             // per-warp partial sums: <dS,S0>, sum etl <dKt,k>
+    // Fixed-order partial sums (the dg and dbeta results are bit-reproducible):
+    float pG[8][C];              // dG terms of a token's own rows, per (column group, lane half)
+    float pB[4][C];              // dbeta terms, per column group
+    float pC[8][C];              // column sums of hP and hA, per 8-row block
+    float red[16], red2[16];     // per-warp sums: <dS, S0>; etl <dKt, k> (enters dG_last)
+    float dgs[C];                // reverse-cumsum scratch
     uint64_t bar_ld, bar_mma;
     uint32_t tmem;
 };
@@ -96,7 +101,8 @@ GDN_DEV void ld_row32(float* v, uint32_t taddr) {
 GDN_DEV void scale_pair_row(__nv_bfloat16* R, int r, int panel, float f) {
     __nv_bfloat16* row = R + panel * PAIR + r * 64;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
+    for (int jj = 0; jj < 8; ++jj) {
+        const int j = (jj + r) & 7;  // per-row rotated order: lanes on different rows, different banks
         uint4 x = *reinterpret_cast<uint4*>(row + 8 * j);
         uint32_t* w = reinterpret_cast<uint32_t*>(&x);
 #pragma unroll
@@ -108,9 +114,23 @@ GDN_DEV void scale_pair_row(__nv_bfloat16* R, int r, int panel, float f) {
     }
 }
 
-// Element (r, c), c < 128, of a pair region's rows (rows 0..63 or 64..127).
-GDN_DEV float pair_at(const __nv_bfloat16* R, int r, int c) {
-    return __bfloat162float(R[(c >> 6) * PAIR + swz<64>(r, c & 63)]);
+// sum_{c < 32} x[c] * R[r][c0 + c] for row r of a pair region (c0 a multiple
+// of 32): four 16-byte loads of the row's swizzled chunks.
+GDN_DEV float dot_row32(const float* x, const __nv_bfloat16* R, int r, int c0) {
+    const __nv_bfloat16* base = R + (c0 >> 6) * PAIR;
+    float acc = 0.f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const uint4 v = *reinterpret_cast<const uint4*>(base + swz<64>(r, (c0 & 63) + 8 * j));
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 f = unpack_bf16(w[i]);
+            acc = fmaf(x[8 * j + 2 * i], f.x, acc);
+            acc = fmaf(x[8 * j + 2 * i + 1], f.y, acc);
+        }
+    }
+    return acc;
 }
 
 __global__ void __launch_bounds__(BL_THREADS, 1) tc5_bwd_local_kernel(const __grid_constant__ BlPtrs p) {
@@ -179,18 +199,22 @@ __global__ void __launch_bounds__(BL_THREADS, 1) tc5_bwd_local_kernel(const __gr
         s.beta[lane] = lane < L ? p.beta[row0 + lane * rs] : 0.f;
         s.beta[lane + 32] = lane + 32 < L ? p.beta[row0 + (lane + 32) * rs] : 0.f;
     }
-    if (tid < C) { s.colG[tid] = 0.f; s.colB[tid] = 0.f; }
+    if (tid < 16) s.red2[tid] = 0.f;
     tc5::fence_before();
     __syncthreads();
     tc5::fence_after();
     const uint32_t tm = s.tmem;
-    const uint32_t trow = tm + ((uint32_t)(32 * warp) << 16);  // this thread's TMEM lane
+    // TMEM lane quarter q, column group cg; row = this thread's token (lanes
+    // 0..63: tokens of the lower half, lanes 64..127: of the upper half)
+    const int q = warp & 3, cg = warp >> 2, row = 32 * (q & 1) + lane;
+    const uint32_t trow = tm + ((uint32_t)(32 * q) << 16);  // this thread's TMEM lane
     const uint32_t sR1 = smem_u32(s.R1), sR2 = smem_u32(s.R2), sR3 = smem_u32(s.R3),
                    sR4 = smem_u32(s.R4), sR5 = smem_u32(s.R5), sT = smem_u32(s.T);
     constexpr uint32_t PB = PAIR * 2;  // bytes of one pair panel (the panel stride of pair regions)
     const float Gl = s.G[C - 1];
     uint32_t mph = 0;  // phase of bar_mma
-    float rowG = 0.f, rowB = 0.f;  // this thread's token: dG and dbeta terms of its own row
+    float myG = 0.f, myB = 0.f;  // this thread's (token, column group) share of dG / dbeta
+    float myC = 0.f;             // this thread's (column, row block) share of the column sums
     // S0 / dS space, reused once both are dead
     float* Mf = reinterpret_cast<float*>(s.R4 + 2 * C * 64);   // M (fp32, [t][j], rotated columns)
     float* Xs = reinterpret_cast<float*>(s.R5 + 2 * C * 64);   // transpose scratch (fp32)
@@ -229,10 +253,10 @@ __global__ void __launch_bounds__(BL_THREADS, 1) tc5_bwd_local_kernel(const __gr
     mph ^= 1;
     if (__syncthreads_or(!ok)) goto done;
     // dO rows *= scale e^{G_i} (the dq rows), U rows *= e^{G_last - G_i} (the dk rows)
-    {
-        const int r = tid >> 1, pn = tid & 1;
-        scale_pair_row(s.R1, C + r, pn, p.scale * __expf(s.G[r]));
-        scale_pair_row(s.R3, r, pn, __expf(Gl - s.G[r]));
+    if (tid < 256) {
+        const int r = (tid >> 1) & 63, pn = tid & 1;
+        if (tid < 128) scale_pair_row(s.R1, C + r, pn, p.scale * __expf(s.G[r]));
+        else scale_pair_row(s.R3, r, pn, __expf(Gl - s.G[r]));
     }
     fence_async_smem();
     tc5::fence_before();
@@ -252,7 +276,6 @@ __global__ void __launch_bounds__(BL_THREADS, 1) tc5_bwd_local_kernel(const __gr
     mph ^= 1;
     if (__syncthreads_or(!ok)) goto done;
     tc5::fence_after();
-
     {
         // ---- <dS, S0> (before S0 / dS space is reused) ------------------------
         float ss = 0.f;
@@ -262,106 +285,79 @@ __global__ void __launch_bounds__(BL_THREADS, 1) tc5_bwd_local_kernel(const __gr
             const uint32_t xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
 #pragma unroll
             for (int t = 0; t < 4; ++t) {
-                const float2 a = unpack_bf16(xs[t]), b = unpack_bf16(ys[t]);
-                ss += a.x * b.x + a.y * b.y;
+                const float2 a2 = unpack_bf16(xs[t]), b2 = unpack_bf16(ys[t]);
+                ss += a2.x * b2.x + a2.y * b2.y;
             }
         }
         ss = warp_sum(ss);
-        if (lane == 0) s.red[warp][0] = ss;
+        if (lane == 0) s.red[warp] = ss;
     }
     __syncthreads();  // S0 and dS are dead from here on
-    // ---- epilogue A -----------------------------------------------------------
-    if (tid >= C) {
-        // token i: dP, Q K^T -> sdPG row i and hP; <dO' S0, q_i>
-        const int i = tid - C;
-        const float Gi = s.G[i];
-        float dp[32], qk[32];
-        float hrow = 0.f;
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            ld_row32(dp, trow + TC2 + 32 * half);
-            ld_row32(qk, trow + TC1 + 32 * half);
+    {
+        // ---- epilogue A -------------------------------------------------------
+        if (q >= 2) {
+            // token i: dP, Q K^T (columns 16cg..) -> sdPG and hP; <dO' S0, q_i> (columns 32cg..)
+            const int i = row;
+            const float Gi = s.G[i];
+            float dp[16], qk[16], x[32];
+            tc5::ld16(dp, trow + TC2 + 16 * cg);
+            tc5::ld16(qk, trow + TC1 + 16 * cg);
+            ld_row32(x, trow + TA + 32 * cg);
             tc5::wait_ld();
-            uint32_t pk[16];
+            float hrow = 0.f;
+            uint32_t pk[8];
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-                const int j = 32 * half + c;
-                const float gdec = j <= i ? __expf(Gi - s.G[j]) : 0.f;
-                const float g = p.scale * dp[c] * gdec;       // scale dP .* Gamma
+            for (int c = 0; c < 16; ++c) {
+                const int j = 16 * cg + c;
+                const float g = j <= i ? p.scale * dp[c] * __expf(Gi - s.G[j]) : 0.f;  // scale dP .* Gamma
                 const float hp = g * qk[c];                    // dP .* (scale Q K^T .* Gamma)
                 hrow += hp;
                 Xs[i * 64 + ((j + i) & 63)] = hp;              // column sums below
                 dp[c] = g;
             }
 #pragma unroll
-            for (int c = 0; c < 16; ++c) pk[c] = pack_bf16(dp[2 * c], dp[2 * c + 1]);
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4)
-                *reinterpret_cast<uint4*>(sdPG + swz<64>(i, 32 * half + 8 * q4)) =
-                    make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
-        }
-        rowG += hrow;
-        float dqq = 0.f;
-#pragma unroll
-        for (int part = 0; part < 4; ++part) {
-            float x[32];
-            ld_row32(x, trow + TA + 32 * part);
-            tc5::wait_ld();
-#pragma unroll
-            for (int c = 0; c < 32; ++c) dqq += x[c] * pair_at(s.R2, C + i, 32 * part + c);
-        }
-        rowG += dqq;  // scale e^{G_i} <dO S0 row i, q_i>
-    } else {
-        // token t: -dW row t -> dW (bf16, into the dO rows of R1); M row t;
-        // <etl dKt row t, k_t>
-        const int t = tid;
-        const float Gt = s.G[t];
-#pragma unroll
-        for (int part = 0; part < 4; ++part) {
-            float x[32];
-            ld_row32(x, trow + TA + 32 * part);
+            for (int c = 0; c < 8; ++c) pk[c] = pack_bf16(dp[2 * c], dp[2 * c + 1]);
+            *reinterpret_cast<uint4*>(sdPG + swz<64>(i, 16 * cg)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            *reinterpret_cast<uint4*>(sdPG + swz<64>(i, 16 * cg + 8)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            // scale e^{G_i} <dO S0 row i, q_i>, this thread's 32 columns
+            const float dqq = dot_row32(x, s.R2, C + i, 32 * cg);
+            myG += hrow + dqq;
+        } else {
+            // token t: -dW (columns 32cg..) -> dW (bf16, into the dO rows of R1);
+            // M (columns 16cg..); <etl dKt row t, k_t> (columns 32cg..)
+            const int t = row;
+            const float Gt = s.G[t];
+            float x[32], kk[16], y[32];
+            ld_row32(x, trow + TA + 32 * cg);
+            tc5::ld16(kk, trow + TC1 + 16 * cg);
+            ld_row32(y, trow + TB + 32 * cg);
             tc5::wait_ld();
             uint32_t pk[16];
 #pragma unroll
             for (int c = 0; c < 16; ++c) pk[c] = pack_bf16(-x[2 * c], -x[2 * c + 1]);
-            __nv_bfloat16* dst = s.R1 + (part >> 1) * PAIR;  // panel of key columns 32*part..
+            __nv_bfloat16* dst = s.R1 + (cg >> 1) * PAIR;  // panel of key columns 32cg..
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4)
-                *reinterpret_cast<uint4*>(dst + swz<64>(C + t, 32 * (part & 1) + 8 * q4)) =
+                *reinterpret_cast<uint4*>(dst + swz<64>(C + t, 32 * (cg & 1) + 8 * q4)) =
                     make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
-        }
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            float kk[32];
-            ld_row32(kk, trow + TC1 + 32 * half);
-            tc5::wait_ld();
-#pragma unroll
-            for (int c = 0; c < 32; ++c) {
-                const int j = 32 * half + c;
+            for (int c = 0; c < 16; ++c) {
+                const int j = 16 * cg + c;
                 Mf[t * 64 + ((j + t) & 63)] = j < t ? kk[c] * __expf(Gt - s.G[j]) : 0.f;
             }
+            float hk = dot_row32(y, s.R2, t, 32 * cg);
+            myG -= hk;  // -etl_t <dKt_t, k_t>; the same enters dG_last
+            hk = warp_sum(hk);
+            if (lane == 0) s.red2[warp] = hk;
         }
-        float hk = 0.f;
-#pragma unroll
-        for (int part = 0; part < 4; ++part) {
-            float x[32];
-            ld_row32(x, trow + TB + 32 * part);
-            tc5::wait_ld();
-#pragma unroll
-            for (int c = 0; c < 32; ++c) hk += x[c] * pair_at(s.R2, t, 32 * part + c);
-        }
-        rowG -= hk;  // -etl_t <dKt_t, k_t>; the same enters dG_last
-        hk = warp_sum(hk);
-        if (lane == 0) s.red[warp][1] = hk;
     }
     fence_async_smem();
     tc5::fence_before();
     __syncthreads();
-    // column sums of hP: dG_j -= sum_i hP_ij
-    if (tid < C) {
-        float cs = 0.f;
-        for (int i = 0; i < C; ++i) cs += Xs[i * 64 + ((tid + i) & 63)];
-        s.colG[tid] -= cs;
+    {   // column sums of hP: dG_j -= sum_i hP_ij (eight row blocks per column)
+        const int j = tid & 63, pb = tid >> 6;
+#pragma unroll
+        for (int i = 8 * pb; i < 8 * pb + 8; ++i) myC -= Xs[i * 64 + ((j + i) & 63)];
     }
     // ---- phase B: [dW ; .] K^T -----------------------------------------------
     if (tid == 0) {
@@ -376,27 +372,22 @@ __global__ void __launch_bounds__(BL_THREADS, 1) tc5_bwd_local_kernel(const __gr
     if (__syncthreads_or(!ok)) goto done;
     tc5::fence_after();
     // ---- epilogue B: dT row t = beta_j (e^{G_j} dW K^T + dU V^T)_tj -----------
-    if (tid < C) {
-        const int t = tid;
+    if (q < 2) {
+        const int t = row;
+        float tw[16], tu[16];
+        tc5::ld16(tw, trow + TW + 16 * cg);
+        tc5::ld16(tu, trow + TU + 16 * cg);
+        tc5::wait_ld();
+        uint32_t pk[8];
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            float tw[32], tu[32];
-            ld_row32(tw, trow + TW + 32 * half);
-            ld_row32(tu, trow + TU + 32 * half);
-            tc5::wait_ld();
-            uint32_t pk[16];
-#pragma unroll
-            for (int c = 0; c < 16; ++c) {
-                const int j0 = 32 * half + 2 * c;
-                const float d0 = s.beta[j0] * (__expf(s.G[j0]) * tw[2 * c] + tu[2 * c]);
-                const float d1 = s.beta[j0 + 1] * (__expf(s.G[j0 + 1]) * tw[2 * c + 1] + tu[2 * c + 1]);
-                pk[c] = pack_bf16(d0, d1);
-            }
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4)
-                *reinterpret_cast<uint4*>(dTt + swz<64>(t, 32 * half + 8 * q4)) =
-                    make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+        for (int c = 0; c < 8; ++c) {
+            const int j0 = 16 * cg + 2 * c;
+            const float d0 = s.beta[j0] * (__expf(s.G[j0]) * tw[2 * c] + tu[2 * c]);
+            const float d1 = s.beta[j0 + 1] * (__expf(s.G[j0 + 1]) * tw[2 * c + 1] + tu[2 * c + 1]);
+            pk[c] = pack_bf16(d0, d1);
         }
+        *reinterpret_cast<uint4*>(dTt + swz<64>(t, 16 * cg)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        *reinterpret_cast<uint4*>(dTt + swz<64>(t, 16 * cg + 8)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
     }
     fence_async_smem();
     tc5::fence_before();
@@ -413,21 +404,16 @@ __global__ void __launch_bounds__(BL_THREADS, 1) tc5_bwd_local_kernel(const __gr
     mph ^= 1;
     if (__syncthreads_or(!ok)) goto done;
     tc5::fence_after();
-    if (tid < C) {
-        const int t = tid;
+    if (q < 2) {
+        const int t = row;
+        float x[16];
+        tc5::ld16(x, trow + TC1 + 16 * cg);
+        tc5::wait_ld();
+        uint32_t pk[8];
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            float x[32];
-            ld_row32(x, trow + TC1 + 32 * half);
-            tc5::wait_ld();
-            uint32_t pk[16];
-#pragma unroll
-            for (int c = 0; c < 16; ++c) pk[c] = pack_bf16(x[2 * c], x[2 * c + 1]);
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4)
-                *reinterpret_cast<uint4*>(Xt + swz<64>(t, 32 * half + 8 * q4)) =
-                    make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
-        }
+        for (int c = 0; c < 8; ++c) pk[c] = pack_bf16(x[2 * c], x[2 * c + 1]);
+        *reinterpret_cast<uint4*>(Xt + swz<64>(t, 16 * cg)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        *reinterpret_cast<uint4*>(Xt + swz<64>(t, 16 * cg + 8)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
     }
     fence_async_smem();
     tc5::fence_before();
@@ -446,44 +432,39 @@ __global__ void __launch_bounds__(BL_THREADS, 1) tc5_bwd_local_kernel(const __gr
     if (__syncthreads_or(!ok)) goto done;
     tc5::fence_after();
     // ---- epilogue D: dA = strict_lower(-T^T X); dMM; hA; dbeta and dG terms ----
-    if (tid < C) {
-        const int i = tid;
+    if (q < 2) {
+        const int i = row;
         const float Gi = s.G[i], bi = s.beta[i];
+        float x[16];
+        tc5::ld16(x, trow + TC2 + 16 * cg);
+        tc5::wait_ld();
         float hrow = 0.f, brow = 0.f;
+        uint32_t pk[8];
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            float x[32];
-            ld_row32(x, trow + TC2 + 32 * half);
-            tc5::wait_ld();
-            uint32_t pk[16];
-#pragma unroll
-            for (int c = 0; c < 32; ++c) {
-                const int j = 32 * half + c;
-                const float dA = j < i ? -x[c] : 0.f;
-                const float m = Mf[i * 64 + ((j + i) & 63)];  // K K^T .* Gamma (strict lower)
-                brow += dA * m;
-                const float hA = dA * bi * m;
-                hrow += hA;
-                Xs[i * 64 + ((j + i) & 63)] = hA;
-                x[c] = j < i ? dA * bi * __expf(Gi - s.G[j]) : 0.f;  // dMM
-            }
-#pragma unroll
-            for (int c = 0; c < 16; ++c) pk[c] = pack_bf16(x[2 * c], x[2 * c + 1]);
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4)
-                *reinterpret_cast<uint4*>(dMM + swz<64>(i, 32 * half + 8 * q4)) =
-                    make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+        for (int c = 0; c < 16; ++c) {
+            const int j = 16 * cg + c;
+            const float dA = j < i ? -x[c] : 0.f;
+            const float m = Mf[i * 64 + ((j + i) & 63)];  // K K^T .* Gamma (strict lower)
+            brow += dA * m;
+            const float hA = dA * bi * m;
+            hrow += hA;
+            Xs[i * 64 + ((j + i) & 63)] = hA;
+            x[c] = j < i ? dA * bi * __expf(Gi - s.G[j]) : 0.f;  // dMM
         }
-        rowG += hrow;
-        rowB += brow;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) pk[c] = pack_bf16(x[2 * c], x[2 * c + 1]);
+        *reinterpret_cast<uint4*>(dMM + swz<64>(i, 16 * cg)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        *reinterpret_cast<uint4*>(dMM + swz<64>(i, 16 * cg + 8)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        myG += hrow;
+        myB += brow;
     }
     fence_async_smem();
     tc5::fence_before();
     __syncthreads();
-    if (tid < C) {  // column sums of hA: dG_j -= sum_i hA_ij
-        float cs = 0.f;
-        for (int i = 0; i < C; ++i) cs += Xs[i * 64 + ((tid + i) & 63)];
-        s.colG[tid] -= cs;
+    {   // column sums of hA: dG_j -= sum_i hA_ij
+        const int j = tid & 63, pb = tid >> 6;
+#pragma unroll
+        for (int i = 8 * pb; i < 8 * pb + 8; ++i) myC -= Xs[i * 64 + ((j + i) & 63)];
     }
     // ---- phase E: the remaining products --------------------------------------------
     if (tid == 0) {
@@ -518,98 +499,91 @@ __global__ void __launch_bounds__(BL_THREADS, 1) tc5_bwd_local_kernel(const __gr
     mph ^= 1;
     if (__syncthreads_or(!ok)) goto done;
     tc5::fence_after();
-    // ---- epilogue E: dk, dv, dq rows; dbeta / dG terms; dg ----------------------------
-    if (tid < C) {
-        const int t = tid;
+    // ---- epilogue E: dk, dv, dq (columns 32cg..); dbeta / dG terms -------------------
+    if (q < 2) {
+        const int t = row;
         const float bt = s.beta[t], egt = __expf(s.G[t]);
-        const bool live = t < L;
-        __nv_bfloat16* dkp = p.dk + (row0 + (size_t)t * rs) * DK;
-        __nv_bfloat16* dvp = p.dv + (row0 + (size_t)t * rs) * DV;
-        float hk = 0.f, hv = 0.f;
+        float a[32], kg[32];
+        ld_row32(a, trow + TB + 32 * cg);
+        ld_row32(kg, trow + TKG + 32 * cg);
+        tc5::wait_ld();
+        const float hk = dot_row32(kg, s.R2, t, 32 * cg);
+        uint32_t pk[16];
 #pragma unroll
-        for (int part = 0; part < 4; ++part) {
-            float a[32], kg[32];
-            ld_row32(a, trow + TB + 32 * part);
-            ld_row32(kg, trow + TKG + 32 * part);
-            tc5::wait_ld();
-            uint32_t pk[16];
+        for (int c = 0; c < 32; ++c) a[c] = fmaf(bt * egt, kg[c], a[c]);
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-                hk += kg[c] * pair_at(s.R2, t, 32 * part + c);
-                a[c] = fmaf(bt * egt, kg[c], a[c]);
-            }
+        for (int c = 0; c < 16; ++c) pk[c] = pack_bf16(a[2 * c], a[2 * c + 1]);
+        if (t < L) {
+            __nv_bfloat16* dkp = p.dk + (row0 + (size_t)t * rs) * DK + 32 * cg;
 #pragma unroll
-            for (int c = 0; c < 16; ++c) pk[c] = pack_bf16(a[2 * c], a[2 * c + 1]);
-            if (live)
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4)
-                    *reinterpret_cast<uint4*>(dkp + 32 * part + 8 * q4) =
-                        make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+            for (int q4 = 0; q4 < 4; ++q4)
+                *reinterpret_cast<uint4*>(dkp + 8 * q4) =
+                    make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
         }
+        ld_row32(a, trow + TVB + 32 * cg);
+        tc5::wait_ld();
+        const float hv = dot_row32(a, s.R3, C + t, 32 * cg);
 #pragma unroll
-        for (int part = 0; part < 4; ++part) {
-            float vb[32];
-            ld_row32(vb, trow + TVB + 32 * part);
-            tc5::wait_ld();
-            uint32_t pk[16];
+        for (int c = 0; c < 16; ++c) pk[c] = pack_bf16(bt * a[2 * c], bt * a[2 * c + 1]);
+        if (t < L) {
+            __nv_bfloat16* dvp = p.dv + (row0 + (size_t)t * rs) * DV + 32 * cg;
 #pragma unroll
-            for (int c = 0; c < 32; ++c) hv += vb[c] * pair_at(s.R3, C + t, 32 * part + c);
-#pragma unroll
-            for (int c = 0; c < 16; ++c) pk[c] = pack_bf16(bt * vb[2 * c], bt * vb[2 * c + 1]);
-            if (live)
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4)
-                    *reinterpret_cast<uint4*>(dvp + 32 * part + 8 * q4) =
-                        make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+            for (int q4 = 0; q4 < 4; ++q4)
+                *reinterpret_cast<uint4*>(dvp + 8 * q4) =
+                    make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
         }
-        rowB += egt * hk + hv;
-        rowG += bt * egt * hk;
+        myB += egt * hk + hv;
+        myG += bt * egt * hk;
     } else {
-        const int i = tid - C;
-        __nv_bfloat16* dqp = p.dq + (row0 + (size_t)i * rs) * DK;
+        const int i = row;
+        float a[32];
+        ld_row32(a, trow + TA + 32 * cg);
+        tc5::wait_ld();
+        uint32_t pk[16];
 #pragma unroll
-        for (int part = 0; part < 4; ++part) {
-            float a[32];
-            ld_row32(a, trow + TA + 32 * part);
-            tc5::wait_ld();
-            uint32_t pk[16];
+        for (int c = 0; c < 16; ++c) pk[c] = pack_bf16(a[2 * c], a[2 * c + 1]);
+        if (i < L) {
+            __nv_bfloat16* dqp = p.dq + (row0 + (size_t)i * rs) * DK + 32 * cg;
 #pragma unroll
-            for (int c = 0; c < 16; ++c) pk[c] = pack_bf16(a[2 * c], a[2 * c + 1]);
-            if (i < L)
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4)
-                    *reinterpret_cast<uint4*>(dqp + 32 * part + 8 * q4) =
-                        make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+            for (int q4 = 0; q4 < 4; ++q4)
+                *reinterpret_cast<uint4*>(dqp + 8 * q4) =
+                    make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
         }
     }
-    // ---- per-token sums: dG (row terms of both halves + column terms), dg -------
-    {
-        // the dq half's row terms belong to token tid - 64
-        if (tid >= C) s.colB[tid - C] = rowG;  // reuse: hand the other half's dG row terms over
-    }
+    // ---- per-token sums in a fixed order: dG (own-row terms + column terms),
+    // dbeta; dg = reverse cumsum of dG -------------------------------------------
+    s.pG[cg + 4 * (q >> 1)][row] = myG;
+    if (q < 2) s.pB[cg][row] = myB;
+    s.pC[tid >> 6][tid & 63] = myC;
     __syncthreads();
     if (warp < 2) {
         const int t = tid;
-        float dG = rowG + s.colB[t] + s.colG[t];
-        if (t == C - 1)  // G_last: e^{G_last} <dS, S0> + sum_i etl_i <dKt_i, k_i>
-            dG += __expf(Gl) * (s.red[0][0] + s.red[1][0] + s.red[2][0] + s.red[3][0]) + s.red[0][1] +
-                  s.red[1][1];
-        // reverse cumsum over the 64 tokens: dg_t = sum_{j >= t} dG_j
+        float dG = 0.f, dB = 0.f;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) dG += s.pG[k][t] + s.pC[k][t];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) dB += s.pB[k][t];
+        if (t == C - 1) {  // G_last: e^{G_last} <dS, S0> + sum_i etl_i <dKt_i, k_i>
+            float ss = 0.f, la = 0.f;
+#pragma unroll
+            for (int w = 0; w < 16; ++w) { ss += s.red[w]; la += s.red2[w]; }
+            dG += __expf(Gl) * ss + la;
+        }
         float x = dG;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const float y = __shfl_down_sync(0xffffffffu, x, o);
             if (lane + o < 32) x += y;
         }
-        s.colG[t] = x;  // per-warp suffix sums (colG is free again)
-        s.colB[t] = rowB;
+        s.dgs[t] = x;  // per-warp suffix sums
+        s.pB[0][t] = dB;
     }
     __syncthreads();
     if (tid < C) {
-        const float x = s.colG[tid] + (tid < 32 ? s.colG[32] : 0.f);
+        const float x = s.dgs[tid] + (tid < 32 ? s.dgs[32] : 0.f);
         if (tid < L) {
             p.dg[row0 + (size_t)tid * rs] = x;
-            p.dbeta[row0 + (size_t)tid * rs] = s.colB[tid];
+            p.dbeta[row0 + (size_t)tid * rs] = s.pB[0][tid];
         }
     }
 done:

@@ -177,8 +177,11 @@ __global__ void __launch_bounds__(P5_THREADS, 3) tc5_prep_kernel(const __grid_co
             __nv_bfloat16* row = s.KQ + pn * KQ_PANEL + r * 64;
             // same swizzled position in the Tma128 image (panel pn at pn * 4096)
             __nv_bfloat16* kt = p.Kt + (size_t)cid * C * DK + pn * (C * 64) + r * 64;
+            // chunks in a per-row rotated order: the 32 lanes of a warp sit on 16
+            // rows, so a common order would put them all on the same four banks
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
+            for (int jj = 0; jj < 8; ++jj) {
+                const int j = (jj + r) & 7;
                 uint4 x = *reinterpret_cast<uint4*>(row + 8 * j), y;
                 uint32_t* w = reinterpret_cast<uint32_t*>(&x);
                 uint32_t* wt = reinterpret_cast<uint32_t*>(&y);
@@ -194,7 +197,8 @@ __global__ void __launch_bounds__(P5_THREADS, 3) tc5_prep_kernel(const __grid_co
             const float b = s.beta[r];
             __nv_bfloat16* vrow = s.V + pn * (C * 64) + r * 64;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
+            for (int jj = 0; jj < 8; ++jj) {
+                const int j = (jj + r) & 7;
                 uint4 x = *reinterpret_cast<uint4*>(vrow + 8 * j);
                 uint32_t* w = reinterpret_cast<uint32_t*>(&x);
 #pragma unroll

@@ -47,7 +47,7 @@
 namespace gdn {
 namespace tc {
 void launch_seg_scan(float* E, const float* Mmap, const float* Nmap, int nseg, int chains,
-                     cudaStream_t st);
+                     unsigned int* status, cudaStream_t st);
 }
 namespace {
 using namespace tc;
@@ -450,39 +450,57 @@ __global__ void __launch_bounds__(W5_THREADS) tc5_walk_kernel(const __grid_const
 
 // ---------------------------------------------------------------------------
 // Scan over the runs of each chain: E_{j+1} = E_j M_j + N_j for j = 1 ..
-// nseg-2, in fp32 (E_1 comes from run 0).  One CTA per (state row block of
-// 8 rows, chain); M_j is staged through shared memory a 64-row half at a time.
+// nseg-2, in fp32 (E_1 comes from run 0).  One CTA per (16-row block of the
+// state, chain).  M_j (64 KB fp32) arrives in shared memory by two bulk copies
+// on an mbarrier, the next step's map one step ahead (two buffers).
 // ---------------------------------------------------------------------------
-constexpr int SC_THREADS = 256, SC_ROWS = 8;
+constexpr int SC_THREADS = 512, SC_ROWS = 16;
+struct ScSmem {
+    float M[2][DK * DK];   // double-buffered map
+    float Er[SC_ROWS][DK];
+    uint64_t bar[2];
+};
 __global__ void __launch_bounds__(SC_THREADS) tc5_seg_scan_kernel(float* E, const float* Mmap,
-                                                                  const float* Nmap, int nseg) {
-    __shared__ __align__(16) float Ms[64][DK];
-    __shared__ __align__(16) float Er[SC_ROWS][DK];
+                                                                  const float* Nmap, int nseg,
+                                                                  unsigned int* status) {
+    extern __shared__ __align__(128) unsigned char sc_raw[];
+    ScSmem& s = *reinterpret_cast<ScSmem*>(sc_raw);
     const int tid = threadIdx.x;
     const int b = blockIdx.y, r0 = blockIdx.x * SC_ROWS;
     const int r = tid >> 5, c0 = (tid & 31) * 4;  // row r0 + r, columns c0 .. c0+3
+    auto slot = [&](int j) { return ((size_t)b * nseg + j) * DV * DK; };
+    auto fetch = [&](int j) {  // map of run j into buffer j & 1
+        uint64_t* bar = &s.bar[j & 1];
+        mbar_arrive_expect(bar, DK * DK * 4);
+        bulk_g2s(s.M[j & 1], Mmap + slot(j), DK * DK * 2, bar);
+        bulk_g2s(s.M[j & 1] + DK * DK / 2, Mmap + slot(j) + DK * DK / 2, DK * DK * 2, bar);
+    };
+    if (tid == 0) {
+        mbar_init(&s.bar[0], 1);
+        mbar_init(&s.bar[1], 1);
+        fence_mbar_init();
+        if (nseg > 2) fetch(1);
+    }
+    __syncthreads();
+    bool ok = true;
     for (int j = 1; j + 1 < nseg; ++j) {
-        const size_t slot = ((size_t)b * nseg + j) * DV * DK;
+        if (tid == 0 && j + 2 < nseg) fetch(j + 1);  // buffer of step j-1, released at its end
         for (int e = tid; e < SC_ROWS * DK / 4; e += SC_THREADS)
-            reinterpret_cast<float4*>(&Er[0][0])[e] =
-                reinterpret_cast<const float4*>(E + slot + (size_t)r0 * DK)[e];
-        float4 acc = reinterpret_cast<const float4*>(Nmap + slot + (size_t)(r0 + r) * DK)[c0 / 4];
-        for (int half = 0; half < 2; ++half) {
-            __syncthreads();
-            for (int e = tid; e < 64 * DK / 4; e += SC_THREADS)
-                reinterpret_cast<float4*>(&Ms[0][0])[e] =
-                    reinterpret_cast<const float4*>(Mmap + slot + (size_t)64 * half * DK)[e];
-            __syncthreads();
+            reinterpret_cast<float4*>(&s.Er[0][0])[e] =
+                reinterpret_cast<const float4*>(E + slot(j) + (size_t)r0 * DK)[e];
+        float4 acc = reinterpret_cast<const float4*>(Nmap + slot(j) + (size_t)(r0 + r) * DK)[c0 / 4];
+        ok = ok && mbar_wait(&s.bar[j & 1], ((j - 1) >> 1) & 1, status);
+        if (__syncthreads_or(!ok)) break;
+        const float* M = s.M[j & 1];
 #pragma unroll 8
-            for (int k = 0; k < 64; ++k) {
-                const float e = Er[r][64 * half + k];
-                const float4 m = *reinterpret_cast<const float4*>(&Ms[k][c0]);
-                acc.x = fmaf(e, m.x, acc.x); acc.y = fmaf(e, m.y, acc.y);
-                acc.z = fmaf(e, m.z, acc.z); acc.w = fmaf(e, m.w, acc.w);
-            }
+        for (int k = 0; k < DK; ++k) {
+            const float e = s.Er[r][k];
+            const float4 m = *reinterpret_cast<const float4*>(M + k * DK + c0);
+            acc.x = fmaf(e, m.x, acc.x); acc.y = fmaf(e, m.y, acc.y);
+            acc.z = fmaf(e, m.z, acc.z); acc.w = fmaf(e, m.w, acc.w);
         }
-        reinterpret_cast<float4*>(E + slot + (size_t)DV * DK + (size_t)(r0 + r) * DK)[c0 / 4] = acc;
-        __syncthreads();
+        reinterpret_cast<float4*>(E + slot(j) + (size_t)DV * DK + (size_t)(r0 + r) * DK)[c0 / 4] = acc;
+        __syncthreads();  // this step's E rows written, its map buffer free
     }
 }
 
@@ -513,17 +531,19 @@ void run_segments(W5Ptrs& w, const TcLayout& L, void* ws, cudaStream_t st) {
     w.Mmap = (float*)((char*)ws + L.segM);
     w.Nmap = (float*)((char*)ws + L.segN);
     launch_w5<KDA, 2>(w, w.B * w.H * (2 * w.nseg - 3), st);
-    if (w.nseg > 2) tc::launch_seg_scan(w.E, w.Mmap, w.Nmap, w.nseg, w.B * w.H, st);
+    if (w.nseg > 2) tc::launch_seg_scan(w.E, w.Mmap, w.Nmap, w.nseg, w.B * w.H, w.status, st);
 }
 
 }  // namespace
 
 namespace tc {
 void launch_seg_scan(float* E, const float* Mmap, const float* Nmap, int nseg, int chains,
-                     cudaStream_t st) {
+                     unsigned int* status, cudaStream_t st) {
+    const int smem = sizeof(ScSmem);
+    cudaFuncSetAttribute(tc5_seg_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     GDN_LAUNCH("tc5_seg_scan", st,
-               (tc5_seg_scan_kernel<<<dim3(DV / SC_ROWS, chains), SC_THREADS, 0, st>>>(
-                   E, Mmap, Nmap, nseg)));
+               (tc5_seg_scan_kernel<<<dim3(DV / SC_ROWS, chains), SC_THREADS, smem, st>>>(
+                   E, Mmap, Nmap, nseg, status)));
 }
 
 void launch_walk5_fwd(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& c, const float* h0,

@@ -365,7 +365,7 @@ void launch_rb(const RbPtrs& p, int grid, cudaStream_t st) {
 
 namespace tc {
 void launch_seg_scan(float* E, const float* Mmap, const float* Nmap, int nseg, int chains,
-                     cudaStream_t st);
+                     unsigned int* status, cudaStream_t st);
 
 bool launch_walk5_bwd(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& c, const void* dO,
                       const float* dhT, float* dh0, void* ws, cudaStream_t st) {
@@ -387,7 +387,7 @@ bool launch_walk5_bwd(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& c, 
         p.Nmap = (float*)((char*)ws + L.segN);
         if (kda) launch_rb<true, 2>(p, chains * (2 * p.nseg - 3), st);
         else launch_rb<false, 2>(p, chains * (2 * p.nseg - 3), st);
-        if (p.nseg > 2) launch_seg_scan(p.E, p.Mmap, p.Nmap, p.nseg, chains, st);
+        if (p.nseg > 2) launch_seg_scan(p.E, p.Mmap, p.Nmap, p.nseg, chains, p.status, st);
     }
     if (kda) launch_rb<true, 0>(p, chains * p.nseg, st);
     else launch_rb<false, 0>(p, chains * p.nseg, st);
