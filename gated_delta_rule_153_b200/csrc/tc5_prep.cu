@@ -151,18 +151,30 @@ __global__ void __launch_bounds__(P5_THREADS, 3) tc5_prep_kernel(const __grid_co
             const float f = is_a ? s.beta[r] : (r < L ? p.scale : 0.f);
             const int lim = is_a ? r : r + 1;
 #pragma unroll
-            for (int c = 0; c < 64; ++c) v[c] = (c < lim) ? f * v[c] * __expf(Gr - s.G[c]) : 0.f;
+            for (int c = 0; c < 32; ++c) v[c] = (c < lim) ? f * v[c] * __expf(Gr - s.G[c]) : 0.f;
+            if (warp & 1) {  // rows 32..63 of A or P: the second half of the row is live
+#pragma unroll
+                for (int c = 32; c < 64; ++c) v[c] = (c < lim) ? f * v[c] * __expf(Gr - s.G[c]) : 0.f;
+            } else {         // rows 0..31: columns 32.. are masked
+#pragma unroll
+                for (int c = 32; c < 64; ++c) v[c] = 0.f;
+            }
             __nv_bfloat16* dst = is_a ? Abf : s.P;
 #pragma unroll
             for (int j = 0; j < 8; ++j)
                 *reinterpret_cast<uint4*>(dst + swz<C>(r, 8 * j)) =
                     make_uint4(pack_bf16(v[8 * j], v[8 * j + 1]), pack_bf16(v[8 * j + 2], v[8 * j + 3]),
                                pack_bf16(v[8 * j + 4], v[8 * j + 5]), pack_bf16(v[8 * j + 6], v[8 * j + 7]));
-            if (is_a) {
-                const int b = r >> 4;
-#pragma unroll
-                for (int c = 0; c < 64; ++c)
-                    if ((c >> 4) == b) Ad[b][r & 15][c & 15] = v[c];
+            if (is_a) {  // the row's diagonal 16x16 block of A, exact in fp32
+                float* ad = &Ad[r >> 4][r & 15][0];
+                switch (r >> 4) {
+#define GDN_DIAG_BLOCK(B)                                          \
+                    case B:                                        \
+                        _Pragma("unroll") for (int c = 0; c < 16; ++c) ad[c] = v[16 * B + c]; \
+                        break;
+                    GDN_DIAG_BLOCK(0) GDN_DIAG_BLOCK(1) GDN_DIAG_BLOCK(2) GDN_DIAG_BLOCK(3)
+#undef GDN_DIAG_BLOCK
+                }
             }
         }
         tc5::fence_before();
