@@ -61,7 +61,9 @@ struct alignas(1024) RbStage {
 struct RbSmem {
     RbStage st[RB_STAGES];
     uint64_t full[RB_STAGES], empty[RB_STAGES];
-    uint64_t ds_ready, q_ready, du_ready, e_done, t_done, fin;
+    // q_ready[k & 1]: Q^ of step k in place (two barriers: the epilogue may
+    // signal step k+1 before the MMA thread has waited for step k)
+    uint64_t ds_ready, q_ready[2], du_ready, e_done, t_done, fin;
     uint32_t tmem;
 };
 
@@ -155,7 +157,8 @@ __global__ void __launch_bounds__(RB_THREADS) tc5_walk_bwd_kernel(const __grid_c
             mbar_init(&s.empty[i], 1 + RB_EPI_WARPS);
         }
         mbar_init(&s.ds_ready, RB_EPI_WARPS);
-        mbar_init(&s.q_ready, RB_EPI_WARPS);
+        mbar_init(&s.q_ready[0], RB_EPI_WARPS);
+        mbar_init(&s.q_ready[1], RB_EPI_WARPS);
         mbar_init(&s.du_ready, RB_EPI_WARPS);
         mbar_init(&s.e_done, 1);
         mbar_init(&s.t_done, 1);
@@ -202,7 +205,7 @@ __global__ void __launch_bounds__(RB_THREADS) tc5_walk_bwd_kernel(const __grid_c
                     tc5::mma_ts(tm + TE, tm + TADS + 8 * kk, tc5::kmajor<C>(sK, kk), ID_E, kk > 0);
                 tc5::commit(&s.e_done);
                 if (use_do) {
-                    if (!mbar_wait(&s.q_ready, k & 1, p.status)) break;
+                    if (!mbar_wait(&s.q_ready[k & 1], (k >> 1) & 1, p.status)) break;
                     tc5::fence_after();
 #pragma unroll
                     for (int kk = 0; kk < C / 16; ++kk)  // T = dO^T Q^
@@ -288,7 +291,7 @@ __global__ void __launch_bounds__(RB_THREADS) tc5_walk_bwd_kernel(const __grid_c
                 }
             }
             tc5::fence_proxy_async();
-            rb_warp_arrive(&s.q_ready);
+            rb_warp_arrive(&s.q_ready[k & 1]);
             // ---- dU = F + E, zero past the sequence end (E = dS K~^T carries
             // the factors e^{G_last - G_i}) ---------------------------------------
             const float gam = KDA ? 1.f : __expf(st.G[C - 1]);
