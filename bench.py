@@ -43,6 +43,8 @@ FWD_FLOP = 140_629
 BWD_FLOP = 281_259
 FWD_BYTES = 1032      # q,k,v,o bf16 + g,beta fp32
 BWD_BYTES = 1808      # q,k,v,dO read; dq,dk,dv written; g,beta,dg,dbeta
+KDA_FWD_EXTRA = 508   # channel gate: g is d_k fp32 values per token-head, not one
+KDA_BWD_EXTRA = 1016  # g read and dg written
 
 
 def peaks():
@@ -194,6 +196,24 @@ def timed(fn, steps, warmup, barrier=lambda: None):
     barrier()
     torch.cuda.synchronize()
     return s.elapsed_time(e) / steps
+
+
+def kernel_breakdown(gdn, fn, steps):
+    """Per-kernel launch counts, mean times and shares over `steps` calls of fn,
+    from the library's launch hook (two events per launch), in a pass of its own."""
+    cap = 32 * steps + 64
+    torch.cuda.synchronize()
+    gdn.gdn_profile_begin(cap)
+    for _ in range(steps):
+        fn()
+    torch.cuda.synchronize()
+    _, launches = gdn.gdn_profile_end(cap)
+    per = {}
+    for name, ms in launches:
+        per.setdefault(name, []).append(ms)
+    total = sum(sum(v) for v in per.values()) or 1.0
+    return {n: {"launches": len(v), "avg_ms": round(statistics.mean(v), 4),
+                "share": round(sum(v) / total, 4)} for n, v in per.items()}
 
 
 def chunk_step_fn(gdn, d, ws_f, ws_b, outs):
@@ -352,6 +372,7 @@ def run_ours(args, rank, world, dev, barrier, max_over_ranks):
         ms_fb = timed(chunk_step_fn(gdn, li, lws_f, workspaces(gdn, li)[1],
                                     dict(o=lo, hT=lh)), 3, 1, barrier)
         extra["long_context_fwd_bwd_ms"] = round(ms_fb, 3)
+        extra["long_context_fwd"]["kernels"] = kernel_breakdown(gdn, fwd, 5)
         del li, lws_f
         # ---- channel gate (KDA) fwd+bwd -------------------------------------
         ki = to_dev(make_chunk_inputs(KDA, seed=replica_seed(KDA.seed, rank)), dev)
@@ -362,6 +383,11 @@ def run_ours(args, rank, world, dev, barrier, max_over_ranks):
         extra["kda_fwd_bwd"] = {"workload": KDA.name, "ms": round(ms_k, 3),
                                 "tokens_per_s": round(KDA.B * KDA.T / (ms_k / 1e3), 1),
                                 "tflops": round((FWD_FLOP + BWD_FLOP) * kth / (ms_k / 1e3) / 1e12, 2)}
+        kbytes = (FWD_BYTES + KDA_FWD_EXTRA + BWD_BYTES + KDA_BWD_EXTRA) * kth
+        extra["kda_fwd_bwd"].update(
+            algorithmic_bytes=kbytes, hbm_gbs=round(kbytes / (ms_k / 1e3) / 1e9, 1),
+            frac_hbm=round(kbytes / (ms_k / 1e3) / 1e9 / pk["hbm"], 4),
+            kernels=kernel_breakdown(gdn, chunk_step_fn(gdn, ki, kws_f, kws_b, ko), 3))
         del ki, kws_f, kws_b
         # ---- gated DeltaProduct, n = 2 steps per token, 350M-scale shape -----
         from gated_delta_rule_153_b200.inputs import make_product_inputs

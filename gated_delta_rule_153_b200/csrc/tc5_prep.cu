@@ -20,9 +20,7 @@
 // memory.  The row scales beta e^G of W and beta of U~ are applied to the K
 // and V tiles in place once Q K^T and K K^T are done, so both transposed
 // products share the B operand T.
-// The triangular solve keeps the 16x16 diagonal blocks of T exact in fp32
-// registers (forward substitution) and combines the off-diagonal blocks one
-// block diagonal at a time with warp-level MMAs (T_IJ = -T_II sum_K A_IK T_KJ).
+// The triangular solve is the shared UT transform of tc5_solve.cuh.
 //
 // One CTA of four warps per chunk; thread t owns TMEM lane t in both
 // epilogues (row t of [K K^T ; Q K^T], then key / value row t of W^T / U~^T).
@@ -36,6 +34,7 @@
 #include "internal.h"
 #include "mma.cuh"
 #include "tc5.cuh"
+#include "tc5_solve.cuh"
 #include "tc_common.cuh"
 
 namespace gdn {
@@ -222,68 +221,8 @@ __global__ void __launch_bounds__(P5_THREADS, 3) tc5_prep_kernel(const __grid_co
             }
         }
 
-        // ---- UT transform, diagonal block `warp`: forward substitution ------
-        // Lane c (< 16) owns column c of T_ww in registers.
-        const int m0 = 16 * warp;
-        {
-            const int c = lane & 15;
-            float t[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                float v = (i == c) ? 1.f : 0.f;
-#pragma unroll
-                for (int j = 0; j < i; ++j) v -= Ad[warp][i][j] * t[j];
-                t[i] = (i < c) ? 0.f : v;
-            }
-            if (lane < 16) {
-#pragma unroll
-                for (int i = 0; i < 16; ++i) s.T[swz<C>(m0 + i, m0 + c)] = __float2bfloat16_rn(t[i]);
-            }
-            // zero this warp's row block right of the diagonal block
-            for (int e = lane; e < 16 * C; e += 32) {
-                const int r = e >> 6, cc = e & 63;
-                if (cc >= m0 + 16) s.T[swz<C>(m0 + r, cc)] = __float2bfloat16_rn(0.f);
-            }
-        }
-        __syncthreads();
-        // ---- off-diagonal blocks, one block diagonal at a time --------------
-        //   T_IJ = -T_II sum_{K=J}^{I-1} A_IK T_KJ
-        for (int dgl = 1; dgl < 4; ++dgl) {
-            const int J = warp, I = warp + dgl;
-            if (I < 4) {
-                float x[2][4] = {};
-                for (int Kb = J; Kb < I; ++Kb) {
-                    uint32_t a[4], bt[4];
-                    lda<Swz<64>>(a, Abf, 16 * I, 16 * Kb);
-                    ldb_kn<Swz<64>>(bt, s.T, 16 * Kb, 16 * J);
-                    mma16816(x[0], a, bt[0], bt[1]);
-                    mma16816(x[1], a, bt[2], bt[3]);
-                }
-#pragma unroll
-                for (int jn = 0; jn < 2; ++jn) {
-                    const int r = lane >> 2, cc = 8 * jn + 2 * (lane & 3);
-                    *reinterpret_cast<uint32_t*>(&Xs[warp][r * 16 + cc]) = pack_bf16(x[jn][0], x[jn][1]);
-                    *reinterpret_cast<uint32_t*>(&Xs[warp][(r + 8) * 16 + cc]) = pack_bf16(x[jn][2], x[jn][3]);
-                }
-                __syncwarp();
-                uint32_t a[4], bx[4];
-                lda<Swz<64>>(a, s.T, 16 * I, 16 * I);
-                {
-                    const int idx = lane >> 3;
-                    const int row = (lane & 7) + (idx & 1) * 8, col = (idx >> 1) * 8;
-                    ldsm_x4_t(bx, smem_u32(&Xs[warp][row * 16 + col]));
-                }
-                float y[2][4] = {};
-                mma16816(y[0], a, bx[0], bx[1]);
-                mma16816(y[1], a, bx[2], bx[3]);
-#pragma unroll
-                for (int jn = 0; jn < 2; ++jn) {
-                    float z[4] = {-y[jn][0], -y[jn][1], -y[jn][2], -y[jn][3]};
-                    st_c<Swz<64>>(s.T, 16 * I, 16 * J + 8 * jn, z);
-                }
-            }
-            __syncthreads();
-        }
+        // ---- UT transform: T = (I + A)^{-1} ---------------------------------
+        ut_solve(Ad, Abf, s.T, Xs);
     }
 
     // ---- W^T = (beta e^G K)^T T^T ; U~^T = (beta V)^T T^T -----------------------

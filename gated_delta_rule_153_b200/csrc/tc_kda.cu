@@ -342,7 +342,9 @@ __global__ void __launch_bounds__(KP_THREADS) tc_prep_kda_kernel(const __grid_co
 
 }  // namespace
 
+void launch_prep5_kda(const ChunkPtrs& p, size_t nchunks, cudaStream_t st);
 void launch_prep_kda(const ChunkPtrs& p, size_t nchunks, cudaStream_t st) {
+    return launch_prep5_kda(p, nchunks, st);
     const int smem = sizeof(KdaPrepSmem) + 1024;
     cudaFuncSetAttribute(tc_prep_kda_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     GDN_LAUNCH("tc_prep_kda", st, tc_prep_kda_kernel<<<(unsigned)nchunks, KP_THREADS, smem, st>>>(p));
