@@ -546,6 +546,25 @@ def run_ours(args, rank, world, dev, barrier, max_over_ranks):
                 gpu_launches=nlaunch, clocks=clk.summary(), peaks=pk, cfg=cfg)
 
 
+def run_case(args, dev):
+    """One workload alone: `warmup` untimed then `steps` timed steps."""
+    import gated_delta_rule_153_b200 as gdn
+    from gated_delta_rule_153_b200.inputs import KDA, LONG, make_chunk_inputs
+    cfg = KDA if args.case == "kda" else LONG
+    d = to_dev(make_chunk_inputs(cfg, seed=cfg.seed), dev)
+    ws_f, ws_b = workspaces(gdn, d)
+    o = torch.empty_like(d["v"])
+    hT = torch.empty(cfg.B, cfg.H, cfg.dv, cfg.dk, device=dev)
+    if args.case == "kda":
+        fn = chunk_step_fn(gdn, d, ws_f, ws_b, dict(o=o, hT=None))
+    else:
+        fn = lambda: gdn.gdn_chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["h0"],
+                                       o=o, hT=hT, workspace=ws_f)
+    ms = timed(fn, args.steps, args.warmup)
+    print(json.dumps({"case": cfg.name, "ms": round(ms, 4), "steps": args.steps,
+                      "warmup": args.warmup}))
+
+
 def cpu_baseline_oracle(sample_B, sample_T=None, inp=None):
     """The fp64 oracle (as it stands) on host cores: fwd + bwd over the first
     `sample_B` sequences (first `sample_T` tokens of each, default all) of the
@@ -572,6 +591,10 @@ def main():
     ap.add_argument("--headline-only", action="store_true",
                     help="skip the long-context, channel-gate and decode extras")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--case", choices=["kda", "long"],
+                    help="run only this workload's step (channel-gate fwd+bwd, or the "
+                         "long-context forward) and print its time: a short command for "
+                         "kernel profilers, not the contract line")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -628,6 +651,9 @@ def main():
     dev = torch.device("cuda", local if world > 1 else 0)
     torch.cuda.set_device(dev)
 
+    if args.case:
+        run_case(args, dev)
+        return
     r = run_ours(args, rank, world, dev, barrier, max_over_ranks)
 
     cpu = None

@@ -41,6 +41,8 @@ bool launch_walk5_bwd(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& c, 
                       const float* dhT, float* dh0, void* ws, cudaStream_t st);
 bool launch_bwd_local5(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& cp, const void* dO,
                        void* dq, void* dk, void* dv, float* dg, float* dbeta, void* ws, cudaStream_t st);
+bool launch_bwd_local5_kda(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& cp, const void* dO,
+                           void* dq, void* dk, void* dv, float* dg, float* dbeta, void* ws, cudaStream_t st);
 }  // namespace tc
 
 namespace {
@@ -893,7 +895,7 @@ bool launch_tc_bwd(const gdn_dims& d, const void* q, const void* k, const void* 
         return false;
     }
     if (kda_gate)
-        return launch_bwd_local_kda(d, L, cp, dO, dq, dk, dv, dg, dbeta, ws, st);
+        return launch_bwd_local5_kda(d, L, cp, dO, dq, dk, dv, dg, dbeta, ws, st);
     return launch_bwd_local5(d, L, cp, dO, dq, dk, dv, dg, dbeta, ws, st);
     LocPtrs lp{};
     lp.qmap = cp.qmap; lp.kmap = cp.kmap; lp.vmap = cp.vmap;
