@@ -65,16 +65,18 @@ def peaks():
 # ratio traffic / algorithmic is reported as the waste factor.
 TH_BYTES = {
     # reads q, k, v (bf16) and g, beta (fp32)
-    "tc_prep": 3 * 256 + 8, "tc5_prep": 3 * 256 + 8,
+    "tc5_prep": 3 * 256 + 8, "tc5_prep_kda": 3 * 256 + 4 + 512,
     # reads q, k; writes o
-    "tc_walk_fwd": 3 * 256, "tc5_walk_fwd": 3 * 256, "tc5_seg_fwd": 3 * 256,
+    "tc_walk_fwd": 3 * 256, "tc5_walk_fwd": 3 * 256,
     # reads k (and v through the prepared images): k only
     "tc_walk_states": 256, "tc5_walk_states": 256, "tc5_seg_map": 256,
+    # the scan over the runs touches only the per-run maps: no layer tensor
+    "tc5_seg_scan": 0,
     # reads q, k, dO
     "tc_walk_bwd": 3 * 256, "tc5_walk_bwd": 3 * 256,
     # reads q, k, v, dO, g, beta; writes dq, dk, dv, dg, dbeta: the whole
     # backward's method bytes
-    "tc_bwd_local": BWD_BYTES, "tc5_bwd_local": BWD_BYTES,
+    "tc5_bwd_local": BWD_BYTES, "tc5_bwd_local_kda": BWD_BYTES + KDA_BWD_EXTRA,
     "simt_bwd": BWD_BYTES, "simt_fwd": FWD_BYTES,
 }
 
@@ -88,14 +90,13 @@ def kernel_work(name, B, T, H):
 
 # Kernel -> source file, for matching a recorded ncu traffic figure to the
 # code it was taken on (profiles/roofline_traffic.md).
-KERNEL_SOURCE = {"tc_prep": "tc_chunk.cu", "tc_walk_fwd": "tc_chunk.cu",
-                 "tc5_prep": "tc5_prep.cu", "tc5_bwd_local": "tc5_bwd_local.cu",
-                 "tc5_seg_fwd": "tc5_walk.cu", "tc5_seg_map": "tc5_walk.cu",
+KERNEL_SOURCE = {"tc_walk_fwd": "tc_chunk.cu", "tc_walk_states": "tc_chunk.cu",
+                 "tc_walk_bwd": "tc_bwd.cu",
+                 "tc5_prep": "tc5_prep.cu", "tc5_prep_kda": "tc5_prep_kda.cu",
+                 "tc5_bwd_local": "tc5_bwd_local.cu", "tc5_bwd_local_kda": "tc5_bwd_local_kda.cu",
+                 "tc5_seg_map": "tc5_walk.cu", "tc5_seg_scan": "tc5_walk.cu",
                  "tc5_walk_fwd": "tc5_walk.cu", "tc5_walk_states": "tc5_walk.cu",
-                 "tc5_walk_bwd": "tc5_walk_bwd.cu",
-                 "tc_walk_states": "tc_chunk.cu", "tc_walk_bwd": "tc_bwd.cu",
-                 "tc_bwd_local": "tc_bwd.cu", "tc_prep_kda": "tc_kda.cu",
-                 "decode_step": "decode.cu"}
+                 "tc5_walk_bwd": "tc5_walk_bwd.cu", "decode_step": "decode.cu"}
 
 
 def recorded_traffic(kernel):
@@ -562,7 +563,7 @@ def run_case(args, dev):
                                        o=o, hT=hT, workspace=ws_f)
     ms = timed(fn, args.steps, args.warmup)
     print(json.dumps({"case": cfg.name, "ms": round(ms, 4), "steps": args.steps,
-                      "warmup": args.warmup}))
+                      "warmup": args.warmup, "kernels": kernel_breakdown(gdn, fn, 2)}))
 
 
 def cpu_baseline_oracle(sample_B, sample_T=None, inp=None):

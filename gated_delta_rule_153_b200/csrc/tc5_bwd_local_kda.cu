@@ -63,10 +63,11 @@ constexpr uint32_t T_QW = 0,   // lane = key: 0..63 (dU S0)^T = -dW^T, 64..127 (
     T_DUV = 256,               // lane = token (rows 0..63): dU V^T
     T_TW = 320,                // lane = token (rows 0..63): dW Kg^T
     T_WT = 384,                // lane = key: (T^T dW)^T
-    T_UT = 448,                // lane = value: (T^T dU)^T
+    T_UT = 128,                // lane = value: (T^T dU)^T
+    T_X = 192,                 // lane = token: dT T^T
     T_TX = 0,                  // lane = token: T^T X
-    T_X = 448,                 // lane = token: dT T^T
     T_PR = 128,                // pair products: 2 x 10 x 16 columns (one round)
+    T_DK = 448,                // lane = key: the dk accumulator, 16 columns per token block
     KB_TCOLS = 512;
 constexpr uint32_t ID_QW = tc5::idesc_bf16(128, 128, true, false);
 constexpr uint32_t ID_MN64 = tc5::idesc_bf16(128, 64, true, false);
@@ -215,7 +216,10 @@ __global__ void __launch_bounds__(KB_THREADS, 1) tc5_bwd_local_kda_kernel(const 
     const uint32_t sKEL = smem_u32(KEL), sQEL = smem_u32(QEL), sKER = smem_u32(KER);
     const uint32_t sdA = smem_u32(Xt), sdMMt = smem_u32(dTt), sdP = smem_u32(s.dP), sdPt = smem_u32(s.dPt);
     uint32_t mph = 0;
-    float dk[16], dG[16];
+    float dG[16];  // this thread's dG terms (dk accumulates in TMEM)
+    const uint32_t tstride = (uint32_t)(rs * DK);  // elements between tokens of a [token][key] tensor
+    // raw log-gate of token t of this thread's block, key c (0 past the sequence end)
+    auto graw = [&](int t) { return i0 + t < L ? p.g[(row0 + (size_t)(i0 + t) * rs) * DK + c] : 0.f; };
     bool ok = mbar_wait(&s.bar_ld, 0, p.status);
     if (__syncthreads_or(!ok)) goto done;
     // dO rows past the sequence end belong to the next sequence: zero them
@@ -253,14 +257,32 @@ __global__ void __launch_bounds__(KB_THREADS, 1) tc5_bwd_local_kda_kernel(const 
     tc5::fence_after();
 
     // ---- epilogue 1 ----------------------------------------------------------------
+    if (q >= 2) {  // dP row i (lanes 64..127), columns of block tg: strict lower; the diagonal apart
+        const int i = 32 * (q - 2) + lane;
+        float pd[16];
+        tc5::ld16(pd, tm + trow + T_DP + i0);
+        tc5::wait_ld();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const int j = i0 + e;
+            if (j == i) s.dPd[i] = pd[e];
+            pd[e] = j < i ? pd[e] : 0.f;
+            s.dPt[swz<64>(j, i)] = __float2bfloat16_rn(pd[e]);
+        }
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh)
+            *reinterpret_cast<uint4*>(s.dP + swz<64>(i, i0 + 8 * hh)) =
+                make_uint4(pack_bf16(pd[8 * hh], pd[8 * hh + 1]), pack_bf16(pd[8 * hh + 2], pd[8 * hh + 3]),
+                           pack_bf16(pd[8 * hh + 4], pd[8 * hh + 5]), pack_bf16(pd[8 * hh + 6], pd[8 * hh + 7]));
+    }
     {
         const float Glast = s.Gl[3][c];
-        float x[16], z[16], pd[16];
+        float x[16], z[16];
         tc5::ld16(x, tm + trow + T_QW + i0);   // -dW^T
         tc5::ld16(z, tm + trow + T_KT + i0);   // (U dS)^T
-        tc5::ld16(pd, tm + trow + T_DP + i0);  // lanes 64..127: dO U^T rows
         tc5::wait_ld();
         float gl = 0.f;
+        uint32_t dku[16];
 #pragma unroll
         for (int r = 0; r < 16; ++r) {
             const int i = i0 + r;
@@ -268,10 +290,13 @@ __global__ void __launch_bounds__(KB_THREADS, 1) tc5_bwd_local_kda_kernel(const 
             const float kv = bf(s.R2, kq);
             s.R1[kq + C * 64] = __float2bfloat16_rn(-x[r]);               // dW, in the dO rows
             s.R3[kq] = __float2bfloat16_rn(kv * __expf(Gr[r]));            // Kg, in the U rows
-            dk[r] = __expf(Glast - Gr[r]) * z[r];                         // etl .* (U dS)
-            dG[r] = -dk[r] * kv;
-            gl += dk[r] * kv;
+            const float dkr = __expf(Glast - Gr[r]) * z[r];               // etl .* (U dS)
+            dku[r] = __float_as_uint(dkr);
+            dG[r] = -dkr * kv;
+            gl += dkr * kv;
         }
+        tc5::st16(tm + trow + T_DK + i0, dku);
+        tc5::wait_st();
         s.glp[tg][c] = gl;
         float ss = 0.f;  // <dS, S0> over value rows 32 tg .. +31 of key c
 #pragma unroll 8
@@ -280,21 +305,6 @@ __global__ void __launch_bounds__(KB_THREADS, 1) tc5_bwd_local_kda_kernel(const 
             ss += bf(s.R5, o) * bf(s.R4, o);
         }
         s.ssp[tg][c] = ss;
-        if (q >= 2) {  // dP row i, columns of block tg: strict lower; the diagonal apart
-            const int i = 32 * (q - 2) + lane;
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-                const int j = i0 + e;
-                if (j == i) s.dPd[i] = pd[e];
-                pd[e] = j < i ? pd[e] : 0.f;
-                s.dPt[swz<64>(j, i)] = __float2bfloat16_rn(pd[e]);
-            }
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh)
-                *reinterpret_cast<uint4*>(s.dP + swz<64>(i, i0 + 8 * hh)) =
-                    make_uint4(pack_bf16(pd[8 * hh], pd[8 * hh + 1]), pack_bf16(pd[8 * hh + 2], pd[8 * hh + 3]),
-                               pack_bf16(pd[8 * hh + 4], pd[8 * hh + 5]), pack_bf16(pd[8 * hh + 6], pd[8 * hh + 7]));
-        }
     }
     fence_async_smem();
     tc5::fence_before();
@@ -321,13 +331,11 @@ __global__ void __launch_bounds__(KB_THREADS, 1) tc5_bwd_local_kda_kernel(const 
 
     // ---- epilogue 2 ----------------------------------------------------------------
     {
-        float wt[16], ut[16], tw[16], du[16];
-        tc5::ld16(wt, tm + trow + T_WT + i0);   // (T^T dW)^T
-        tc5::ld16(ut, tm + trow + T_UT + i0);   // (T^T dU)^T, lane = value c
-        tc5::ld16(tw, tm + trow + T_TW + i0);   // lanes 0..63: dW Kg^T rows
-        tc5::ld16(du, tm + trow + T_DUV + i0);  // lanes 0..63: dU V^T rows
-        tc5::wait_ld();
-        if (q < 2) {  // dT row i, columns of block tg
+        if (q < 2) {  // dT row i, columns of block tg (lanes 0..63)
+            float tw[16], du[16];
+            tc5::ld16(tw, tm + trow + T_TW + i0);   // dW Kg^T
+            tc5::ld16(du, tm + trow + T_DUV + i0);  // dU V^T
+            tc5::wait_ld();
             const int i = 32 * q + lane;
             uint32_t pk[8];
 #pragma unroll
@@ -337,6 +345,10 @@ __global__ void __launch_bounds__(KB_THREADS, 1) tc5_bwd_local_kda_kernel(const 
             *reinterpret_cast<uint4*>(dTt + swz<64>(i, i0)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
             *reinterpret_cast<uint4*>(dTt + swz<64>(i, i0 + 8)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
         }
+        float wt[16], ut[16];
+        tc5::ld16(wt, tm + trow + T_WT + i0);   // (T^T dW)^T
+        tc5::ld16(ut, tm + trow + T_UT + i0);   // (T^T dU)^T, lane = value c
+        tc5::wait_ld();
         const float Gf0 = Gr[0], Gl0 = Gr[15];
         __nv_bfloat16* dvp = p.dv + row0 * DV + c;
 #pragma unroll
@@ -346,18 +358,25 @@ __global__ void __launch_bounds__(KB_THREADS, 1) tc5_bwd_local_kda_kernel(const 
             const uint32_t kq = (c >> 6) * PAIR + swz<64>(i, c & 63);
             const float kv = bf(s.R2, kq), qv = bf(s.R2, kq + C * 64), vv = bf(s.R3, kq + C * 64);
             const float w = eg * wt[r];
-            dk[r] += bi * w;
             dG[r] += bi * w * kv;
-            if (i < L) dvp[(size_t)i * rs * DV] = __float2bfloat16_rn(bi * ut[r]);
-            wt[r] = w * kv + ut[r] * vv;  // dbeta term, summed over keys below
+            if (i < L) dvp[(uint32_t)i * tstride] = __float2bfloat16_rn(bi * ut[r]);
+            ut[r] = w * kv + ut[r] * vv;  // dbeta term, summed over keys below
+            wt[r] = bi * w;               // dk term
             const float el = __expf(Gr[r] - Gf0), er = __expf(Gl0 - Gr[r]);
             const uint32_t o = Tma128::off(i, c);
             KEL[o] = __float2bfloat16_rn(kv * el);
             QEL[o] = __float2bfloat16_rn(qv * el);
             KER[o] = __float2bfloat16_rn(kv * er);
         }
-        const float b = reduce16(wt, lane);
+        const float b = reduce16(ut, lane);
         if (!(lane & 1)) s.dbp[0][q][i0 + (lane >> 1)] = b;
+        tc5::ld16(ut, tm + trow + T_DK + i0);
+        tc5::wait_ld();
+        uint32_t dku[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) dku[r] = __float_as_uint(ut[r] + wt[r]);
+        tc5::st16(tm + trow + T_DK + i0, dku);
+        tc5::wait_st();
     }
     fence_async_smem();
     tc5::fence_before();
@@ -460,25 +479,38 @@ __global__ void __launch_bounds__(KB_THREADS, 1) tc5_bwd_local_kda_kernel(const 
         }
 #pragma unroll
         for (int r = 0; r < 16; ++r) acc[r] *= __expf(Gr[r] - GfI);
-        if (exact) {
+        if (exact) {  // e^{G_r - G_jj} from the in-block partial sums of g
 #pragma unroll
-            for (int r = 1; r < 16; ++r)
-#pragma unroll
-                for (int jj = 0; jj < r; ++jj)
-                    acc[r] += bf(Xt, swz<64>(i0 + r, i0 + jj)) * __expf(Gr[r] - Gr[jj]) *
+            for (int r = 1; r < 16; ++r) {
+                float sg = 0.f;
+#pragma unroll 1
+                for (int jj = r - 1; jj >= 0; --jj) {
+                    sg += graw(jj + 1);
+                    acc[r] += bf(Xt, swz<64>(i0 + r, i0 + jj)) * __expf(sg) *
                               bf(s.R2, (c >> 6) * PAIR + swz<64>(i0 + jj, c & 63));
+                }
+            }
         }
         // X1' -> dk, dG, dbeta
 #pragma unroll
         for (int r = 0; r < 16; ++r) {
             const int i = i0 + r;
             const float bi = s.beta[i], kv = bf(s.R2, (c >> 6) * PAIR + swz<64>(i, c & 63));
-            dk[r] = fmaf(bi, acc[r], dk[r]);
             dG[r] = fmaf(bi * kv, acc[r], dG[r]);
+            a[r] = bi * acc[r];  // dk term
             acc[r] *= kv;
         }
         const float b = reduce16(acc, lane);
         if (!(lane & 1)) s.dbp[1][q][i0 + (lane >> 1)] = b;
+        {
+            tc5::ld16(acc, tm + trow + T_DK + i0);
+            tc5::wait_ld();
+            uint32_t dku[16];
+#pragma unroll
+            for (int r = 0; r < 16; ++r) dku[r] = __float_as_uint(acc[r] + a[r]);
+            tc5::st16(tm + trow + T_DK + i0, dku);
+            tc5::wait_st();
+        }
         // X4 -> dq (with scale e^G (dO S0) and the diagonal of dP), dG
 #pragma unroll
         for (int r = 0; r < 16; ++r) acc[r] = 0.f;
@@ -493,11 +525,15 @@ __global__ void __launch_bounds__(KB_THREADS, 1) tc5_bwd_local_kda_kernel(const 
         for (int r = 0; r < 16; ++r) acc[r] *= __expf(Gr[r] - GfI);
         if (exact) {
 #pragma unroll
-            for (int r = 1; r < 16; ++r)
-#pragma unroll
-                for (int jj = 0; jj < r; ++jj)
-                    acc[r] += bf(s.dP, swz<64>(i0 + r, i0 + jj)) * __expf(Gr[r] - Gr[jj]) *
+            for (int r = 1; r < 16; ++r) {
+                float sg = 0.f;
+#pragma unroll 1
+                for (int jj = r - 1; jj >= 0; --jj) {
+                    sg += graw(jj + 1);
+                    acc[r] += bf(s.dP, swz<64>(i0 + r, i0 + jj)) * __expf(sg) *
                               bf(s.R2, (c >> 6) * PAIR + swz<64>(i0 + jj, c & 63));
+                }
+            }
         }
         tc5::ld16(a, tm + trow + T_QW + 64 + i0);  // (dO S0)^T
         tc5::wait_ld();
@@ -509,7 +545,7 @@ __global__ void __launch_bounds__(KB_THREADS, 1) tc5_bwd_local_kda_kernel(const 
             const float kv = bf(s.R2, kq), qv = bf(s.R2, kq + C * 64);
             const float d = fmaf(__expf(Gr[r]), a[r], acc[r]);  // e^G (dO S0) + X4
             dG[r] = fmaf(p.scale * qv, d, dG[r]);
-            if (i < L) dqp[(size_t)i * rs * DK] = __float2bfloat16_rn(p.scale * fmaf(s.dPd[i], kv, d));
+            if (i < L) dqp[(uint32_t)i * tstride] = __float2bfloat16_rn(p.scale * fmaf(s.dPd[i], kv, d));
         }
     }
     tc5::fence_before();
@@ -539,9 +575,10 @@ __global__ void __launch_bounds__(KB_THREADS, 1) tc5_bwd_local_kda_kernel(const 
         const int J = tg;
         const float GlJ = Gr[15];
         const bool exact = Gr[0] - GlJ > 80.f;
-        float a2[16], a3[16], x2[16], x3[16];
+        // X2 + scale X3 share their factors: one accumulator
+        float a2[16], a3[16], side[16];
 #pragma unroll
-        for (int r = 0; r < 16; ++r) x2[r] = x3[r] = 0.f;
+        for (int r = 0; r < 16; ++r) side[r] = 0.f;
         for (int I = J; I < 4; ++I) {
             const int pi = I * (I + 1) / 2 + J;
             tc5::ld16(a2, tm + trow + T_PR + 16 * pi);
@@ -549,38 +586,35 @@ __global__ void __launch_bounds__(KB_THREADS, 1) tc5_bwd_local_kda_kernel(const 
             tc5::wait_ld();
             const float F = (I == J && exact) ? 0.f : __expf(s.Gf[I][c] - GlJ);
 #pragma unroll
-            for (int r = 0; r < 16; ++r) {
-                x2[r] = fmaf(F, a2[r], x2[r]);
-                x3[r] = fmaf(F, a3[r], x3[r]);
+            for (int r = 0; r < 16; ++r) side[r] = fmaf(F, fmaf(p.scale, a3[r], a2[r]), side[r]);
+        }
+#pragma unroll
+        for (int r = 0; r < 16; ++r) side[r] *= __expf(GlJ - Gr[r]);
+        if (exact) {  // e^{G_ii - G_r} from the in-block partial sums of g
+#pragma unroll
+            for (int r = 0; r < 15; ++r) {
+                float sg = 0.f;
+#pragma unroll 1
+                for (int ii = r + 1; ii < 16; ++ii) {
+                    sg += graw(ii);
+                    const float d = __expf(sg);
+                    const uint32_t kq = (c >> 6) * PAIR + swz<64>(i0 + ii, c & 63);
+                    side[r] += d * fmaf(p.scale * bf(s.dPt, swz<64>(i0 + r, i0 + ii)), bf(s.R2, kq + C * 64),
+                                        bf(dTt, swz<64>(i0 + r, i0 + ii)) * bf(s.R2, kq));
+                }
             }
         }
-#pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            const float er = __expf(GlJ - Gr[r]);
-            x2[r] *= er;
-            x3[r] *= er;
-        }
-        if (exact) {
-#pragma unroll
-            for (int r = 0; r < 15; ++r)
-#pragma unroll
-                for (int ii = r + 1; ii < 16; ++ii) {
-                    const float d = __expf(Gr[ii] - Gr[r]);
-                    const uint32_t kq = (c >> 6) * PAIR + swz<64>(i0 + ii, c & 63);
-                    x2[r] += bf(dTt, swz<64>(i0 + r, i0 + ii)) * d * bf(s.R2, kq);
-                    x3[r] += bf(s.dPt, swz<64>(i0 + r, i0 + ii)) * d * bf(s.R2, kq + C * 64);
-                }
-        }
         __nv_bfloat16* dkp = p.dk + row0 * DK + c;
+        tc5::ld16(a2, tm + trow + T_DK + i0);
+        tc5::wait_ld();
 #pragma unroll
         for (int r = 0; r < 16; ++r) {
             const int j = i0 + r;
             const uint32_t kq = (c >> 6) * PAIR + swz<64>(j, c & 63);
             const float kv = bf(s.R2, kq), qv = bf(s.R2, kq + C * 64);
-            const float side = fmaf(p.scale, x3[r], x2[r]);
-            dG[r] = fmaf(-kv, side, dG[r]);
-            const float dkj = dk[r] + side + p.scale * s.dPd[j] * qv;
-            if (j < L) dkp[(size_t)j * rs * DK] = __float2bfloat16_rn(dkj);
+            dG[r] = fmaf(-kv, side[r], dG[r]);
+            const float dkj = a2[r] + side[r] + p.scale * s.dPd[j] * qv;
+            if (j < L) dkp[(uint32_t)j * tstride] = __float2bfloat16_rn(dkj);
         }
     }
 
@@ -604,7 +638,7 @@ __global__ void __launch_bounds__(KB_THREADS, 1) tc5_bwd_local_kda_kernel(const 
 #pragma unroll
         for (int r = 0; r < 16; ++r) {
             const int i = i0 + r;
-            if (i < L) dgp[(size_t)i * rs * DK] = dG[r] + suf;
+            if (i < L) dgp[(uint32_t)i * tstride] = dG[r] + suf;
         }
         if (tid < C && tid < L) {
             float b = 0.f;

@@ -12,8 +12,8 @@
 //   O  = scale diag(e^G) Q S0^T + P U
 //   S1 = e^{G_last} S0 + U^T diag(e^{G_last - G}) K
 //
-// Kernels (one pass each over the chunks):
-//   prep   -- grid over all (b, h, chunk): G, A, T, W, U~, P  ->  workspace
+// This file holds the 16-row walk and the forward driver (the preparation is
+// tc5_prep.cu / tc5_prep_kda.cu, the whole-head walks tc5_walk.cu):
 //   walk   -- grid over (b, h, 16-row tile of S): the sequential chain
 //             U -> S1 -> ... in fp32, plus O (forward) or the chunk-start
 //             states and U (backward recompute).
@@ -29,7 +29,7 @@
 
 namespace gdn {
 namespace tc {
-void launch_prep_kda(const ChunkPtrs& p, size_t nchunks, cudaStream_t st);
+void launch_prep5_kda(const ChunkPtrs& p, size_t nchunks, cudaStream_t st);
 void launch_prep5(const ChunkPtrs& p, size_t nchunks, cudaStream_t st);
 void launch_walk5_fwd(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& c, const float* h0,
                       void* o, float* hT, void* ws, cudaStream_t st);
@@ -41,238 +41,6 @@ using namespace tc;
 using S128 = Swz<128>;
 using S64 = Swz<64>;
 using P128 = Pad<128>;
-
-// ---------------------------------------------------------------------------
-// prep: one CTA (4 warps) per chunk.  Warp w owns row block 16w..16w+15.
-// ---------------------------------------------------------------------------
-struct PrepSmem {
-    __nv_bfloat16 K[C * DK];   // Tma128; later: U~^T staging (Swz<64>, 128 rows)
-    __nv_bfloat16 Q[C * DK];   // Tma128; then the fp32 diagonal blocks of A and the
-                               // 16x16 scratch of the block solve; then W staging
-    __nv_bfloat16 V[C * DV];   // Tma128
-    __nv_bfloat16 P[C * C];    // Swz<64> image
-    __nv_bfloat16 Ab[C * C];   // bf16 A (Swz<64>), strictly lower blocks used
-    __nv_bfloat16 Tb[C * C];   // bf16 T (Swz<64>)
-    float G[C];
-    float beta[C];
-    float sc1[C];              // beta_j e^{G_j}
-    uint64_t bar;
-};
-
-// Scale the k-columns of an A fragment (16x16 at k0) by f[k].
-GDN_DEV void scale_a_cols(uint32_t (&a)[4], const float* f, int k0) {
-    const int l = threadIdx.x & 31;
-    const int k = k0 + 2 * (l & 3);
-#pragma unroll
-    for (int r = 0; r < 4; ++r) {
-        const int kk = k + (r >> 1) * 8;
-        float2 v = unpack_bf16(a[r]);
-        a[r] = pack_bf16(v.x * f[kk], v.y * f[kk + 1]);
-    }
-}
-
-__global__ void __launch_bounds__(128) tc_prep_kernel(const __grid_constant__ ChunkPtrs p) {
-    extern __shared__ __align__(1024) unsigned char smem_raw[];
-    PrepSmem& s = *reinterpret_cast<PrepSmem*>(align1k(smem_raw));
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int cid = blockIdx.x;
-    const int bh = cid / p.NT, n = cid % p.NT, h = bh % p.H;
-    const ChunkLoc cl = chunk_loc(p.seq, p.T, p.H, bh, n);
-    if (!cl.valid) return;  // past the last chunk of a packed batch
-    const int L = cl.L;
-    const size_t row0 = (size_t)cl.tok * p.H + h;  // token-head index of row 0
-    const size_t rs = (size_t)p.H;                 // token-head stride between rows
-
-    if (tid == 0) {
-        mbar_init(&s.bar, 1);
-        fence_mbar_init();
-        // rows past L hold the next sequence's tokens (or zeros past the
-        // tensor): finite, and annihilated by beta = 0 on those rows
-        mbar_arrive_expect(&s.bar, 3 * C * DK * 2);
-        const int tok = cl.tok;
-        tma_load_tile(s.K, &p.kmap, h, tok, &s.bar);
-        tma_load_tile(s.Q, &p.qmap, h, tok, &s.bar);
-        tma_load_tile(s.V, &p.vmap, h, tok, &s.bar);
-    }
-    if (warp == 0) {
-        // inclusive cumsum of the log-gate over the chunk (rows past L add 0)
-        float g0 = lane < L ? p.g[row0 + lane * rs] : 0.f;
-        float g1 = lane + 32 < L ? p.g[row0 + (lane + 32) * rs] : 0.f;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            float x0 = __shfl_up_sync(0xffffffffu, g0, o);
-            float x1 = __shfl_up_sync(0xffffffffu, g1, o);
-            if (lane >= o) { g0 += x0; g1 += x1; }
-        }
-        g1 += __shfl_sync(0xffffffffu, g0, 31);
-        const float b0 = lane < L ? p.beta[row0 + lane * rs] : 0.f;
-        const float b1 = lane + 32 < L ? p.beta[row0 + (lane + 32) * rs] : 0.f;
-        s.G[lane] = g0;
-        s.G[lane + 32] = g1;
-        s.beta[lane] = b0;
-        s.beta[lane + 32] = b1;
-        s.sc1[lane] = b0 * __expf(g0);
-        s.sc1[lane + 32] = b1 * __expf(g1);
-    }
-    __syncthreads();
-    if (__syncthreads_or(!mbar_wait(&s.bar, 0, p.status))) return;
-
-    const int m0 = 16 * warp;
-    // Q is dead once Q K^T is formed: its space holds the diagonal blocks of A
-    // (fp32, padded rows) and each warp's 16x16 bf16 scratch.
-    auto Ad = reinterpret_cast<float(*)[16][17]>(s.Q);
-    auto Xs = reinterpret_cast<__nv_bfloat16(*)[16 * 16]>(reinterpret_cast<unsigned char*>(s.Q) +
-                                                          4 * 16 * 17 * sizeof(float));
-    // ---- decayed K K^T (-> A) and Q K^T (-> P) for row block `warp` --------
-    {
-        float acck[8][4], accq[8][4];
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) acck[j][e] = accq[j][e] = 0.f;
-#pragma unroll
-        for (int kk = 0; kk < DK / 16; ++kk) {
-            uint32_t ak[4], aq[4];
-            lda<Tma128>(ak, s.K, m0, 16 * kk);
-            lda<Tma128>(aq, s.Q, m0, 16 * kk);
-#pragma unroll
-            for (int np = 0; np < 4; ++np) {
-                if (np > warp) break;  // blocks above the diagonal are masked
-                uint32_t bf[4];
-                ldb_nk<Tma128>(bf, s.K, 16 * np, 16 * kk);
-                mma16816(acck[2 * np], ak, bf[0], bf[1]);
-                mma16816(acck[2 * np + 1], ak, bf[2], bf[3]);
-                mma16816(accq[2 * np], aq, bf[0], bf[1]);
-                mma16816(accq[2 * np + 1], aq, bf[2], bf[3]);
-            }
-        }
-        __syncthreads();  // every warp is done reading Q
-        const int ra = m0 + (lane >> 2), rb2 = ra + 8;
-        const float Gra = s.G[ra], Grb = s.G[rb2], bra = s.beta[ra], brb = s.beta[rb2];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int c0 = 8 * j + 2 * (lane & 3);
-            const bool live = (j >> 1) <= warp;
-            float a[4], pv[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int r = (e < 2) ? ra : rb2, c = c0 + (e & 1);
-                const float dec = (live && c <= r) ? __expf(((e < 2) ? Gra : Grb) - s.G[c]) : 0.f;
-                a[e] = (c < r) ? ((e < 2) ? bra : brb) * acck[j][e] * dec : 0.f;
-                // rows past the sequence end are zero (their q rows are not ours)
-                pv[e] = (r < L) ? accq[j][e] * dec * p.scale : 0.f;
-                if ((j >> 1) == warp) Ad[warp][r - m0][c - m0] = a[e];
-            }
-            st_c<S64>(s.Ab, m0, 8 * j, a);
-            st_c<S64>(s.P, m0, 8 * j, pv);
-        }
-    }
-    __syncwarp();
-
-    // ---- UT transform, diagonal block `warp`: forward substitution ---------
-    // Lane c (< 16) owns column c of T_ww in registers.
-    {
-        const int c = lane & 15;
-        float t[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            float v = (i == c) ? 1.f : 0.f;
-#pragma unroll
-            for (int j = 0; j < i; ++j) v -= Ad[warp][i][j] * t[j];
-            t[i] = (i < c) ? 0.f : v;
-        }
-        if (lane < 16) {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) s.Tb[swz<C>(m0 + i, m0 + c)] = __float2bfloat16_rn(t[i]);
-        }
-        // zero this warp's row block right of the diagonal block
-        for (int e = lane; e < 16 * C; e += 32) {
-            const int r = e >> 6, cc = e & 63;
-            if (cc >= m0 + 16) s.Tb[swz<C>(m0 + r, cc)] = __float2bfloat16_rn(0.f);
-        }
-    }
-    __syncthreads();
-    // ---- off-diagonal blocks, one block diagonal at a time -----------------
-    //   T_IJ = -T_II sum_{K=J}^{I-1} A_IK T_KJ
-    for (int dgl = 1; dgl < 4; ++dgl) {
-        const int J = warp, I = warp + dgl;
-        if (I < 4) {
-            float x[2][4] = {};
-            for (int Kb = J; Kb < I; ++Kb) {
-                uint32_t a[4], bt[4];
-                lda<S64>(a, s.Ab, 16 * I, 16 * Kb);
-                ldb_kn<S64>(bt, s.Tb, 16 * Kb, 16 * J);
-                mma16816(x[0], a, bt[0], bt[1]);
-                mma16816(x[1], a, bt[2], bt[3]);
-            }
-            // X -> bf16 scratch, row-major 16x16 (rows of 32 bytes)
-#pragma unroll
-            for (int jn = 0; jn < 2; ++jn) {
-                const int r = lane >> 2, cc = 8 * jn + 2 * (lane & 3);
-                *reinterpret_cast<uint32_t*>(&Xs[warp][r * 16 + cc]) = pack_bf16(x[jn][0], x[jn][1]);
-                *reinterpret_cast<uint32_t*>(&Xs[warp][(r + 8) * 16 + cc]) = pack_bf16(x[jn][2], x[jn][3]);
-            }
-            __syncwarp();
-            uint32_t a[4], bx[4];
-            lda<S64>(a, s.Tb, 16 * I, 16 * I);
-            {
-                // B[k][n] = X[k][n]
-                const int idx = lane >> 3;
-                const int row = (lane & 7) + (idx & 1) * 8, col = (idx >> 1) * 8;
-                ldsm_x4_t(bx, smem_u32(&Xs[warp][row * 16 + col]));
-            }
-            float y[2][4] = {};
-            mma16816(y[0], a, bx[0], bx[1]);
-            mma16816(y[1], a, bx[2], bx[3]);
-#pragma unroll
-            for (int jn = 0; jn < 2; ++jn) {
-                float z[4] = {-y[jn][0], -y[jn][1], -y[jn][2], -y[jn][3]};
-                st_c<S64>(s.Tb, 16 * I, 16 * J + 8 * jn, z);
-            }
-        }
-        __syncthreads();
-    }
-
-    // ---- W = T diag(beta e^G) K,  U~ = T diag(beta) V  (T lower triangular) -
-    float aw[16][4], au[16][4];
-#pragma unroll
-    for (int j = 0; j < 16; ++j)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) aw[j][e] = au[j][e] = 0.f;
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-        if (kk > warp) break;
-        uint32_t a1[4], a2[4];
-        lda<S64>(a1, s.Tb, m0, 16 * kk);
-#pragma unroll
-        for (int r = 0; r < 4; ++r) a2[r] = a1[r];
-        scale_a_cols(a1, s.sc1, 16 * kk);
-        scale_a_cols(a2, s.beta, 16 * kk);
-#pragma unroll
-        for (int np = 0; np < 8; ++np) {
-            uint32_t bk[4], bv[4];
-            ldb_kn<Tma128>(bk, s.K, 16 * kk, 16 * np);
-            ldb_kn<Tma128>(bv, s.V, 16 * kk, 16 * np);
-            mma16816(aw[2 * np], a1, bk[0], bk[1]);
-            mma16816(aw[2 * np + 1], a1, bk[2], bk[3]);
-            mma16816(au[2 * np], a2, bv[0], bv[1]);
-            mma16816(au[2 * np + 1], a2, bv[2], bv[3]);
-        }
-    }
-    __syncthreads();  // every warp is done reading K and V
-    stage_w_ut(s.Q, s.K, aw, au, m0);  // W image in Q's slot, U~^T image in K's
-    fence_async_smem();
-    __syncthreads();
-    if (tid == 0) {
-        bulk_s2g(p.W + (size_t)cid * C * DK, s.Q, C * DK * 2);
-        bulk_s2g(p.Ut + (size_t)cid * C * DV, s.K, C * DV * 2);
-        bulk_s2g(p.P + (size_t)cid * C * C, s.P, C * C * 2);
-        bulk_s2g(p.G + (size_t)cid * C, s.G, C * 4);
-        if (p.Tb) bulk_s2g(p.Tb + (size_t)cid * C * C, s.Tb, C * C * 2);
-        bulk_commit();
-        bulk_wait_read<0>();
-    }
-}
 
 // ---------------------------------------------------------------------------
 // walk: the sequential chain over chunks for 16 rows of S, 8 warps.
@@ -686,7 +454,7 @@ bool launch_tc_fwd(const gdn_dims& d, const void* q, const void* k, const void* 
         cp.seq = SeqMap{cu, cstart, nseq};
     }
     const bool kda = d.gate == GDN_GATE_CHANNEL;
-    if (kda) launch_prep_kda(cp, L.nchunks, st);
+    if (kda) launch_prep5_kda(cp, L.nchunks, st);
     else launch_prep(cp, L.nchunks, st);
     if (tc::whole_head_fwd(d, L, cp.seq)) {
         launch_walk5_fwd(d, L, cp, h0, o, hT, ws, st);
