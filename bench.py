@@ -217,10 +217,22 @@ def kernel_breakdown(gdn, fn, steps):
                 "share": round(sum(v) / total, 4)} for n, v in per.items()}
 
 
-def chunk_step_fn(gdn, d, ws_f, ws_b, outs):
+def chunk_step_fn(gdn, d, ws_f, ws_b, outs, saved=True):
+    """One training step of the layer: the forward, then the backward.  With
+    saved=True (the training pair) the forward keeps its chunk products and
+    states in ws_b and the backward reads them; with saved=False both calls
+    are stateless and the backward recomputes them."""
+    if saved:
+        def step():
+            gdn.gdn_chunk_fwd_save(d["q"], d["k"], d["v"], d["g"], d["beta"], d["h0"],
+                                   o=outs["o"], hT=outs["hT"], workspace=ws_b)
+            gdn.gdn_chunk_bwd_saved(d["q"], d["k"], d["v"], d["g"], d["beta"], d["dO"], ws_b,
+                                    d["h0"], d["dhT"])
+        return step
+
     def step():
-        o, hT = gdn.gdn_chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["h0"],
-                                  o=outs["o"], hT=outs["hT"], workspace=ws_f)
+        gdn.gdn_chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["h0"],
+                          o=outs["o"], hT=outs["hT"], workspace=ws_f)
         gdn.gdn_chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["dO"], d["h0"],
                           d["dhT"], workspace=ws_b)
     return step
@@ -234,7 +246,7 @@ def workspaces(gdn, d):
     dims = gdn.make_dims(d["q"], d["v"], d["g"])
     wf = torch.empty(max(gdn.gdn_chunk_fwd_workspace(dims), 256), dtype=torch.uint8,
                      device=d["q"].device)
-    wb = torch.empty(max(gdn.gdn_chunk_bwd_workspace(dims), 256), dtype=torch.uint8,
+    wb = torch.empty(max(gdn.gdn_chunk_saved_workspace(dims), 256), dtype=torch.uint8,
                      device=d["q"].device)
     return wf, wb
 
@@ -344,6 +356,10 @@ def run_ours(args, rank, world, dev, barrier, max_over_ranks):
 
     extra = {}
     if not args.headline_only:
+        # the same step through the stateless pair (the backward recomputes
+        # the chunk products and states), for comparison
+        extra["stateless_step_ms"] = round(timed(chunk_step_fn(gdn, d, ws_f, ws_b, outs, saved=False),
+                                                 max(args.steps // 2, 5), args.warmup, barrier), 4)
         # ---- long-context forward (the 50%-of-tensor-peak target) ----------
         li = to_dev(make_chunk_inputs(LONG, seed=replica_seed(LONG.seed, rank)), dev)
         lws_f, _ = workspaces(gdn, li)
@@ -529,10 +545,11 @@ def run_ours(args, rank, world, dev, barrier, max_over_ranks):
     def e2e_step():
         for n in names_in:
             dbuf[n].copy_(host[n], non_blocking=True)
-        o, _ = gdn.gdn_chunk_fwd(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["g"], dbuf["beta"], h0,
-                                 o=outs["o"], hT=outs["hT"], workspace=ws_f)
-        r = gdn.gdn_chunk_bwd(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["g"], dbuf["beta"],
-                              dbuf["dO"], h0, None, workspace=ws_b)
+        o, _, _ = gdn.gdn_chunk_fwd_save(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["g"],
+                                         dbuf["beta"], h0, o=outs["o"], hT=outs["hT"],
+                                         workspace=ws_b)
+        r = gdn.gdn_chunk_bwd_saved(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["g"], dbuf["beta"],
+                                    dbuf["dO"], ws_b, h0, None)
         hout["o"].copy_(o, non_blocking=True)
         for n in ("dq", "dk", "dv", "dg", "dbeta"):
             hout[n].copy_(r[n], non_blocking=True)

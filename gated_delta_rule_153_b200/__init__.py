@@ -26,7 +26,7 @@ GDN_GATE_SCALAR, GDN_GATE_CHANNEL = 0, 1
 
 # Every symbol include/gdn.h declares.
 EXPORTS = ("gdn_chunk_fwd_workspace", "gdn_chunk_fwd", "gdn_chunk_bwd_workspace",
-           "gdn_chunk_bwd", "gdn_recurrent_step", "gdn_query_device_status",
+           "gdn_chunk_bwd", "gdn_chunk_fwd_save", "gdn_chunk_bwd_saved", "gdn_recurrent_step", "gdn_query_device_status",
            "gdn_status_string", "gdn_profile_begin", "gdn_profile_end",
            "gdn_chunk_fwd_noalloc", "gdn_noalloc_device_status", "gdn_test_stalled_fwd", "gdn_product_fwd_workspace", "gdn_product_fwd",
            "gdn_product_bwd_workspace", "gdn_product_bwd", "gdn_chunk_fwd_varlen_workspace",
@@ -73,6 +73,10 @@ def lib() -> ctypes.CDLL:
             L.gdn_chunk_bwd.argtypes = [dp, vp, vp, vp, fp, fp, fp, vp, fp, vp, vp, vp,
                                         fp, fp, fp, vp, sz, vp]
             L.gdn_chunk_bwd.restype = i
+            L.gdn_chunk_fwd_save.argtypes = L.gdn_chunk_fwd.argtypes
+            L.gdn_chunk_fwd_save.restype = i
+            L.gdn_chunk_bwd_saved.argtypes = L.gdn_chunk_bwd.argtypes
+            L.gdn_chunk_bwd_saved.restype = i
             L.gdn_recurrent_step.argtypes = [i, i, i, i, i, i, f, vp, vp, vp, fp, fp, fp,
                                              vp, vp]
             L.gdn_recurrent_step.restype = i
@@ -253,6 +257,57 @@ def gdn_chunk_bwd(q, k, v, g, beta, dO, h0=None, dhT=None, *, chunk=64, scale=1.
                              nbytes if ws is None else ws.numel() * ws.element_size(),
                              _stream(stream))
     _check(st, "gdn_chunk_bwd")
+    return out
+
+
+def gdn_chunk_saved_workspace(dims: gdn_dims) -> int:
+    """Bytes of the workspace gdn_chunk_fwd_save fills and gdn_chunk_bwd_saved reads."""
+    return max(gdn_chunk_bwd_workspace(dims), gdn_chunk_fwd_workspace(dims))
+
+
+def gdn_chunk_fwd_save(q, k, v, g, beta, h0=None, *, chunk=64, scale=1.0,
+                       output_final_state=True, o=None, hT=None, workspace=None, stream=None):
+    """Forward of a training step.  Returns (o, hT, workspace): pass the
+    workspace, and the same inputs, to gdn_chunk_bwd_saved."""
+    import torch
+    B, T, H, dk, dv = _validate_chunk_inputs(q, k, v, g, beta, h0)
+    dims = make_dims(q, v, g, chunk, scale)
+    if o is None:
+        o = torch.empty(B, T, H, dv, dtype=q.dtype, device=q.device)
+    if output_final_state and hT is None:
+        hT = torch.empty(B, H, dv, dk, dtype=torch.float32, device=q.device)
+    nbytes = gdn_chunk_saved_workspace(dims)
+    ws = _workspace(nbytes, q.device, workspace)
+    st = lib().gdn_chunk_fwd_save(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
+                                  _ptr(beta), _ptr(h0), _ptr(o), _ptr(hT), _ptr(ws),
+                                  nbytes if ws is None else ws.numel() * ws.element_size(),
+                                  _stream(stream))
+    _check(st, "gdn_chunk_fwd_save")
+    return o, hT, ws
+
+
+def gdn_chunk_bwd_saved(q, k, v, g, beta, dO, workspace, h0=None, dhT=None, *, chunk=64,
+                        scale=1.0, stream=None):
+    """Backward from gdn_chunk_fwd_save's workspace; results as gdn_chunk_bwd."""
+    import torch
+    B, T, H, dk, dv = _validate_chunk_inputs(q, k, v, g, beta, h0)
+    _need(dO, "dO", q.dtype, (B, T, H, dv))
+    if dhT is not None:
+        _need(dhT, "dhT", torch.float32, (B, H, dv, dk))
+    dims = make_dims(q, v, g, chunk, scale)
+    out = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dv=torch.empty_like(v),
+               dg=torch.empty_like(g), dbeta=torch.empty_like(beta),
+               dh0=None if h0 is None else torch.empty_like(h0))
+    nbytes = gdn_chunk_saved_workspace(dims)
+    if nbytes and (workspace is None or workspace.numel() * workspace.element_size() < nbytes):
+        raise ValueError(f"workspace must be gdn_chunk_fwd_save's ({nbytes} bytes)")
+    st = lib().gdn_chunk_bwd_saved(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
+                                   _ptr(beta), _ptr(h0), _ptr(dO), _ptr(dhT), _ptr(out["dq"]),
+                                   _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dg"]),
+                                   _ptr(out["dbeta"]), _ptr(out["dh0"]), _ptr(workspace),
+                                   0 if workspace is None else workspace.numel() * workspace.element_size(),
+                                   _stream(stream))
+    _check(st, "gdn_chunk_bwd_saved")
     return out
 
 

@@ -6,6 +6,7 @@
 // supported shape and GDN_F32 go to the fp32 SIMT kernels.  Both run on the
 // GPU; there is no host fallback.
 #include <math.h>
+#include <algorithm>
 #include <stdint.h>
 
 #include "common.cuh"
@@ -140,6 +141,57 @@ gdn_status gdn_chunk_bwd(const gdn_dims* d, const void* q, const void* k, const 
         return GDN_ERR_CUDA;
     if (tc_bwd_supported(*d)) {
         if (!launch_tc_bwd(*d, q, k, v, g, beta, h0, dO, dhT, dq, dk, dv, dg, dbeta, dh0, ws, st))
+            return GDN_ERR_CUDA;
+    } else
+        launch_simt_bwd(*d, q, k, v, g, beta, h0, dO, dhT, dq, dk, dv, dg, dbeta, dh0, ws, st);
+    return launch_status();
+}
+
+gdn_status gdn_chunk_fwd_save(const gdn_dims* d, const void* q, const void* k, const void* v,
+                              const float* g, const float* beta, const float* h0, void* o,
+                              float* hT, void* ws, size_t ws_bytes, gdn_stream_t stream) {
+    gdn_status s = check_dims(d);
+    if (s != GDN_OK) return s;
+    if (!q || !k || !v || !g || !beta || !o) return GDN_ERR_INVALID_ARG;
+    if (!all_aligned({q, k, v, g, beta, h0, o, hT})) return GDN_ERR_INVALID_ARG;
+    if (h0 && hT && h0 == hT) return GDN_ERR_INVALID_ARG;
+    const size_t need = std::max(gdn_chunk_bwd_workspace(d), gdn_chunk_fwd_workspace(d));
+    if (ws_bytes < need || (need && !ws)) return GDN_ERR_WORKSPACE;
+    if (ws && ((uintptr_t)ws & 255u)) return GDN_ERR_WORKSPACE;
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaGetLastError();
+    if (ws && cudaMemsetAsync(ws, 0, sizeof(unsigned int), st) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    if (tc_supported(*d)) {
+        if (!launch_tc_fwd_save(*d, q, k, v, g, beta, h0, o, hT, ws, st)) return GDN_ERR_CUDA;
+    } else {  // the general-shape backward recomputes: nothing to keep
+        launch_simt_fwd(*d, q, k, v, g, beta, h0, o, hT, ws, st);
+    }
+    return launch_status();
+}
+
+gdn_status gdn_chunk_bwd_saved(const gdn_dims* d, const void* q, const void* k, const void* v,
+                               const float* g, const float* beta, const float* h0, const void* dO,
+                               const float* dhT, void* dq, void* dk, void* dv, float* dg,
+                               float* dbeta, float* dh0, void* ws, size_t ws_bytes,
+                               gdn_stream_t stream) {
+    gdn_status s = check_dims(d);
+    if (s != GDN_OK) return s;
+    if (!q || !k || !v || !g || !beta || !dO || !dq || !dk || !dv || !dg || !dbeta)
+        return GDN_ERR_INVALID_ARG;
+    if ((h0 == nullptr) != (dh0 == nullptr)) return GDN_ERR_INVALID_ARG;
+    if (!all_aligned({q, k, v, g, beta, h0, dO, dhT, dq, dk, dv, dg, dbeta, dh0}))
+        return GDN_ERR_INVALID_ARG;
+    const size_t need = std::max(gdn_chunk_bwd_workspace(d), gdn_chunk_fwd_workspace(d));
+    if (ws_bytes < need || (need && !ws)) return GDN_ERR_WORKSPACE;
+    if (ws && ((uintptr_t)ws & 255u)) return GDN_ERR_WORKSPACE;
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaGetLastError();
+    if (ws && cudaMemsetAsync(ws, 0, sizeof(unsigned int), st) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    if (tc_bwd_supported(*d)) {
+        if (!launch_tc_bwd(*d, q, k, v, g, beta, h0, dO, dhT, dq, dk, dv, dg, dbeta, dh0, ws, st,
+                           nullptr, 0, true))
             return GDN_ERR_CUDA;
     } else
         launch_simt_bwd(*d, q, k, v, g, beta, h0, dO, dhT, dq, dk, dv, dg, dbeta, dh0, ws, st);

@@ -44,12 +44,19 @@ bool launch_tc_fwd(const gdn_dims& d, const void* q, const void* k, const void* 
                    const float* g, const float* beta, const float* h0, void* o, float* hT,
                    void* ws, cudaStream_t st, const int* cu = nullptr, int nseq = 0,
                    unsigned long long wait_ns = 1000000000ull, int stall_at = -1);
+// The forward of a training step: launch_tc_fwd's results, plus, in `ws` (a
+// backward-layout workspace), what launch_tc_bwd(..., saved = true) reads
+// back instead of recomputing it.
+bool launch_tc_fwd_save(const gdn_dims& d, const void* q, const void* k, const void* v,
+                        const float* g, const float* beta, const float* h0, void* o, float* hT,
+                        void* ws, cudaStream_t st);
 // True when the forward of these dims runs its chain on the tcgen05 whole-head walk.
 bool tc_fwd_whole_head(const gdn_dims& d);
 bool launch_tc_bwd(const gdn_dims& d, const void* q, const void* k, const void* v,
                    const float* g, const float* beta, const float* h0, const void* dO,
                    const float* dhT, void* dq, void* dk, void* dv, float* dg, float* dbeta,
-                   float* dh0, void* ws, cudaStream_t st, const int* cu = nullptr, int nseq = 0);
+                   float* dh0, void* ws, cudaStream_t st, const int* cu = nullptr, int nseq = 0,
+                   bool saved = false);
 // Chunk offsets of a packed batch: cstart[s] = sum over s' < s of ceil(len_s' / 64).
 // An offset table that is not non-decreasing from 0 to T sets status bit 1 and
 // yields no chunks.

@@ -30,7 +30,9 @@
 // MODE 1 (state recompute for the backward) has no output: it fetches
 // neither Q nor P, runs X alone in place of [X|Y], skips Z, and stores each
 // chunk's entering state (bf16, Kp<128> image: two 64-key panels of 128
-// rows) and U (Tma128, token rows) for the backward kernels.
+// rows) and U (Tma128, token rows) for the backward kernels.  MODE 3 (the
+// forward of a training step) does both: the outputs of MODE 0 and the
+// stores of MODE 1, so the backward need not walk the chain again.
 //
 // Channel gate: Q arrives as the prepared image scale Q .* e^G, K~ is
 // K .* e^{G_last - G} per key channel, G holds e^{G_last,c}, and the decay of
@@ -65,6 +67,7 @@ constexpr uint32_t ID_Z = tc5::idesc_bf16(128, 64, false, false);
 
 // MODE 0: forward (O, hT).  MODE 1: state recompute for the backward (chunk
 // states S0 and U stored).  MODE 2: a segment's affine map (final state only).
+// MODE 3: forward that also stores S0 and U.
 // Forward stage: [W p0 | Q p0 | W p1 | Q p1] (K-major B of [X|Y], 128 rows per
 // 64-key panel, 8 KB each), K~, U~^T, P.
 struct alignas(1024) W5Stage {
@@ -82,7 +85,8 @@ struct alignas(1024) W5LeanStage {
 
 template <int MODE>
 struct W5Cfg {
-    static constexpr bool FULL = MODE == 0;
+    static constexpr bool FULL = MODE == 0 || MODE == 3;  // outputs: Q, P, [X|Y], Z
+    static constexpr bool SAVE = MODE == 1 || MODE == 3;  // S0 and U images stored
     static constexpr int STAGES = FULL ? 3 : 2;
     // tensor-memory columns.  Forward: [X|Y] 0..127, D, Z, then the A operands
     // S (bf16 pairs) and U.  Lean: X and D share columns 0..127 (D is issued
@@ -109,7 +113,7 @@ struct W5Ptrs {
     const float* G;
     __nv_bfloat16* o;
     float* hT;
-    __nv_bfloat16 *S0out, *Uout;  // MODE 1
+    __nv_bfloat16 *S0out, *Uout;  // MODE 1 and 3
     unsigned int* status;
     int B, T, H, NT;
     float scale;
@@ -136,7 +140,7 @@ __device__ void w5_issue(typename W5Smem<MODE>::Stage& st, float* G, uint64_t* b
     constexpr int PANEL = C * 64;  // elements of one 64x64 panel
     const __nv_bfloat16* W = p.W + cid * C * DK;
     const int tok = ch.tok0 + n * C;
-    if constexpr (MODE == 0) {
+    if constexpr (W5Cfg<MODE>::FULL) {
         mbar_arrive_expect(bar, (3 * C * DK + DV * C + C * C) * 2 + GW * 4);  // W, Q, K~, U~^T, P
         bulk_g2s(st.WQ, W, PANEL * 2, bar);
         bulk_g2s(st.WQ + 2 * PANEL, W + PANEL, PANEL * 2, bar);
@@ -207,7 +211,7 @@ GDN_DEV W5Job w5_job(const W5Ptrs& p, int nsteps_of_chain_unused) {
         jb.n_end = (j + 1) * p.seglen;  // clipped to the chain below
         jb.start = j == 0 ? kStartH0 : kStartE;
         jb.use_u = true;
-        jb.out = (MODE == 0 && j == p.nseg - 1 && p.hT) ? p.hT + (size_t)b * DV * DK : nullptr;
+        jb.out = (W5Cfg<MODE>::FULL && j == p.nseg - 1 && p.hT) ? p.hT + (size_t)b * DV * DK : nullptr;
     }
     return jb;
 }
@@ -278,7 +282,7 @@ __global__ void __launch_bounds__(W5_THREADS) tc5_walk_kernel(const __grid_const
                 const uint32_t sK = smem_u32(st.K), sU = smem_u32(st.Ut);
                 // [X|Y] = -S0 [W;Q]^T (X alone without outputs), then X += U~^T:
                 // X is U itself
-                if constexpr (MODE == 0) {
+                if constexpr (Cfg::FULL) {
                     const uint32_t sWQ = smem_u32(st.WQ);
 #pragma unroll
                     for (int kk = 0; kk < DK / 16; ++kk)
@@ -305,7 +309,7 @@ __global__ void __launch_bounds__(W5_THREADS) tc5_walk_kernel(const __grid_const
                     tc5::mma_ts(tm + Cfg::TD, tm + Cfg::TAU + 8 * kk, tc5::mnmajor(sK, kk, C * 128), ID_D,
                                 kk > 0);
                 tc5::commit(&s.d_done);
-                if constexpr (MODE == 0) {
+                if constexpr (Cfg::FULL) {
                     const uint32_t sP = smem_u32(st.P);
 #pragma unroll
                     for (int kk = 0; kk < C / 16; ++kk)
@@ -348,7 +352,7 @@ __global__ void __launch_bounds__(W5_THREADS) tc5_walk_kernel(const __grid_const
             tc5::st16(trow + Cfg::TAS + 16 * cg, r);
             tc5::wait_st();
         };
-        // MODE 1: bf16 state entering chain step n, Kp<128> image (64 contiguous bytes)
+        // MODE 1 / 3: bf16 state entering chain step n, Kp<128> image (64 contiguous bytes)
         auto store_s0 = [&](int n) {
             __nv_bfloat16* dst = p.S0out + ((size_t)ch.img * p.NT + ch.n0 + n) * DV * DK;
 #pragma unroll
@@ -360,7 +364,7 @@ __global__ void __launch_bounds__(W5_THREADS) tc5_walk_kernel(const __grid_const
             }
         };
         store_state();
-        if (MODE == 1 && nsteps > 0) store_s0(n_begin);
+        if (Cfg::SAVE && nsteps > 0) store_s0(n_begin);
         tc5::fence_before();
         warp_arrive(&s.s_ready);
 
@@ -377,7 +381,7 @@ __global__ void __launch_bounds__(W5_THREADS) tc5_walk_kernel(const __grid_const
             {
                 float x[16];
                 tc5::ld16(x, trow + Cfg::TXY + t0);
-                if (MODE == 0) tc5::ld16(y, trow + Cfg::TXY + C + t0);
+                if (Cfg::FULL) tc5::ld16(y, trow + Cfg::TXY + C + t0);
                 tc5::wait_ld();
                 uint32_t ru[8];
 #pragma unroll
@@ -386,7 +390,7 @@ __global__ void __launch_bounds__(W5_THREADS) tc5_walk_kernel(const __grid_const
                 tc5::wait_st();
                 tc5::fence_before();
                 warp_arrive(&s.u_ready);
-                if (MODE == 1) {  // U image, Tma128 token rows (64 contiguous bytes per warp store)
+                if (Cfg::SAVE) {  // U image, Tma128 token rows (64 contiguous bytes per warp store)
                     __nv_bfloat16* dst = p.Uout + ((size_t)ch.img * p.NT + ch.n0 + cn) * C * DV;
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
@@ -410,9 +414,9 @@ __global__ void __launch_bounds__(W5_THREADS) tc5_walk_kernel(const __grid_const
             store_state();
             tc5::fence_before();
             warp_arrive(&s.s_ready);
-            if (MODE != 0) {
+            if (Cfg::SAVE && n + 1 < nsteps) store_s0(cn + 1);
+            if (!Cfg::FULL) {
                 warp_arrive(&s.empty[sn]);
-                if (MODE == 1 && n + 1 < nsteps) store_s0(cn + 1);
                 continue;
             }
             // ---- O^T = scale e^{G_i} S0 Q^T + U^T P^T, tokens t0 .. t0+15 of row a
@@ -508,7 +512,9 @@ template <bool KDA, int MODE>
 void launch_w5(const W5Ptrs& p, int grid, cudaStream_t st) {
     const int smem = sizeof(W5Smem<MODE>) + 1024;
     cudaFuncSetAttribute(tc5_walk_kernel<KDA, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    GDN_LAUNCH(MODE == 0 ? "tc5_walk_fwd" : MODE == 1 ? "tc5_walk_states" : "tc5_seg_map", st,
+    GDN_LAUNCH(MODE == 0 ? "tc5_walk_fwd" : MODE == 1 ? "tc5_walk_states" : MODE == 2 ? "tc5_seg_map"
+                                                                             : "tc5_walk_fwd_save",
+               st,
                (tc5_walk_kernel<KDA, MODE><<<grid, W5_THREADS, smem, st>>>(p)));
 }
 
@@ -547,9 +553,13 @@ void launch_seg_scan(float* E, const float* Mmap, const float* Nmap, int nseg, i
 }
 
 void launch_walk5_fwd(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& c, const float* h0,
-                      void* o, float* hT, void* ws, cudaStream_t st) {
+                      void* o, float* hT, void* ws, cudaStream_t st, bool save) {
     W5Ptrs w = w5_ptrs(d, L, c, h0);
     w.o = (__nv_bfloat16*)o; w.hT = hT;
+    if (save) {  // a backward layout: keep the chunk states and U
+        w.S0out = (__nv_bfloat16*)((char*)ws + L.S0);
+        w.Uout = (__nv_bfloat16*)((char*)ws + L.U);
+    }
     const bool kda = d.gate == GDN_GATE_CHANNEL;
     w.nseg = L.nseg;
     w.seglen = L.seglen;
@@ -557,8 +567,13 @@ void launch_walk5_fwd(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& c, 
         if (kda) run_segments<true>(w, L, ws, st);
         else run_segments<false>(w, L, ws, st);
     }
-    if (kda) launch_w5<true, 0>(w, w.B * w.H * w.nseg, st);
-    else launch_w5<false, 0>(w, w.B * w.H * w.nseg, st);
+    if (save) {
+        if (kda) launch_w5<true, 3>(w, w.B * w.H * w.nseg, st);
+        else launch_w5<false, 3>(w, w.B * w.H * w.nseg, st);
+    } else {
+        if (kda) launch_w5<true, 0>(w, w.B * w.H * w.nseg, st);
+        else launch_w5<false, 0>(w, w.B * w.H * w.nseg, st);
+    }
 }
 
 void launch_walk5_states(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& c, const float* h0,

@@ -328,7 +328,7 @@ bool tc_bwd_supported(const gdn_dims& d) { return tc_supported(d); }
 bool launch_tc_bwd(const gdn_dims& d, const void* q, const void* k, const void* v,
                    const float* g, const float* beta, const float* h0, const void* dO,
                    const float* dhT, void* dq, void* dk, void* dv, float* dg, float* dbeta,
-                   float* dh0, void* ws, cudaStream_t st, const int* cu, int nseq) {
+                   float* dh0, void* ws, cudaStream_t st, const int* cu, int nseq, bool saved) {
     const TcLayout L = tc_layout(d, true, nseq);
     char* base = (char*)ws;
     ChunkPtrs cp;
@@ -340,9 +340,11 @@ bool launch_tc_bwd(const gdn_dims& d, const void* q, const void* k, const void* 
         cp.seq = SeqMap{cu, cstart, nseq};
     }
     const bool kda_gate = d.gate == GDN_GATE_CHANNEL;
-    if (kda_gate) launch_prep5_kda(cp, L.nchunks, st);
-    else launch_prep(cp, L.nchunks, st);
-    launch_walk_states(d, L, cp, h0, ws, st);
+    if (!saved) {  // else launch_tc_fwd_save left these in ws
+        if (kda_gate) launch_prep5_kda(cp, L.nchunks, st);
+        else launch_prep(cp, L.nchunks, st);
+        launch_walk_states(d, L, cp, h0, ws, st);
+    }
 
     BwPtrs bp{};
     bp.dSout = (__nv_bfloat16*)(base + L.dS);

@@ -32,7 +32,7 @@ namespace tc {
 void launch_prep5_kda(const ChunkPtrs& p, size_t nchunks, cudaStream_t st);
 void launch_prep5(const ChunkPtrs& p, size_t nchunks, cudaStream_t st);
 void launch_walk5_fwd(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& c, const float* h0,
-                      void* o, float* hT, void* ws, cudaStream_t st);
+                      void* o, float* hT, void* ws, cudaStream_t st, bool save = false);
 void launch_walk5_states(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& c, const float* h0,
                          void* ws, cudaStream_t st);
 }
@@ -464,6 +464,32 @@ bool launch_tc_fwd(const gdn_dims& d, const void* q, const void* k, const void* 
         w.hT = hT;
         if (kda) launch_walk<0, true>(w, st);
         else launch_walk<0, false>(w, st);
+    }
+    return true;
+}
+
+// The forward of a training step: as launch_tc_fwd, in a backward-layout
+// workspace, keeping what the backward would recompute (T, the chunk-start
+// states and U) next to the prepared images.
+bool launch_tc_fwd_save(const gdn_dims& d, const void* q, const void* k, const void* v,
+                        const float* g, const float* beta, const float* h0, void* o, float* hT,
+                        void* ws, cudaStream_t st) {
+    const TcLayout L = tc_layout(d, true);
+    ChunkPtrs cp;
+    if (!make_chunk_ptrs(cp, d, L, q, k, v, g, beta, ws)) return false;
+    cp.Tb = (__nv_bfloat16*)((char*)ws + L.Tb);
+    const bool kda = d.gate == GDN_GATE_CHANNEL;
+    if (kda) launch_prep5_kda(cp, L.nchunks, st);
+    else launch_prep(cp, L.nchunks, st);
+    if (tc::whole_head_fwd(d, L, cp.seq)) {
+        launch_walk5_fwd(d, L, cp, h0, o, hT, ws, st, true);
+    } else {  // the 16-row walk: outputs, then the states pass the backward would run
+        WalkPtrs w = make_walk_ptrs(d, L, cp, h0);
+        w.o = (__nv_bfloat16*)o;
+        w.hT = hT;
+        if (kda) launch_walk<0, true>(w, st);
+        else launch_walk<0, false>(w, st);
+        launch_walk_states(d, L, cp, h0, ws, st);
     }
     return true;
 }

@@ -113,6 +113,32 @@ gdn_status gdn_chunk_bwd(const gdn_dims *dims, const void *q, const void *k,
                          float *dh0, void *ws, size_t ws_bytes,
                          gdn_stream_t stream);
 
+/* The forward and backward of a training step, with the forward's chunk
+ * products kept for the backward instead of recomputed ("Gated Delta
+ * Networks: Improving Mamba2 with Delta Rule" (paper review), section
+ * "Method": the per-chunk WY factors, the UT transform T and the state
+ * entering each chunk are functions of the forward's inputs alone).
+ * gdn_chunk_fwd_save returns what gdn_chunk_fwd returns and leaves in `ws`
+ * the prepared chunk images, T, and every chunk's entering state and U;
+ * gdn_chunk_bwd_saved then returns what gdn_chunk_bwd returns for the same
+ * primal inputs, reading those from `ws` instead of recomputing them.  Both
+ * take the same workspace: ws_bytes >= max(gdn_chunk_bwd_workspace(dims),
+ * gdn_chunk_fwd_workspace(dims)), 256-byte aligned; the caller owns it and
+ * must keep it, and q, k, v, g, beta, h0, unchanged from the forward until
+ * the backward has run (stream order suffices).  Arguments are otherwise those
+ * of gdn_chunk_fwd / gdn_chunk_bwd, with the same error returns.  For shapes
+ * outside the tensor-core path the backward recomputes, as gdn_chunk_bwd. */
+gdn_status gdn_chunk_fwd_save(const gdn_dims *dims, const void *q, const void *k,
+                              const void *v, const float *g, const float *beta,
+                              const float *h0, void *o, float *hT, void *ws,
+                              size_t ws_bytes, gdn_stream_t stream);
+gdn_status gdn_chunk_bwd_saved(const gdn_dims *dims, const void *q, const void *k,
+                               const void *v, const float *g, const float *beta,
+                               const float *h0, const void *dO, const float *dhT,
+                               void *dq, void *dk, void *dv, float *dg, float *dbeta,
+                               float *dh0, void *ws, size_t ws_bytes,
+                               gdn_stream_t stream);
+
 /* Packed variable-length batches.  Each sequence of a packed batch is its own
  * instance of the recurrence of "Gated Delta Networks: Improving Mamba2 with
  * Delta Rule" (paper review), section "Method": its state starts from its
