@@ -55,9 +55,9 @@ namespace {
 using namespace tc;
 
 constexpr int W5_EPI_WARPS = 16;
-constexpr int W5_THREADS = 32 * (W5_EPI_WARPS + 2);
 constexpr int W5_CTRL = W5_EPI_WARPS;      // MMA warp
 constexpr int W5_PROD = W5_EPI_WARPS + 1;  // load warp
+constexpr int W5_SAVE = W5_EPI_WARPS + 2;  // MODE 3: bulk stores of the chunk states
 constexpr uint32_t NEG_B = 1u << 14;       // instruction descriptor: negate B
 constexpr uint32_t ID_XY = tc5::idesc_bf16(128, 128, false, false) | NEG_B;
 constexpr uint32_t ID_X = tc5::idesc_bf16(128, 64, false, false) | NEG_B;
@@ -87,7 +87,11 @@ template <int MODE>
 struct W5Cfg {
     static constexpr bool FULL = MODE == 0 || MODE == 3;  // outputs: Q, P, [X|Y], Z
     static constexpr bool SAVE = MODE == 1 || MODE == 3;  // S0 and U images stored
-    static constexpr int STAGES = FULL ? 3 : 2;
+    // MODE 3 stages each chunk state in shared memory (two 32 KiB buffers) for
+    // a bulk store by a warp of its own, so its ring has two stages
+    static constexpr bool STAGED = MODE == 3;
+    static constexpr int STAGES = MODE == 0 ? 3 : 2;
+    static constexpr int THREADS = 32 * (W5_EPI_WARPS + 2 + (STAGED ? 1 : 0));
     // tensor-memory columns.  Forward: [X|Y] 0..127, D, Z, then the A operands
     // S (bf16 pairs) and U.  Lean: X and D share columns 0..127 (D is issued
     // only after the epilogue has read X), so two CTAs fit an SM.
@@ -95,8 +99,18 @@ struct W5Cfg {
                          TAU = FULL ? 384 : 192, TCOLS = FULL ? 512 : 256;
 };
 
+// The staged state images of MODE 3 and their hand-off barriers
+template <bool STAGED>
+struct W5Save {
+    __nv_bfloat16 S0[2][DV * DK];  // Kp<128> image of the state entering a step
+    uint64_t full[2], empty[2];
+};
+template <>
+struct W5Save<false> {};
+
 template <int MODE>
 struct W5Smem {
+    W5Save<W5Cfg<MODE>::STAGED> sv;
     using Stage = typename std::conditional<W5Cfg<MODE>::FULL, W5Stage, W5LeanStage>::type;
     Stage st[W5Cfg<MODE>::STAGES];
     __nv_bfloat16 I16[16 * 64];  // 16x16 identity, Swz<64> rows: B of X += U~^T
@@ -217,7 +231,7 @@ GDN_DEV W5Job w5_job(const W5Ptrs& p, int nsteps_of_chain_unused) {
 }
 
 template <bool KDA, int MODE>
-__global__ void __launch_bounds__(W5_THREADS) tc5_walk_kernel(const __grid_constant__ W5Ptrs p) {
+__global__ void __launch_bounds__(W5Cfg<MODE>::THREADS) tc5_walk_kernel(const __grid_constant__ W5Ptrs p) {
     using Cfg = W5Cfg<MODE>;
     using Smem = W5Smem<MODE>;
     constexpr int NST = Cfg::STAGES;
@@ -241,10 +255,16 @@ __global__ void __launch_bounds__(W5_THREADS) tc5_walk_kernel(const __grid_const
         mbar_init(&s.d_done, 1);
         mbar_init(&s.o_done, 1);
         mbar_init(&s.fin, 1);
+        if constexpr (Cfg::STAGED) {
+            for (int i = 0; i < 2; ++i) {
+                mbar_init(&s.sv.full[i], W5_EPI_WARPS);
+                mbar_init(&s.sv.empty[i], 1);
+            }
+        }
         fence_mbar_init();
     }
     // the 16x16 identity (rows of 64 elements, 128-byte swizzle)
-    for (int e = tid; e < 16 * 64; e += W5_THREADS) {
+    for (int e = tid; e < 16 * 64; e += Cfg::THREADS) {
         const int r = e >> 6, c = e & 63;
         s.I16[swz<64>(r, c)] = __float2bfloat16_rn(r == c ? 1.f : 0.f);
     }
@@ -323,6 +343,26 @@ __global__ void __launch_bounds__(W5_THREADS) tc5_walk_kernel(const __grid_const
             mbar_wait(&s.fin, 0, p.status);
         }
         __syncwarp();
+    } else if (warp == W5_SAVE) {
+        // MODE 3: bulk-store each staged chunk state to its image, then hand the
+        // buffer back (state m of this CTA in buffer m & 1)
+        if constexpr (Cfg::STAGED) {
+            if (lane == 0) {
+                int issued = 0;
+                for (int m = 0; m < nsteps; ++m) {
+                    if (!mbar_wait(&s.sv.full[m & 1], (m >> 1) & 1, p.status, p.wait_ns)) break;
+                    bulk_s2g(p.S0out + ((size_t)ch.img * p.NT + ch.n0 + n_begin + m) * DV * DK, s.sv.S0[m & 1],
+                             DV * DK * 2);
+                    bulk_commit();
+                    issued = m + 1;
+                    bulk_wait_read<0>();
+                    mbar_arrive(&s.sv.empty[m & 1]);
+                }
+                (void)issued;
+                bulk_wait<0>();  // every store complete before the CTA exits
+            }
+            __syncwarp();
+        }
     } else {
         // ---- epilogue: thread = state row a; key columns 32*cg .. +31 of the
         // state, tokens 16*cg .. +15 of U and O ---------------------------------
@@ -352,9 +392,18 @@ __global__ void __launch_bounds__(W5_THREADS) tc5_walk_kernel(const __grid_const
             tc5::st16(trow + Cfg::TAS + 16 * cg, r);
             tc5::wait_st();
         };
-        // MODE 1 / 3: bf16 state entering chain step n, Kp<128> image (64 contiguous bytes)
+        // MODE 1: bf16 state entering chain step n, Kp<128> image (64 contiguous
+        // bytes per thread).  MODE 3: the same image staged in shared memory
+        // (buffer m & 1 for this CTA's m-th state, m = n - n_begin) for the
+        // saver warp's bulk store.
         auto store_s0 = [&](int n) {
             __nv_bfloat16* dst = p.S0out + ((size_t)ch.img * p.NT + ch.n0 + n) * DV * DK;
+            if constexpr (Cfg::STAGED) {
+                const int m = n - n_begin;
+                if (m >= 2 && !wait_all(&s.sv.empty[m & 1], ((m >> 1) - 1) & 1, p.status, p.wait_ns))
+                    return false;
+                dst = s.sv.S0[m & 1];
+            }
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const int c = 32 * cg + 8 * j;
@@ -362,6 +411,11 @@ __global__ void __launch_bounds__(W5_THREADS) tc5_walk_kernel(const __grid_const
                     make_uint4(pack_bf16(S[8 * j], S[8 * j + 1]), pack_bf16(S[8 * j + 2], S[8 * j + 3]),
                                pack_bf16(S[8 * j + 4], S[8 * j + 5]), pack_bf16(S[8 * j + 6], S[8 * j + 7]));
             }
+            if constexpr (Cfg::STAGED) {
+                fence_async_smem();
+                warp_arrive(&s.sv.full[(n - n_begin) & 1]);
+            }
+            return true;
         };
         store_state();
         if (Cfg::SAVE && nsteps > 0) store_s0(n_begin);
@@ -374,6 +428,16 @@ __global__ void __launch_bounds__(W5_THREADS) tc5_walk_kernel(const __grid_const
             const int cn = n_begin + n;  // chain step
             const int L = min(C, ch.end - (ch.tok0 + cn * C));
             if (!wait_all(&s.full[sn], (n / NST) & 1, p.status, p.wait_ns)) break;
+            // Scalar gate: the epilogue's only reads of the stage are two gate
+            // factors; with them in registers it releases the stage at once (the
+            // MMA thread releases it after the step's last product), so the next
+            // loads need not wait for the output stores.
+            float gam = 1.f, sce = 1.f;
+            if constexpr (!KDA) {
+                gam = __expf(G[C - 1]);
+                sce = p.scale * __expf(G[t0 + (lane & 15)]);
+                warp_arrive(&s.empty[sn]);
+            }
             // ---- U = X (= U~ - S0 W^T); -Y kept for the output -------------
             if (!wait_all(&s.x_done, n & 1, p.status, p.wait_ns)) break;
             tc5::fence_after();
@@ -407,20 +471,18 @@ __global__ void __launch_bounds__(W5_THREADS) tc5_walk_kernel(const __grid_const
                 float d[32];
                 tc5::ld32(d, trow + Cfg::TD + 32 * cg);
                 tc5::wait_ld();
-                const float gam = KDA ? 1.f : __expf(G[C - 1]);
 #pragma unroll
                 for (int j = 0; j < 32; ++j) S[j] = fmaf(KDA ? G[32 * cg + j] : gam, S[j], d[j]);
             }
             store_state();
             tc5::fence_before();
             warp_arrive(&s.s_ready);
-            if (Cfg::SAVE && n + 1 < nsteps) store_s0(cn + 1);
+            if (Cfg::SAVE && n + 1 < nsteps && !store_s0(cn + 1)) break;
             if (!Cfg::FULL) {
-                warp_arrive(&s.empty[sn]);
+                if (KDA) warp_arrive(&s.empty[sn]);
                 continue;
             }
             // ---- O^T = scale e^{G_i} S0 Q^T + U^T P^T, tokens t0 .. t0+15 of row a
-            const float sce = KDA ? 1.f : p.scale * __expf(G[t0 + (lane & 15)]);
             if (!wait_all(&s.o_done, n & 1, p.status, p.wait_ns)) break;
             tc5::fence_after();
             {
@@ -434,8 +496,10 @@ __global__ void __launch_bounds__(W5_THREADS) tc5_walk_kernel(const __grid_const
                     if (t0 + j < L) o[(size_t)j * p.H * DV] = __float2bfloat16_rn(fmaf(-f, y[j], z[j]));
                 }
             }
-            tc5::fence_before();
-            warp_arrive(&s.empty[sn]);
+            if (KDA) {
+                tc5::fence_before();
+                warp_arrive(&s.empty[sn]);
+            }
         }
         if (jb.out) {
             float* out = jb.out + (size_t)a * DK + 32 * cg;
@@ -515,7 +579,7 @@ void launch_w5(const W5Ptrs& p, int grid, cudaStream_t st) {
     GDN_LAUNCH(MODE == 0 ? "tc5_walk_fwd" : MODE == 1 ? "tc5_walk_states" : MODE == 2 ? "tc5_seg_map"
                                                                              : "tc5_walk_fwd_save",
                st,
-               (tc5_walk_kernel<KDA, MODE><<<grid, W5_THREADS, smem, st>>>(p)));
+               (tc5_walk_kernel<KDA, MODE><<<grid, W5Cfg<MODE>::THREADS, smem, st>>>(p)));
 }
 
 W5Ptrs w5_ptrs(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& c, const float* h0) {
