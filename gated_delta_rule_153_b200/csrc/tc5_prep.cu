@@ -22,8 +22,9 @@
 // products share the B operand T.
 // The triangular solve is the shared UT transform of tc5_solve.cuh.
 //
-// One CTA of four warps per chunk; thread t owns TMEM lane t in both
-// epilogues (row t of [K K^T ; Q K^T], then key / value row t of W^T / U~^T).
+// One CTA of eight warps per chunk; warps w and w + 4 share TMEM lane
+// quarter w: in the first epilogue they split a row's columns, in the second
+// one takes W^T and the other U~^T.
 // Shared memory 74 KB and 128 TMEM columns, so three CTAs share an SM.
 // Outputs (bulk stores into the workspace): the W image (Tma128), the U~^T
 // image (Swz<64>, 128 value rows), P (Swz<64>), G, and optionally T (Swz<64>);
@@ -41,7 +42,7 @@ namespace gdn {
 namespace {
 using namespace tc;
 
-constexpr int P5_THREADS = 128;
+constexpr int P5_THREADS = 256;  // warp w: TMEM lane quarter w % 4, column half w / 4
 constexpr uint32_t P5_TCOLS = 128;  // D1 = [KK^T; QK^T] in 0..63; then W^T 0..63, U~^T 64..127
 constexpr uint32_t ID_KQ = tc5::idesc_bf16(128, 64, false, false);
 constexpr uint32_t ID_WU = tc5::idesc_bf16(128, 64, true, false);
@@ -135,44 +136,44 @@ __global__ void __launch_bounds__(P5_THREADS, 3) tc5_prep_kernel(const __grid_co
         auto Xs = reinterpret_cast<__nv_bfloat16(*)[16 * 16]>(
             reinterpret_cast<unsigned char*>(s.KQ + KQ_PANEL + C * 64) + 4 * 16 * 17 * sizeof(float));
 
-        // ---- epilogue 1: thread t = row t of [K K^T ; Q K^T] ---------------
+        // ---- epilogue 1: row r of [K K^T ; Q K^T] (TMEM lane), columns
+        // 32 hf .. +31, two threads per row ----------------------------------
         {
-            const uint32_t trow = tm + ((uint32_t)(32 * warp) << 16);
-            float v[64];
-            tc5::ld32(*reinterpret_cast<float(*)[32]>(&v[0]), trow);
-            tc5::ld32(*reinterpret_cast<float(*)[32]>(&v[32]), trow + 32);
-            tc5::wait_ld();
-            const bool is_a = tid < C;
-            const int r = is_a ? tid : tid - C;
-            const float Gr = s.G[r];
-            // A row r: beta_r (k_r . k_c) e^{G_r - G_c} for c < r;
-            // P row r: scale (q_r . k_c) e^{G_r - G_c} for c <= r (rows past L zero)
-            const float f = is_a ? s.beta[r] : (r < L ? p.scale : 0.f);
-            const int lim = is_a ? r : r + 1;
+            const int ql = warp & 3, hf = warp >> 2, lr = 32 * ql + lane;
+            const uint32_t trow = tm + ((uint32_t)(32 * ql) << 16);
+            const bool is_a = lr < C;
+            const int r = is_a ? lr : lr - C, c0 = 32 * hf;
+            float v[32];
+            // rows 0..31 have their columns 32.. masked: no load, no exponentials
+            const bool live = (ql & 1) || hf == 0;
+            if (live) {
+                tc5::ld32(v, trow + c0);
+                tc5::wait_ld();
+                const float Gr = s.G[r];
+                // A row r: beta_r (k_r . k_c) e^{G_r - G_c} for c < r;
+                // P row r: scale (q_r . k_c) e^{G_r - G_c} for c <= r (rows past L zero)
+                const float f = is_a ? s.beta[r] : (r < L ? p.scale : 0.f);
+                const int lim = is_a ? r : r + 1;
 #pragma unroll
-            for (int c = 0; c < 32; ++c) v[c] = (c < lim) ? f * v[c] * __expf(Gr - s.G[c]) : 0.f;
-            if (warp & 1) {  // rows 32..63 of A or P: the second half of the row is live
+                for (int c = 0; c < 32; ++c) v[c] = (c0 + c < lim) ? f * v[c] * __expf(Gr - s.G[c0 + c]) : 0.f;
+            } else {
 #pragma unroll
-                for (int c = 32; c < 64; ++c) v[c] = (c < lim) ? f * v[c] * __expf(Gr - s.G[c]) : 0.f;
-            } else {         // rows 0..31: columns 32.. are masked
-#pragma unroll
-                for (int c = 32; c < 64; ++c) v[c] = 0.f;
+                for (int c = 0; c < 32; ++c) v[c] = 0.f;
             }
             __nv_bfloat16* dst = is_a ? Abf : s.P;
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-                *reinterpret_cast<uint4*>(dst + swz<C>(r, 8 * j)) =
+            for (int j = 0; j < 4; ++j)
+                *reinterpret_cast<uint4*>(dst + swz<C>(r, c0 + 8 * j)) =
                     make_uint4(pack_bf16(v[8 * j], v[8 * j + 1]), pack_bf16(v[8 * j + 2], v[8 * j + 3]),
                                pack_bf16(v[8 * j + 4], v[8 * j + 5]), pack_bf16(v[8 * j + 6], v[8 * j + 7]));
-            if (is_a) {  // the row's diagonal 16x16 block of A, exact in fp32
+            if (is_a && (r >> 5) == hf) {  // the row's diagonal 16x16 block of A, exact in fp32
                 float* ad = &Ad[r >> 4][r & 15][0];
-                switch (r >> 4) {
-#define GDN_DIAG_BLOCK(B)                                          \
-                    case B:                                        \
-                        _Pragma("unroll") for (int c = 0; c < 16; ++c) ad[c] = v[16 * B + c]; \
-                        break;
-                    GDN_DIAG_BLOCK(0) GDN_DIAG_BLOCK(1) GDN_DIAG_BLOCK(2) GDN_DIAG_BLOCK(3)
-#undef GDN_DIAG_BLOCK
+                if (r & 16) {
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) ad[c] = v[16 + c];
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) ad[c] = v[c];
                 }
             }
         }
@@ -182,7 +183,7 @@ __global__ void __launch_bounds__(P5_THREADS, 3) tc5_prep_kernel(const __grid_co
         // ---- K~ = diag(e^{G_last - G}) K to the workspace (the walks' B of
         // the state update); K <- diag(beta e^G) K and V <- diag(beta) V in
         // place (the row scales of W and U~)
-        {
+        if (tid < 128) {  // threads 0..127: K rows; 128..255: V rows (below)
             const int r = tid >> 1, pn = tid & 1;
             const float e = s.beta[r] * __expf(s.G[r]), dec = __expf(s.G[C - 1] - s.G[r]);
             __nv_bfloat16* row = s.KQ + pn * KQ_PANEL + r * 64;
@@ -205,6 +206,8 @@ __global__ void __launch_bounds__(P5_THREADS, 3) tc5_prep_kernel(const __grid_co
                 *reinterpret_cast<uint4*>(row + 8 * j) = x;
                 *reinterpret_cast<uint4*>(kt + 8 * j) = y;
             }
+        } else {
+            const int r = (tid - 128) >> 1, pn = tid & 1;
             const float b = s.beta[r];
             __nv_bfloat16* vrow = s.V + pn * (C * 64) + r * 64;
 #pragma unroll
@@ -244,28 +247,32 @@ __global__ void __launch_bounds__(P5_THREADS, 3) tc5_prep_kernel(const __grid_co
     if (__syncthreads_or(!ok)) goto done;
     tc5::fence_after();
 
-    // ---- epilogue 2: thread t = key row t of W^T and value row t of U~^T -----
+    // ---- epilogue 2: warps 0..3 key rows of W^T, warps 4..7 value rows of U~^T
     {
         __nv_bfloat16* Wimg = s.KQ;             // Tma128, 16 KB
         __nv_bfloat16* Uimg = s.KQ + C * DK;    // Swz<64>, 128 rows x 64 tokens
-        const uint32_t trow = tm + ((uint32_t)(32 * warp) << 16);
+        const int ql = warp & 3, row = 32 * ql + lane;
+        const uint32_t trow = tm + ((uint32_t)(32 * ql) << 16);
         float x[32];
+        if (warp < 4) {
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            tc5::ld32(x, trow + 32 * half);
-            tc5::wait_ld();
+            for (int half = 0; half < 2; ++half) {
+                tc5::ld32(x, trow + 32 * half);
+                tc5::wait_ld();
 #pragma unroll
-            for (int t = 0; t < 32; ++t) Wimg[Tma128::off(32 * half + t, tid)] = __float2bfloat16_rn(x[t]);
-        }
+                for (int t = 0; t < 32; ++t) Wimg[Tma128::off(32 * half + t, row)] = __float2bfloat16_rn(x[t]);
+            }
+        } else {
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            tc5::ld32(x, trow + 64 + 32 * half);
-            tc5::wait_ld();
+            for (int half = 0; half < 2; ++half) {
+                tc5::ld32(x, trow + 64 + 32 * half);
+                tc5::wait_ld();
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-                *reinterpret_cast<uint4*>(Uimg + swz<C>(tid, 32 * half + 8 * j)) =
-                    make_uint4(pack_bf16(x[8 * j], x[8 * j + 1]), pack_bf16(x[8 * j + 2], x[8 * j + 3]),
-                               pack_bf16(x[8 * j + 4], x[8 * j + 5]), pack_bf16(x[8 * j + 6], x[8 * j + 7]));
+                for (int j = 0; j < 4; ++j)
+                    *reinterpret_cast<uint4*>(Uimg + swz<C>(row, 32 * half + 8 * j)) =
+                        make_uint4(pack_bf16(x[8 * j], x[8 * j + 1]), pack_bf16(x[8 * j + 2], x[8 * j + 3]),
+                                   pack_bf16(x[8 * j + 4], x[8 * j + 5]), pack_bf16(x[8 * j + 6], x[8 * j + 7]));
+            }
         }
     }
     fence_async_smem();
