@@ -70,7 +70,7 @@ struct alignas(1024) PkSmem {
     __nv_bfloat16 Bx[B_ELEMS];
     __nv_bfloat16 Kw[C * DK];  // Tma128: beta e^G .* K (MN-major A of W^T)
     __nv_bfloat16 V[C * DV];   // Tma128, scaled by beta in place
-    float htot[DK];            // G at row 31, per key
+    float btot[4][DK];         // per-block sums of g, per key
     float Gf[4][DK], Gl[4][DK];  // G at the first and the last row of each block
     float gl[DK];              // e^{G_last}
     float beta[C];
@@ -112,76 +112,100 @@ __global__ void __launch_bounds__(PK_THREADS, 2) tc5_prep_kda_kernel(const __gri
     if (tid < C) s.beta[tid] = tid < L ? p.beta[row0 + tid * rs] : 0.f;
     if (warp == 0) tc5::alloc(&s.tmem, PK_TCOLS);
 
-    // ---- per-key cumsum: thread (c, hf) holds key c of rows 32 hf .. +31 -----
-    const int c = tid & (DK - 1), hf = tid >> 7;
-    float G[32];
+    // ---- per-key cumsum: thread (key pair kp, block bq) holds keys 2 kp and
+    // 2 kp + 1 of the 16 rows of block bq (a warp: 32 key pairs of one block)
+    const int kp = tid & 63, bq = tid >> 6, c = 2 * kp, i0 = 16 * bq;
+    float G0[16], G1[16];
 #pragma unroll
-    for (int r = 0; r < 32; ++r) {
-        const int i = 32 * hf + r;
-        G[r] = i < L ? p.g[(row0 + (size_t)i * rs) * DK + c] : 0.f;  // rows past L add 0
+    for (int r = 0; r < 16; ++r) {
+        const int i = i0 + r;
+        float2 gv = make_float2(0.f, 0.f);  // rows past L add 0
+        if (i < L) gv = *reinterpret_cast<const float2*>(p.g + (row0 + (size_t)i * rs) * DK + c);
+        G0[r] = gv.x;
+        G1[r] = gv.y;
     }
 #pragma unroll
-    for (int r = 1; r < 32; ++r) G[r] += G[r - 1];
-    if (hf == 0) s.htot[c] = G[31];
+    for (int r = 1; r < 16; ++r) {
+        G0[r] += G0[r - 1];
+        G1[r] += G1[r - 1];
+    }
+    s.btot[bq][c] = G0[15];
+    s.btot[bq][c + 1] = G1[15];
     tc5::fence_before();
     __syncthreads();
     tc5::fence_after();
     const uint32_t tm = s.tmem;
-    if (hf == 1) {
-        const float off = s.htot[c];
+    {
+        float p0 = 0.f, p1 = 0.f;
+        for (int t = 0; t < bq; ++t) {
+            p0 += s.btot[t][c];
+            p1 += s.btot[t][c + 1];
+        }
 #pragma unroll
-        for (int r = 0; r < 32; ++r) G[r] += off;
-        s.gl[c] = __expf(G[31]);
+        for (int r = 0; r < 16; ++r) {
+            G0[r] += p0;
+            G1[r] += p1;
+        }
     }
-#pragma unroll
-    for (int blk = 0; blk < 2; ++blk) {
-        const int b = 2 * hf + blk;
-        s.Gf[b][c] = G[16 * blk];
-        s.Gl[b][c] = G[16 * blk + 15];
-        float sp = G[16 * blk] - G[16 * blk + 15];
+    s.Gf[bq][c] = G0[0];
+    s.Gf[bq][c + 1] = G1[0];
+    s.Gl[bq][c] = G0[15];
+    s.Gl[bq][c + 1] = G1[15];
+    if (bq == 3) {
+        s.gl[c] = __expf(G0[15]);
+        s.gl[c + 1] = __expf(G1[15]);
+    }
+    {
+        float sp = fmaxf(G0[0] - G0[15], G1[0] - G1[15]);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) sp = fmaxf(sp, __shfl_xor_sync(0xffffffffu, sp, o));
         // unsigned order of the float bits: negative spans and NaN compare above 80
-        if (lane == 0) atomicMax(&s.span[b], __float_as_uint(sp));
+        if (lane == 0) atomicMax(&s.span[bq], __float_as_uint(sp));
     }
     __syncthreads();
     if (__syncthreads_or(!mbar_wait(&s.bar_ld, 0, p.status))) goto done;
 
-    // ---- every operand from one pass over the tiles --------------------------
+    // ---- every operand from one pass over the tiles (bf16 pairs) ------------
     {
-        const float Glast = s.Gl[3][c];
+        auto ld2 = [](const __nv_bfloat16* t, uint32_t o) {
+            return unpack_bf16(*reinterpret_cast<const uint32_t*>(t + o));
+        };
+        auto st2 = [](__nv_bfloat16* t, uint32_t o, float x, float y) {
+            *reinterpret_cast<uint32_t*>(t + o) = pack_bf16(x, y);
+        };
+        const float Gf0 = G0[0], Gl0 = G0[15], Gf1 = G1[0], Gl1 = G1[15];
+        const float ef0 = __expf(Gf0), ef1 = __expf(Gf1);
+        const float ekt0 = __expf(s.Gl[3][c] - Gl0), ekt1 = __expf(s.Gl[3][c + 1] - Gl1);
+        const float esp0 = Gf0 - Gl0 <= 80.f ? __expf(Gf0 - Gl0) : 0.f;
+        const float esp1 = Gf1 - Gl1 <= 80.f ? __expf(Gf1 - Gl1) : 0.f;
+        float F0[4], F1[4];
+#pragma unroll
+        for (int I = 0; I < 4; ++I) {
+            F0[I] = I > bq ? __expf(s.Gf[I][c] - Gl0) : 0.f;
+            F1[I] = I > bq ? __expf(s.Gf[I][c + 1] - Gl1) : 0.f;
+        }
         __nv_bfloat16* qg = p.Qg + (size_t)cid * C * DK;
         __nv_bfloat16* kt = p.Kt + (size_t)cid * C * DK;
 #pragma unroll
-        for (int blk = 0; blk < 2; ++blk) {
-            const int b = 2 * hf + blk;
-            const float Gfb = G[16 * blk], Glb = G[16 * blk + 15];
-            const float ef = __expf(Gfb), ekt = __expf(Glast - Glb);
-            const float esp = Gfb - Glb <= 80.f ? __expf(Gfb - Glb) : 0.f;
-            float F[4];
+        for (int r = 0; r < 16; ++r) {
+            const int i = i0 + r;
+            const float el0 = __expf(G0[r] - Gf0), er0 = __expf(Gl0 - G0[r]);
+            const float el1 = __expf(G1[r] - Gf1), er1 = __expf(Gl1 - G1[r]);
+            const uint32_t ok_ = Kp<128>::off(i, c), oq = Kp<128>::off(C + i, c), ot = Tma128::off(i, c);
+            const float2 kv = ld2(s.KQ, ok_), qv = ld2(s.KQ, oq), vv = ld2(s.V, ot);
+            const float bi = s.beta[i];
+            st2(s.KQ, ok_, kv.x * el0, kv.y * el1);
+            st2(s.KQ, oq, qv.x * el0, qv.y * el1);
+            const float k0 = kv.x * er0, k1 = kv.y * er1;
+            st2(s.Bx, b_off(bq, i, c), k0 * esp0, k1 * esp1);
 #pragma unroll
-            for (int I = 0; I < 4; ++I) F[I] = I > b ? __expf(s.Gf[I][c] - Glb) : 0.f;
-#pragma unroll
-            for (int r = 0; r < 16; ++r) {
-                const int i = 16 * b + r;
-                const float gi = G[16 * blk + r];
-                const float el = __expf(gi - Gfb), er = __expf(Glb - gi);
-                const uint32_t ok_ = Kp<128>::off(i, c), oq = Kp<128>::off(C + i, c), ot = Tma128::off(i, c);
-                const float kv = __bfloat162float(s.KQ[ok_]), qv = __bfloat162float(s.KQ[oq]);
-                const float bi = s.beta[i];
-                s.KQ[ok_] = __float2bfloat16_rn(kv * el);
-                s.KQ[oq] = __float2bfloat16_rn(qv * el);
-                const float ker = kv * er;
-                s.Bx[b_off(b, i, c)] = __float2bfloat16_rn(ker * esp);
-#pragma unroll
-                for (int I = 1; I < 4; ++I)
-                    if (I > b) s.Bx[b_off(I, i, c)] = __float2bfloat16_rn(ker * F[I]);
-                const float eg = el * ef;  // e^{G_i}
-                s.Kw[ot] = __float2bfloat16_rn(kv * bi * eg);
-                s.V[ot] = __float2bfloat16_rn(__bfloat162float(s.V[ot]) * bi);
-                qg[ot] = __float2bfloat16_rn(p.scale * qv * eg);
-                kt[ot] = __float2bfloat16_rn(ker * ekt);
-            }
+            for (int I = 1; I < 4; ++I)
+                if (I > bq) st2(s.Bx, b_off(I, i, c), k0 * F0[I], k1 * F1[I]);
+            const float eg0 = el0 * ef0, eg1 = el1 * ef1;  // e^{G_i}
+            st2(s.Kw, ot, kv.x * bi * eg0, kv.y * bi * eg1);
+            st2(s.V, ot, vv.x * bi, vv.y * bi);
+            st2(qg, ot, p.scale * qv.x * eg0, p.scale * qv.y * eg1);
+            st2(kt, ot, k0 * ekt0, k1 * ekt1);
         }
     }
     fence_async_smem();  // generic writes -> tensor-core reads
