@@ -530,7 +530,35 @@ def run_ours(args, rank, world, dev, barrier, max_over_ranks):
             "bwd_us": round(ms_pb * 1e3, 1), "bwd_bytes": pb_bytes,
             "bwd_hbm_gbs": round(pb_bytes / (ms_pb / 1e3) / 1e9, 1),
             "bwd_frac_hbm_peak": round(pb_bytes / (ms_pb / 1e3) / 1e9 / pk["hbm"], 4)}
-        del pr, py, pws
+        # ---- the layer's training step from the raw projections: the prologue
+        # fused into the chunk preparation, against the prologue as separate passes
+        xs = {n: pr[n]["x"] for n in "qkv"}
+        ws_ = {n: pr[n]["w"] for n in "qkv"}
+        cws = [None]
+
+        def fused_step():
+            _, _, cws[0] = gdn.gdn_chunk_fwd_save_conv(xs["q"], xs["k"], xs["v"], ws_["q"], ws_["k"],
+                                                       ws_["v"], d["g"], d["beta"], d["h0"],
+                                                       o=outs["o"], hT=outs["hT"], workspace=cws[0])
+            gdn.gdn_chunk_bwd_saved_conv(xs["q"], xs["k"], xs["v"], ws_["q"], ws_["k"], ws_["v"],
+                                         d["g"], d["beta"], d["dO"], cws[0], d["h0"], d["dhT"])
+
+        def unfused_step():
+            f = {n: gdn.gdn_short_conv_fwd(xs[n], ws_[n], l2norm=n != "v", y=py[n]) for n in "qkv"}
+            gdn.gdn_chunk_fwd_save(f["q"], f["k"], f["v"], d["g"], d["beta"], d["h0"],
+                                   o=outs["o"], hT=outs["hT"], workspace=ws_b)
+            r = gdn.gdn_chunk_bwd_saved(f["q"], f["k"], f["v"], d["g"], d["beta"], d["dO"], ws_b,
+                                        d["h0"], d["dhT"])
+            for n in "qkv":
+                gdn.gdn_short_conv_bwd(xs[n], ws_[n], r["d" + n], l2norm=n != "v", workspace=pws)
+        ms_fu = timed(fused_step, max(args.steps // 2, 5), args.warmup, barrier)
+        ms_un = timed(unfused_step, max(args.steps // 2, 5), args.warmup, barrier)
+        extra["prologue_fused_step"] = {
+            "workload": f"{cfg.name} from raw q/k/v projections, K = 4 taps, fwd+bwd",
+            "fused_ms": round(ms_fu, 4), "separate_passes_ms": round(ms_un, 4),
+            "tokens_per_s": round(cfg.B * cfg.T / (ms_fu / 1e3), 1),
+            "kernels": kernel_breakdown(gdn, fused_step, 3)}
+        del pr, py, pws, cws
 
     # ---- end to end through host buffers ------------------------------------
     names_in = ("q", "k", "v", "g", "beta", "dO")

@@ -26,7 +26,8 @@ GDN_GATE_SCALAR, GDN_GATE_CHANNEL = 0, 1
 
 # Every symbol include/gdn.h declares.
 EXPORTS = ("gdn_chunk_fwd_workspace", "gdn_chunk_fwd", "gdn_chunk_bwd_workspace",
-           "gdn_chunk_bwd", "gdn_chunk_fwd_save", "gdn_chunk_bwd_saved", "gdn_recurrent_step", "gdn_query_device_status",
+           "gdn_chunk_bwd", "gdn_chunk_fwd_save", "gdn_chunk_bwd_saved",
+           "gdn_chunk_conv_saved_workspace", "gdn_chunk_fwd_save_conv", "gdn_chunk_bwd_saved_conv", "gdn_recurrent_step", "gdn_query_device_status",
            "gdn_status_string", "gdn_profile_begin", "gdn_profile_end",
            "gdn_chunk_fwd_noalloc", "gdn_noalloc_device_status", "gdn_test_stalled_fwd", "gdn_product_fwd_workspace", "gdn_product_fwd",
            "gdn_product_bwd_workspace", "gdn_product_bwd", "gdn_chunk_fwd_varlen_workspace",
@@ -77,6 +78,14 @@ def lib() -> ctypes.CDLL:
             L.gdn_chunk_fwd_save.restype = i
             L.gdn_chunk_bwd_saved.argtypes = L.gdn_chunk_bwd.argtypes
             L.gdn_chunk_bwd_saved.restype = i
+            L.gdn_chunk_conv_saved_workspace.argtypes = [dp, i]
+            L.gdn_chunk_conv_saved_workspace.restype = sz
+            L.gdn_chunk_fwd_save_conv.argtypes = [dp, i, vp, vp, vp, fp, fp, fp, fp, fp, fp, vp, fp,
+                                                  vp, sz, vp]
+            L.gdn_chunk_fwd_save_conv.restype = i
+            L.gdn_chunk_bwd_saved_conv.argtypes = [dp, i, vp, vp, vp, fp, fp, fp, fp, fp, fp, vp, fp,
+                                                   vp, vp, vp, fp, fp, fp, fp, fp, fp, vp, sz, vp]
+            L.gdn_chunk_bwd_saved_conv.restype = i
             L.gdn_recurrent_step.argtypes = [i, i, i, i, i, i, f, vp, vp, vp, fp, fp, fp,
                                              vp, vp]
             L.gdn_recurrent_step.restype = i
@@ -308,6 +317,62 @@ def gdn_chunk_bwd_saved(q, k, v, g, beta, dO, workspace, h0=None, dhT=None, *, c
                                    0 if workspace is None else workspace.numel() * workspace.element_size(),
                                    _stream(stream))
     _check(st, "gdn_chunk_bwd_saved")
+    return out
+
+
+def _validate_conv_chunk(xq, xk, xv, wq, wk, wv, g, beta, h0):
+    import torch
+    B, T, H, dk, dv = _validate_chunk_inputs(xq, xk, xv, g, beta, h0)
+    K = wq.shape[-1] if wq.dim() == 3 else 0
+    for w, name, d in ((wq, "wq", dk), (wk, "wk", dk), (wv, "wv", dv)):
+        _need(w, name, torch.float32, (H, d, K))
+    return B, T, H, dk, dv, K
+
+
+def gdn_chunk_fwd_save_conv(xq, xk, xv, wq, wk, wv, g, beta, h0=None, *, chunk=64, scale=1.0,
+                            output_final_state=True, o=None, hT=None, workspace=None, stream=None):
+    """Forward of a training step from the raw projections: the short
+    convolution, SiLU and (q, k) L2 norm, then the gated delta rule.  Returns
+    (o, hT, workspace); pass the workspace to gdn_chunk_bwd_saved_conv."""
+    import torch
+    B, T, H, dk, dv, K = _validate_conv_chunk(xq, xk, xv, wq, wk, wv, g, beta, h0)
+    dims = make_dims(xq, xv, g, chunk, scale)
+    if o is None:
+        o = torch.empty(B, T, H, dv, dtype=xq.dtype, device=xq.device)
+    if output_final_state and hT is None:
+        hT = torch.empty(B, H, dv, dk, dtype=torch.float32, device=xq.device)
+    nbytes = int(lib().gdn_chunk_conv_saved_workspace(ctypes.byref(dims), K))
+    ws = _workspace(nbytes, xq.device, workspace)
+    st = lib().gdn_chunk_fwd_save_conv(ctypes.byref(dims), K, _ptr(xq), _ptr(xk), _ptr(xv),
+                                       _ptr(wq), _ptr(wk), _ptr(wv), _ptr(g), _ptr(beta), _ptr(h0),
+                                       _ptr(o), _ptr(hT), _ptr(ws),
+                                       0 if ws is None else ws.numel() * ws.element_size(),
+                                       _stream(stream))
+    _check(st, "gdn_chunk_fwd_save_conv")
+    return o, hT, ws
+
+
+def gdn_chunk_bwd_saved_conv(xq, xk, xv, wq, wk, wv, g, beta, dO, workspace, h0=None, dhT=None,
+                             *, chunk=64, scale=1.0, stream=None):
+    """Backward from gdn_chunk_fwd_save_conv's workspace.  Returns a dict with
+    dxq, dxk, dxv, dwq, dwk, dwv, dg, dbeta, dh0."""
+    import torch
+    B, T, H, dk, dv, K = _validate_conv_chunk(xq, xk, xv, wq, wk, wv, g, beta, h0)
+    _need(dO, "dO", xq.dtype, (B, T, H, dv))
+    if dhT is not None:
+        _need(dhT, "dhT", torch.float32, (B, H, dv, dk))
+    dims = make_dims(xq, xv, g, chunk, scale)
+    out = dict(dxq=torch.empty_like(xq), dxk=torch.empty_like(xk), dxv=torch.empty_like(xv),
+               dwq=torch.empty_like(wq), dwk=torch.empty_like(wk), dwv=torch.empty_like(wv),
+               dg=torch.empty_like(g), dbeta=torch.empty_like(beta),
+               dh0=None if h0 is None else torch.empty_like(h0))
+    st = lib().gdn_chunk_bwd_saved_conv(
+        ctypes.byref(dims), K, _ptr(xq), _ptr(xk), _ptr(xv), _ptr(wq), _ptr(wk), _ptr(wv), _ptr(g),
+        _ptr(beta), _ptr(h0), _ptr(dO), _ptr(dhT), _ptr(out["dxq"]), _ptr(out["dxk"]),
+        _ptr(out["dxv"]), _ptr(out["dwq"]), _ptr(out["dwk"]), _ptr(out["dwv"]), _ptr(out["dg"]),
+        _ptr(out["dbeta"]), _ptr(out["dh0"]), _ptr(workspace),
+        0 if workspace is None else workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "gdn_chunk_bwd_saved_conv")
     return out
 
 

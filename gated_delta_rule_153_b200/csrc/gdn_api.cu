@@ -71,6 +71,25 @@ gdn_status validate_fwd_args(const gdn_dims* d, const void* q, const void* k, co
     if (h0 && hT && h0 == hT) return GDN_ERR_INVALID_ARG;
     return GDN_OK;
 }
+
+ConvLayout conv_layout(const gdn_dims& d, int K, size_t base) {
+    auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    const size_t es = d.dtype == GDN_BF16 ? 2 : 4;
+    const size_t tq = al((size_t)d.B * d.T * d.H * d.dk * es), tv = al((size_t)d.B * d.T * d.H * d.dv * es);
+    ConvLayout c{};
+    size_t o = al(base);
+    c.qf = o; o += tq;
+    c.kf = o; o += tq;
+    c.vf = o; o += tv;
+    c.dqf = o; o += tq;
+    c.dkf = o; o += tq;
+    c.dvf = o; o += tv;
+    c.cws = o;
+    o += al(std::max(gdn_short_conv_bwd_workspace(d.B, d.T, d.H, d.dk, K),
+                     gdn_short_conv_bwd_workspace(d.B, d.T, d.H, d.dv, K)));
+    c.end = o;
+    return c;
+}
 }  // namespace gdn
 
 extern "C" {
@@ -196,6 +215,83 @@ gdn_status gdn_chunk_bwd_saved(const gdn_dims* d, const void* q, const void* k, 
     } else
         launch_simt_bwd(*d, q, k, v, g, beta, h0, dO, dhT, dq, dk, dv, dg, dbeta, dh0, ws, st);
     return launch_status();
+}
+
+static size_t saved_base(const gdn_dims* d) {
+    return std::max(gdn_chunk_bwd_workspace(d), gdn_chunk_fwd_workspace(d));
+}
+
+size_t gdn_chunk_conv_saved_workspace(const gdn_dims* d, int K) {
+    if (check_dims(d) != GDN_OK || K < 1 || K > 4) return 0;
+    return conv_layout(*d, K, saved_base(d)).end;
+}
+
+gdn_status gdn_chunk_fwd_save_conv(const gdn_dims* d, int K, const void* xq, const void* xk,
+                                   const void* xv, const float* wq, const float* wk, const float* wv,
+                                   const float* g, const float* beta, const float* h0, void* o,
+                                   float* hT, void* ws, size_t ws_bytes, gdn_stream_t stream) {
+    gdn_status s = validate_fwd_args(d, xq, xk, xv, g, beta, h0, o, hT);
+    if (s != GDN_OK) return s;
+    if (K < 1 || K > 4 || !wq || !wk || !wv) return GDN_ERR_INVALID_ARG;
+    if (!all_aligned({wq, wk, wv})) return GDN_ERR_INVALID_ARG;
+    const size_t need = gdn_chunk_conv_saved_workspace(d, K);
+    if (!ws || ws_bytes < need) return GDN_ERR_WORKSPACE;
+    if ((uintptr_t)ws & 255u) return GDN_ERR_WORKSPACE;
+    const ConvLayout CL = conv_layout(*d, K, saved_base(d));
+    char* base = (char*)ws;
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaGetLastError();
+    if (tc_supported(*d) && d->gate == GDN_GATE_SCALAR) {  // the prologue fused into the preparation
+        if (cudaMemsetAsync(ws, 0, sizeof(unsigned int), st) != cudaSuccess) return GDN_ERR_CUDA;
+        if (!launch_tc_fwd_save_conv(*d, K, xq, xk, xv, wq, wk, wv, g, beta, h0, o, hT, ws, st))
+            return GDN_ERR_CUDA;
+        return launch_status();
+    }
+    // other shapes: the prologue as its own pass, then the saving forward
+    const int B = d->B, T = d->T, H = d->H;
+    if ((s = gdn_short_conv_fwd(B, T, H, d->dk, K, d->dtype, 1, xq, wq, base + CL.qf, stream)) != GDN_OK ||
+        (s = gdn_short_conv_fwd(B, T, H, d->dk, K, d->dtype, 1, xk, wk, base + CL.kf, stream)) != GDN_OK ||
+        (s = gdn_short_conv_fwd(B, T, H, d->dv, K, d->dtype, 0, xv, wv, base + CL.vf, stream)) != GDN_OK)
+        return s;
+    return gdn_chunk_fwd_save(d, base + CL.qf, base + CL.kf, base + CL.vf, g, beta, h0, o, hT, ws,
+                              saved_base(d), stream);
+}
+
+gdn_status gdn_chunk_bwd_saved_conv(const gdn_dims* d, int K, const void* xq, const void* xk,
+                                    const void* xv, const float* wq, const float* wk, const float* wv,
+                                    const float* g, const float* beta, const float* h0, const void* dO,
+                                    const float* dhT, void* dxq, void* dxk, void* dxv, float* dwq,
+                                    float* dwk, float* dwv, float* dg, float* dbeta, float* dh0,
+                                    void* ws, size_t ws_bytes, gdn_stream_t stream) {
+    gdn_status s = check_dims(d);
+    if (s != GDN_OK) return s;
+    if (K < 1 || K > 4) return GDN_ERR_INVALID_ARG;
+    if (!xq || !xk || !xv || !wq || !wk || !wv || !dxq || !dxk || !dxv || !dwq || !dwk || !dwv)
+        return GDN_ERR_INVALID_ARG;
+    if (!all_aligned({xq, xk, xv, wq, wk, wv, dxq, dxk, dxv, dwq, dwk, dwv}))
+        return GDN_ERR_INVALID_ARG;
+    const size_t need = gdn_chunk_conv_saved_workspace(d, K);
+    if (!ws || ws_bytes < need) return GDN_ERR_WORKSPACE;
+    if ((uintptr_t)ws & 255u) return GDN_ERR_WORKSPACE;
+    const ConvLayout CL = conv_layout(*d, K, saved_base(d));
+    char* base = (char*)ws;
+    // the chunk backward for the filtered q, k, v kept by the forward ...
+    s = gdn_chunk_bwd_saved(d, base + CL.qf, base + CL.kf, base + CL.vf, g, beta, h0, dO, dhT,
+                            base + CL.dqf, base + CL.dkf, base + CL.dvf, dg, dbeta, dh0, ws,
+                            saved_base(d), stream);
+    if (s != GDN_OK) return s;
+    // ... then the prologue's backward from their gradients
+    const int B = d->B, T = d->T, H = d->H;
+    void* cws = base + CL.cws;
+    const size_t cb = CL.end - CL.cws;
+    if ((s = gdn_short_conv_bwd(B, T, H, d->dk, K, d->dtype, 1, xq, wq, base + CL.dqf, dxq, dwq, cws, cb,
+                                stream)) != GDN_OK ||
+        (s = gdn_short_conv_bwd(B, T, H, d->dk, K, d->dtype, 1, xk, wk, base + CL.dkf, dxk, dwk, cws, cb,
+                                stream)) != GDN_OK ||
+        (s = gdn_short_conv_bwd(B, T, H, d->dv, K, d->dtype, 0, xv, wv, base + CL.dvf, dxv, dwv, cws, cb,
+                                stream)) != GDN_OK)
+        return s;
+    return GDN_OK;
 }
 
 gdn_status gdn_recurrent_step(int N, int H, int dk, int dv, gdn_dtype dtype, gdn_gate gate,

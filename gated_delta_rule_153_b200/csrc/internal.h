@@ -50,6 +50,18 @@ bool launch_tc_fwd(const gdn_dims& d, const void* q, const void* k, const void* 
 bool launch_tc_fwd_save(const gdn_dims& d, const void* q, const void* k, const void* v,
                         const float* g, const float* beta, const float* h0, void* o, float* hT,
                         void* ws, cudaStream_t st);
+// The training pair with the q/k/v prologue (gdn_chunk_fwd_save_conv): after
+// the `base` bytes of the saved chunk workspace come the filtered q, k, v,
+// their gradients, and the prologue backward's workspace.
+struct ConvLayout {
+    size_t qf, kf, vf, dqf, dkf, dvf, cws, end;
+};
+ConvLayout conv_layout(const gdn_dims& d, int K, size_t base);
+// The fused forward (scalar gate on the tensor-core shapes).
+bool launch_tc_fwd_save_conv(const gdn_dims& d, int K, const void* xq, const void* xk, const void* xv,
+                             const float* wq, const float* wk, const float* wv, const float* g,
+                             const float* beta, const float* h0, void* o, float* hT, void* ws,
+                             cudaStream_t st);
 // True when the forward of these dims runs its chain on the tcgen05 whole-head walk.
 bool tc_fwd_whole_head(const gdn_dims& d);
 bool launch_tc_bwd(const gdn_dims& d, const void* q, const void* k, const void* v,

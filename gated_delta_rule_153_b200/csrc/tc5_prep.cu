@@ -64,6 +64,75 @@ struct alignas(1024) P5Smem {
     uint32_t tmem;
 };
 
+// The q/k/v prologue of the block design ("Gated Delta Networks: Improving
+// Mamba2 with Delta Rule" (paper review), section "Method": a short causal
+// depthwise convolution, SiLU, and for q and k an L2 norm over the head's
+// channels), applied in place to a raw 64-token tile in shared memory:
+//   z_t[c] = sum_{j<K} w[h, c, j] x_{t-j}[c],  s = z sigmoid(z),
+//   y = s / sqrt(sum_c s_c^2 + 1e-6)  (norm), else y = s.
+// The tile's own raw rows give the history of its rows 3..63; the `halo`
+// rows before the chunk (0 at a sequence's first chunk) come from x.  Thread
+// (row, 8-channel group); the norm's sum is a 16-lane reduction.  All rows'
+// raw values are read before any is overwritten (results wait in registers
+// as bf16 pairs).  Rows below L also go to `out`.
+template <typename Off>
+GDN_DEV void conv_tile(__nv_bfloat16* tile, Off off, const __nv_bfloat16* x, __nv_bfloat16* out,
+                       const float* w, int K, bool norm, int h, size_t row0, size_t rs, int L,
+                       int halo) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int c0 = 8 * (lane & 15);
+    float wr[8][4];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) wr[i][j] = j < K ? w[((size_t)h * DK + c0 + i) * K + j] : 0.f;
+    uint4 res[4];
+#pragma unroll
+    for (int ps = 0; ps < 4; ++ps) {
+        const int r = 16 * ps + 2 * warp + (lane >> 4);
+        float z[8] = {};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            if (j >= K) break;
+            const int rr = r - j;  // tile row of tap j
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (rr >= 0) v = *reinterpret_cast<const uint4*>(tile + off(rr, c0));
+            else if (-rr <= halo)
+                v = *reinterpret_cast<const uint4*>(x + (row0 - (size_t)(-rr) * rs) * DK + c0);
+            const uint32_t e[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float2 f = unpack_bf16(e[i]);
+                z[2 * i] = fmaf(wr[2 * i][j], f.x, z[2 * i]);
+                z[2 * i + 1] = fmaf(wr[2 * i + 1][j], f.y, z[2 * i + 1]);
+            }
+        }
+        float ss = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            z[i] = __fdividef(z[i], 1.f + __expf(-z[i]));
+            ss += z[i] * z[i];
+        }
+        if (norm) {
+#pragma unroll
+            for (int o = 8; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+            const float inv = rsqrtf(ss + 1e-6f);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) z[i] *= inv;
+        }
+        res[ps] = make_uint4(pack_bf16(z[0], z[1]), pack_bf16(z[2], z[3]), pack_bf16(z[4], z[5]),
+                             pack_bf16(z[6], z[7]));
+    }
+    __syncthreads();  // every raw row read
+#pragma unroll
+    for (int ps = 0; ps < 4; ++ps) {
+        const int r = 16 * ps + 2 * warp + (lane >> 4);
+        *reinterpret_cast<uint4*>(tile + off(r, c0)) = res[ps];
+        if (r < L) *reinterpret_cast<uint4*>(out + (row0 + (size_t)r * rs) * DK + c0) = res[ps];
+    }
+}
+
+template <bool CONV>
 __global__ void __launch_bounds__(P5_THREADS, 3) tc5_prep_kernel(const __grid_constant__ ChunkPtrs p) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     P5Smem& s = *reinterpret_cast<P5Smem*>(align1k(smem_raw));
@@ -113,10 +182,25 @@ __global__ void __launch_bounds__(P5_THREADS, 3) tc5_prep_kernel(const __grid_co
     const uint32_t sKQ = smem_u32(s.KQ);
     bool ok = true;
 
+    if constexpr (CONV) {  // the tiles are raw projections: filter them in place
+        ok = mbar_wait(&s.bar_ld, 0, p.status);
+        if (__syncthreads_or(!ok)) goto done;
+        const int halo = n > 0 ? 3 : 0;  // a dense batch: one sequence per row b
+        conv_tile(s.KQ, [](int r, int c) { return (c >> 6) * KQ_PANEL + swz<64>(r, c & 63); }, p.conv.xk,
+                  p.conv.kf, p.conv.wk, p.conv.K, true, h, row0, rs, L, halo);
+        conv_tile(s.KQ, [](int r, int c) { return (c >> 6) * KQ_PANEL + swz<64>(C + r, c & 63); }, p.conv.xq,
+                  p.conv.qf, p.conv.wq, p.conv.K, true, h, row0, rs, L, halo);
+        conv_tile(s.V, [](int r, int c) { return (c >> 6) * (C * 64) + swz<64>(r, c & 63); }, p.conv.xv,
+                  p.conv.vf, p.conv.wv, p.conv.K, false, h, row0, rs, L, halo);
+        fence_async_smem();  // filtered tiles (generic writes) -> tensor-core reads
+        tc5::fence_before();
+        __syncthreads();
+    }
     // ---- [K K^T ; Q K^T] ---------------------------------------------------
     if (tid == 0) {
-        ok = mbar_wait(&s.bar_ld, 0, p.status);
+        if (!CONV) ok = mbar_wait(&s.bar_ld, 0, p.status);
         if (ok) {
+            tc5::fence_after();
 #pragma unroll
             for (int kk = 0; kk < DK / 16; ++kk)
                 tc5::mma(tm, tc5::kmajor<2 * C>(sKQ, kk), tc5::kmajor<2 * C>(sKQ, kk), ID_KQ, kk > 0);
@@ -300,8 +384,15 @@ done:
 namespace tc {
 void launch_prep5(const ChunkPtrs& p, size_t nchunks, cudaStream_t st) {
     const int smem = sizeof(P5Smem) + 1024;
-    cudaFuncSetAttribute(tc5_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    GDN_LAUNCH("tc5_prep", st, tc5_prep_kernel<<<(unsigned)nchunks, P5_THREADS, smem, st>>>(p));
+    cudaFuncSetAttribute(tc5_prep_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    GDN_LAUNCH("tc5_prep", st, tc5_prep_kernel<false><<<(unsigned)nchunks, P5_THREADS, smem, st>>>(p));
+}
+// The preparation with the q/k/v prologue fused into its load stage (p.conv set,
+// the token maps over the raw projections).
+void launch_prep5_conv(const ChunkPtrs& p, size_t nchunks, cudaStream_t st) {
+    const int smem = sizeof(P5Smem) + 1024;
+    cudaFuncSetAttribute(tc5_prep_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    GDN_LAUNCH("tc5_prep_conv", st, tc5_prep_kernel<true><<<(unsigned)nchunks, P5_THREADS, smem, st>>>(p));
 }
 }  // namespace tc
 }  // namespace gdn

@@ -31,6 +31,7 @@ namespace gdn {
 namespace tc {
 void launch_prep5_kda(const ChunkPtrs& p, size_t nchunks, cudaStream_t st);
 void launch_prep5(const ChunkPtrs& p, size_t nchunks, cudaStream_t st);
+void launch_prep5_conv(const ChunkPtrs& p, size_t nchunks, cudaStream_t st);
 void launch_walk5_fwd(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& c, const float* h0,
                       void* o, float* hT, void* ws, cudaStream_t st, bool save = false);
 void launch_walk5_states(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& c, const float* h0,
@@ -490,6 +491,40 @@ bool launch_tc_fwd_save(const gdn_dims& d, const void* q, const void* k, const v
         if (kda) launch_walk<0, true>(w, st);
         else launch_walk<0, false>(w, st);
         launch_walk_states(d, L, cp, h0, ws, st);
+    }
+    return true;
+}
+
+// The training-step forward with the q/k/v prologue fused into the
+// preparation's load stage: the preparation reads the raw projections,
+// filters its tiles in shared memory and writes the filtered q, k, v to the
+// workspace, where the walk (and later the backward) read them.
+bool launch_tc_fwd_save_conv(const gdn_dims& d, int K, const void* xq, const void* xk, const void* xv,
+                             const float* wq, const float* wk, const float* wv, const float* g,
+                             const float* beta, const float* h0, void* o, float* hT, void* ws,
+                             cudaStream_t st) {
+    const TcLayout L = tc_layout(d, true);
+    const ConvLayout CL = conv_layout(d, K, L.end);
+    char* base = (char*)ws;
+    __nv_bfloat16 *qf = (__nv_bfloat16*)(base + CL.qf), *kf = (__nv_bfloat16*)(base + CL.kf),
+                  *vf = (__nv_bfloat16*)(base + CL.vf);
+    ChunkPtrs cp;  // token maps over the raw projections
+    if (!make_chunk_ptrs(cp, d, L, xq, xk, xv, g, beta, ws)) return false;
+    cp.Tb = (__nv_bfloat16*)(base + L.Tb);
+    cp.conv = ChunkPtrs::Conv{(const __nv_bfloat16*)xq, (const __nv_bfloat16*)xk, (const __nv_bfloat16*)xv,
+                              wq, wk, wv, qf, kf, vf, K};
+    launch_prep5_conv(cp, L.nchunks, st);
+    ChunkPtrs cw;  // token maps over the filtered tensors
+    if (!make_chunk_ptrs(cw, d, L, qf, kf, vf, g, beta, ws)) return false;
+    cw.Tb = cp.Tb;
+    if (tc::whole_head_fwd(d, L, cw.seq)) {
+        launch_walk5_fwd(d, L, cw, h0, o, hT, ws, st, true);
+    } else {
+        WalkPtrs w = make_walk_ptrs(d, L, cw, h0);
+        w.o = (__nv_bfloat16*)o;
+        w.hT = hT;
+        launch_walk<0, false>(w, st);
+        launch_walk_states(d, L, cw, h0, ws, st);
     }
     return true;
 }

@@ -174,6 +174,16 @@ struct ChunkPtrs {
     // bounded waits of the tcgen05 forward walks (see tc5_walk.cu)
     unsigned long long wait_ns = kWaitNs;
     int stall_at = -1;
+    // The q/k/v prologue fused into the preparation's load stage: the token
+    // maps above then cover the raw projections, whose rows before a chunk
+    // (the filter's history) are read from xq, xk, xv; the filtered tensors
+    // ([B, T, H, 128] bf16) go to qf, kf, vf for the later kernels.
+    struct Conv {
+        const __nv_bfloat16 *xq, *xk, *xv;
+        const float *wq, *wk, *wv;  // [H, 128, K] filters
+        __nv_bfloat16 *qf, *kf, *vf;
+        int K;
+    } conv{};
 };
 
 // Stage the W and U~ images from a warp's 16-row block of the W = T diag(.) K

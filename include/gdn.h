@@ -139,6 +139,41 @@ gdn_status gdn_chunk_bwd_saved(const gdn_dims *dims, const void *q, const void *
                                float *dh0, void *ws, size_t ws_bytes,
                                gdn_stream_t stream);
 
+/* The training pair with the block's q/k/v prologue ("Gated Delta Networks:
+ * Improving Mamba2 with Delta Rule" (paper review), section "Method": q and k
+ * pass through a short convolution, SiLU and L2 normalisation, v through the
+ * convolution and SiLU; gdn_short_conv_fwd below defines the filter).  The
+ * forward takes the raw projections xq, xk [B,T,H,dk] and xv [B,T,H,dv] (the
+ * dtype of dims) and the filters wq, wk [H,dk,K], wv [H,dv,K] fp32 (1 <= K <=
+ * 4), and returns o and hT of gdn_chunk_fwd applied to the filtered q, k, v;
+ * the backward returns the gradients of <dO, o> + <dhT, hT> with respect to
+ * xq, xk, xv (dtype of dims), wq, wk, wv (fp32, overwritten), g, beta and h0.
+ * On the tensor-core shapes with the scalar gate the filter runs inside the
+ * chunk preparation's load stage: it reads the raw tiles (and the 3 tokens
+ * before each chunk), filters them in shared memory and writes the filtered
+ * q, k, v once for the later kernels; elsewhere the prologue runs as its own
+ * pass.  Both calls take the same caller-owned workspace of
+ * gdn_chunk_conv_saved_workspace(dims, K) bytes (256-byte aligned), which
+ * keeps the filtered tensors, the chunk products and the chunk states between
+ * them; inputs must stay unchanged from the forward until the backward has
+ * run.  The batch is dims->B sequences of dims->T tokens (the filter sees
+ * zeros before each sequence's first token). */
+size_t gdn_chunk_conv_saved_workspace(const gdn_dims *dims, int K);
+gdn_status gdn_chunk_fwd_save_conv(const gdn_dims *dims, int K, const void *xq,
+                                   const void *xk, const void *xv, const float *wq,
+                                   const float *wk, const float *wv, const float *g,
+                                   const float *beta, const float *h0, void *o,
+                                   float *hT, void *ws, size_t ws_bytes,
+                                   gdn_stream_t stream);
+gdn_status gdn_chunk_bwd_saved_conv(const gdn_dims *dims, int K, const void *xq,
+                                    const void *xk, const void *xv, const float *wq,
+                                    const float *wk, const float *wv, const float *g,
+                                    const float *beta, const float *h0, const void *dO,
+                                    const float *dhT, void *dxq, void *dxk, void *dxv,
+                                    float *dwq, float *dwk, float *dwv, float *dg,
+                                    float *dbeta, float *dh0, void *ws, size_t ws_bytes,
+                                    gdn_stream_t stream);
+
 /* Packed variable-length batches.  Each sequence of a packed batch is its own
  * instance of the recurrence of "Gated Delta Networks: Improving Mamba2 with
  * Delta Rule" (paper review), section "Method": its state starts from its

@@ -241,3 +241,22 @@ def test_stalled_fwd_hook_checks():
     assert call(wide, 2, 2_000_000_000) == gdn.GDN_ERR_INVALID_ARG
     assert call(narrow, 2, 1000) == gdn.GDN_ERR_UNSUPPORTED
     assert call(f32, 2, 1000) == gdn.GDN_ERR_UNSUPPORTED
+
+
+def test_training_pair_bindings_reject_host_tensors():
+    """The training-pair bindings run their argument checks before any device
+    work: host tensors are refused with TypeError."""
+    import torch
+    import gated_delta_rule_153_b200 as gdn
+    B, T, H, d, K = 1, 8, 2, 128, 4
+    x = torch.zeros(B, T, H, d, dtype=torch.bfloat16)
+    w = torch.zeros(H, d, K)
+    g, beta = torch.zeros(B, T, H), torch.zeros(B, T, H)
+    with pytest.raises(TypeError):
+        gdn.gdn_chunk_fwd_save(x, x, x, g, beta)
+    with pytest.raises(TypeError):
+        gdn.gdn_chunk_bwd_saved(x, x, x, g, beta, x, None)
+    with pytest.raises(TypeError):
+        gdn.gdn_chunk_fwd_save_conv(x, x, x, w, w, w, g, beta)
+    with pytest.raises(TypeError):
+        gdn.gdn_chunk_bwd_saved_conv(x, x, x, w, w, w, g, beta, x, None)
