@@ -70,23 +70,26 @@ struct alignas(1024) P5Smem {
 // channels), applied in place to a raw 64-token tile in shared memory:
 //   z_t[c] = sum_{j<K} w[h, c, j] x_{t-j}[c],  s = z sigmoid(z),
 //   y = s / sqrt(sum_c s_c^2 + 1e-6)  (norm), else y = s.
-// The tile's own raw rows give the history of its rows 3..63; the `halo`
-// rows before the chunk (0 at a sequence's first chunk) come from x.  Thread
-// (row, 8-channel group); the norm's sum is a 16-lane reduction.  All rows'
-// raw values are read before any is overwritten (results wait in registers
-// as bf16 pairs).  Rows below L also go to `out`.
+// The tile's own raw rows give the history of its rows 3..63; the 3 rows
+// before the chunk (zero at a sequence's first chunk) and the filter, 4 taps
+// per channel (zero past K), were staged in shared memory while the tiles
+// loaded.  Thread (row, 8-channel group); the norm's sum is a 16-lane
+// reduction.  The caller reads every raw row of a tile (results in registers
+// as bf16 pairs) before any is overwritten.
+// Filtered rows of one tile into res (bf16 pairs): compute only, no write.
 template <typename Off>
-GDN_DEV void conv_tile(__nv_bfloat16* tile, Off off, const __nv_bfloat16* x, __nv_bfloat16* out,
-                       const float* w, int K, bool norm, int h, size_t row0, size_t rs, int L,
-                       int halo) {
+GDN_DEV void conv_rows(uint4 (&res)[4], const __nv_bfloat16* tile, Off off, const __nv_bfloat16* hal,
+                       const float* wsm, int K, bool norm) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int c0 = 8 * (lane & 15);
-    float wr[8][4];
+    float wr[8][4];  // [channel][tap]; wsm is [tap][channel]: a half-warp reads 512 contiguous bytes
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) wr[i][j] = j < K ? w[((size_t)h * DK + c0 + i) * K + j] : 0.f;
-    uint4 res[4];
+    for (int j = 0; j < 4; ++j) {
+        const float4 a = *reinterpret_cast<const float4*>(wsm + j * DK + c0);
+        const float4 b = *reinterpret_cast<const float4*>(wsm + j * DK + c0 + 4);
+        wr[0][j] = a.x; wr[1][j] = a.y; wr[2][j] = a.z; wr[3][j] = a.w;
+        wr[4][j] = b.x; wr[5][j] = b.y; wr[6][j] = b.z; wr[7][j] = b.w;
+    }
 #pragma unroll
     for (int ps = 0; ps < 4; ++ps) {
         const int r = 16 * ps + 2 * warp + (lane >> 4);
@@ -95,10 +98,8 @@ GDN_DEV void conv_tile(__nv_bfloat16* tile, Off off, const __nv_bfloat16* x, __n
         for (int j = 0; j < 4; ++j) {
             if (j >= K) break;
             const int rr = r - j;  // tile row of tap j
-            uint4 v = make_uint4(0, 0, 0, 0);
-            if (rr >= 0) v = *reinterpret_cast<const uint4*>(tile + off(rr, c0));
-            else if (-rr <= halo)
-                v = *reinterpret_cast<const uint4*>(x + (row0 - (size_t)(-rr) * rs) * DK + c0);
+            const uint4 v = rr >= 0 ? *reinterpret_cast<const uint4*>(tile + off(rr, c0))
+                                    : *reinterpret_cast<const uint4*>(hal + (3 + rr) * DK + c0);
             const uint32_t e[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
@@ -123,7 +124,13 @@ GDN_DEV void conv_tile(__nv_bfloat16* tile, Off off, const __nv_bfloat16* x, __n
         res[ps] = make_uint4(pack_bf16(z[0], z[1]), pack_bf16(z[2], z[3]), pack_bf16(z[4], z[5]),
                              pack_bf16(z[6], z[7]));
     }
-    __syncthreads();  // every raw row read
+}
+// ... and their write-back into the tile and, for rows below L, to `out`.
+template <typename Off>
+GDN_DEV void conv_store(const uint4 (&res)[4], __nv_bfloat16* tile, Off off, __nv_bfloat16* out,
+                        size_t row0, size_t rs, int L) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int c0 = 8 * (lane & 15);
 #pragma unroll
     for (int ps = 0; ps < 4; ++ps) {
         const int r = 16 * ps + 2 * warp + (lane >> 4);
@@ -158,6 +165,27 @@ __global__ void __launch_bounds__(P5_THREADS, 3) tc5_prep_kernel(const __grid_co
         tma_load_3d(s.KQ + KQ_PANEL + C * 64, &p.qmap, 64, h, cl.tok, &s.bar_ld);
         tma_load_tile(s.V, &p.vmap, h, cl.tok, &s.bar_ld);
     }
+    if constexpr (CONV) {
+        // the filters [tensor][tap][channel] fp32 in P's space and the 3
+        // rows before the chunk [tensor][row][channel] bf16 in T's (both free
+        // until the first epilogue), while the tiles load
+        float* wsm = reinterpret_cast<float*>(s.P);
+        __nv_bfloat16* hal = s.T;
+        for (int e = tid; e < 3 * DK; e += P5_THREADS) {
+            const int t = e / DK, c = e % DK;
+            const float* src = (t == 0 ? p.conv.wk : t == 1 ? p.conv.wq : p.conv.wv) + ((size_t)h * DK + c) * p.conv.K;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) wsm[(t * 4 + j) * DK + c] = j < p.conv.K ? src[j] : 0.f;
+        }
+        const int halo = n > 0 ? 3 : 0;  // a dense batch: one sequence per row b
+        for (int e = tid; e < 3 * 3 * 16; e += P5_THREADS) {
+            const int t = e / 48, j = (e / 16) % 3, c = 8 * (e % 16);  // row j: token tok - 3 + j
+            uint4 v = make_uint4(0, 0, 0, 0);
+            const __nv_bfloat16* xs = t == 0 ? p.conv.xk : t == 1 ? p.conv.xq : p.conv.xv;
+            if (3 - j <= halo) v = *reinterpret_cast<const uint4*>(xs + (row0 - (size_t)(3 - j) * rs) * DK + c);
+            *reinterpret_cast<uint4*>(hal + (t * 3 + j) * DK + c) = v;
+        }
+    }
     if (warp == 0) {
         tc5::alloc(&s.tmem, P5_TCOLS);
         // inclusive cumsum of the log-gate over the chunk (rows past L add 0)
@@ -185,13 +213,20 @@ __global__ void __launch_bounds__(P5_THREADS, 3) tc5_prep_kernel(const __grid_co
     if constexpr (CONV) {  // the tiles are raw projections: filter them in place
         ok = mbar_wait(&s.bar_ld, 0, p.status);
         if (__syncthreads_or(!ok)) goto done;
-        const int halo = n > 0 ? 3 : 0;  // a dense batch: one sequence per row b
-        conv_tile(s.KQ, [](int r, int c) { return (c >> 6) * KQ_PANEL + swz<64>(r, c & 63); }, p.conv.xk,
-                  p.conv.kf, p.conv.wk, p.conv.K, true, h, row0, rs, L, halo);
-        conv_tile(s.KQ, [](int r, int c) { return (c >> 6) * KQ_PANEL + swz<64>(C + r, c & 63); }, p.conv.xq,
-                  p.conv.qf, p.conv.wq, p.conv.K, true, h, row0, rs, L, halo);
-        conv_tile(s.V, [](int r, int c) { return (c >> 6) * (C * 64) + swz<64>(r, c & 63); }, p.conv.xv,
-                  p.conv.vf, p.conv.wv, p.conv.K, false, h, row0, rs, L, halo);
+        const float* wsm = reinterpret_cast<const float*>(s.P);
+        auto offk = [](int r, int c) { return (c >> 6) * KQ_PANEL + swz<64>(r, c & 63); };
+        auto offq = [](int r, int c) { return (c >> 6) * KQ_PANEL + swz<64>(C + r, c & 63); };
+        auto offv = [](int r, int c) { return (c >> 6) * (C * 64) + swz<64>(r, c & 63); };
+        uint4 rr[4];  // a tile's raw rows are all read before any is overwritten
+        conv_rows(rr, s.KQ, offk, s.T, wsm, p.conv.K, true);
+        __syncthreads();
+        conv_store(rr, s.KQ, offk, p.conv.kf, row0, rs, L);
+        conv_rows(rr, s.KQ, offq, s.T + 3 * DK, wsm + 4 * DK, p.conv.K, true);
+        __syncthreads();
+        conv_store(rr, s.KQ, offq, p.conv.qf, row0, rs, L);
+        conv_rows(rr, s.V, offv, s.T + 6 * DK, wsm + 8 * DK, p.conv.K, false);
+        __syncthreads();
+        conv_store(rr, s.V, offv, p.conv.vf, row0, rs, L);
         fence_async_smem();  // filtered tiles (generic writes) -> tensor-core reads
         tc5::fence_before();
         __syncthreads();

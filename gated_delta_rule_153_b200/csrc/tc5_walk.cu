@@ -522,12 +522,15 @@ __global__ void __launch_bounds__(W5Cfg<MODE>::THREADS) tc5_walk_kernel(const __
 // state, chain).  M_j (64 KB fp32) arrives in shared memory by two bulk copies
 // on an mbarrier, the next step's map one step ahead (two buffers).
 // ---------------------------------------------------------------------------
-constexpr int SC_THREADS = 512, SC_ROWS = 16;
+constexpr int SC_THREADS = 128, SC_ROWS = 16;
 struct ScSmem {
     float M[2][DK * DK];   // double-buffered map
-    float Er[SC_ROWS][DK];
+    float Er[SC_ROWS][DK]; // this CTA's rows of the entry state of the current run
     uint64_t bar[2];
 };
+// Thread t: rows 4 (t / 32) .. +3 and columns 4 (t % 32) .. +3 of the CTA's
+// 16 x 128 block, so each map element read from shared memory feeds four rows
+// (a warp reads 512 contiguous bytes of a map row; the state rows broadcast).
 __global__ void __launch_bounds__(SC_THREADS) tc5_seg_scan_kernel(float* E, const float* Mmap,
                                                                   const float* Nmap, int nseg,
                                                                   unsigned int* status) {
@@ -535,7 +538,7 @@ __global__ void __launch_bounds__(SC_THREADS) tc5_seg_scan_kernel(float* E, cons
     ScSmem& s = *reinterpret_cast<ScSmem*>(sc_raw);
     const int tid = threadIdx.x;
     const int b = blockIdx.y, r0 = blockIdx.x * SC_ROWS;
-    const int r = tid >> 5, c0 = (tid & 31) * 4;  // row r0 + r, columns c0 .. c0+3
+    const int rg = 4 * (tid >> 5), c0 = (tid & 31) * 4;
     auto slot = [&](int j) { return ((size_t)b * nseg + j) * DV * DK; };
     auto fetch = [&](int j) {  // map of run j into buffer j & 1
         uint64_t* bar = &s.bar[j & 1];
@@ -549,26 +552,40 @@ __global__ void __launch_bounds__(SC_THREADS) tc5_seg_scan_kernel(float* E, cons
         fence_mbar_init();
         if (nseg > 2) fetch(1);
     }
+    // E_1 (from run 0's walk), this CTA's rows
+    for (int e = tid; e < SC_ROWS * DK / 4; e += SC_THREADS)
+        reinterpret_cast<float4*>(&s.Er[0][0])[e] = reinterpret_cast<const float4*>(E + slot(1) + (size_t)r0 * DK)[e];
     __syncthreads();
     bool ok = true;
     for (int j = 1; j + 1 < nseg; ++j) {
         if (tid == 0 && j + 2 < nseg) fetch(j + 1);  // buffer of step j-1, released at its end
-        for (int e = tid; e < SC_ROWS * DK / 4; e += SC_THREADS)
-            reinterpret_cast<float4*>(&s.Er[0][0])[e] =
-                reinterpret_cast<const float4*>(E + slot(j) + (size_t)r0 * DK)[e];
-        float4 acc = reinterpret_cast<const float4*>(Nmap + slot(j) + (size_t)(r0 + r) * DK)[c0 / 4];
+        float acc[4][4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float4 nv = reinterpret_cast<const float4*>(Nmap + slot(j) + (size_t)(r0 + rg + i) * DK)[c0 / 4];
+            acc[i][0] = nv.x; acc[i][1] = nv.y; acc[i][2] = nv.z; acc[i][3] = nv.w;
+        }
         ok = ok && mbar_wait(&s.bar[j & 1], ((j - 1) >> 1) & 1, status);
         if (__syncthreads_or(!ok)) break;
         const float* M = s.M[j & 1];
-#pragma unroll 8
+#pragma unroll 4
         for (int k = 0; k < DK; ++k) {
-            const float e = s.Er[r][k];
             const float4 m = *reinterpret_cast<const float4*>(M + k * DK + c0);
-            acc.x = fmaf(e, m.x, acc.x); acc.y = fmaf(e, m.y, acc.y);
-            acc.z = fmaf(e, m.z, acc.z); acc.w = fmaf(e, m.w, acc.w);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float e = s.Er[rg + i][k];
+                acc[i][0] = fmaf(e, m.x, acc[i][0]); acc[i][1] = fmaf(e, m.y, acc[i][1]);
+                acc[i][2] = fmaf(e, m.z, acc[i][2]); acc[i][3] = fmaf(e, m.w, acc[i][3]);
+            }
         }
-        reinterpret_cast<float4*>(E + slot(j) + (size_t)DV * DK + (size_t)(r0 + r) * DK)[c0 / 4] = acc;
-        __syncthreads();  // this step's E rows written, its map buffer free
+        __syncthreads();  // every read of this step's entry rows and map done
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float4 v = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+            reinterpret_cast<float4*>(&s.Er[rg + i][0])[c0 / 4] = v;
+            reinterpret_cast<float4*>(E + slot(j + 1) + (size_t)(r0 + rg + i) * DK)[c0 / 4] = v;
+        }
+        __syncthreads();  // the next entry rows in place
     }
 }
 
