@@ -24,6 +24,8 @@
 // write of each state row.
 #include <math.h>
 
+#include <type_traits>
+
 #include "async.cuh"
 #include "common.cuh"
 #include "internal.h"
@@ -36,7 +38,7 @@ constexpr int TD = 128;           // d_k = d_v
 constexpr int TREE_THREADS = 256;  // 8 warps
 constexpr int kMaxTreeNodes = 64;
 
-template <int MP>
+template <int MP, bool KDA>
 struct TreeSmem {
     __nv_bfloat16 K[MP * TD];  // Swz<128>; rows of U (value index as column) once W is built
     __nv_bfloat16 Q[MP * TD];
@@ -53,10 +55,15 @@ struct TreeSmem {
     unsigned long long anc[MP];
     int par[MP], depth[MP];
     int maxdepth;
+    alignas(16) float Gc[KDA ? MP : 1][TD];  // channel gate: per-key sums of g over each root path (16-byte copies)
 };
 
 // One CTA per (sequence n, head h).  MB = number of 16-node blocks.
-template <int MB>
+// Channel gate (KDA): g_i is a vector over the keys, G_i its sum over the root
+// path, and every decay e^{G_i - G_j} (j an ancestor of i) carries the key
+// index, so A and P sum k_i k_j e^{G_i - G_j} (q_i k_j e^{G_i - G_j}) over the
+// keys pair by pair; W and the read-out take K .* e^G and Q .* e^G.
+template <int MB, bool KDA>
 __global__ void __launch_bounds__(TREE_THREADS, MB <= 2 ? 4 : 2)  // 4 CTAs per SM up to 32 nodes
 tree_verify_kernel(int M, int H, float scale, const int* __restrict__ parent,
                    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
@@ -65,7 +72,7 @@ tree_verify_kernel(int M, int H, float scale, const int* __restrict__ parent,
                    __nv_bfloat16* __restrict__ o, unsigned int* status) {
     constexpr int MP = 16 * MB;
     extern __shared__ __align__(128) unsigned char smem_raw[];
-    TreeSmem<MP>& s = *reinterpret_cast<TreeSmem<MP>*>(smem_raw);
+    TreeSmem<MP, KDA>& s = *reinterpret_cast<TreeSmem<MP, KDA>*>(smem_raw);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int nh = blockIdx.x, n = nh / H, h = nh % H;
     const size_t rs = (size_t)H * TD;                        // token row stride
@@ -89,15 +96,28 @@ tree_verify_kernel(int M, int H, float scale, const int* __restrict__ parent,
                 if (status) atomicOr(status, 2u);
                 p = -1;
             }
-            gi = g[((size_t)n * M + tid) * H + h];
+            if (!KDA) gi = g[((size_t)n * M + tid) * H + h];
             bi = beta[((size_t)n * M + tid) * H + h];
         }
         s.par[tid] = p;
         s.g[tid] = gi;
         s.beta[tid] = bi;
     }
+    if constexpr (KDA) {  // per-key gates of every node (zero past M)
+        for (int e = tid; e < MP * TD / 4; e += TREE_THREADS) {
+            const int i = e / (TD / 4), c4 = e % (TD / 4);
+            cp_async16_zfill(&s.Gc[i][4 * c4], g + (((size_t)n * M + (i < M ? i : 0)) * H + h) * TD + 4 * c4,
+                             i < M);
+        }
+        cp_async_commit();
+    }
     cp_async_wait<0>();
     __syncthreads();
+    if constexpr (KDA) {  // path sums, parents first: thread = key
+        if (tid < TD)
+            for (int i = 0; i < M; ++i)
+                if (s.par[i] >= 0) s.Gc[i][tid] += s.Gc[s.par[i]][tid];
+    }
 
     // ---- path sums of g and ancestor sets (parents precede children) ------
     if (tid < MP) {
@@ -115,6 +135,41 @@ tree_verify_kernel(int M, int H, float scale, const int* __restrict__ parent,
     __syncthreads();
 
     // ---- A (warps 0-3) and P (warps 4-7): 16 node rows each -----------------
+    if constexpr (KDA) {
+        // ancestor pairs (and, for P, the node itself) only; a warp per pair,
+        // a lane per 4 keys; the decays are e^{G_i - G_j} <= 1 key by key
+        for (int e = tid; e < MP * MP; e += TREE_THREADS) {
+            const int i = e / MP, j = e % MP;
+            s.A[i][j] = 0.f;
+            s.P[swz<64>(i, j)] = __float2bfloat16_rn(0.f);
+        }
+        __syncthreads();
+        int pc = 0;
+        const int c = 4 * lane;
+        for (int i = 0; i < M; ++i) {
+            for (unsigned long long m = s.anc[i] | (1ull << i); m; m &= m - 1ull, ++pc) {
+                if ((pc & 7) != warp) continue;
+                const int j = __ffsll((long long)m) - 1;
+                const uint2 ki = *reinterpret_cast<const uint2*>(&s.K[swz<TD>(i, c)]);
+                const uint2 kj = *reinterpret_cast<const uint2*>(&s.K[swz<TD>(j, c)]);
+                const uint2 qi = *reinterpret_cast<const uint2*>(&s.Q[swz<TD>(i, c)]);
+                const float2 ki0 = unpack_bf16(ki.x), ki1 = unpack_bf16(ki.y);
+                const float2 kj0 = unpack_bf16(kj.x), kj1 = unpack_bf16(kj.y);
+                const float2 qi0 = unpack_bf16(qi.x), qi1 = unpack_bf16(qi.y);
+                const float d0 = __expf(s.Gc[i][c] - s.Gc[j][c]), d1 = __expf(s.Gc[i][c + 1] - s.Gc[j][c + 1]);
+                const float d2 = __expf(s.Gc[i][c + 2] - s.Gc[j][c + 2]), d3 = __expf(s.Gc[i][c + 3] - s.Gc[j][c + 3]);
+                const float w0 = kj0.x * d0, w1 = kj0.y * d1, w2 = kj1.x * d2, w3 = kj1.y * d3;
+                float sa = ki0.x * w0 + ki0.y * w1 + ki1.x * w2 + ki1.y * w3;
+                float sq = qi0.x * w0 + qi0.y * w1 + qi1.x * w2 + qi1.y * w3;
+                sa = warp_sum(sa);
+                sq = warp_sum(sq);
+                if (lane == 0) {
+                    if (j != i) s.A[i][j] = s.beta[i] * sa;
+                    s.P[swz<64>(i, j)] = __float2bfloat16_rn(scale * sq);
+                }
+            }
+        }
+    } else {
     {
         const int mat = warp >> 2, mb = warp & 3;
         if (mb < MB) {
@@ -153,6 +208,7 @@ tree_verify_kernel(int M, int H, float scale, const int* __restrict__ parent,
     }
     __syncthreads();
 
+    }
     // ---- T = (I + A)^{-1}, one tree level at a time --------------------------
     // Row i of T is e_i - sum over ancestors l of A_il T_l, and T_ic is non-zero
     // only for c an ancestor of i or i itself; so every node of one depth is
@@ -181,8 +237,19 @@ tree_verify_kernel(int M, int H, float scale, const int* __restrict__ parent,
     for (int e = tid; e < MP * MP; e += TREE_THREADS) {
         const int i = e / MP, j = e % MP;
         const float t = s.T[i][j] * s.beta[j];
-        s.Tw[swz<64>(i, j)] = __float2bfloat16_rn(t * __expf(s.G[j]));
+        s.Tw[swz<64>(i, j)] = __float2bfloat16_rn(KDA ? t : t * __expf(s.G[j]));
         s.Tu[swz<64>(i, j)] = __float2bfloat16_rn(t);
+    }
+    if constexpr (KDA) {  // K .* e^G (the rows of W) and Q .* e^G (the read-out), in place
+        for (int e = tid; e < MP * TD / 2; e += TREE_THREADS) {
+            const int i = e / (TD / 2), c = 2 * (e % (TD / 2));
+            const float d0 = __expf(s.Gc[i][c]), d1 = __expf(s.Gc[i][c + 1]);
+            uint32_t* kp = reinterpret_cast<uint32_t*>(&s.K[swz<TD>(i, c)]);
+            uint32_t* qp = reinterpret_cast<uint32_t*>(&s.Q[swz<TD>(i, c)]);
+            const float2 kv = unpack_bf16(*kp), qv = unpack_bf16(*qp);
+            *kp = pack_bf16(kv.x * d0, kv.y * d1);
+            *qp = pack_bf16(qv.x * d0, qv.y * d1);
+        }
     }
     __syncthreads();
 
@@ -266,7 +333,7 @@ tree_verify_kernel(int M, int H, float scale, const int* __restrict__ parent,
         st_c<TD>(Ub, 16 * mb, a0, accu[mb][0]);
         st_c<TD>(Ub, 16 * mb, a0 + 8, accu[mb][1]);
         const int r = 16 * mb + (lane >> 2);
-        const float f0 = scale * __expf(s.G[r]), f1 = scale * __expf(s.G[r + 8]);
+        const float f0 = KDA ? scale : scale * __expf(s.G[r]), f1 = KDA ? scale : scale * __expf(s.G[r + 8]);
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
             acco[mb][nt][0] *= f0; acco[mb][nt][1] *= f0;
@@ -299,10 +366,11 @@ tree_verify_kernel(int M, int H, float scale, const int* __restrict__ parent,
 }
 
 // ---- commit: the recurrent form along the accepted node's root path --------
+template <bool KDA>
 struct CommitSmem {
     float k[kMaxTreeNodes][TD];  // keys of the path tokens, in path order
     float v[kMaxTreeNodes][TD];
-    float alpha[kMaxTreeNodes], beta[kMaxTreeNodes];
+    float alpha[kMaxTreeNodes][KDA ? TD : 1], beta[kMaxTreeNodes];  // decay per token (per key: channel gate)
     int path[kMaxTreeNodes];
     int len;
 };
@@ -310,13 +378,14 @@ struct CommitSmem {
 // One CTA per (n, h); a state row is covered by 8 lanes of 16 columns each
 // (column 4*(sub + 8j) + e), and each thread keeps four rows in registers for
 // the whole path: one streaming read and one streaming write per element.
+template <bool KDA>
 __global__ void __launch_bounds__(TREE_THREADS)
 tree_commit_kernel(int M, int H, const int* __restrict__ parent, const int* __restrict__ accepted,
                    const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
                    const float* __restrict__ g, const float* __restrict__ beta,
                    float* __restrict__ state, unsigned int* status) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
-    CommitSmem& s = *reinterpret_cast<CommitSmem*>(smem_raw);
+    CommitSmem<KDA>& s = *reinterpret_cast<CommitSmem<KDA>*>(smem_raw);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int nh = blockIdx.x, n = nh / H, h = nh % H;
     if (tid == 0) {
@@ -353,8 +422,14 @@ tree_commit_kernel(int M, int H, const int* __restrict__ parent, const int* __re
     }
     if (tid < len) {
         const size_t i = ((size_t)n * M + s.path[tid]) * H + h;
-        s.alpha[tid] = __expf(g[i]);
+        if (!KDA) s.alpha[tid][0] = __expf(g[i]);
         s.beta[tid] = beta[i];
+    }
+    if constexpr (KDA) {
+        for (int e = tid; e < len * TD; e += TREE_THREADS) {
+            const int p = e / TD, c = e % TD;
+            s.alpha[p][c] = __expf(g[(((size_t)n * M + s.path[p]) * H + h) * TD + c]);
+        }
     }
     float* S = state + (size_t)nh * TD * TD;
     const int sub = lane & 7, grp = lane >> 3;
@@ -373,13 +448,25 @@ tree_commit_kernel(int M, int H, const int* __restrict__ parent, const int* __re
             const float4 x = *reinterpret_cast<const float4*>(&s.k[p][4 * (sub + 8 * j)]);
             kr[4 * j] = x.x; kr[4 * j + 1] = x.y; kr[4 * j + 2] = x.z; kr[4 * j + 3] = x.w;
         }
-        const float al = s.alpha[p], be = s.beta[p];
+        float al[16];  // this thread's 16 key columns' decays
+        if constexpr (KDA) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float4 x = *reinterpret_cast<const float4*>(&s.alpha[p][4 * (sub + 8 * j)]);
+                al[4 * j] = x.x; al[4 * j + 1] = x.y; al[4 * j + 2] = x.z; al[4 * j + 3] = x.w;
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) al[j] = s.alpha[p][0];
+        }
+        const float be = s.beta[p];
 #pragma unroll
         for (int rr = 0; rr < 4; ++rr) {
             float dot = 0.f;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                st[rr][j].x *= al; st[rr][j].y *= al; st[rr][j].z *= al; st[rr][j].w *= al;
+                st[rr][j].x *= al[4 * j]; st[rr][j].y *= al[4 * j + 1];
+                st[rr][j].z *= al[4 * j + 2]; st[rr][j].w *= al[4 * j + 3];
                 dot += st[rr][j].x * kr[4 * j] + st[rr][j].y * kr[4 * j + 1] +
                        st[rr][j].z * kr[4 * j + 2] + st[rr][j].w * kr[4 * j + 3];
             }
@@ -402,14 +489,14 @@ tree_commit_kernel(int M, int H, const int* __restrict__ parent, const int* __re
     }
 }
 
-template <int MB>
+template <int MB, bool KDA>
 void launch_verify(int N, int M, int H, float scale, const int* parent, const void* q,
                    const void* k, const void* v, const float* g, const float* beta,
                    const float* state, void* o, unsigned int* status, cudaStream_t st) {
-    const int smem = sizeof(TreeSmem<16 * MB>);
-    cudaFuncSetAttribute(tree_verify_kernel<MB>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    const int smem = sizeof(TreeSmem<16 * MB, KDA>);
+    cudaFuncSetAttribute(tree_verify_kernel<MB, KDA>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     GDN_LAUNCH("tree_verify", st,
-               (tree_verify_kernel<MB><<<(unsigned)(N * H), TREE_THREADS, smem, st>>>(
+               (tree_verify_kernel<MB, KDA><<<(unsigned)(N * H), TREE_THREADS, smem, st>>>(
                    M, H, scale, parent, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k,
                    (const __nv_bfloat16*)v, g, beta, state, (__nv_bfloat16*)o, status)));
 }
@@ -422,8 +509,7 @@ gdn_status check_tree(int N, int M, int H, int dk, int dv, gdn_dtype dtype, gdn_
     if (dtype != GDN_BF16 && dtype != GDN_F32) return GDN_ERR_INVALID_ARG;
     if (gate != GDN_GATE_SCALAR && gate != GDN_GATE_CHANNEL) return GDN_ERR_INVALID_ARG;
     if (M > kMaxTreeNodes) return GDN_ERR_UNSUPPORTED;
-    if (dtype != GDN_BF16 || gate != GDN_GATE_SCALAR || dk != TD || dv != TD)
-        return GDN_ERR_UNSUPPORTED;
+    if (dtype != GDN_BF16 || dk != TD || dv != TD) return GDN_ERR_UNSUPPORTED;
     return GDN_OK;
 }
 
@@ -447,14 +533,20 @@ gdn_status gdn_tree_verify(int N, int M, int H, int dk, int dv, gdn_dtype dtype,
         !aligned(o, 16) || !aligned(parent, 4) || !aligned(g, 4) || !aligned(beta, 4) ||
         !aligned(status, 4))
         return GDN_ERR_INVALID_ARG;
+    if (gate == GDN_GATE_CHANNEL && !aligned(g, 16)) return GDN_ERR_INVALID_ARG;  // 16-byte copies of g rows
     cudaStream_t st = (cudaStream_t)stream;
     cudaGetLastError();
-    switch ((M + 15) / 16) {
-        case 1: launch_verify<1>(N, M, H, scale, parent, q, k, v, g, beta, state, o, status, st); break;
-        case 2: launch_verify<2>(N, M, H, scale, parent, q, k, v, g, beta, state, o, status, st); break;
-        case 3: launch_verify<3>(N, M, H, scale, parent, q, k, v, g, beta, state, o, status, st); break;
-        default: launch_verify<4>(N, M, H, scale, parent, q, k, v, g, beta, state, o, status, st); break;
-    }
+    auto run = [&](auto kda) {
+        constexpr bool K = decltype(kda)::value;
+        switch ((M + 15) / 16) {
+            case 1: launch_verify<1, K>(N, M, H, scale, parent, q, k, v, g, beta, state, o, status, st); break;
+            case 2: launch_verify<2, K>(N, M, H, scale, parent, q, k, v, g, beta, state, o, status, st); break;
+            case 3: launch_verify<3, K>(N, M, H, scale, parent, q, k, v, g, beta, state, o, status, st); break;
+            default: launch_verify<4, K>(N, M, H, scale, parent, q, k, v, g, beta, state, o, status, st); break;
+        }
+    };
+    if (gate == GDN_GATE_CHANNEL) run(std::true_type{});
+    else run(std::false_type{});
     return launched();
 }
 
@@ -471,12 +563,17 @@ gdn_status gdn_tree_commit(int N, int M, int H, int dk, int dv, gdn_dtype dtype,
         return GDN_ERR_INVALID_ARG;
     cudaStream_t st = (cudaStream_t)stream;
     cudaGetLastError();
-    const int smem = sizeof(CommitSmem);
-    cudaFuncSetAttribute(tree_commit_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    GDN_LAUNCH("tree_commit", st,
-               (tree_commit_kernel<<<(unsigned)(N * H), TREE_THREADS, smem, st>>>(
-                   M, H, parent, accepted, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, g,
-                   beta, state, status)));
+    auto run = [&](auto kda) {
+        constexpr bool K = decltype(kda)::value;
+        const int smem = sizeof(CommitSmem<K>);
+        cudaFuncSetAttribute(tree_commit_kernel<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        GDN_LAUNCH("tree_commit", st,
+                   (tree_commit_kernel<K><<<(unsigned)(N * H), TREE_THREADS, smem, st>>>(
+                       M, H, parent, accepted, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, g,
+                       beta, state, status)));
+    };
+    if (gate == GDN_GATE_CHANNEL) run(std::true_type{});
+    else run(std::false_type{});
     return launched();
 }
 

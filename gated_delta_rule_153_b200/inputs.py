@@ -198,12 +198,13 @@ def tree_parents(N: int, M: int, shape: str = "random", seed: int = 0) -> torch.
 
 def make_tree_inputs(N: int, M: int, H: int, shape: str = "random", seed: int = 1200,
                      g_shift: float = 0.0, beta_max: float = 1.0,
-                     state_std: float = 0.02) -> dict:
+                     state_std: float = 0.02, gate: str = "scalar") -> dict:
     """Host tensors for draft-tree verification: q, k [N,M,H,128] and v
-    [N,M,H,128] bf16 (q, k L2-normalised), g, beta [N,M,H] fp32 drawn as in
-    make_chunk_inputs, state [N,H,128,128] fp32, parent [N,M] int32 and
-    accepted [N] int32 (uniform over -1 .. M-1)."""
-    cfg = ChunkConfig("tree", N, M, H, 128, 128, 64, "bf16", "scalar", g_shift, None,
+    [N,M,H,128] bf16 (q, k L2-normalised), g [N,M,H] (or [N,M,H,128] for the
+    channel gate) and beta [N,M,H] fp32 drawn as in make_chunk_inputs, state
+    [N,H,128,128] fp32, parent [N,M] int32 and accepted [N] int32 (uniform
+    over -1 .. M-1)."""
+    cfg = ChunkConfig("tree", N, M, H, 128, 128, 64, "bf16", gate, g_shift, None,
                       False, None, seed, beta_max)
     tok = make_chunk_inputs(cfg)
     state = torch.randn(N, H, 128, 128, generator=_gen(seed, 12)) * state_std

@@ -248,11 +248,14 @@ gdn_status gdn_short_conv_bwd(int B, int T, int H, int d, int K, gdn_dtype dtype
  * accepted[n] (-1 or nothing accepted: S is left untouched), by the
  * recurrent form along that path on the fp32 state.
  * Layouts (contiguous): parent [N, M] int32; accepted [N] int32; q, k
- * [N, M, H, dk]; v, o [N, M, H, dv]; g, beta [N, M, H] fp32; state
- * [N, H, dv, dk] fp32 (row = value index).  All device pointers.
- * Supported: GDN_BF16, GDN_GATE_SCALAR, dk = dv = 128, 1 <= M <= 64 (else
+ * [N, M, H, dk]; v, o [N, M, H, dv]; g [N, M, H] fp32 (scalar gate) or
+ * [N, M, H, dk] fp32 (channel gate: the decay of node t is Diag(e^{g_t}) on
+ * the key index); beta [N, M, H] fp32; state [N, H, dv, dk] fp32 (row =
+ * value index).  All device pointers.
+ * Supported: GDN_BF16, either gate, dk = dv = 128, 1 <= M <= 64 (else
  * GDN_ERR_UNSUPPORTED); N, H, M < 1, null pointers or misalignment (16 bytes
- * for q, k, v, o, state; 4 for the rest) are GDN_ERR_INVALID_ARG.
+ * for q, k, v, o, state and a channel-gate g; 4 for the rest) are
+ * GDN_ERR_INVALID_ARG.
  * Tree indices are device data and are checked on the device: a parent out
  * of [-1, i) is read as -1 and an accepted index out of [-1, M) as -1; either
  * sets bit 1 (value 2) of the optional device word *status (may be NULL),

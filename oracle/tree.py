@@ -56,9 +56,10 @@ def root_path(parent, i):
 
 
 def _run_path(S, path, k, v, g, beta):
-    """Token loop of the gated delta rule over the nodes of `path` (scalar
-    gate), one (sequence, head) pair: S [dv, dk]; k [M, dk]; v [M, dv];
-    g, beta [M]."""
+    """Token loop of the gated delta rule over the nodes of `path`, one
+    (sequence, head) pair: S [dv, dk]; k [M, dk]; v [M, dv]; beta [M]; g [M]
+    (scalar gate) or [M, dk] (channel gate: the decay Diag(e^{g_t}) acts on the
+    key index, i.e. scales the columns of S)."""
     S = S.copy()
     for t in path:
         S = S * np.exp(g[t])
@@ -68,8 +69,8 @@ def _run_path(S, path, k, v, g, beta):
 
 
 def verify(parent, q, k, v, g, beta, state, scale=1.0):
-    """parent [N, M] ints; q, k [N, M, H, dk]; v [N, M, H, dv]; g, beta
-    [N, M, H]; state [N, H, dv, dk].  Returns o [N, M, H, dv] (float64): the
+    """parent [N, M] ints; q, k [N, M, H, dk]; v [N, M, H, dv]; g [N, M, H]
+    or [N, M, H, dk]; beta [N, M, H]; state [N, H, dv, dk].  Returns o [N, M, H, dv] (float64): the
     read-out of every node after the tokens of its root path."""
     parent = np.asarray(parent)
     q, k, v, g, beta, state = map(_f64, (q, k, v, g, beta, state))

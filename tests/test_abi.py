@@ -175,7 +175,9 @@ def test_tree_checks():
     assert v(2, 65, 4, 128, 128, bf, sc, 1.0, *args) == gdn.GDN_ERR_UNSUPPORTED
     assert v(2, 8, 4, 64, 128, bf, sc, 1.0, *args) == gdn.GDN_ERR_UNSUPPORTED
     assert v(2, 8, 4, 128, 128, gdn.GDN_F32, sc, 1.0, *args) == gdn.GDN_ERR_UNSUPPORTED
-    assert v(2, 8, 4, 128, 128, bf, ch, 1.0, *args) == gdn.GDN_ERR_UNSUPPORTED
+    # the channel gate is supported, with its g rows 16-byte aligned
+    assert v(2, 8, 4, 128, 128, bf, ch, 1.0, p, p, p, p, ctypes.c_void_p(260), p, p, p, None,
+             None) == gdn.GDN_ERR_INVALID_ARG
     assert v(2, 8, 4, 128, 128, bf, sc, float("nan"), *args) == gdn.GDN_ERR_INVALID_ARG
     assert v(2, 8, 4, 128, 128, bf, sc, 1.0, None, *args[1:]) == gdn.GDN_ERR_INVALID_ARG
     assert v(2, 8, 4, 128, 128, bf, sc, 1.0, p, ctypes.c_void_p(264), *args[2:]) == \

@@ -27,8 +27,10 @@ def _verify(d, scale=1.0, status=None):
 
 @pytest.mark.parametrize("M", [1, 5, 16, 17, 33, 48, 64])
 @pytest.mark.parametrize("shape", ["random", "kary4"])
-def test_verify_matches_oracle(dev, M, shape):
-    inp = make_tree_inputs(3, M, 4, shape=shape, seed=1200 + M, g_shift=-1.0, state_std=0.05)
+@pytest.mark.parametrize("gate", ["scalar", "channel"])
+def test_verify_matches_oracle(dev, M, shape, gate):
+    inp = make_tree_inputs(3, M, 4, shape=shape, seed=1200 + M, g_shift=-1.0, state_std=0.05,
+                           gate=gate)
     o = _verify(_dev(inp, dev), scale=0.9)
     ref = tree_oracle.verify(inp["parent"].numpy(), inp["q"], inp["k"], inp["v"], inp["g"],
                              inp["beta"], inp["state"], scale=0.9)
@@ -37,9 +39,10 @@ def test_verify_matches_oracle(dev, M, shape):
 
 
 @pytest.mark.parametrize("M", [1, 7, 64])
-def test_commit_matches_oracle(dev, M):
+@pytest.mark.parametrize("gate", ["scalar", "channel"])
+def test_commit_matches_oracle(dev, M, gate):
     """fp32 recurrent form along the accepted path: held to the fp32 bar."""
-    inp = make_tree_inputs(6, M, 3, seed=1300 + M, g_shift=-1.0, state_std=0.05)
+    inp = make_tree_inputs(6, M, 3, seed=1300 + M, g_shift=-1.0, state_std=0.05, gate=gate)
     inp["accepted"][0] = -1
     inp["accepted"][1] = M - 1
     d = _dev(inp, dev)
@@ -116,3 +119,16 @@ def test_invalid_tree_indices_are_reported(dev):
                         status=status)
     assert gdn.gdn_query_device_status(status) == gdn.GDN_ERR_INVALID_ARG
     assert torch.equal(d["state"], before)
+
+
+def test_channel_gate_chain_equals_chunkwise_forward(dev):
+    """Channel gate: a 64-node chain agrees with gdn_chunk_fwd from the same
+    state, the decays acting per key."""
+    inp = make_tree_inputs(2, 64, 4, shape="chain", seed=23, g_shift=-2.0, state_std=0.05,
+                           gate="channel")
+    d = _dev(inp, dev)
+    o = _verify(d)
+    q, k, v, g, beta = (d[n].contiguous() for n in ("q", "k", "v", "g", "beta"))
+    o2, _ = gdn.gdn_chunk_fwd(q, k, v, g, beta, d["state"])
+    torch.cuda.synchronize()
+    assert rel_err(o, o2.double().cpu().numpy()) < 2e-2

@@ -17,11 +17,11 @@ def _unit(rng, shape):
     return x / np.linalg.norm(x, axis=-1, keepdims=True)
 
 
-def _inputs(rng, N=2, M=7, H=2, dk=5, dv=3):
+def _inputs(rng, N=2, M=7, H=2, dk=5, dv=3, channel=False):
     q = _unit(rng, (N, M, H, dk))
     k = _unit(rng, (N, M, H, dk))
     v = rng.standard_normal((N, M, H, dv))
-    g = -np.log1p(np.exp(rng.standard_normal((N, M, H))))
+    g = -np.log1p(np.exp(rng.standard_normal((N, M, H) + ((dk,) if channel else ()))))
     beta = 1 / (1 + np.exp(-rng.standard_normal((N, M, H))))
     S0 = 0.5 * rng.standard_normal((N, H, dv, dk))
     return q, k, v, g, beta, S0
@@ -31,11 +31,12 @@ def _random_parents(rng, N, M):
     return np.array([[rng.integers(-1, i) for i in range(M)] for _ in range(N)])
 
 
-def test_chain_is_the_token_loop():
+def test_chain_is_the_token_loop(channel=False):
     """parent[i] = i - 1: node i reads out token i of one sequence; committing
-    node j gives the state after its first j + 1 tokens."""
+    node j gives the state after its first j + 1 tokens (scalar gate, and the
+    channel gate against the C oracle's per-key decay)."""
     rng = np.random.default_rng(31)
-    q, k, v, g, beta, S0 = _inputs(rng)
+    q, k, v, g, beta, S0 = _inputs(rng, channel=channel)
     N, M = q.shape[:2]
     par = np.tile(np.arange(M) - 1, (N, 1))
     o = tree.verify(par, q, k, v, g, beta, S0, scale=0.8)
@@ -48,10 +49,10 @@ def test_chain_is_the_token_loop():
         assert np.abs(S - S2).max() < 1e-12
 
 
-def test_star_is_one_decode_step_per_node():
+def test_star_is_one_decode_step_per_node(channel=False):
     """Every parent -1: each node is one decode step from S0."""
     rng = np.random.default_rng(32)
-    q, k, v, g, beta, S0 = _inputs(rng, N=1, M=6)
+    q, k, v, g, beta, S0 = _inputs(rng, N=1, M=6, channel=channel)
     par = -np.ones((1, 6), dtype=int)
     o = tree.verify(par, q, k, v, g, beta, S0, scale=1.3)
     for i in range(6):
@@ -59,6 +60,14 @@ def test_star_is_one_decode_step_per_node():
         assert np.abs(o[:, i] - oi).max() < 1e-12
         S = tree.commit(par, [i], k, v, g, beta, S0)
         assert np.abs(S - Si).max() < 1e-12
+
+
+def test_chain_is_the_token_loop_channel_gate():
+    test_chain_is_the_token_loop(channel=True)
+
+
+def test_star_is_one_decode_step_per_node_channel_gate():
+    test_star_is_one_decode_step_per_node(channel=True)
 
 
 def test_random_trees_follow_their_root_paths():
