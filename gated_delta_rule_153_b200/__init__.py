@@ -296,17 +296,25 @@ def gdn_chunk_fwd_save(q, k, v, g, beta, h0=None, *, chunk=64, scale=1.0,
 
 
 def gdn_chunk_bwd_saved(q, k, v, g, beta, dO, workspace, h0=None, dhT=None, *, chunk=64,
-                        scale=1.0, stream=None):
-    """Backward from gdn_chunk_fwd_save's workspace; results as gdn_chunk_bwd."""
+                        scale=1.0, out=None, stream=None):
+    """Backward from gdn_chunk_fwd_save's workspace; results as gdn_chunk_bwd.
+    ``out``: optional dict of preallocated result tensors (dq, dk, dv, dg,
+    dbeta, dh0), filled in place."""
     import torch
     B, T, H, dk, dv = _validate_chunk_inputs(q, k, v, g, beta, h0)
     _need(dO, "dO", q.dtype, (B, T, H, dv))
     if dhT is not None:
         _need(dhT, "dhT", torch.float32, (B, H, dv, dk))
     dims = make_dims(q, v, g, chunk, scale)
-    out = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dv=torch.empty_like(v),
-               dg=torch.empty_like(g), dbeta=torch.empty_like(beta),
-               dh0=None if h0 is None else torch.empty_like(h0))
+    if out is None:
+        out = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dv=torch.empty_like(v),
+                   dg=torch.empty_like(g), dbeta=torch.empty_like(beta),
+                   dh0=None if h0 is None else torch.empty_like(h0))
+    else:
+        for n, ref in (("dq", q), ("dk", k), ("dv", v), ("dg", g), ("dbeta", beta)):
+            _need(out[n], n, ref.dtype, tuple(ref.shape))
+        if h0 is not None:
+            _need(out["dh0"], "dh0", torch.float32, tuple(h0.shape))
     nbytes = gdn_chunk_saved_workspace(dims)
     if nbytes and (workspace is None or workspace.numel() * workspace.element_size() < nbytes):
         raise ValueError(f"workspace must be gdn_chunk_fwd_save's ({nbytes} bytes)")

@@ -177,6 +177,14 @@ __global__ void __launch_bounds__(KB_THREADS, 1) tc5_bwd_local_kda_kernel(const 
     }
     if (warp == 0) tc5::alloc(&s.tmem, KB_TCOLS);
     if (tid < C) s.beta[tid] = tid < L ? p.beta[row0 + tid * rs] : 0.f;
+    // the per-key gate rows of the chunk a wave ahead (512 bytes each) into L2
+    if (tid >= 64 && tid < 64 + C && p.pf_stride > 0 && cid + p.pf_stride < (int)gridDim.x) {
+        const int pc = cid + p.pf_stride, pbh = pc / p.NT;
+        const ChunkLoc pl = chunk_loc(p.seq, p.T, p.H, pbh, pc % p.NT);
+        const int r = tid - 64;
+        if (pl.valid && r < pl.L)
+            bulk_prefetch_l2(p.g + (((size_t)pl.tok + r) * p.H + pbh % p.H) * DK, DK * 4);
+    }
 
     // Thread (c, tg): key / value / TMEM lane c = 32 (warp % 4) + lane, token
     // block tg = warp / 4 (tokens 16 tg .. +15).  Lane-token epilogues: token

@@ -110,6 +110,14 @@ __global__ void __launch_bounds__(PK_THREADS, 2) tc5_prep_kda_kernel(const __gri
     }
     if (tid < 4) s.span[tid] = 0u;
     if (tid < C) s.beta[tid] = tid < L ? p.beta[row0 + tid * rs] : 0.f;
+    // the per-key gate rows of the chunk a wave ahead (512 bytes each) into L2
+    if (tid >= 64 && tid < 64 + C && p.pf_stride > 0 && cid + p.pf_stride < (int)gridDim.x) {
+        const int pc = cid + p.pf_stride, pbh = pc / p.NT;
+        const ChunkLoc pl = chunk_loc(p.seq, p.T, p.H, pbh, pc % p.NT);
+        const int r = tid - 64;
+        if (pl.valid && r < pl.L)
+            bulk_prefetch_l2(p.g + (((size_t)pl.tok + r) * p.H + pbh % p.H) * DK, DK * 4);
+    }
     if (warp == 0) tc5::alloc(&s.tmem, PK_TCOLS);
 
     // ---- per-key cumsum: thread (key pair kp, block bq) holds keys 2 kp and
@@ -402,7 +410,9 @@ done:
 }  // namespace
 
 namespace tc {
-void launch_prep5_kda(const ChunkPtrs& p, size_t nchunks, cudaStream_t st) {
+void launch_prep5_kda(const ChunkPtrs& pin, size_t nchunks, cudaStream_t st) {
+    ChunkPtrs p = pin;
+    p.pf_stride = 2 * sm_count();  // two CTAs per SM
     const int smem = sizeof(PkSmem) + 1024;
     cudaFuncSetAttribute(tc5_prep_kda_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     GDN_LAUNCH("tc5_prep_kda", st, tc5_prep_kda_kernel<<<(unsigned)nchunks, PK_THREADS, smem, st>>>(p));

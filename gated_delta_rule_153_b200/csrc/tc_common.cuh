@@ -174,6 +174,7 @@ struct ChunkPtrs {
     // bounded waits of the tcgen05 forward walks (see tc5_walk.cu)
     unsigned long long wait_ns = kWaitNs;
     int stall_at = -1;
+    int pf_stride = 0;  // preparation: chunks a wave ahead whose gate rows go to L2 (0: none)
     // The q/k/v prologue fused into the preparation's load stage: the token
     // maps above then cover the raw projections, whose rows before a chunk
     // (the filter's history) are read from xq, xk, xv; the filtered tensors
