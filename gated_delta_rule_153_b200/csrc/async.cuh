@@ -85,6 +85,11 @@ GDN_DEV void bulk_prefetch_l2(const void* gmem, uint32_t bytes) {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(gmem), "r"(bytes) : "memory");
 }
 
+// Hint: pull the cache line holding `gmem` into L2.
+GDN_DEV void prefetch_l2(const void* gmem) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(gmem) : "memory");
+}
+
 // Bulk copy from shared memory to global memory (bulk-group completion).
 GDN_DEV void bulk_s2g(void* gmem, const void* smem, uint32_t bytes) {
     asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"

@@ -4,16 +4,21 @@
 // Reverse mode through the chunk equations of "Gated Delta Networks:
 // Improving Mamba2 with Delta Rule" (paper review), section "Method" (the WY /
 // UT-transform form; see tc_chunk.cu).  Given a chunk's entering state S0 and
-// U (from the forward recompute) and its dS (gradient of the state leaving it)
-// and dU (from the reverse walk), with Gamma_ij = e^{G_i - G_j}, etl_i =
+// U (from the forward), its dS (gradient of the state leaving it) and dU
+// (from the reverse walk), with Gamma_ij = e^{G_i - G_j}, etl_i =
 // e^{G_last - G_i} and gamma = e^{G_last}:
 //   dq  = scale e^G .* (dO S0) + sdPG K,        sdPG = scale lower(dO U^T) .* Gamma
-//   dW  = -dU S0,   dT = dW (beta e^G .* K)^T + dU (beta .* V)^T
-//   dA  = strict_lower(-T^T dT T^T),   dMM = dA .* beta_i .* Gamma
-//   dk  = etl .* (U dS) + beta e^G .* (T^T dW) + dMM K + dMM^T K + sdPG^T Q
-//   dv  = beta .* (T^T dU)
+//   dW  = -dU S0,   Gk = T^T dW,   Gv = T^T dU
+//   dA  = strict_lower(-T^T dT T^T) = strict_lower(-(Gk W^T + Gv U~^T)),
+//   dMM = dA .* beta_i .* Gamma
+//   dk  = etl .* (U dS) + beta e^G .* Gk + dMM K + dMM^T K + sdPG^T Q
+//   dv  = beta .* Gv
 // and the gate and beta gradients from the matching row and column sums, with
-// dg the reverse within-chunk cumsum of dG.
+// dg the reverse within-chunk cumsum of dG.  The dA line uses the WY factors
+// themselves: dT = dW (beta e^G .* K)^T + dU (beta .* V)^T, so
+// T^T dT T^T = Gk (T beta e^G K)^T + Gv (T beta V)^T = Gk W^T + Gv U~^T, and
+// the W and U~ images of the forward's preparation serve as operands.  One
+// product replaces the chain dT -> dT T^T -> T^T (dT T^T).
 //
 // Every product is one tcgen05 MMA group with M = 128 and an fp32 accumulator
 // in tensor memory.  The 64-token tiles sit in pairs in 128-row K-major panels
@@ -24,13 +29,13 @@
 //                        scale e^{G_i}: the dq accumulator, lanes 64..127)
 //   [U ; V] dS        -> etl .* (U dS) (U rows pre-scaled: the dk accumulator)
 //   [K ; Q] K^T       -> K K^T, Q K^T       [dU ; dO] U^T -> dO U^T
-//   [dU ; dO] V^T     -> dU V^T             [dW ; .] K^T  -> dW K^T
-//   [dT ; .] T^T -> X,  [T^T ; .] X -> T^T X,  [T^T ; .] dW,  [T^T ; .] dU
+//   [T^T ; .] dW -> Gk,  [T^T ; .] dU -> Gv,  [Gk ; .] W^T + [Gv ; .] U~^T -> -dA
 //   dk += [dMM ; .] K + [dMM^T ; .] K + [sdPG^T ; .] Q,   dq += [. ; sdPG] K
 // In every epilogue four warps share a TMEM lane quarter (one token row per
-// thread) and split the row's columns; per-token sums meet in shared-memory
-// atomics, and column sums over tokens go through a shared-memory transpose.
-// One CTA of sixteen warps per chunk; thread 0 issues the loads and the MMAs.
+// thread) and split the row's columns; per-token sums meet in fixed-order
+// shared-memory partials, and column sums over tokens go through a
+// shared-memory transpose.  One CTA of sixteen warps per chunk; thread 0
+// issues the loads and the MMAs.
 #include "async.cuh"
 #include "common.cuh"
 #include "internal.h"
@@ -47,71 +52,65 @@ constexpr int PAIR = 128 * 64;  // elements of one 128-row, 64-column panel
 // tensor-memory columns
 constexpr uint32_t TA = 0,     // [-dW ; dq accumulator]          128
     TB = 128,                  // [dk accumulator ; .]            128
-    TC1 = 256,                 // [K K^T ; Q K^T]                  64  (then X)
-    TC2 = 320,                 // [. ; dO U^T]                     64  (then T^T X)
-    TW = 384,                  // [dW K^T ; .]                     64
-    TU = 448,                  // [dU V^T ; .]                     64
-    TKG = 256,                 // [T^T dW ; .]                    128 (phase E)
-    TVB = 384,                 // [T^T dU ; .]                    128 (phase E)
+    TC1 = 256,                 // [K K^T ; Q K^T]                  64
+    TC2 = 320,                 // [. ; dO U^T]                     64
+    TKG = 256,                 // [Gk = T^T dW ; .]               128 (after the first epilogue)
+    TVB = 384,                 // [Gv = T^T dU ; .]               128 (after the first epilogue)
+    TD = 384,                  // [Gk W^T + Gv U~^T ; .]           64 (after Gv is read)
+    TKK = 448,                 // [K K^T ; .] again                64 (after Gv is read)
     BL_TCOLS = 512;
 constexpr uint32_t ID_N64 = tc5::idesc_bf16(128, 64, false, false);     // A, B K-major
+constexpr uint32_t ID_N64_BMN = tc5::idesc_bf16(128, 64, false, true);   // B MN-major
 constexpr uint32_t ID_N128_BMN = tc5::idesc_bf16(128, 128, false, true); // B MN-major
-constexpr uint32_t ID_N64_AMN_BMN = tc5::idesc_bf16(128, 64, true, true);
 constexpr uint32_t ID_N128_AMN_BMN = tc5::idesc_bf16(128, 128, true, true);
 
+// Shared memory (one CTA per SM).  The CTA is persistent: it takes the chunks
+// blockIdx.x, blockIdx.x + gridDim.x, ... and loads each buffer of the next
+// chunk as soon as the current chunk is done with it (S0, dS and U after the
+// first products, T and Q after E1, dU, dO, W and U~ after C, K after E2),
+// so the loads of a chunk overlap the work of the one before.
 struct alignas(1024) BlSmem {
-    __nv_bfloat16 R1[2 * PAIR];  // [dU | dO] panels; later dW in the dO rows
+    __nv_bfloat16 R4[DV * DK];   // S0 (Kp<128>)
+    __nv_bfloat16 R5[DV * DK];   // dS (Kp<128>)
+    __nv_bfloat16 R1[2 * PAIR];  // [dU | dO] panels; dW in the dO rows; then Gk (rows 0..63)
+                                 // and Gv (from 8 KB on: rows 64..127 and the next panel)
     __nv_bfloat16 R2[2 * PAIR];  // [K | Q]
-    __nv_bfloat16 R3[2 * PAIR];  // [U | V]; later dMM in the U rows of panel 0
-    __nv_bfloat16 R4[DV * DK];   // S0 (Kp<128>); later dT | X | M (fp32)
-    __nv_bfloat16 R5[DV * DK];   // dS (Kp<128>); later . | sdPG | transpose scratch (fp32)
-    // Swz<64> T, then 8 KB that the MN-major T^T operands read as their unused
-    // rows 64..127
-    __nv_bfloat16 T[2 * C * C];
-    float G[C], beta[C];
+    __nv_bfloat16 R3[2 * PAIR];  // [U | .]: U rows; sdPG in the other rows of panel 0, dMM in
+                                 // those of panel 1 (V is not held: its rows are read from L2)
+    // Swz<64> T; the MN-major T^T operands read the 8 KB after it (W) as their
+    // unused rows 64..127
+    __nv_bfloat16 T[C * C];
+    __nv_bfloat16 W[C * DK];     // Tma128 image of W (two 64-key K-major panels)
+    __nv_bfloat16 Ut[DV * C];    // Swz<64> image of U~^T (value rows x tokens)
+    float Xs[C * C];             // transpose scratch for column sums (fp32, rotated columns)
+    float G[2][C], beta[2][C];   // per chunk, alternating
     // Fixed-order partial sums (the dg and dbeta results are bit-reproducible):
     float pG[8][C];              // dG terms of a token's own rows, per (column group, lane half)
     float pB[4][C];              // dbeta terms, per column group
     float pC[8][C];              // column sums of hP and hA, per 8-row block
     float red[16], red2[16];     // per-warp sums: <dS, S0>; etl <dKt, k> (enters dG_last)
     float dgs[C];                // reverse-cumsum scratch
-    uint64_t bar_ld, bar_mma;
+    // one load barrier per buffer group (one phase per chunk), one for the MMAs
+    uint64_t bar_s, bar_u, bar_tq, bar_r1, bar_wu, bar_k, bar_mma;
     uint32_t tmem;
 };
 
 struct BlPtrs {
-    CUtensorMap qmap, kmap, vmap, dOmap;
+    CUtensorMap qmap, kmap, dOmap;
     const float *g, *beta;
-    const __nv_bfloat16 *S0, *U, *dS, *dU, *Tb;
+    const __nv_bfloat16 *v;
+    const __nv_bfloat16 *S0, *U, *dS, *dU, *Tb, *W, *Ut;
     __nv_bfloat16 *dq, *dk, *dv;
     float *dg, *dbeta;
     unsigned int* status;
-    int B, T, H, NT;
+    int B, T, H, NT, nchunks;
     float scale;
-    int pf_stride;  // chunks a wave ahead to pull into L2; 0: no prefetch
     SeqMap seq;
 };
 
 // 32 consecutive TMEM columns of this thread's lane into v[0..31].
 GDN_DEV void ld_row32(float* v, uint32_t taddr) {
     tc5::ld32(*reinterpret_cast<float(*)[32]>(v), taddr);
-}
-
-// Scale the 64 elements of row r (0..127) of a pair region's panel by f.
-GDN_DEV void scale_pair_row(__nv_bfloat16* R, int r, int panel, float f) {
-    __nv_bfloat16* row = R + panel * PAIR + r * 64;
-#pragma unroll
-    for (int jj = 0; jj < 8; ++jj) {
-        const int j = (jj + r) & 7;  // per-row rotated order: lanes on different rows, different banks
-        uint4 x = *reinterpret_cast<uint4*>(row + 8 * j);
-        uint32_t* w = reinterpret_cast<uint32_t*>(&x);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float2 v = unpack_bf16(w[i]);
-            w[i] = pack_bf16(v.x * f, v.y * f);
-        }
-        *reinterpret_cast<uint4*>(row + 8 * j) = x;
-    }
 }
 
 // sum_{c < 32} x[c] * R[r][c0 + c] for row r of a pair region (c0 a multiple
@@ -133,73 +132,156 @@ GDN_DEV float dot_row32(const float* x, const __nv_bfloat16* R, int r, int c0) {
     return acc;
 }
 
+// The chunk of this CTA at or after c (grid stride) that holds tokens, or
+// p.nchunks when none is left.
+GDN_DEV int next_chunk(const BlPtrs& p, int c) {
+    for (; c < p.nchunks; c += gridDim.x) {
+        const int bh = c / p.NT;
+        if (chunk_loc(p.seq, p.T, p.H, bh, c % p.NT).valid) break;
+    }
+    return c < p.nchunks ? c : p.nchunks;
+}
+
+struct BlChunk {
+    int cid, h, tok, L;
+    size_t row0;  // (first token of the chunk) * H + h
+};
+
+GDN_DEV BlChunk bl_chunk(const BlPtrs& p, int cid) {
+    BlChunk c;
+    c.cid = cid;
+    const int bh = cid / p.NT;
+    const ChunkLoc cl = chunk_loc(p.seq, p.T, p.H, bh, cid % p.NT);
+    c.h = bh % p.H;
+    c.tok = cl.tok;
+    c.L = cl.L;
+    c.row0 = (size_t)cl.tok * p.H + c.h;
+    return c;
+}
+
+// Loads of one buffer group of chunk c (thread 0).
+GDN_DEV void load_s(BlSmem& s, const BlPtrs& p, const BlChunk& c) {  // S0, dS
+    mbar_arrive_expect(&s.bar_s, 2 * DV * DK * 2);
+    bulk_g2s(s.R4, p.S0 + (size_t)c.cid * DV * DK, DV * DK * 2, &s.bar_s);
+    bulk_g2s(s.R5, p.dS + (size_t)c.cid * DV * DK, DV * DK * 2, &s.bar_s);
+}
+GDN_DEV void load_u(BlSmem& s, const BlPtrs& p, const BlChunk& c) {  // U (rows 0..63 of R3)
+    mbar_arrive_expect(&s.bar_u, C * DV * 2);
+    bulk_g2s(s.R3, p.U + (size_t)c.cid * C * DV, C * 64 * 2, &s.bar_u);
+    bulk_g2s(s.R3 + PAIR, p.U + (size_t)c.cid * C * DV + C * 64, C * 64 * 2, &s.bar_u);
+}
+GDN_DEV void load_tq(BlSmem& s, const BlPtrs& p, const BlChunk& c) {  // T, Q (rows 64..127 of R2)
+    mbar_arrive_expect(&s.bar_tq, (C * C + C * DK) * 2);
+    bulk_g2s(s.T, p.Tb + (size_t)c.cid * C * C, C * C * 2, &s.bar_tq);
+    tma_load_3d(s.R2 + C * 64, &p.qmap, 0, c.h, c.tok, &s.bar_tq);
+    tma_load_3d(s.R2 + PAIR + C * 64, &p.qmap, 64, c.h, c.tok, &s.bar_tq);
+}
+GDN_DEV void load_r1(BlSmem& s, const BlPtrs& p, const BlChunk& c) {  // dU, dO; W, U~
+    mbar_arrive_expect(&s.bar_r1, 2 * C * DV * 2);
+    bulk_g2s(s.R1, p.dU + (size_t)c.cid * C * DV, C * 64 * 2, &s.bar_r1);
+    bulk_g2s(s.R1 + PAIR, p.dU + (size_t)c.cid * C * DV + C * 64, C * 64 * 2, &s.bar_r1);
+    tma_load_3d(s.R1 + C * 64, &p.dOmap, 0, c.h, c.tok, &s.bar_r1);
+    tma_load_3d(s.R1 + PAIR + C * 64, &p.dOmap, 64, c.h, c.tok, &s.bar_r1);
+    mbar_arrive_expect(&s.bar_wu, (C * DK + DV * C) * 2);
+    bulk_g2s(s.W, p.W + (size_t)c.cid * C * DK, C * DK * 2, &s.bar_wu);
+    bulk_g2s(s.Ut, p.Ut + (size_t)c.cid * DV * C, DV * C * 2, &s.bar_wu);
+}
+GDN_DEV void load_k(BlSmem& s, const BlPtrs& p, const BlChunk& c) {  // K (rows 0..63 of R2)
+    mbar_arrive_expect(&s.bar_k, C * DK * 2);
+    tma_load_3d(s.R2, &p.kmap, 0, c.h, c.tok, &s.bar_k);
+    tma_load_3d(s.R2 + PAIR, &p.kmap, 64, c.h, c.tok, &s.bar_k);
+}
+// Everything chunk c reads, into L2 (thread 0, a chunk ahead of its loads).
+GDN_DEV void prefetch_chunk(const BlPtrs& p, const BlChunk& c) {
+    tma_prefetch_tile(&p.dOmap, c.h, c.tok);
+    tma_prefetch_tile(&p.qmap, c.h, c.tok);
+    tma_prefetch_tile(&p.kmap, c.h, c.tok);
+    bulk_prefetch_l2(p.U + (size_t)c.cid * C * DV, C * DV * 2);
+    bulk_prefetch_l2(p.dU + (size_t)c.cid * C * DV, C * DV * 2);
+    bulk_prefetch_l2(p.S0 + (size_t)c.cid * DV * DK, DV * DK * 2);
+    bulk_prefetch_l2(p.dS + (size_t)c.cid * DV * DK, DV * DK * 2);
+    bulk_prefetch_l2(p.Tb + (size_t)c.cid * C * C, C * C * 2);
+    bulk_prefetch_l2(p.W + (size_t)c.cid * C * DK, C * DK * 2);
+    bulk_prefetch_l2(p.Ut + (size_t)c.cid * DV * C, DV * C * 2);
+}
+
+// G (within-chunk cumsum of g) and beta of chunk c into slot b (one warp).
+GDN_DEV void load_gb(BlSmem& s, const BlPtrs& p, const BlChunk& c, int b) {
+    const int lane = threadIdx.x & 31;
+    const size_t rs = (size_t)p.H;
+    float g0 = lane < c.L ? p.g[c.row0 + lane * rs] : 0.f;
+    float g1 = lane + 32 < c.L ? p.g[c.row0 + (lane + 32) * rs] : 0.f;
+    const float b0 = lane < c.L ? p.beta[c.row0 + lane * rs] : 0.f;
+    const float b1 = lane + 32 < c.L ? p.beta[c.row0 + (lane + 32) * rs] : 0.f;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const float x0 = __shfl_up_sync(0xffffffffu, g0, o);
+        const float x1 = __shfl_up_sync(0xffffffffu, g1, o);
+        if (lane >= o) { g0 += x0; g1 += x1; }
+    }
+    g1 += __shfl_sync(0xffffffffu, g0, 31);
+    s.G[b][lane] = g0;
+    s.G[b][lane + 32] = g1;
+    s.beta[b][lane] = b0;
+    s.beta[b][lane + 32] = b1;
+}
+
+GDN_DEV void store_row32(__nv_bfloat16* dst, const float* a, float f) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int c = 0; c < 16; ++c) pk[c] = pack_bf16(f * a[2 * c], f * a[2 * c + 1]);
+#pragma unroll
+    for (int q4 = 0; q4 < 4; ++q4)
+        *reinterpret_cast<uint4*>(dst + 8 * q4) = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+}
+
+// Row t, columns c0..c0+31 (c0 a multiple of 32) of a pair region's panel, bf16.
+GDN_DEV void put_pair_row32(__nv_bfloat16* R, int t, int c0, const float* a, float f) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int c = 0; c < 16; ++c) pk[c] = pack_bf16(f * a[2 * c], f * a[2 * c + 1]);
+    __nv_bfloat16* dst = R + (c0 >> 6) * PAIR;
+#pragma unroll
+    for (int q4 = 0; q4 < 4; ++q4)
+        *reinterpret_cast<uint4*>(dst + swz<64>(t, (c0 & 63) + 8 * q4)) =
+            make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+}
+
+// 32 fp32 values back into this thread's TMEM lane (two 16-column stores).
+GDN_DEV void st_row32(uint32_t taddr, const float* a) {
+    uint32_t r0[16], r1[16];
+#pragma unroll
+    for (int c = 0; c < 16; ++c) { r0[c] = __float_as_uint(a[c]); r1[c] = __float_as_uint(a[16 + c]); }
+    tc5::st16(taddr, r0);
+    tc5::st16(taddr + 16, r1);
+}
+
 __global__ void __launch_bounds__(BL_THREADS, 1) tc5_bwd_local_kernel(const __grid_constant__ BlPtrs p) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     BlSmem& s = *reinterpret_cast<BlSmem*>(align1k(smem_raw));
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int cid = blockIdx.x;
-    const int bh = cid / p.NT, n = cid % p.NT, h = bh % p.H;
-    const ChunkLoc cl = chunk_loc(p.seq, p.T, p.H, bh, n);
-    if (!cl.valid) return;  // past the last chunk of a packed batch
-    const int L = cl.L;
-    const size_t row0 = (size_t)cl.tok * p.H + h;
-    const size_t rs = (size_t)p.H;
-
+    int cid = next_chunk(p, blockIdx.x);
+    if (cid >= p.nchunks) return;  // nothing for this CTA (before any barrier or TMEM)
+    BlChunk ch = bl_chunk(p, cid);
     if (tid == 0) {
-        mbar_init(&s.bar_ld, 1);
+        mbar_init(&s.bar_s, 1);
+        mbar_init(&s.bar_u, 1);
+        mbar_init(&s.bar_tq, 1);
+        mbar_init(&s.bar_r1, 1);
+        mbar_init(&s.bar_wu, 1);
+        mbar_init(&s.bar_k, 1);
         mbar_init(&s.bar_mma, 1);
         fence_mbar_init();
-        const int tok = cl.tok;
-        mbar_arrive_expect(&s.bar_ld, (6 * C * DK + 2 * DV * DK + C * C) * 2);
-        bulk_g2s(s.R1, p.dU + (size_t)cid * C * DV, C * 64 * 2, &s.bar_ld);
-        bulk_g2s(s.R1 + PAIR, p.dU + (size_t)cid * C * DV + C * 64, C * 64 * 2, &s.bar_ld);
-        tma_load_3d(s.R1 + C * 64, &p.dOmap, 0, h, tok, &s.bar_ld);
-        tma_load_3d(s.R1 + PAIR + C * 64, &p.dOmap, 64, h, tok, &s.bar_ld);
-        tma_load_3d(s.R2, &p.kmap, 0, h, tok, &s.bar_ld);
-        tma_load_3d(s.R2 + PAIR, &p.kmap, 64, h, tok, &s.bar_ld);
-        tma_load_3d(s.R2 + C * 64, &p.qmap, 0, h, tok, &s.bar_ld);
-        tma_load_3d(s.R2 + PAIR + C * 64, &p.qmap, 64, h, tok, &s.bar_ld);
-        bulk_g2s(s.R3, p.U + (size_t)cid * C * DV, C * 64 * 2, &s.bar_ld);
-        bulk_g2s(s.R3 + PAIR, p.U + (size_t)cid * C * DV + C * 64, C * 64 * 2, &s.bar_ld);
-        tma_load_3d(s.R3 + C * 64, &p.vmap, 0, h, tok, &s.bar_ld);
-        tma_load_3d(s.R3 + PAIR + C * 64, &p.vmap, 64, h, tok, &s.bar_ld);
-        bulk_g2s(s.R4, p.S0 + (size_t)cid * DV * DK, DV * DK * 2, &s.bar_ld);
-        bulk_g2s(s.R5, p.dS + (size_t)cid * DV * DK, DV * DK * 2, &s.bar_ld);
-        bulk_g2s(s.T, p.Tb + (size_t)cid * C * C, C * C * 2, &s.bar_ld);
-        // the chunk a wave ahead: its tiles and images wait in L2 when its CTA starts
-        const int pc = cid + p.pf_stride;
-        if (p.pf_stride > 0 && pc < (int)gridDim.x) {
-            const int pbh = pc / p.NT, pn = pc % p.NT, ph = pbh % p.H;
-            const ChunkLoc pl = chunk_loc(p.seq, p.T, p.H, pbh, pn);
-            const int ptok = pl.valid ? pl.tok : 0;
-            tma_prefetch_tile(&p.dOmap, ph, ptok);
-            tma_prefetch_tile(&p.qmap, ph, ptok);
-            tma_prefetch_tile(&p.kmap, ph, ptok);
-            tma_prefetch_tile(&p.vmap, ph, ptok);
-            bulk_prefetch_l2(p.U + (size_t)pc * C * DV, C * DV * 2);
-            bulk_prefetch_l2(p.dU + (size_t)pc * C * DV, C * DV * 2);
-            bulk_prefetch_l2(p.S0 + (size_t)pc * DV * DK, DV * DK * 2);
-            bulk_prefetch_l2(p.dS + (size_t)pc * DV * DK, DV * DK * 2);
-            bulk_prefetch_l2(p.Tb + (size_t)pc * C * C, C * C * 2);
-        }
+        load_r1(s, p, ch);
+        load_s(s, p, ch);
+        load_u(s, p, ch);
+        load_k(s, p, ch);
+        load_tq(s, p, ch);
     }
     if (warp == 0) {
         tc5::alloc(&s.tmem, BL_TCOLS);
-        float g0 = lane < L ? p.g[row0 + lane * rs] : 0.f;
-        float g1 = lane + 32 < L ? p.g[row0 + (lane + 32) * rs] : 0.f;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const float x0 = __shfl_up_sync(0xffffffffu, g0, o);
-            const float x1 = __shfl_up_sync(0xffffffffu, g1, o);
-            if (lane >= o) { g0 += x0; g1 += x1; }
-        }
-        g1 += __shfl_sync(0xffffffffu, g0, 31);
-        s.G[lane] = g0;
-        s.G[lane + 32] = g1;
-        s.beta[lane] = lane < L ? p.beta[row0 + lane * rs] : 0.f;
-        s.beta[lane + 32] = lane + 32 < L ? p.beta[row0 + (lane + 32) * rs] : 0.f;
+        load_gb(s, p, ch, 0);
     }
-    if (tid < 16) s.red2[tid] = 0.f;
     tc5::fence_before();
     __syncthreads();
     tc5::fence_after();
@@ -211,105 +293,114 @@ __global__ void __launch_bounds__(BL_THREADS, 1) tc5_bwd_local_kernel(const __gr
     const uint32_t sR1 = smem_u32(s.R1), sR2 = smem_u32(s.R2), sR3 = smem_u32(s.R3),
                    sR4 = smem_u32(s.R4), sR5 = smem_u32(s.R5), sT = smem_u32(s.T);
     constexpr uint32_t PB = PAIR * 2;  // bytes of one pair panel (the panel stride of pair regions)
-    const float Gl = s.G[C - 1];
+    const size_t rs = (size_t)p.H;
+    __nv_bfloat16* sdPG = s.R3 + C * 64;         // scale dP .* Gamma (Swz<64>), panel 0 rows 64..127
+    __nv_bfloat16* dMM = s.R3 + PAIR + C * 64;   // dMM (Swz<64>), panel 1 rows 64..127
+    float* Xs = s.Xs;
     uint32_t mph = 0;  // phase of bar_mma
-    float myG = 0.f, myB = 0.f;  // this thread's (token, column group) share of dG / dbeta
-    float myC = 0.f;             // this thread's (column, row block) share of the column sums
-    // S0 / dS space, reused once both are dead
-    float* Mf = reinterpret_cast<float*>(s.R4 + 2 * C * 64);   // M (fp32, [t][j], rotated columns)
-    float* Xs = reinterpret_cast<float*>(s.R5 + 2 * C * 64);   // transpose scratch (fp32)
-    __nv_bfloat16* dTt = s.R4;                                 // dT (Swz<64>)
-    __nv_bfloat16* Xt = s.R4 + C * 64;                         // X (Swz<64>)
-    __nv_bfloat16* sdPG = s.R5 + C * 64;                       // scale dP .* Gamma (Swz<64>)
-    __nv_bfloat16* dMM = s.R3;                                 // dMM (Swz<64>), in the U rows
-    bool ok = mbar_wait(&s.bar_ld, 0, p.status);
-    if (__syncthreads_or(!ok)) goto done;
-    // dO rows past the sequence end belong to the next sequence: zero them
-    if (L < C) {
-        for (int e = tid; e < (C - L) * 16; e += BL_THREADS) {
-            const int r = L + (e >> 4), pc = e & 15;
-            *reinterpret_cast<uint4*>(s.R1 + (pc >> 3) * PAIR + (C + r) * 64 + (pc & 7) * 8) =
-                make_uint4(0, 0, 0, 0);
-        }
-        fence_async_smem();
-    }
-    __syncthreads();
-
-    // ---- phase A1: products of the unscaled tiles ----------------------------
-    if (tid == 0) {
-        tc5::fence_after();
-#pragma unroll
-        for (int kk = 0; kk < DV / 16; ++kk)  // [dU ; dO] U^T
-            tc5::mma(tm + TC2, tc5::kmajor<128>(sR1, kk), tc5::kmajor<128>(sR3, kk), ID_N64, kk > 0);
-#pragma unroll
-        for (int kk = 0; kk < DK / 16; ++kk)  // [K ; Q] K^T
-            tc5::mma(tm + TC1, tc5::kmajor<128>(sR2, kk), tc5::kmajor<128>(sR2, kk), ID_N64, kk > 0);
-#pragma unroll
-        for (int kk = 0; kk < DV / 16; ++kk)  // [dU ; dO] V^T
-            tc5::mma(tm + TU, tc5::kmajor<128>(sR1, kk), tc5::kmajor<128>(sR3 + C * 128, kk), ID_N64, kk > 0);
-        tc5::commit(&s.bar_mma);
-    }
-    ok = mbar_wait(&s.bar_mma, mph, p.status);
-    mph ^= 1;
-    if (__syncthreads_or(!ok)) goto done;
-    // dO rows *= scale e^{G_i} (the dq rows), U rows *= e^{G_last - G_i} (the dk rows)
-    if (tid < 256) {
-        const int r = (tid >> 1) & 63, pn = tid & 1;
-        if (tid < 128) scale_pair_row(s.R1, C + r, pn, p.scale * __expf(s.G[r]));
-        else scale_pair_row(s.R3, r, pn, __expf(Gl - s.G[r]));
-    }
-    fence_async_smem();
-    tc5::fence_before();
-    __syncthreads();
-    // ---- phase A2: [dU ; dO'] S0 and [U' ; V] dS -------------------------------
-    if (tid == 0) {
-        tc5::fence_after();
-#pragma unroll
-        for (int kk = 0; kk < DV / 16; ++kk)
-            tc5::mma(tm + TA, tc5::kmajor<128>(sR1, kk), tc5::mnmajor(sR4, kk, 128 * 128), ID_N128_BMN, kk > 0);
-#pragma unroll
-        for (int kk = 0; kk < DV / 16; ++kk)
-            tc5::mma(tm + TB, tc5::kmajor<128>(sR3, kk), tc5::mnmajor(sR5, kk, 128 * 128), ID_N128_BMN, kk > 0);
-        tc5::commit(&s.bar_mma);
-    }
-    ok = mbar_wait(&s.bar_mma, mph, p.status);
-    mph ^= 1;
-    if (__syncthreads_or(!ok)) goto done;
-    tc5::fence_after();
-    {
-        // ---- <dS, S0> (before S0 / dS space is reused) ------------------------
-        float ss = 0.f;
-        for (int e = tid; e < DV * DK / 8; e += BL_THREADS) {
-            const uint4 x = reinterpret_cast<const uint4*>(s.R5)[e];
-            const uint4 y = reinterpret_cast<const uint4*>(s.R4)[e];
-            const uint32_t xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
-#pragma unroll
-            for (int t = 0; t < 4; ++t) {
-                const float2 a2 = unpack_bf16(xs[t]), b2 = unpack_bf16(ys[t]);
-                ss += a2.x * b2.x + a2.y * b2.y;
+    bool ok = true;
+    for (int it = 0;; ++it) {
+        const uint32_t lp = it & 1;  // phase of the load barriers for this chunk
+        const int L = ch.L;
+        const size_t row0 = ch.row0;
+        const float* G = s.G[it & 1];
+        const float* beta = s.beta[it & 1];
+        const float Gl = G[C - 1];
+        const int ncid = next_chunk(p, cid + gridDim.x);
+        const bool has_next = ncid < p.nchunks;
+        const BlChunk nch = bl_chunk(p, has_next ? ncid : cid);
+        float myG = 0.f, myB = 0.f;  // this thread's (token, column group) share of dG / dbeta
+        float myC = 0.f;             // this thread's (column, row block) share of the column sums
+        if (tid == 0 && has_next) prefetch_chunk(p, nch);
+        if (warp == 2 && has_next) {  // the next chunk's g and beta rows, into L2
+            for (int t = lane; t < nch.L; t += 32) {
+                prefetch_l2(p.g + nch.row0 + (size_t)t * rs);
+                prefetch_l2(p.beta + nch.row0 + (size_t)t * rs);
             }
         }
-        ss = warp_sum(ss);
-        if (lane == 0) s.red[warp] = ss;
-    }
-    __syncthreads();  // S0 and dS are dead from here on
-    {
-        // ---- epilogue A -------------------------------------------------------
+        if (tid < 16) s.red2[tid] = 0.f;
+        ok = mbar_wait(&s.bar_r1, lp, p.status) && mbar_wait(&s.bar_s, lp, p.status) &&
+             mbar_wait(&s.bar_u, lp, p.status) && mbar_wait(&s.bar_tq, lp, p.status);
+        if (__syncthreads_or(!ok)) break;
+        // dO rows past the sequence end belong to the next sequence: zero them
+        if (L < C) {
+            for (int e = tid; e < (C - L) * 16; e += BL_THREADS) {
+                const int r = L + (e >> 4), pc = e & 15;
+                *reinterpret_cast<uint4*>(s.R1 + (pc >> 3) * PAIR + (C + r) * 64 + (pc & 7) * 8) =
+                    make_uint4(0, 0, 0, 0);
+            }
+            fence_async_smem();
+        }
+        __syncthreads();
+        // ---- phase A: every product of the loaded tiles --------------------------------
+        bool kfail = false;
+        if (tid == 0) {
+            tc5::fence_after();
+#pragma unroll
+            for (int kk = 0; kk < DV / 16; ++kk)  // [dU ; dO] S0 -> [-dW ; dO S0]
+                tc5::mma(tm + TA, tc5::kmajor<128>(sR1, kk), tc5::mnmajor(sR4, kk, 128 * 128), ID_N128_BMN,
+                         kk > 0);
+#pragma unroll
+            for (int kk = 0; kk < DV / 16; ++kk)  // [U ; .] dS
+                tc5::mma(tm + TB, tc5::kmajor<128>(sR3, kk), tc5::mnmajor(sR5, kk, 128 * 128), ID_N128_BMN,
+                         kk > 0);
+#pragma unroll
+            for (int kk = 0; kk < DV / 16; ++kk)  // [dU ; dO] U^T
+                tc5::mma(tm + TC2, tc5::kmajor<128>(sR1, kk), tc5::kmajor<128>(sR3, kk), ID_N64, kk > 0);
+            if (mbar_wait(&s.bar_k, lp, p.status)) {
+#pragma unroll
+                for (int kk = 0; kk < DK / 16; ++kk)  // [K ; Q] K^T
+                    tc5::mma(tm + TC1, tc5::kmajor<128>(sR2, kk), tc5::kmajor<128>(sR2, kk), ID_N64, kk > 0);
+            } else {
+                kfail = true;
+            }
+            tc5::commit(&s.bar_mma);
+        }
+        {   // <dS, S0> under the products (both are only read until the next chunk's loads)
+            float ss = 0.f;
+            for (int e = tid; e < DV * DK / 8; e += BL_THREADS) {
+                const uint4 x = reinterpret_cast<const uint4*>(s.R5)[e];
+                const uint4 y = reinterpret_cast<const uint4*>(s.R4)[e];
+                const uint32_t xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    const float2 a2 = unpack_bf16(xs[t]), b2 = unpack_bf16(ys[t]);
+                    ss += a2.x * b2.x + a2.y * b2.y;
+                }
+            }
+            ss = warp_sum(ss);
+            if (lane == 0) s.red[warp] = ss;
+        }
+        fence_async_smem();
+        ok = mbar_wait(&s.bar_mma, mph, p.status);
+        mph ^= 1;
+        if (__syncthreads_or(!ok || kfail)) break;
+        tc5::fence_after();
+        // S0, dS and U are done with: the next chunk's go in
+        if (tid == 0 && has_next) {
+            load_s(s, p, nch);
+            load_u(s, p, nch);
+        }
+        // ---- epilogue A --------------------------------------------------------------
         if (q >= 2) {
-            // token i: dP, Q K^T (columns 16cg..) -> sdPG and hP; <dO' S0, q_i> (columns 32cg..)
+            // token i: dP, Q K^T (columns 16cg..) -> sdPG and hP; dq accumulator
+            // (columns 32cg..) *= scale e^{G_i}, and <scale e^{G_i} dO S0 row i, q_i>
             const int i = row;
-            const float Gi = s.G[i];
+            const float Gi = G[i], fi = p.scale * __expf(Gi);
             float dp[16], qk[16], x[32];
             tc5::ld16(dp, trow + TC2 + 16 * cg);
             tc5::ld16(qk, trow + TC1 + 16 * cg);
             ld_row32(x, trow + TA + 32 * cg);
             tc5::wait_ld();
+#pragma unroll
+            for (int c = 0; c < 32; ++c) x[c] *= fi;
+            st_row32(trow + TA + 32 * cg, x);
             float hrow = 0.f;
             uint32_t pk[8];
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
                 const int j = 16 * cg + c;
-                const float g = j <= i ? p.scale * dp[c] * __expf(Gi - s.G[j]) : 0.f;  // scale dP .* Gamma
+                const float g = j <= i ? p.scale * dp[c] * __expf(Gi - G[j]) : 0.f;  // scale dP .* Gamma
                 const float hp = g * qk[c];                    // dP .* (scale Q K^T .* Gamma)
                 hrow += hp;
                 Xs[i * 64 + ((j + i) & 63)] = hp;              // column sums below
@@ -319,274 +410,242 @@ __global__ void __launch_bounds__(BL_THREADS, 1) tc5_bwd_local_kernel(const __gr
             for (int c = 0; c < 8; ++c) pk[c] = pack_bf16(dp[2 * c], dp[2 * c + 1]);
             *reinterpret_cast<uint4*>(sdPG + swz<64>(i, 16 * cg)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
             *reinterpret_cast<uint4*>(sdPG + swz<64>(i, 16 * cg + 8)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-            // scale e^{G_i} <dO S0 row i, q_i>, this thread's 32 columns
             const float dqq = dot_row32(x, s.R2, C + i, 32 * cg);
             myG += hrow + dqq;
         } else {
-            // token t: -dW (columns 32cg..) -> dW (bf16, into the dO rows of R1);
-            // M (columns 16cg..); <etl dKt row t, k_t> (columns 32cg..)
+            // token t: -dW (columns 32cg..) -> dW (bf16, into the dO rows of R1); the dk
+            // accumulator (U dS, columns 32cg..) *= etl_t, and <etl dKt row t, k_t>
             const int t = row;
-            const float Gt = s.G[t];
-            float x[32], kk[16], y[32];
+            float x[32], y[32];
             ld_row32(x, trow + TA + 32 * cg);
-            tc5::ld16(kk, trow + TC1 + 16 * cg);
             ld_row32(y, trow + TB + 32 * cg);
             tc5::wait_ld();
-            uint32_t pk[16];
+            const float et = __expf(Gl - G[t]);
 #pragma unroll
-            for (int c = 0; c < 16; ++c) pk[c] = pack_bf16(-x[2 * c], -x[2 * c + 1]);
-            __nv_bfloat16* dst = s.R1 + (cg >> 1) * PAIR;  // panel of key columns 32cg..
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4)
-                *reinterpret_cast<uint4*>(dst + swz<64>(C + t, 32 * (cg & 1) + 8 * q4)) =
-                    make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
-#pragma unroll
-            for (int c = 0; c < 16; ++c) {
-                const int j = 16 * cg + c;
-                Mf[t * 64 + ((j + t) & 63)] = j < t ? kk[c] * __expf(Gt - s.G[j]) : 0.f;
-            }
+            for (int c = 0; c < 32; ++c) y[c] *= et;
+            st_row32(trow + TB + 32 * cg, y);
+            put_pair_row32(s.R1 + C * 64, t, 32 * cg, x, -1.f);
             float hk = dot_row32(y, s.R2, t, 32 * cg);
             myG -= hk;  // -etl_t <dKt_t, k_t>; the same enters dG_last
             hk = warp_sum(hk);
             if (lane == 0) s.red2[warp] = hk;
         }
-    }
-    fence_async_smem();
-    tc5::fence_before();
-    __syncthreads();
-    {   // column sums of hP: dG_j -= sum_i hP_ij (eight row blocks per column)
-        const int j = tid & 63, pb = tid >> 6;
+        tc5::wait_st();
+        fence_async_smem();
+        tc5::fence_before();
+        __syncthreads();
+        {   // column sums of hP: dG_j -= sum_i hP_ij (eight row blocks per column)
+            const int j = tid & 63, pb = tid >> 6;
 #pragma unroll
-        for (int i = 8 * pb; i < 8 * pb + 8; ++i) myC -= Xs[i * 64 + ((j + i) & 63)];
-    }
-    // ---- phase B: [dW ; .] K^T -----------------------------------------------
-    if (tid == 0) {
+            for (int i = 8 * pb; i < 8 * pb + 8; ++i) myC -= Xs[i * 64 + ((j + i) & 63)];
+        }
+        // ---- phase E1: Gk = T^T dW, Gv = T^T dU; dq += [. ; sdPG] K; dk += sdPG^T Q
+        if (tid == 0) {
+            tc5::fence_after();
+            const uint32_t ssdPG = smem_u32(sdPG);
+#pragma unroll
+            for (int kk = 0; kk < C / 16; ++kk)
+                tc5::mma(tm + TKG, tc5::mnmajor(sT, kk, C * 128), tc5::mnmajor(sR1 + C * 128, kk, PB),
+                         ID_N128_AMN_BMN, kk > 0);
+#pragma unroll
+            for (int kk = 0; kk < C / 16; ++kk)
+                tc5::mma(tm + TVB, tc5::mnmajor(sT, kk, C * 128), tc5::mnmajor(sR1, kk, PB), ID_N128_AMN_BMN,
+                         kk > 0);
+            // (rows 0..63 of this A view are the 8 KB before sdPG)
+#pragma unroll
+            for (int kk = 0; kk < C / 16; ++kk)
+                tc5::mma(tm + TA, tc5::kmajor<128>(ssdPG - C * 128, kk), tc5::mnmajor(sR2, kk, PB), ID_N128_BMN,
+                         true);
+#pragma unroll
+            for (int kk = 0; kk < C / 16; ++kk)
+                tc5::mma(tm + TB, tc5::mnmajor(ssdPG, kk, C * 128), tc5::mnmajor(sR2 + C * 128, kk, PB),
+                         ID_N128_AMN_BMN, true);
+            tc5::commit(&s.bar_mma);
+        }
+        ok = mbar_wait(&s.bar_mma, mph, p.status);
+        mph ^= 1;
+        if (__syncthreads_or(!ok)) break;
         tc5::fence_after();
+        if (tid == 0 && has_next) load_tq(s, p, nch);  // T and Q are done with
+        // ---- epilogue E1: Gk, Gv -> bf16 A operands (R1); dv; <Gk_t, k_t>, <Gv_t, v_t>;
+        // dq (complete after E1) -----------------------------------------------------
+        if (q < 2) {
+            const int t = row;
+            const float bt = beta[t], egt = __expf(G[t]);
+            uint4 vr[4];  // v_t, columns 32cg.. (from L2)
+            if (t < L) {
+                const uint4* vp = reinterpret_cast<const uint4*>(p.v + (row0 + (size_t)t * rs) * DV + 32 * cg);
 #pragma unroll
-        for (int kk = 0; kk < DK / 16; ++kk)
-            tc5::mma(tm + TW, tc5::kmajor<128>(sR1 + C * 128, kk), tc5::kmajor<128>(sR2, kk), ID_N64, kk > 0);
-        tc5::commit(&s.bar_mma);
-    }
-    ok = mbar_wait(&s.bar_mma, mph, p.status);
-    mph ^= 1;
-    if (__syncthreads_or(!ok)) goto done;
-    tc5::fence_after();
-    // ---- epilogue B: dT row t = beta_j (e^{G_j} dW K^T + dU V^T)_tj -----------
-    if (q < 2) {
-        const int t = row;
-        float tw[16], tu[16];
-        tc5::ld16(tw, trow + TW + 16 * cg);
-        tc5::ld16(tu, trow + TU + 16 * cg);
-        tc5::wait_ld();
-        uint32_t pk[8];
+                for (int j = 0; j < 4; ++j) vr[j] = __ldg(vp + j);
+            } else {
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            const int j0 = 16 * cg + 2 * c;
-            const float d0 = s.beta[j0] * (__expf(s.G[j0]) * tw[2 * c] + tu[2 * c]);
-            const float d1 = s.beta[j0 + 1] * (__expf(s.G[j0 + 1]) * tw[2 * c + 1] + tu[2 * c + 1]);
-            pk[c] = pack_bf16(d0, d1);
+                for (int j = 0; j < 4; ++j) vr[j] = make_uint4(0, 0, 0, 0);
+            }
+            float gk[32], gv[32];
+            ld_row32(gk, trow + TKG + 32 * cg);
+            ld_row32(gv, trow + TVB + 32 * cg);
+            tc5::wait_ld();
+            const float hk = dot_row32(gk, s.R2, t, 32 * cg);
+            float hv = 0.f;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const uint32_t w[4] = {vr[j].x, vr[j].y, vr[j].z, vr[j].w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float2 f = unpack_bf16(w[i]);
+                    hv = fmaf(gv[8 * j + 2 * i], f.x, hv);
+                    hv = fmaf(gv[8 * j + 2 * i + 1], f.y, hv);
+                }
+            }
+            // Gk: rows 0..63 of the two K-major panels of R1; Gv: the same from 8 KB on
+            put_pair_row32(s.R1, t, 32 * cg, gk, 1.f);
+            put_pair_row32(s.R1 + C * 64, t, 32 * cg, gv, 1.f);
+            if (t < L) store_row32(p.dv + (row0 + (size_t)t * rs) * DV + 32 * cg, gv, bt);
+            myB += egt * hk + hv;
+            myG += bt * egt * hk;
+        } else {
+            const int i = row;
+            float a[32];
+            ld_row32(a, trow + TA + 32 * cg);
+            tc5::wait_ld();
+            if (i < L) store_row32(p.dq + (row0 + (size_t)i * rs) * DK + 32 * cg, a, 1.f);
         }
-        *reinterpret_cast<uint4*>(dTt + swz<64>(t, 16 * cg)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        *reinterpret_cast<uint4*>(dTt + swz<64>(t, 16 * cg + 8)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-    }
-    fence_async_smem();
-    tc5::fence_before();
-    __syncthreads();
-    // ---- phase C1: X = [dT ; .] T^T ---------------------------------------------
-    if (tid == 0) {
+        fence_async_smem();
+        tc5::fence_before();
+        ok = mbar_wait(&s.bar_wu, lp, p.status);
+        if (__syncthreads_or(!ok)) break;
+        // ---- phase C: [Gk ; .] W^T + [Gv ; .] U~^T = T^T dT T^T; [K ; .] K^T again -------
+        if (tid == 0) {
+            tc5::fence_after();
+            const uint32_t sW = smem_u32(s.W), sUt = smem_u32(s.Ut);
+#pragma unroll
+            for (int kk = 0; kk < DK / 16; ++kk)
+                tc5::mma(tm + TD, tc5::kmajor<128>(sR1, kk), tc5::kmajor<C>(sW, kk), ID_N64, kk > 0);
+#pragma unroll
+            for (int kk = 0; kk < DV / 16; ++kk)
+                tc5::mma(tm + TD, tc5::kmajor<128>(sR1 + C * 128, kk), tc5::mnmajor(sUt, kk, C * 128),
+                         ID_N64_BMN, true);
+#pragma unroll
+            for (int kk = 0; kk < DK / 16; ++kk)
+                tc5::mma(tm + TKK, tc5::kmajor<128>(sR2, kk), tc5::kmajor<128>(sR2, kk), ID_N64, kk > 0);
+            tc5::commit(&s.bar_mma);
+        }
+        ok = mbar_wait(&s.bar_mma, mph, p.status);
+        mph ^= 1;
+        if (__syncthreads_or(!ok)) break;
         tc5::fence_after();
+        if (tid == 0 && has_next) load_r1(s, p, nch);  // R1, W and U~ are done with
+        // ---- epilogue D: dA = strict_lower(-(Gk W^T + Gv U~^T)); M = K K^T .* Gamma;
+        // dMM; hA; dbeta and dG terms --------------------------------------------------
+        if (q < 2) {
+            const int i = row;
+            const float Gi = G[i], bi = beta[i];
+            float x[16], kk[16];
+            tc5::ld16(x, trow + TD + 16 * cg);
+            tc5::ld16(kk, trow + TKK + 16 * cg);
+            tc5::wait_ld();
+            float hrow = 0.f, brow = 0.f;
+            uint32_t pk[8];
 #pragma unroll
-        for (int kk = 0; kk < C / 16; ++kk)
-            tc5::mma(tm + TC1, tc5::kmajor<128>(smem_u32(dTt), kk), tc5::kmajor<C>(sT, kk), ID_N64, kk > 0);
-        tc5::commit(&s.bar_mma);
-    }
-    ok = mbar_wait(&s.bar_mma, mph, p.status);
-    mph ^= 1;
-    if (__syncthreads_or(!ok)) goto done;
-    tc5::fence_after();
-    if (q < 2) {
-        const int t = row;
-        float x[16];
-        tc5::ld16(x, trow + TC1 + 16 * cg);
-        tc5::wait_ld();
-        uint32_t pk[8];
+            for (int c = 0; c < 16; ++c) {
+                const int j = 16 * cg + c;
+                const float gam = j < i ? __expf(Gi - G[j]) : 0.f;
+                const float dA = j < i ? -x[c] : 0.f;
+                const float m = kk[c] * gam;  // K K^T .* Gamma (strict lower)
+                brow += dA * m;
+                const float hA = dA * bi * m;
+                hrow += hA;
+                Xs[i * 64 + ((j + i) & 63)] = hA;
+                x[c] = dA * bi * gam;  // dMM
+            }
 #pragma unroll
-        for (int c = 0; c < 8; ++c) pk[c] = pack_bf16(x[2 * c], x[2 * c + 1]);
-        *reinterpret_cast<uint4*>(Xt + swz<64>(t, 16 * cg)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        *reinterpret_cast<uint4*>(Xt + swz<64>(t, 16 * cg + 8)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-    }
-    fence_async_smem();
-    tc5::fence_before();
-    __syncthreads();
-    // ---- phase C2: T^T X ----------------------------------------------------------
-    if (tid == 0) {
+            for (int c = 0; c < 8; ++c) pk[c] = pack_bf16(x[2 * c], x[2 * c + 1]);
+            *reinterpret_cast<uint4*>(dMM + swz<64>(i, 16 * cg)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            *reinterpret_cast<uint4*>(dMM + swz<64>(i, 16 * cg + 8)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            myG += hrow;
+            myB += brow;
+        }
+        fence_async_smem();
+        tc5::fence_before();
+        __syncthreads();
+        // ---- phase E2: dk += dMM K + dMM^T K ---------------------------------------------
+        if (tid == 0) {
+            tc5::fence_after();
+            const uint32_t sdMM = smem_u32(dMM);
+#pragma unroll
+            for (int kk = 0; kk < C / 16; ++kk)
+                tc5::mma(tm + TB, tc5::kmajor<128>(sdMM, kk), tc5::mnmajor(sR2, kk, PB), ID_N128_BMN, true);
+#pragma unroll
+            for (int kk = 0; kk < C / 16; ++kk)
+                tc5::mma(tm + TB, tc5::mnmajor(sdMM, kk, C * 128), tc5::mnmajor(sR2, kk, PB), ID_N128_AMN_BMN,
+                         true);
+            tc5::commit(&s.bar_mma);
+        }
+        {   // column sums of hA (under the E2 products): dG_j -= sum_i hA_ij
+            const int j = tid & 63, pb = tid >> 6;
+#pragma unroll
+            for (int i = 8 * pb; i < 8 * pb + 8; ++i) myC -= Xs[i * 64 + ((j + i) & 63)];
+        }
+        ok = mbar_wait(&s.bar_mma, mph, p.status);
+        mph ^= 1;
+        if (__syncthreads_or(!ok)) break;
         tc5::fence_after();
+        if (tid == 0 && has_next) load_k(s, p, nch);  // K is done with
+        // ---- epilogue E2: dk = TB + beta e^G .* Gk; the next chunk's G and beta ----------
+        if (q < 2) {
+            const int t = row;
+            const float f = beta[t] * __expf(G[t]);
+            float a[32], kg[32];
+            ld_row32(a, trow + TB + 32 * cg);
+            ld_row32(kg, trow + TKG + 32 * cg);
+            tc5::wait_ld();
 #pragma unroll
-        for (int kk = 0; kk < C / 16; ++kk)
-            tc5::mma(tm + TC2, tc5::mnmajor(sT, kk, C * 128), tc5::mnmajor(smem_u32(Xt), kk, C * 128),
-                     ID_N64_AMN_BMN, kk > 0);
-        tc5::commit(&s.bar_mma);
-    }
-    ok = mbar_wait(&s.bar_mma, mph, p.status);
-    mph ^= 1;
-    if (__syncthreads_or(!ok)) goto done;
-    tc5::fence_after();
-    // ---- epilogue D: dA = strict_lower(-T^T X); dMM; hA; dbeta and dG terms ----
-    if (q < 2) {
-        const int i = row;
-        const float Gi = s.G[i], bi = s.beta[i];
-        float x[16];
-        tc5::ld16(x, trow + TC2 + 16 * cg);
-        tc5::wait_ld();
-        float hrow = 0.f, brow = 0.f;
-        uint32_t pk[8];
-#pragma unroll
-        for (int c = 0; c < 16; ++c) {
-            const int j = 16 * cg + c;
-            const float dA = j < i ? -x[c] : 0.f;
-            const float m = Mf[i * 64 + ((j + i) & 63)];  // K K^T .* Gamma (strict lower)
-            brow += dA * m;
-            const float hA = dA * bi * m;
-            hrow += hA;
-            Xs[i * 64 + ((j + i) & 63)] = hA;
-            x[c] = j < i ? dA * bi * __expf(Gi - s.G[j]) : 0.f;  // dMM
+            for (int c = 0; c < 32; ++c) a[c] = fmaf(f, kg[c], a[c]);
+            if (t < L) store_row32(p.dk + (row0 + (size_t)t * rs) * DK + 32 * cg, a, 1.f);
+        } else if (warp == 2 && has_next) {
+            load_gb(s, p, nch, (it + 1) & 1);
         }
+        // ---- per-token sums in a fixed order: dG (own-row terms + column terms),
+        // dbeta; dg = reverse cumsum of dG ------------------------------------------------
+        s.pG[cg + 4 * (q >> 1)][row] = myG;
+        if (q < 2) s.pB[cg][row] = myB;
+        s.pC[tid >> 6][tid & 63] = myC;
+        __syncthreads();
+        if (warp < 2) {
+            const int t = tid;
+            float dG = 0.f, dB = 0.f;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) pk[c] = pack_bf16(x[2 * c], x[2 * c + 1]);
-        *reinterpret_cast<uint4*>(dMM + swz<64>(i, 16 * cg)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        *reinterpret_cast<uint4*>(dMM + swz<64>(i, 16 * cg + 8)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-        myG += hrow;
-        myB += brow;
-    }
-    fence_async_smem();
-    tc5::fence_before();
-    __syncthreads();
-    {   // column sums of hA: dG_j -= sum_i hA_ij
-        const int j = tid & 63, pb = tid >> 6;
+            for (int k = 0; k < 8; ++k) dG += s.pG[k][t] + s.pC[k][t];
 #pragma unroll
-        for (int i = 8 * pb; i < 8 * pb + 8; ++i) myC -= Xs[i * 64 + ((j + i) & 63)];
-    }
-    // ---- phase E: the remaining products --------------------------------------------
-    if (tid == 0) {
-        tc5::fence_after();
-        const uint32_t sdMM = smem_u32(dMM), ssdPG = smem_u32(sdPG);
-        // dk += dMM K + dMM^T K + sdPG^T Q
+            for (int k = 0; k < 4; ++k) dB += s.pB[k][t];
+            if (t == C - 1) {  // G_last: e^{G_last} <dS, S0> + sum_i etl_i <dKt_i, k_i>
+                float ss = 0.f, la = 0.f;
 #pragma unroll
-        for (int kk = 0; kk < C / 16; ++kk)
-            tc5::mma(tm + TB, tc5::kmajor<128>(sdMM, kk), tc5::mnmajor(sR2, kk, PB), ID_N128_BMN, true);
+                for (int w = 0; w < 16; ++w) { ss += s.red[w]; la += s.red2[w]; }
+                dG += __expf(Gl) * ss + la;
+            }
+            float x = dG;
 #pragma unroll
-        for (int kk = 0; kk < C / 16; ++kk)
-            tc5::mma(tm + TB, tc5::mnmajor(sdMM, kk, C * 128), tc5::mnmajor(sR2, kk, PB), ID_N128_AMN_BMN, true);
-#pragma unroll
-        for (int kk = 0; kk < C / 16; ++kk)
-            tc5::mma(tm + TB, tc5::mnmajor(ssdPG, kk, C * 128), tc5::mnmajor(sR2 + C * 128, kk, PB),
-                     ID_N128_AMN_BMN, true);
-        // dq += [. ; sdPG] K   (rows 0..63 of the A view are the 8 KB before sdPG)
-#pragma unroll
-        for (int kk = 0; kk < C / 16; ++kk)
-            tc5::mma(tm + TA, tc5::kmajor<128>(ssdPG - C * 128, kk), tc5::mnmajor(sR2, kk, PB), ID_N128_BMN, true);
-        // T^T dW and T^T dU
-#pragma unroll
-        for (int kk = 0; kk < C / 16; ++kk)
-            tc5::mma(tm + TKG, tc5::mnmajor(sT, kk, C * 128), tc5::mnmajor(sR1 + C * 128, kk, PB),
-                     ID_N128_AMN_BMN, kk > 0);
-#pragma unroll
-        for (int kk = 0; kk < C / 16; ++kk)
-            tc5::mma(tm + TVB, tc5::mnmajor(sT, kk, C * 128), tc5::mnmajor(sR1, kk, PB), ID_N128_AMN_BMN, kk > 0);
-        tc5::commit(&s.bar_mma);
-    }
-    ok = mbar_wait(&s.bar_mma, mph, p.status);
-    mph ^= 1;
-    if (__syncthreads_or(!ok)) goto done;
-    tc5::fence_after();
-    // ---- epilogue E: dk, dv, dq (columns 32cg..); dbeta / dG terms -------------------
-    if (q < 2) {
-        const int t = row;
-        const float bt = s.beta[t], egt = __expf(s.G[t]);
-        float a[32], kg[32];
-        ld_row32(a, trow + TB + 32 * cg);
-        ld_row32(kg, trow + TKG + 32 * cg);
-        tc5::wait_ld();
-        const float hk = dot_row32(kg, s.R2, t, 32 * cg);
-        uint32_t pk[16];
-#pragma unroll
-        for (int c = 0; c < 32; ++c) a[c] = fmaf(bt * egt, kg[c], a[c]);
-#pragma unroll
-        for (int c = 0; c < 16; ++c) pk[c] = pack_bf16(a[2 * c], a[2 * c + 1]);
-        if (t < L) {
-            __nv_bfloat16* dkp = p.dk + (row0 + (size_t)t * rs) * DK + 32 * cg;
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4)
-                *reinterpret_cast<uint4*>(dkp + 8 * q4) =
-                    make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+            for (int o = 1; o < 32; o <<= 1) {
+                const float y = __shfl_down_sync(0xffffffffu, x, o);
+                if (lane + o < 32) x += y;
+            }
+            s.dgs[t] = x;  // per-warp suffix sums
+            s.pB[0][t] = dB;
         }
-        ld_row32(a, trow + TVB + 32 * cg);
-        tc5::wait_ld();
-        const float hv = dot_row32(a, s.R3, C + t, 32 * cg);
-#pragma unroll
-        for (int c = 0; c < 16; ++c) pk[c] = pack_bf16(bt * a[2 * c], bt * a[2 * c + 1]);
-        if (t < L) {
-            __nv_bfloat16* dvp = p.dv + (row0 + (size_t)t * rs) * DV + 32 * cg;
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4)
-                *reinterpret_cast<uint4*>(dvp + 8 * q4) =
-                    make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+        __syncthreads();
+        if (tid < C) {
+            const float x = s.dgs[tid] + (tid < 32 ? s.dgs[32] : 0.f);
+            if (tid < L) {
+                p.dg[row0 + (size_t)tid * rs] = x;
+                p.dbeta[row0 + (size_t)tid * rs] = s.pB[0][tid];
+            }
         }
-        myB += egt * hk + hv;
-        myG += bt * egt * hk;
-    } else {
-        const int i = row;
-        float a[32];
-        ld_row32(a, trow + TA + 32 * cg);
-        tc5::wait_ld();
-        uint32_t pk[16];
-#pragma unroll
-        for (int c = 0; c < 16; ++c) pk[c] = pack_bf16(a[2 * c], a[2 * c + 1]);
-        if (i < L) {
-            __nv_bfloat16* dqp = p.dq + (row0 + (size_t)i * rs) * DK + 32 * cg;
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4)
-                *reinterpret_cast<uint4*>(dqp + 8 * q4) =
-                    make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
-        }
+        __syncthreads();  // the sums' scratch and this chunk's G are free
+        if (!has_next) break;
+        cid = ncid;
+        ch = nch;
     }
-    // ---- per-token sums in a fixed order: dG (own-row terms + column terms),
-    // dbeta; dg = reverse cumsum of dG -------------------------------------------
-    s.pG[cg + 4 * (q >> 1)][row] = myG;
-    if (q < 2) s.pB[cg][row] = myB;
-    s.pC[tid >> 6][tid & 63] = myC;
-    __syncthreads();
-    if (warp < 2) {
-        const int t = tid;
-        float dG = 0.f, dB = 0.f;
-#pragma unroll
-        for (int k = 0; k < 8; ++k) dG += s.pG[k][t] + s.pC[k][t];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) dB += s.pB[k][t];
-        if (t == C - 1) {  // G_last: e^{G_last} <dS, S0> + sum_i etl_i <dKt_i, k_i>
-            float ss = 0.f, la = 0.f;
-#pragma unroll
-            for (int w = 0; w < 16; ++w) { ss += s.red[w]; la += s.red2[w]; }
-            dG += __expf(Gl) * ss + la;
-        }
-        float x = dG;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const float y = __shfl_down_sync(0xffffffffu, x, o);
-            if (lane + o < 32) x += y;
-        }
-        s.dgs[t] = x;  // per-warp suffix sums
-        s.pB[0][t] = dB;
-    }
-    __syncthreads();
-    if (tid < C) {
-        const float x = s.dgs[tid] + (tid < 32 ? s.dgs[32] : 0.f);
-        if (tid < L) {
-            p.dg[row0 + (size_t)tid * rs] = x;
-            p.dbeta[row0 + (size_t)tid * rs] = s.pB[0][tid];
-        }
-    }
-done:
     tc5::fence_before();
     __syncthreads();
     if (warp == 0) {
@@ -601,24 +660,27 @@ namespace tc {
 bool launch_bwd_local5(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& cp, const void* dO,
                        void* dq, void* dk, void* dv, float* dg, float* dbeta, void* ws, cudaStream_t st) {
     BlPtrs lp{};
-    lp.qmap = cp.qmap; lp.kmap = cp.kmap; lp.vmap = cp.vmap;
+    lp.qmap = cp.qmap; lp.kmap = cp.kmap;
     if (!encode_token_map(&lp.dOmap, dO, d.B, d.T, d.H)) return false;
     char* base = (char*)ws;
-    lp.g = cp.g; lp.beta = cp.beta; lp.status = cp.status;
+    lp.g = cp.g; lp.beta = cp.beta; lp.v = cp.v; lp.status = cp.status;
     lp.S0 = (const __nv_bfloat16*)(base + L.S0);
     lp.U = (const __nv_bfloat16*)(base + L.U);
     lp.dS = (const __nv_bfloat16*)(base + L.dS);
     lp.dU = (const __nv_bfloat16*)(base + L.dU);
     lp.Tb = cp.Tb;
+    lp.W = cp.W; lp.Ut = cp.Ut;
     lp.dq = (__nv_bfloat16*)dq; lp.dk = (__nv_bfloat16*)dk; lp.dv = (__nv_bfloat16*)dv;
     lp.dg = dg; lp.dbeta = dbeta;
     lp.B = d.B; lp.T = d.T; lp.H = d.H; lp.NT = L.NT; lp.scale = d.scale;
+    lp.nchunks = (int)L.nchunks;
     lp.seq = cp.seq;
-    lp.pf_stride = sm_count();  // one CTA per SM
+    if (L.nchunks == 0) return true;
+    // persistent: one CTA per SM, each taking every gridDim.x-th chunk
+    const unsigned grid = (unsigned)std::min<size_t>(L.nchunks, (size_t)sm_count());
     const int smem = sizeof(BlSmem) + 1024;
     cudaFuncSetAttribute(tc5_bwd_local_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    GDN_LAUNCH("tc5_bwd_local", st,
-               tc5_bwd_local_kernel<<<(unsigned)L.nchunks, BL_THREADS, smem, st>>>(lp));
+    GDN_LAUNCH("tc5_bwd_local", st, tc5_bwd_local_kernel<<<grid, BL_THREADS, smem, st>>>(lp));
     return true;
 }
 }  // namespace tc
