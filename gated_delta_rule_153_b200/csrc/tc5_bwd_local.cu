@@ -96,7 +96,7 @@ struct alignas(1024) BlSmem {
 };
 
 struct BlPtrs {
-    CUtensorMap qmap, kmap, dOmap;
+    CUtensorMap qmap, kmap, vmap, dOmap;
     const float *g, *beta;
     const __nv_bfloat16 *v;
     const __nv_bfloat16 *S0, *U, *dS, *dU, *Tb, *W, *Ut;
@@ -196,6 +196,7 @@ GDN_DEV void prefetch_chunk(const BlPtrs& p, const BlChunk& c) {
     tma_prefetch_tile(&p.dOmap, c.h, c.tok);
     tma_prefetch_tile(&p.qmap, c.h, c.tok);
     tma_prefetch_tile(&p.kmap, c.h, c.tok);
+    tma_prefetch_tile(&p.vmap, c.h, c.tok);  // v rows are read from L2 by the E1 epilogue
     bulk_prefetch_l2(p.U + (size_t)c.cid * C * DV, C * DV * 2);
     bulk_prefetch_l2(p.dU + (size_t)c.cid * C * DV, C * DV * 2);
     bulk_prefetch_l2(p.S0 + (size_t)c.cid * DV * DK, DV * DK * 2);
@@ -277,6 +278,7 @@ __global__ void __launch_bounds__(BL_THREADS, 1) tc5_bwd_local_kernel(const __gr
         load_u(s, p, ch);
         load_k(s, p, ch);
         load_tq(s, p, ch);
+        tma_prefetch_tile(&p.vmap, ch.h, ch.tok);
     }
     if (warp == 0) {
         tc5::alloc(&s.tmem, BL_TCOLS);
@@ -299,6 +301,9 @@ __global__ void __launch_bounds__(BL_THREADS, 1) tc5_bwd_local_kernel(const __gr
     float* Xs = s.Xs;
     uint32_t mph = 0;  // phase of bar_mma
     bool ok = true;
+    // The next chunk's loads are issued by a lane of warp 2, whose epilogue
+    // share is light or empty where they go out (thread 0 issues the MMAs).
+    const bool loader = warp == 2 && lane == 0;
     for (int it = 0;; ++it) {
         const uint32_t lp = it & 1;  // phase of the load barriers for this chunk
         const int L = ch.L;
@@ -311,7 +316,7 @@ __global__ void __launch_bounds__(BL_THREADS, 1) tc5_bwd_local_kernel(const __gr
         const BlChunk nch = bl_chunk(p, has_next ? ncid : cid);
         float myG = 0.f, myB = 0.f;  // this thread's (token, column group) share of dG / dbeta
         float myC = 0.f;             // this thread's (column, row block) share of the column sums
-        if (tid == 0 && has_next) prefetch_chunk(p, nch);
+        if (loader && has_next) prefetch_chunk(p, nch);
         if (warp == 2 && has_next) {  // the next chunk's g and beta rows, into L2
             for (int t = lane; t < nch.L; t += 32) {
                 prefetch_l2(p.g + nch.row0 + (size_t)t * rs);
@@ -377,7 +382,7 @@ __global__ void __launch_bounds__(BL_THREADS, 1) tc5_bwd_local_kernel(const __gr
         if (__syncthreads_or(!ok || kfail)) break;
         tc5::fence_after();
         // S0, dS and U are done with: the next chunk's go in
-        if (tid == 0 && has_next) {
+        if (loader && has_next) {
             load_s(s, p, nch);
             load_u(s, p, nch);
         }
@@ -466,7 +471,7 @@ __global__ void __launch_bounds__(BL_THREADS, 1) tc5_bwd_local_kernel(const __gr
         mph ^= 1;
         if (__syncthreads_or(!ok)) break;
         tc5::fence_after();
-        if (tid == 0 && has_next) load_tq(s, p, nch);  // T and Q are done with
+        if (loader && has_next) load_tq(s, p, nch);  // T and Q are done with
         // ---- epilogue E1: Gk, Gv -> bf16 A operands (R1); dv; <Gk_t, k_t>, <Gv_t, v_t>;
         // dq (complete after E1) -----------------------------------------------------
         if (q < 2) {
@@ -534,7 +539,7 @@ __global__ void __launch_bounds__(BL_THREADS, 1) tc5_bwd_local_kernel(const __gr
         mph ^= 1;
         if (__syncthreads_or(!ok)) break;
         tc5::fence_after();
-        if (tid == 0 && has_next) load_r1(s, p, nch);  // R1, W and U~ are done with
+        if (loader && has_next) load_r1(s, p, nch);  // R1, W and U~ are done with
         // ---- epilogue D: dA = strict_lower(-(Gk W^T + Gv U~^T)); M = K K^T .* Gamma;
         // dMM; hA; dbeta and dG terms --------------------------------------------------
         if (q < 2) {
@@ -590,7 +595,7 @@ __global__ void __launch_bounds__(BL_THREADS, 1) tc5_bwd_local_kernel(const __gr
         mph ^= 1;
         if (__syncthreads_or(!ok)) break;
         tc5::fence_after();
-        if (tid == 0 && has_next) load_k(s, p, nch);  // K is done with
+        if (loader && has_next) load_k(s, p, nch);  // K is done with
         // ---- epilogue E2: dk = TB + beta e^G .* Gk; the next chunk's G and beta ----------
         if (q < 2) {
             const int t = row;
@@ -660,7 +665,7 @@ namespace tc {
 bool launch_bwd_local5(const gdn_dims& d, const TcLayout& L, const ChunkPtrs& cp, const void* dO,
                        void* dq, void* dk, void* dv, float* dg, float* dbeta, void* ws, cudaStream_t st) {
     BlPtrs lp{};
-    lp.qmap = cp.qmap; lp.kmap = cp.kmap;
+    lp.qmap = cp.qmap; lp.kmap = cp.kmap; lp.vmap = cp.vmap;
     if (!encode_token_map(&lp.dOmap, dO, d.B, d.T, d.H)) return false;
     char* base = (char*)ws;
     lp.g = cp.g; lp.beta = cp.beta; lp.v = cp.v; lp.status = cp.status;
