@@ -50,7 +50,8 @@ using namespace tc;
 constexpr int BL_THREADS = 512;  // warp w: TMEM lane quarter w % 4, column group w / 4
 constexpr int PAIR = 128 * 64;  // elements of one 128-row, 64-column panel
 // tensor-memory columns
-constexpr uint32_t TA = 0,     // [-dW ; dq accumulator]          128
+constexpr uint32_t TA = 0,     // [-dW ; dq accumulator]          128; after E1 its lanes
+                               // 0..63 hold bf16 Gk (columns 0..63) and Gv (64..127)
     TB = 128,                  // [dk accumulator ; .]            128
     TC1 = 256,                 // [K K^T ; Q K^T]                  64
     TC2 = 320,                 // [. ; dO U^T]                     64
@@ -66,14 +67,15 @@ constexpr uint32_t ID_N128_AMN_BMN = tc5::idesc_bf16(128, 128, true, true);
 
 // Shared memory (one CTA per SM).  The CTA is persistent: it takes the chunks
 // blockIdx.x, blockIdx.x + gridDim.x, ... and loads each buffer of the next
-// chunk as soon as the current chunk is done with it (S0, dS and U after the
-// first products, T and Q after E1, dU, dO, W and U~ after C, K after E2),
-// so the loads of a chunk overlap the work of the one before.
+// chunk as soon as the current chunk is done with it (U after the first
+// products, T, Q, dU and dO after E1, S0 and dS after the E1 epilogue, W and
+// U~ after C, K after E2), so the loads of a chunk overlap the work of the
+// one before.  Between the first products and the E1 epilogue the S0 space
+// holds this chunk's V tile.
 struct alignas(1024) BlSmem {
-    __nv_bfloat16 R4[DV * DK];   // S0 (Kp<128>)
+    __nv_bfloat16 R4[DV * DK];   // S0 (Kp<128>); then V (Tma128) in its first 16 KB
     __nv_bfloat16 R5[DV * DK];   // dS (Kp<128>)
-    __nv_bfloat16 R1[2 * PAIR];  // [dU | dO] panels; dW in the dO rows; then Gk (rows 0..63)
-                                 // and Gv (from 8 KB on: rows 64..127 and the next panel)
+    __nv_bfloat16 R1[2 * PAIR];  // [dU | dO] panels; dW in the dO rows
     __nv_bfloat16 R2[2 * PAIR];  // [K | Q]
     __nv_bfloat16 R3[2 * PAIR];  // [U | .]: U rows; sdPG in the other rows of panel 0, dMM in
                                  // those of panel 1 (V is not held: its rows are read from L2)
@@ -91,7 +93,7 @@ struct alignas(1024) BlSmem {
     float red[16], red2[16];     // per-warp sums: <dS, S0>; etl <dKt, k> (enters dG_last)
     float dgs[C];                // reverse-cumsum scratch
     // one load barrier per buffer group (one phase per chunk), one for the MMAs
-    uint64_t bar_s, bar_u, bar_tq, bar_r1, bar_wu, bar_k, bar_mma;
+    uint64_t bar_s, bar_u, bar_tq, bar_r1, bar_wu, bar_k, bar_v, bar_mma;
     uint32_t tmem;
 };
 
@@ -176,15 +178,22 @@ GDN_DEV void load_tq(BlSmem& s, const BlPtrs& p, const BlChunk& c) {  // T, Q (r
     tma_load_3d(s.R2 + C * 64, &p.qmap, 0, c.h, c.tok, &s.bar_tq);
     tma_load_3d(s.R2 + PAIR + C * 64, &p.qmap, 64, c.h, c.tok, &s.bar_tq);
 }
-GDN_DEV void load_r1(BlSmem& s, const BlPtrs& p, const BlChunk& c) {  // dU, dO; W, U~
+GDN_DEV void load_r1(BlSmem& s, const BlPtrs& p, const BlChunk& c) {  // dU, dO
     mbar_arrive_expect(&s.bar_r1, 2 * C * DV * 2);
     bulk_g2s(s.R1, p.dU + (size_t)c.cid * C * DV, C * 64 * 2, &s.bar_r1);
     bulk_g2s(s.R1 + PAIR, p.dU + (size_t)c.cid * C * DV + C * 64, C * 64 * 2, &s.bar_r1);
     tma_load_3d(s.R1 + C * 64, &p.dOmap, 0, c.h, c.tok, &s.bar_r1);
     tma_load_3d(s.R1 + PAIR + C * 64, &p.dOmap, 64, c.h, c.tok, &s.bar_r1);
+}
+GDN_DEV void load_wu(BlSmem& s, const BlPtrs& p, const BlChunk& c) {  // W, U~
     mbar_arrive_expect(&s.bar_wu, (C * DK + DV * C) * 2);
     bulk_g2s(s.W, p.W + (size_t)c.cid * C * DK, C * DK * 2, &s.bar_wu);
     bulk_g2s(s.Ut, p.Ut + (size_t)c.cid * DV * C, DV * C * 2, &s.bar_wu);
+}
+GDN_DEV void load_v(BlSmem& s, const BlPtrs& p, const BlChunk& c) {  // V (Tma128, in the S0 space)
+    mbar_arrive_expect(&s.bar_v, C * DV * 2);
+    tma_load_3d(s.R4, &p.vmap, 0, c.h, c.tok, &s.bar_v);
+    tma_load_3d(s.R4 + C * 64, &p.vmap, 64, c.h, c.tok, &s.bar_v);
 }
 GDN_DEV void load_k(BlSmem& s, const BlPtrs& p, const BlChunk& c) {  // K (rows 0..63 of R2)
     mbar_arrive_expect(&s.bar_k, C * DK * 2);
@@ -225,6 +234,25 @@ GDN_DEV void load_gb(BlSmem& s, const BlPtrs& p, const BlChunk& c, int b) {
     s.G[b][lane + 32] = g1;
     s.beta[b][lane] = b0;
     s.beta[b][lane + 32] = b1;
+}
+
+// sum_{c < 32} x[c] * V[r][c0 + c] for row r of a Tma128 tile pair (two
+// 64-column panels of 64 rows).
+GDN_DEV float dot_tile32(const float* x, const __nv_bfloat16* V, int r, int c0) {
+    const __nv_bfloat16* base = V + (c0 >> 6) * (C * 64);
+    float acc = 0.f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const uint4 v = *reinterpret_cast<const uint4*>(base + swz<64>(r, (c0 & 63) + 8 * j));
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 f = unpack_bf16(w[i]);
+            acc = fmaf(x[8 * j + 2 * i], f.x, acc);
+            acc = fmaf(x[8 * j + 2 * i + 1], f.y, acc);
+        }
+    }
+    return acc;
 }
 
 GDN_DEV void store_row32(__nv_bfloat16* dst, const float* a, float f) {
@@ -271,14 +299,15 @@ __global__ void __launch_bounds__(BL_THREADS, 1) tc5_bwd_local_kernel(const __gr
         mbar_init(&s.bar_r1, 1);
         mbar_init(&s.bar_wu, 1);
         mbar_init(&s.bar_k, 1);
+        mbar_init(&s.bar_v, 1);
         mbar_init(&s.bar_mma, 1);
         fence_mbar_init();
         load_r1(s, p, ch);
+        load_wu(s, p, ch);
         load_s(s, p, ch);
         load_u(s, p, ch);
         load_k(s, p, ch);
         load_tq(s, p, ch);
-        tma_prefetch_tile(&p.vmap, ch.h, ch.tok);
     }
     if (warp == 0) {
         tc5::alloc(&s.tmem, BL_TCOLS);
@@ -381,10 +410,10 @@ __global__ void __launch_bounds__(BL_THREADS, 1) tc5_bwd_local_kernel(const __gr
         mph ^= 1;
         if (__syncthreads_or(!ok || kfail)) break;
         tc5::fence_after();
-        // S0, dS and U are done with: the next chunk's go in
-        if (loader && has_next) {
-            load_s(s, p, nch);
-            load_u(s, p, nch);
+        // S0 and U are done with: this chunk's V, the next chunk's U
+        if (loader) {
+            load_v(s, p, ch);
+            if (has_next) load_u(s, p, nch);
         }
         // ---- epilogue A --------------------------------------------------------------
         if (q >= 2) {
@@ -471,41 +500,31 @@ __global__ void __launch_bounds__(BL_THREADS, 1) tc5_bwd_local_kernel(const __gr
         mph ^= 1;
         if (__syncthreads_or(!ok)) break;
         tc5::fence_after();
-        if (loader && has_next) load_tq(s, p, nch);  // T and Q are done with
-        // ---- epilogue E1: Gk, Gv -> bf16 A operands (R1); dv; <Gk_t, k_t>, <Gv_t, v_t>;
-        // dq (complete after E1) -----------------------------------------------------
+        if (loader && has_next) {  // T, Q, dU and dO are done with
+            load_tq(s, p, nch);
+            load_r1(s, p, nch);
+        }
+        // ---- epilogue E1: Gk, Gv -> bf16 A operands in TMEM (lanes 0..63 of TA); dv;
+        // <Gk_t, k_t>, <Gv_t, v_t>; dq (complete after E1) -----------------------------
         if (q < 2) {
             const int t = row;
             const float bt = beta[t], egt = __expf(G[t]);
-            uint4 vr[4];  // v_t, columns 32cg.. (from L2)
-            if (t < L) {
-                const uint4* vp = reinterpret_cast<const uint4*>(p.v + (row0 + (size_t)t * rs) * DV + 32 * cg);
-#pragma unroll
-                for (int j = 0; j < 4; ++j) vr[j] = __ldg(vp + j);
-            } else {
-#pragma unroll
-                for (int j = 0; j < 4; ++j) vr[j] = make_uint4(0, 0, 0, 0);
-            }
             float gk[32], gv[32];
             ld_row32(gk, trow + TKG + 32 * cg);
             ld_row32(gv, trow + TVB + 32 * cg);
             tc5::wait_ld();
             const float hk = dot_row32(gk, s.R2, t, 32 * cg);
-            float hv = 0.f;
+            uint32_t pk[16];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const uint32_t w[4] = {vr[j].x, vr[j].y, vr[j].z, vr[j].w};
+            for (int c = 0; c < 16; ++c) pk[c] = pack_bf16(gk[2 * c], gk[2 * c + 1]);
+            tc5::st16(trow + TA + 16 * cg, pk);
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float2 f = unpack_bf16(w[i]);
-                    hv = fmaf(gv[8 * j + 2 * i], f.x, hv);
-                    hv = fmaf(gv[8 * j + 2 * i + 1], f.y, hv);
-                }
-            }
-            // Gk: rows 0..63 of the two K-major panels of R1; Gv: the same from 8 KB on
-            put_pair_row32(s.R1, t, 32 * cg, gk, 1.f);
-            put_pair_row32(s.R1 + C * 64, t, 32 * cg, gv, 1.f);
+            for (int c = 0; c < 16; ++c) pk[c] = pack_bf16(gv[2 * c], gv[2 * c + 1]);
+            tc5::st16(trow + TA + 64 + 16 * cg, pk);
             if (t < L) store_row32(p.dv + (row0 + (size_t)t * rs) * DV + 32 * cg, gv, bt);
+            const bool vok = mbar_wait(&s.bar_v, lp, p.status);
+            const float hv = vok ? dot_tile32(gv, s.R4, t, 32 * cg) : 0.f;
+            ok = ok && vok;
             myB += egt * hk + hv;
             myG += bt * egt * hk;
         } else {
@@ -515,21 +534,22 @@ __global__ void __launch_bounds__(BL_THREADS, 1) tc5_bwd_local_kernel(const __gr
             tc5::wait_ld();
             if (i < L) store_row32(p.dq + (row0 + (size_t)i * rs) * DK + 32 * cg, a, 1.f);
         }
-        fence_async_smem();
+        tc5::wait_st();
+        fence_async_smem();  // the V reads above, before the next chunk's S0 lands there
         tc5::fence_before();
-        ok = mbar_wait(&s.bar_wu, lp, p.status);
+        ok = ok && mbar_wait(&s.bar_wu, lp, p.status);
         if (__syncthreads_or(!ok)) break;
-        // ---- phase C: [Gk ; .] W^T + [Gv ; .] U~^T = T^T dT T^T; [K ; .] K^T again -------
+        if (loader && has_next) load_s(s, p, nch);  // V (in the S0 space) is done with
+        // ---- phase C: [Gk ; .] W^T + [Gv ; .] U~^T = T^T dT T^T (A from TMEM); [K ; .] K^T
         if (tid == 0) {
             tc5::fence_after();
             const uint32_t sW = smem_u32(s.W), sUt = smem_u32(s.Ut);
 #pragma unroll
             for (int kk = 0; kk < DK / 16; ++kk)
-                tc5::mma(tm + TD, tc5::kmajor<128>(sR1, kk), tc5::kmajor<C>(sW, kk), ID_N64, kk > 0);
+                tc5::mma_ts(tm + TD, tm + TA + 8 * kk, tc5::kmajor<C>(sW, kk), ID_N64, kk > 0);
 #pragma unroll
             for (int kk = 0; kk < DV / 16; ++kk)
-                tc5::mma(tm + TD, tc5::kmajor<128>(sR1 + C * 128, kk), tc5::mnmajor(sUt, kk, C * 128),
-                         ID_N64_BMN, true);
+                tc5::mma_ts(tm + TD, tm + TA + 64 + 8 * kk, tc5::mnmajor(sUt, kk, C * 128), ID_N64_BMN, true);
 #pragma unroll
             for (int kk = 0; kk < DK / 16; ++kk)
                 tc5::mma(tm + TKK, tc5::kmajor<128>(sR2, kk), tc5::kmajor<128>(sR2, kk), ID_N64, kk > 0);
@@ -539,7 +559,7 @@ __global__ void __launch_bounds__(BL_THREADS, 1) tc5_bwd_local_kernel(const __gr
         mph ^= 1;
         if (__syncthreads_or(!ok)) break;
         tc5::fence_after();
-        if (loader && has_next) load_r1(s, p, nch);  // R1, W and U~ are done with
+        if (loader && has_next) load_wu(s, p, nch);  // W and U~ are done with
         // ---- epilogue D: dA = strict_lower(-(Gk W^T + Gv U~^T)); M = K K^T .* Gamma;
         // dMM; hA; dbeta and dG terms --------------------------------------------------
         if (q < 2) {
