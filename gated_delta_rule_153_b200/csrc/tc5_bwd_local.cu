@@ -22,20 +22,25 @@
 //
 // Every product is one tcgen05 MMA group with M = 128 and an fp32 accumulator
 // in tensor memory.  The 64-token tiles sit in pairs in 128-row K-major panels
-// ([dU ; dO], [K ; Q], [U ; V]), so a product whose A is a pair yields two
-// results at once (lanes 0..63 and 64..127), and a 64-row A reads its partner
-// tile (or a neighbouring buffer) as rows 64..127 whose result is ignored:
-//   [dU ; dO] S0      -> -dW (lanes 0..63) and dO S0 (dO rows pre-scaled by
-//                        scale e^{G_i}: the dq accumulator, lanes 64..127)
-//   [U ; V] dS        -> etl .* (U dS) (U rows pre-scaled: the dk accumulator)
-//   [K ; Q] K^T       -> K K^T, Q K^T       [dU ; dO] U^T -> dO U^T
-//   [T^T ; .] dW -> Gk,  [T^T ; .] dU -> Gv,  [Gk ; .] W^T + [Gv ; .] U~^T -> -dA
-//   dk += [dMM ; .] K + [dMM^T ; .] K + [sdPG^T ; .] Q,   dq += [. ; sdPG] K
-// In every epilogue four warps share a TMEM lane quarter (one token row per
-// thread) and split the row's columns; per-token sums meet in fixed-order
-// shared-memory partials, and column sums over tokens go through a
-// shared-memory transpose.  One CTA of sixteen warps per chunk; thread 0
-// issues the loads and the MMAs.
+// ([dU ; dO], [K ; Q]), so a product whose A is a pair yields two results at
+// once (lanes 0..63 and 64..127), and a 64-row A reads its partner tile (or a
+// neighbouring buffer) as rows 64..127 whose result is ignored:
+//   A:  [dU ; dO] S0 -> -dW and dO S0 (the dq accumulator)
+//       [U ; .] dS   -> U dS (the dk accumulator)
+//       [dU ; dO] U^T -> dO U^T        [K ; Q] K^T -> K K^T, Q K^T
+//   E1: [T^T ; .] dW -> Gk,  [T^T ; .] dU -> Gv,
+//       dq += [. ; sdPG] K,  dk += [sdPG^T ; .] Q
+//   C:  [Gk ; .] W^T + [Gv ; .] U~^T -> -dA (Gk and Gv as bf16 A operands in
+//       tensor memory),  [K ; .] K^T again (for M = K K^T .* Gamma)
+//   E2: dk += [dMM ; .] K + [dMM^T ; .] K
+// The row scalings of the first products (scale e^{G_i} of the dq rows,
+// e^{G_last - G_i} of the dk rows) are applied to the accumulators in the
+// first epilogue (a TMEM load, scale, store), so every product of phase A
+// reads the tiles as loaded and goes out in one group.  In every epilogue
+// four warps share a TMEM lane quarter (one token row per thread) and split
+// the row's columns; per-token sums meet in fixed-order shared-memory
+// partials, and column sums over tokens go through a shared-memory transpose.
+// Sixteen warps per CTA; thread 0 issues the MMAs, a lane of warp 2 the loads.
 #include "async.cuh"
 #include "common.cuh"
 #include "internal.h"
@@ -67,18 +72,18 @@ constexpr uint32_t ID_N128_AMN_BMN = tc5::idesc_bf16(128, 128, true, true);
 
 // Shared memory (one CTA per SM).  The CTA is persistent: it takes the chunks
 // blockIdx.x, blockIdx.x + gridDim.x, ... and loads each buffer of the next
-// chunk as soon as the current chunk is done with it (U after the first
-// products, T, Q, dU and dO after E1, S0 and dS after the E1 epilogue, W and
+// chunk as soon as the current chunk is done with it (S0 and U after the
+// first products, T, Q, dU and dO after E1, dS after the E1 epilogue, W and
 // U~ after C, K after E2), so the loads of a chunk overlap the work of the
-// one before.  Between the first products and the E1 epilogue the S0 space
-// holds this chunk's V tile.
+// one before.  Between the first products and the E1 epilogue the dS space
+// holds this chunk's V tile (for <Gv_t, v_t>).
 struct alignas(1024) BlSmem {
-    __nv_bfloat16 R4[DV * DK];   // S0 (Kp<128>); then V (Tma128) in its first 16 KB
-    __nv_bfloat16 R5[DV * DK];   // dS (Kp<128>)
+    __nv_bfloat16 R4[DV * DK];   // S0 (Kp<128>)
+    __nv_bfloat16 R5[DV * DK];   // dS (Kp<128>); then V (Tma128) in its first 16 KB
     __nv_bfloat16 R1[2 * PAIR];  // [dU | dO] panels; dW in the dO rows
     __nv_bfloat16 R2[2 * PAIR];  // [K | Q]
     __nv_bfloat16 R3[2 * PAIR];  // [U | .]: U rows; sdPG in the other rows of panel 0, dMM in
-                                 // those of panel 1 (V is not held: its rows are read from L2)
+                                 // those of panel 1
     // Swz<64> T; the MN-major T^T operands read the 8 KB after it (W) as their
     // unused rows 64..127
     __nv_bfloat16 T[C * C];
@@ -93,7 +98,7 @@ struct alignas(1024) BlSmem {
     float red[16], red2[16];     // per-warp sums: <dS, S0>; etl <dKt, k> (enters dG_last)
     float dgs[C];                // reverse-cumsum scratch
     // one load barrier per buffer group (one phase per chunk), one for the MMAs
-    uint64_t bar_s, bar_u, bar_tq, bar_r1, bar_wu, bar_k, bar_v, bar_mma;
+    uint64_t bar_s, bar_ds, bar_u, bar_tq, bar_r1, bar_wu, bar_k, bar_v, bar_mma;
     uint32_t tmem;
 };
 
@@ -162,10 +167,13 @@ GDN_DEV BlChunk bl_chunk(const BlPtrs& p, int cid) {
 }
 
 // Loads of one buffer group of chunk c (thread 0).
-GDN_DEV void load_s(BlSmem& s, const BlPtrs& p, const BlChunk& c) {  // S0, dS
-    mbar_arrive_expect(&s.bar_s, 2 * DV * DK * 2);
+GDN_DEV void load_s0(BlSmem& s, const BlPtrs& p, const BlChunk& c) {  // S0
+    mbar_arrive_expect(&s.bar_s, DV * DK * 2);
     bulk_g2s(s.R4, p.S0 + (size_t)c.cid * DV * DK, DV * DK * 2, &s.bar_s);
-    bulk_g2s(s.R5, p.dS + (size_t)c.cid * DV * DK, DV * DK * 2, &s.bar_s);
+}
+GDN_DEV void load_ds(BlSmem& s, const BlPtrs& p, const BlChunk& c) {  // dS
+    mbar_arrive_expect(&s.bar_ds, DV * DK * 2);
+    bulk_g2s(s.R5, p.dS + (size_t)c.cid * DV * DK, DV * DK * 2, &s.bar_ds);
 }
 GDN_DEV void load_u(BlSmem& s, const BlPtrs& p, const BlChunk& c) {  // U (rows 0..63 of R3)
     mbar_arrive_expect(&s.bar_u, C * DV * 2);
@@ -190,10 +198,10 @@ GDN_DEV void load_wu(BlSmem& s, const BlPtrs& p, const BlChunk& c) {  // W, U~
     bulk_g2s(s.W, p.W + (size_t)c.cid * C * DK, C * DK * 2, &s.bar_wu);
     bulk_g2s(s.Ut, p.Ut + (size_t)c.cid * DV * C, DV * C * 2, &s.bar_wu);
 }
-GDN_DEV void load_v(BlSmem& s, const BlPtrs& p, const BlChunk& c) {  // V (Tma128, in the S0 space)
+GDN_DEV void load_v(BlSmem& s, const BlPtrs& p, const BlChunk& c) {  // V (Tma128, in the dS space)
     mbar_arrive_expect(&s.bar_v, C * DV * 2);
-    tma_load_3d(s.R4, &p.vmap, 0, c.h, c.tok, &s.bar_v);
-    tma_load_3d(s.R4 + C * 64, &p.vmap, 64, c.h, c.tok, &s.bar_v);
+    tma_load_3d(s.R5, &p.vmap, 0, c.h, c.tok, &s.bar_v);
+    tma_load_3d(s.R5 + C * 64, &p.vmap, 64, c.h, c.tok, &s.bar_v);
 }
 GDN_DEV void load_k(BlSmem& s, const BlPtrs& p, const BlChunk& c) {  // K (rows 0..63 of R2)
     mbar_arrive_expect(&s.bar_k, C * DK * 2);
@@ -205,7 +213,7 @@ GDN_DEV void prefetch_chunk(const BlPtrs& p, const BlChunk& c) {
     tma_prefetch_tile(&p.dOmap, c.h, c.tok);
     tma_prefetch_tile(&p.qmap, c.h, c.tok);
     tma_prefetch_tile(&p.kmap, c.h, c.tok);
-    tma_prefetch_tile(&p.vmap, c.h, c.tok);  // v rows are read from L2 by the E1 epilogue
+    tma_prefetch_tile(&p.vmap, c.h, c.tok);
     bulk_prefetch_l2(p.U + (size_t)c.cid * C * DV, C * DV * 2);
     bulk_prefetch_l2(p.dU + (size_t)c.cid * C * DV, C * DV * 2);
     bulk_prefetch_l2(p.S0 + (size_t)c.cid * DV * DK, DV * DK * 2);
@@ -295,6 +303,7 @@ __global__ void __launch_bounds__(BL_THREADS, 1) tc5_bwd_local_kernel(const __gr
     if (tid == 0) {
         mbar_init(&s.bar_s, 1);
         mbar_init(&s.bar_u, 1);
+        mbar_init(&s.bar_ds, 1);
         mbar_init(&s.bar_tq, 1);
         mbar_init(&s.bar_r1, 1);
         mbar_init(&s.bar_wu, 1);
@@ -304,7 +313,8 @@ __global__ void __launch_bounds__(BL_THREADS, 1) tc5_bwd_local_kernel(const __gr
         fence_mbar_init();
         load_r1(s, p, ch);
         load_wu(s, p, ch);
-        load_s(s, p, ch);
+        load_s0(s, p, ch);
+        load_ds(s, p, ch);
         load_u(s, p, ch);
         load_k(s, p, ch);
         load_tq(s, p, ch);
@@ -354,6 +364,7 @@ __global__ void __launch_bounds__(BL_THREADS, 1) tc5_bwd_local_kernel(const __gr
         }
         if (tid < 16) s.red2[tid] = 0.f;
         ok = mbar_wait(&s.bar_r1, lp, p.status) && mbar_wait(&s.bar_s, lp, p.status) &&
+             mbar_wait(&s.bar_ds, lp, p.status) &&
              mbar_wait(&s.bar_u, lp, p.status) && mbar_wait(&s.bar_tq, lp, p.status);
         if (__syncthreads_or(!ok)) break;
         // dO rows past the sequence end belong to the next sequence: zero them
@@ -413,7 +424,10 @@ __global__ void __launch_bounds__(BL_THREADS, 1) tc5_bwd_local_kernel(const __gr
         // S0 and U are done with: this chunk's V, the next chunk's U
         if (loader) {
             load_v(s, p, ch);
-            if (has_next) load_u(s, p, nch);
+            if (has_next) {
+                load_u(s, p, nch);
+                load_s0(s, p, nch);
+            }
         }
         // ---- epilogue A --------------------------------------------------------------
         if (q >= 2) {
@@ -523,7 +537,7 @@ __global__ void __launch_bounds__(BL_THREADS, 1) tc5_bwd_local_kernel(const __gr
             tc5::st16(trow + TA + 64 + 16 * cg, pk);
             if (t < L) store_row32(p.dv + (row0 + (size_t)t * rs) * DV + 32 * cg, gv, bt);
             const bool vok = mbar_wait(&s.bar_v, lp, p.status);
-            const float hv = vok ? dot_tile32(gv, s.R4, t, 32 * cg) : 0.f;
+            const float hv = vok ? dot_tile32(gv, s.R5, t, 32 * cg) : 0.f;
             ok = ok && vok;
             myB += egt * hk + hv;
             myG += bt * egt * hk;
@@ -539,7 +553,7 @@ __global__ void __launch_bounds__(BL_THREADS, 1) tc5_bwd_local_kernel(const __gr
         tc5::fence_before();
         ok = ok && mbar_wait(&s.bar_wu, lp, p.status);
         if (__syncthreads_or(!ok)) break;
-        if (loader && has_next) load_s(s, p, nch);  // V (in the S0 space) is done with
+        if (loader && has_next) load_ds(s, p, nch);  // V (in the dS space) is done with
         // ---- phase C: [Gk ; .] W^T + [Gv ; .] U~^T = T^T dT T^T (A from TMEM); [K ; .] K^T
         if (tid == 0) {
             tc5::fence_after();
