@@ -401,9 +401,10 @@ __global__ void __launch_bounds__(BL_THREADS, 1) tc5_bwd_local_kernel(const __gr
             }
             tc5::commit(&s.bar_mma);
         }
-        {   // <dS, S0> under the products (both are only read until the next chunk's loads)
+        {   // <dS, S0> under the products (both are only read until the next chunk's loads),
+            // by warps 1..15: warp 0 holds the thread that issues the products
             float ss = 0.f;
-            for (int e = tid; e < DV * DK / 8; e += BL_THREADS) {
+            for (int e = tid - 32; warp > 0 && e < DV * DK / 8; e += BL_THREADS - 32) {
                 const uint4 x = reinterpret_cast<const uint4*>(s.R5)[e];
                 const uint4 y = reinterpret_cast<const uint4*>(s.R4)[e];
                 const uint32_t xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
@@ -482,11 +483,6 @@ __global__ void __launch_bounds__(BL_THREADS, 1) tc5_bwd_local_kernel(const __gr
         fence_async_smem();
         tc5::fence_before();
         __syncthreads();
-        {   // column sums of hP: dG_j -= sum_i hP_ij (eight row blocks per column)
-            const int j = tid & 63, pb = tid >> 6;
-#pragma unroll
-            for (int i = 8 * pb; i < 8 * pb + 8; ++i) myC -= Xs[i * 64 + ((j + i) & 63)];
-        }
         // ---- phase E1: Gk = T^T dW, Gv = T^T dU; dq += [. ; sdPG] K; dk += sdPG^T Q
         if (tid == 0) {
             tc5::fence_after();
@@ -509,6 +505,12 @@ __global__ void __launch_bounds__(BL_THREADS, 1) tc5_bwd_local_kernel(const __gr
                 tc5::mma(tm + TB, tc5::mnmajor(ssdPG, kk, C * 128), tc5::mnmajor(sR2 + C * 128, kk, PB),
                          ID_N128_AMN_BMN, true);
             tc5::commit(&s.bar_mma);
+        }
+        {   // column sums of hP (under the E1 products): dG_j -= sum_i hP_ij (eight row
+            // blocks per column)
+            const int j = tid & 63, pb = tid >> 6;
+#pragma unroll
+            for (int i = 8 * pb; i < 8 * pb + 8; ++i) myC -= Xs[i * 64 + ((j + i) & 63)];
         }
         ok = mbar_wait(&s.bar_mma, mph, p.status);
         mph ^= 1;
