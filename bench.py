@@ -96,6 +96,7 @@ KERNEL_SOURCE = {"tc_walk_fwd": "tc_chunk.cu", "tc_walk_states": "tc_chunk.cu",
                  "tc5_bwd_local": "tc5_bwd_local.cu", "tc5_bwd_local_kda": "tc5_bwd_local_kda.cu",
                  "tc5_seg_map": "tc5_walk.cu", "tc5_seg_scan": "tc5_walk.cu",
                  "tc5_walk_fwd": "tc5_walk.cu", "tc5_walk_states": "tc5_walk.cu",
+                 "tc5_walk_fwd_save": "tc5_walk.cu", "tc5_prep_conv": "tc5_prep.cu",
                  "tc5_walk_bwd": "tc5_walk_bwd.cu", "decode_step": "decode.cu"}
 
 
