@@ -231,18 +231,57 @@ __global__ void __launch_bounds__(P5_THREADS, 3) tc5_prep_kernel(const __grid_co
         tc5::fence_before();
         __syncthreads();
     }
+    if (!CONV) {
+        ok = mbar_wait(&s.bar_ld, 0, p.status);
+        if (__syncthreads_or(!ok)) goto done;
+    }
     // ---- [K K^T ; Q K^T] ---------------------------------------------------
     if (tid == 0) {
-        if (!CONV) ok = mbar_wait(&s.bar_ld, 0, p.status);
-        if (ok) {
-            tc5::fence_after();
+        tc5::fence_after();
 #pragma unroll
-            for (int kk = 0; kk < DK / 16; ++kk)
-                tc5::mma(tm, tc5::kmajor<2 * C>(sKQ, kk), tc5::kmajor<2 * C>(sKQ, kk), ID_KQ, kk > 0);
-            tc5::commit(&s.bar_mma);
+        for (int kk = 0; kk < DK / 16; ++kk)
+            tc5::mma(tm, tc5::kmajor<2 * C>(sKQ, kk), tc5::kmajor<2 * C>(sKQ, kk), ID_KQ, kk > 0);
+        tc5::commit(&s.bar_mma);
+    }
+    // ---- under the product: K~ = diag(e^{G_last - G}) K to the workspace (the
+    // walks' B of the state update) from the K tile as loaded, and V <- diag(beta) V
+    // in place (the row scale of U~; V is not read before the second product)
+    if (tid < 128) {  // threads 0..127: K~ rows; 128..255: V rows
+        const int r = tid >> 1, pn = tid & 1;
+        const float dec = __expf(s.G[C - 1] - s.G[r]);
+        const __nv_bfloat16* row = s.KQ + pn * KQ_PANEL + r * 64;
+        // same swizzled position in the Tma128 image (panel pn at pn * 4096)
+        __nv_bfloat16* kt = p.Kt + (size_t)cid * C * DK + pn * (C * 64) + r * 64;
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+            const int j = (jj + r) & 7;  // per-row rotated order (banks)
+            const uint4 x = *reinterpret_cast<const uint4*>(row + 8 * j);
+            const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+            uint32_t wt[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float2 f2 = unpack_bf16(w[i]);
+                wt[i] = pack_bf16(f2.x * dec, f2.y * dec);
+            }
+            *reinterpret_cast<uint4*>(kt + 8 * j) = make_uint4(wt[0], wt[1], wt[2], wt[3]);
+        }
+    } else {
+        const int r = (tid - 128) >> 1, pn = tid & 1;
+        const float b = s.beta[r];
+        __nv_bfloat16* vrow = s.V + pn * (C * 64) + r * 64;
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+            const int j = (jj + r) & 7;
+            uint4 x = *reinterpret_cast<uint4*>(vrow + 8 * j);
+            uint32_t* w = reinterpret_cast<uint32_t*>(&x);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float2 f2 = unpack_bf16(w[i]);
+                w[i] = pack_bf16(f2.x * b, f2.y * b);
+            }
+            *reinterpret_cast<uint4*>(vrow + 8 * j) = x;
         }
     }
-    if (__syncthreads_or(!ok)) goto done;
     ok = mbar_wait(&s.bar_mma, 0, p.status);
     if (__syncthreads_or(!ok)) goto done;
     tc5::fence_after();
@@ -296,50 +335,32 @@ __global__ void __launch_bounds__(P5_THREADS, 3) tc5_prep_kernel(const __grid_co
                 }
             }
         }
+        fence_async_smem();  // P (generic writes) -> its bulk store
         tc5::fence_before();
         __syncthreads();
+        if (tid == 0) {  // P and G are final: out now, under the solve
+            bulk_s2g(p.P + (size_t)cid * C * C, s.P, C * C * 2);
+            bulk_s2g(p.G + (size_t)cid * C, s.G, C * 4);
+            bulk_commit();
+        }
 
-        // ---- K~ = diag(e^{G_last - G}) K to the workspace (the walks' B of
-        // the state update); K <- diag(beta e^G) K and V <- diag(beta) V in
-        // place (the row scales of W and U~)
-        if (tid < 128) {  // threads 0..127: K rows; 128..255: V rows (below)
-            const int r = tid >> 1, pn = tid & 1;
-            const float e = s.beta[r] * __expf(s.G[r]), dec = __expf(s.G[C - 1] - s.G[r]);
+        // ---- K <- diag(beta e^G) K in place (the row scale of W): thread =
+        // (row, quarter of the row's 128 channels)
+        {
+            const int r = tid >> 2, qc = tid & 3, pn = qc >> 1;
+            const float e = s.beta[r] * __expf(s.G[r]);
             __nv_bfloat16* row = s.KQ + pn * KQ_PANEL + r * 64;
-            // same swizzled position in the Tma128 image (panel pn at pn * 4096)
-            __nv_bfloat16* kt = p.Kt + (size_t)cid * C * DK + pn * (C * 64) + r * 64;
-            // chunks in a per-row rotated order: the 32 lanes of a warp sit on 16
-            // rows, so a common order would put them all on the same four banks
 #pragma unroll
-            for (int jj = 0; jj < 8; ++jj) {
-                const int j = (jj + r) & 7;
-                uint4 x = *reinterpret_cast<uint4*>(row + 8 * j), y;
+            for (int jj = 0; jj < 4; ++jj) {
+                const int j = 4 * (qc & 1) + ((jj + r) & 3);  // rotated order within the half row
+                uint4 x = *reinterpret_cast<uint4*>(row + 8 * j);
                 uint32_t* w = reinterpret_cast<uint32_t*>(&x);
-                uint32_t* wt = reinterpret_cast<uint32_t*>(&y);
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const float2 f2 = unpack_bf16(w[i]);
                     w[i] = pack_bf16(f2.x * e, f2.y * e);
-                    wt[i] = pack_bf16(f2.x * dec, f2.y * dec);
                 }
                 *reinterpret_cast<uint4*>(row + 8 * j) = x;
-                *reinterpret_cast<uint4*>(kt + 8 * j) = y;
-            }
-        } else {
-            const int r = (tid - 128) >> 1, pn = tid & 1;
-            const float b = s.beta[r];
-            __nv_bfloat16* vrow = s.V + pn * (C * 64) + r * 64;
-#pragma unroll
-            for (int jj = 0; jj < 8; ++jj) {
-                const int j = (jj + r) & 7;
-                uint4 x = *reinterpret_cast<uint4*>(vrow + 8 * j);
-                uint32_t* w = reinterpret_cast<uint32_t*>(&x);
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float2 f2 = unpack_bf16(w[i]);
-                    w[i] = pack_bf16(f2.x * b, f2.y * b);
-                }
-                *reinterpret_cast<uint4*>(vrow + 8 * j) = x;
             }
         }
 
@@ -352,6 +373,10 @@ __global__ void __launch_bounds__(P5_THREADS, 3) tc5_prep_kernel(const __grid_co
     tc5::fence_before();
     __syncthreads();
     if (tid == 0) {
+        if (p.Tb) {  // T is final: out now, under the second product
+            bulk_s2g(p.Tb + (size_t)cid * C * C, s.T, C * C * 2);
+            bulk_commit();
+        }
         tc5::fence_after();
         const uint32_t sT = smem_u32(s.T), sV = smem_u32(s.V);
 #pragma unroll
@@ -399,9 +424,6 @@ __global__ void __launch_bounds__(P5_THREADS, 3) tc5_prep_kernel(const __grid_co
     if (tid == 0) {
         bulk_s2g(p.W + (size_t)cid * C * DK, s.KQ, C * DK * 2);
         bulk_s2g(p.Ut + (size_t)cid * C * DV, s.KQ + C * DK, C * DV * 2);
-        bulk_s2g(p.P + (size_t)cid * C * C, s.P, C * C * 2);
-        bulk_s2g(p.G + (size_t)cid * C, s.G, C * 4);
-        if (p.Tb) bulk_s2g(p.Tb + (size_t)cid * C * C, s.T, C * C * 2);
         bulk_commit();
         bulk_wait_read<0>();
     }
