@@ -650,7 +650,17 @@ def run_ours(args, rank, world, dev, barrier, max_over_ranks):
 def run_case(args, dev):
     """One workload alone: `warmup` untimed then `steps` timed steps."""
     import gated_delta_rule_153_b200 as gdn
-    from gated_delta_rule_153_b200.inputs import KDA, LONG, make_chunk_inputs
+    from gated_delta_rule_153_b200.inputs import DECODE, KDA, LONG, make_chunk_inputs, make_tree_inputs
+    if args.case == "tree":  # draft-tree verification, the decode-sized batch of 32-node 4-ary trees
+        tr = to_dev(make_tree_inputs(DECODE.N, 32, DECODE.H, shape="kary4", seed=1200), dev)
+        to = torch.empty_like(tr["v"])
+        fn = lambda: gdn.gdn_tree_verify(tr["parent"], tr["q"], tr["k"], tr["v"], tr["g"], tr["beta"],
+                                         tr["state"], o=to)
+        ms = timed(fn, args.steps, args.warmup)
+        print(json.dumps({"case": f"tree verify N{DECODE.N} H{DECODE.H} d128, 32-node 4-ary trees",
+                          "ms": round(ms, 4), "steps": args.steps, "warmup": args.warmup,
+                          "kernels": kernel_breakdown(gdn, fn, 2)}))
+        return
     cfg = KDA if args.case == "kda" else LONG
     d = to_dev(make_chunk_inputs(cfg, seed=cfg.seed), dev)
     ws_f, ws_b = workspaces(gdn, d)
@@ -692,10 +702,10 @@ def main():
     ap.add_argument("--headline-only", action="store_true",
                     help="skip the long-context, channel-gate and decode extras")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--case", choices=["kda", "long"],
-                    help="run only this workload's step (channel-gate fwd+bwd, or the "
-                         "long-context forward) and print its time: a short command for "
-                         "kernel profilers, not the contract line")
+    ap.add_argument("--case", choices=["kda", "long", "tree"],
+                    help="run only this workload's step (channel-gate fwd+bwd, the "
+                         "long-context forward, or the draft-tree verification) and print "
+                         "its time: a short command for kernel profilers, not the contract line")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 

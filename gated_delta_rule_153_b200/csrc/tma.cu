@@ -21,12 +21,12 @@ static PFN_cuTensorMapEncodeTiled_v12000 encoder() {
     return fn;
 }
 
-bool encode_token_map(CUtensorMap* map, const void* base, int B, int T, int H, int box_cols) {
+bool encode_token_map(CUtensorMap* map, const void* base, int B, int T, int H, int box_cols, int box_rows) {
     PFN_cuTensorMapEncodeTiled_v12000 fn = encoder();
     if (!fn) return false;
     const cuuint64_t dims[3] = {128, (cuuint64_t)H, (cuuint64_t)B * (cuuint64_t)T};
     const cuuint64_t strides[2] = {128 * 2, (cuuint64_t)H * 128 * 2};
-    const cuuint32_t box[3] = {(cuuint32_t)box_cols, 1, 64};
+    const cuuint32_t box[3] = {(cuuint32_t)box_cols, 1, (cuuint32_t)box_rows};
     const cuuint32_t estr[3] = {1, 1, 1};
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,

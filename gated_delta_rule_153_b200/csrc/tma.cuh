@@ -54,10 +54,10 @@ GDN_DEV void tma_prefetch_tile(const CUtensorMap* map, int head, int token) {
 }
 
 // Host: encode the token map of a [B, T, H, 128] bf16 tensor.  box_cols 64
-// gives 128-byte-swizzled 64x64 boxes (Tma128 tiles); box_cols 16 gives
-// unswizzled 64-row x 16-column boxes (32-byte rows).  Returns false
-// if the driver entry point is unavailable or the encoder rejects the map.
+// gives 128-byte-swizzled boxes of box_rows x 64 (Tma128 tiles at 64 rows);
+// box_cols 16 gives unswizzled box_rows x 16 boxes (32-byte rows).  Returns
+// false if the driver entry point is unavailable or the encoder rejects the map.
 bool encode_token_map(CUtensorMap* map, const void* base, int B, int T, int H,
-                      int box_cols = 64);
+                      int box_cols = 64, int box_rows = 64);
 
 }  // namespace gdn

@@ -30,6 +30,8 @@
 #include "common.cuh"
 #include "internal.h"
 #include "mma.cuh"
+#include "tc5.cuh"
+#include "tma.cuh"
 
 namespace gdn {
 namespace {
@@ -38,87 +40,90 @@ constexpr int TD = 128;           // d_k = d_v
 constexpr int TREE_THREADS = 256;  // 8 warps
 constexpr int kMaxTreeNodes = 64;
 
+// Verification on the fifth-generation tensor cores.  The node tiles (MP = 32
+// or 64 rows) arrive by TMA; the products whose rows would be nodes run
+// transposed where they touch the state, so the 128 value (or key) rows sit
+// on the TMEM lanes and every warp has work in their epilogues:
+//   [K] K^T, [Q] K^T                 lane = node        (A and P; scalar gate)
+//   W^T  = K^T Tw^T,  U~^T = V^T Tu^T lane = key / value (Tw = T diag(beta e^G),
+//                                                         Tu = T diag(beta))
+//   U^T  = U~^T - S0 W^T,  Y^T = S0 Q^T   lane = value   (S0 as a bf16 A operand
+//                                                         in tensor memory)
+//   O^T  = diag-scaled Y^T + U^T P^T     lane = value   (U^T likewise)
+// Each thread converts its own state row (value lane, 64 keys) from fp32 to
+// bf16 straight into tensor memory, so the state never occupies shared memory.
+// The ancestor masks, the decays and the level-by-level solve for T stay on
+// CUDA cores: they are the tree's small dependent steps, not contractions.
 template <int MP, bool KDA>
-struct TreeSmem {
-    __nv_bfloat16 K[MP * TD];  // Swz<128>; rows of U (value index as column) once W is built
-    __nv_bfloat16 Q[MP * TD];
+struct alignas(1024) TreeSmem {
+    __nv_bfloat16 K[MP * TD];      // TMA tiles: two 64-column panels of MP node rows,
+    __nv_bfloat16 Q[MP * TD];      // 128-byte swizzle
     __nv_bfloat16 V[MP * TD];
-    union {
-        float A[MP][MP + 1];          // masked, decayed beta K K^T
-        __nv_bfloat16 Wn[MP * TD];    // -W, Swz<128>
-    };
-    float T[MP][MP + 1];              // (I + A)^{-1}
-    alignas(128) __nv_bfloat16 Tw[MP * 64];  // T diag(beta e^G), Swz<64> (columns < MP used)
-    __nv_bfloat16 Tu[MP * 64];        // T diag(beta)
-    __nv_bfloat16 P[MP * 64];
+    __nv_bfloat16 WnT[TD * 64];    // -W^T: [key][node], rows of 64 nodes (MN-major B)
+    __nv_bfloat16 Tw[MP * 64];     // T diag(beta e^G) (channel gate: T diag(beta)): [i][j]
+    __nv_bfloat16 Tu[MP * 64];     // T diag(beta)
+    __nv_bfloat16 P[MP * 64];      // scale e^{G_i - G_j} q_i.k_j on ancestors and the diagonal
+    float A[MP][MP + 1];           // masked, decayed beta K K^T
+    float T[MP][MP + 1];           // (I + A)^{-1}
     float G[MP], g[MP], beta[MP];
     unsigned long long anc[MP];
     int par[MP], depth[MP];
     int maxdepth;
-    alignas(16) float Gc[KDA ? MP : 1][TD];  // channel gate: per-key sums of g over each root path (16-byte copies)
+    uint64_t bar_ld, bar_mma;
+    uint32_t tmem;
+    alignas(16) float Gc[KDA ? MP : 1][TD];  // channel gate: per-key sums of g over each root path
 };
 
-// One CTA per (sequence n, head h).  MB = number of 16-node blocks.
-// Channel gate (KDA): g_i is a vector over the keys, G_i its sum over the root
-// path, and every decay e^{G_i - G_j} (j an ancestor of i) carries the key
-// index, so A and P sum k_i k_j e^{G_i - G_j} (q_i k_j e^{G_i - G_j}) over the
-// keys pair by pair; W and the read-out take K .* e^G and Q .* e^G.
-template <int MB, bool KDA>
-__global__ void __launch_bounds__(TREE_THREADS, MB <= 2 ? 4 : 2)  // 4 CTAs per SM up to 32 nodes
-tree_verify_kernel(int M, int H, float scale, const int* __restrict__ parent,
-                   const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
-                   const __nv_bfloat16* __restrict__ v, const float* __restrict__ g,
-                   const float* __restrict__ beta, const float* __restrict__ state,
-                   __nv_bfloat16* __restrict__ o, unsigned int* status) {
-    constexpr int MP = 16 * MB;
-    extern __shared__ __align__(128) unsigned char smem_raw[];
-    TreeSmem<MP, KDA>& s = *reinterpret_cast<TreeSmem<MP, KDA>*>(smem_raw);
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int nh = blockIdx.x, n = nh / H, h = nh % H;
-    const size_t rs = (size_t)H * TD;                        // token row stride
-    const size_t row0 = ((size_t)n * M * H + h) * TD;       // node 0 of (n, h)
+struct TreePtrs {
+    CUtensorMap qmap, kmap, vmap;  // [N, M, H, 128] node maps, boxes of MP rows
+    int M, H;
+    float scale;
+    const int* parent;
+    const float *g, *beta, *state;
+    __nv_bfloat16* o;
+    unsigned int* status;
+};
 
-    // ---- loads: node tokens into shared tiles; the state is pulled into L2
-    // now and read as MMA fragments in the last phase ------------------------
-    const float* S0 = state + (size_t)nh * TD * TD;
-    if (tid < 4) bulk_prefetch_l2(S0 + tid * (TD * TD / 4), TD * TD);  // 4 x 16 KiB
-    if (tid == 0) s.maxdepth = 0;
-    load_tile_async<TD>(s.K, k + row0, rs, MP, M, tid, TREE_THREADS);
-    load_tile_async<TD>(s.Q, q + row0, rs, MP, M, tid, TREE_THREADS);
-    load_tile_async<TD>(s.V, v + row0, rs, MP, M, tid, TREE_THREADS);
-    cp_async_commit();
-    if (tid < MP) {
-        int p = -1;
-        float gi = 0.f, bi = 0.f;
-        if (tid < M) {
-            p = parent[(size_t)n * M + tid];
-            if (p < -1 || p >= tid) {  // not a tree in topological order
-                if (status) atomicOr(status, 2u);
-                p = -1;
-            }
-            if (!KDA) gi = g[((size_t)n * M + tid) * H + h];
-            bi = beta[((size_t)n * M + tid) * H + h];
-        }
-        s.par[tid] = p;
-        s.g[tid] = gi;
-        s.beta[tid] = bi;
-    }
-    if constexpr (KDA) {  // per-key gates of every node (zero past M)
-        for (int e = tid; e < MP * TD / 4; e += TREE_THREADS) {
-            const int i = e / (TD / 4), c4 = e % (TD / 4);
-            cp_async16_zfill(&s.Gc[i][4 * c4], g + (((size_t)n * M + (i < M ? i : 0)) * H + h) * TD + 4 * c4,
-                             i < M);
-        }
-        cp_async_commit();
-    }
-    cp_async_wait<0>();
-    __syncthreads();
+GDN_DEV unsigned char* align_1k(unsigned char* p) {
+    return reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// Element (row, column) of an MP-row TMA tile (two 64-column panels).
+template <int MP>
+GDN_DEV int toff(int r, int c) { return (c >> 6) * (MP * 64) + swz<64>(r, c & 63); }
+
+template <int MP>
+GDN_DEV void ldcols(float* v, uint32_t taddr) {  // MP / 2 columns of this thread's lane
+    if constexpr (MP == 32) tc5::ld16(*reinterpret_cast<float(*)[16]>(v), taddr);
+    else tc5::ld32(*reinterpret_cast<float(*)[32]>(v), taddr);
+}
+
+template <int MP, bool KDA>
+GDN_DEV void verify_body(TreeSmem<MP, KDA>& s, const TreePtrs& p, uint32_t tm) {
+    // tensor-memory columns: the bf16 state (64), then X and Y (MP each); U^T in
+    // bf16 takes the state's columns once the state products are done
+    constexpr uint32_t TS0 = 0, TX = 64, TY = 64 + MP, TUP = 0;
+    constexpr uint32_t ID_NN = tc5::idesc_bf16(128, MP, false, false);
+    constexpr uint32_t ID_MK = tc5::idesc_bf16(128, MP, true, false);
+    constexpr uint32_t ID_KM = tc5::idesc_bf16(128, MP, false, true);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int M = p.M, H = p.H;
+    const int nh = blockIdx.x, n = nh / H, h = nh % H;
+    const size_t rs = (size_t)H * TD;                   // node row stride
+    const size_t row0 = ((size_t)n * M * H + h) * TD;  // node 0 of (n, h)
+    const float scale = p.scale;
+    const uint32_t sK = smem_u32(s.K), sQ = smem_u32(s.Q), sV = smem_u32(s.V);
+    const uint32_t sWnT = smem_u32(s.WnT), sTw = smem_u32(s.Tw), sTu = smem_u32(s.Tu), sP = smem_u32(s.P);
+    // epilogue thread roles on the 128 lanes: lane quarter warp % 4, column half warp / 4
+    const int lr = 32 * (warp & 3) + lane, hh = warp >> 2;
+    const uint32_t trow = tm + ((uint32_t)(32 * (warp & 3)) << 16);
+    uint32_t mph = 0;
+
     if constexpr (KDA) {  // path sums, parents first: thread = key
         if (tid < TD)
             for (int i = 0; i < M; ++i)
                 if (s.par[i] >= 0) s.Gc[i][tid] += s.Gc[s.par[i]][tid];
     }
-
     // ---- path sums of g and ancestor sets (parents precede children) ------
     if (tid < MP) {
         float Gi = s.g[tid];
@@ -132,9 +137,10 @@ tree_verify_kernel(int M, int H, float scale, const int* __restrict__ parent,
         s.depth[tid] = __popcll(m);
         atomicMax(&s.maxdepth, __popcll(m));
     }
-    __syncthreads();
+    bool ok = mbar_wait(&s.bar_ld, 0, p.status);
+    if (__syncthreads_or(!ok)) return;
 
-    // ---- A (warps 0-3) and P (warps 4-7): 16 node rows each -----------------
+    // ---- A and P ---------------------------------------------------------
     if constexpr (KDA) {
         // ancestor pairs (and, for P, the node itself) only; a warp per pair,
         // a lane per 4 keys; the decays are e^{G_i - G_j} <= 1 key by key
@@ -150,9 +156,9 @@ tree_verify_kernel(int M, int H, float scale, const int* __restrict__ parent,
             for (unsigned long long m = s.anc[i] | (1ull << i); m; m &= m - 1ull, ++pc) {
                 if ((pc & 7) != warp) continue;
                 const int j = __ffsll((long long)m) - 1;
-                const uint2 ki = *reinterpret_cast<const uint2*>(&s.K[swz<TD>(i, c)]);
-                const uint2 kj = *reinterpret_cast<const uint2*>(&s.K[swz<TD>(j, c)]);
-                const uint2 qi = *reinterpret_cast<const uint2*>(&s.Q[swz<TD>(i, c)]);
+                const uint2 ki = *reinterpret_cast<const uint2*>(&s.K[toff<MP>(i, c)]);
+                const uint2 kj = *reinterpret_cast<const uint2*>(&s.K[toff<MP>(j, c)]);
+                const uint2 qi = *reinterpret_cast<const uint2*>(&s.Q[toff<MP>(i, c)]);
                 const float2 ki0 = unpack_bf16(ki.x), ki1 = unpack_bf16(ki.y);
                 const float2 kj0 = unpack_bf16(kj.x), kj1 = unpack_bf16(kj.y);
                 const float2 qi0 = unpack_bf16(qi.x), qi1 = unpack_bf16(qi.y);
@@ -170,45 +176,46 @@ tree_verify_kernel(int M, int H, float scale, const int* __restrict__ parent,
             }
         }
     } else {
-    {
-        const int mat = warp >> 2, mb = warp & 3;
-        if (mb < MB) {
-            float acc[2 * MB][4];
+        if (tid == 0) {  // [K] K^T and [Q] K^T: node rows on lanes 0..MP-1
+            tc5::fence_after();
 #pragma unroll
-            for (int t = 0; t < 2 * MB; ++t)
+            for (int kk = 0; kk < TD / 16; ++kk)
+                tc5::mma(tm + TX, tc5::kmajor<MP>(sK, kk), tc5::kmajor<MP>(sK, kk), ID_NN, kk > 0);
 #pragma unroll
-                for (int e = 0; e < 4; ++e) acc[t][e] = 0.f;
+            for (int kk = 0; kk < TD / 16; ++kk)
+                tc5::mma(tm + TY, tc5::kmajor<MP>(sQ, kk), tc5::kmajor<MP>(sK, kk), ID_NN, kk > 0);
+            tc5::commit(&s.bar_mma);
+        }
+        ok = mbar_wait(&s.bar_mma, mph, p.status);
+        mph ^= 1;
+        if (__syncthreads_or(!ok)) return;
+        tc5::fence_after();
+        if (lr < MP) {  // node i = lane row, columns hh * MP/2 ..
+            const int i = lr, j0 = hh * (MP / 2);
+            float kk[MP / 2], qk[MP / 2];
+            ldcols<MP>(kk, trow + TX + j0);
+            ldcols<MP>(qk, trow + TY + j0);
+            tc5::wait_ld();
+            const unsigned long long ai = s.anc[i];
+            const float Gi = s.G[i], bi = s.beta[i];
 #pragma unroll
-            for (int kk = 0; kk < TD / 16; ++kk) {
-                uint32_t a[4];
-                lda<TD>(a, mat ? s.Q : s.K, 16 * mb, 16 * kk);
-#pragma unroll
-                for (int np = 0; np < MB; ++np) {
-                    uint32_t b[4];
-                    ldb_nk<TD>(b, s.K, 16 * np, 16 * kk);
-                    mma16816(acc[2 * np], a, b[0], b[1]);
-                    mma16816(acc[2 * np + 1], a, b[2], b[3]);
-                }
+            for (int c = 0; c < MP / 2; ++c) {
+                const int j = j0 + c;
+                const float d = __expf(Gi - s.G[j]);
+                const bool is_anc = (ai >> j) & 1ull;
+                s.A[i][j] = is_anc ? bi * d * kk[c] : 0.f;
+                qk[c] = (is_anc || j == i) ? scale * d * qk[c] : 0.f;
             }
 #pragma unroll
-            for (int t = 0; t < 2 * MB; ++t)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int i = 16 * mb + (lane >> 2) + 8 * (e >> 1);
-                    const int j = 8 * t + 2 * (lane & 3) + (e & 1);
-                    const bool is_anc = (s.anc[i] >> j) & 1ull;
-                    if (mat == 0) {
-                        s.A[i][j] = is_anc ? s.beta[i] * __expf(s.G[i] - s.G[j]) * acc[t][e] : 0.f;
-                    } else {
-                        const float pv = (is_anc || j == i) ? scale * __expf(s.G[i] - s.G[j]) * acc[t][e] : 0.f;
-                        s.P[swz<64>(i, j)] = __float2bfloat16_rn(pv);
-                    }
-                }
+            for (int c8 = 0; c8 < MP / 16; ++c8)
+                *reinterpret_cast<uint4*>(&s.P[swz<64>(i, j0 + 8 * c8)]) =
+                    make_uint4(pack_bf16(qk[8 * c8], qk[8 * c8 + 1]), pack_bf16(qk[8 * c8 + 2], qk[8 * c8 + 3]),
+                               pack_bf16(qk[8 * c8 + 4], qk[8 * c8 + 5]), pack_bf16(qk[8 * c8 + 6], qk[8 * c8 + 7]));
         }
+        tc5::fence_before();
     }
     __syncthreads();
 
-    }
     // ---- T = (I + A)^{-1}, one tree level at a time --------------------------
     // Row i of T is e_i - sum over ancestors l of A_il T_l, and T_ic is non-zero
     // only for c an ancestor of i or i itself; so every node of one depth is
@@ -244,124 +251,190 @@ tree_verify_kernel(int M, int H, float scale, const int* __restrict__ parent,
         for (int e = tid; e < MP * TD / 2; e += TREE_THREADS) {
             const int i = e / (TD / 2), c = 2 * (e % (TD / 2));
             const float d0 = __expf(s.Gc[i][c]), d1 = __expf(s.Gc[i][c + 1]);
-            uint32_t* kp = reinterpret_cast<uint32_t*>(&s.K[swz<TD>(i, c)]);
-            uint32_t* qp = reinterpret_cast<uint32_t*>(&s.Q[swz<TD>(i, c)]);
+            uint32_t* kp = reinterpret_cast<uint32_t*>(&s.K[toff<MP>(i, c)]);
+            uint32_t* qp = reinterpret_cast<uint32_t*>(&s.Q[toff<MP>(i, c)]);
             const float2 kv = unpack_bf16(*kp), qv = unpack_bf16(*qp);
             *kp = pack_bf16(kv.x * d0, kv.y * d1);
             *qp = pack_bf16(qv.x * d0, qv.y * d1);
         }
     }
+    fence_async_smem();  // P, Tw, Tu (and the scaled tiles) -> tensor-core reads
+    tc5::fence_before();
     __syncthreads();
 
-    // ---- -W = -T diag(beta e^G) K: 16 node rows x 64 key columns per warp ----
-    {
-        const int mb = warp & 3, c0 = 64 * (warp >> 2);
-        if (mb < MB) {
-            float acc[8][4];
+    // ---- W^T = K^T Tw^T (lane = key), U~^T = V^T Tu^T (lane = value) ---------
+    if (tid == 0) {
+        tc5::fence_after();
 #pragma unroll
-            for (int t = 0; t < 8; ++t)
+        for (int kk = 0; kk < MP / 16; ++kk)
+            tc5::mma(tm + TX, tc5::mnmajor(sK, kk, MP * 128), tc5::kmajor<MP>(sTw, kk), ID_MK, kk > 0);
 #pragma unroll
-                for (int e = 0; e < 4; ++e) acc[t][e] = 0.f;
-#pragma unroll
-            for (int kk = 0; kk < MB; ++kk) {
-                uint32_t a[4];
-                lda<64>(a, s.Tw, 16 * mb, 16 * kk);
-#pragma unroll
-                for (int np = 0; np < 4; ++np) {
-                    uint32_t b[4];
-                    ldb_kn<TD>(b, s.K, 16 * kk, c0 + 16 * np);
-                    mma16816(acc[2 * np], a, b[0], b[1]);
-                    mma16816(acc[2 * np + 1], a, b[2], b[3]);
-                }
-            }
-#pragma unroll
-            for (int t = 0; t < 8; ++t) {
-                float ng[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) ng[e] = -acc[t][e];
-                st_c<TD>(s.Wn, 16 * mb, c0 + 8 * t, ng);
-            }
-        }
+        for (int kk = 0; kk < MP / 16; ++kk)
+            tc5::mma(tm + TY, tc5::mnmajor(sV, kk, MP * 128), tc5::kmajor<MP>(sTu, kk), ID_MK, kk > 0);
+        tc5::commit(&s.bar_mma);
     }
-    __syncthreads();  // K is read for the last time above; U takes its place
+    ok = mbar_wait(&s.bar_mma, mph, p.status);
+    mph ^= 1;
+    if (__syncthreads_or(!ok)) return;
+    tc5::fence_after();
+    {   // -W^T (key row lr, nodes hh * MP/2 ..) -> bf16, [key][node]
+        const int j0 = hh * (MP / 2);
+        float w[MP / 2];
+        ldcols<MP>(w, trow + TX + j0);
+        tc5::wait_ld();
+#pragma unroll
+        for (int c8 = 0; c8 < MP / 16; ++c8)
+            *reinterpret_cast<uint4*>(&s.WnT[swz<64>(lr, j0 + 8 * c8)]) =
+                make_uint4(pack_bf16(-w[8 * c8], -w[8 * c8 + 1]), pack_bf16(-w[8 * c8 + 2], -w[8 * c8 + 3]),
+                           pack_bf16(-w[8 * c8 + 4], -w[8 * c8 + 5]), pack_bf16(-w[8 * c8 + 6], -w[8 * c8 + 7]));
+    }
+    fence_async_smem();
+    tc5::fence_before();
+    __syncthreads();
 
-    // ---- U = U~ - W S0^T and O = scale e^G Q S0^T + P U, value rows a0..a0+15 ----
-    const int a0 = 16 * warp;
-    __nv_bfloat16* Ub = s.K;
-    float accu[MB][2][4], acco[MB][2][4];
+    // ---- U^T = U~^T + S0 (-W^T),  Y^T = S0 Q^T (lane = value) ----------------
+    if (tid == 0) {
+        tc5::fence_after();
 #pragma unroll
-    for (int mb = 0; mb < MB; ++mb)
+        for (int kk = 0; kk < TD / 16; ++kk)
+            tc5::mma_ts(tm + TY, tm + TS0 + 8 * kk, tc5::mnmajor(sWnT, kk, TD * 128), ID_KM, true);
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
+        for (int kk = 0; kk < TD / 16; ++kk)
+            tc5::mma_ts(tm + TX, tm + TS0 + 8 * kk, tc5::kmajor<MP>(sQ, kk), ID_NN, kk > 0);
+        tc5::commit(&s.bar_mma);
+    }
+    ok = mbar_wait(&s.bar_mma, mph, p.status);
+    mph ^= 1;
+    if (__syncthreads_or(!ok)) return;
+    tc5::fence_after();
+    {   // U^T -> bf16 A operand (TMEM); Y^T columns *= scale e^{G_i}
+        const int j0 = hh * (MP / 2);
+        float u[MP / 2], y[MP / 2];
+        ldcols<MP>(u, trow + TY + j0);
+        ldcols<MP>(y, trow + TX + j0);
+        tc5::wait_ld();
+        uint32_t pk[MP / 4], yb[MP / 2];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) { accu[mb][nt][e] = 0.f; acco[mb][nt][e] = 0.f; }
+        for (int c = 0; c < MP / 4; ++c) pk[c] = pack_bf16(u[2 * c], u[2 * c + 1]);
 #pragma unroll
-    for (int mb = 0; mb < MB; ++mb)
-#pragma unroll
-        for (int kk = 0; kk <= mb; ++kk) {  // T is lower triangular
-            uint32_t a[4], b[4];
-            lda<64>(a, s.Tu, 16 * mb, 16 * kk);
-            ldb_kn<TD>(b, s.V, 16 * kk, a0);
-            mma16816(accu[mb][0], a, b[0], b[1]);
-            mma16816(accu[mb][1], a, b[2], b[3]);
+        for (int c = 0; c < MP / 2; ++c)
+            yb[c] = __float_as_uint(y[c] * (KDA ? scale : scale * __expf(s.G[j0 + c])));
+        if constexpr (MP == 32) {
+            tc5::st8(trow + TUP + j0 / 2, *reinterpret_cast<uint32_t(*)[8]>(pk));
+            tc5::st16(trow + TX + j0, *reinterpret_cast<uint32_t(*)[16]>(yb));
+        } else {
+            tc5::st16(trow + TUP + j0 / 2, *reinterpret_cast<uint32_t(*)[16]>(pk));
+            tc5::st16(trow + TX + j0, *reinterpret_cast<uint32_t(*)[16]>(yb));
+            tc5::st16(trow + TX + j0 + 16, *reinterpret_cast<uint32_t(*)[16]>(yb + 16));
         }
-    // B fragments of S0^T (B[k = c][n = a] = S0[a][c]) straight from L2, one
-    // K = 16 step at a time, shared by every node block.
-    const float* srow0 = S0 + (size_t)(a0 + (lane >> 2)) * TD + 2 * (lane & 3);
-    const float* srow1 = srow0 + 8 * TD;
+        tc5::wait_st();
+    }
+    tc5::fence_before();
+    __syncthreads();
+
+    // ---- O^T += U^T P^T (A from tensor memory) --------------------------------
+    if (tid == 0) {
+        tc5::fence_after();
 #pragma unroll
-    for (int kk = 0; kk < TD / 16; ++kk) {
-        const float2 x0 = __ldcs(reinterpret_cast<const float2*>(srow0 + 16 * kk));
-        const float2 y0 = __ldcs(reinterpret_cast<const float2*>(srow0 + 16 * kk + 8));
-        const float2 x1 = __ldcs(reinterpret_cast<const float2*>(srow1 + 16 * kk));
-        const float2 y1 = __ldcs(reinterpret_cast<const float2*>(srow1 + 16 * kk + 8));
-        const uint32_t b00 = pack_bf16(x0.x, x0.y), b01 = pack_bf16(y0.x, y0.y);
-        const uint32_t b10 = pack_bf16(x1.x, x1.y), b11 = pack_bf16(y1.x, y1.y);
+        for (int kk = 0; kk < MP / 16; ++kk)
+            tc5::mma_ts(tm + TX, tm + TUP + 8 * kk, tc5::kmajor<MP>(sP, kk), ID_NN, true);
+        tc5::commit(&s.bar_mma);
+    }
+    ok = mbar_wait(&s.bar_mma, mph, p.status);
+    mph ^= 1;
+    if (__syncthreads_or(!ok)) return;
+    tc5::fence_after();
+    {   // O[i][v] for v = lr, nodes hh * MP/2 ..: a warp writes 32 consecutive values
+        const int j0 = hh * (MP / 2);
+        float x[MP / 2];
+        ldcols<MP>(x, trow + TX + j0);
+        tc5::wait_ld();
 #pragma unroll
-        for (int mb = 0; mb < MB; ++mb) {
-            uint32_t a[4];
-            lda<TD>(a, s.Wn, 16 * mb, 16 * kk);
-            mma16816(accu[mb][0], a, b00, b01);
-            mma16816(accu[mb][1], a, b10, b11);
-            lda<TD>(a, s.Q, 16 * mb, 16 * kk);
-            mma16816(acco[mb][0], a, b00, b01);
-            mma16816(acco[mb][1], a, b10, b11);
+        for (int c = 0; c < MP / 2; ++c)
+            if (j0 + c < M) p.o[row0 + (size_t)(j0 + c) * rs + lr] = __float2bfloat16_rn(x[c]);
+    }
+}
+
+// One CTA per (sequence n, head h), MP = 32 (two CTAs per SM) or 64 node rows.
+template <int MP, bool KDA>
+__global__ void __launch_bounds__(TREE_THREADS, MP == 32 ? (KDA ? 2 : 3) : 1)
+tree_verify_kernel(const __grid_constant__ TreePtrs p) {
+    constexpr uint32_t TCOLS = MP == 32 ? 128 : 256;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    TreeSmem<MP, KDA>& s = *reinterpret_cast<TreeSmem<MP, KDA>*>(align_1k(smem_raw));
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int M = p.M, H = p.H;
+    const int nh = blockIdx.x, n = nh / H, h = nh % H;
+    if (tid == 0) {
+        mbar_init(&s.bar_ld, 1);
+        mbar_init(&s.bar_mma, 1);
+        fence_mbar_init();
+        // rows past M hold the next sequence's nodes (or zeros past the
+        // tensor): finite, and masked out of every product that reaches O
+        mbar_arrive_expect(&s.bar_ld, 3 * MP * TD * 2);
+        const int tok = n * M;
+        tma_load_3d(s.K, &p.kmap, 0, h, tok, &s.bar_ld);
+        tma_load_3d(s.K + MP * 64, &p.kmap, 64, h, tok, &s.bar_ld);
+        tma_load_3d(s.Q, &p.qmap, 0, h, tok, &s.bar_ld);
+        tma_load_3d(s.Q + MP * 64, &p.qmap, 64, h, tok, &s.bar_ld);
+        tma_load_3d(s.V, &p.vmap, 0, h, tok, &s.bar_ld);
+        tma_load_3d(s.V + MP * 64, &p.vmap, 64, h, tok, &s.bar_ld);
+        s.maxdepth = 0;
+    }
+    if (warp == 0) tc5::alloc(&s.tmem, TCOLS);
+    if (tid < MP) {
+        int pa = -1;
+        float gi = 0.f, bi = 0.f;
+        if (tid < M) {
+            pa = p.parent[(size_t)n * M + tid];
+            if (pa < -1 || pa >= tid) {  // not a tree in topological order
+                if (p.status) atomicOr(p.status, 2u);
+                pa = -1;
+            }
+            if (!KDA) gi = p.g[((size_t)n * M + tid) * H + h];
+            bi = p.beta[((size_t)n * M + tid) * H + h];
+        }
+        s.par[tid] = pa;
+        s.g[tid] = gi;
+        s.beta[tid] = bi;
+    }
+    if constexpr (KDA) {  // per-key gates of every node (zero past M)
+        for (int e = tid; e < MP * TD / 4; e += TREE_THREADS) {
+            const int i = e / (TD / 4), c4 = e % (TD / 4);
+            cp_async16_zfill(&s.Gc[i][4 * c4], p.g + (((size_t)n * M + (i < M ? i : 0)) * H + h) * TD + 4 * c4,
+                             i < M);
+        }
+        cp_async_commit();
+    }
+    // the state row of this thread's lane (value 32 (warp % 4) + lane), keys
+    // 64 (warp / 4) .. +63, from fp32 to bf16 pairs, into registers now ...
+    uint32_t srow[32];
+    {
+        const int vr = 32 * (warp & 3) + (tid & 31), c0 = 64 * (warp >> 2);
+        const float4* src = reinterpret_cast<const float4*>(p.state + ((size_t)nh * TD + vr) * TD + c0);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            const float4 a = __ldcs(src + j);
+            srow[2 * j] = pack_bf16(a.x, a.y);
+            srow[2 * j + 1] = pack_bf16(a.z, a.w);
         }
     }
-#pragma unroll
-    for (int mb = 0; mb < MB; ++mb) {
-        st_c<TD>(Ub, 16 * mb, a0, accu[mb][0]);
-        st_c<TD>(Ub, 16 * mb, a0 + 8, accu[mb][1]);
-        const int r = 16 * mb + (lane >> 2);
-        const float f0 = KDA ? scale : scale * __expf(s.G[r]), f1 = KDA ? scale : scale * __expf(s.G[r + 8]);
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-            acco[mb][nt][0] *= f0; acco[mb][nt][1] *= f0;
-            acco[mb][nt][2] *= f1; acco[mb][nt][3] *= f1;
-        }
-    }
-    __syncwarp();  // this warp's U columns, written above, are all it reads below
-#pragma unroll
-    for (int mb = 0; mb < MB; ++mb) {
-#pragma unroll
-        for (int kk = 0; kk <= mb; ++kk) {  // P is lower triangular
-            uint32_t a[4], b[4];
-            lda<64>(a, s.P, 16 * mb, 16 * kk);
-            ldb_kn<TD>(b, Ub, 16 * kk, a0);
-            mma16816(acco[mb][0], a, b[0], b[1]);
-            mma16816(acco[mb][1], a, b[2], b[3]);
-        }
-        const int r = 16 * mb + (lane >> 2);
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-            const int col = a0 + 8 * nt + 2 * (lane & 3);
-            if (r < M)
-                *reinterpret_cast<uint32_t*>(o + row0 + (size_t)r * rs + col) =
-                    pack_bf16(acco[mb][nt][0], acco[mb][nt][1]);
-            if (r + 8 < M)
-                *reinterpret_cast<uint32_t*>(o + row0 + (size_t)(r + 8) * rs + col) =
-                    pack_bf16(acco[mb][nt][2], acco[mb][nt][3]);
-        }
+    if constexpr (KDA) cp_async_wait<0>();
+    tc5::fence_before();
+    __syncthreads();
+    tc5::fence_after();
+    const uint32_t tm = s.tmem;
+    // ... and into tensor memory as the A operand of the state products
+    tc5::st16(tm + ((uint32_t)(32 * (warp & 3)) << 16) + 32 * (warp >> 2), *reinterpret_cast<uint32_t(*)[16]>(srow));
+    tc5::st16(tm + ((uint32_t)(32 * (warp & 3)) << 16) + 32 * (warp >> 2) + 16,
+              *reinterpret_cast<uint32_t(*)[16]>(srow + 16));
+    tc5::wait_st();
+    verify_body<MP, KDA>(s, p, tm);
+    tc5::fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc5::fence_after();
+        tc5::dealloc(tm, TCOLS);
     }
 }
 
@@ -384,7 +457,7 @@ tree_commit_kernel(int M, int H, const int* __restrict__ parent, const int* __re
                    const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
                    const float* __restrict__ g, const float* __restrict__ beta,
                    float* __restrict__ state, unsigned int* status) {
-    extern __shared__ __align__(128) unsigned char smem_raw[];
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
     CommitSmem<KDA>& s = *reinterpret_cast<CommitSmem<KDA>*>(smem_raw);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int nh = blockIdx.x, n = nh / H, h = nh % H;
@@ -489,18 +562,22 @@ tree_commit_kernel(int M, int H, const int* __restrict__ parent, const int* __re
     }
 }
 
-template <int MB, bool KDA>
-void launch_verify(int N, int M, int H, float scale, const int* parent, const void* q,
+template <int MP, bool KDA>
+bool launch_verify(int N, int M, int H, float scale, const int* parent, const void* q,
                    const void* k, const void* v, const float* g, const float* beta,
                    const float* state, void* o, unsigned int* status, cudaStream_t st) {
-    const int smem = sizeof(TreeSmem<16 * MB, KDA>);
-    cudaFuncSetAttribute(tree_verify_kernel<MB, KDA>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    GDN_LAUNCH("tree_verify", st,
-               (tree_verify_kernel<MB, KDA><<<(unsigned)(N * H), TREE_THREADS, smem, st>>>(
-                   M, H, scale, parent, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k,
-                   (const __nv_bfloat16*)v, g, beta, state, (__nv_bfloat16*)o, status)));
+    TreePtrs tp{};
+    if (!encode_token_map(&tp.qmap, q, N, M, H, 64, MP) || !encode_token_map(&tp.kmap, k, N, M, H, 64, MP) ||
+        !encode_token_map(&tp.vmap, v, N, M, H, 64, MP))
+        return false;
+    tp.M = M; tp.H = H; tp.scale = scale;
+    tp.parent = parent; tp.g = g; tp.beta = beta; tp.state = state;
+    tp.o = (__nv_bfloat16*)o; tp.status = status;
+    const int smem = sizeof(TreeSmem<MP, KDA>) + 1024;
+    cudaFuncSetAttribute(tree_verify_kernel<MP, KDA>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    GDN_LAUNCH("tree_verify", st, (tree_verify_kernel<MP, KDA><<<(unsigned)(N * H), TREE_THREADS, smem, st>>>(tp)));
+    return true;
 }
-
 bool aligned(const void* p, unsigned a) { return ((uintptr_t)p & (a - 1)) == 0; }
 
 gdn_status check_tree(int N, int M, int H, int dk, int dv, gdn_dtype dtype, gdn_gate gate) {
@@ -538,15 +615,11 @@ gdn_status gdn_tree_verify(int N, int M, int H, int dk, int dv, gdn_dtype dtype,
     cudaGetLastError();
     auto run = [&](auto kda) {
         constexpr bool K = decltype(kda)::value;
-        switch ((M + 15) / 16) {
-            case 1: launch_verify<1, K>(N, M, H, scale, parent, q, k, v, g, beta, state, o, status, st); break;
-            case 2: launch_verify<2, K>(N, M, H, scale, parent, q, k, v, g, beta, state, o, status, st); break;
-            case 3: launch_verify<3, K>(N, M, H, scale, parent, q, k, v, g, beta, state, o, status, st); break;
-            default: launch_verify<4, K>(N, M, H, scale, parent, q, k, v, g, beta, state, o, status, st); break;
-        }
+        if (M <= 32) return launch_verify<32, K>(N, M, H, scale, parent, q, k, v, g, beta, state, o, status, st);
+        return launch_verify<64, K>(N, M, H, scale, parent, q, k, v, g, beta, state, o, status, st);
     };
-    if (gate == GDN_GATE_CHANNEL) run(std::true_type{});
-    else run(std::false_type{});
+    const bool fine = gate == GDN_GATE_CHANNEL ? run(std::true_type{}) : run(std::false_type{});
+    if (!fine) return GDN_ERR_CUDA;
     return launched();
 }
 
