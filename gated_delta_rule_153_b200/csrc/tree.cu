@@ -59,7 +59,7 @@ struct alignas(1024) TreeSmem {
     __nv_bfloat16 K[MP * TD];      // TMA tiles: two 64-column panels of MP node rows,
     __nv_bfloat16 Q[MP * TD];      // 128-byte swizzle
     __nv_bfloat16 V[MP * TD];
-    __nv_bfloat16 WnT[TD * 64];    // -W^T: [key][node], rows of 64 nodes (MN-major B)
+    __nv_bfloat16 Wn[MP * TD];     // -W: [node][key], laid out like the node tiles (K-major B)
     __nv_bfloat16 Tw[MP * 64];     // T diag(beta e^G) (channel gate: T diag(beta)): [i][j]
     __nv_bfloat16 Tu[MP * 64];     // T diag(beta)
     __nv_bfloat16 P[MP * 64];      // scale e^{G_i - G_j} q_i.k_j on ancestors and the diagonal
@@ -105,7 +105,6 @@ GDN_DEV void verify_body(TreeSmem<MP, KDA>& s, const TreePtrs& p, uint32_t tm) {
     constexpr uint32_t TS0 = 0, TX = 64, TY = 64 + MP, TUP = 0;
     constexpr uint32_t ID_NN = tc5::idesc_bf16(128, MP, false, false);
     constexpr uint32_t ID_MK = tc5::idesc_bf16(128, MP, true, false);
-    constexpr uint32_t ID_KM = tc5::idesc_bf16(128, MP, false, true);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int M = p.M, H = p.H;
     const int nh = blockIdx.x, n = nh / H, h = nh % H;
@@ -113,7 +112,7 @@ GDN_DEV void verify_body(TreeSmem<MP, KDA>& s, const TreePtrs& p, uint32_t tm) {
     const size_t row0 = ((size_t)n * M * H + h) * TD;  // node 0 of (n, h)
     const float scale = p.scale;
     const uint32_t sK = smem_u32(s.K), sQ = smem_u32(s.Q), sV = smem_u32(s.V);
-    const uint32_t sWnT = smem_u32(s.WnT), sTw = smem_u32(s.Tw), sTu = smem_u32(s.Tu), sP = smem_u32(s.P);
+    const uint32_t sWn = smem_u32(s.Wn), sTw = smem_u32(s.Tw), sTu = smem_u32(s.Tu), sP = smem_u32(s.P);
     // epilogue thread roles on the 128 lanes: lane quarter warp % 4, column half warp / 4
     const int lr = 32 * (warp & 3) + lane, hh = warp >> 2;
     const uint32_t trow = tm + ((uint32_t)(32 * (warp & 3)) << 16);
@@ -176,35 +175,44 @@ GDN_DEV void verify_body(TreeSmem<MP, KDA>& s, const TreePtrs& p, uint32_t tm) {
             }
         }
     } else {
-        if (tid == 0) {  // [K] K^T and [Q] K^T: node rows on lanes 0..MP-1
+        if (tid == 0) {  // [K ; .] K^T (lanes 0..MP-1) and [. ; Q] K^T (lanes 64..64+MP-1)
             tc5::fence_after();
 #pragma unroll
             for (int kk = 0; kk < TD / 16; ++kk)
                 tc5::mma(tm + TX, tc5::kmajor<MP>(sK, kk), tc5::kmajor<MP>(sK, kk), ID_NN, kk > 0);
+            // (rows 0..63 of this A view are the 8 KB before the Q tile)
 #pragma unroll
             for (int kk = 0; kk < TD / 16; ++kk)
-                tc5::mma(tm + TY, tc5::kmajor<MP>(sQ, kk), tc5::kmajor<MP>(sK, kk), ID_NN, kk > 0);
+                tc5::mma(tm + TY, tc5::kmajor<MP>(sQ - 64 * 128, kk), tc5::kmajor<MP>(sK, kk), ID_NN, kk > 0);
             tc5::commit(&s.bar_mma);
         }
         ok = mbar_wait(&s.bar_mma, mph, p.status);
         mph ^= 1;
         if (__syncthreads_or(!ok)) return;
         tc5::fence_after();
-        if (lr < MP) {  // node i = lane row, columns hh * MP/2 ..
+        if (lr < MP) {  // A row i = lr, columns hh * MP/2 ..
             const int i = lr, j0 = hh * (MP / 2);
-            float kk[MP / 2], qk[MP / 2];
+            float kk[MP / 2];
             ldcols<MP>(kk, trow + TX + j0);
-            ldcols<MP>(qk, trow + TY + j0);
             tc5::wait_ld();
             const unsigned long long ai = s.anc[i];
             const float Gi = s.G[i], bi = s.beta[i];
 #pragma unroll
             for (int c = 0; c < MP / 2; ++c) {
                 const int j = j0 + c;
-                const float d = __expf(Gi - s.G[j]);
-                const bool is_anc = (ai >> j) & 1ull;
-                s.A[i][j] = is_anc ? bi * d * kk[c] : 0.f;
-                qk[c] = (is_anc || j == i) ? scale * d * qk[c] : 0.f;
+                s.A[i][j] = ((ai >> j) & 1ull) ? bi * __expf(Gi - s.G[j]) * kk[c] : 0.f;
+            }
+        } else if (lr >= 64 && lr < 64 + MP) {  // P row i = lr - 64
+            const int i = lr - 64, j0 = hh * (MP / 2);
+            float qk[MP / 2];
+            ldcols<MP>(qk, trow + TY + j0);
+            tc5::wait_ld();
+            const unsigned long long ai = s.anc[i];
+            const float Gi = s.G[i];
+#pragma unroll
+            for (int c = 0; c < MP / 2; ++c) {
+                const int j = j0 + c;
+                qk[c] = (((ai >> j) & 1ull) || j == i) ? scale * __expf(Gi - s.G[j]) * qk[c] : 0.f;
             }
 #pragma unroll
             for (int c8 = 0; c8 < MP / 16; ++c8)
@@ -220,23 +228,27 @@ GDN_DEV void verify_body(TreeSmem<MP, KDA>& s, const TreePtrs& p, uint32_t tm) {
     // Row i of T is e_i - sum over ancestors l of A_il T_l, and T_ic is non-zero
     // only for c an ancestor of i or i itself; so every node of one depth is
     // solved at once from the rows of shallower nodes (a chain: one per level).
-    {
-        const int levels = s.maxdepth;
+    {   // thread = (node i, NC consecutive columns): fixed for every level
+        constexpr int NC = MP * MP / TREE_THREADS;
+        const int i = tid / (MP / NC), c0 = NC * (tid % (MP / NC));
+        const unsigned long long ai = s.anc[i];
+        const int di = s.depth[i], levels = s.maxdepth;
         for (int d = 0; d <= levels; ++d) {
-            for (int e = tid; e < MP * MP; e += TREE_THREADS) {
-                const int i = e / MP, c = e % MP;
-                if (s.depth[i] != d) continue;
-                const unsigned long long ai = s.anc[i];
-                float t = c == i ? 1.f : 0.f;
-                if ((ai >> c) & 1ull) {
-                    float sum = 0.f;
-                    for (unsigned long long m = ai & ~((1ull << c) - 1ull); m; m &= m - 1ull) {
-                        const int l = __ffsll((long long)m) - 1;  // ancestors l >= c
-                        sum += s.A[i][l] * s.T[l][c];
+            if (di == d) {
+#pragma unroll
+                for (int cc = 0; cc < NC; ++cc) {
+                    const int c = c0 + cc;
+                    float t = c == i ? 1.f : 0.f;
+                    if ((ai >> c) & 1ull) {
+                        float sum = 0.f;
+                        for (unsigned long long m = ai & ~((1ull << c) - 1ull); m; m &= m - 1ull) {
+                            const int l = __ffsll((long long)m) - 1;  // ancestors l >= c
+                            sum += s.A[i][l] * s.T[l][c];
+                        }
+                        t = -sum;
                     }
-                    t = -sum;
+                    s.T[i][c] = t;
                 }
-                s.T[i][c] = t;
             }
             __syncthreads();
         }
@@ -273,20 +285,33 @@ GDN_DEV void verify_body(TreeSmem<MP, KDA>& s, const TreePtrs& p, uint32_t tm) {
             tc5::mma(tm + TY, tc5::mnmajor(sV, kk, MP * 128), tc5::kmajor<MP>(sTu, kk), ID_MK, kk > 0);
         tc5::commit(&s.bar_mma);
     }
+    {   // under these products: this lane's state row (value lr, keys 64 hh ..
+        // +63) from fp32 to bf16 pairs, into tensor memory as the A operand of
+        // the state products
+        const float4* src = reinterpret_cast<const float4*>(p.state + ((size_t)nh * TD + lr) * TD + 64 * hh);
+        uint32_t srow[32];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            const float4 a = __ldcs(src + j);
+            srow[2 * j] = pack_bf16(a.x, a.y);
+            srow[2 * j + 1] = pack_bf16(a.z, a.w);
+        }
+        tc5::st16(trow + TS0 + 32 * hh, *reinterpret_cast<uint32_t(*)[16]>(srow));
+        tc5::st16(trow + TS0 + 32 * hh + 16, *reinterpret_cast<uint32_t(*)[16]>(srow + 16));
+        tc5::wait_st();
+    }
     ok = mbar_wait(&s.bar_mma, mph, p.status);
     mph ^= 1;
     if (__syncthreads_or(!ok)) return;
     tc5::fence_after();
-    {   // -W^T (key row lr, nodes hh * MP/2 ..) -> bf16, [key][node]
+    {   // -W (key lr, nodes hh * MP/2 ..) -> bf16 [node][key]: a warp writes 32
+        // consecutive keys of one node row per store
         const int j0 = hh * (MP / 2);
         float w[MP / 2];
         ldcols<MP>(w, trow + TX + j0);
         tc5::wait_ld();
 #pragma unroll
-        for (int c8 = 0; c8 < MP / 16; ++c8)
-            *reinterpret_cast<uint4*>(&s.WnT[swz<64>(lr, j0 + 8 * c8)]) =
-                make_uint4(pack_bf16(-w[8 * c8], -w[8 * c8 + 1]), pack_bf16(-w[8 * c8 + 2], -w[8 * c8 + 3]),
-                           pack_bf16(-w[8 * c8 + 4], -w[8 * c8 + 5]), pack_bf16(-w[8 * c8 + 6], -w[8 * c8 + 7]));
+        for (int c = 0; c < MP / 2; ++c) s.Wn[toff<MP>(j0 + c, lr)] = __float2bfloat16_rn(-w[c]);
     }
     fence_async_smem();
     tc5::fence_before();
@@ -297,7 +322,7 @@ GDN_DEV void verify_body(TreeSmem<MP, KDA>& s, const TreePtrs& p, uint32_t tm) {
         tc5::fence_after();
 #pragma unroll
         for (int kk = 0; kk < TD / 16; ++kk)
-            tc5::mma_ts(tm + TY, tm + TS0 + 8 * kk, tc5::mnmajor(sWnT, kk, TD * 128), ID_KM, true);
+            tc5::mma_ts(tm + TY, tm + TS0 + 8 * kk, tc5::kmajor<MP>(sWn, kk), ID_NN, true);
 #pragma unroll
         for (int kk = 0; kk < TD / 16; ++kk)
             tc5::mma_ts(tm + TX, tm + TS0 + 8 * kk, tc5::kmajor<MP>(sQ, kk), ID_NN, kk > 0);
@@ -406,29 +431,13 @@ tree_verify_kernel(const __grid_constant__ TreePtrs p) {
         }
         cp_async_commit();
     }
-    // the state row of this thread's lane (value 32 (warp % 4) + lane), keys
-    // 64 (warp / 4) .. +63, from fp32 to bf16 pairs, into registers now ...
-    uint32_t srow[32];
-    {
-        const int vr = 32 * (warp & 3) + (tid & 31), c0 = 64 * (warp >> 2);
-        const float4* src = reinterpret_cast<const float4*>(p.state + ((size_t)nh * TD + vr) * TD + c0);
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            const float4 a = __ldcs(src + j);
-            srow[2 * j] = pack_bf16(a.x, a.y);
-            srow[2 * j + 1] = pack_bf16(a.z, a.w);
-        }
-    }
+    if (tid < 4)  // the state, into L2 now; read once the node-side products are under way
+        bulk_prefetch_l2(p.state + (size_t)nh * TD * TD + tid * (TD * TD / 4), TD * TD);
     if constexpr (KDA) cp_async_wait<0>();
     tc5::fence_before();
     __syncthreads();
     tc5::fence_after();
     const uint32_t tm = s.tmem;
-    // ... and into tensor memory as the A operand of the state products
-    tc5::st16(tm + ((uint32_t)(32 * (warp & 3)) << 16) + 32 * (warp >> 2), *reinterpret_cast<uint32_t(*)[16]>(srow));
-    tc5::st16(tm + ((uint32_t)(32 * (warp & 3)) << 16) + 32 * (warp >> 2) + 16,
-              *reinterpret_cast<uint32_t(*)[16]>(srow + 16));
-    tc5::wait_st();
     verify_body<MP, KDA>(s, p, tm);
     tc5::fence_before();
     __syncthreads();
