@@ -41,30 +41,33 @@ constexpr int TREE_THREADS = 256;  // 8 warps
 constexpr int kMaxTreeNodes = 64;
 
 // Verification on the fifth-generation tensor cores.  The node tiles (MP = 32
-// or 64 rows) arrive by TMA; the products whose rows would be nodes run
-// transposed where they touch the state, so the 128 value (or key) rows sit
-// on the TMEM lanes and every warp has work in their epilogues:
-//   [K] K^T, [Q] K^T                 lane = node        (A and P; scalar gate)
-//   W^T  = K^T Tw^T,  U~^T = V^T Tu^T lane = key / value (Tw = T diag(beta e^G),
-//                                                         Tu = T diag(beta))
-//   U^T  = U~^T - S0 W^T,  Y^T = S0 Q^T   lane = value   (S0 as a bf16 A operand
-//                                                         in tensor memory)
-//   O^T  = diag-scaled Y^T + U^T P^T     lane = value   (U^T likewise)
-// Each thread converts its own state row (value lane, 64 keys) from fp32 to
-// bf16 straight into tensor memory, so the state never occupies shared memory.
-// The ancestor masks, the decays and the level-by-level solve for T stay on
-// CUDA cores: they are the tree's small dependent steps, not contractions.
+// or 64 rows) arrive by TMA, K and Q interleaved panel by panel so that one
+// M = 128 product [K ; Q] K^T gives A's rows (lanes 0..MP-1) and P's rows
+// (lanes MP..2MP-1).  W is never formed: with Tu = T diag(beta),
+//   U = U~ - W S0^T = Tu (V - diag(e^G) K S0^T) = Tu Z,
+// so the products that touch the state run transposed, the 128 value rows on
+// the TMEM lanes (every warp has work in their epilogues):
+//   [K ; Q] K^T                 lane = node    A and P (scalar gate)
+//   S0 K^T                      lane = value   -> Z^T = V^T - (S0 K^T) diag(e^G),
+//                                                 written over the V tile
+//   U^T = Z^T Tu^T,  Y^T = S0 Q^T  lane = value
+//   O^T = Y^T diag(scale e^G) + U^T P^T  lane = value
+// The state enters as a bf16 A operand in tensor memory (each thread converts
+// its own row), and so does U^T.  The ancestor masks, the decays and the
+// level-by-level solve for T stay on CUDA cores: they are the tree's small
+// dependent steps, not contractions.  Channel gate: A and P are sums over the
+// keys pair by pair on CUDA cores, and K and Q are scaled by e^G per key in
+// place before the state products (Z = V - (K .* e^G) S0^T, O = scale
+// (Q .* e^G) S0^T + P U).
 template <int MP, bool KDA>
 struct alignas(1024) TreeSmem {
-    __nv_bfloat16 K[MP * TD];      // TMA tiles: two 64-column panels of MP node rows,
-    __nv_bfloat16 Q[MP * TD];      // 128-byte swizzle
-    __nv_bfloat16 V[MP * TD];
-    __nv_bfloat16 Wn[MP * TD];     // -W: [node][key], laid out like the node tiles (K-major B)
-    __nv_bfloat16 Tw[MP * 64];     // T diag(beta e^G) (channel gate: T diag(beta)): [i][j]
-    __nv_bfloat16 Tu[MP * 64];     // T diag(beta)
-    __nv_bfloat16 P[MP * 64];      // scale e^{G_i - G_j} q_i.k_j on ancestors and the diagonal
-    float A[MP][MP + 1];           // masked, decayed beta K K^T
-    float T[MP][MP + 1];           // (I + A)^{-1}
+    __nv_bfloat16 KQ[2 * MP * TD];  // TMA tiles [K p0 | Q p0 | K p1 | Q p1]: 64-column panels of
+                                    // MP node rows, 128-byte swizzle
+    __nv_bfloat16 V[MP * TD];       // two 64-column panels of MP rows; then Z in place
+    __nv_bfloat16 Tu[MP * 64];      // T diag(beta): [i][j] (K-major B: N = i)
+    __nv_bfloat16 P[MP * 64];       // scale e^{G_i - G_j} q_i.k_j on ancestors and the diagonal
+    float A[MP][MP + 1];            // masked, decayed beta K K^T
+    float T[MP][MP + 1];            // (I + A)^{-1}
     float G[MP], g[MP], beta[MP];
     unsigned long long anc[MP];
     int par[MP], depth[MP];
@@ -88,21 +91,32 @@ GDN_DEV unsigned char* align_1k(unsigned char* p) {
     return reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-// Element (row, column) of an MP-row TMA tile (two 64-column panels).
+// Elements (row, column) of K (Q at + MP * 64) in the interleaved tile, and of V.
 template <int MP>
-GDN_DEV int toff(int r, int c) { return (c >> 6) * (MP * 64) + swz<64>(r, c & 63); }
+GDN_DEV int kqoff(int r, int c) { return (c >> 6) * (2 * MP * 64) + swz<64>(r, c & 63); }
+template <int MP>
+GDN_DEV int voff(int r, int c) { return (c >> 6) * (MP * 64) + swz<64>(r, c & 63); }
 
 template <int MP>
 GDN_DEV void ldcols(float* v, uint32_t taddr) {  // MP / 2 columns of this thread's lane
     if constexpr (MP == 32) tc5::ld16(*reinterpret_cast<float(*)[16]>(v), taddr);
     else tc5::ld32(*reinterpret_cast<float(*)[32]>(v), taddr);
 }
+template <int MP>
+GDN_DEV void stcols(uint32_t taddr, const uint32_t* r) {  // MP / 2 32-bit columns
+    if constexpr (MP == 32) {
+        tc5::st16(taddr, *reinterpret_cast<const uint32_t(*)[16]>(r));
+    } else {
+        tc5::st16(taddr, *reinterpret_cast<const uint32_t(*)[16]>(r));
+        tc5::st16(taddr + 16, *reinterpret_cast<const uint32_t(*)[16]>(r + 16));
+    }
+}
 
 template <int MP, bool KDA>
 GDN_DEV void verify_body(TreeSmem<MP, KDA>& s, const TreePtrs& p, uint32_t tm) {
-    // tensor-memory columns: the bf16 state (64), then X and Y (MP each); U^T in
-    // bf16 takes the state's columns once the state products are done
-    constexpr uint32_t TS0 = 0, TX = 64, TY = 64 + MP, TUP = 0;
+    // tensor-memory columns: the bf16 state (64); then [K K^T ; Q K^T] and S0 K^T;
+    // then U^T and Y^T (becoming O^T); U^T in bf16 takes the state's columns
+    constexpr uint32_t TS0 = 0, TKQ = 64, TSK = 64 + MP, TU = 64, TY = 64 + MP, TUP = 0;
     constexpr uint32_t ID_NN = tc5::idesc_bf16(128, MP, false, false);
     constexpr uint32_t ID_MK = tc5::idesc_bf16(128, MP, true, false);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -111,10 +125,10 @@ GDN_DEV void verify_body(TreeSmem<MP, KDA>& s, const TreePtrs& p, uint32_t tm) {
     const size_t rs = (size_t)H * TD;                   // node row stride
     const size_t row0 = ((size_t)n * M * H + h) * TD;  // node 0 of (n, h)
     const float scale = p.scale;
-    const uint32_t sK = smem_u32(s.K), sQ = smem_u32(s.Q), sV = smem_u32(s.V);
-    const uint32_t sWn = smem_u32(s.Wn), sTw = smem_u32(s.Tw), sTu = smem_u32(s.Tu), sP = smem_u32(s.P);
+    const uint32_t sKQ = smem_u32(s.KQ), sQ = sKQ + MP * 128, sV = smem_u32(s.V);
+    const uint32_t sTu = smem_u32(s.Tu), sP = smem_u32(s.P);
     // epilogue thread roles on the 128 lanes: lane quarter warp % 4, column half warp / 4
-    const int lr = 32 * (warp & 3) + lane, hh = warp >> 2;
+    const int lr = 32 * (warp & 3) + lane, hh = warp >> 2, j0 = hh * (MP / 2);
     const uint32_t trow = tm + ((uint32_t)(32 * (warp & 3)) << 16);
     uint32_t mph = 0;
 
@@ -139,10 +153,9 @@ GDN_DEV void verify_body(TreeSmem<MP, KDA>& s, const TreePtrs& p, uint32_t tm) {
     bool ok = mbar_wait(&s.bar_ld, 0, p.status);
     if (__syncthreads_or(!ok)) return;
 
-    // ---- A and P ---------------------------------------------------------
     if constexpr (KDA) {
-        // ancestor pairs (and, for P, the node itself) only; a warp per pair,
-        // a lane per 4 keys; the decays are e^{G_i - G_j} <= 1 key by key
+        // ---- A and P: ancestor pairs (and, for P, the node itself) only; a
+        // warp per pair, a lane per 4 keys; the decays e^{G_i - G_j} <= 1 key by key
         for (int e = tid; e < MP * MP; e += TREE_THREADS) {
             const int i = e / MP, j = e % MP;
             s.A[i][j] = 0.f;
@@ -155,9 +168,9 @@ GDN_DEV void verify_body(TreeSmem<MP, KDA>& s, const TreePtrs& p, uint32_t tm) {
             for (unsigned long long m = s.anc[i] | (1ull << i); m; m &= m - 1ull, ++pc) {
                 if ((pc & 7) != warp) continue;
                 const int j = __ffsll((long long)m) - 1;
-                const uint2 ki = *reinterpret_cast<const uint2*>(&s.K[toff<MP>(i, c)]);
-                const uint2 kj = *reinterpret_cast<const uint2*>(&s.K[toff<MP>(j, c)]);
-                const uint2 qi = *reinterpret_cast<const uint2*>(&s.Q[toff<MP>(i, c)]);
+                const uint2 ki = *reinterpret_cast<const uint2*>(&s.KQ[kqoff<MP>(i, c)]);
+                const uint2 kj = *reinterpret_cast<const uint2*>(&s.KQ[kqoff<MP>(j, c)]);
+                const uint2 qi = *reinterpret_cast<const uint2*>(&s.KQ[MP * 64 + kqoff<MP>(i, c)]);
                 const float2 ki0 = unpack_bf16(ki.x), ki1 = unpack_bf16(ki.y);
                 const float2 kj0 = unpack_bf16(kj.x), kj1 = unpack_bf16(kj.y);
                 const float2 qi0 = unpack_bf16(qi.x), qi1 = unpack_bf16(qi.y);
@@ -174,26 +187,43 @@ GDN_DEV void verify_body(TreeSmem<MP, KDA>& s, const TreePtrs& p, uint32_t tm) {
                 }
             }
         }
-    } else {
-        if (tid == 0) {  // [K ; .] K^T (lanes 0..MP-1) and [. ; Q] K^T (lanes 64..64+MP-1)
-            tc5::fence_after();
-#pragma unroll
-            for (int kk = 0; kk < TD / 16; ++kk)
-                tc5::mma(tm + TX, tc5::kmajor<MP>(sK, kk), tc5::kmajor<MP>(sK, kk), ID_NN, kk > 0);
-            // (rows 0..63 of this A view are the 8 KB before the Q tile)
-#pragma unroll
-            for (int kk = 0; kk < TD / 16; ++kk)
-                tc5::mma(tm + TY, tc5::kmajor<MP>(sQ - 64 * 128, kk), tc5::kmajor<MP>(sK, kk), ID_NN, kk > 0);
-            tc5::commit(&s.bar_mma);
+        __syncthreads();
+        // K .* e^G (for Z) and Q .* e^G (the read-out), in place
+        for (int e = tid; e < MP * TD / 2; e += TREE_THREADS) {
+            const int i = e / (TD / 2), c2 = 2 * (e % (TD / 2));
+            const float d0 = __expf(s.Gc[i][c2]), d1 = __expf(s.Gc[i][c2 + 1]);
+            uint32_t* kp = reinterpret_cast<uint32_t*>(&s.KQ[kqoff<MP>(i, c2)]);
+            uint32_t* qp = reinterpret_cast<uint32_t*>(&s.KQ[MP * 64 + kqoff<MP>(i, c2)]);
+            const float2 kv = unpack_bf16(*kp), qv = unpack_bf16(*qp);
+            *kp = pack_bf16(kv.x * d0, kv.y * d1);
+            *qp = pack_bf16(qv.x * d0, qv.y * d1);
         }
-        ok = mbar_wait(&s.bar_mma, mph, p.status);
-        mph ^= 1;
-        if (__syncthreads_or(!ok)) return;
+        fence_async_smem();
+        tc5::fence_before();
+        __syncthreads();
+    }
+    // ---- [K ; Q] K^T (scalar gate) and S0 K^T -----------------------------------
+    if (tid == 0) {
         tc5::fence_after();
-        if (lr < MP) {  // A row i = lr, columns hh * MP/2 ..
-            const int i = lr, j0 = hh * (MP / 2);
+        if constexpr (!KDA) {
+#pragma unroll
+            for (int kk = 0; kk < TD / 16; ++kk)
+                tc5::mma(tm + TKQ, tc5::kmajor<2 * MP>(sKQ, kk), tc5::kmajor<2 * MP>(sKQ, kk), ID_NN, kk > 0);
+        }
+#pragma unroll
+        for (int kk = 0; kk < TD / 16; ++kk)
+            tc5::mma_ts(tm + TSK, tm + TS0 + 8 * kk, tc5::kmajor<2 * MP>(sKQ, kk), ID_NN, kk > 0);
+        tc5::commit(&s.bar_mma);
+    }
+    ok = mbar_wait(&s.bar_mma, mph, p.status);
+    mph ^= 1;
+    if (__syncthreads_or(!ok)) return;
+    tc5::fence_after();
+    if constexpr (!KDA) {
+        if (lr < MP) {  // A row i = lr, columns j0 ..
+            const int i = lr;
             float kk[MP / 2];
-            ldcols<MP>(kk, trow + TX + j0);
+            ldcols<MP>(kk, trow + TKQ + j0);
             tc5::wait_ld();
             const unsigned long long ai = s.anc[i];
             const float Gi = s.G[i], bi = s.beta[i];
@@ -202,10 +232,10 @@ GDN_DEV void verify_body(TreeSmem<MP, KDA>& s, const TreePtrs& p, uint32_t tm) {
                 const int j = j0 + c;
                 s.A[i][j] = ((ai >> j) & 1ull) ? bi * __expf(Gi - s.G[j]) * kk[c] : 0.f;
             }
-        } else if (lr >= 64 && lr < 64 + MP) {  // P row i = lr - 64
-            const int i = lr - 64, j0 = hh * (MP / 2);
+        } else if (lr < 2 * MP) {  // P row i = lr - MP
+            const int i = lr - MP;
             float qk[MP / 2];
-            ldcols<MP>(qk, trow + TY + j0);
+            ldcols<MP>(qk, trow + TKQ + j0);
             tc5::wait_ld();
             const unsigned long long ai = s.anc[i];
             const float Gi = s.G[i];
@@ -220,8 +250,19 @@ GDN_DEV void verify_body(TreeSmem<MP, KDA>& s, const TreePtrs& p, uint32_t tm) {
                     make_uint4(pack_bf16(qk[8 * c8], qk[8 * c8 + 1]), pack_bf16(qk[8 * c8 + 2], qk[8 * c8 + 3]),
                                pack_bf16(qk[8 * c8 + 4], qk[8 * c8 + 5]), pack_bf16(qk[8 * c8 + 6], qk[8 * c8 + 7]));
         }
-        tc5::fence_before();
     }
+    {   // Z^T = V^T - (S0 K^T) diag(e^G): value lr, nodes j0 .., over the V tile
+        float sk[MP / 2];
+        ldcols<MP>(sk, trow + TSK + j0);
+        tc5::wait_ld();
+#pragma unroll
+        for (int c = 0; c < MP / 2; ++c) {
+            __nv_bfloat16& vz = s.V[voff<MP>(j0 + c, lr)];
+            const float f = KDA ? 1.f : __expf(s.G[j0 + c]);
+            vz = __float2bfloat16_rn(__bfloat162float(vz) - f * sk[c]);
+        }
+    }
+    tc5::fence_before();
     __syncthreads();
 
     // ---- T = (I + A)^{-1}, one tree level at a time --------------------------
@@ -255,88 +296,31 @@ GDN_DEV void verify_body(TreeSmem<MP, KDA>& s, const TreePtrs& p, uint32_t tm) {
     }
     for (int e = tid; e < MP * MP; e += TREE_THREADS) {
         const int i = e / MP, j = e % MP;
-        const float t = s.T[i][j] * s.beta[j];
-        s.Tw[swz<64>(i, j)] = __float2bfloat16_rn(KDA ? t : t * __expf(s.G[j]));
-        s.Tu[swz<64>(i, j)] = __float2bfloat16_rn(t);
+        s.Tu[swz<64>(i, j)] = __float2bfloat16_rn(s.T[i][j] * s.beta[j]);
     }
-    if constexpr (KDA) {  // K .* e^G (the rows of W) and Q .* e^G (the read-out), in place
-        for (int e = tid; e < MP * TD / 2; e += TREE_THREADS) {
-            const int i = e / (TD / 2), c = 2 * (e % (TD / 2));
-            const float d0 = __expf(s.Gc[i][c]), d1 = __expf(s.Gc[i][c + 1]);
-            uint32_t* kp = reinterpret_cast<uint32_t*>(&s.K[toff<MP>(i, c)]);
-            uint32_t* qp = reinterpret_cast<uint32_t*>(&s.Q[toff<MP>(i, c)]);
-            const float2 kv = unpack_bf16(*kp), qv = unpack_bf16(*qp);
-            *kp = pack_bf16(kv.x * d0, kv.y * d1);
-            *qp = pack_bf16(qv.x * d0, qv.y * d1);
-        }
-    }
-    fence_async_smem();  // P, Tw, Tu (and the scaled tiles) -> tensor-core reads
+    fence_async_smem();  // Z, P and Tu (generic writes) -> tensor-core reads
     tc5::fence_before();
     __syncthreads();
 
-    // ---- W^T = K^T Tw^T (lane = key), U~^T = V^T Tu^T (lane = value) ---------
+    // ---- U^T = Z^T Tu^T,  Y^T = S0 Q^T (lane = value) ----------------------------
     if (tid == 0) {
         tc5::fence_after();
 #pragma unroll
         for (int kk = 0; kk < MP / 16; ++kk)
-            tc5::mma(tm + TX, tc5::mnmajor(sK, kk, MP * 128), tc5::kmajor<MP>(sTw, kk), ID_MK, kk > 0);
-#pragma unroll
-        for (int kk = 0; kk < MP / 16; ++kk)
-            tc5::mma(tm + TY, tc5::mnmajor(sV, kk, MP * 128), tc5::kmajor<MP>(sTu, kk), ID_MK, kk > 0);
-        tc5::commit(&s.bar_mma);
-    }
-    {   // under these products: this lane's state row (value lr, keys 64 hh ..
-        // +63) from fp32 to bf16 pairs, into tensor memory as the A operand of
-        // the state products
-        const float4* src = reinterpret_cast<const float4*>(p.state + ((size_t)nh * TD + lr) * TD + 64 * hh);
-        uint32_t srow[32];
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            const float4 a = __ldcs(src + j);
-            srow[2 * j] = pack_bf16(a.x, a.y);
-            srow[2 * j + 1] = pack_bf16(a.z, a.w);
-        }
-        tc5::st16(trow + TS0 + 32 * hh, *reinterpret_cast<uint32_t(*)[16]>(srow));
-        tc5::st16(trow + TS0 + 32 * hh + 16, *reinterpret_cast<uint32_t(*)[16]>(srow + 16));
-        tc5::wait_st();
-    }
-    ok = mbar_wait(&s.bar_mma, mph, p.status);
-    mph ^= 1;
-    if (__syncthreads_or(!ok)) return;
-    tc5::fence_after();
-    {   // -W (key lr, nodes hh * MP/2 ..) -> bf16 [node][key]: a warp writes 32
-        // consecutive keys of one node row per store
-        const int j0 = hh * (MP / 2);
-        float w[MP / 2];
-        ldcols<MP>(w, trow + TX + j0);
-        tc5::wait_ld();
-#pragma unroll
-        for (int c = 0; c < MP / 2; ++c) s.Wn[toff<MP>(j0 + c, lr)] = __float2bfloat16_rn(-w[c]);
-    }
-    fence_async_smem();
-    tc5::fence_before();
-    __syncthreads();
-
-    // ---- U^T = U~^T + S0 (-W^T),  Y^T = S0 Q^T (lane = value) ----------------
-    if (tid == 0) {
-        tc5::fence_after();
+            tc5::mma(tm + TU, tc5::mnmajor(sV, kk, MP * 128), tc5::kmajor<MP>(sTu, kk), ID_MK, kk > 0);
 #pragma unroll
         for (int kk = 0; kk < TD / 16; ++kk)
-            tc5::mma_ts(tm + TY, tm + TS0 + 8 * kk, tc5::kmajor<MP>(sWn, kk), ID_NN, true);
-#pragma unroll
-        for (int kk = 0; kk < TD / 16; ++kk)
-            tc5::mma_ts(tm + TX, tm + TS0 + 8 * kk, tc5::kmajor<MP>(sQ, kk), ID_NN, kk > 0);
+            tc5::mma_ts(tm + TY, tm + TS0 + 8 * kk, tc5::kmajor<2 * MP>(sQ, kk), ID_NN, kk > 0);
         tc5::commit(&s.bar_mma);
     }
     ok = mbar_wait(&s.bar_mma, mph, p.status);
     mph ^= 1;
     if (__syncthreads_or(!ok)) return;
     tc5::fence_after();
-    {   // U^T -> bf16 A operand (TMEM); Y^T columns *= scale e^{G_i}
-        const int j0 = hh * (MP / 2);
+    {   // U^T -> bf16 A operand (over the state's columns); Y^T columns *= scale e^{G_i}
         float u[MP / 2], y[MP / 2];
-        ldcols<MP>(u, trow + TY + j0);
-        ldcols<MP>(y, trow + TX + j0);
+        ldcols<MP>(u, trow + TU + j0);
+        ldcols<MP>(y, trow + TY + j0);
         tc5::wait_ld();
         uint32_t pk[MP / 4], yb[MP / 2];
 #pragma unroll
@@ -344,35 +328,29 @@ GDN_DEV void verify_body(TreeSmem<MP, KDA>& s, const TreePtrs& p, uint32_t tm) {
 #pragma unroll
         for (int c = 0; c < MP / 2; ++c)
             yb[c] = __float_as_uint(y[c] * (KDA ? scale : scale * __expf(s.G[j0 + c])));
-        if constexpr (MP == 32) {
-            tc5::st8(trow + TUP + j0 / 2, *reinterpret_cast<uint32_t(*)[8]>(pk));
-            tc5::st16(trow + TX + j0, *reinterpret_cast<uint32_t(*)[16]>(yb));
-        } else {
-            tc5::st16(trow + TUP + j0 / 2, *reinterpret_cast<uint32_t(*)[16]>(pk));
-            tc5::st16(trow + TX + j0, *reinterpret_cast<uint32_t(*)[16]>(yb));
-            tc5::st16(trow + TX + j0 + 16, *reinterpret_cast<uint32_t(*)[16]>(yb + 16));
-        }
+        if constexpr (MP == 32) tc5::st8(trow + TUP + j0 / 2, *reinterpret_cast<uint32_t(*)[8]>(pk));
+        else tc5::st16(trow + TUP + j0 / 2, *reinterpret_cast<uint32_t(*)[16]>(pk));
+        stcols<MP>(trow + TY + j0, yb);
         tc5::wait_st();
     }
     tc5::fence_before();
     __syncthreads();
 
-    // ---- O^T += U^T P^T (A from tensor memory) --------------------------------
+    // ---- O^T = Y^T + U^T P^T (A from tensor memory) ------------------------------
     if (tid == 0) {
         tc5::fence_after();
 #pragma unroll
         for (int kk = 0; kk < MP / 16; ++kk)
-            tc5::mma_ts(tm + TX, tm + TUP + 8 * kk, tc5::kmajor<MP>(sP, kk), ID_NN, true);
+            tc5::mma_ts(tm + TY, tm + TUP + 8 * kk, tc5::kmajor<MP>(sP, kk), ID_NN, true);
         tc5::commit(&s.bar_mma);
     }
     ok = mbar_wait(&s.bar_mma, mph, p.status);
     mph ^= 1;
     if (__syncthreads_or(!ok)) return;
     tc5::fence_after();
-    {   // O[i][v] for v = lr, nodes hh * MP/2 ..: a warp writes 32 consecutive values
-        const int j0 = hh * (MP / 2);
+    {   // O[i][v] for v = lr, nodes j0 ..: a warp writes 32 consecutive values
         float x[MP / 2];
-        ldcols<MP>(x, trow + TX + j0);
+        ldcols<MP>(x, trow + TY + j0);
         tc5::wait_ld();
 #pragma unroll
         for (int c = 0; c < MP / 2; ++c)
@@ -380,9 +358,9 @@ GDN_DEV void verify_body(TreeSmem<MP, KDA>& s, const TreePtrs& p, uint32_t tm) {
     }
 }
 
-// One CTA per (sequence n, head h), MP = 32 (two CTAs per SM) or 64 node rows.
+// One CTA per (sequence n, head h), MP = 32 (three CTAs per SM) or 64 node rows.
 template <int MP, bool KDA>
-__global__ void __launch_bounds__(TREE_THREADS, MP == 32 ? (KDA ? 2 : 3) : 1)
+__global__ void __launch_bounds__(TREE_THREADS, MP == 32 ? 3 : 1)
 tree_verify_kernel(const __grid_constant__ TreePtrs p) {
     constexpr uint32_t TCOLS = MP == 32 ? 128 : 256;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -398,10 +376,10 @@ tree_verify_kernel(const __grid_constant__ TreePtrs p) {
         // tensor): finite, and masked out of every product that reaches O
         mbar_arrive_expect(&s.bar_ld, 3 * MP * TD * 2);
         const int tok = n * M;
-        tma_load_3d(s.K, &p.kmap, 0, h, tok, &s.bar_ld);
-        tma_load_3d(s.K + MP * 64, &p.kmap, 64, h, tok, &s.bar_ld);
-        tma_load_3d(s.Q, &p.qmap, 0, h, tok, &s.bar_ld);
-        tma_load_3d(s.Q + MP * 64, &p.qmap, 64, h, tok, &s.bar_ld);
+        tma_load_3d(s.KQ, &p.kmap, 0, h, tok, &s.bar_ld);
+        tma_load_3d(s.KQ + MP * 64, &p.qmap, 0, h, tok, &s.bar_ld);
+        tma_load_3d(s.KQ + 2 * MP * 64, &p.kmap, 64, h, tok, &s.bar_ld);
+        tma_load_3d(s.KQ + 3 * MP * 64, &p.qmap, 64, h, tok, &s.bar_ld);
         tma_load_3d(s.V, &p.vmap, 0, h, tok, &s.bar_ld);
         tma_load_3d(s.V + MP * 64, &p.vmap, 64, h, tok, &s.bar_ld);
         s.maxdepth = 0;
@@ -431,13 +409,30 @@ tree_verify_kernel(const __grid_constant__ TreePtrs p) {
         }
         cp_async_commit();
     }
-    if (tid < 4)  // the state, into L2 now; read once the node-side products are under way
-        bulk_prefetch_l2(p.state + (size_t)nh * TD * TD + tid * (TD * TD / 4), TD * TD);
+    // the state row of this thread's lane (value 32 (warp % 4) + lane), keys
+    // 64 (warp / 4) .. +63, from fp32 to bf16 pairs ...
+    uint32_t srow[32];
+    {
+        const float4* src = reinterpret_cast<const float4*>(
+            p.state + ((size_t)nh * TD + 32 * (warp & 3) + (tid & 31)) * TD + 64 * (warp >> 2));
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            const float4 a = __ldcs(src + j);
+            srow[2 * j] = pack_bf16(a.x, a.y);
+            srow[2 * j + 1] = pack_bf16(a.z, a.w);
+        }
+    }
     if constexpr (KDA) cp_async_wait<0>();
     tc5::fence_before();
     __syncthreads();
     tc5::fence_after();
     const uint32_t tm = s.tmem;
+    {   // ... into tensor memory as the A operand of the state products
+        const uint32_t ta = tm + ((uint32_t)(32 * (warp & 3)) << 16) + 32 * (warp >> 2);
+        tc5::st16(ta, *reinterpret_cast<uint32_t(*)[16]>(srow));
+        tc5::st16(ta + 16, *reinterpret_cast<uint32_t(*)[16]>(srow + 16));
+        tc5::wait_st();
+    }
     verify_body<MP, KDA>(s, p, tm);
     tc5::fence_before();
     __syncthreads();
@@ -445,6 +440,23 @@ tree_verify_kernel(const __grid_constant__ TreePtrs p) {
         tc5::fence_after();
         tc5::dealloc(tm, TCOLS);
     }
+}
+
+template <int MP, bool KDA>
+bool launch_verify(int N, int M, int H, float scale, const int* parent, const void* q,
+                   const void* k, const void* v, const float* g, const float* beta,
+                   const float* state, void* o, unsigned int* status, cudaStream_t st) {
+    TreePtrs tp{};
+    if (!encode_token_map(&tp.qmap, q, N, M, H, 64, MP) || !encode_token_map(&tp.kmap, k, N, M, H, 64, MP) ||
+        !encode_token_map(&tp.vmap, v, N, M, H, 64, MP))
+        return false;
+    tp.M = M; tp.H = H; tp.scale = scale;
+    tp.parent = parent; tp.g = g; tp.beta = beta; tp.state = state;
+    tp.o = (__nv_bfloat16*)o; tp.status = status;
+    const int smem = sizeof(TreeSmem<MP, KDA>) + 1024;
+    cudaFuncSetAttribute(tree_verify_kernel<MP, KDA>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    GDN_LAUNCH("tree_verify", st, (tree_verify_kernel<MP, KDA><<<(unsigned)(N * H), TREE_THREADS, smem, st>>>(tp)));
+    return true;
 }
 
 // ---- commit: the recurrent form along the accepted node's root path --------
@@ -571,22 +583,6 @@ tree_commit_kernel(int M, int H, const int* __restrict__ parent, const int* __re
     }
 }
 
-template <int MP, bool KDA>
-bool launch_verify(int N, int M, int H, float scale, const int* parent, const void* q,
-                   const void* k, const void* v, const float* g, const float* beta,
-                   const float* state, void* o, unsigned int* status, cudaStream_t st) {
-    TreePtrs tp{};
-    if (!encode_token_map(&tp.qmap, q, N, M, H, 64, MP) || !encode_token_map(&tp.kmap, k, N, M, H, 64, MP) ||
-        !encode_token_map(&tp.vmap, v, N, M, H, 64, MP))
-        return false;
-    tp.M = M; tp.H = H; tp.scale = scale;
-    tp.parent = parent; tp.g = g; tp.beta = beta; tp.state = state;
-    tp.o = (__nv_bfloat16*)o; tp.status = status;
-    const int smem = sizeof(TreeSmem<MP, KDA>) + 1024;
-    cudaFuncSetAttribute(tree_verify_kernel<MP, KDA>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    GDN_LAUNCH("tree_verify", st, (tree_verify_kernel<MP, KDA><<<(unsigned)(N * H), TREE_THREADS, smem, st>>>(tp)));
-    return true;
-}
 bool aligned(const void* p, unsigned a) { return ((uintptr_t)p & (a - 1)) == 0; }
 
 gdn_status check_tree(int N, int M, int H, int dk, int dv, gdn_dtype dtype, gdn_gate gate) {
