@@ -358,9 +358,10 @@ GDN_DEV void verify_body(TreeSmem<MP, KDA>& s, const TreePtrs& p, uint32_t tm) {
     }
 }
 
-// One CTA per (sequence n, head h), MP = 32 (three CTAs per SM) or 64 node rows.
+// One CTA per (sequence n, head h), MP = 32 (four CTAs per SM; three with the
+// channel gate's per-key path sums) or 64 node rows.
 template <int MP, bool KDA>
-__global__ void __launch_bounds__(TREE_THREADS, MP == 32 ? 3 : 1)
+__global__ void __launch_bounds__(TREE_THREADS, MP == 32 ? (KDA ? 3 : 4) : 1)
 tree_verify_kernel(const __grid_constant__ TreePtrs p) {
     constexpr uint32_t TCOLS = MP == 32 ? 128 : 256;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
