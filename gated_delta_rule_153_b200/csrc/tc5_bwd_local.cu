@@ -208,19 +208,14 @@ GDN_DEV void load_k(BlSmem& s, const BlPtrs& p, const BlChunk& c) {  // K (rows 
     tma_load_3d(s.R2, &p.kmap, 0, c.h, c.tok, &s.bar_k);
     tma_load_3d(s.R2 + PAIR, &p.kmap, 64, c.h, c.tok, &s.bar_k);
 }
-// Everything chunk c reads, into L2 (thread 0, a chunk ahead of its loads).
+// The first buffers chunk c loads (U, S0, dS: 80 KB), into L2 a chunk ahead.
+// The prefetches run on the TMA engine with the loads themselves; the rest of
+// the chunk's buffers load late enough from DRAM (measured: prefetching the
+// tiles and the other images as well is slower).
 GDN_DEV void prefetch_chunk(const BlPtrs& p, const BlChunk& c) {
-    tma_prefetch_tile(&p.dOmap, c.h, c.tok);
-    tma_prefetch_tile(&p.qmap, c.h, c.tok);
-    tma_prefetch_tile(&p.kmap, c.h, c.tok);
-    tma_prefetch_tile(&p.vmap, c.h, c.tok);
     bulk_prefetch_l2(p.U + (size_t)c.cid * C * DV, C * DV * 2);
-    bulk_prefetch_l2(p.dU + (size_t)c.cid * C * DV, C * DV * 2);
     bulk_prefetch_l2(p.S0 + (size_t)c.cid * DV * DK, DV * DK * 2);
     bulk_prefetch_l2(p.dS + (size_t)c.cid * DV * DK, DV * DK * 2);
-    bulk_prefetch_l2(p.Tb + (size_t)c.cid * C * C, C * C * 2);
-    bulk_prefetch_l2(p.W + (size_t)c.cid * C * DK, C * DK * 2);
-    bulk_prefetch_l2(p.Ut + (size_t)c.cid * DV * C, DV * C * 2);
 }
 
 // G (within-chunk cumsum of g) and beta of chunk c into slot b (one warp).
