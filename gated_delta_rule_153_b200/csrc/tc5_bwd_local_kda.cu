@@ -159,21 +159,8 @@ __global__ void __launch_bounds__(KB_THREADS, 1) tc5_bwd_local_kda_kernel(const 
         bulk_g2s(s.R4, p.S0 + (size_t)cid * DV * DK, DV * DK * 2, &s.bar_ld);
         bulk_g2s(s.R5, p.dS + (size_t)cid * DV * DK, DV * DK * 2, &s.bar_ld);
         bulk_g2s(s.T, p.Tb + (size_t)cid * C * C, C * C * 2, &s.bar_ld);
-        const int pc = cid + p.pf_stride;  // the chunk a wave ahead waits in L2
-        if (p.pf_stride > 0 && pc < (int)gridDim.x) {
-            const int pbh = pc / p.NT, pn = pc % p.NT, ph = pbh % p.H;
-            const ChunkLoc pl = chunk_loc(p.seq, p.T, p.H, pbh, pn);
-            const int ptok = pl.valid ? pl.tok : 0;
-            tma_prefetch_tile(&p.dOmap, ph, ptok);
-            tma_prefetch_tile(&p.qmap, ph, ptok);
-            tma_prefetch_tile(&p.kmap, ph, ptok);
-            tma_prefetch_tile(&p.vmap, ph, ptok);
-            bulk_prefetch_l2(p.U + (size_t)pc * C * DV, C * DV * 2);
-            bulk_prefetch_l2(p.dU + (size_t)pc * C * DV, C * DV * 2);
-            bulk_prefetch_l2(p.S0 + (size_t)pc * DV * DK, DV * DK * 2);
-            bulk_prefetch_l2(p.dS + (size_t)pc * DV * DK, DV * DK * 2);
-            bulk_prefetch_l2(p.Tb + (size_t)pc * C * C, C * C * 2);
-        }
+        // (no L2 prefetch of the next wave's tiles and images: measured slower,
+        // the prefetches share the TMA engine with the loads themselves)
     }
     if (warp == 0) tc5::alloc(&s.tmem, KB_TCOLS);
     if (tid < C) s.beta[tid] = tid < L ? p.beta[row0 + tid * rs] : 0.f;

@@ -92,11 +92,12 @@ struct W5Cfg {
     static constexpr bool STAGED = MODE == 3;
     static constexpr int STAGES = MODE == 0 ? 3 : 2;
     static constexpr int THREADS = 32 * (W5_EPI_WARPS + 2 + (STAGED ? 1 : 0));
-    // tensor-memory columns.  Forward: [X|Y] 0..127, D, Z, then the A operands
-    // S (bf16 pairs) and U.  Lean: X and D share columns 0..127 (D is issued
-    // only after the epilogue has read X), so two CTAs fit an SM.
+    // tensor-memory columns.  Forward: [X|Y] 0..127, D, Z (two buffers, by
+    // step parity: a step's output is read during the next step), then the A
+    // operands S (bf16 pairs) and U.  Lean: X and D share columns 0..127 (D is
+    // issued only after the epilogue has read X), so two CTAs fit an SM.
     static constexpr int TXY = 0, TD = FULL ? 128 : 0, TZ = 256, TAS = FULL ? 320 : 128,
-                         TAU = FULL ? 384 : 192, TCOLS = FULL ? 512 : 256;
+                         TAU = FULL ? 384 : 192, TZ2 = 448, TCOLS = FULL ? 512 : 256;
 };
 
 // The staged state images of MODE 3 and their hand-off barriers
@@ -116,7 +117,7 @@ struct W5Smem {
     __nv_bfloat16 I16[16 * 64];  // 16x16 identity, Swz<64> rows: B of X += U~^T
     float G[W5Cfg<MODE>::STAGES][DK];  // G (scalar gate, C used) or e^{G_last,c}
     uint64_t full[W5Cfg<MODE>::STAGES], empty[W5Cfg<MODE>::STAGES];
-    uint64_t s_ready, u_ready, x_done, d_done, o_done, fin;
+    uint64_t s_ready, u_ready, x_done, d_done, o_done[2], fin;
     uint32_t tmem;
 };
 
@@ -253,7 +254,8 @@ __global__ void __launch_bounds__(W5Cfg<MODE>::THREADS) tc5_walk_kernel(const __
         mbar_init(&s.u_ready, W5_EPI_WARPS);
         mbar_init(&s.x_done, 1);
         mbar_init(&s.d_done, 1);
-        mbar_init(&s.o_done, 1);
+        mbar_init(&s.o_done[0], 1);
+        mbar_init(&s.o_done[1], 1);
         mbar_init(&s.fin, 1);
         if constexpr (Cfg::STAGED) {
             for (int i = 0; i < 2; ++i) {
@@ -329,12 +331,12 @@ __global__ void __launch_bounds__(W5Cfg<MODE>::THREADS) tc5_walk_kernel(const __
                     tc5::mma_ts(tm + Cfg::TD, tm + Cfg::TAU + 8 * kk, tc5::mnmajor(sK, kk, C * 128), ID_D,
                                 kk > 0);
                 tc5::commit(&s.d_done);
-                if constexpr (Cfg::FULL) {
-                    const uint32_t sP = smem_u32(st.P);
+                if constexpr (Cfg::FULL) {  // onto -scale e^{G_i} Y, stored by the epilogue
+                    const uint32_t sP = smem_u32(st.P), tz = tm + ((n & 1) ? Cfg::TZ2 : Cfg::TZ);
 #pragma unroll
                     for (int kk = 0; kk < C / 16; ++kk)
-                        tc5::mma_ts(tm + Cfg::TZ, tm + Cfg::TAU + 8 * kk, tc5::kmajor<C>(sP, kk), ID_Z, kk > 0);
-                    tc5::commit(&s.o_done);
+                        tc5::mma_ts(tz, tm + Cfg::TAU + 8 * kk, tc5::kmajor<C>(sP, kk), ID_Z, true);
+                    tc5::commit(&s.o_done[n & 1]);
                 }
                 tc5::commit(&s.empty[sn]);
             }
@@ -417,6 +419,22 @@ __global__ void __launch_bounds__(W5Cfg<MODE>::THREADS) tc5_walk_kernel(const __
             }
             return true;
         };
+        // O^T of step m (tokens t0 .. t0+15 of value row a) from its Z buffer
+        auto store_out = [&](int m) {
+            if (!wait_all(&s.o_done[m & 1], (m >> 1) & 1, p.status, p.wait_ns)) return false;
+            tc5::fence_after();
+            const int cm = n_begin + m;
+            const int Lm = min(C, ch.end - (ch.tok0 + cm * C));
+            float z[16];
+            tc5::ld16(z, trow + ((m & 1) ? Cfg::TZ2 : Cfg::TZ) + t0);
+            tc5::wait_ld();
+            __nv_bfloat16* o = p.o + (((size_t)ch.tok0 + cm * C + t0) * p.H + h) * DV + a;
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+                if (t0 + j < Lm) o[(size_t)j * p.H * DV] = __float2bfloat16_rn(z[j]);
+            return true;
+        };
+        int done_steps = 0;
         store_state();
         if (Cfg::SAVE && nsteps > 0) store_s0(n_begin);
         tc5::fence_before();
@@ -438,12 +456,12 @@ __global__ void __launch_bounds__(W5Cfg<MODE>::THREADS) tc5_walk_kernel(const __
                 sce = p.scale * __expf(G[t0 + (lane & 15)]);
                 warp_arrive(&s.empty[sn]);
             }
-            // ---- U = X (= U~ - S0 W^T); -Y kept for the output -------------
+            // ---- U = X (= U~ - S0 W^T); -scale e^{G_i} Y into this step's Z
+            // buffer, onto which the MMA thread adds U^T P^T: the output ----------
             if (!wait_all(&s.x_done, n & 1, p.status, p.wait_ns)) break;
             tc5::fence_after();
-            float y[16];
             {
-                float x[16];
+                float x[16], y[16];
                 tc5::ld16(x, trow + Cfg::TXY + t0);
                 if (Cfg::FULL) tc5::ld16(y, trow + Cfg::TXY + C + t0);
                 tc5::wait_ld();
@@ -451,6 +469,15 @@ __global__ void __launch_bounds__(W5Cfg<MODE>::THREADS) tc5_walk_kernel(const __
 #pragma unroll
                 for (int j = 0; j < 8; ++j) ru[j] = pack_bf16(x[2 * j], x[2 * j + 1]);
                 tc5::st8(trow + Cfg::TAU + 8 * cg, ru);
+                if constexpr (Cfg::FULL) {
+                    uint32_t ry[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const float f = KDA ? 1.f : __shfl_sync(0xffffffffu, sce, j);
+                        ry[j] = __float_as_uint(-f * y[j]);
+                    }
+                    tc5::st16(trow + ((n & 1) ? Cfg::TZ2 : Cfg::TZ) + t0, ry);
+                }
                 tc5::wait_st();
                 tc5::fence_before();
                 warp_arrive(&s.u_ready);
@@ -464,6 +491,8 @@ __global__ void __launch_bounds__(W5Cfg<MODE>::THREADS) tc5_walk_kernel(const __
                     }
                 }
             }
+            // ---- the previous step's output, under this step's D product ----------
+            if (Cfg::FULL && n > 0 && !store_out(n - 1)) break;
             // ---- S1 = gamma S0 + D, and the bf16 state image -------------------
             if (!wait_all(&s.d_done, n & 1, p.status, p.wait_ns)) break;
             tc5::fence_after();
@@ -477,30 +506,12 @@ __global__ void __launch_bounds__(W5Cfg<MODE>::THREADS) tc5_walk_kernel(const __
             store_state();
             tc5::fence_before();
             warp_arrive(&s.s_ready);
+            if (KDA) warp_arrive(&s.empty[sn]);  // the per-key decays were its last stage reads
             if (Cfg::SAVE && n + 1 < nsteps && !store_s0(cn + 1)) break;
-            if (!Cfg::FULL) {
-                if (KDA) warp_arrive(&s.empty[sn]);
-                continue;
-            }
-            // ---- O^T = scale e^{G_i} S0 Q^T + U^T P^T, tokens t0 .. t0+15 of row a
-            if (!wait_all(&s.o_done, n & 1, p.status, p.wait_ns)) break;
-            tc5::fence_after();
-            {
-                float z[16];
-                tc5::ld16(z, trow + Cfg::TZ + t0);
-                tc5::wait_ld();
-                __nv_bfloat16* o = p.o + (((size_t)ch.tok0 + cn * C + t0) * p.H + h) * DV + a;
-#pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const float f = KDA ? 1.f : __shfl_sync(0xffffffffu, sce, j);
-                    if (t0 + j < L) o[(size_t)j * p.H * DV] = __float2bfloat16_rn(fmaf(-f, y[j], z[j]));
-                }
-            }
-            if (KDA) {
-                tc5::fence_before();
-                warp_arrive(&s.empty[sn]);
-            }
+            done_steps = n + 1;
         }
+        // the last step's output
+        if (Cfg::FULL && done_steps == nsteps && nsteps > 0) store_out(nsteps - 1);
         if (jb.out) {
             float* out = jb.out + (size_t)a * DK + 32 * cg;
 #pragma unroll
