@@ -15,7 +15,14 @@
 // as an MN-major A operand from shared memory; Q is scaled in place to
 // Q^ = scale e^{G_i} Q (rows past the sequence end zeroed) before T.
 // Each chunk's dS (bf16, Kp<128>) and dU (Tma128, token rows) are stored
-// for the local-gradient kernel; dh0 is the dS left after chunk 0.
+// for the local-gradient kernel; dh0 is the dS left after chunk 0.  From the
+// second step on, the epilogue writes these two images into the stage of the
+// step before (dead once that step's T product and epilogue are done: dS over
+// its Q and K~ tiles, dU over its W tile) and the load thread sends them out
+// with bulk stores before it refills the stage.  The threads themselves then
+// issue no global stores on the chain: per-thread 16-byte stores of dS rows
+// fill each 32-byte sector in two halves and stalled the epilogue behind the
+// store path.
 //
 // Warp roles as in tc5_walk.cu: 16 epilogue warps (TMEM lane quarter =
 // warp % 4, column group = warp / 4), one MMA warp, one load warp with a
@@ -62,8 +69,9 @@ struct RbSmem {
     RbStage st[RB_STAGES];
     uint64_t full[RB_STAGES], empty[RB_STAGES];
     // q_ready[k & 1]: Q^ of step k in place (two barriers: the epilogue may
-    // signal step k+1 before the MMA thread has waited for step k)
-    uint64_t ds_ready, q_ready[2], du_ready, e_done, t_done, fin;
+    // signal step k+1 before the MMA thread has waited for step k).
+    // staged[k & 1]: the dS and dU images of step k >= 1 are in stage k-1.
+    uint64_t ds_ready, q_ready[2], du_ready, e_done, t_done, fin, staged[2];
     uint32_t tmem;
 };
 
@@ -154,7 +162,8 @@ __global__ void __launch_bounds__(RB_THREADS) tc5_walk_bwd_kernel(const __grid_c
     if (tid == 0) {
         for (int i = 0; i < RB_STAGES; ++i) {
             mbar_init(&s.full[i], 1);
-            mbar_init(&s.empty[i], 1 + RB_EPI_WARPS);
+            // MODE 0: the MMA commit; the epilogue's part is known from staged
+            mbar_init(&s.empty[i], MODE == 0 ? 1 : 1 + RB_EPI_WARPS);
         }
         mbar_init(&s.ds_ready, RB_EPI_WARPS);
         mbar_init(&s.q_ready[0], RB_EPI_WARPS);
@@ -163,6 +172,8 @@ __global__ void __launch_bounds__(RB_THREADS) tc5_walk_bwd_kernel(const __grid_c
         mbar_init(&s.e_done, 1);
         mbar_init(&s.t_done, 1);
         mbar_init(&s.fin, 1);
+        mbar_init(&s.staged[0], RB_EPI_WARPS);
+        mbar_init(&s.staged[1], RB_EPI_WARPS);
         fence_mbar_init();
     }
     if (warp == RB_CTRL) tc5::alloc(&s.tmem, RCOLS);
@@ -173,15 +184,34 @@ __global__ void __launch_bounds__(RB_THREADS) tc5_walk_bwd_kernel(const __grid_c
 
     if (warp == RB_PROD) {
         if (lane == 0) {
+            // MODE 0: bulk stores of the dS and dU images of step m >= 1, staged
+            // in stage m-1; the stage is free again once they have been read
+            auto flush = [&](int m) -> bool {
+                if (!mbar_wait(&s.staged[m & 1], ((m - 1) >> 1) & 1, p.status)) return false;
+                const RbStage& sg = s.st[(m - 1) % RB_STAGES];
+                const size_t cid = (size_t)ch.img * p.NT + ch.n0 + (c_hi - 1 - m);
+                bulk_s2g(p.dSout + cid * DV * DK, sg.Q, DV * DK * 2);  // Q and K~ tiles: 32 KiB
+                bulk_s2g(p.dUout + cid * C * DV, sg.W, C * DV * 2);
+                bulk_commit();
+                bulk_wait_read<0>();
+                return true;
+            };
             int issued = 0;
+            bool ok = true;
             for (int k = 0; k < nsteps; ++k) {  // step k carries chunk c_hi-1-k of the chain
                 const int sk = k % RB_STAGES;
-                if (k >= RB_STAGES && !mbar_wait(&s.empty[sk], ((k / RB_STAGES) - 1) & 1, p.status)) break;
+                if (k >= RB_STAGES) {
+                    if (MODE == 0 && !(ok = flush(k - 2))) break;
+                    if (!(ok = mbar_wait(&s.empty[sk], ((k / RB_STAGES) - 1) & 1, p.status))) break;
+                }
                 rb_issue<KDA>(s.st[sk], &s.full[sk], p, ch, h, c_hi - 1 - k, use_do);
                 issued = k + 1;
             }
+            if (MODE == 0 && ok)
+                for (int m = max(1, issued - 2); m < issued && flush(m); ++m) {}
             for (int k = max(0, issued - RB_STAGES); k < issued; ++k)
                 mbar_wait(&s.full[k % RB_STAGES], (k / RB_STAGES) & 1, p.status);
+            bulk_wait<0>();
         }
         __syncwarp();
     } else if (warp == RB_CTRL) {
@@ -264,14 +294,6 @@ __global__ void __launch_bounds__(RB_THREADS) tc5_walk_bwd_kernel(const __grid_c
             const int L = min(C, ch.end - (ch.tok0 + j * C));
             const size_t cid = (size_t)ch.img * p.NT + ch.n0 + j;
             if (!rb_wait_all(&s.full[sk], (k / RB_STAGES) & 1, p.status)) break;
-            if (MODE == 0) {   // dS leaving chunk n: bf16 Kp<128> image, 64 contiguous bytes
-                __nv_bfloat16* dst = p.dSout + cid * DV * DK;
-#pragma unroll
-                for (int jj = 0; jj < 4; ++jj)
-                    *reinterpret_cast<uint4*>(dst + Kp<DV>::off(a, 32 * cg + 8 * jj)) =
-                        make_uint4(pack_bf16(dS[8 * jj], dS[8 * jj + 1]), pack_bf16(dS[8 * jj + 2], dS[8 * jj + 3]),
-                                   pack_bf16(dS[8 * jj + 4], dS[8 * jj + 5]), pack_bf16(dS[8 * jj + 6], dS[8 * jj + 7]));
-            }
             // Q^ = scale e^{G_i} Q in place, rows past the sequence end zeroed
             if (use_do && (!KDA || L < C)) {
 #pragma unroll
@@ -292,6 +314,17 @@ __global__ void __launch_bounds__(RB_THREADS) tc5_walk_bwd_kernel(const __grid_c
             }
             tc5::fence_proxy_async();
             rb_warp_arrive(&s.q_ready[k & 1]);
+            // the dS image of chunk j (the gradient leaving it), bf16 Kp<128>:
+            // into stage k-1 for the load thread's bulk store, or to global
+            // memory at the first step
+            if (MODE == 0) {
+                __nv_bfloat16* dst = k > 0 ? s.st[(k + RB_STAGES - 1) % RB_STAGES].Q : p.dSout + cid * DV * DK;
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj)
+                    *reinterpret_cast<uint4*>(dst + Kp<DV>::off(a, 32 * cg + 8 * jj)) =
+                        make_uint4(pack_bf16(dS[8 * jj], dS[8 * jj + 1]), pack_bf16(dS[8 * jj + 2], dS[8 * jj + 3]),
+                                   pack_bf16(dS[8 * jj + 4], dS[8 * jj + 5]), pack_bf16(dS[8 * jj + 6], dS[8 * jj + 7]));
+            }
             // ---- dU = F + E, zero past the sequence end (E = dS K~^T carries
             // the factors e^{G_last - G_i}) ---------------------------------------
             const float gam = KDA ? 1.f : __expf(st.G[C - 1]);
@@ -313,13 +346,17 @@ __global__ void __launch_bounds__(RB_THREADS) tc5_walk_bwd_kernel(const __grid_c
                 tc5::wait_st();
                 tc5::fence_before();
                 rb_warp_arrive(&s.du_ready);
-                if (MODE == 0) {
-                    __nv_bfloat16* dst = p.dUout + cid * C * DV;  // dU image, Tma128 token rows
+                if (MODE == 0) {  // dU image, Tma128 token rows: over stage k-1's W, or global
+                    __nv_bfloat16* dst = k > 0 ? s.st[(k + RB_STAGES - 1) % RB_STAGES].W : p.dUout + cid * C * DV;
 #pragma unroll
                     for (int jj = 0; jj < 8; ++jj) {
                         const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(&ru[jj]);
                         dst[Tma128::off(t0 + 2 * jj, a)] = v.x;
                         dst[Tma128::off(t0 + 2 * jj + 1, a)] = v.y;
+                    }
+                    if (k > 0) {
+                        tc5::fence_proxy_async();
+                        rb_warp_arrive(&s.staged[k & 1]);
                     }
                 }
             }
@@ -339,7 +376,7 @@ __global__ void __launch_bounds__(RB_THREADS) tc5_walk_bwd_kernel(const __grid_c
             store_ds_tmem();
             tc5::fence_before();
             rb_warp_arrive(&s.ds_ready);
-            rb_warp_arrive(&s.empty[sk]);
+            if (MODE != 0) rb_warp_arrive(&s.empty[sk]);
         }
         if (out) {
             float* dst = out + (size_t)a * DK + 32 * cg;
