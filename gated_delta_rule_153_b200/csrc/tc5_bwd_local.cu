@@ -258,13 +258,35 @@ GDN_DEV float dot_tile32(const float* x, const __nv_bfloat16* V, int r, int c0) 
     return acc;
 }
 
-GDN_DEV void store_row32(__nv_bfloat16* dst, const float* a, float f) {
+// f * a[0..31] as bf16 to dst (this lane's row, 64 bytes at a 32-byte
+// boundary) if ok.  Lanes 2i and 2i+1 hold neighbouring rows, pitch elements
+// apart.  Each 32-byte sector is written by one instruction: the two lanes
+// trade a 16-byte piece, so that in one store the pair writes both halves of
+// the even row's sector and in the next both halves of the odd row's.  (A
+// lane writing its own row alone fills every sector in two halves, which
+// costs the store path twice.)  Called by all lanes of the warp.
+GDN_DEV void store_row32(__nv_bfloat16* dst, size_t pitch, bool ok, const float* a, float f) {
     uint32_t pk[16];
 #pragma unroll
     for (int c = 0; c < 16; ++c) pk[c] = pack_bf16(f * a[2 * c], f * a[2 * c + 1]);
+    const bool odd = threadIdx.x & 1;
+    const bool pok = __shfl_xor_sync(0xffffffffu, ok, 1);
+    __nv_bfloat16* const even_row = odd ? dst - pitch : dst;
+    __nv_bfloat16* const odd_row = odd ? dst : dst + pitch;
 #pragma unroll
-    for (int q4 = 0; q4 < 4; ++q4)
-        *reinterpret_cast<uint4*>(dst + 8 * q4) = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+    for (int hs = 0; hs < 2; ++hs) {  // sector hs: columns 16hs .. 16hs+15 (pieces 2hs, 2hs+1)
+        uint32_t x[4];
+#pragma unroll
+        for (int w = 0; w < 4; ++w) x[w] = __shfl_xor_sync(0xffffffffu, odd ? pk[8 * hs + w] : pk[8 * hs + 4 + w], 1);
+        // the even row's sector: its piece 2hs from the even lane, 2hs+1 from the odd lane
+        const uint4 ve = odd ? make_uint4(x[0], x[1], x[2], x[3])
+                             : make_uint4(pk[8 * hs], pk[8 * hs + 1], pk[8 * hs + 2], pk[8 * hs + 3]);
+        if (odd ? pok : ok) *reinterpret_cast<uint4*>(even_row + 16 * hs + (odd ? 8 : 0)) = ve;
+        // the odd row's sector
+        const uint4 vo = odd ? make_uint4(pk[8 * hs + 4], pk[8 * hs + 5], pk[8 * hs + 6], pk[8 * hs + 7])
+                             : make_uint4(x[0], x[1], x[2], x[3]);
+        if (odd ? ok : pok) *reinterpret_cast<uint4*>(odd_row + 16 * hs + (odd ? 8 : 0)) = vo;
+    }
 }
 
 // Row t, columns c0..c0+31 (c0 a multiple of 32) of a pair region's panel, bf16.
@@ -532,7 +554,7 @@ __global__ void __launch_bounds__(BL_THREADS, 1) tc5_bwd_local_kernel(const __gr
 #pragma unroll
             for (int c = 0; c < 16; ++c) pk[c] = pack_bf16(gv[2 * c], gv[2 * c + 1]);
             tc5::st16(trow + TA + 64 + 16 * cg, pk);
-            if (t < L) store_row32(p.dv + (row0 + (size_t)t * rs) * DV + 32 * cg, gv, bt);
+            store_row32(p.dv + (row0 + (size_t)t * rs) * DV + 32 * cg, rs * DV, t < L, gv, bt);
             const bool vok = mbar_wait(&s.bar_v, lp, p.status);
             const float hv = vok ? dot_tile32(gv, s.R5, t, 32 * cg) : 0.f;
             ok = ok && vok;
@@ -543,7 +565,7 @@ __global__ void __launch_bounds__(BL_THREADS, 1) tc5_bwd_local_kernel(const __gr
             float a[32];
             ld_row32(a, trow + TA + 32 * cg);
             tc5::wait_ld();
-            if (i < L) store_row32(p.dq + (row0 + (size_t)i * rs) * DK + 32 * cg, a, 1.f);
+            store_row32(p.dq + (row0 + (size_t)i * rs) * DK + 32 * cg, rs * DK, i < L, a, 1.f);
         }
         tc5::wait_st();
         fence_async_smem();  // the V reads above, before the next chunk's S0 lands there
@@ -637,7 +659,7 @@ __global__ void __launch_bounds__(BL_THREADS, 1) tc5_bwd_local_kernel(const __gr
             tc5::wait_ld();
 #pragma unroll
             for (int c = 0; c < 32; ++c) a[c] = fmaf(f, kg[c], a[c]);
-            if (t < L) store_row32(p.dk + (row0 + (size_t)t * rs) * DK + 32 * cg, a, 1.f);
+            store_row32(p.dk + (row0 + (size_t)t * rs) * DK + 32 * cg, rs * DK, t < L, a, 1.f);
         } else if (warp == 2 && has_next) {
             load_gb(s, p, nch, (it + 1) & 1);
         }
