@@ -25,6 +25,20 @@ struct Kp {
     GDN_DEV static uint32_t off(int r, int c) { return (c >> 6) * (R * 64) + swz<64>(r, c & 63); }
 };
 
+// Transposed epilogue rows: a lane holds 16 consecutive rows r0 .. r0+15 of
+// its own column c as bf16 pairs v[jj] = (row r0+2jj, row r0+2jj+1).  Lanes
+// 2i and 2i+1 (columns c, c+1, c even) trade halves, so that w[jj] is the
+// 32-bit word (column c, c+1) of row r0 + 2jj + (lane & 1): one store of it
+// per row replaces two 2-byte stores.
+GDN_DEV void pair_columns(const uint32_t (&v)[8], uint32_t (&w)[8]) {
+    const bool odd = threadIdx.x & 1;
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj) {
+        const uint32_t o = __shfl_xor_sync(0xffffffffu, v[jj], 1);
+        w[jj] = odd ? __byte_perm(o, v[jj], 0x7632) : __byte_perm(v[jj], o, 0x5410);
+    }
+}
+
 namespace tc5 {
 
 // Shared-memory descriptor: start address, leading and stride byte offsets,

@@ -428,10 +428,15 @@ __global__ void __launch_bounds__(W5Cfg<MODE>::THREADS) tc5_walk_kernel(const __
             float z[16];
             tc5::ld16(z, trow + ((m & 1) ? Cfg::TZ2 : Cfg::TZ) + t0);
             tc5::wait_ld();
-            __nv_bfloat16* o = p.o + (((size_t)ch.tok0 + cm * C + t0) * p.H + h) * DV + a;
+            uint32_t v[8], w[8];
 #pragma unroll
-            for (int j = 0; j < 16; ++j)
-                if (t0 + j < Lm) o[(size_t)j * p.H * DV] = __float2bfloat16_rn(z[j]);
+            for (int j = 0; j < 8; ++j) v[j] = pack_bf16(z[2 * j], z[2 * j + 1]);
+            pair_columns(v, w);  // w[j]: values a & ~1, (a & ~1) + 1 of token t0 + 2j + (lane & 1)
+            const int t1 = t0 + (lane & 1);
+            __nv_bfloat16* o = p.o + (((size_t)ch.tok0 + cm * C + t1) * p.H + h) * DV + (a & ~1);
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                if (t1 + 2 * j < Lm) *reinterpret_cast<uint32_t*>(o + (size_t)(2 * j) * p.H * DV) = w[j];
             return true;
         };
         int done_steps = 0;
@@ -483,12 +488,11 @@ __global__ void __launch_bounds__(W5Cfg<MODE>::THREADS) tc5_walk_kernel(const __
                 warp_arrive(&s.u_ready);
                 if (Cfg::SAVE) {  // U image, Tma128 token rows (64 contiguous bytes per warp store)
                     __nv_bfloat16* dst = p.Uout + ((size_t)ch.img * p.NT + ch.n0 + cn) * C * DV;
+                    uint32_t w[8];
+                    pair_columns(ru, w);
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(&ru[j]);
-                        dst[Tma128::off(t0 + 2 * j, a)] = v.x;
-                        dst[Tma128::off(t0 + 2 * j + 1, a)] = v.y;
-                    }
+                    for (int j = 0; j < 8; ++j)
+                        *reinterpret_cast<uint32_t*>(dst + Tma128::off(t0 + 2 * j + (lane & 1), a & ~1)) = w[j];
                 }
             }
             // ---- the previous step's output, under this step's D product ----------

@@ -348,12 +348,11 @@ __global__ void __launch_bounds__(RB_THREADS) tc5_walk_bwd_kernel(const __grid_c
                 rb_warp_arrive(&s.du_ready);
                 if (MODE == 0) {  // dU image, Tma128 token rows: over stage k-1's W, or global
                     __nv_bfloat16* dst = k > 0 ? s.st[(k + RB_STAGES - 1) % RB_STAGES].W : p.dUout + cid * C * DV;
+                    uint32_t w[8];
+                    pair_columns(ru, w);
 #pragma unroll
-                    for (int jj = 0; jj < 8; ++jj) {
-                        const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(&ru[jj]);
-                        dst[Tma128::off(t0 + 2 * jj, a)] = v.x;
-                        dst[Tma128::off(t0 + 2 * jj + 1, a)] = v.y;
-                    }
+                    for (int jj = 0; jj < 8; ++jj)
+                        *reinterpret_cast<uint32_t*>(dst + Tma128::off(t0 + 2 * jj + (lane & 1), a & ~1)) = w[jj];
                     if (k > 0) {
                         tc5::fence_proxy_async();
                         rb_warp_arrive(&s.staged[k & 1]);
