@@ -113,6 +113,23 @@ __device__ void rb_issue(RbStage& st, uint64_t* bar, const RbPtrs& p, const Chai
     bulk_g2s(st.G, p.G + cid * GW, GW * 4, bar);
 }
 
+// The same tiles of chunk j, pulled into L2 a step before the ring reaches them.
+template <bool KDA>
+__device__ void rb_prefetch(const RbPtrs& p, const Chain& ch, int h, int j, bool use_do) {
+    const size_t cid = (size_t)ch.img * p.NT + ch.n0 + j;
+    constexpr int GW = KDA ? DK : C;
+    const int tok = ch.tok0 + j * C;
+    if (use_do) {
+        if (KDA) bulk_prefetch_l2(p.Qg + cid * C * DK, C * DK * 2);
+        else tma_prefetch_tile(&p.qmap, h, tok);
+        tma_prefetch_tile(&p.dOmap, h, tok);
+        bulk_prefetch_l2(p.P + cid * C * C, C * C * 2);
+    }
+    bulk_prefetch_l2(p.Kt + cid * C * DK, C * DK * 2);
+    bulk_prefetch_l2(p.W + cid * C * DK, C * DK * 2);
+    bulk_prefetch_l2(p.G + cid * GW, GW * 4);
+}
+
 GDN_DEV bool rb_wait_all(uint64_t* bar, uint32_t parity, unsigned int* status) {
     return __all_sync(0xffffffffu, mbar_wait(bar, parity, status));
 }
@@ -205,6 +222,8 @@ __global__ void __launch_bounds__(RB_THREADS) tc5_walk_bwd_kernel(const __grid_c
                     if (!(ok = mbar_wait(&s.empty[sk], ((k / RB_STAGES) - 1) & 1, p.status))) break;
                 }
                 rb_issue<KDA>(s.st[sk], &s.full[sk], p, ch, h, c_hi - 1 - k, use_do);
+                if (k + RB_STAGES < nsteps)  // the step after the ring (the backward: 260 -> 256 us)
+                    rb_prefetch<KDA>(p, ch, h, c_hi - 1 - (k + RB_STAGES), use_do);
                 issued = k + 1;
             }
             if (MODE == 0 && ok)
