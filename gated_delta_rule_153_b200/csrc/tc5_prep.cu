@@ -29,7 +29,7 @@
 // Outputs (bulk stores into the workspace): the W image (Tma128), the U~^T
 // image (Swz<64>, 128 value rows), P (Swz<64>), G, and optionally T (Swz<64>);
 // the K~ = diag(e^{G_last - G}) K image (Tma128) goes out with plain 16-byte
-// stores straight from the K tile.
+// stores straight from the K tile, four whole 128-byte rows per warp store.
 #include "async.cuh"
 #include "common.cuh"
 #include "internal.h"
@@ -247,15 +247,17 @@ __global__ void __launch_bounds__(P5_THREADS, 3) tc5_prep_kernel(const __grid_co
     // walks' B of the state update) from the K tile as loaded, and V <- diag(beta) V
     // in place (the row scale of U~; V is not read before the second product)
     if (tid < 128) {  // threads 0..127: K~ rows; 128..255: V rows
-        const int r = tid >> 1, pn = tid & 1;
-        const float dec = __expf(s.G[C - 1] - s.G[r]);
-        const __nv_bfloat16* row = s.KQ + pn * KQ_PANEL + r * 64;
-        // same swizzled position in the Tma128 image (panel pn at pn * 4096)
-        __nv_bfloat16* kt = p.Kt + (size_t)cid * C * DK + pn * (C * 64) + r * 64;
+        // 16-byte piece e = tid + 128 it of the image: piece e & 7 of row e >> 4,
+        // panel (e >> 3) & 1, so that every warp store writes four whole 128-byte
+        // rows (a thread writing a row piece by piece fills each 32-byte sector
+        // in two halves)
+        __nv_bfloat16* kt = p.Kt + (size_t)cid * C * DK;
 #pragma unroll
-        for (int jj = 0; jj < 8; ++jj) {
-            const int j = (jj + r) & 7;  // per-row rotated order (banks)
-            const uint4 x = *reinterpret_cast<const uint4*>(row + 8 * j);
+        for (int it = 0; it < 8; ++it) {
+            const int e = tid + 128 * it, j = e & 7, pn = (e >> 3) & 1, r = e >> 4;
+            const float dec = __expf(s.G[C - 1] - s.G[r]);
+            // same swizzled position in the Tma128 image (panel pn at pn * 4096)
+            const uint4 x = *reinterpret_cast<const uint4*>(s.KQ + pn * KQ_PANEL + r * 64 + 8 * j);
             const uint32_t w[4] = {x.x, x.y, x.z, x.w};
             uint32_t wt[4];
 #pragma unroll
@@ -263,7 +265,7 @@ __global__ void __launch_bounds__(P5_THREADS, 3) tc5_prep_kernel(const __grid_co
                 const float2 f2 = unpack_bf16(w[i]);
                 wt[i] = pack_bf16(f2.x * dec, f2.y * dec);
             }
-            *reinterpret_cast<uint4*>(kt + 8 * j) = make_uint4(wt[0], wt[1], wt[2], wt[3]);
+            *reinterpret_cast<uint4*>(kt + pn * (C * 64) + r * 64 + 8 * j) = make_uint4(wt[0], wt[1], wt[2], wt[3]);
         }
     } else {
         const int r = (tid - 128) >> 1, pn = tid & 1;
