@@ -348,13 +348,23 @@ GDN_DEV void verify_body(TreeSmem<MP, KDA>& s, const TreePtrs& p, uint32_t tm) {
     mph ^= 1;
     if (__syncthreads_or(!ok)) return;
     tc5::fence_after();
-    {   // O[i][v] for v = lr, nodes j0 ..: a warp writes 32 consecutive values
+    {   // O[i][v] for v = lr, nodes j0 ..: a warp writes 32 consecutive values of a
+        // node, lane pairs trading halves so that each store is a 32-bit word
         float x[MP / 2];
         ldcols<MP>(x, trow + TY + j0);
         tc5::wait_ld();
 #pragma unroll
-        for (int c = 0; c < MP / 2; ++c)
-            if (j0 + c < M) p.o[row0 + (size_t)(j0 + c) * rs + lr] = __float2bfloat16_rn(x[c]);
+        for (int g = 0; g < MP / 32; ++g) {
+            uint32_t v[8], w[8];
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj) v[jj] = pack_bf16(x[16 * g + 2 * jj], x[16 * g + 2 * jj + 1]);
+            pair_columns(v, w);  // w[jj]: values lr & ~1, +1 of node j0 + 16g + 2jj + (lane & 1)
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj) {
+                const int node = j0 + 16 * g + 2 * jj + (lane & 1);
+                if (node < M) *reinterpret_cast<uint32_t*>(p.o + row0 + (size_t)node * rs + (lr & ~1)) = w[jj];
+            }
+        }
     }
 }
 
