@@ -421,14 +421,16 @@ tree_verify_kernel(const __grid_constant__ TreePtrs p) {
         cp_async_commit();
     }
     // the state row of this thread's lane (value 32 (warp % 4) + lane), keys
-    // 64 (warp / 4) .. +63, from fp32 to bf16 pairs ...
+    // 64 (warp / 4) .. +63, from fp32 to bf16 pairs.  The loads go through L1:
+    // a warp's 16-byte loads touch half of each of 32 sectors, and the next
+    // load of the same lanes finds the other half there ...
     uint32_t srow[32];
     {
         const float4* src = reinterpret_cast<const float4*>(
             p.state + ((size_t)nh * TD + 32 * (warp & 3) + (tid & 31)) * TD + 64 * (warp >> 2));
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-            const float4 a = __ldcs(src + j);
+            const float4 a = __ldg(src + j);
             srow[2 * j] = pack_bf16(a.x, a.y);
             srow[2 * j + 1] = pack_bf16(a.z, a.w);
         }
