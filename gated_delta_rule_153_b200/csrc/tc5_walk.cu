@@ -231,6 +231,22 @@ GDN_DEV W5Job w5_job(const W5Ptrs& p, int nsteps_of_chain_unused) {
     return jb;
 }
 
+// The same tiles of chain step n, pulled into L2 ahead of the ring (the saving
+// forward with the scalar gate: 350M-scale forward 176.6 -> 174.3 us; with the
+// channel gate it measured slower and is left out).
+template <bool KDA, int MODE>
+__device__ void w5_prefetch(const W5Ptrs& p, const Chain& ch, int h, int n) {
+    const size_t cid = (size_t)ch.img * p.NT + ch.n0 + n;
+    constexpr int GW = KDA ? DK : C;
+    const int tok = ch.tok0 + n * C;
+    bulk_prefetch_l2(p.W + cid * C * DK, C * DK * 2);
+    if (KDA) bulk_prefetch_l2(p.Qg + cid * C * DK, C * DK * 2);
+    else tma_prefetch_tile(&p.qmap, h, tok);
+    bulk_prefetch_l2(p.P + cid * C * C, C * C * 2);
+    bulk_prefetch_l2(p.Ut + cid * C * DV, DV * C * 2);
+    bulk_prefetch_l2(p.Kt + cid * C * DK, C * DK * 2);
+    bulk_prefetch_l2(p.G + cid * GW, GW * 4);
+}
 template <bool KDA, int MODE>
 __global__ void __launch_bounds__(W5Cfg<MODE>::THREADS) tc5_walk_kernel(const __grid_constant__ W5Ptrs p) {
     using Cfg = W5Cfg<MODE>;
@@ -285,6 +301,7 @@ __global__ void __launch_bounds__(W5Cfg<MODE>::THREADS) tc5_walk_kernel(const __
                 if (n == p.stall_at) break;  // test hook: leave this stage unloaded
                 if (n >= NST && !mbar_wait(&s.empty[sn], ((n / NST) - 1) & 1, p.status, p.wait_ns)) break;
                 w5_issue<KDA, MODE>(s.st[sn], s.G[sn], &s.full[sn], p, ch, h, n_begin + n, jb.use_u);
+                if (MODE == 3 && !KDA && n + NST < nsteps) w5_prefetch<KDA, MODE>(p, ch, h, n_begin + n + NST);
                 issued = n + 1;
             }
             // Leave no load in flight (returns at once for stages already consumed).
