@@ -411,10 +411,10 @@ __global__ void __launch_bounds__(W5Cfg<MODE>::THREADS) tc5_walk_kernel(const __
             tc5::st16(trow + Cfg::TAS + 16 * cg, r);
             tc5::wait_st();
         };
-        // MODE 1: bf16 state entering chain step n, Kp<128> image (64 contiguous
-        // bytes per thread).  MODE 3: the same image staged in shared memory
-        // (buffer m & 1 for this CTA's m-th state, m = n - n_begin) for the
-        // saver warp's bulk store.
+        // MODE 1: bf16 state entering chain step n, Kp<128> image (64 bytes of a
+        // row per thread, whole sectors per store).  MODE 3: the same image
+        // staged in shared memory (buffer m & 1 for this CTA's m-th state,
+        // m = n - n_begin) for the saver warp's bulk store.
         auto store_s0 = [&](int n) {
             __nv_bfloat16* dst = p.S0out + ((size_t)ch.img * p.NT + ch.n0 + n) * DV * DK;
             if constexpr (Cfg::STAGED) {
@@ -423,12 +423,36 @@ __global__ void __launch_bounds__(W5Cfg<MODE>::THREADS) tc5_walk_kernel(const __
                     return false;
                 dst = s.sv.S0[m & 1];
             }
+            if constexpr (Cfg::STAGED) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int c = 32 * cg + 8 * j;
-                *reinterpret_cast<uint4*>(dst + Kp<DV>::off(a, c)) =
-                    make_uint4(pack_bf16(S[8 * j], S[8 * j + 1]), pack_bf16(S[8 * j + 2], S[8 * j + 3]),
-                               pack_bf16(S[8 * j + 4], S[8 * j + 5]), pack_bf16(S[8 * j + 6], S[8 * j + 7]));
+                for (int j = 0; j < 4; ++j) {
+                    const int c = 32 * cg + 8 * j;
+                    *reinterpret_cast<uint4*>(dst + Kp<DV>::off(a, c)) =
+                        make_uint4(pack_bf16(S[8 * j], S[8 * j + 1]), pack_bf16(S[8 * j + 2], S[8 * j + 3]),
+                                   pack_bf16(S[8 * j + 4], S[8 * j + 5]), pack_bf16(S[8 * j + 6], S[8 * j + 7]));
+                }
+            } else {
+                // global memory: lanes 2i, 2i+1 (rows a, a+1 of one swizzle group) trade
+                // a 16-byte piece so that each store covers whole 32-byte sectors
+                uint32_t pk[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) pk[j] = pack_bf16(S[2 * j], S[2 * j + 1]);
+                const bool odd = lane & 1;
+                const int re = odd ? a - 1 : a, ro = odd ? a : a + 1;
+#pragma unroll
+                for (int hs = 0; hs < 2; ++hs) {
+                    uint32_t x[4];
+#pragma unroll
+                    for (int w = 0; w < 4; ++w)
+                        x[w] = __shfl_xor_sync(0xffffffffu, odd ? pk[8 * hs + w] : pk[8 * hs + 4 + w], 1);
+                    const int c = 32 * cg + 16 * hs + (odd ? 8 : 0);
+                    *reinterpret_cast<uint4*>(dst + Kp<DV>::off(re, c)) =
+                        odd ? make_uint4(x[0], x[1], x[2], x[3])
+                            : make_uint4(pk[8 * hs], pk[8 * hs + 1], pk[8 * hs + 2], pk[8 * hs + 3]);
+                    *reinterpret_cast<uint4*>(dst + Kp<DV>::off(ro, c)) =
+                        odd ? make_uint4(pk[8 * hs + 4], pk[8 * hs + 5], pk[8 * hs + 6], pk[8 * hs + 7])
+                            : make_uint4(x[0], x[1], x[2], x[3]);
+                }
             }
             if constexpr (Cfg::STAGED) {
                 fence_async_smem();
